@@ -1,0 +1,247 @@
+"""fp64 CPU oracle of the FastVim SSM layer (pooled selective scan).
+
+TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only the test suite, the package smoke check and the
+benchmark's CPU-baseline / reference leg may import this module.  It wraps the plain C library
+built from ``fastvim_oracle.c`` (fp64, nested loops, no GPU code, no code shared with the CUDA
+library); see that file for the method passages each step follows and the readings taken where
+the method description is silent.
+
+Every function takes numpy arrays in the layouts of ``fastvim_oracle.h`` and returns fp64 arrays.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fastvim_oracle.c")
+_HDR = os.path.join(_HERE, "fastvim_oracle.h")
+_LIB_PATH = os.path.join(_HERE, "libfastvim_oracle.so")
+
+FVO_OK, FVO_BAD_SHAPE, FVO_BAD_INDEX, FVO_NO_MEMORY = 0, 2, 4, 8
+POOL_W, POOL_H = 0, 1
+FWD, BWD = 1, 2
+
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``libfastvim_oracle.so`` (gcc, -O2, OpenMP over images)."""
+    newest_src = max(os.path.getmtime(_SRC), os.path.getmtime(_HDR))
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < newest_src:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-std=c99", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            I = ctypes.c_int
+            U = ctypes.c_uint
+            Dbl = ctypes.c_double
+            sigs = {
+                "fvo_pool": [P, I, I, I, I, I, Dbl, P],
+                "fvo_mask_rows": [P, I, I, I, I, I, P, P, P],
+                "fvo_pool_masked": [P, P, P, I, I, I, I, I, Dbl, P],
+                "fvo_proj": [P, I, I, I, I, I, I, P, P, P, P, P],
+                "fvo_scan": [P, P, P, P, I, I, I, I, I, I, U, I, P],
+                "fvo_gate_dense": [P, P, P, P, I, I, I, I, I, I, P],
+                "fvo_gate_masked": [P, P, P, P, P, I, I, I, I, I, P],
+                "fvo_forward": [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, U, Dbl, I, I, P],
+            }
+            for name, argtypes in sigs.items():
+                fn = getattr(lib, name)
+                fn.argtypes = argtypes
+                fn.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+class OracleError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"oracle {where} returned status {status}")
+        self.status = status
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _f64(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _i32(a):
+    return np.ascontiguousarray(a, dtype=np.int32)
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(st, where, allow=()):
+    if st != FVO_OK and st not in allow:
+        raise OracleError(st, where)
+    return st
+
+
+def nd_of(dir_flags: int) -> int:
+    return int(bool(dir_flags & FWD)) + int(bool(dir_flags & BWD))
+
+
+def pooled_len(h: int, w: int, pool_axis: int) -> int:
+    return h if pool_axis == POOL_W else w
+
+
+def pooled_over(h: int, w: int, pool_axis: int) -> int:
+    return w if pool_axis == POOL_W else h
+
+
+def pool(x, pool_axis, pool_scale=1.0):
+    """Dense mean pooling: x [B,h,w,E] -> xbar [B,T,E]."""
+    x = _f32(x)
+    B, h, w, E = x.shape
+    out = np.empty((B, pooled_len(h, w, pool_axis), E), np.float64)
+    _check(_load().fvo_pool(_p(x), B, h, w, E, pool_axis, float(pool_scale), _p(out)), "pool")
+    return out
+
+
+def mask_rows(keep_idx, h, w, pool_axis):
+    """Row bucketing of kept-token ids -> (status, row_of [B,K], row_off [B,T+1], row_tok [B,K])."""
+    idx = _i32(keep_idx)
+    B, K = idx.shape
+    T = pooled_len(h, w, pool_axis)
+    row_of = np.empty((B, K), np.int32)
+    row_off = np.empty((B, T + 1), np.int32)
+    row_tok = np.empty((B, K), np.int32)
+    st = _load().fvo_mask_rows(_p(idx), B, K, h, w, pool_axis, _p(row_of), _p(row_off), _p(row_tok))
+    _check(st, "mask_rows", allow=(FVO_BAD_INDEX,))
+    return st, row_of, row_off, row_tok
+
+
+def pool_masked(x, row_off, row_tok, S, pool_scale=1.0):
+    """Masked mean pooling: x [B,K,E] + row CSR -> xbar [B,T,E] (divisor S, fixed)."""
+    x = _f32(x)
+    B, K, E = x.shape
+    row_off = _i32(row_off)
+    row_tok = _i32(row_tok)
+    T = row_off.shape[1] - 1
+    out = np.empty((B, T, E), np.float64)
+    st = _load().fvo_pool_masked(_p(x), _p(row_off), _p(row_tok), B, K, T, S, E, float(pool_scale), _p(out))
+    _check(st, "pool_masked")
+    return out
+
+
+def proj(xbar, W_x, W_dt, b_dt, R, N):
+    """x_proj + dt_proj + softplus: xbar [B,T,E] -> u [nd,B,T,R+2N], delta [nd,B,T,E]."""
+    xbar = _f64(xbar)
+    W_x, W_dt, b_dt = _f32(W_x), _f32(W_dt), _f32(b_dt)
+    B, T, E = xbar.shape
+    nd = W_x.shape[0]
+    u = np.empty((nd, B, T, R + 2 * N), np.float64)
+    delta = np.empty((nd, B, T, E), np.float64)
+    st = _load().fvo_proj(_p(xbar), B, T, E, nd, R, N, _p(W_x), _p(W_dt), _p(b_dt), _p(u), _p(delta))
+    _check(st, "proj")
+    return u, delta
+
+
+def scan(xbar, delta, u, A_log, R, N, dir_flags, zoh_exact=False):
+    """ZOH + forward/backward selective scans, directions summed -> ys [B,T,E]."""
+    xbar, delta, u = _f64(xbar), _f64(delta), _f64(u)
+    A_log = _f32(A_log)
+    B, T, E = xbar.shape
+    nd = nd_of(dir_flags)
+    ys = np.empty((B, T, E), np.float64)
+    st = _load().fvo_scan(_p(xbar), _p(delta), _p(u), _p(A_log), B, T, E, nd, R, N,
+                          int(dir_flags), int(bool(zoh_exact)), _p(ys))
+    _check(st, "scan")
+    return ys
+
+
+def gate_dense(x, z, ys, D, pool_axis):
+    """Repeat + D x skip + SiLU(z) gate on the dense grid -> y [B,h,w,E]."""
+    x, z, D = _f32(x), _f32(z), _f32(D)
+    ys = _f64(ys)
+    B, h, w, E = x.shape
+    y = np.empty(x.shape, np.float64)
+    st = _load().fvo_gate_dense(_p(x), _p(z), _p(ys), _p(D), B, h, w, E, D.shape[0], pool_axis, _p(y))
+    _check(st, "gate_dense")
+    return y
+
+
+def gate_masked(x, z, ys, D, row_of):
+    """Repeat to kept tokens + skip + gate -> y [B,K,E]."""
+    x, z, D = _f32(x), _f32(z), _f32(D)
+    ys = _f64(ys)
+    row_of = _i32(row_of)
+    B, K, E = x.shape
+    T = ys.shape[1]
+    y = np.empty(x.shape, np.float64)
+    st = _load().fvo_gate_masked(_p(x), _p(z), _p(ys), _p(D), _p(row_of), B, K, T, E, D.shape[0], _p(y))
+    _check(st, "gate_masked")
+    return y
+
+
+def forward(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis, dir_flags, keep_idx=None, h=None,
+            w=None, pool_scale=1.0, zoh_exact=False, nthreads=1, allow_bad_index=False):
+    """The whole layer, image by image.
+
+    Dense: x, z [B,h,w,E] -> y [B,h,w,E].  Masked: x, z [B,K,E], keep_idx [B,K] with the grid
+    given by h, w -> y [B,K,E].  Returns fp64 y (and the status when allow_bad_index is set).
+    """
+    x, z = _f32(x), _f32(z)
+    A_log, D, W_x, W_dt, b_dt = map(_f32, (A_log, D, W_x, W_dt, b_dt))
+    N = A_log.shape[2]
+    E = A_log.shape[1]
+    R = W_dt.shape[2]
+    if keep_idx is None:
+        B, h, w, E2 = x.shape
+        K = 0
+        idx = None
+    else:
+        B, K, E2 = x.shape
+        idx = _i32(keep_idx)
+        assert h is not None and w is not None and idx.shape == (B, K)
+    assert E2 == E and z.shape == x.shape
+    y = np.empty(x.shape, np.float64)
+    st = _load().fvo_forward(_p(x), _p(z), _p(A_log), _p(D), _p(W_x), _p(W_dt), _p(b_dt), _p(idx),
+                             B, h, w, E, N, R, K, pool_axis, int(dir_flags), float(pool_scale),
+                             int(bool(zoh_exact)), int(nthreads), _p(y))
+    _check(st, "forward", allow=(FVO_BAD_INDEX,) if allow_bad_index else ())
+    return (y, st) if allow_bad_index else y
+
+
+def forward_intermediates(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis, dir_flags, keep_idx=None,
+                          h=None, w=None, pool_scale=1.0, zoh_exact=False):
+    """The same chain step by step, returning every intermediate as a dict (small sizes only)."""
+    A_log, W_dt = _f32(A_log), _f32(W_dt)
+    N = A_log.shape[2]
+    R = W_dt.shape[2]
+    out = {}
+    if keep_idx is None:
+        xbar = pool(x, pool_axis, pool_scale)
+    else:
+        st, row_of, row_off, row_tok = mask_rows(keep_idx, h, w, pool_axis)
+        if st != FVO_OK:
+            raise OracleError(st, "mask_rows")
+        out.update(row_of=row_of, row_off=row_off, row_tok=row_tok)
+        xbar = pool_masked(x, row_off, row_tok, pooled_over(h, w, pool_axis), pool_scale)
+    u, delta = proj(xbar, W_x, W_dt, b_dt, R, N)
+    ys = scan(xbar, delta, u, A_log, R, N, dir_flags, zoh_exact)
+    if keep_idx is None:
+        y = gate_dense(x, z, ys, D, pool_axis)
+    else:
+        y = gate_masked(x, z, ys, D, out["row_of"])
+    out.update(xbar=xbar, u=u, delta=delta, ys=ys, y=y)
+    return out

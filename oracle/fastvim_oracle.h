@@ -1,0 +1,85 @@
+/*
+ * fastvim_oracle.h -- fp64 CPU oracle of the FastVim SSM layer ("pooled selective scan").
+ *
+ * TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only the test suite, the package's smoke check and
+ * the benchmark's CPU-baseline / reference leg may load or call this library.  It shares no
+ * code, header, table or helper with the CUDA library; the two only ever meet through the
+ * seeded synthetic inputs that both are handed.
+ *
+ * What it computes follows the method description of FastVim (Kapse et al., arXiv 2502.00594):
+ *   - gptget.net summary of 2502.00594, section "方法详解" (method details), items 1-6:
+ *     reshape to (B,h,w,D), mean-pool along one grid axis to (B,h,1,D), input-dependent
+ *     B, C and Delta = softplus(Parameter + s_Delta(x)), ZOH discretisation, forward and
+ *     backward selective scan of the pooled sequence, repeat along the pooled axis, skip;
+ *   - same page, glossary "State Space Model": h_t = A h_{t-1} + B x_t, y_t = C h_t + D x_t;
+ *   - pith.science verdict on 2502.00594, field "key_machinery": the repeat restores the token
+ *     count before the D x_t skip connection (so the skip uses full-resolution x);
+ *   - ijyty.com Vision Mamba article, section 2.1 code: the block gates the sum of the forward
+ *     and backward SSM outputs with z.
+ *
+ * All arithmetic is fp64; inputs are fp32 arrays as the GPU library sees them.
+ * Layouts (row-major, last index fastest):
+ *   dense  x, z        [B][h][w][E]          masked x, z      [B][K][E]
+ *   keep_idx           [B][K] int32, grid id r*w + c
+ *   A_log              [nd][E][N]            D                [nd][E]
+ *   W_x                [nd][R+2N][E]  (rows: dt_low | B | C)
+ *   W_dt               [nd][E][R]            b_dt             [nd][E]
+ *   xbar               [B][T][E]             u                [nd][B][T][R+2N]
+ *   delta              [nd][B][T][E]         ys               [B][T][E]
+ * Parameter slot k (0..nd-1) belongs to the k-th enabled direction in the order FWD, BWD.
+ */
+#ifndef FASTVIM_ORACLE_H
+#define FASTVIM_ORACLE_H
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum { FVO_OK = 0, FVO_BAD_SHAPE = 2, FVO_BAD_INDEX = 4, FVO_NO_MEMORY = 8 };
+enum { FVO_POOL_W = 0, FVO_POOL_H = 1 };
+enum { FVO_FWD = 1, FVO_BWD = 2 };
+
+/* Mean pooling of a dense grid along one axis (pooled length T, pooled-over length S). */
+int fvo_pool(const float* x, int B, int h, int w, int E, int pool_axis, double pool_scale,
+             double* xbar);
+
+/* Row bucketing of kept-token indices: row_of[B][K] (pooled token of each kept token),
+ * row_off[B][T+1] and row_tok[B][K] (kept-token ordinals grouped by row, ascending k). */
+int fvo_mask_rows(const int32_t* keep_idx, int B, int K, int h, int w, int pool_axis,
+                  int32_t* row_of, int32_t* row_off, int32_t* row_tok);
+
+/* Masked pooling: xbar[b][t] = pool_scale * (sum of kept tokens in row t) / S. */
+int fvo_pool_masked(const float* x, const int32_t* row_off, const int32_t* row_tok, int B,
+                    int K, int T, int S, int E, double pool_scale, double* xbar);
+
+/* x_proj and dt_proj + softplus on the pooled tokens. */
+int fvo_proj(const double* xbar, int B, int T, int E, int nd, int R, int N, const float* W_x,
+             const float* W_dt, const float* b_dt, double* u, double* delta);
+
+/* ZOH discretisation + forward/backward selective scans, directions summed. zoh_exact = 0:
+ * Bbar x = Delta B x; zoh_exact = 1: Bbar = (exp(Delta A) - 1) / A * B. */
+int fvo_scan(const double* xbar, const double* delta, const double* u, const float* A_log,
+             int B, int T, int E, int nd, int R, int N, unsigned dir_flags, int zoh_exact,
+             double* ys);
+
+/* Repeat + D x skip + SiLU(z) gate on the dense grid. */
+int fvo_gate_dense(const float* x, const float* z, const double* ys, const float* D, int B,
+                   int h, int w, int E, int nd, int pool_axis, double* y);
+
+/* Same on the kept tokens, each taking the pooled output of its row. */
+int fvo_gate_masked(const float* x, const float* z, const double* ys, const float* D,
+                    const int32_t* row_of, int B, int K, int T, int E, int nd, double* y);
+
+/* The whole layer, one image at a time (OpenMP over images when nthreads > 1).
+ * keep_idx == NULL: dense x, z, y [B][h][w][E]; otherwise masked [B][K][E]. */
+int fvo_forward(const float* x, const float* z, const float* A_log, const float* D,
+                const float* W_x, const float* W_dt, const float* b_dt,
+                const int32_t* keep_idx, int B, int h, int w, int E, int N, int R, int K,
+                int pool_axis, unsigned dir_flags, double pool_scale, int zoh_exact,
+                int nthreads, double* y);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
