@@ -1,0 +1,431 @@
+#!/usr/bin/env python
+"""Benchmark of the FastVim SSM layer (pooled selective scan) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config NAME]
+
+One step = one fastvim_ssm_forward call over the whole batch of the workload (pool ->
+projections -> scans -> repeat/skip/gate), inputs resident in HBM.  The default workload is the
+FastVim-T layer at 2048 px: B = 128, a 128 x 128 token grid, E = 384, N = 16, R = 12, column
+pooling, forward + backward scans, fp32.  Its x, z and y take 9.7 GB, far above the 126 MB L2,
+so no L2 flush is needed between steps.
+
+Under torchrun (N > 1) every rank runs its own full batch on its own GPU (the images are
+independent, so there is no data-path collective: weak scaling); the step time is the maximum
+over ranks of each rank's CUDA-event time.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (rank 0 only), on a bounded
+sample of images of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "SSM-layer grid tokens/s at 2048² FastVim-T (fp32, B=128); HBM GB/s vs peak"
+UNIT = "grid tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+# Algorithmic bytes per processed token of each kernel, in units of E*4 bytes (fp32 channels):
+# what the kernel must move at minimum for its step of the layer.
+KERNEL_BYTES_PER_TOKEN_E4 = {
+    "pool_dense_kernel": 1,        # read x
+    "epilogue_dense_kernel": 3,    # read x, read z, write y
+    "mask_pool_kernel": 1,         # read kept x
+    "mask_epilogue_kernel": 3,     # read kept x and z, write y
+    "fused_layer_kernel": 3,       # the whole layer: x once, z, y
+}
+
+
+def parse(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="fastvim_t_2048")
+    ap.add_argument("--pool-axis", type=int, default=None, help="override the workload's pool axis")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) leg")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    a = ap.parse_args(argv)
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if a.steps < 1:
+        ap.error("--steps must be >= 1")
+    return a
+
+
+def workload_desc(cfg, pool_axis):
+    axis = "w (column pooling, T = h)" if pool_axis == 0 else "h (row pooling, T = w)"
+    dirs = {1: "forward", 2: "backward", 3: "forward+backward"}[cfg.dir_flags]
+    d = {
+        "workload": f"{cfg.name}: {cfg.note}",
+        "B": cfg.B, "grid": [cfg.h, cfg.w], "E": cfg.E, "N": cfg.N, "R": cfg.R,
+        "pool": axis, "scan": dirs,
+    }
+    if cfg.masked:
+        d["kept_tokens_per_sample"] = cfg.K
+    return d
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s earlier pool measurement)"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "pooled_selective_scan_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, cfg_name):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on the
+    current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+    except Exception:
+        return None
+    if j.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    ent = j.get("kernels", {}).get(f"{cfg_name}/{kernel}")
+    if not ent:
+        return None
+    return ent.get("dram_bytes_per_full_launch")
+
+
+# ------------------------------------------------------------------------------------------------
+# Clock sampling (NVML, read-only) during the timed region.
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+               0x1: "gpu_idle", 0x10: "sync_boost", 0x100: "display_clock_setting"}
+
+    def __init__(self, torch_device_index, period_s=0.02):
+        self.ok = False
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml as nv
+            import torch
+            nv.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_device_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = nv.nvmlDeviceGetHandleByUUID(uuid)
+            self.nv = nv
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self._reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.ok = True
+        except Exception as e:  # sampling is best effort; the JSON says when it was unavailable
+            self.err = f"{type(e).__name__}: {e}"
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = self._reasons(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": getattr(self, "err", "unavailable")}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [m for m, _ in self.samples]
+        mask = 0
+        for _, r in self.samples:
+            mask |= int(r)
+        reasons = sorted(n for bit, n in self.REASONS.items() if mask & bit and n != "gpu_idle")
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(mhz), "sm_mhz_min": min(mhz)}
+
+
+# ------------------------------------------------------------------------------------------------
+# Multi-rank plumbing
+# ------------------------------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a per-rank float over the process group (identity without one)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: int, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return units_per_rank * world / max_seconds
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline of our arm, and the reference arm)
+# ------------------------------------------------------------------------------------------------
+def oracle_sample(cfg, pool_axis, n_images):
+    import oracle
+    from pooled_selective_scan_b200 import inputs
+    which = list(range(min(n_images, cfg.B)))
+    d = inputs.layer_inputs(cfg, which=which)
+    oracle.build()
+
+    def step(nthreads):
+        oracle.forward(d["x"], d["z"], d["A_log"], d["D"], d["W_x"], d["W_dt"], d["b_dt"], pool_axis,
+                       cfg.dir_flags, keep_idx=d.get("keep_idx"), h=cfg.h, w=cfg.w, nthreads=nthreads)
+    return which, step
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(cfg, pool_axis, min_seconds=10.0):
+    cores = host_cores()
+    n_img = min(cfg.B, max(1, cores), 32)
+    which, step = oracle_sample(cfg, pool_axis, n_img)
+    threads = min(cores, len(which))
+    step(threads)  # warm
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        step(threads)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el * threads >= min_seconds or el >= min_seconds:
+            break
+    tok = len(which) * (cfg.K if cfg.masked else cfg.h * cfg.w)
+    return {"value": tok * reps / el, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{len(which)} images of {cfg.name} x {reps} passes, fp64 C oracle, OpenMP over images "
+                      f"({el:.1f} s wall, {el * threads:.1f} core-s)"}
+
+
+def run_reference(a, cfg, pool_axis):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    cores = host_cores()
+    n_img = min(cfg.B, max(1, cores), 16)
+    which, step = oracle_sample(cfg, pool_axis, n_img)
+    threads = min(cores, len(which))
+    for _ in range(a.warmup):
+        step(threads)
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        step(threads)
+    el = time.perf_counter() - t0
+    tok = len(which) * (cfg.K if cfg.masked else cfg.h * cfg.w)
+    value = tok * a.steps / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * el / a.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": dict(workload_desc(cfg, pool_axis), sample_per_step=f"{len(which)} of {cfg.B} images"),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{len(which)} images of {cfg.name} per step, fp64 C oracle, OpenMP over images"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------------------
+# Our arm
+# ------------------------------------------------------------------------------------------------
+def run_ours(a, cfg, pool_axis):
+    import torch
+    import torch.distributed as dist
+
+    from pooled_selective_scan_b200 import build as fvbuild
+    from pooled_selective_scan_b200 import ssm, workload
+
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the layer has no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    if not os.path.exists(os.path.join(ROOT, "pooled_selective_scan_b200", "libfastvim_ssm.so")):
+        if rank == 0:
+            fvbuild.build()
+        if world > 1:
+            dist.barrier()
+
+    t = workload.layer_tensors(cfg, dev)
+    keep = t.get("keep_idx")
+    shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, cfg.dir_flags, keep, cfg.h, cfg.w)
+    y = torch.empty_like(t["x"])
+    ws = ssm.alloc_workspace(shape, dev)
+    stream = torch.cuda.current_stream(dev)
+    fwd = ssm.BoundForward(shape, t, y, ws, stream)
+    names = ssm.launch_names(shape)
+    nl = len(names)
+
+    for _ in range(a.warmup):
+        fwd.run()
+    torch.cuda.synchronize(dev)
+    if ssm.device_status(ws) != 0:
+        raise SystemExit("device status reported an error during warm-up")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nl + 1)] for _ in range(a.steps)]
+    for evs in events:  # materialise the event handles outside the timed region
+        for e in evs:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for i in range(a.steps):
+        fwd.run_events(events[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks.stop()
+    local_ms = start.elapsed_time(end)
+    max_ms = reduce_max(local_ms, dev)
+    per_kernel = {n: [] for n in names}
+    for evs in events:
+        for j, n in enumerate(names):
+            per_kernel[n].append(evs[j].elapsed_time(evs[j + 1]))
+    if ssm.device_status(ws) != 0:
+        raise SystemExit("device status reported an error in the timed region")
+
+    tokens = cfg.tokens_per_call()
+    ms_step = max_ms / a.steps
+    value = weak_scaling_value(tokens * a.steps, world, max_ms / 1e3)
+    peak, peak_src = load_peaks()
+    alg_bytes_call = cfg.algorithmic_bytes_per_call()
+
+    total_k = sum(sum(v) for v in per_kernel.values())
+    kern = {n: {"launches": len(v), "avg_us": 1e3 * statistics.mean(v), "share": sum(v) / total_k}
+            for n, v in per_kernel.items()}
+    dom = max(kern, key=lambda n: kern[n]["share"])
+    dom_alg = KERNEL_BYTES_PER_TOKEN_E4.get(dom, 0) * 4 * cfg.E * tokens
+    dom_s = kern[dom]["avg_us"] / 1e6
+    achieved = dom_alg / dom_s / 1e9 if dom_alg else None
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": (achieved / peak) if achieved else None, "traffic": recorded_traffic(dom, cfg.name),
+                "algorithmic_bytes_per_launch": dom_alg, "peak_source": peak_src,
+                "note": "achieved = algorithmic bytes per launch / mean CUDA-event duration of the launch"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic (seeded N(0,1) x, z; Mamba-style parameter init)",
+        "config": dict(workload_desc(cfg, pool_axis),
+                       l2=f"inputs {alg_bytes_call / 1e9:.2f} GB per step > 126 MB L2; no flush",
+                       parallelism=f"replicas: each of {world} GPU(s) runs its own batch of {cfg.B}"),
+        "layer_hbm": {"achieved_gbs": alg_bytes_call / (ms_step / 1e3) / 1e9, "peak_gbs": peak,
+                      "frac": alg_bytes_call / (ms_step / 1e3) / 1e9 / peak,
+                      "algorithmic_bytes_per_step": alg_bytes_call},
+        "roofline": roofline,
+        "kernels": kern,
+        "gpu_launches": nl * a.steps,
+        "clocks": clocks.summary(),
+    }
+
+    del events
+    # end-to-end leg: host buffers through fastvim_ssm_forward_host (every rank runs it; max over ranks)
+    if not a.no_e2e:
+        del fwd
+        dev_keep = None
+        del t, y
+        torch.cuda.empty_cache()
+        host = workload.layer_tensors(cfg, dev, pinned_host=True)
+        run = ssm.HostForward(shape, dev)
+        y_host = torch.empty(host["x"].shape, dtype=torch.float32).pin_memory()
+        run(host, y_host)  # warm
+        if world > 1:
+            dist.barrier()
+        t0 = time.perf_counter()
+        for _ in range(a.e2e_steps):
+            run(host, y_host)
+        el = reduce_max(time.perf_counter() - t0, dev)
+        line["e2e"] = {"value": weak_scaling_value(tokens * a.e2e_steps, world, el), "unit": UNIT,
+                       "h2d_bytes_per_step": run.h2d_bytes(), "d2h_bytes_per_step": run.d2h_bytes(),
+                       "steps": a.e2e_steps,
+                       "note": "pinned host x, z, params -> device, layer, y -> pinned host; per-step wall time"}
+        del run, host, y_host, dev_keep
+    else:
+        line["e2e"] = None
+
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, pool_axis)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    a = parse(argv)
+    from pooled_selective_scan_b200.configs import by_name
+    cfg = by_name(a.config)
+    pool_axis = cfg.pool_axes[0] if a.pool_axis is None else a.pool_axis
+    if a.impl == "reference":
+        return run_reference(a, cfg, pool_axis)
+    return run_ours(a, cfg, pool_axis)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,170 @@
+/*
+ * fastvim_ssm.h -- C ABI of the B200 (sm_100a) FastVim SSM layer, the "pooled selective scan".
+ *
+ * The layer (FastVim, Kapse et al., arXiv 2502.00594; gptget.net summary of the paper, section
+ * "方法详解" (method details), items 1-6, and glossary "State Space Model"):
+ *
+ *   1. grid index map   x[B][h][w][E] is the post-Conv1D activation of an h x w token grid
+ *                       (channels last).  No copy, transpose or flip is made: the pooled axis
+ *                       is the pool_axis flag, the scan direction is a loop order.
+ *   2. mean pooling     POOL_W: xbar[b][t] = pool_scale/w * sum_j x[b][t][j], T = h tokens
+ *                       ("(B,h,w,D) -> (B,h,1,D)");  POOL_H: mean over i, T = w tokens.
+ *   3. projections      per direction k: [dt_low | B | C] = W_x[k] xbar  (R, N, N values),
+ *                       Delta[e] = softplus(W_dt[k][e] . dt_low + b_dt[k][e]).
+ *   4. ZOH              A = -exp(A_log[k]);  Abar = exp(Delta A);  Bbar x = Delta B xbar
+ *                       (FV_FLAG_ZOH_EXACT: Bbar = (Abar - 1) / A * B).
+ *   5. scans            forward  h_t = Abar_t h_{t-1} + Bbar_t x_t, t = 0 .. T-1;
+ *                       backward the same for t = T-1 .. 0; both from a zero state;
+ *                       ys[t] = sum over enabled directions of C_t . h_t.
+ *   6. repeat+skip+gate y[b][i][j] = SiLU(z[b][i][j]) * (ys[b][t(i,j)] + (sum_k D[k]) * x[b][i][j])
+ *                       (pith.science verdict on 2502.00594, "key_machinery": the repeat comes
+ *                       before the D x skip; ijyty.com Vision Mamba article, section 2.1: the
+ *                       gate is applied to the sum of the two directions).
+ *   masked (FastMaskVim; "方法详解" item 6): x, z, y are [B][K][E] kept tokens with grid ids
+ *                       keep_idx[B][K] = r*w + c.  A kept token pools into row r (POOL_W) or
+ *                       column c (POOL_H); each pooled token is the sum of its kept tokens
+ *                       divided by the FIXED full length (w for POOL_W, h for POOL_H); an
+ *                       empty row pools to 0 and is still scanned; each kept token takes the
+ *                       output of its row.  Ids must be in [0, h*w) and unique per sample.
+ *
+ * Conventions for every entry point:
+ *   - All tensors are fp32 (keep_idx int32), row-major, and live in DEVICE memory unless an
+ *     entry point says otherwise.  Every pointer must be 16-byte aligned.
+ *   - Parameters are stacked per enabled direction on a leading nd axis (nd = number of bits
+ *     set in dir_flags), slot 0 = FWD when enabled, then BWD:
+ *       A_log [nd][E][N], D [nd][E], W_x [nd][R+2N][E] (rows dt_low | B | C),
+ *       W_dt [nd][E][R], b_dt [nd][E].
+ *   - Ownership: the caller allocates and frees every buffer, including the workspace.  The
+ *     library never allocates device memory, never frees, and (except fastvim_ssm_forward_host
+ *     and fastvim_get_device_status) never synchronises.  Work is queued on the caller's
+ *     stream (a cudaStream_t passed as void*, NULL = the legacy default stream).
+ *   - Errors: argument errors are detected on the host and returned before anything is
+ *     queued.  Launch failures return FV_ERR_CUDA (fastvim_last_error() has the CUDA
+ *     message).  Errors found on the device (a bad keep index) never trap: the kernels skip
+ *     the bad token, record FV_ERR_INDEX in the workspace, and fastvim_get_device_status()
+ *     reports it; the output of a call that recorded a device error is unspecified.
+ *   - Limits: E % 4 == 0, 1 <= N <= 16, 1 <= R, R + 2N <= 96, T <= 4096, h*w <= 2^20 for the
+ *     masked layer, and the per-image scan tile must fit in shared memory (checked; returns
+ *     FV_ERR_UNSUPPORTED otherwise).
+ */
+#ifndef FASTVIM_SSM_H
+#define FASTVIM_SSM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FASTVIM_SSM_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define FV_API __attribute__((visibility("default")))
+#else
+#define FV_API
+#endif
+
+typedef enum {
+    FV_OK = 0,
+    FV_ERR_NULL = 1,        /* a required pointer is NULL                                  */
+    FV_ERR_SHAPE = 2,       /* a size or flag is out of range                              */
+    FV_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned                            */
+    FV_ERR_INDEX = 4,       /* (device) a keep index is out of range or repeated           */
+    FV_ERR_WORKSPACE = 5,   /* workspace missing, too small or not 256-byte aligned        */
+    FV_ERR_CUDA = 6,        /* a CUDA call failed; see fastvim_last_error()                */
+    FV_ERR_TIMEOUT = 7,     /* (device) a bounded wait gave up                             */
+    FV_ERR_UNSUPPORTED = 8, /* valid layer, but beyond this build's limits                 */
+    FV_ERR_ALIAS = 9        /* y overlaps x or z                                           */
+} fv_status;
+
+enum { FV_POOL_W = 0, /* mean over w, T = h tokens (column pooling) */
+       FV_POOL_H = 1  /* mean over h, T = w tokens (row pooling)    */ };
+enum { FV_DIR_FWD = 1u, FV_DIR_BWD = 2u };
+enum { FV_FLAG_ZOH_EXACT = 1u /* Bbar = (exp(Delta A) - 1) / A * B instead of Delta B */ };
+
+typedef struct {
+    int B, h, w, E, N, R;    /* batch, grid height/width, channels, d_state, dt_rank        */
+    int pool_axis;           /* FV_POOL_W or FV_POOL_H                                       */
+    unsigned dir_flags;      /* FV_DIR_FWD | FV_DIR_BWD, at least one                        */
+    int K;                   /* kept tokens per sample (masked layer); 0 = dense grid        */
+    float pool_scale;        /* factor on the pooled mean; 0 is read as 1 (plain mean)       */
+    unsigned flags;          /* FV_FLAG_*                                                    */
+    const float* x;          /* dense [B][h][w][E] | masked [B][K][E]                        */
+    const float* z;          /* same shape as x                                              */
+    const float* A_log;      /* [nd][E][N]                                                   */
+    const float* D;          /* [nd][E]                                                      */
+    const float* W_x;        /* [nd][R+2N][E]                                                */
+    const float* W_dt;       /* [nd][E][R]                                                   */
+    const float* b_dt;       /* [nd][E]                                                      */
+    const int32_t* keep_idx; /* NULL (dense) or [B][K] grid ids r*w + c                      */
+    float* y;                /* same shape as x; must not overlap x or z                     */
+} fv_ssm_args;
+
+/* Byte offsets of the intermediates inside a workspace (for inspection and tests). */
+typedef struct {
+    size_t total_bytes;  /* what fastvim_ssm_workspace_size returns                          */
+    size_t status;       /* uint32 device status word                                        */
+    size_t xbar;         /* fp32 [B][T][E] pooled tokens                                     */
+    size_t u;            /* fp32 [nd][B][T][R+2N] projections dt_low | B | C                 */
+    size_t ys;           /* fp32 [B][T][E] scan output summed over directions                */
+    size_t row_of;       /* int32 [B][K] pooled row of each kept token (masked), else 0      */
+    size_t row_off;      /* int32 [B][T+1] CSR row offsets (masked), else 0                  */
+    size_t row_tok;      /* int32 [B][K] kept-token ordinals grouped by row, ascending       */
+    int T, S, nd;        /* pooled length, pooled-over length, number of directions          */
+} fv_ws_layout;
+
+/* Human-readable name of a status code (static string, never NULL). */
+FV_API const char* fastvim_status_string(fv_status s);
+
+/* Message of the last CUDA failure seen by this thread ("" if none). */
+FV_API const char* fastvim_last_error(void);
+
+/* ABI version (FASTVIM_SSM_ABI_VERSION). */
+FV_API int fastvim_abi_version(void);
+
+/* Host-side argument check of a forward call, without touching the GPU or dereferencing any
+ * tensor pointer.  Returns FV_OK or the first error found. */
+FV_API fv_status fastvim_ssm_validate(const fv_ssm_args* args);
+
+/* Workspace bytes a forward call needs (0 when the arguments are invalid). */
+FV_API size_t fastvim_ssm_workspace_size(const fv_ssm_args* args);
+
+/* Where each intermediate sits inside the workspace. */
+FV_API fv_status fastvim_ssm_workspace_layout(const fv_ssm_args* args, fv_ws_layout* out);
+
+/* Number of kernel launches one fastvim_ssm_forward call queues (memsets excluded; 0 when the
+ * arguments are invalid or B == 0). */
+FV_API int fastvim_ssm_launch_count(const fv_ssm_args* args);
+
+/* Name of the i-th kernel launch of a forward call ("" when out of range); static string. */
+FV_API const char* fastvim_ssm_launch_name(const fv_ssm_args* args, int i);
+
+/* The layer: queue pool -> projections -> scans -> repeat/skip/gate on `stream`.
+ * ws: device workspace of at least fastvim_ssm_workspace_size(args) bytes, 256-byte aligned,
+ * no initial contents required, not shared with a concurrently running call. */
+FV_API fv_status fastvim_ssm_forward(const fv_ssm_args* args, void* ws, size_t ws_bytes, void* stream);
+
+/* fastvim_ssm_forward with timing marks: `events` holds n_events >= launch_count + 1 CUDA
+ * events (cudaEvent_t, created by the caller); events[i] is recorded on `stream` just before
+ * the i-th kernel launch and events[launch_count] after the last one, so the elapsed time
+ * between events i and i+1 is the device duration of launch i.  Same results as
+ * fastvim_ssm_forward. */
+FV_API fv_status fastvim_ssm_forward_events(const fv_ssm_args* args, void* ws, size_t ws_bytes,
+                                            void* stream, void* const* events, int n_events);
+
+/* End-to-end variant for host-resident data.  `host` names pinned HOST buffers for x, z,
+ * the parameters, keep_idx and y; `dev` names DEVICE buffers of the same shapes (its sizes
+ * and flags must equal host's).  Copies the inputs host -> device, runs the layer, copies y
+ * device -> host and waits for the stream, so y is ready in host memory on return. */
+FV_API fv_status fastvim_ssm_forward_host(const fv_ssm_args* host, const fv_ssm_args* dev, void* ws,
+                                   size_t ws_bytes, void* stream);
+
+/* Waits for `stream`, then reads the device status word of a workspace used by the last
+ * forward call: FV_OK, FV_ERR_INDEX or FV_ERR_TIMEOUT (or FV_ERR_CUDA if the read fails). */
+FV_API fv_status fastvim_get_device_status(const void* ws, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FASTVIM_SSM_H */

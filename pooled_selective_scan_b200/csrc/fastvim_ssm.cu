@@ -1,0 +1,383 @@
+// fastvim_ssm.cu -- C ABI of the FastVim SSM layer: validation, workspace planning, launches.
+// The layer's definition, the argument layouts and the error contract are in fastvim_ssm.h.
+#include "fastvim_ssm.h"
+
+#include <stdio.h>
+#include <string.h>
+
+#include "fv_common.cuh"
+#include "fv_kernels.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+void note_cuda(cudaError_t e, const char* where) {
+    snprintf(g_last_error, sizeof g_last_error, "%s: %s (%d)", where, cudaGetErrorString(e), (int)e);
+}
+
+int popc2(unsigned f) { return (int)((f & 1u) != 0) + (int)((f & 2u) != 0); }
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+size_t round256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+constexpr int kMaxT = 4096;
+constexpr long long kMaxMaskGrid = 1ll << 20;
+
+// Lanes per (direction, channel) in the scan: 4 states per lane.
+int scan_lanes(int N) { return N <= 4 ? 1 : (N <= 8 ? 2 : 4); }
+
+size_t scan_smem_bytes(const fv::Shape& sh) {
+    return fv::scan_smem_floats(sh.T, sh.J, sh.R, scan_lanes(sh.N), sh.nd) * sizeof(float);
+}
+size_t proj_smem_bytes(const fv::Shape& sh) {
+    return (size_t)(fv::kProjRows * 33 + sh.NJ * 33) * sizeof(float);
+}
+size_t bucket_smem_bytes(const fv::Shape& sh) {
+    const long long G = (long long)sh.h * sh.w;
+    return (size_t)(((G + 31) >> 5) + 2ll * sh.T) * sizeof(unsigned);
+}
+
+int max_optin_smem() {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 0;
+    return v;
+}
+
+// Sizes and flags only; no pointer is dereferenced.
+fv_status make_shape(const fv_ssm_args* a, fv::Shape* sh) {
+    if (!a) return FV_ERR_NULL;
+    if (a->B < 0 || a->h < 1 || a->w < 1 || a->E < 4 || a->N < 1 || a->R < 1) return FV_ERR_SHAPE;
+    if (a->pool_axis != FV_POOL_W && a->pool_axis != FV_POOL_H) return FV_ERR_SHAPE;
+    if (a->dir_flags == 0 || (a->dir_flags & ~3u) != 0) return FV_ERR_SHAPE;
+    if ((a->flags & ~(unsigned)FV_FLAG_ZOH_EXACT) != 0) return FV_ERR_SHAPE;
+    if (a->E % 4 != 0) return FV_ERR_SHAPE;
+    if (a->K < 0 || (long long)a->K > (long long)a->h * a->w) return FV_ERR_SHAPE;
+    if (!(a->pool_scale == a->pool_scale) || a->pool_scale > 3.0e38f || a->pool_scale < -3.0e38f)
+        return FV_ERR_SHAPE;
+    if (a->N > fv::kMaxN || a->R + 2 * a->N > fv::kMaxJ) return FV_ERR_UNSUPPORTED;
+    const long long tok = a->K > 0 ? (long long)a->K : (long long)a->h * a->w;
+    if ((long long)a->B * tok * a->E >= (1ll << 40)) return FV_ERR_UNSUPPORTED;
+    sh->B = a->B; sh->h = a->h; sh->w = a->w; sh->E = a->E; sh->N = a->N; sh->R = a->R;
+    sh->pool_axis = a->pool_axis;
+    sh->T = a->pool_axis == FV_POOL_W ? a->h : a->w;
+    sh->S = a->pool_axis == FV_POOL_W ? a->w : a->h;
+    sh->nd = popc2(a->dir_flags);
+    sh->J = a->R + 2 * a->N;
+    sh->NJ = sh->nd * sh->J;
+    sh->K = a->K;
+    sh->dir_flags = a->dir_flags;
+    sh->zoh_exact = (a->flags & FV_FLAG_ZOH_EXACT) ? 1 : 0;
+    sh->pool_scale = a->pool_scale == 0.f ? 1.f : a->pool_scale;
+    sh->SL = a->E / 4;
+    if (sh->T > kMaxT) return FV_ERR_UNSUPPORTED;
+    if (a->K > 0 && (long long)a->h * a->w > kMaxMaskGrid) return FV_ERR_UNSUPPORTED;
+    if ((long long)sh->B * sh->T >= (1ll << 31)) return FV_ERR_UNSUPPORTED;
+    return FV_OK;
+}
+
+fv_status check_pointers(const fv_ssm_args* a, const fv::Shape& sh) {
+    if (!a->A_log || !a->D || !a->W_x || !a->W_dt || !a->b_dt) return FV_ERR_NULL;
+    if (sh.B > 0 && (!a->x || !a->z || !a->y)) return FV_ERR_NULL;
+    if (sh.K > 0 && sh.B > 0 && !a->keep_idx) return FV_ERR_NULL;
+    if (sh.K == 0 && a->keep_idx) return FV_ERR_SHAPE;  // a keep list needs K
+    const void* ps[] = {a->x, a->z, a->y, a->A_log, a->D, a->W_x, a->W_dt, a->b_dt, a->keep_idx};
+    for (const void* p : ps)
+        if (p && !aligned16(p)) return FV_ERR_ALIGN;
+    if (sh.B > 0) {
+        const size_t tok = sh.K > 0 ? (size_t)sh.K : (size_t)sh.h * sh.w;
+        const size_t bytes = (size_t)sh.B * tok * sh.E * sizeof(float);
+        const uintptr_t y0 = (uintptr_t)a->y, y1 = y0 + bytes;
+        const uintptr_t x0 = (uintptr_t)a->x, z0 = (uintptr_t)a->z;
+        if ((x0 < y1 && y0 < x0 + bytes) || (z0 < y1 && y0 < z0 + bytes)) return FV_ERR_ALIAS;
+    }
+    return FV_OK;
+}
+
+fv_status plan_layout(const fv::Shape& sh, fv_ws_layout* L) {
+    memset(L, 0, sizeof *L);
+    size_t off = 0;
+    L->status = off; off = round256(off + sizeof(unsigned));
+    L->xbar = off; off = round256(off + (size_t)sh.B * sh.T * sh.E * sizeof(float));
+    L->u = off; off = round256(off + (size_t)sh.nd * sh.B * sh.T * sh.J * sizeof(float));
+    L->ys = off; off = round256(off + (size_t)sh.B * sh.T * sh.E * sizeof(float));
+    if (sh.K > 0) {
+        L->row_of = off; off = round256(off + (size_t)sh.B * sh.K * sizeof(int32_t));
+        L->row_off = off; off = round256(off + (size_t)sh.B * (sh.T + 1) * sizeof(int32_t));
+        L->row_tok = off; off = round256(off + (size_t)sh.B * sh.K * sizeof(int32_t));
+    }
+    L->total_bytes = off;
+    L->T = sh.T; L->S = sh.S; L->nd = sh.nd;
+    return FV_OK;
+}
+
+fv_status check_limits(const fv::Shape& sh) {
+    const size_t optin = (size_t)max_optin_smem();
+    const size_t lim = optin ? optin : (size_t)(227 * 1024);
+    if (scan_smem_bytes(sh) > lim) return FV_ERR_UNSUPPORTED;
+    if (sh.K > 0 && bucket_smem_bytes(sh) > lim) return FV_ERR_UNSUPPORTED;
+    return FV_OK;
+}
+
+// Kernels that take more than 48 KB of dynamic shared memory need an opt-in per device.
+template <typename Kern>
+cudaError_t ensure_smem(Kern kernel, size_t bytes) {
+    if (bytes <= 48 * 1024) return cudaSuccess;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+#define FV_LAUNCH_CHECK(where)                         \
+    do {                                               \
+        cudaError_t e_ = cudaGetLastError();           \
+        if (e_ != cudaSuccess) {                       \
+            note_cuda(e_, where);                      \
+            return FV_ERR_CUDA;                        \
+        }                                              \
+    } while (0)
+
+template <int G, int ND, bool Z>
+fv_status launch_scan_t(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws,
+                        cudaStream_t st) {
+    constexpr int ECH = fv::scan_ech<G, ND>();
+    const size_t smem = scan_smem_bytes(sh);
+    auto kern = fv::scan_kernel<G, ND, Z>;
+    cudaError_t e = ensure_smem(kern, smem);
+    if (e != cudaSuccess) { note_cuda(e, "scan smem attribute"); return FV_ERR_CUDA; }
+    const int ntile = (sh.E + ECH - 1) / ECH;
+    kern<<<sh.B * ntile, fv::kThreads, smem, st>>>(sh, (const float*)(ws + L.xbar), (const float*)(ws + L.u),
+                                                  a->A_log, a->W_dt, a->b_dt, (float*)(ws + L.ys));
+    FV_LAUNCH_CHECK("scan_kernel");
+    return FV_OK;
+}
+
+template <int G, int ND>
+fv_status launch_scan_z(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st) {
+    return sh.zoh_exact ? launch_scan_t<G, ND, true>(sh, a, L, ws, st) : launch_scan_t<G, ND, false>(sh, a, L, ws, st);
+}
+
+template <int G>
+fv_status launch_scan_g(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st) {
+    return sh.nd == 2 ? launch_scan_z<G, 2>(sh, a, L, ws, st) : launch_scan_z<G, 1>(sh, a, L, ws, st);
+}
+
+fv_status launch_scan(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st) {
+    switch (scan_lanes(sh.N)) {
+        case 1: return launch_scan_g<1>(sh, a, L, ws, st);
+        case 2: return launch_scan_g<2>(sh, a, L, ws, st);
+        default: return launch_scan_g<4>(sh, a, L, ws, st);
+    }
+}
+
+// Records events[i] just before the i-th kernel launch and events[n] after the last one when an
+// event list is given (n = the call's launch count).
+struct EventMarks {
+    void* const* ev;
+    int n, next;
+    cudaError_t mark(cudaStream_t st) {
+        if (!ev || next > n) return cudaSuccess;
+        return cudaEventRecord((cudaEvent_t)ev[next++], st);
+    }
+};
+
+#define FV_MARK(marks, st)                                   \
+    do {                                                     \
+        cudaError_t e_ = (marks).mark(st);                   \
+        if (e_ != cudaSuccess) {                             \
+            note_cuda(e_, "event record");                   \
+            return FV_ERR_CUDA;                              \
+        }                                                    \
+    } while (0)
+
+int launch_count_of(const fv::Shape& sh) { return sh.B == 0 ? 0 : (sh.K > 0 ? 5 : 4); }
+
+const char* launch_name_of(const fv::Shape& sh, int i) {
+    static const char* dense[] = {"pool_dense_kernel", "proj_kernel", "scan_kernel", "epilogue_dense_kernel"};
+    static const char* masked[] = {"mask_bucket_kernel", "mask_pool_kernel", "proj_kernel", "scan_kernel",
+                                   "mask_epilogue_kernel"};
+    if (i < 0 || i >= launch_count_of(sh)) return "";
+    return sh.K > 0 ? masked[i] : dense[i];
+}
+
+fv_status forward_impl(const fv_ssm_args* a, void* ws_v, size_t ws_bytes, cudaStream_t st,
+                       void* const* events = nullptr, int n_events = 0) {
+    fv::Shape sh;
+    fv_status s = make_shape(a, &sh);
+    if (s != FV_OK) return s;
+    if ((s = check_pointers(a, sh)) != FV_OK) return s;
+    fv_ws_layout L;
+    plan_layout(sh, &L);
+    if (!ws_v || ws_bytes < L.total_bytes || ((uintptr_t)ws_v & 255u) != 0) return FV_ERR_WORKSPACE;
+    if ((s = check_limits(sh)) != FV_OK) return s;
+    if (events && n_events < launch_count_of(sh) + 1) return FV_ERR_SHAPE;
+    EventMarks marks{events, launch_count_of(sh), 0};
+    char* ws = (char*)ws_v;
+    unsigned* status = (unsigned*)(ws + L.status);
+    if (sh.B == 0) {
+        cudaError_t e = cudaMemsetAsync(status, 0, sizeof(unsigned), st);
+        if (e != cudaSuccess) { note_cuda(e, "status reset"); return FV_ERR_CUDA; }
+        return FV_OK;
+    }
+    const int M = sh.B * sh.T;
+    float* xbar = (float*)(ws + L.xbar);
+    if (sh.K == 0) {
+        FV_MARK(marks, st);
+        fv::pool_dense_kernel<<<M, fv::kThreads, 0, st>>>(sh, a->x, xbar, status);
+        FV_LAUNCH_CHECK("pool_dense_kernel");
+    } else {
+        cudaError_t e = cudaMemsetAsync(status, 0, sizeof(unsigned), st);
+        if (e != cudaSuccess) { note_cuda(e, "status reset"); return FV_ERR_CUDA; }
+        const size_t bsm = bucket_smem_bytes(sh);
+        e = ensure_smem(fv::mask_bucket_kernel, bsm);
+        if (e != cudaSuccess) { note_cuda(e, "bucket smem attribute"); return FV_ERR_CUDA; }
+        FV_MARK(marks, st);
+        fv::mask_bucket_kernel<<<sh.B, fv::kThreads, bsm, st>>>(sh, a->keep_idx, (int32_t*)(ws + L.row_of),
+                                                                (int32_t*)(ws + L.row_off),
+                                                                (int32_t*)(ws + L.row_tok), status);
+        FV_LAUNCH_CHECK("mask_bucket_kernel");
+        FV_MARK(marks, st);
+        fv::mask_pool_kernel<<<M, fv::kThreads, 0, st>>>(sh, a->x, (const int32_t*)(ws + L.row_off),
+                                                         (const int32_t*)(ws + L.row_tok), xbar);
+        FV_LAUNCH_CHECK("mask_pool_kernel");
+    }
+    FV_MARK(marks, st);
+    fv::proj_kernel<<<(M + fv::kProjRows - 1) / fv::kProjRows, fv::kThreads, proj_smem_bytes(sh), st>>>(
+        sh, xbar, a->W_x, (float*)(ws + L.u));
+    FV_LAUNCH_CHECK("proj_kernel");
+    FV_MARK(marks, st);
+    if ((s = launch_scan(sh, a, L, ws, st)) != FV_OK) return s;
+    FV_MARK(marks, st);
+    if (sh.K == 0) {
+        fv::epilogue_dense_kernel<<<M, fv::kThreads, 0, st>>>(sh, a->x, a->z, (const float*)(ws + L.ys), a->D, a->y);
+        FV_LAUNCH_CHECK("epilogue_dense_kernel");
+    } else {
+        const int nkb = (sh.K + fv::kMaskEpiTokens - 1) / fv::kMaskEpiTokens;
+        fv::mask_epilogue_kernel<<<sh.B * nkb, fv::kThreads, 0, st>>>(sh, a->x, a->z, (const float*)(ws + L.ys),
+                                                                     a->D, (const int32_t*)(ws + L.row_of), a->y);
+        FV_LAUNCH_CHECK("mask_epilogue_kernel");
+    }
+    FV_MARK(marks, st);
+    return FV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fastvim_status_string(fv_status s) {
+    switch (s) {
+        case FV_OK: return "FV_OK";
+        case FV_ERR_NULL: return "FV_ERR_NULL: a required pointer is NULL";
+        case FV_ERR_SHAPE: return "FV_ERR_SHAPE: a size or flag is out of range";
+        case FV_ERR_ALIGN: return "FV_ERR_ALIGN: a pointer is not 16-byte aligned";
+        case FV_ERR_INDEX: return "FV_ERR_INDEX: a keep index is out of range or repeated";
+        case FV_ERR_WORKSPACE: return "FV_ERR_WORKSPACE: workspace missing, too small or misaligned";
+        case FV_ERR_CUDA: return "FV_ERR_CUDA: a CUDA call failed";
+        case FV_ERR_TIMEOUT: return "FV_ERR_TIMEOUT: a bounded device wait gave up";
+        case FV_ERR_UNSUPPORTED: return "FV_ERR_UNSUPPORTED: beyond this build's limits";
+        case FV_ERR_ALIAS: return "FV_ERR_ALIAS: y overlaps x or z";
+    }
+    return "unknown fv_status";
+}
+
+const char* fastvim_last_error(void) { return g_last_error; }
+
+int fastvim_abi_version(void) { return FASTVIM_SSM_ABI_VERSION; }
+
+fv_status fastvim_ssm_validate(const fv_ssm_args* args) {
+    fv::Shape sh;
+    fv_status s = make_shape(args, &sh);
+    if (s != FV_OK) return s;
+    return check_pointers(args, sh);
+}
+
+size_t fastvim_ssm_workspace_size(const fv_ssm_args* args) {
+    fv::Shape sh;
+    if (make_shape(args, &sh) != FV_OK) return 0;
+    fv_ws_layout L;
+    plan_layout(sh, &L);
+    return L.total_bytes;
+}
+
+fv_status fastvim_ssm_workspace_layout(const fv_ssm_args* args, fv_ws_layout* out) {
+    if (!out) return FV_ERR_NULL;
+    fv::Shape sh;
+    fv_status s = make_shape(args, &sh);
+    if (s != FV_OK) return s;
+    return plan_layout(sh, out);
+}
+
+int fastvim_ssm_launch_count(const fv_ssm_args* args) {
+    fv::Shape sh;
+    if (make_shape(args, &sh) != FV_OK) return 0;
+    return launch_count_of(sh);
+}
+
+const char* fastvim_ssm_launch_name(const fv_ssm_args* args, int i) {
+    fv::Shape sh;
+    if (make_shape(args, &sh) != FV_OK) return "";
+    return launch_name_of(sh, i);
+}
+
+fv_status fastvim_ssm_forward(const fv_ssm_args* args, void* ws, size_t ws_bytes, void* stream) {
+    return forward_impl(args, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+fv_status fastvim_ssm_forward_events(const fv_ssm_args* args, void* ws, size_t ws_bytes, void* stream,
+                                     void* const* events, int n_events) {
+    if (!events) return FV_ERR_NULL;
+    return forward_impl(args, ws, ws_bytes, (cudaStream_t)stream, events, n_events);
+}
+
+fv_status fastvim_ssm_forward_host(const fv_ssm_args* host, const fv_ssm_args* dev, void* ws,
+                                   size_t ws_bytes, void* stream) {
+    if (!host || !dev) return FV_ERR_NULL;
+    fv::Shape sh, shd;
+    fv_status s = make_shape(host, &sh);
+    if (s != FV_OK) return s;
+    if ((s = make_shape(dev, &shd)) != FV_OK) return s;
+    if (host->B != dev->B || host->h != dev->h || host->w != dev->w || host->E != dev->E ||
+        host->N != dev->N || host->R != dev->R || host->K != dev->K || host->pool_axis != dev->pool_axis ||
+        host->dir_flags != dev->dir_flags || host->flags != dev->flags || host->pool_scale != dev->pool_scale)
+        return FV_ERR_SHAPE;
+    if ((s = check_pointers(host, sh)) != FV_OK) return s;
+    if ((s = check_pointers(dev, shd)) != FV_OK) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t tok = sh.K > 0 ? (size_t)sh.K : (size_t)sh.h * sh.w;
+    const size_t act = (size_t)sh.B * tok * sh.E * sizeof(float);
+    const size_t nd = (size_t)sh.nd;
+    struct Copy { void* dst; const void* src; size_t bytes; } copies[] = {
+        {(void*)dev->x, host->x, act},
+        {(void*)dev->z, host->z, act},
+        {(void*)dev->A_log, host->A_log, nd * sh.E * sh.N * sizeof(float)},
+        {(void*)dev->D, host->D, nd * sh.E * sizeof(float)},
+        {(void*)dev->W_x, host->W_x, nd * sh.J * sh.E * sizeof(float)},
+        {(void*)dev->W_dt, host->W_dt, nd * sh.E * sh.R * sizeof(float)},
+        {(void*)dev->b_dt, host->b_dt, nd * sh.E * sizeof(float)},
+        {(void*)dev->keep_idx, host->keep_idx, sh.K > 0 ? (size_t)sh.B * sh.K * sizeof(int32_t) : 0},
+    };
+    for (const Copy& c : copies) {
+        if (c.bytes == 0 || !c.dst) continue;
+        cudaError_t e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, st);
+        if (e != cudaSuccess) { note_cuda(e, "host->device copy"); return FV_ERR_CUDA; }
+    }
+    if ((s = forward_impl(dev, ws, ws_bytes, st)) != FV_OK) return s;
+    if (act > 0) {
+        cudaError_t e = cudaMemcpyAsync(host->y, dev->y, act, cudaMemcpyDeviceToHost, st);
+        if (e != cudaSuccess) { note_cuda(e, "device->host copy"); return FV_ERR_CUDA; }
+    }
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) { note_cuda(e, "stream synchronize"); return FV_ERR_CUDA; }
+    return FV_OK;
+}
+
+fv_status fastvim_get_device_status(const void* ws, void* stream) {
+    if (!ws) return FV_ERR_NULL;
+    cudaStream_t st = (cudaStream_t)stream;
+    unsigned v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) { note_cuda(e, "status read"); return FV_ERR_CUDA; }
+    return (fv_status)v;
+}
+
+}  // extern "C"

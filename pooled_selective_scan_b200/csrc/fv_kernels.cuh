@@ -1,0 +1,445 @@
+// fv_kernels.cuh -- the staged kernels of the FastVim SSM layer (sm_100a, fp32).
+//
+// Step map (FastVim, arXiv 2502.00594; gptget.net summary of the paper, section "方法详解"):
+//   pool_dense_kernel / mask_bucket_kernel + mask_pool_kernel   item 2 (and item 6, masked)
+//   proj_kernel                                                 item 3 (x_proj)
+//   scan_kernel                                                 items 3-4 (dt_proj + softplus,
+//                                                               ZOH, forward/backward scans)
+//   epilogue_dense_kernel / mask_epilogue_kernel                item 5 (repeat, skip, gate)
+// The work is HBM-streaming except the projection and the scan, which are small; none of it
+// is a dense contraction large enough for tensor cores (the x_proj GEMM has N = nd(R+2N) <= 192
+// columns and K = E, and must stay fp32 to meet the layer's tolerance).
+#pragma once
+
+#include "fv_common.cuh"
+
+namespace fv {
+
+// ------------------------------------------------------------------------------------------
+// Pooling
+// ------------------------------------------------------------------------------------------
+
+// Sum of tokens s0, s0+G, s0+2G, ... < S of one float4 column; four loads in flight.
+__device__ __forceinline__ float4 sum_line(const float4* __restrict__ p, size_t st4, int s0, int G,
+                                           int S) {
+    float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+    int s = s0;
+    for (; s + 3 * G < S; s += 4 * G) {
+        const float4 v0 = ld_stream(p + (size_t)s * st4);
+        const float4 v1 = ld_stream(p + (size_t)(s + G) * st4);
+        const float4 v2 = ld_stream(p + (size_t)(s + 2 * G) * st4);
+        const float4 v3 = ld_stream(p + (size_t)(s + 3 * G) * st4);
+        f4_add(a0, v0); f4_add(a1, v1); f4_add(a0, v2); f4_add(a1, v3);
+    }
+    for (; s < S; s += G) f4_add(a0, ld_stream(p + (size_t)s * st4));
+    f4_add(a0, a1);
+    return a0;
+}
+
+__device__ __forceinline__ float4 f4_scale(float4 v, float s) {
+    return make_float4(v.x * s, v.y * s, v.z * s, v.w * s);
+}
+
+// One CTA per pooled token (b, t): mean of the S grid tokens of line t, 128-bit loads, no copy
+// or transpose of the grid (the pooled axis only changes the base/stride of the index map).
+__global__ void __launch_bounds__(kThreads)
+pool_dense_kernel(Shape sh, const float* __restrict__ x, float* __restrict__ xbar, unsigned* status) {
+    __shared__ float4 part[kThreads];
+    const int bt = blockIdx.x;
+    const int b = bt / sh.T, t = bt - b * sh.T;
+    if (bt == 0 && threadIdx.x == 0) *status = 0u;  // a dense call records no device error
+    const float4* base = reinterpret_cast<const float4*>(x + dense_base(sh, b, t));
+    const size_t st4 = dense_stride(sh) >> 2;
+    const float scale = sh.pool_scale / (float)sh.S;
+    float4* out = reinterpret_cast<float4*>(xbar + (size_t)bt * sh.E);
+    const int SL = sh.SL;
+    if (SL <= kThreads) {
+        const int G = kThreads / SL;
+        const int slot = threadIdx.x % SL, g = threadIdx.x / SL;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (g < G) acc = sum_line(base + slot, st4, g, G, sh.S);
+        part[threadIdx.x] = acc;
+        __syncthreads();
+        if (threadIdx.x < SL) {
+            float4 s = part[threadIdx.x];
+            for (int q = 1; q < G; ++q) f4_add(s, part[q * SL + threadIdx.x]);
+            out[threadIdx.x] = f4_scale(s, scale);
+        }
+    } else {
+        for (int slot = threadIdx.x; slot < SL; slot += kThreads)
+            out[slot] = f4_scale(sum_line(base + slot, st4, 0, 1, sh.S), scale);
+    }
+}
+
+// Per-sample row bucketing of kept-token ids (one CTA per sample).  Validates every id (in
+// range, not repeated), writes row_of[k] (-1 for a rejected id), the CSR offsets row_off[0..T]
+// and row_tok (the sample's kept-token ordinals grouped by row, ascending k inside a row; the
+// tail past the valid count is -1).  The stable scatter runs in one warp, 32 ids at a time,
+// ranking equal rows with __match_any_sync, so the result does not depend on timing.
+__global__ void __launch_bounds__(kThreads)
+mask_bucket_kernel(Shape sh, const int32_t* __restrict__ keep_idx, int32_t* row_of, int32_t* row_off,
+                   int32_t* row_tok, unsigned* status) {
+    extern __shared__ unsigned smem_u[];
+    const int G = sh.h * sh.w;
+    const int nwords = (G + 31) >> 5;
+    const int T = sh.T, K = sh.K;
+    unsigned* bitmap = smem_u;
+    int* cnt = reinterpret_cast<int*>(bitmap + nwords);  // [T]
+    int* cursor = cnt + T;                               // [T]
+    const int b = blockIdx.x;
+    int32_t* rof = row_of + (size_t)b * K;
+    for (int i = threadIdx.x; i < nwords; i += kThreads) bitmap[i] = 0u;
+    for (int i = threadIdx.x; i < T; i += kThreads) cnt[i] = 0;
+    __syncthreads();
+    bool bad = false;
+    for (int k = threadIdx.x; k < K; k += kThreads) {
+        const int g = keep_idx[(size_t)b * K + k];
+        int r = -1;
+        if (g >= 0 && g < G) {
+            const unsigned bit = 1u << (g & 31);
+            const unsigned old = atomicOr(&bitmap[g >> 5], bit);
+            if (!(old & bit)) r = (sh.pool_axis == 0) ? g / sh.w : g % sh.w;
+        }
+        if (r < 0) bad = true;
+        else atomicAdd(&cnt[r], 1);
+        rof[k] = r;
+    }
+    if (bad) set_status(status, kStatusIndex);
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        int32_t* off = row_off + (size_t)b * (T + 1);
+        int carry = 0;
+        for (int base = 0; base < T; base += 32) {
+            const int r = base + lane;
+            const int v = (r < T) ? cnt[r] : 0;
+            int incl = v;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, incl, d);
+                if (lane >= d) incl += n;
+            }
+            if (r < T) {
+                cursor[r] = carry + incl - v;
+                off[r] = carry + incl - v;
+            }
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) off[T] = carry;
+        __syncwarp();
+        int32_t* tok = row_tok + (size_t)b * K;
+        const unsigned lt = (1u << lane) - 1u;
+        for (int k0 = 0; k0 < K; k0 += 32) {
+            const int k = k0 + lane;
+            const int r = (k < K) ? rof[k] : -1;
+            const unsigned peers = __match_any_sync(0xffffffffu, r);
+            const int rank = __popc(peers & lt);
+            const int pos = (r >= 0) ? cursor[r] + rank : 0;
+            __syncwarp();
+            if (r >= 0) {
+                tok[pos] = k;
+                if (lane == 31 - __clz(peers)) cursor[r] = pos + 1;
+            }
+            __syncwarp();
+        }
+        for (int p = carry + lane; p < K; p += 32) tok[p] = -1;
+    }
+}
+
+// One CTA per pooled row (b, t) of a masked sample: sum of the row's kept tokens divided by the
+// fixed full length S (an empty row pools to 0).
+__global__ void __launch_bounds__(kThreads)
+mask_pool_kernel(Shape sh, const float* __restrict__ x, const int32_t* __restrict__ row_off,
+                 const int32_t* __restrict__ row_tok, float* __restrict__ xbar) {
+    __shared__ float4 part[kThreads];
+    const int bt = blockIdx.x;
+    const int b = bt / sh.T, t = bt - b * sh.T;
+    const int32_t* off = row_off + (size_t)b * (sh.T + 1);
+    const int p0 = off[t], p1 = off[t + 1];
+    const int32_t* tok = row_tok + (size_t)b * sh.K;
+    const float4* xb = reinterpret_cast<const float4*>(x + (size_t)b * sh.K * sh.E);
+    const float scale = sh.pool_scale / (float)sh.S;
+    float4* out = reinterpret_cast<float4*>(xbar + (size_t)bt * sh.E);
+    const int SL = sh.SL;
+    if (SL <= kThreads) {
+        const int G = kThreads / SL;
+        const int slot = threadIdx.x % SL, g = threadIdx.x / SL;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (g < G)
+            for (int p = p0 + g; p < p1; p += G) f4_add(acc, ld_stream(xb + (size_t)tok[p] * SL + slot));
+        part[threadIdx.x] = acc;
+        __syncthreads();
+        if (threadIdx.x < SL) {
+            float4 s = part[threadIdx.x];
+            for (int q = 1; q < G; ++q) f4_add(s, part[q * SL + threadIdx.x]);
+            out[threadIdx.x] = f4_scale(s, scale);
+        }
+    } else {
+        for (int slot = threadIdx.x; slot < SL; slot += kThreads) {
+            float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+            int p = p0;
+            for (; p + 1 < p1; p += 2) {
+                const float4 v0 = ld_stream(xb + (size_t)tok[p] * SL + slot);
+                const float4 v1 = ld_stream(xb + (size_t)tok[p + 1] * SL + slot);
+                f4_add(a0, v0); f4_add(a1, v1);
+            }
+            if (p < p1) f4_add(a0, ld_stream(xb + (size_t)tok[p] * SL + slot));
+            f4_add(a0, a1);
+            out[slot] = f4_scale(a0, scale);
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// x_proj: u[k][m][0:J] = W_x[k] . xbar[m] for the pooled tokens m = b*T + t (fp32 FFMA).
+// One CTA per 32 pooled tokens, all nd*J outputs; channels staged 32 at a time in shared memory.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads)
+proj_kernel(Shape sh, const float* __restrict__ xbar, const float* __restrict__ W_x, float* __restrict__ u) {
+    extern __shared__ float smem_f[];
+    float* xs = smem_f;                        // [32][33]
+    float* wsm = smem_f + kProjRows * 33;      // [NJ][33]
+    const int M = sh.B * sh.T, E = sh.E, NJ = sh.NJ, J = sh.J;
+    const int m0 = blockIdx.x * kProjRows;
+    const int ml = threadIdx.x & 31, jg = threadIdx.x >> 5;
+    float acc[kProjQ];
+#pragma unroll
+    for (int q = 0; q < kProjQ; ++q) acc[q] = 0.f;
+    for (int e0 = 0; e0 < E; e0 += kProjChunk) {
+        for (int i = threadIdx.x; i < kProjRows * kProjChunk; i += kThreads) {
+            const int r = i >> 5, c = i & 31;
+            const int m = m0 + r, e = e0 + c;
+            xs[r * 33 + c] = (m < M && e < E) ? xbar[(size_t)m * E + e] : 0.f;
+        }
+        for (int i = threadIdx.x; i < NJ * kProjChunk; i += kThreads) {
+            const int jj = i >> 5, c = i & 31;
+            const int e = e0 + c;
+            wsm[jj * 33 + c] = (e < E) ? W_x[(size_t)jj * E + e] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int c = 0; c < kProjChunk; ++c) {
+            const float xv = xs[ml * 33 + c];
+#pragma unroll
+            for (int q = 0; q < kProjQ; ++q) {
+                const int jj = jg + 8 * q;
+                if (jj < NJ) acc[q] = fmaf(wsm[jj * 33 + c], xv, acc[q]);
+            }
+        }
+        __syncthreads();
+    }
+    const int m = m0 + ml;
+    if (m < M) {
+#pragma unroll
+        for (int q = 0; q < kProjQ; ++q) {
+            const int jj = jg + 8 * q;
+            if (jj < NJ) {
+                const int k = jj / J, j = jj - k * J;
+                u[((size_t)k * M + m) * J + j] = acc[q];
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// dt_proj + softplus, ZOH and the forward/backward selective scans in one launch.
+// One CTA per (image b, tile of ECH channels).  Thread = (state group g, direction kd, channel c):
+// G lanes of 4 states each cover the N <= 16 states of one (kd, c), so the state lives in
+// registers and is never written; the G partial C.h sums meet through __shfl_xor, and the two
+// directions meet in a shared-memory accumulator (two fp32 adds onto zero commute exactly, so
+// the sum does not depend on their order).
+// ------------------------------------------------------------------------------------------
+template <int G, int ND>
+__host__ __device__ constexpr int scan_ech() { return kThreads / (G * ND); }
+
+__host__ __forceinline__ size_t scan_smem_floats(int T, int J, int R, int G, int ND) {
+    const int ech = kThreads / (G * ND);
+    return (size_t)ND * T * J + (size_t)T * ech + (size_t)ND * T * ech + (size_t)ND * ech * R +
+           (size_t)T * ech;
+}
+
+template <int G, int ND, bool ZOH_EXACT>
+__global__ void __launch_bounds__(kThreads)
+scan_kernel(Shape sh, const float* __restrict__ xbar, const float* __restrict__ u,
+            const float* __restrict__ A_log, const float* __restrict__ W_dt,
+            const float* __restrict__ b_dt, float* __restrict__ ys) {
+    constexpr int ECH = scan_ech<G, ND>();
+    extern __shared__ float smem_f[];
+    const int T = sh.T, J = sh.J, R = sh.R, N = sh.N, E = sh.E;
+    const int M = sh.B * T;
+    const int ntile = (E + ECH - 1) / ECH;
+    const int b = blockIdx.x / ntile;
+    const int e0 = (blockIdx.x - b * ntile) * ECH;
+    float* us = smem_f;                  // [ND][T][J]   projections of this image
+    float* xs = us + ND * T * J;         // [T][ECH]     pooled tokens, this channel tile
+    float* dts = xs + T * ECH;           // [ND][T][ECH] Delta
+    float* wdt = dts + ND * T * ECH;     // [ND][ECH][R] dt_proj rows of this tile
+    float* ysum = wdt + ND * ECH * R;    // [T][ECH]     output, summed over directions
+
+    for (int k = 0; k < ND; ++k) {
+        const float* src = u + ((size_t)k * M + (size_t)b * T) * J;
+        for (int i = threadIdx.x; i < T * J; i += kThreads) us[k * T * J + i] = src[i];
+    }
+    for (int i = threadIdx.x; i < T * ECH; i += kThreads) {
+        const int t = i / ECH, c = i - t * ECH;
+        const int e = e0 + c;
+        xs[i] = (e < E) ? xbar[((size_t)b * T + t) * E + e] : 0.f;
+        ysum[i] = 0.f;
+    }
+    for (int i = threadIdx.x; i < ND * ECH * R; i += kThreads) {
+        const int k = i / (ECH * R);
+        const int rem = i - k * ECH * R;
+        const int c = rem / R, r = rem - c * R;
+        const int e = e0 + c;
+        wdt[i] = (e < E) ? W_dt[((size_t)k * E + e) * R + r] : 0.f;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < ND * T * ECH; i += kThreads) {
+        const int k = i / (T * ECH);
+        const int rem = i - k * T * ECH;
+        const int t = rem / ECH, c = rem - t * ECH;
+        const int e = e0 + c;
+        float acc = (e < E) ? b_dt[(size_t)k * E + e] : 0.f;
+        const float* ur = us + (k * T + t) * J;
+        const float* wr = wdt + (k * ECH + c) * R;
+        for (int r = 0; r < R; ++r) acc = fmaf(wr[r], ur[r], acc);
+        dts[i] = softplus_f(acc);
+    }
+    __syncthreads();
+
+    const int g = threadIdx.x % G;
+    const int kd = (threadIdx.x / G) % ND;
+    const int c = threadIdx.x / (G * ND);
+    const int e = e0 + c;
+    const bool active = e < E;
+    const bool fwd = (ND == 2) ? (kd == 0) : ((sh.dir_flags & 1u) != 0);
+    constexpr float kLog2e = 1.4426950408889634f;
+    float An[4], A2[4], Ainv[4], hs[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int n = 4 * g + i;
+        const float A = (active && n < N) ? -expf(A_log[((size_t)kd * E + e) * N + n]) : -1.f;
+        An[i] = A;
+        A2[i] = A * kLog2e;
+        Ainv[i] = 1.f / A;
+        hs[i] = 0.f;
+    }
+    const float* ub = us + kd * T * J;
+    const float* dcol = dts + kd * T * ECH + c;
+    for (int step = 0; step < T; ++step) {
+        const int t = fwd ? step : T - 1 - step;
+        const float dt = dcol[t * ECH];
+        const float xv = xs[t * ECH + c];
+        const float dtx = dt * xv;
+        const float* Brow = ub + t * J + R;
+        const float* Crow = Brow + N;
+        float yp = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int n = 4 * g + i;
+            if (n < N) {
+                const float dA = exp2f(dt * A2[i]);
+                float bx;
+                if (ZOH_EXACT) bx = expm1f(dt * An[i]) * Ainv[i] * Brow[n] * xv;
+                else bx = dtx * Brow[n];
+                hs[i] = fmaf(dA, hs[i], bx);
+                yp = fmaf(Crow[n], hs[i], yp);
+            }
+        }
+        if (G >= 2) yp += __shfl_xor_sync(0xffffffffu, yp, 1);
+        if (G >= 4) yp += __shfl_xor_sync(0xffffffffu, yp, 2);
+        if (g == 0 && active) atomicAdd(&ysum[t * ECH + c], yp);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < T * ECH; i += kThreads) {
+        const int t = i / ECH, cc = i - t * ECH;
+        const int ee = e0 + cc;
+        if (ee < E) ys[((size_t)b * T + t) * E + ee] = ysum[i];
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// Repeat + skip + gate: y = SiLU(z) * (ys[row] + (sum_k D_k) x), streamed with 128-bit accesses.
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ float4 gate4(const float4& xv, const float4& zv, const float4& ysv, const float4& dv) {
+    return make_float4(silu_f(zv.x) * fmaf(dv.x, xv.x, ysv.x), silu_f(zv.y) * fmaf(dv.y, xv.y, ysv.y),
+                       silu_f(zv.z) * fmaf(dv.z, xv.z, ysv.z), silu_f(zv.w) * fmaf(dv.w, xv.w, ysv.w));
+}
+
+__device__ __forceinline__ float4 dsum4(const float* __restrict__ D, int nd, int SL, int slot) {
+    const float4* D4 = reinterpret_cast<const float4*>(D);
+    float4 dv = D4[slot];
+    if (nd == 2) f4_add(dv, D4[SL + slot]);
+    return dv;
+}
+
+__device__ __forceinline__ void gate_line(const float4* __restrict__ x4, const float4* __restrict__ z4,
+                                          float4* __restrict__ y4, size_t st4, int s0, int G, int S,
+                                          const float4& ysv, const float4& dv) {
+    int s = s0;
+    for (; s + G < S; s += 2 * G) {
+        const size_t o0 = (size_t)s * st4, o1 = (size_t)(s + G) * st4;
+        const float4 x0 = ld_stream(x4 + o0), z0 = ld_stream(z4 + o0);
+        const float4 x1 = ld_stream(x4 + o1), z1 = ld_stream(z4 + o1);
+        st_stream(y4 + o0, gate4(x0, z0, ysv, dv));
+        st_stream(y4 + o1, gate4(x1, z1, ysv, dv));
+    }
+    if (s < S) {
+        const size_t o0 = (size_t)s * st4;
+        st_stream(y4 + o0, gate4(ld_stream(x4 + o0), ld_stream(z4 + o0), ysv, dv));
+    }
+}
+
+// One CTA per pooled token (b, t): writes the S grid tokens of line t.
+__global__ void __launch_bounds__(kThreads)
+epilogue_dense_kernel(Shape sh, const float* __restrict__ x, const float* __restrict__ z,
+                      const float* __restrict__ ys, const float* __restrict__ D, float* __restrict__ y) {
+    const int bt = blockIdx.x;
+    const int b = bt / sh.T, t = bt - b * sh.T;
+    const size_t off4 = dense_base(sh, b, t) >> 2;
+    const size_t st4 = dense_stride(sh) >> 2;
+    const float4* x4 = reinterpret_cast<const float4*>(x) + off4;
+    const float4* z4 = reinterpret_cast<const float4*>(z) + off4;
+    float4* y4 = reinterpret_cast<float4*>(y) + off4;
+    const float4* ys4 = reinterpret_cast<const float4*>(ys + (size_t)bt * sh.E);
+    const int SL = sh.SL;
+    if (SL <= kThreads) {
+        const int G = kThreads / SL;
+        const int slot = threadIdx.x % SL, g = threadIdx.x / SL;
+        if (g < G) gate_line(x4 + slot, z4 + slot, y4 + slot, st4, g, G, sh.S, ys4[slot], dsum4(D, sh.nd, SL, slot));
+    } else {
+        for (int slot = threadIdx.x; slot < SL; slot += kThreads)
+            gate_line(x4 + slot, z4 + slot, y4 + slot, st4, 0, 1, sh.S, ys4[slot], dsum4(D, sh.nd, SL, slot));
+    }
+}
+
+constexpr int kMaskEpiTokens = 16;  // kept tokens per masked-epilogue CTA
+
+// One CTA per (sample b, block of kMaskEpiTokens kept tokens); a rejected token gets 0.
+__global__ void __launch_bounds__(kThreads)
+mask_epilogue_kernel(Shape sh, const float* __restrict__ x, const float* __restrict__ z,
+                     const float* __restrict__ ys, const float* __restrict__ D,
+                     const int32_t* __restrict__ row_of, float* __restrict__ y) {
+    const int nkb = (sh.K + kMaskEpiTokens - 1) / kMaskEpiTokens;
+    const int b = blockIdx.x / nkb;
+    const int k0 = (blockIdx.x - b * nkb) * kMaskEpiTokens;
+    const int SL = sh.SL;
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    const float4* z4 = reinterpret_cast<const float4*>(z);
+    const float4* ys4 = reinterpret_cast<const float4*>(ys);
+    float4* y4 = reinterpret_cast<float4*>(y);
+    for (int f = threadIdx.x; f < kMaskEpiTokens * SL; f += kThreads) {
+        const int kk = f / SL, slot = f - kk * SL;
+        const int k = k0 + kk;
+        if (k >= sh.K) break;
+        const int r = row_of[(size_t)b * sh.K + k];
+        const size_t o = ((size_t)b * sh.K + k) * SL + slot;
+        float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r >= 0)
+            res = gate4(ld_stream(x4 + o), ld_stream(z4 + o), ys4[((size_t)b * sh.T + r) * SL + slot],
+                        dsum4(D, sh.nd, SL, slot));
+        st_stream(y4 + o, res);
+    }
+}
+
+}  // namespace fv

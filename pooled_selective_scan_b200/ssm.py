@@ -1,0 +1,238 @@
+"""PyTorch-facing binding of the FastVim SSM layer (argument marshalling only).
+
+Every step of the layer runs in the CUDA library (``libfastvim_ssm.so``); PyTorch only provides
+device memory and the stream.  Tensors must be contiguous fp32 (keep_idx int32) on the current
+CUDA device; parameters are stacked per enabled direction (slot 0 = forward when enabled):
+
+    A_log [nd,E,N]   D [nd,E]   W_x [nd,R+2N,E]   W_dt [nd,E,R]   b_dt [nd,E]
+
+Dense layer:  x, z [B,h,w,E] -> y [B,h,w,E].
+Masked layer: x, z [B,K,E] with keep_idx [B,K] (grid ids r*w + c of an h x w grid) -> y [B,K,E].
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _native as nat
+from .configs import DIR_BWD, DIR_FWD, POOL_H, POOL_W  # noqa: F401
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_tensor(name, t, dtype, device=None, host=False):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if host:
+        if t.is_cuda:
+            raise ValueError(f"{name} must be a host tensor")
+    else:
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if device is not None and t.device != device:
+            raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+@dataclass
+class LayerShape:
+    B: int
+    h: int
+    w: int
+    E: int
+    N: int
+    R: int
+    pool_axis: int
+    dir_flags: int
+    K: int = 0
+    pool_scale: float = 1.0
+    zoh_exact: bool = False
+
+    @property
+    def nd(self) -> int:
+        return int(bool(self.dir_flags & DIR_FWD)) + int(bool(self.dir_flags & DIR_BWD))
+
+    @property
+    def T(self) -> int:
+        return self.h if self.pool_axis == POOL_W else self.w
+
+    def token_shape(self):
+        return (self.B, self.K, self.E) if self.K else (self.B, self.h, self.w, self.E)
+
+    def args(self, x=None, z=None, A_log=None, D=None, W_x=None, W_dt=None, b_dt=None, keep_idx=None,
+             y=None) -> nat.FvSsmArgs:
+        a = nat.FvSsmArgs()
+        a.B, a.h, a.w, a.E, a.N, a.R = self.B, self.h, self.w, self.E, self.N, self.R
+        a.pool_axis = self.pool_axis
+        a.dir_flags = self.dir_flags
+        a.K = self.K
+        a.pool_scale = float(self.pool_scale)
+        a.flags = nat.FV_FLAG_ZOH_EXACT if self.zoh_exact else 0
+        a.x, a.z, a.A_log, a.D, a.W_x, a.W_dt, a.b_dt, a.keep_idx, a.y = (
+            _ptr(x), _ptr(z), _ptr(A_log), _ptr(D), _ptr(W_x), _ptr(W_dt), _ptr(b_dt), _ptr(keep_idx), _ptr(y))
+        return a
+
+
+def infer_shape(x, A_log, W_dt, pool_axis, dir_flags, keep_idx=None, h=None, w=None, pool_scale=1.0,
+                zoh_exact=False) -> LayerShape:
+    nd, E, N = A_log.shape
+    R = W_dt.shape[2]
+    if keep_idx is None:
+        if x.dim() != 4:
+            raise ValueError("dense x must be [B,h,w,E]")
+        B, h, w, E2 = x.shape
+        K = 0
+    else:
+        if x.dim() != 3 or h is None or w is None:
+            raise ValueError("masked x must be [B,K,E] and the grid h, w must be given")
+        B, K, E2 = x.shape
+        if K == 0:
+            raise ValueError("a masked layer needs K >= 1 kept tokens")
+    if E2 != E:
+        raise ValueError(f"x has E={E2}, parameters have E={E}")
+    s = LayerShape(B, h, w, E, N, R, pool_axis, dir_flags, K, pool_scale, zoh_exact)
+    if s.nd != nd:
+        raise ValueError(f"dir_flags={dir_flags} enables {s.nd} directions, parameters stack {nd}")
+    return s
+
+
+def workspace_size(shape: LayerShape) -> int:
+    a = shape.args()
+    n = nat.lib().fastvim_ssm_workspace_size(ctypes.byref(a))
+    if n == 0:
+        nat.check(nat.lib().fastvim_ssm_validate(ctypes.byref(a)), "fastvim_ssm_workspace_size")
+    return int(n)
+
+
+def workspace_layout(shape: LayerShape) -> dict:
+    a = shape.args()
+    L = nat.FvWsLayout()
+    nat.check(nat.lib().fastvim_ssm_workspace_layout(ctypes.byref(a), ctypes.byref(L)), "fastvim_ssm_workspace_layout")
+    return {name: getattr(L, name) for name, _ in L._fields_}
+
+
+def launch_count(shape: LayerShape) -> int:
+    a = shape.args()
+    return int(nat.lib().fastvim_ssm_launch_count(ctypes.byref(a)))
+
+
+def launch_names(shape: LayerShape) -> list:
+    a = shape.args()
+    return [nat.lib().fastvim_ssm_launch_name(ctypes.byref(a), i).decode() for i in range(launch_count(shape))]
+
+
+def alloc_workspace(shape: LayerShape, device=None) -> torch.Tensor:
+    return torch.empty(max(workspace_size(shape), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def forward(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis=POOL_W, dir_flags=DIR_FWD | DIR_BWD, keep_idx=None,
+            h=None, w=None, pool_scale=1.0, zoh_exact=False, y=None, workspace=None, stream=None):
+    """Queue the layer on ``stream`` (default: the current stream) and return y."""
+    dev = x.device
+    for name, t in (("x", x), ("z", z), ("A_log", A_log), ("D", D), ("W_x", W_x), ("W_dt", W_dt), ("b_dt", b_dt)):
+        _check_tensor(name, t, torch.float32, dev)
+    if keep_idx is not None:
+        _check_tensor("keep_idx", keep_idx, torch.int32, dev)
+    shape = infer_shape(x, A_log, W_dt, pool_axis, dir_flags, keep_idx, h, w, pool_scale, zoh_exact)
+    if z.shape != x.shape:
+        raise ValueError("z must have the shape of x")
+    if y is None:
+        y = torch.empty_like(x)
+    else:
+        _check_tensor("y", y, torch.float32, dev)
+        if y.shape != x.shape:
+            raise ValueError("y must have the shape of x")
+    if workspace is None:
+        workspace = alloc_workspace(shape, dev)
+    a = shape.args(x, z, A_log, D, W_x, W_dt, b_dt, keep_idx, y)
+    st = nat.lib().fastvim_ssm_forward(ctypes.byref(a), ctypes.c_void_p(workspace.data_ptr()),
+                                       ctypes.c_size_t(workspace.numel()), _stream_handle(stream))
+    nat.check(st, "fastvim_ssm_forward")
+    return y
+
+
+class BoundForward:
+    """A forward call with its tensors, workspace and argument block bound once, for repeated
+    launches (benchmark loops): ``run()`` queues the layer, ``run_events(evs)`` also records
+    ``evs[i]`` before the i-th kernel launch and ``evs[-1]`` after the last one."""
+
+    def __init__(self, shape: LayerShape, t: dict, y, workspace, stream=None):
+        self.shape = shape
+        self.workspace = workspace
+        self._keep = (t, y, workspace)
+        self._args = shape.args(t["x"], t["z"], t["A_log"], t["D"], t["W_x"], t["W_dt"], t["b_dt"], t.get("keep_idx"), y)
+        self._stream = _stream_handle(stream)
+        self._ws = ctypes.c_void_p(workspace.data_ptr())
+        self._wsn = ctypes.c_size_t(workspace.numel())
+        self.n_launch = launch_count(shape)
+        self._evbuf = (ctypes.c_void_p * (self.n_launch + 1))()
+        L = nat.lib()
+        nat.check(L.fastvim_ssm_validate(ctypes.byref(self._args)), "fastvim_ssm_validate")
+
+    def run(self):
+        nat.check(nat.lib().fastvim_ssm_forward(ctypes.byref(self._args), self._ws, self._wsn, self._stream),
+                  "fastvim_ssm_forward")
+
+    def run_events(self, events):
+        for i, e in enumerate(events):
+            self._evbuf[i] = e.cuda_event
+        nat.check(nat.lib().fastvim_ssm_forward_events(ctypes.byref(self._args), self._ws, self._wsn, self._stream,
+                                                       self._evbuf, len(events)), "fastvim_ssm_forward_events")
+
+
+def device_status(workspace, stream=None) -> int:
+    """Wait for the stream and return the device status word of the last call (0 = FV_OK)."""
+    return int(nat.lib().fastvim_get_device_status(ctypes.c_void_p(workspace.data_ptr()), _stream_handle(stream)))
+
+
+class HostForward:
+    """End-to-end calls on pinned host buffers through ``fastvim_ssm_forward_host``: each call
+    copies the inputs host -> device, runs the layer and copies y back, returning when y is in
+    host memory.  Device buffers and the workspace are allocated once here."""
+
+    def __init__(self, shape: LayerShape, device=None):
+        self.shape = shape
+        dev = torch.device(device or "cuda")
+        nd, E, N, R = shape.nd, shape.E, shape.N, shape.R
+        mk = lambda *s: torch.empty(s, dtype=torch.float32, device=dev)  # noqa: E731
+        self.dev = dict(x=mk(*shape.token_shape()), z=mk(*shape.token_shape()), y=mk(*shape.token_shape()),
+                        A_log=mk(nd, E, N), D=mk(nd, E), W_x=mk(nd, R + 2 * N, E), W_dt=mk(nd, E, R), b_dt=mk(nd, E))
+        self.dev["keep_idx"] = (torch.empty((shape.B, shape.K), dtype=torch.int32, device=dev) if shape.K else None)
+        self.workspace = alloc_workspace(shape, dev)
+
+    def h2d_bytes(self) -> int:
+        s = self.shape
+        act = 2 * s.B * (s.K if s.K else s.h * s.w) * s.E * 4
+        par = s.nd * (s.E * s.N + 2 * s.E + (s.R + 2 * s.N) * s.E + s.E * s.R) * 4
+        return act + par + (s.B * s.K * 4 if s.K else 0)
+
+    def d2h_bytes(self) -> int:
+        s = self.shape
+        return s.B * (s.K if s.K else s.h * s.w) * s.E * 4
+
+    def __call__(self, host: dict, y_host, stream=None):
+        for name in ("x", "z", "A_log", "D", "W_x", "W_dt", "b_dt"):
+            _check_tensor(name, host[name], torch.float32, host=True)
+        _check_tensor("y", y_host, torch.float32, host=True)
+        d = self.dev
+        ha = self.shape.args(host["x"], host["z"], host["A_log"], host["D"], host["W_x"], host["W_dt"], host["b_dt"],
+                             host.get("keep_idx"), y_host)
+        da = self.shape.args(d["x"], d["z"], d["A_log"], d["D"], d["W_x"], d["W_dt"], d["b_dt"], d["keep_idx"], d["y"])
+        st = nat.lib().fastvim_ssm_forward_host(ctypes.byref(ha), ctypes.byref(da),
+                                                ctypes.c_void_p(self.workspace.data_ptr()),
+                                                ctypes.c_size_t(self.workspace.numel()), _stream_handle(stream))
+        nat.check(st, "fastvim_ssm_forward_host")
+        return y_host

@@ -1,0 +1,47 @@
+"""Device-resident synthetic workloads (seeded, image by image from ``inputs``).
+
+Builds the full-batch tensors of a ``LayerConfig`` on a CUDA device without ever holding more
+than one image of x or z on the host, so the 3.2 GB-per-tensor 2048 px layer can be set up on
+any host.  Pinned host copies (for end-to-end runs) are built the same way on request.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import inputs
+from .configs import LayerConfig
+
+
+def params_tensors(cfg: LayerConfig, device) -> dict:
+    p = inputs.params(cfg.E, cfg.N, cfg.R, cfg.nd, cfg.seed)
+    return {k: torch.from_numpy(v).to(device) for k, v in p.items()}
+
+
+def activations(cfg: LayerConfig, device, pinned_host: bool = False) -> dict:
+    """x, z (and keep_idx) for every image of ``cfg`` on ``device`` (or in pinned host memory)."""
+    shp = inputs.token_shape(cfg)
+    kw = dict(dtype=torch.float32)
+    if pinned_host:
+        x = torch.empty((cfg.B,) + shp, pin_memory=True, **kw)
+        z = torch.empty((cfg.B,) + shp, pin_memory=True, **kw)
+    else:
+        x = torch.empty((cfg.B,) + shp, device=device, **kw)
+        z = torch.empty((cfg.B,) + shp, device=device, **kw)
+    for b in range(cfg.B):
+        x[b].copy_(torch.from_numpy(inputs.image_x(cfg.seed, b, shp)), non_blocking=False)
+        z[b].copy_(torch.from_numpy(inputs.image_z(cfg.seed, b, shp)), non_blocking=False)
+    out = dict(x=x, z=z)
+    if cfg.masked:
+        idx = np.stack([inputs.image_keep_idx(cfg.seed, b, cfg.h, cfg.w, cfg.K) for b in range(cfg.B)])
+        t = torch.from_numpy(idx)
+        out["keep_idx"] = t.pin_memory() if pinned_host else t.to(device)
+    return out
+
+
+def layer_tensors(cfg: LayerConfig, device, pinned_host: bool = False) -> dict:
+    d = params_tensors(cfg, "cpu" if pinned_host else device)
+    if pinned_host:
+        d = {k: v.pin_memory() for k, v in d.items()}
+    d.update(activations(cfg, device, pinned_host))
+    return d

@@ -1,0 +1,166 @@
+"""The C ABI on the host, without a GPU: the library loads, exports exactly what the header
+declares, and the host-side checks reject bad arguments before anything would be queued."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from pooled_selective_scan_b200 import _native as nat
+from pooled_selective_scan_b200 import build as fvbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fastvim_ssm.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fvbuild.build()
+    return nat.lib()
+
+
+def header_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"FV_API\s+[\w\s\*]+?\b(fastvim_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    fns = header_functions()
+    for must in ("fastvim_ssm_forward", "fastvim_ssm_workspace_size", "fastvim_get_device_status",
+                 "fastvim_status_string"):
+        assert must in fns
+    assert sorted(nat.EXPORTS) == fns
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", nat.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = sorted(set(re.findall(r"\sT\s(fastvim_\w+)$", out, re.M)))
+    assert exported == header_functions()
+    for name in header_functions():
+        assert getattr(lib, name) is not None
+
+
+def test_header_compiles_as_plain_c(tmp_path):
+    src = tmp_path / "use.c"
+    src.write_text('#include "fastvim_ssm.h"\nint main(void){fv_ssm_args a={0}; (void)a; '
+                   'return (int)fastvim_ssm_workspace_size(&a);}\n')
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-c", "-I", os.path.dirname(HEADER), str(src),
+                    "-o", str(tmp_path / "use.o")], check=True)
+
+
+def test_struct_layout_matches_header(tmp_path):
+    src = tmp_path / "off.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "fastvim_ssm.h"\n'
+                   'int main(void){printf("%zu %zu %zu %zu %zu\\n", sizeof(fv_ssm_args), '
+                   'offsetof(fv_ssm_args, pool_scale), offsetof(fv_ssm_args, x), offsetof(fv_ssm_args, y), '
+                   'sizeof(fv_ws_layout)); return 0;}\n')
+    exe = tmp_path / "off"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    want = [ctypes.sizeof(nat.FvSsmArgs), nat.FvSsmArgs.pool_scale.offset, nat.FvSsmArgs.x.offset,
+            nat.FvSsmArgs.y.offset, ctypes.sizeof(nat.FvWsLayout)]
+    assert got == want
+
+
+def test_status_strings(lib):
+    assert nat.status_string(0) == "FV_OK"
+    for s in range(1, 10):
+        assert nat.status_string(s).startswith("FV_ERR_")
+    assert lib.fastvim_abi_version() == 1
+
+
+# ---------------------------------------------------------------------------------------------
+# Host validation with fake (never dereferenced) aligned addresses.
+# ---------------------------------------------------------------------------------------------
+FAKE = 1 << 40
+
+
+def good_args(**kw):
+    a = nat.FvSsmArgs()
+    a.B, a.h, a.w, a.E, a.N, a.R = 2, 14, 14, 384, 16, 12
+    a.pool_axis, a.dir_flags, a.K, a.pool_scale, a.flags = 0, 3, 0, 1.0, 0
+    base = FAKE
+    for i, name in enumerate(("x", "z", "A_log", "D", "W_x", "W_dt", "b_dt", "y")):
+        setattr(a, name, base + i * (1 << 32))
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def validate(a):
+    return nat.lib().fastvim_ssm_validate(ctypes.byref(a))
+
+
+def test_valid_dense_and_masked(lib):
+    assert validate(good_args()) == nat.FV_OK
+    assert validate(good_args(K=49, keep_idx=FAKE + (9 << 32))) == nat.FV_OK
+    assert validate(good_args(B=0, x=None, z=None, y=None)) == nat.FV_OK
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("E", 382, nat.FV_ERR_SHAPE), ("E", 0, nat.FV_ERR_SHAPE), ("B", -1, nat.FV_ERR_SHAPE),
+    ("h", 0, nat.FV_ERR_SHAPE), ("N", 0, nat.FV_ERR_SHAPE), ("R", 0, nat.FV_ERR_SHAPE),
+    ("N", 17, nat.FV_ERR_UNSUPPORTED), ("R", 70, nat.FV_ERR_UNSUPPORTED),
+    ("pool_axis", 2, nat.FV_ERR_SHAPE), ("dir_flags", 0, nat.FV_ERR_SHAPE), ("dir_flags", 4, nat.FV_ERR_SHAPE),
+    ("flags", 2, nat.FV_ERR_SHAPE), ("K", 14 * 14 + 1, nat.FV_ERR_SHAPE), ("K", -3, nat.FV_ERR_SHAPE),
+    ("pool_scale", float("nan"), nat.FV_ERR_SHAPE),
+    ("x", None, nat.FV_ERR_NULL), ("y", None, nat.FV_ERR_NULL), ("W_x", None, nat.FV_ERR_NULL),
+    ("b_dt", None, nat.FV_ERR_NULL), ("x", FAKE + 4, nat.FV_ERR_ALIGN), ("D", FAKE + 8, nat.FV_ERR_ALIGN),
+    ("keep_idx", FAKE + (9 << 32), nat.FV_ERR_SHAPE),  # a keep list without K
+])
+def test_bad_arguments_rejected(lib, field, value, status):
+    assert validate(good_args(**{field: value})) == status
+
+
+def test_masked_without_indices_rejected(lib):
+    assert validate(good_args(K=10)) == nat.FV_ERR_NULL
+
+
+def test_alias_rejected(lib):
+    a = good_args()
+    a.y = a.x + 1024 * 16
+    assert validate(a) == nat.FV_ERR_ALIAS
+    a = good_args()
+    a.y = a.z
+    assert validate(a) == nat.FV_ERR_ALIAS
+
+
+def test_null_args_and_outputs(lib):
+    assert lib.fastvim_ssm_validate(None) == nat.FV_ERR_NULL
+    assert lib.fastvim_ssm_workspace_size(None) == 0
+    assert lib.fastvim_ssm_workspace_layout(ctypes.byref(good_args()), None) == nat.FV_ERR_NULL
+    assert lib.fastvim_get_device_status(None, None) == nat.FV_ERR_NULL
+
+
+def test_forward_rejects_before_touching_the_gpu(lib):
+    a = good_args(E=382)
+    assert lib.fastvim_ssm_forward(ctypes.byref(a), None, 0, None) == nat.FV_ERR_SHAPE
+    a = good_args()
+    assert lib.fastvim_ssm_forward(ctypes.byref(a), None, 0, None) == nat.FV_ERR_WORKSPACE
+    assert lib.fastvim_ssm_forward(ctypes.byref(a), ctypes.c_void_p(FAKE + 16), 1 << 30, None) == nat.FV_ERR_WORKSPACE
+    need = lib.fastvim_ssm_workspace_size(ctypes.byref(a))
+    assert lib.fastvim_ssm_forward(ctypes.byref(a), ctypes.c_void_p(FAKE), need - 1, None) == nat.FV_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("pool_axis", [0, 1])
+@pytest.mark.parametrize("K", [0, 37])
+def test_workspace_layout(lib, pool_axis, K):
+    kw = dict(pool_axis=pool_axis, h=6, w=9, E=64, N=16, R=4, B=3)
+    if K:
+        kw.update(K=K, keep_idx=FAKE + (9 << 32))
+    a = good_args(**kw)
+    L = nat.FvWsLayout()
+    assert lib.fastvim_ssm_workspace_layout(ctypes.byref(a), ctypes.byref(L)) == nat.FV_OK
+    T = 6 if pool_axis == 0 else 9
+    assert (L.T, L.S, L.nd) == (T, 15 - T, 2)
+    regions = [(L.status, 4), (L.xbar, 3 * T * 64 * 4), (L.u, 2 * 3 * T * 36 * 4), (L.ys, 3 * T * 64 * 4)]
+    if K:
+        regions += [(L.row_of, 3 * K * 4), (L.row_off, 3 * (T + 1) * 4), (L.row_tok, 3 * K * 4)]
+    end = 0
+    for off, size in regions:
+        assert off % 256 == 0 and off >= end
+        end = off + size
+    assert L.total_bytes >= end
+    assert lib.fastvim_ssm_workspace_size(ctypes.byref(a)) == L.total_bytes
+    assert lib.fastvim_ssm_launch_count(ctypes.byref(a)) == (5 if K else 4)
