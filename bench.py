@@ -54,6 +54,8 @@ def parse(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="fastvim_t_2048")
     ap.add_argument("--pool-axis", type=int, default=None, help="override the workload's pool axis")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the batch (small cases for profiler captures; not a benchmark line)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -421,6 +423,9 @@ def main(argv=None):
     a = parse(argv)
     from pooled_selective_scan_b200.configs import by_name
     cfg = by_name(a.config)
+    if a.batch is not None:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, B=a.batch)
     pool_axis = cfg.pool_axes[0] if a.pool_axis is None else a.pool_axis
     if a.impl == "reference":
         return run_reference(a, cfg, pool_axis)
