@@ -160,6 +160,28 @@ FV_API fv_status fastvim_ssm_forward_events(const fv_ssm_args* args, void* ws, s
 FV_API fv_status fastvim_ssm_forward_host(const fv_ssm_args* host, const fv_ssm_args* dev, void* ws,
                                    size_t ws_bytes, void* stream);
 
+/* fastvim_ssm_forward for callers that cannot allocate device memory.  There is no counterpart
+ * in the paper; this is an interface convenience.  Some callers only ever receive device
+ * buffers for their inputs and outputs from a host framework that owns all device memory and
+ * offers them no allocator, or must not call cudaMalloc/cudaFree because those calls can stall
+ * the whole device.  This entry point needs no workspace argument: its scratch is a fixed
+ * 16 MiB array in device memory that the library reserves on every GPU that loads it, held
+ * until the process exits.
+ *   - Limit: fastvim_ssm_workspace_size(args) must be <= 16 MiB (e.g. the 224 px FastVim-T
+ *     layer at batch 128: about 6 MiB); larger layers return FV_ERR_UNSUPPORTED with a message
+ *     in fastvim_last_error() and queue nothing; split the batch or use fastvim_ssm_forward.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - The first call on a device looks up that device's scratch address (with the device
+ *     current); make that first call before any stream capture begins.
+ *   - All calls on a device share the one scratch array: calls that may overlap on the GPU
+ *     (different streams, no ordering between them) race and give wrong results.  Calls
+ *     queued on one stream are ordered and safe.  The contents left by a previous call need
+ *     no clearing.
+ *   - The device status word lives in the shared scratch and is not readable through this
+ *     entry point; use fastvim_ssm_forward with a workspace where FV_ERR_INDEX must be seen.
+ * Inputs, outputs and the returned status are as for fastvim_ssm_forward. */
+FV_API fv_status fastvim_ssm_forward_noalloc(const fv_ssm_args* args, void* stream);
+
 /* Waits for `stream`, then reads the device status word of a workspace used by the last
  * forward call: FV_OK, FV_ERR_INDEX or FV_ERR_TIMEOUT (or FV_ERR_CUDA if the read fails). */
 FV_API fv_status fastvim_get_device_status(const void* ws, void* stream);

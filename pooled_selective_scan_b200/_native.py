@@ -38,6 +38,7 @@ EXPORTS = (
     "fastvim_ssm_forward",
     "fastvim_ssm_forward_events",
     "fastvim_ssm_forward_host",
+    "fastvim_ssm_forward_noalloc",
     "fastvim_get_device_status",
 )
 
@@ -116,6 +117,8 @@ def lib() -> ctypes.CDLL:
             L.fastvim_ssm_forward_host.argtypes = [P(FvSsmArgs), P(FvSsmArgs), ctypes.c_void_p, ctypes.c_size_t,
                                                    ctypes.c_void_p]
             L.fastvim_ssm_forward_host.restype = ctypes.c_int
+            L.fastvim_ssm_forward_noalloc.argtypes = [P(FvSsmArgs), ctypes.c_void_p]
+            L.fastvim_ssm_forward_noalloc.restype = ctypes.c_int
             L.fastvim_get_device_status.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
             L.fastvim_get_device_status.restype = ctypes.c_int
             _lib = L

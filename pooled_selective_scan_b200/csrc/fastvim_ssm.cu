@@ -5,6 +5,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "fv_common.cuh"
 #include "fv_kernels.cuh"
 
@@ -381,3 +383,62 @@ fv_status fastvim_get_device_status(const void* ws, void* stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------------
+// Allocation-free entry point: the forward call with its workspace in a fixed static device
+// array instead of caller-provided memory.
+// ------------------------------------------------------------------------------------------------
+namespace {
+
+// 16 MiB, reserved on every GPU that loads this library, for as long as the process lives.
+constexpr size_t kStaticScratchBytes = (size_t)16 << 20;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxScratchDevices] = {};
+
+// Device address of g_static_scratch on the current device.  Host code only sees a host-side
+// stand-in under that name, so the real address is asked from the runtime, once per device,
+// with that device current.
+fv_status static_scratch_address(void** out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) { note_cuda(e, "cudaGetDevice"); return FV_ERR_CUDA; }
+    if (dev < 0 || dev >= kMaxScratchDevices) return FV_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (e != cudaSuccess || !p) {
+            note_cuda(e, "cudaGetSymbolAddress(static scratch)");
+            return FV_ERR_CUDA;
+        }
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return FV_OK;
+}
+
+}  // namespace
+
+extern "C" fv_status fastvim_ssm_forward_noalloc(const fv_ssm_args* args, void* stream) {
+    fv::Shape sh;
+    fv_status s = make_shape(args, &sh);
+    if (s != FV_OK) return s;
+    if ((s = check_pointers(args, sh)) != FV_OK) return s;
+    fv_ws_layout L;
+    plan_layout(sh, &L);
+    if (L.total_bytes > kStaticScratchBytes) {
+        snprintf(g_last_error, sizeof g_last_error,
+                 "fastvim_ssm_forward_noalloc: this layer needs %zu bytes of scratch, above the %zu-byte "
+                 "static scratch; split the batch or use fastvim_ssm_forward with a workspace",
+                 L.total_bytes, kStaticScratchBytes);
+        return FV_ERR_UNSUPPORTED;
+    }
+    void* scratch = nullptr;
+    if ((s = static_scratch_address(&scratch)) != FV_OK) return s;
+    // Every region of the workspace is written before it is read within one call, and each call
+    // resets the status word itself, so the contents left by an earlier call need no clearing.
+    return forward_impl(args, scratch, kStaticScratchBytes, (cudaStream_t)stream);
+}
