@@ -56,6 +56,8 @@ def parse(argv=None):
     ap.add_argument("--pool-axis", type=int, default=None, help="override the workload's pool axis")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the batch (small cases for profiler captures; not a benchmark line)")
+    ap.add_argument("--path", choices=["auto", "staged", "fused"], default="auto",
+                    help="implementation of the layer (auto picks the fused launch for this workload)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -307,7 +309,7 @@ def run_ours(a, cfg, pool_axis):
 
     t = workload.layer_tensors(cfg, dev)
     keep = t.get("keep_idx")
-    shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, cfg.dir_flags, keep, cfg.h, cfg.w)
+    shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, cfg.dir_flags, keep, cfg.h, cfg.w, path=a.path)
     y = torch.empty_like(t["x"])
     ws = ssm.alloc_workspace(shape, dev)
     stream = torch.cuda.current_stream(dev)

@@ -81,7 +81,19 @@ typedef enum {
 enum { FV_POOL_W = 0, /* mean over w, T = h tokens (column pooling) */
        FV_POOL_H = 1  /* mean over h, T = w tokens (row pooling)    */ };
 enum { FV_DIR_FWD = 1u, FV_DIR_BWD = 2u };
-enum { FV_FLAG_ZOH_EXACT = 1u /* Bbar = (exp(Delta A) - 1) / A * B instead of Delta B */ };
+enum {
+    FV_FLAG_ZOH_EXACT = 1u,   /* Bbar = (exp(Delta A) - 1) / A * B instead of Delta B            */
+    FV_FLAG_PATH_STAGED = 2u, /* force the staged kernels (pool, proj, scan, epilogue launches)  */
+    FV_FLAG_PATH_FUSED = 4u,  /* force the single persistent launch (dense layers only;
+                                 FV_ERR_UNSUPPORTED when the layer does not fit it)             */
+    FV_FLAG_TRACE = 8u        /* fused launch: record one entry per task in the workspace
+                                 (fv_ws_layout.trace); costs a little time, for profiling      */
+};
+/* Without a PATH flag a dense layer whose images hold >= 1 MiB of x runs the fused launch, every
+ * other layer the staged kernels; both compute the same layer.  The fused launch keeps each
+ * image's x in L2 between pooling and the epilogue; the environment variable FASTVIM_FUSED_LAG
+ * (2..64, read per call) overrides how many images it lets lie between the two, and
+ * FASTVIM_FUSED_LP (1..4) how many grid lines one streaming task covers (tuning only). */
 
 typedef struct {
     int B, h, w, E, N, R;    /* batch, grid height/width, channels, d_state, dt_rank        */
@@ -106,11 +118,19 @@ typedef struct {
     size_t total_bytes;  /* what fastvim_ssm_workspace_size returns                          */
     size_t status;       /* uint32 device status word                                        */
     size_t xbar;         /* fp32 [B][T][E] pooled tokens                                     */
-    size_t u;            /* fp32 [nd][B][T][R+2N] projections dt_low | B | C                 */
+    size_t u;            /* fp32 projections dt_low | B | C: [nd][B] blocks of [T][R+2N], each
+                            block starting every ceil(T (R+2N) / 32) * 32 floats            */
     size_t ys;           /* fp32 [B][T][E] scan output summed over directions                */
     size_t row_of;       /* int32 [B][K] pooled row of each kept token (masked), else 0      */
     size_t row_off;      /* int32 [B][T+1] CSR row offsets (masked), else 0                  */
     size_t row_tok;      /* int32 [B][K] kept-token ordinals grouped by row, ascending       */
+    size_t delta;        /* reserved (0): step sizes stay on chip                            */
+    size_t ctrl;         /* uint32 control block of the fused launch (dense layers), else 0  */
+    size_t trace;        /* FV_FLAG_TRACE on the fused launch: uint64 [trace_records][4]:
+                            w0 = kind << 60 | image << 32 | index (kind 0 pool, 1 scan, 2 gate, 3 x_proj),
+                            w1 = SM id << 32 | CTA id, w2 = start (ns, %globaltimer),
+                            w3 = wait_ns << 40 | total_ns (from start to the task's end)        */
+    size_t trace_records;  /* number of trace entries (tasks of the call), else 0               */
     int T, S, nd;        /* pooled length, pooled-over length, number of directions          */
 } fv_ws_layout;
 
@@ -168,7 +188,7 @@ FV_API fv_status fastvim_ssm_forward_host(const fv_ssm_args* host, const fv_ssm_
  * 16 MiB array in device memory that the library reserves on every GPU that loads it, held
  * until the process exits.
  *   - Limit: fastvim_ssm_workspace_size(args) must be <= 16 MiB (e.g. the 224 px FastVim-T
- *     layer at batch 128: about 6 MiB); larger layers return FV_ERR_UNSUPPORTED with a message
+ *     layer at batch 128: about 12 MiB); larger layers return FV_ERR_UNSUPPORTED with a message
  *     in fastvim_last_error() and queue nothing; split the batch or use fastvim_ssm_forward.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  *   - The first call on a device looks up that device's scratch address (with the device
@@ -181,6 +201,12 @@ FV_API fv_status fastvim_ssm_forward_host(const fv_ssm_args* host, const fv_ssm_
  *     entry point; use fastvim_ssm_forward with a workspace where FV_ERR_INDEX must be seen.
  * Inputs, outputs and the returned status are as for fastvim_ssm_forward. */
 FV_API fv_status fastvim_ssm_forward_noalloc(const fv_ssm_args* args, void* stream);
+
+/* Self-test of the bounded wait that the fused launch uses between its tasks: queues one CTA
+ * that waits on a counter nothing increments, for limit_us microseconds (1 .. 10^7), after which
+ * it records FV_ERR_TIMEOUT in the status word of `ws` (>= 1 KB, 256-byte aligned) and exits.
+ * fastvim_get_device_status(ws, stream) then returns FV_ERR_TIMEOUT; the context stays usable. */
+FV_API fv_status fastvim_selftest_bounded_wait(void* ws, size_t ws_bytes, unsigned limit_us, void* stream);
 
 /* Waits for `stream`, then reads the device status word of a workspace used by the last
  * forward call: FV_OK, FV_ERR_INDEX or FV_ERR_TIMEOUT (or FV_ERR_CUDA if the read fails). */

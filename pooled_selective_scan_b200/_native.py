@@ -24,6 +24,9 @@ FV_ERR_UNSUPPORTED = 8
 FV_ERR_ALIAS = 9
 
 FV_FLAG_ZOH_EXACT = 1
+FV_FLAG_PATH_STAGED = 2
+FV_FLAG_PATH_FUSED = 4
+FV_FLAG_TRACE = 8
 
 # Every exported symbol of the ABI, as the header declares it.
 EXPORTS = (
@@ -39,6 +42,7 @@ EXPORTS = (
     "fastvim_ssm_forward_events",
     "fastvim_ssm_forward_host",
     "fastvim_ssm_forward_noalloc",
+    "fastvim_selftest_bounded_wait",
     "fastvim_get_device_status",
 )
 
@@ -65,6 +69,8 @@ class FvWsLayout(ctypes.Structure):
         ("total_bytes", ctypes.c_size_t), ("status", ctypes.c_size_t), ("xbar", ctypes.c_size_t),
         ("u", ctypes.c_size_t), ("ys", ctypes.c_size_t), ("row_of", ctypes.c_size_t),
         ("row_off", ctypes.c_size_t), ("row_tok", ctypes.c_size_t),
+        ("delta", ctypes.c_size_t), ("ctrl", ctypes.c_size_t), ("trace", ctypes.c_size_t),
+        ("trace_records", ctypes.c_size_t),
         ("T", ctypes.c_int), ("S", ctypes.c_int), ("nd", ctypes.c_int),
     ]
 
@@ -119,6 +125,8 @@ def lib() -> ctypes.CDLL:
             L.fastvim_ssm_forward_host.restype = ctypes.c_int
             L.fastvim_ssm_forward_noalloc.argtypes = [P(FvSsmArgs), ctypes.c_void_p]
             L.fastvim_ssm_forward_noalloc.restype = ctypes.c_int
+            L.fastvim_selftest_bounded_wait.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint, ctypes.c_void_p]
+            L.fastvim_selftest_bounded_wait.restype = ctypes.c_int
             L.fastvim_get_device_status.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
             L.fastvim_get_device_status.restype = ctypes.c_int
             _lib = L

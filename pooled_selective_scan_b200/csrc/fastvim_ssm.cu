@@ -5,9 +5,12 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <stdlib.h>
+
 #include <mutex>
 
 #include "fv_common.cuh"
+#include "fv_fused.cuh"
 #include "fv_kernels.cuh"
 
 namespace {
@@ -39,20 +42,15 @@ size_t bucket_smem_bytes(const fv::Shape& sh) {
     return (size_t)(((G + 31) >> 5) + 2ll * sh.T) * sizeof(unsigned);
 }
 
-int max_optin_smem() {
-    int dev = 0, v = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 0;
-    return v;
-}
-
 // Sizes and flags only; no pointer is dereferenced.
 fv_status make_shape(const fv_ssm_args* a, fv::Shape* sh) {
     if (!a) return FV_ERR_NULL;
     if (a->B < 0 || a->h < 1 || a->w < 1 || a->E < 4 || a->N < 1 || a->R < 1) return FV_ERR_SHAPE;
     if (a->pool_axis != FV_POOL_W && a->pool_axis != FV_POOL_H) return FV_ERR_SHAPE;
     if (a->dir_flags == 0 || (a->dir_flags & ~3u) != 0) return FV_ERR_SHAPE;
-    if ((a->flags & ~(unsigned)FV_FLAG_ZOH_EXACT) != 0) return FV_ERR_SHAPE;
+    if ((a->flags & ~(unsigned)(FV_FLAG_ZOH_EXACT | FV_FLAG_PATH_STAGED | FV_FLAG_PATH_FUSED | FV_FLAG_TRACE)) != 0)
+        return FV_ERR_SHAPE;
+    if ((a->flags & FV_FLAG_PATH_STAGED) && (a->flags & FV_FLAG_PATH_FUSED)) return FV_ERR_SHAPE;
     if (a->E % 4 != 0) return FV_ERR_SHAPE;
     if (a->K < 0 || (long long)a->K > (long long)a->h * a->w) return FV_ERR_SHAPE;
     if (!(a->pool_scale == a->pool_scale) || a->pool_scale > 3.0e38f || a->pool_scale < -3.0e38f)
@@ -70,6 +68,8 @@ fv_status make_shape(const fv_ssm_args* a, fv::Shape* sh) {
     sh->K = a->K;
     sh->dir_flags = a->dir_flags;
     sh->zoh_exact = (a->flags & FV_FLAG_ZOH_EXACT) ? 1 : 0;
+    sh->path_flags = a->flags & (FV_FLAG_PATH_STAGED | FV_FLAG_PATH_FUSED);
+    sh->trace = (a->flags & FV_FLAG_TRACE) ? 1 : 0;
     sh->pool_scale = a->pool_scale == 0.f ? 1.f : a->pool_scale;
     sh->SL = a->E / 4;
     if (sh->T > kMaxT) return FV_ERR_UNSUPPORTED;
@@ -96,29 +96,122 @@ fv_status check_pointers(const fv_ssm_args* a, const fv::Shape& sh) {
     return FV_OK;
 }
 
+enum class Path { Staged, Fused, Invalid };
+Path choose_path(const fv::Shape& sh);
+fv::FusedPlan plan_fused(const fv::Shape& sh);
+
 fv_status plan_layout(const fv::Shape& sh, fv_ws_layout* L) {
     memset(L, 0, sizeof *L);
     size_t off = 0;
     L->status = off; off = round256(off + sizeof(unsigned));
     L->xbar = off; off = round256(off + (size_t)sh.B * sh.T * sh.E * sizeof(float));
-    L->u = off; off = round256(off + (size_t)sh.nd * sh.B * sh.T * sh.J * sizeof(float));
+    L->u = off; off = round256(off + (size_t)sh.nd * sh.B * fv::u_block_stride(sh.T, sh.J) * sizeof(float));
     L->ys = off; off = round256(off + (size_t)sh.B * sh.T * sh.E * sizeof(float));
     if (sh.K > 0) {
         L->row_of = off; off = round256(off + (size_t)sh.B * sh.K * sizeof(int32_t));
         L->row_off = off; off = round256(off + (size_t)sh.B * (sh.T + 1) * sizeof(int32_t));
         L->row_tok = off; off = round256(off + (size_t)sh.B * sh.K * sizeof(int32_t));
+    } else {
+        // dense layers: the control block of the fused single-launch path
+        L->ctrl = off; off = round256(off + (size_t)(fv::kCtrlHeaderWords + fv::kCtrlCounters * (size_t)sh.B) * sizeof(unsigned));
+        if (sh.trace && choose_path(sh) == Path::Fused) {
+            const fv::FusedPlan pl = plan_fused(sh);
+            L->trace = off;
+            L->trace_records = pl.total;
+            off = round256(off + (size_t)pl.total * 4 * sizeof(unsigned long long));
+        }
     }
     L->total_bytes = off;
     L->T = sh.T; L->S = sh.S; L->nd = sh.nd;
     return FV_OK;
 }
 
+// The library is built for sm_100a only: 227 KB of opt-in shared memory per CTA.
+constexpr size_t kMaxSmemOptin = 227 * 1024;
+// Latency of one image's pool -> x_proj -> scan chain inside the fused launch (trace, B200).
+constexpr double kChainLatencyUs = 60.0;
+
 fv_status check_limits(const fv::Shape& sh) {
-    const size_t optin = (size_t)max_optin_smem();
-    const size_t lim = optin ? optin : (size_t)(227 * 1024);
-    if (scan_smem_bytes(sh) > lim) return FV_ERR_UNSUPPORTED;
-    if (sh.K > 0 && bucket_smem_bytes(sh) > lim) return FV_ERR_UNSUPPORTED;
+    if (scan_smem_bytes(sh) > kMaxSmemOptin) return FV_ERR_UNSUPPORTED;
+    if (sh.K > 0 && bucket_smem_bytes(sh) > kMaxSmemOptin) return FV_ERR_UNSUPPORTED;
     return FV_OK;
+}
+
+
+// Grid lines per P/E task: the fewest that give each task at least 96 KB of x (short tasks keep
+// the per-image dependency chain short).  FASTVIM_FUSED_LP (1..4) overrides it (tuning only).
+int fused_lines_per_task(const fv::Shape& sh) {
+    const size_t line = (size_t)sh.S * sh.E * sizeof(float);
+    int lp = 1;
+    while (lp < fv::kMaxLP && lp < sh.T && (size_t)lp * line < ((size_t)96 << 10)) ++lp;
+    if (const char* env = getenv("FASTVIM_FUSED_LP")) {
+        const int v = atoi(env);
+        if (v >= 1 && v <= fv::kMaxLP) lp = v < sh.T ? v : sh.T;
+    }
+    return lp;
+}
+
+bool fused_possible(const fv::Shape& sh) {
+    if (sh.K > 0 || sh.B < 1) return false;
+    // a token row of x (and of z) must fit half a ring stage; a thread holds at most 2 float4 slots
+    if ((size_t)sh.E * sizeof(float) > (size_t)fv::kStageBytes / 2) return false;
+    if (sh.SL > fv::kMaxSlots * fv::kFusedThreads) return false;
+    if (fv::fused_smem_floats(sh, fused_lines_per_task(sh)) * sizeof(float) > kMaxSmemOptin) return false;
+    // tickets are 32-bit: every task of the call must be numbered
+    const long long per_image = 2ll * sh.T + (sh.T + fv::kQT - 1) / fv::kQT +
+                                (sh.E + fv::fused_ech(sh.nd) - 1) / fv::fused_ech(sh.nd);
+    if ((long long)sh.B * per_image >= (1ll << 31)) return false;
+    return true;
+}
+
+// Which implementation runs: the fused single launch for dense layers whose images are large
+// enough to stream (>= 1 MiB of x per image), the staged kernels otherwise; flags can force either.
+Path choose_path(const fv::Shape& sh) {
+    const bool ok = fused_possible(sh);
+    if (sh.path_flags & FV_FLAG_PATH_STAGED) return Path::Staged;
+    if (sh.path_flags & FV_FLAG_PATH_FUSED) return ok ? Path::Fused : Path::Invalid;
+    const size_t img = (size_t)sh.h * sh.w * sh.E * sizeof(float);
+    return (ok && img >= ((size_t)1 << 20)) ? Path::Fused : Path::Staged;
+}
+
+fv::FusedPlan plan_fused(const fv::Shape& sh) {
+    fv::FusedPlan pl;
+    pl.LP = fused_lines_per_task(sh);
+    pl.nP = (sh.T + pl.LP - 1) / pl.LP;
+    pl.nQ = (sh.T + fv::kQT - 1) / fv::kQT;
+    pl.ECH = fv::fused_ech(sh.nd);
+    pl.nS = (sh.E + pl.ECH - 1) / pl.ECH;
+    pl.CL = (sh.T + fv::kScanChunks - 1) / fv::kScanChunks;
+    pl.ctP = fv::kStageBytes / (sh.E * (int)sizeof(float));
+    pl.ctE = fv::kStageBytes / 2 / (sh.E * (int)sizeof(float));
+    // Lag: enough rounds to cover one image's pool -> proj -> scan chain (about 60 us measured on
+    // B200) at the rate one round streams (x twice, z and y once: 16 E bytes per grid token at
+    // ~6.5 TB/s).  (Keeping x in L2 across that window does not happen: traffic of this size
+    // evicts first-touch lines whatever their L2 eviction priority.)
+    const double round_us = (double)sh.h * sh.w * sh.E * 16.0 / 6.5e6;
+    long long lag = (long long)(kChainLatencyUs / (round_us > 0.01 ? round_us : 0.01)) + 2;
+    if (const char* env = getenv("FASTVIM_FUSED_LAG")) {
+        const long long v = atoll(env);
+        if (v >= 2 && v <= 64) lag = v;
+    }
+    // E of image r-L is dequeued before S of image r-1 within round r, so L >= 2 keeps every
+    // consumer after its producers in ticket order (the deadlock-freedom argument above).
+    pl.L = (int)(lag < 2 ? 2 : (lag > 64 ? 64 : lag));
+    pl.B = sh.B;
+    // rounds r = 0 .. B+L-1; [R1, R2) hold Q, P, E and S alike
+    const int rounds = sh.B + pl.L;
+    pl.R1 = pl.L > 1 ? pl.L : 1;
+    pl.R2 = sh.B > pl.R1 ? sh.B : pl.R1;
+    unsigned c = 0;
+    for (int r = 0; r < pl.R1; ++r) c += fv::fused_round_size(pl, r);
+    pl.c1 = c;
+    pl.c2 = c + (unsigned)(pl.R2 - pl.R1) * fv::fused_round_size(pl, pl.R1);
+    c = pl.c2;
+    for (int r = pl.R2; r < rounds; ++r) c += fv::fused_round_size(pl, r);
+    pl.total = c;
+    pl.smem_bytes = fv::fused_smem_floats(sh, pl.LP) * sizeof(float);
+    pl.wait_limit_ns = fv::kWaitLimitNs;
+    return pl;
 }
 
 // Kernels that take more than 48 KB of dynamic shared memory need an opt-in per device.
@@ -190,14 +283,56 @@ struct EventMarks {
         }                                                    \
     } while (0)
 
-int launch_count_of(const fv::Shape& sh) { return sh.B == 0 ? 0 : (sh.K > 0 ? 5 : 4); }
+int launch_count_of(const fv::Shape& sh) {
+    if (sh.B == 0) return 0;
+    const Path path = choose_path(sh);
+    if (path == Path::Invalid) return 0;
+    if (path == Path::Fused) return 1;
+    return sh.K > 0 ? 5 : 4;
+}
 
 const char* launch_name_of(const fv::Shape& sh, int i) {
     static const char* dense[] = {"pool_dense_kernel", "proj_kernel", "scan_kernel", "epilogue_dense_kernel"};
     static const char* masked[] = {"mask_bucket_kernel", "mask_pool_kernel", "proj_kernel", "scan_kernel",
                                    "mask_epilogue_kernel"};
     if (i < 0 || i >= launch_count_of(sh)) return "";
+    if (choose_path(sh) == Path::Fused) return "fused_layer_kernel";
     return sh.K > 0 ? masked[i] : dense[i];
+}
+
+template <int ND, bool Z>
+fv_status launch_fused_t(const fv::Shape& sh, const fv::FusedPlan& pl, const fv::FusedPtrs& ptrs, cudaStream_t st) {
+    auto kern = fv::fused_layer_kernel<ND, Z>;
+    cudaError_t e = ensure_smem(kern, pl.smem_bytes);
+    if (e != cudaSuccess) { note_cuda(e, "fused smem attribute"); return FV_ERR_CUDA; }
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, fv::kFusedThreads, pl.smem_bytes)) != cudaSuccess) {
+        note_cuda(e, "fused occupancy query");
+        return FV_ERR_CUDA;
+    }
+    if (per_sm < 1) return FV_ERR_UNSUPPORTED;
+    long long grid = (long long)sms * per_sm;
+    if (grid > (long long)pl.total) grid = pl.total;
+    kern<<<(unsigned)grid, fv::kFusedThreads, pl.smem_bytes, st>>>(sh, pl, ptrs);
+    FV_LAUNCH_CHECK("fused_layer_kernel");
+    return FV_OK;
+}
+
+fv_status launch_fused(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st) {
+    const fv::FusedPlan pl = plan_fused(sh);
+    fv::FusedPtrs p;
+    p.x = a->x; p.z = a->z; p.A_log = a->A_log; p.D = a->D; p.W_x = a->W_x; p.W_dt = a->W_dt; p.b_dt = a->b_dt;
+    p.y = a->y;
+    p.xbar = (float*)(ws + L.xbar);
+    p.u = (float*)(ws + L.u);
+    p.ys = (float*)(ws + L.ys);
+    p.status = (unsigned*)(ws + L.status);
+    p.ctrl = (unsigned*)(ws + L.ctrl);
+    p.trace = L.trace_records ? (unsigned long long*)(ws + L.trace) : nullptr;
+    if (sh.nd == 2) return sh.zoh_exact ? launch_fused_t<2, true>(sh, pl, p, st) : launch_fused_t<2, false>(sh, pl, p, st);
+    return sh.zoh_exact ? launch_fused_t<1, true>(sh, pl, p, st) : launch_fused_t<1, false>(sh, pl, p, st);
 }
 
 fv_status forward_impl(const fv_ssm_args* a, void* ws_v, size_t ws_bytes, cudaStream_t st,
@@ -217,6 +352,19 @@ fv_status forward_impl(const fv_ssm_args* a, void* ws_v, size_t ws_bytes, cudaSt
     if (sh.B == 0) {
         cudaError_t e = cudaMemsetAsync(status, 0, sizeof(unsigned), st);
         if (e != cudaSuccess) { note_cuda(e, "status reset"); return FV_ERR_CUDA; }
+        return FV_OK;
+    }
+    const Path path = choose_path(sh);
+    if (path == Path::Invalid) return FV_ERR_UNSUPPORTED;
+    if (path == Path::Fused) {
+        // status word and control block (ticket, abort flag, per-image counters) start at zero
+        cudaError_t e = cudaMemsetAsync(status, 0, sizeof(unsigned), st);
+        if (e == cudaSuccess)
+            e = cudaMemsetAsync(ws + L.ctrl, 0, (fv::kCtrlHeaderWords + fv::kCtrlCounters * (size_t)sh.B) * sizeof(unsigned), st);
+        if (e != cudaSuccess) { note_cuda(e, "control reset"); return FV_ERR_CUDA; }
+        FV_MARK(marks, st);
+        if ((s = launch_fused(sh, a, L, ws, st)) != FV_OK) return s;
+        FV_MARK(marks, st);
         return FV_OK;
     }
     const int M = sh.B * sh.T;
@@ -369,6 +517,20 @@ fv_status fastvim_ssm_forward_host(const fv_ssm_args* host, const fv_ssm_args* d
     }
     cudaError_t e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) { note_cuda(e, "stream synchronize"); return FV_ERR_CUDA; }
+    return FV_OK;
+}
+
+fv_status fastvim_selftest_bounded_wait(void* ws, size_t ws_bytes, unsigned limit_us, void* stream) {
+    if (!ws) return FV_ERR_NULL;
+    if (ws_bytes < 1024 || ((uintptr_t)ws & 255u) != 0) return FV_ERR_WORKSPACE;
+    if (limit_us == 0 || limit_us > 10u * 1000u * 1000u) return FV_ERR_SHAPE;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaMemsetAsync(ws, 0, 1024, st);
+    if (e != cudaSuccess) { note_cuda(e, "selftest reset"); return FV_ERR_CUDA; }
+    unsigned* status = (unsigned*)ws;
+    unsigned* ctrl = (unsigned*)((char*)ws + 256);
+    fv::bounded_wait_selftest_kernel<<<1, 32, 0, st>>>(status, ctrl, (unsigned long long)limit_us * 1000ull);
+    FV_LAUNCH_CHECK("bounded_wait_selftest_kernel");
     return FV_OK;
 }
 

@@ -26,9 +26,19 @@ struct Shape {
     int pool_axis;     // 0 = POOL_W (T = h), 1 = POOL_H (T = w)
     unsigned dir_flags;
     int zoh_exact;
+    unsigned path_flags;  // FV_FLAG_PATH_* of the call
+    int trace;            // FV_FLAG_TRACE: record one trace entry per fused task
     float pool_scale;
     int SL;            // float4 slots per token row: E / 4
 };
+
+// Projections u of (direction k, image b) are one block of T x J floats; blocks start every
+// u_block_stride floats (T J rounded up to 32 floats = 128 bytes), so no cache line holds
+// projections of two images.
+__host__ __device__ __forceinline__ size_t u_block_stride(int T, int J) { return (((size_t)T * J + 31) / 32) * 32; }
+__host__ __device__ __forceinline__ size_t u_offset(const Shape& sh, int k, int b, int t) {
+    return ((size_t)k * sh.B + b) * u_block_stride(sh.T, sh.J) + (size_t)t * sh.J;
+}
 
 // Offset (in floats) of token s of pooled token (b, t) on the dense grid, and the stride
 // between consecutive s.  POOL_W: token (t, s); POOL_H: token (s, t).
@@ -43,6 +53,118 @@ __host__ __device__ __forceinline__ size_t dense_stride(const Shape& sh) {
 // Streaming (evict-first) 128-bit accesses for data touched once.
 __device__ __forceinline__ float4 ld_stream(const float4* p) { return __ldcs(p); }
 __device__ __forceinline__ void st_stream(float4* p, const float4& v) { __stcs(p, v); }
+
+// L2 eviction-priority policies (createpolicy) and 128-bit accesses that carry them.  Loads skip
+// L1 allocation: every byte is used once per CTA.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t p;
+    asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t p;
+    asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// For tensors that stay read-only for the whole kernel (x, z): the compiler may schedule these
+// loads freely.
+__device__ __forceinline__ float4 ld_nc_hint(const float4* p, uint64_t pol) {
+    float4 v;
+    asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p), "l"(pol));
+    return v;
+}
+__device__ __forceinline__ void st_hint(float4* p, const float4& v, uint64_t pol) {
+    asm volatile("st.global.L1::no_allocate.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;"
+                 :
+                 : "l"(p), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "l"(pol)
+                 : "memory");
+}
+
+// Cross-CTA handshakes inside one launch: acquire loads of counters, release increments.
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(unsigned* p, unsigned v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" : : "l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ---- shared-memory mbarriers and TMA bulk copies (global -> shared) ----------------------------
+__device__ __forceinline__ unsigned smem_u32(const void* p) {
+    return static_cast<unsigned>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(unsigned long long* bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" : : "r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" : : : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" : : : "memory");
+}
+// One arrival that also announces `bytes` of asynchronous transfers completing on this barrier.
+__device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long* bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" : : "r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, unsigned parity) {
+    unsigned ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) into this CTA's shared
+// memory, completing on `bar`, with an L2 eviction-priority policy on the global reads.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, unsigned long long* bar,
+                                         uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+        :
+        : "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
+}
+// 2^x on the SFU (ex2.approx.ftz: results below 2^-126 flush to zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// 1/x on the SFU (rcp.approx.ftz).
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// SiLU(v) = v / (1 + e^-v) with the SFU exponential and reciprocal: about 3e-7 relative error;
+// v -> -inf gives -0 (e^-v overflows to inf, its reciprocal is 0).
+__device__ __forceinline__ float silu_fast(float v) {
+    return v * rcp_approx(1.f + ex2_approx(v * -1.4426950408889634f));
+}
+
+// 16-byte asynchronous global -> shared copies (cp.async); src_bytes = 0 fills zeros.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, unsigned src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" : : "r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" : : "r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" : : : "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" : : "n"(N) : "memory"); }
 
 __device__ __forceinline__ float softplus_f(float v) { return v > 20.f ? v : log1pf(expf(v)); }
 __device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); }

@@ -230,12 +230,13 @@ proj_kernel(Shape sh, const float* __restrict__ xbar, const float* __restrict__ 
     }
     const int m = m0 + ml;
     if (m < M) {
+        const int bm = m / sh.T, tm = m - bm * sh.T;
 #pragma unroll
         for (int q = 0; q < kProjQ; ++q) {
             const int jj = jg + 8 * q;
             if (jj < NJ) {
                 const int k = jj / J, j = jj - k * J;
-                u[((size_t)k * M + m) * J + j] = acc[q];
+                u[u_offset(sh, k, bm, tm) + j] = acc[q];
             }
         }
     }
@@ -266,7 +267,6 @@ scan_kernel(Shape sh, const float* __restrict__ xbar, const float* __restrict__ 
     constexpr int ECH = scan_ech<G, ND>();
     extern __shared__ float smem_f[];
     const int T = sh.T, J = sh.J, R = sh.R, N = sh.N, E = sh.E;
-    const int M = sh.B * T;
     const int ntile = (E + ECH - 1) / ECH;
     const int b = blockIdx.x / ntile;
     const int e0 = (blockIdx.x - b * ntile) * ECH;
@@ -277,7 +277,7 @@ scan_kernel(Shape sh, const float* __restrict__ xbar, const float* __restrict__ 
     float* ysum = wdt + ND * ECH * R;    // [T][ECH]     output, summed over directions
 
     for (int k = 0; k < ND; ++k) {
-        const float* src = u + ((size_t)k * M + (size_t)b * T) * J;
+        const float* src = u + u_offset(sh, k, b, 0);
         for (int i = threadIdx.x; i < T * J; i += kThreads) us[k * T * J + i] = src[i];
     }
     for (int i = threadIdx.x; i < T * ECH; i += kThreads) {

@@ -20,6 +20,9 @@ from . import _native as nat
 from .configs import DIR_BWD, DIR_FWD, POOL_H, POOL_W  # noqa: F401
 
 
+_PATH_FLAGS = {"auto": 0, "staged": 2, "fused": 4}
+
+
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -60,6 +63,7 @@ class LayerShape:
     K: int = 0
     pool_scale: float = 1.0
     zoh_exact: bool = False
+    path: str = "auto"  # "auto", "staged" or "fused" (FV_FLAG_PATH_*)
 
     @property
     def nd(self) -> int:
@@ -80,14 +84,14 @@ class LayerShape:
         a.dir_flags = self.dir_flags
         a.K = self.K
         a.pool_scale = float(self.pool_scale)
-        a.flags = nat.FV_FLAG_ZOH_EXACT if self.zoh_exact else 0
+        a.flags = (nat.FV_FLAG_ZOH_EXACT if self.zoh_exact else 0) | _PATH_FLAGS[self.path]
         a.x, a.z, a.A_log, a.D, a.W_x, a.W_dt, a.b_dt, a.keep_idx, a.y = (
             _ptr(x), _ptr(z), _ptr(A_log), _ptr(D), _ptr(W_x), _ptr(W_dt), _ptr(b_dt), _ptr(keep_idx), _ptr(y))
         return a
 
 
 def infer_shape(x, A_log, W_dt, pool_axis, dir_flags, keep_idx=None, h=None, w=None, pool_scale=1.0,
-                zoh_exact=False) -> LayerShape:
+                zoh_exact=False, path="auto") -> LayerShape:
     nd, E, N = A_log.shape
     R = W_dt.shape[2]
     if keep_idx is None:
@@ -103,7 +107,9 @@ def infer_shape(x, A_log, W_dt, pool_axis, dir_flags, keep_idx=None, h=None, w=N
             raise ValueError("a masked layer needs K >= 1 kept tokens")
     if E2 != E:
         raise ValueError(f"x has E={E2}, parameters have E={E}")
-    s = LayerShape(B, h, w, E, N, R, pool_axis, dir_flags, K, pool_scale, zoh_exact)
+    if path not in _PATH_FLAGS:
+        raise ValueError(f"path must be one of {sorted(_PATH_FLAGS)}")
+    s = LayerShape(B, h, w, E, N, R, pool_axis, dir_flags, K, pool_scale, zoh_exact, path)
     if s.nd != nd:
         raise ValueError(f"dir_flags={dir_flags} enables {s.nd} directions, parameters stack {nd}")
     return s
@@ -139,14 +145,14 @@ def alloc_workspace(shape: LayerShape, device=None) -> torch.Tensor:
 
 
 def forward(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis=POOL_W, dir_flags=DIR_FWD | DIR_BWD, keep_idx=None,
-            h=None, w=None, pool_scale=1.0, zoh_exact=False, y=None, workspace=None, stream=None):
+            h=None, w=None, pool_scale=1.0, zoh_exact=False, y=None, workspace=None, stream=None, path="auto"):
     """Queue the layer on ``stream`` (default: the current stream) and return y."""
     dev = x.device
     for name, t in (("x", x), ("z", z), ("A_log", A_log), ("D", D), ("W_x", W_x), ("W_dt", W_dt), ("b_dt", b_dt)):
         _check_tensor(name, t, torch.float32, dev)
     if keep_idx is not None:
         _check_tensor("keep_idx", keep_idx, torch.int32, dev)
-    shape = infer_shape(x, A_log, W_dt, pool_axis, dir_flags, keep_idx, h, w, pool_scale, zoh_exact)
+    shape = infer_shape(x, A_log, W_dt, pool_axis, dir_flags, keep_idx, h, w, pool_scale, zoh_exact, path)
     if z.shape != x.shape:
         raise ValueError("z must have the shape of x")
     if y is None:

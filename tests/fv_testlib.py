@@ -39,7 +39,7 @@ def assert_close(got, ref, what="y"):
 
 
 def gpu_forward(inp: dict, pool_axis: int, dir_flags: int, h=None, w=None, pool_scale=1.0, zoh_exact=False,
-                intermediates=True):
+                intermediates=True, path="auto"):
     """Run the CUDA layer on numpy inputs; return y (and workspace intermediates) as numpy."""
     import torch
 
@@ -48,12 +48,14 @@ def gpu_forward(inp: dict, pool_axis: int, dir_flags: int, h=None, w=None, pool_
     dev = torch.device("cuda")
     t = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev) for k, v in inp.items() if v is not None}
     keep = t.get("keep_idx")
-    shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, dir_flags, keep, h, w, pool_scale, zoh_exact)
+    shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, dir_flags, keep, h, w, pool_scale, zoh_exact,
+                            path)
     ws = ssm.alloc_workspace(shape, dev)
+    ws.fill_(0xFF)  # poison: every intermediate must be written before it is read
     y = ssm.forward(t["x"], t["z"], t["A_log"], t["D"], t["W_x"], t["W_dt"], t["b_dt"], pool_axis, dir_flags,
-                    keep_idx=keep, h=h, w=w, pool_scale=pool_scale, zoh_exact=zoh_exact, workspace=ws)
+                    keep_idx=keep, h=h, w=w, pool_scale=pool_scale, zoh_exact=zoh_exact, workspace=ws, path=path)
     status = ssm.device_status(ws)
-    out = dict(y=y.cpu().numpy(), status=status)
+    out = dict(y=y.cpu().numpy(), status=status, launches=ssm.launch_names(shape))
     if intermediates:
         L = ssm.workspace_layout(shape)
         B, T, E, nd, J = shape.B, L["T"], shape.E, L["nd"], shape.R + 2 * shape.N
@@ -63,7 +65,8 @@ def gpu_forward(inp: dict, pool_axis: int, dir_flags: int, h=None, w=None, pool_
             return ws[off:off + nbytes].cpu().numpy().view(dtype).copy()
 
         out["xbar"] = view(L["xbar"], B * T * E, np.float32).reshape(B, T, E)
-        out["u"] = view(L["u"], nd * B * T * J, np.float32).reshape(nd, B, T, J)
+        ub = -(-T * J // 32) * 32  # per (direction, image) block stride, floats
+        out["u"] = view(L["u"], nd * B * ub, np.float32).reshape(nd, B, ub)[:, :, :T * J].reshape(nd, B, T, J)
         out["ys"] = view(L["ys"], B * T * E, np.float32).reshape(B, T, E)
         if shape.K:
             out["row_of"] = view(L["row_of"], B * shape.K, np.int32).reshape(B, shape.K)

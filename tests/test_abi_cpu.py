@@ -103,7 +103,7 @@ def test_valid_dense_and_masked(lib):
     ("h", 0, nat.FV_ERR_SHAPE), ("N", 0, nat.FV_ERR_SHAPE), ("R", 0, nat.FV_ERR_SHAPE),
     ("N", 17, nat.FV_ERR_UNSUPPORTED), ("R", 70, nat.FV_ERR_UNSUPPORTED),
     ("pool_axis", 2, nat.FV_ERR_SHAPE), ("dir_flags", 0, nat.FV_ERR_SHAPE), ("dir_flags", 4, nat.FV_ERR_SHAPE),
-    ("flags", 2, nat.FV_ERR_SHAPE), ("K", 14 * 14 + 1, nat.FV_ERR_SHAPE), ("K", -3, nat.FV_ERR_SHAPE),
+    ("flags", 16, nat.FV_ERR_SHAPE), ("flags", 6, nat.FV_ERR_SHAPE), ("K", 14 * 14 + 1, nat.FV_ERR_SHAPE), ("K", -3, nat.FV_ERR_SHAPE),
     ("pool_scale", float("nan"), nat.FV_ERR_SHAPE),
     ("x", None, nat.FV_ERR_NULL), ("y", None, nat.FV_ERR_NULL), ("W_x", None, nat.FV_ERR_NULL),
     ("b_dt", None, nat.FV_ERR_NULL), ("x", FAKE + 4, nat.FV_ERR_ALIGN), ("D", FAKE + 8, nat.FV_ERR_ALIGN),
@@ -154,9 +154,12 @@ def test_workspace_layout(lib, pool_axis, K):
     assert lib.fastvim_ssm_workspace_layout(ctypes.byref(a), ctypes.byref(L)) == nat.FV_OK
     T = 6 if pool_axis == 0 else 9
     assert (L.T, L.S, L.nd) == (T, 15 - T, 2)
-    regions = [(L.status, 4), (L.xbar, 3 * T * 64 * 4), (L.u, 2 * 3 * T * 36 * 4), (L.ys, 3 * T * 64 * 4)]
+    ub = -(-T * 36 // 32) * 32
+    regions = [(L.status, 4), (L.xbar, 3 * T * 64 * 4), (L.u, 2 * 3 * ub * 4), (L.ys, 3 * T * 64 * 4)]
     if K:
         regions += [(L.row_of, 3 * K * 4), (L.row_off, 3 * (T + 1) * 4), (L.row_tok, 3 * K * 4)]
+    else:
+        regions += [(L.ctrl, (64 + 3 * 3) * 4)]
     end = 0
     for off, size in regions:
         assert off % 256 == 0 and off >= end
@@ -164,3 +167,21 @@ def test_workspace_layout(lib, pool_axis, K):
     assert L.total_bytes >= end
     assert lib.fastvim_ssm_workspace_size(ctypes.byref(a)) == L.total_bytes
     assert lib.fastvim_ssm_launch_count(ctypes.byref(a)) == (5 if K else 4)
+
+
+@pytest.mark.parametrize("flags,want", [(0, ["fused_layer_kernel"]), (4, ["fused_layer_kernel"]),
+                                        (2, ["pool_dense_kernel", "proj_kernel", "scan_kernel",
+                                             "epilogue_dense_kernel"])])
+def test_path_selection_is_host_side(lib, flags, want):
+    a = good_args(h=128, w=128, B=4, flags=flags)  # 2048 px FastVim-T images: fused by default
+    n = lib.fastvim_ssm_launch_count(ctypes.byref(a))
+    names = [lib.fastvim_ssm_launch_name(ctypes.byref(a), i).decode() for i in range(n)]
+    assert names == want
+    small = good_args(flags=flags)  # 224 px: staged unless forced
+    n = lib.fastvim_ssm_launch_count(ctypes.byref(small))
+    assert n == (1 if flags == 4 else 4)
+
+
+def test_forced_fused_path_refuses_masked_layers(lib):
+    a = good_args(K=49, keep_idx=FAKE + (9 << 32), flags=4)
+    assert lib.fastvim_ssm_launch_count(ctypes.byref(a)) == 0

@@ -39,20 +39,26 @@ def rand_layer(seed, B, h, w, E, N, R, dir_flags, K=0, dt_hi=0.1):
 
 
 def check_layer(p, pool_axis, dir_flags, h=None, w=None, pool_scale=1.0, zoh_exact=False):
+    """Both implementations of a dense layer (staged kernels and the fused launch), or the staged
+    masked one, against the oracle: intermediates and output."""
     keep = p.get("keep_idx")
     ref = oracle.forward_intermediates(p["x"], p["z"], p["A_log"], p["D"], p["W_x"], p["W_dt"], p["b_dt"],
                                        pool_axis, dir_flags, keep_idx=keep, h=h, w=w, pool_scale=pool_scale,
                                        zoh_exact=zoh_exact)
-    got = gpu_forward(p, pool_axis, dir_flags, h=h, w=w, pool_scale=pool_scale, zoh_exact=zoh_exact)
-    assert got["status"] == 0
-    if keep is not None:
-        assert np.array_equal(got["row_of"], ref["row_of"])
-        assert np.array_equal(got["row_off"], ref["row_off"])
-        assert np.array_equal(got["row_tok"], ref["row_tok"])
-    assert_close(got["xbar"], ref["xbar"], "xbar")
-    assert_close(got["u"], ref["u"], "u")
-    assert_close(got["ys"], ref["ys"], "ys")
-    return assert_close(got["y"], ref["y"], "y")
+    rep = None
+    for path in (("staged",) if keep is not None else ("staged", "fused")):
+        got = gpu_forward(p, pool_axis, dir_flags, h=h, w=w, pool_scale=pool_scale, zoh_exact=zoh_exact, path=path)
+        assert got["status"] == 0, path
+        assert (got["launches"] == ["fused_layer_kernel"]) == (path == "fused")
+        if keep is not None:
+            assert np.array_equal(got["row_of"], ref["row_of"])
+            assert np.array_equal(got["row_off"], ref["row_off"])
+            assert np.array_equal(got["row_tok"], ref["row_tok"])
+        assert_close(got["xbar"], ref["xbar"], f"{path} xbar")
+        assert_close(got["u"], ref["u"], f"{path} u")
+        assert_close(got["ys"], ref["ys"], f"{path} ys")
+        rep = assert_close(got["y"], ref["y"], f"{path} y")
+    return rep
 
 
 def test_config0_tiny_fastvim_t():
@@ -111,6 +117,26 @@ def test_masked_nonsquare_and_wide():
     p = rand_layer(120, B=2, h=5, w=12, E=1040, N=16, R=16, dir_flags=3, K=33)
     check_layer(p, 0, 3, h=5, w=12)
     check_layer(p, 1, 3, h=5, w=12)
+
+
+@pytest.mark.parametrize("lag", ["2", "3", "4", "9"])
+def test_fused_pipeline_lags(lag, monkeypatch):
+    monkeypatch.setenv("FASTVIM_FUSED_LAG", lag)
+    p = rand_layer(125, B=7, h=24, w=20, E=136, N=16, R=6, dir_flags=3)
+    ref = oracle.forward(p["x"], p["z"], p["A_log"], p["D"], p["W_x"], p["W_dt"], p["b_dt"], 0, 3)
+    got = gpu_forward(p, 0, 3, path="fused", intermediates=False)
+    assert got["status"] == 0 and got["launches"] == ["fused_layer_kernel"]
+    assert_close(got["y"], ref)
+
+
+def test_path_auto_choice():
+    from pooled_selective_scan_b200 import ssm
+    big = ssm.LayerShape(B=2, h=64, w=64, E=384, N=16, R=12, pool_axis=0, dir_flags=3)
+    small = ssm.LayerShape(B=2, h=14, w=14, E=384, N=16, R=12, pool_axis=0, dir_flags=3)
+    masked = ssm.LayerShape(B=2, h=64, w=64, E=384, N=16, R=12, pool_axis=0, dir_flags=3, K=100)
+    assert ssm.launch_names(big) == ["fused_layer_kernel"]
+    assert ssm.launch_names(small) == ["pool_dense_kernel", "proj_kernel", "scan_kernel", "epilogue_dense_kernel"]
+    assert ssm.launch_names(masked)[0] == "mask_bucket_kernel"
 
 
 def test_masked_all_kept_equals_dense():
