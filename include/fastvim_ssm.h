@@ -89,7 +89,7 @@ enum {
     FV_FLAG_TRACE = 8u        /* fused launch: record one entry per task in the workspace
                                  (fv_ws_layout.trace); costs a little time, for profiling      */
 };
-/* Without a PATH flag a dense layer whose images hold >= 1 MiB of x runs the fused launch, every
+/* Without a PATH flag a dense layer whose images hold >= 16 MiB of x runs the fused launch, every
  * other layer the staged kernels; both compute the same layer.  The fused launch keeps each
  * image's x in L2 between pooling and the epilogue; the environment variable FASTVIM_FUSED_LAG
  * (2..64, read per call) overrides how many images it lets lie between the two, and
@@ -131,6 +131,8 @@ typedef struct {
                             w1 = SM id << 32 | CTA id, w2 = start (ns, %globaltimer),
                             w3 = wait_ns << 40 | total_ns (from start to the task's end)        */
     size_t trace_records;  /* number of trace entries (tasks of the call), else 0               */
+    size_t scan_bc;      /* dense layers: fused launch's B | C rows in scan order, else 0        */
+    size_t scan_dt;      /* dense layers: fused launch's dt_low rows, else 0                     */
     int T, S, nd;        /* pooled length, pooled-over length, number of directions          */
 } fv_ws_layout;
 

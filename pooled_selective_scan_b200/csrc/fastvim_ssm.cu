@@ -28,15 +28,6 @@ size_t round256(size_t v) { return (v + 255) & ~(size_t)255; }
 constexpr int kMaxT = 4096;
 constexpr long long kMaxMaskGrid = 1ll << 20;
 
-// Lanes per (direction, channel) in the scan: 4 states per lane.
-int scan_lanes(int N) { return N <= 4 ? 1 : (N <= 8 ? 2 : 4); }
-
-size_t scan_smem_bytes(const fv::Shape& sh) {
-    return fv::scan_smem_floats(sh.T, sh.J, sh.R, scan_lanes(sh.N), sh.nd) * sizeof(float);
-}
-size_t proj_smem_bytes(const fv::Shape& sh) {
-    return (size_t)(fv::kProjRows * 33 + sh.NJ * 33) * sizeof(float);
-}
 size_t bucket_smem_bytes(const fv::Shape& sh) {
     const long long G = (long long)sh.h * sh.w;
     return (size_t)(((G + 31) >> 5) + 2ll * sh.T) * sizeof(unsigned);
@@ -107,12 +98,15 @@ fv_status plan_layout(const fv::Shape& sh, fv_ws_layout* L) {
     L->xbar = off; off = round256(off + (size_t)sh.B * sh.T * sh.E * sizeof(float));
     L->u = off; off = round256(off + (size_t)sh.nd * sh.B * fv::u_block_stride(sh.T, sh.J) * sizeof(float));
     L->ys = off; off = round256(off + (size_t)sh.B * sh.T * sh.E * sizeof(float));
+    // scan-ready copies of B | C (chunk-interleaved rows) and dt_low, written by the projections
+    L->scan_bc = off; off = round256(off + (size_t)sh.nd * sh.B * fv::fused_bcs_stride(sh.T) * sizeof(float));
+    L->scan_dt = off; off = round256(off + (size_t)sh.nd * sh.B * fv::fused_dts_stride(sh.T, sh.R) * sizeof(float));
     if (sh.K > 0) {
         L->row_of = off; off = round256(off + (size_t)sh.B * sh.K * sizeof(int32_t));
         L->row_off = off; off = round256(off + (size_t)sh.B * (sh.T + 1) * sizeof(int32_t));
         L->row_tok = off; off = round256(off + (size_t)sh.B * sh.K * sizeof(int32_t));
     } else {
-        // dense layers: the control block of the fused single-launch path
+        // dense layers: the control block of the fused launch
         L->ctrl = off; off = round256(off + (size_t)(fv::kCtrlHeaderWords + fv::kCtrlCounters * (size_t)sh.B) * sizeof(unsigned));
         if (sh.trace && choose_path(sh) == Path::Fused) {
             const fv::FusedPlan pl = plan_fused(sh);
@@ -132,7 +126,8 @@ constexpr size_t kMaxSmemOptin = 227 * 1024;
 constexpr double kChainLatencyUs = 60.0;
 
 fv_status check_limits(const fv::Shape& sh) {
-    if (scan_smem_bytes(sh) > kMaxSmemOptin) return FV_ERR_UNSUPPORTED;
+    if (fv::fused_scan_smem_floats(sh) * sizeof(float) > kMaxSmemOptin) return FV_ERR_UNSUPPORTED;
+    if (fv::fused_proj_smem_floats(sh) * sizeof(float) > kMaxSmemOptin) return FV_ERR_UNSUPPORTED;
     if (sh.K > 0 && bucket_smem_bytes(sh) > kMaxSmemOptin) return FV_ERR_UNSUPPORTED;
     return FV_OK;
 }
@@ -164,14 +159,16 @@ bool fused_possible(const fv::Shape& sh) {
     return true;
 }
 
-// Which implementation runs: the fused single launch for dense layers whose images are large
-// enough to stream (>= 1 MiB of x per image), the staged kernels otherwise; flags can force either.
+// Which implementation runs: the fused single launch for dense layers with large images (>= 16 MiB
+// of x per image: there the overlap of projections and scans with streaming pays; measured on B200,
+// 2.19 vs 2.35 ms at 2048 px, while at 1024 px the staged kernels win, 1.41 vs 1.83 ms), the staged
+// kernels otherwise; flags can force either.
 Path choose_path(const fv::Shape& sh) {
     const bool ok = fused_possible(sh);
     if (sh.path_flags & FV_FLAG_PATH_STAGED) return Path::Staged;
     if (sh.path_flags & FV_FLAG_PATH_FUSED) return ok ? Path::Fused : Path::Invalid;
     const size_t img = (size_t)sh.h * sh.w * sh.E * sizeof(float);
-    return (ok && img >= ((size_t)1 << 20)) ? Path::Fused : Path::Staged;
+    return (ok && img >= ((size_t)16 << 20)) ? Path::Fused : Path::Staged;
 }
 
 fv::FusedPlan plan_fused(const fv::Shape& sh) {
@@ -189,14 +186,14 @@ fv::FusedPlan plan_fused(const fv::Shape& sh) {
     // ~6.5 TB/s).  (Keeping x in L2 across that window does not happen: traffic of this size
     // evicts first-touch lines whatever their L2 eviction priority.)
     const double round_us = (double)sh.h * sh.w * sh.E * 16.0 / 6.5e6;
-    long long lag = (long long)(kChainLatencyUs / (round_us > 0.01 ? round_us : 0.01)) + 2;
+    long long lag = (long long)(kChainLatencyUs / (round_us > 0.01 ? round_us : 0.01)) + 3;
     if (const char* env = getenv("FASTVIM_FUSED_LAG")) {
         const long long v = atoll(env);
-        if (v >= 2 && v <= 64) lag = v;
+        if (v >= 3 && v <= 64) lag = v;
     }
-    // E of image r-L is dequeued before S of image r-1 within round r, so L >= 2 keeps every
-    // consumer after its producers in ticket order (the deadlock-freedom argument above).
-    pl.L = (int)(lag < 2 ? 2 : (lag > 64 ? 64 : lag));
+    // Image b's scans come in round b+2, its gates in round b+L: L >= 3 keeps every consumer after
+    // its producers in ticket order (the deadlock-freedom argument of the fused kernel).
+    pl.L = (int)(lag < 3 ? 3 : (lag > 64 ? 64 : lag));
     pl.B = sh.B;
     // rounds r = 0 .. B+L-1; [R1, R2) hold Q, P, E and S alike
     const int rounds = sh.B + pl.L;
@@ -230,39 +227,6 @@ cudaError_t ensure_smem(Kern kernel, size_t bytes) {
         }                                              \
     } while (0)
 
-template <int G, int ND, bool Z>
-fv_status launch_scan_t(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws,
-                        cudaStream_t st) {
-    constexpr int ECH = fv::scan_ech<G, ND>();
-    const size_t smem = scan_smem_bytes(sh);
-    auto kern = fv::scan_kernel<G, ND, Z>;
-    cudaError_t e = ensure_smem(kern, smem);
-    if (e != cudaSuccess) { note_cuda(e, "scan smem attribute"); return FV_ERR_CUDA; }
-    const int ntile = (sh.E + ECH - 1) / ECH;
-    kern<<<sh.B * ntile, fv::kThreads, smem, st>>>(sh, (const float*)(ws + L.xbar), (const float*)(ws + L.u),
-                                                  a->A_log, a->W_dt, a->b_dt, (float*)(ws + L.ys));
-    FV_LAUNCH_CHECK("scan_kernel");
-    return FV_OK;
-}
-
-template <int G, int ND>
-fv_status launch_scan_z(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st) {
-    return sh.zoh_exact ? launch_scan_t<G, ND, true>(sh, a, L, ws, st) : launch_scan_t<G, ND, false>(sh, a, L, ws, st);
-}
-
-template <int G>
-fv_status launch_scan_g(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st) {
-    return sh.nd == 2 ? launch_scan_z<G, 2>(sh, a, L, ws, st) : launch_scan_z<G, 1>(sh, a, L, ws, st);
-}
-
-fv_status launch_scan(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st) {
-    switch (scan_lanes(sh.N)) {
-        case 1: return launch_scan_g<1>(sh, a, L, ws, st);
-        case 2: return launch_scan_g<2>(sh, a, L, ws, st);
-        default: return launch_scan_g<4>(sh, a, L, ws, st);
-    }
-}
-
 // Records events[i] just before the i-th kernel launch and events[n] after the last one when an
 // event list is given (n = the call's launch count).
 struct EventMarks {
@@ -292,8 +256,9 @@ int launch_count_of(const fv::Shape& sh) {
 }
 
 const char* launch_name_of(const fv::Shape& sh, int i) {
-    static const char* dense[] = {"pool_dense_kernel", "proj_kernel", "scan_kernel", "epilogue_dense_kernel"};
-    static const char* masked[] = {"mask_bucket_kernel", "mask_pool_kernel", "proj_kernel", "scan_kernel",
+    static const char* dense[] = {"pool_dense_kernel", "proj_tasks_kernel", "scan_tasks_kernel",
+                                  "epilogue_dense_kernel"};
+    static const char* masked[] = {"mask_bucket_kernel", "mask_pool_kernel", "proj_tasks_kernel", "scan_tasks_kernel",
                                    "mask_epilogue_kernel"};
     if (i < 0 || i >= launch_count_of(sh)) return "";
     if (choose_path(sh) == Path::Fused) return "fused_layer_kernel";
@@ -320,19 +285,59 @@ fv_status launch_fused_t(const fv::Shape& sh, const fv::FusedPlan& pl, const fv:
     return FV_OK;
 }
 
-fv_status launch_fused(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st) {
-    const fv::FusedPlan pl = plan_fused(sh);
+fv::FusedPtrs fused_ptrs(const fv_ssm_args* a, const fv_ws_layout& L, char* ws) {
     fv::FusedPtrs p;
     p.x = a->x; p.z = a->z; p.A_log = a->A_log; p.D = a->D; p.W_x = a->W_x; p.W_dt = a->W_dt; p.b_dt = a->b_dt;
     p.y = a->y;
     p.xbar = (float*)(ws + L.xbar);
     p.u = (float*)(ws + L.u);
     p.ys = (float*)(ws + L.ys);
+    p.bcs = (float*)(ws + L.scan_bc);
+    p.dts = (float*)(ws + L.scan_dt);
     p.status = (unsigned*)(ws + L.status);
-    p.ctrl = (unsigned*)(ws + L.ctrl);
+    p.ctrl = L.ctrl ? (unsigned*)(ws + L.ctrl) : nullptr;
     p.trace = L.trace_records ? (unsigned long long*)(ws + L.trace) : nullptr;
+    return p;
+}
+
+fv_status launch_fused(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st) {
+    const fv::FusedPlan pl = plan_fused(sh);
+    const fv::FusedPtrs p = fused_ptrs(a, L, ws);
     if (sh.nd == 2) return sh.zoh_exact ? launch_fused_t<2, true>(sh, pl, p, st) : launch_fused_t<2, false>(sh, pl, p, st);
     return sh.zoh_exact ? launch_fused_t<1, true>(sh, pl, p, st) : launch_fused_t<1, false>(sh, pl, p, st);
+}
+
+// Staged: x_proj over every pooled token (one CTA per 16 tokens of an image).
+fv_status launch_proj_tasks(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st) {
+    const fv::FusedPlan pl = plan_fused(sh);
+    fv::FusedPtrs p = fused_ptrs(a, L, ws);
+    p.ctrl = nullptr;
+    const size_t smem = fv::fused_proj_smem_floats(sh) * sizeof(float);
+    cudaError_t e = ensure_smem(fv::proj_tasks_kernel, smem);
+    if (e != cudaSuccess) { note_cuda(e, "proj smem attribute"); return FV_ERR_CUDA; }
+    fv::proj_tasks_kernel<<<sh.B * pl.nQ, fv::kFusedThreads, smem, st>>>(sh, pl, p);
+    FV_LAUNCH_CHECK("proj_tasks_kernel");
+    return FV_OK;
+}
+
+// Staged: scans of every channel tile of every image (one CTA per tile).
+template <int ND, bool Z>
+fv_status launch_scan_tasks_t(const fv::Shape& sh, const fv::FusedPlan& pl, const fv::FusedPtrs& p, cudaStream_t st) {
+    const size_t smem = fv::fused_scan_smem_floats(sh) * sizeof(float);
+    auto kern = fv::scan_tasks_kernel<ND, Z>;
+    cudaError_t e = ensure_smem(kern, smem);
+    if (e != cudaSuccess) { note_cuda(e, "scan smem attribute"); return FV_ERR_CUDA; }
+    kern<<<sh.B * pl.nS, fv::kFusedThreads, smem, st>>>(sh, pl, p);
+    FV_LAUNCH_CHECK("scan_tasks_kernel");
+    return FV_OK;
+}
+fv_status launch_scan_tasks(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st) {
+    const fv::FusedPlan pl = plan_fused(sh);
+    fv::FusedPtrs p = fused_ptrs(a, L, ws);
+    p.ctrl = nullptr;
+    if (sh.nd == 2)
+        return sh.zoh_exact ? launch_scan_tasks_t<2, true>(sh, pl, p, st) : launch_scan_tasks_t<2, false>(sh, pl, p, st);
+    return sh.zoh_exact ? launch_scan_tasks_t<1, true>(sh, pl, p, st) : launch_scan_tasks_t<1, false>(sh, pl, p, st);
 }
 
 fv_status forward_impl(const fv_ssm_args* a, void* ws_v, size_t ws_bytes, cudaStream_t st,
@@ -390,11 +395,9 @@ fv_status forward_impl(const fv_ssm_args* a, void* ws_v, size_t ws_bytes, cudaSt
         FV_LAUNCH_CHECK("mask_pool_kernel");
     }
     FV_MARK(marks, st);
-    fv::proj_kernel<<<(M + fv::kProjRows - 1) / fv::kProjRows, fv::kThreads, proj_smem_bytes(sh), st>>>(
-        sh, xbar, a->W_x, (float*)(ws + L.u));
-    FV_LAUNCH_CHECK("proj_kernel");
+    if ((s = launch_proj_tasks(sh, a, L, ws, st)) != FV_OK) return s;
     FV_MARK(marks, st);
-    if ((s = launch_scan(sh, a, L, ws, st)) != FV_OK) return s;
+    if ((s = launch_scan_tasks(sh, a, L, ws, st)) != FV_OK) return s;
     FV_MARK(marks, st);
     if (sh.K == 0) {
         fv::epilogue_dense_kernel<<<M, fv::kThreads, 0, st>>>(sh, a->x, a->z, (const float*)(ws + L.ys), a->D, a->y);

@@ -9,9 +9,6 @@ namespace fv {
 constexpr int kThreads = 256;       // every kernel of the layer runs 256-thread CTAs
 constexpr int kMaxN = 16;           // d_state limit: 4 lanes x 4 states in the scan
 constexpr int kMaxJ = 96;           // R + 2N limit per direction
-constexpr int kProjRows = 32;       // pooled tokens per projection CTA
-constexpr int kProjChunk = 32;      // channels per projection K-step
-constexpr int kProjQ = (2 * kMaxJ + 7) / 8;  // outputs per thread in the projection
 
 // Device status codes (the values of fv_status that kernels may record).
 constexpr unsigned kStatusIndex = 4u;

@@ -1,21 +1,22 @@
-// fv_fused.cuh -- the dense FastVim SSM layer as ONE persistent, image-pipelined launch (sm_100a).
+// fv_fused.cuh -- the dense FastVim SSM layer as ONE persistent, image-pipelined launch (sm_100a),
+// and the task bodies that the staged launches reuse.
 //
-// Why: the layer's algorithmic traffic is x read once, z read once, y written once (12 E bytes
-// per grid token), but the pooled tokens of an image depend on ALL of its x and every output
-// token depends on the whole image's scan.  Run as separate kernels, x is read from HBM twice
-// (pool, then epilogue).  Here one launch streams the images through four task kinds,
+// The layer's pooled tokens depend on ALL of an image's x, and every output token depends on the
+// whole image's scan, so x must be read once for pooling and once more for the D x skip.  One
+// persistent launch (two 256-thread CTAs per SM) streams the images through four task kinds,
 //
-//   P(b, g)  pool LP grid lines of image b into pooled tokens     (TMA ring: reads x, keeps it in L2)
-//   Q(b, q)  x_proj of 16 pooled tokens of image b                (fp32 GEMM, cp.async tiles)
+//   P(b, g)  pool LP grid lines of image b into pooled tokens     (TMA bulk-copy ring over x)
+//   Q(b, q)  x_proj of 16 pooled tokens of image b                (fp32 GEMM, cp.async pipeline)
 //   S(b, c)  dt_proj + softplus, ZOH and the forward/backward scans of a channel tile of image b
-//   E(b, g)  repeat + D x skip + SiLU(z) gate for LP grid lines  (TMA ring: x from L2, z; y stored)
+//   E(b, g)  repeat + D x skip + SiLU(z) gate for LP grid lines  (TMA ring over x and z; y stored)
 //
-// taken from a global ticket counter in the order  [Q_{r-1}][P_r][E_{r-L}][S_{r-1}]  for r = 0, 1,
-// ... so that image b's x is loaded by P_b with an L2 evict-last policy and consumed by E_b about L
-// rounds later while the GPU keeps streaming other images: x crosses HBM once as long as the x of
-// the images in between fits in L2 (126 MB on B200; 25 MB per 2048 px FastVim-T image).  Within a
-// round the projections of the previous image come first (its pools finished during the previous
-// round) and its scans come last (after the round's streaming tasks), so that neither waits long.
+// taken from a global ticket counter in the order  [Q_{r-1}][P_r][E_{r-L}][S_{r-2}]  for r = 0, 1,
+// ..., so that every CTA keeps streaming while other CTAs project and scan: the x_proj GEMMs, the
+// scans and all the waits between them overlap the HBM traffic of other images.  Each image's
+// projections come one round after its pools and its scans one round after that, and its gates
+// L >= 3 rounds after its pools, so that consumers rarely wait.  (Keeping x in the 126 MB L2
+// between pool and gate does not work at these traffic volumes: first-touch lines are evicted
+// whatever their eviction priority, so x is simply streamed twice.)
 //
 // Dependencies are per-image counters (pool, proj, scan) released by producer CTAs and acquired by
 // consumer CTAs.  A CTA only ever waits for tasks with smaller tickets, which were handed to CTAs
@@ -47,6 +48,9 @@ constexpr int kMaxSlots = 2;             // float4 slots per thread in P tasks: 
 constexpr int kQT = 16;                  // pooled tokens per projection task
 constexpr int kQK = 32;                  // channels per projection K-step
 constexpr int kQPad = kQK + 4;           // padded row of a projection tile (16-byte aligned)
+// cp.async pipeline depth of the projection K-loop for TN = 3, 4, 6 outputs per thread
+__host__ __device__ constexpr int q_stages(int TN) { return TN <= 3 ? 5 : (TN == 4 ? 4 : 3); }
+__host__ __device__ constexpr int q_tn(int NJ) { return NJ <= 96 ? 3 : (NJ <= 128 ? 4 : 6); }
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
 // Control block at the start of the fused workspace region (zeroed before every call):
@@ -84,8 +88,10 @@ struct FusedPtrs {
     const float* b_dt;
     float* y;
     float* xbar;   // [B][T][E]
-    float* u;      // [nd][B*T][J]
+    float* u;      // [nd][B] blocks of [T][J] (see u_offset)
     float* ys;     // [B][T][E]
+    float* bcs;    // [nd][B][8 CL][kBCStride]: B | C rows in the scan's chunk-interleaved order
+    float* dts;    // [nd][B][Tr]: dt_low rows [T][R], block padded to Tr = ceil(T R / 32) * 32
     unsigned* status;
     unsigned* ctrl;
     unsigned long long* trace;  // NULL, or 4 words per ticket
@@ -99,19 +105,32 @@ struct Ring {
 };
 
 __host__ __device__ __forceinline__ int fused_ech(int nd) { return kFusedThreads / (kScanChunks * nd); }
+// Per-(direction, image) block strides of the scan-ready copies, in floats.
+__host__ __device__ __forceinline__ size_t fused_bcs_stride(int T) {
+    return (size_t)kScanChunks * ((T + kScanChunks - 1) / kScanChunks) * kBCStride;
+}
+__host__ __device__ __forceinline__ size_t fused_dts_stride(int T, int R) { return (((size_t)T * R + 31) / 32) * 32; }
 __host__ __device__ __forceinline__ int fused_xstride(int nd) { return fused_ech(nd) + 4; }
 
-// Dynamic shared memory (floats) per task kind; the launch takes the maximum.
-__host__ __device__ __forceinline__ size_t fused_smem_floats(const Shape& sh, int LP) {
+// Dynamic shared memory (floats) per task kind; the fused launch takes the maximum.
+__host__ __device__ __forceinline__ size_t fused_proj_smem_floats(const Shape& sh) {
+    const int tn = q_tn(sh.NJ);
+    return (size_t)q_stages(tn) * ((size_t)kQT * kQPad + (size_t)32 * tn * kQPad);
+}
+__host__ __device__ __forceinline__ size_t fused_scan_smem_floats(const Shape& sh) {
     const int CL = (sh.T + kScanChunks - 1) / kScanChunks;
     const size_t rows = (size_t)kScanChunks * CL;
     const int XS = fused_xstride(sh.nd);
+    return (size_t)sh.nd * rows * kBCStride + (size_t)(sh.nd + 1) * rows * XS +
+           (size_t)sh.nd * fused_dts_stride(sh.T, sh.R) + (size_t)sh.nd * fused_ech(sh.nd) * (sh.R + 1) +
+           (size_t)sh.T;
+}
+__host__ __device__ __forceinline__ size_t fused_smem_floats(const Shape& sh, int LP) {
     const size_t ring = (size_t)kRingStages * kStageBytes / 4;
     const size_t pool = ring + (size_t)kFusedThreads * 4;
     const size_t gate = ring + (size_t)(LP + 1) * sh.E;
-    const size_t proj = 2 * ((size_t)kQT * kQPad + (size_t)sh.NJ * kQPad);
-    const size_t scan = (size_t)sh.nd * rows * kBCStride + (size_t)(sh.nd + 1) * rows * XS +
-                        (size_t)sh.nd * sh.T * sh.R + (size_t)sh.nd * fused_ech(sh.nd) * (sh.R + 1) + (size_t)sh.T;
+    const size_t proj = fused_proj_smem_floats(sh);
+    const size_t scan = fused_scan_smem_floats(sh);
     size_t m = pool > gate ? pool : gate;
     m = m > proj ? m : proj;
     return m > scan ? m : scan;
@@ -119,7 +138,7 @@ __host__ __device__ __forceinline__ size_t fused_smem_floats(const Shape& sh, in
 
 // Ticket -> (task kind, image, index within the image).  Round r holds, in this order,
 //   Q of image r-1 (if 0 <= r-1 < B), P of image r (if r < B), E of image r-L (if 0 <= r-L < B),
-//   S of image r-1 (if 0 <= r-1 < B),
+//   S of image r-2 (if 0 <= r-2 < B),
 // for r = 0 .. B+L-1.  Rounds [R1, R2) all have the same composition; the few rounds outside are
 // walked one by one.
 __host__ __device__ __forceinline__ void fused_round_parts(const FusedPlan& pl, int r, bool& q, bool& pp, bool& ee,
@@ -127,7 +146,7 @@ __host__ __device__ __forceinline__ void fused_round_parts(const FusedPlan& pl, 
     q = (r >= 1 && r - 1 < pl.B);
     pp = r < pl.B;
     ee = (r >= pl.L && r - pl.L < pl.B);
-    ss = q;
+    ss = (r >= 2 && r - 2 < pl.B);
 }
 __host__ __device__ __forceinline__ unsigned fused_round_size(const FusedPlan& pl, int r) {
     bool q, pp, ee, ss;
@@ -170,7 +189,7 @@ __device__ __forceinline__ void fused_decode(const FusedPlan& pl, unsigned tk, i
         off -= pl.nP;
     }
     kind = kTaskScan;
-    b = r - 1;
+    b = r - 2;
     idx = (int)off;
 }
 
@@ -198,10 +217,11 @@ __device__ __forceinline__ bool cta_wait(const unsigned* cnt, unsigned target, u
     return *s_flag != 0;
 }
 
-// All of this CTA's global writes so far become visible before the counter moves.
+// All of this CTA's global writes so far become visible before the counter moves (no counter:
+// the task runs in a staged launch, where the launch boundary orders it).
 __device__ __forceinline__ void cta_signal(unsigned* cnt) {
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && cnt) {
         __threadfence();
         red_release_gpu_add(cnt, 1u);
     }
@@ -363,94 +383,122 @@ __device__ __forceinline__ bool fused_pool(const Shape& sh, const FusedPlan& pl,
                        pol_keep);
     }
     rg.count = g0 + nq;
-    cta_signal(p.ctrl + kCtrlHeaderWords + b);
+    cta_signal(p.ctrl ? p.ctrl + kCtrlHeaderWords + b : nullptr);
     return true;
 }
 
 // ---- Q: x_proj of pooled tokens [q*16, q*16+16) of image b ------------------------------------
-// u = W_x . xbar as a register-blocked fp32 GEMM (2 tokens x TN outputs per thread: TN = 3 for
-// nd(R+2N) <= 96 outputs, 6 up to 192), 32-channel K-steps double-buffered through cp.async.
-template <int TN>
-__device__ __forceinline__ void fused_proj_t(const Shape& sh, const FusedPtrs& p, int b, int q, float* smem) {
-    const int T = sh.T, E = sh.E, J = sh.J, NJ = sh.NJ;
+// u = W_x . xbar as a register-blocked fp32 GEMM (2 tokens x TN outputs per thread: TN = 3, 4 or
+// 6 for nd(R+2N) <= 96, 128 or 192 outputs; weight rows past nd(R+2N) are zero-filled), 32-channel
+// K-steps in a 5-, 4- or 3-stage cp.async pipeline.  Besides u, the task writes the scan-ready copies: B | C
+// of each token into its chunk-interleaved row, dt_low into a dense [T][R] block.
+template <int TN, int kQStages>
+__device__ __forceinline__ void fused_proj_t(const Shape& sh, const FusedPlan& pl, const FusedPtrs& p, int b, int q,
+                                             float* smem) {
+    const int T = sh.T, E = sh.E, J = sh.J, NJ = sh.NJ, R = sh.R, N = sh.N;
+    constexpr int WROWS = 32 * TN;
+    constexpr int TM = kQT / 8;
     const int tq0 = q * kQT;
     const int mt = min(kQT, T - tq0);
     const size_t m0 = (size_t)b * T + tq0;
-    float* xs = smem;                          // [2][kQT][kQPad]
-    float* ws = xs + 2 * kQT * kQPad;          // [2][NJ][kQPad]
+    float* xs = smem;                                // [kQStages][kQT][kQPad]
+    float* ws = xs + kQStages * kQT * kQPad;         // [kQStages][WROWS][kQPad]
     const int tg = threadIdx.x & 7, cg = threadIdx.x >> 3;   // tokens tg + 8 i, outputs cg + 32 j
-    constexpr int TM = kQT / 8;
     const int nk = (E + kQK - 1) / kQK;
-    auto load = [&](int kk, int buf) {
+    auto load = [&](int kk) {
         const int e0 = kk * kQK;
-        float* xb = xs + buf * kQT * kQPad;
-        float* wb = ws + buf * NJ * kQPad;
+        const int st = kk % kQStages;
+        float* xb = xs + st * kQT * kQPad;
+        float* wb = ws + st * WROWS * kQPad;
         for (int v = threadIdx.x; v < kQT * (kQK / 4); v += kFusedThreads) {
             const int r = v >> 3, c4 = (v & 7) * 4;
             const bool ok = r < mt && e0 + c4 < E;
             cp_async16(xb + r * kQPad + c4, ok ? (const void*)(p.xbar + (m0 + r) * E + e0 + c4) : (const void*)p.xbar,
                        ok ? 16u : 0u);
         }
-        for (int v = threadIdx.x; v < NJ * (kQK / 4); v += kFusedThreads) {
+        for (int v = threadIdx.x; v < WROWS * (kQK / 4); v += kFusedThreads) {
             const int r = v >> 3, c4 = (v & 7) * 4;
-            const bool ok = e0 + c4 < E;
+            const bool ok = r < NJ && e0 + c4 < E;
             cp_async16(wb + r * kQPad + c4, ok ? (const void*)(p.W_x + (size_t)r * E + e0 + c4) : (const void*)p.W_x,
                        ok ? 16u : 0u);
         }
-        cp_async_commit();
     };
     float acc[TM][TN];
 #pragma unroll
     for (int i = 0; i < TM; ++i)
 #pragma unroll
         for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
-    load(0, 0);
+#pragma unroll
+    for (int kk = 0; kk < kQStages - 1; ++kk) {
+        if (kk < nk) load(kk);
+        cp_async_commit();
+    }
     for (int kk = 0; kk < nk; ++kk) {
-        const int buf = kk & 1;
-        if (kk + 1 < nk) {
-            load(kk + 1, buf ^ 1);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncthreads();
-        const float* xb = xs + buf * kQT * kQPad;
-        const float* wb = ws + buf * NJ * kQPad;
-#pragma unroll 8
-        for (int c = 0; c < kQK; ++c) {
-            float xv[TM], wv[TN];
+        cp_async_wait<kQStages - 2>();
+        __syncthreads();  // K-step kk has landed for every thread; step kk-1's buffer is free
+        if (kk + kQStages - 1 < nk) load(kk + kQStages - 1);
+        cp_async_commit();
+        const int st = kk % kQStages;
+        const float* xb = xs + st * kQT * kQPad;
+        const float* wb = ws + st * WROWS * kQPad;
+#pragma unroll 2
+        for (int c = 0; c < kQK; c += 4) {
+            float4 xv[TM], wv[TN];
 #pragma unroll
-            for (int i = 0; i < TM; ++i) xv[i] = xb[(tg + 8 * i) * kQPad + c];
+            for (int i = 0; i < TM; ++i) xv[i] = *reinterpret_cast<const float4*>(xb + (tg + 8 * i) * kQPad + c);
 #pragma unroll
-            for (int j = 0; j < TN; ++j) {
-                const int jj = cg + 32 * j;
-                wv[j] = jj < NJ ? wb[jj * kQPad + c] : 0.f;
-            }
+            for (int j = 0; j < TN; ++j) wv[j] = *reinterpret_cast<const float4*>(wb + (cg + 32 * j) * kQPad + c);
 #pragma unroll
             for (int i = 0; i < TM; ++i)
 #pragma unroll
-                for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(wv[j], xv[i], acc[i][j]);
+                for (int j = 0; j < TN; ++j)
+                    acc[i][j] = fmaf(wv[j].w, xv[i].w,
+                                     fmaf(wv[j].z, xv[i].z, fmaf(wv[j].y, xv[i].y, fmaf(wv[j].x, xv[i].x, acc[i][j]))));
         }
-        __syncthreads();  // the buffer is refilled two steps later
     }
+    cp_async_wait<0>();
+    const int CL = pl.CL;
+    const size_t bstride = fused_bcs_stride(T), dstride = fused_dts_stride(T, R);
 #pragma unroll
     for (int j = 0; j < TN; ++j) {
         const int jj = cg + 32 * j;
         if (jj < NJ) {
             const int k = jj / J, jc = jj - k * J;
+            float* bcb = p.bcs + ((size_t)k * sh.B + b) * bstride;
+            float* dtb = p.dts + ((size_t)k * sh.B + b) * dstride;
 #pragma unroll
             for (int i = 0; i < TM; ++i) {
                 const int r = tg + 8 * i;
-                if (r < mt) p.u[u_offset(sh, k, b, tq0 + r) + jc] = acc[i][j];
+                if (r < mt) {
+                    const int t = tq0 + r;
+                    const float v = acc[i][j];
+                    p.u[u_offset(sh, k, b, t) + jc] = v;
+                    if (jc < R) {
+                        dtb[(size_t)t * R + jc] = v;
+                    } else {
+                        const int nb = jc - R;
+                        float* row = bcb + (size_t)((t % CL) * kScanChunks + t / CL) * kBCStride;
+                        row[nb < N ? nb : kScanStates + (nb - N)] = v;
+                        if (nb == 0)  // unused state slots of this token read as zero
+                            for (int n = N; n < kScanStates; ++n) {
+                                row[n] = 0.f;
+                                row[kScanStates + n] = 0.f;
+                            }
+                    }
+                }
             }
         }
     }
-    cta_signal(p.ctrl + kCtrlHeaderWords + sh.B + b);
+    cta_signal(p.ctrl ? p.ctrl + kCtrlHeaderWords + sh.B + b : nullptr);
 }
 
-__device__ __forceinline__ void fused_proj(const Shape& sh, const FusedPtrs& p, int b, int q, float* smem) {
-    if (sh.NJ <= 96) fused_proj_t<3>(sh, p, b, q, smem);
-    else fused_proj_t<6>(sh, p, b, q, smem);
+__device__ __forceinline__ void fused_proj(const Shape& sh, const FusedPlan& pl, const FusedPtrs& p, int b, int q,
+                                           float* smem) {
+    switch (q_tn(sh.NJ)) {
+        case 3: fused_proj_t<3, q_stages(3)>(sh, pl, p, b, q, smem); break;
+        case 4: fused_proj_t<4, q_stages(4)>(sh, pl, p, b, q, smem); break;
+        default: fused_proj_t<6, q_stages(6)>(sh, pl, p, b, q, smem); break;
+    }
 }
 
 // ---- S: dt_proj + softplus, ZOH and scans of channels [e0, e0 + ECH) of image b -----------------
@@ -462,71 +510,65 @@ __device__ __forceinline__ void fused_scan(const Shape& sh, const FusedPlan& pl,
     constexpr int ECH = kFusedThreads / (kScanChunks * ND);
     constexpr int XS = ECH + 4;
     constexpr int NS = kScanStates;
-    const int T = sh.T, E = sh.E, N = sh.N, J = sh.J, R = sh.R;
+    const int T = sh.T, E = sh.E, N = sh.N, R = sh.R;
     const int CL = pl.CL;
     const int rows = kScanChunks * CL;
     const int e0 = tile * ECH;
     float* bc = smem;                          // [ND][rows][kBCStride]: B_0..B_15 | C_0..C_15
     float* dx = bc + ND * rows * kBCStride;    // [ND][rows][XS]: Delta, then y of that direction
     float* xsm = dx + ND * rows * XS;          // [rows][XS]: pooled tokens
-    float* dtl = xsm + rows * XS;              // [ND][T][R]: dt_low
-    float* wdt = dtl + ND * T * R;             // [ND][ECH][R+1]: dt_proj rows (+ bias)
+    const int DTS = (int)fused_dts_stride(T, R);
+    float* dtl = xsm + rows * XS;              // [ND][DTS]: dt_low rows [T][R]
+    float* wdt = dtl + ND * DTS;               // [ND][ECH][R+1]: dt_proj rows (+ bias)
     int* post = reinterpret_cast<int*>(wdt + ND * ECH * (R + 1));  // [T]: p(t)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     constexpr int kWarps = kFusedThreads / 32;
-    for (int t = threadIdx.x; t < T; t += kFusedThreads) post[t] = (t % CL) * kScanChunks + t / CL;
-    if (N < NS)
-        for (int i = threadIdx.x; i < ND * rows * kBCStride; i += kFusedThreads) bc[i] = 0.f;
-    __syncthreads();
-    // Stage this tile's inputs with asynchronous copies (all in flight together): dt_low and
-    // B | C of every token (B | C straight into the chunk-interleaved rows), the pooled tokens of
-    // the tile's channels, and the tile's dt_proj rows and biases.
-    for (int k = 0; k < ND; ++k) {
-        const float* src = p.u + u_offset(sh, k, b, 0);
-        for (int t = warp; t < T; t += kWarps) {
-            const int pos = post[t];
-            for (int j = lane; j < J; j += 32) {
-                float* dst;
-                if (j < R) {
-                    dst = dtl + (k * T + t) * R + j;
-                } else {
-                    const int jb = j - R;
-                    dst = bc + (k * rows + pos) * kBCStride + (jb < N ? jb : NS + (jb - N));
-                }
-                cp_async4(dst, src + (size_t)t * J + j);
-            }
+    // Stage the tile's inputs with 16-byte asynchronous copies (all in flight together): the
+    // scan-ready B | C rows and dt_low rows written by the projection tasks, the pooled tokens of
+    // the tile's channels; and the tile's dt_proj rows and biases.
+    {
+        const int nbc = rows * kBCStride / 4, ndt = DTS / 4;
+        for (int k = 0; k < ND; ++k) {
+            const float* sb = p.bcs + ((size_t)k * sh.B + b) * fused_bcs_stride(T);
+            const float* sd = p.dts + ((size_t)k * sh.B + b) * DTS;
+            for (int v = threadIdx.x; v < nbc; v += kFusedThreads) cp_async16(bc + k * rows * kBCStride + 4 * v, sb + 4 * v, 16u);
+            for (int v = threadIdx.x; v < ndt; v += kFusedThreads) cp_async16(dtl + k * DTS + 4 * v, sd + 4 * v, 16u);
         }
+        for (int t = threadIdx.x; t < T; t += kFusedThreads) post[t] = (t % CL) * kScanChunks + t / CL;
+        __syncthreads();
+        for (int v = threadIdx.x; v < T * (ECH / 4); v += kFusedThreads) {
+            const int t = v / (ECH / 4), c4 = (v % (ECH / 4)) * 4;
+            const bool ok = e0 + c4 < E;
+            cp_async16(xsm + post[t] * XS + c4, ok ? (const void*)(p.xbar + ((size_t)b * T + t) * E + e0 + c4)
+                                                   : (const void*)p.xbar, ok ? 16u : 0u);
+        }
+        cp_async_commit();
+        for (int i = threadIdx.x; i < ND * ECH * (R + 1); i += kFusedThreads) {
+            const int k = i / (ECH * (R + 1));
+            const int rem = i - k * ECH * (R + 1);
+            const int c = rem / (R + 1), r = rem - c * (R + 1);
+            const int e = e0 + c;
+            float v = 0.f;
+            if (e < E) v = r < R ? __ldg(p.W_dt + ((size_t)k * E + e) * R + r) : __ldg(p.b_dt + (size_t)k * E + e);
+            wdt[i] = v;
+        }
+        cp_async_wait<0>();
+        __syncthreads();
     }
-    for (int v = threadIdx.x; v < T * (ECH / 4); v += kFusedThreads) {
-        const int t = v / (ECH / 4), c4 = (v % (ECH / 4)) * 4;
-        const bool ok = e0 + c4 < E;
-        cp_async16(xsm + post[t] * XS + c4, ok ? (const void*)(p.xbar + ((size_t)b * T + t) * E + e0 + c4)
-                                               : (const void*)p.xbar, ok ? 16u : 0u);
-    }
-    cp_async_commit();
-    for (int i = threadIdx.x; i < ND * ECH * (R + 1); i += kFusedThreads) {
-        const int k = i / (ECH * (R + 1));
-        const int rem = i - k * ECH * (R + 1);
-        const int c = rem / (R + 1), r = rem - c * (R + 1);
-        const int e = e0 + c;
-        float v = 0.f;
-        if (e < E) v = r < R ? __ldg(p.W_dt + ((size_t)k * E + e) * R + r) : __ldg(p.b_dt + (size_t)k * E + e);
-        wdt[i] = v;
-    }
-    cp_async_wait<0>();
-    __syncthreads();
-    // Delta = softplus(W_dt . dt_low + b_dt) for this tile: lane -> channel, warps -> (direction, token)
+    // Delta = softplus(W_dt . dt_low + b_dt) for this tile: lane -> channel, warps -> tokens
     {
         constexpr int kTPerWarpPass = 32 / ECH > 0 ? 32 / ECH : 1;
         const int c = lane % ECH;
         const int tsub = lane / ECH;
+        const bool live = e0 + c < E;
         for (int k = 0; k < ND; ++k) {
             const float* wr = wdt + (k * ECH + c) * (R + 1);
             for (int t = warp * kTPerWarpPass + tsub; t < T; t += kWarps * kTPerWarpPass) {
-                const float* dl = dtl + (k * T + t) * R;
+                const float* dl = dtl + k * DTS + t * R;
                 float a = wr[R];
+#pragma unroll 4
                 for (int r = 0; r < R; ++r) a = fmaf(wr[r], dl[r], a);
-                dx[(k * rows + post[t]) * XS + c] = (e0 + c < E) ? softplus_f(a) : 0.f;
+                dx[(k * rows + post[t]) * XS + c] = live ? softplus_f(a) : 0.f;
             }
         }
     }
@@ -579,28 +621,40 @@ __device__ __forceinline__ void fused_scan(const Shape& sh, const FusedPlan& pl,
             }
         }
     }
-    // compose the chunk maps h -> P h + H along the scan order (lanes 0..7 forward, 7..0 backward)
+    // compose the chunk maps h -> P h + H along the scan order (lanes 0..7 forward, 7..0 backward;
+    // the direction is uniform within a warp)
+    if (fwd) {
 #pragma unroll
-    for (int n = 0; n < NS; ++n) {
-        float P = ex2_approx(A2[n] * sdt);
-        float H = h[n];
+        for (int n = 0; n < NS; ++n) {
+            float P = ex2_approx(A2[n] * sdt), H = h[n];
 #pragma unroll
-        for (int d = 1; d < kScanChunks; d <<= 1) {
-            const float Pp = fwd ? __shfl_up_sync(0xffffffffu, P, d, kScanChunks)
-                                 : __shfl_down_sync(0xffffffffu, P, d, kScanChunks);
-            const float Hp = fwd ? __shfl_up_sync(0xffffffffu, H, d, kScanChunks)
-                                 : __shfl_down_sync(0xffffffffu, H, d, kScanChunks);
-            const bool has = fwd ? (chunk >= d) : (chunk + d < kScanChunks);
-            if (has) {
-                H = fmaf(P, Hp, H);
-                P = P * Pp;
+            for (int d = 1; d < kScanChunks; d <<= 1) {
+                const float Pp = __shfl_up_sync(0xffffffffu, P, d, kScanChunks);
+                const float Hp = __shfl_up_sync(0xffffffffu, H, d, kScanChunks);
+                if (chunk >= d) {
+                    H = fmaf(P, Hp, H);
+                    P = P * Pp;
+                }
             }
+            const float Hin = __shfl_up_sync(0xffffffffu, H, 1, kScanChunks);
+            h[n] = chunk == 0 ? 0.f : Hin;
         }
-        // incoming state = inclusive result of the previous chunk in scan order
-        const float Hin = fwd ? __shfl_up_sync(0xffffffffu, H, 1, kScanChunks)
-                              : __shfl_down_sync(0xffffffffu, H, 1, kScanChunks);
-        const bool first = fwd ? (chunk == 0) : (chunk == kScanChunks - 1);
-        h[n] = first ? 0.f : Hin;
+    } else {
+#pragma unroll
+        for (int n = 0; n < NS; ++n) {
+            float P = ex2_approx(A2[n] * sdt), H = h[n];
+#pragma unroll
+            for (int d = 1; d < kScanChunks; d <<= 1) {
+                const float Pp = __shfl_down_sync(0xffffffffu, P, d, kScanChunks);
+                const float Hp = __shfl_down_sync(0xffffffffu, H, d, kScanChunks);
+                if (chunk + d < kScanChunks) {
+                    H = fmaf(P, Hp, H);
+                    P = P * Pp;
+                }
+            }
+            const float Hin = __shfl_down_sync(0xffffffffu, H, 1, kScanChunks);
+            h[n] = chunk == kScanChunks - 1 ? 0.f : Hin;
+        }
     }
     // pass 2: rerun the chunk from its incoming state and emit C_t . h_t
     for (int s = 0; s < len; ++s) {
@@ -638,7 +692,7 @@ __device__ __forceinline__ void fused_scan(const Shape& sh, const FusedPlan& pl,
             if (ee < E) p.ys[((size_t)b * T + t) * E + ee] = sum;
         }
     }
-    cta_signal(p.ctrl + kCtrlHeaderWords + 2 * sh.B + b);
+    cta_signal(p.ctrl ? p.ctrl + kCtrlHeaderWords + 2 * sh.B + b : nullptr);
 }
 
 // ---- E: repeat + skip + gate for grid lines [t0, t0+LP) of image b -------------------------------
@@ -718,7 +772,7 @@ fused_layer_kernel(Shape sh, FusedPlan pl, FusedPtrs p) {
     __shared__ int s_flag;
     __shared__ unsigned s_ticket;
     __shared__ unsigned long long s_t0, s_t1;
-    const uint64_t pol_keep = l2_policy_evict_last();
+    const uint64_t pol_keep = l2_policy_evict_first();  // x is re-read by the gate tasks from HBM
     const uint64_t pol_stream = l2_policy_evict_first();
     unsigned* abort_flag = p.ctrl + 1;
     unsigned* cnt_pool = p.ctrl + kCtrlHeaderWords;
@@ -753,7 +807,7 @@ fused_layer_kernel(Shape sh, FusedPlan pl, FusedPtrs p) {
         } else if (kind == kTaskProj) {
             if (!cta_wait(cnt_pool + b, (unsigned)pl.nP, p.status, abort_flag, pl.wait_limit_ns, &s_flag)) return;
             if (p.trace && threadIdx.x == 0) s_t1 = globaltimer_ns();
-            fused_proj(sh, p, b, idx, smem_f);
+            fused_proj(sh, pl, p, b, idx, smem_f);
         } else if (kind == kTaskScan) {
             if (!cta_wait(cnt_proj + b, (unsigned)pl.nQ, p.status, abort_flag, pl.wait_limit_ns, &s_flag)) return;
             if (p.trace && threadIdx.x == 0) s_t1 = globaltimer_ns();
@@ -776,6 +830,18 @@ fused_layer_kernel(Shape sh, FusedPlan pl, FusedPtrs p) {
             }
         }
     }
+}
+
+// Staged launches of the same task bodies: one CTA per projection task / per scan task, ordered by
+// the launch boundaries instead of counters.
+__global__ void __launch_bounds__(kFusedThreads, 2) proj_tasks_kernel(Shape sh, FusedPlan pl, FusedPtrs p) {
+    extern __shared__ __align__(128) float smem_f[];
+    fused_proj(sh, pl, p, blockIdx.x / pl.nQ, blockIdx.x % pl.nQ, smem_f);
+}
+template <int ND, bool ZOH_EXACT>
+__global__ void __launch_bounds__(kFusedThreads, 2) scan_tasks_kernel(Shape sh, FusedPlan pl, FusedPtrs p) {
+    extern __shared__ __align__(128) float smem_f[];
+    fused_scan<ND, ZOH_EXACT>(sh, pl, p, blockIdx.x / pl.nS, blockIdx.x % pl.nS, smem_f);
 }
 
 // A single CTA that waits, with the layer's bounded wait, on a counter that nothing increments:

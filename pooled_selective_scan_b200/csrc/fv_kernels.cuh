@@ -2,13 +2,10 @@
 //
 // Step map (FastVim, arXiv 2502.00594; gptget.net summary of the paper, section "方法详解"):
 //   pool_dense_kernel / mask_bucket_kernel + mask_pool_kernel   item 2 (and item 6, masked)
-//   proj_kernel                                                 item 3 (x_proj)
-//   scan_kernel                                                 items 3-4 (dt_proj + softplus,
-//                                                               ZOH, forward/backward scans)
+//   (x_proj, dt_proj + softplus, ZOH and the scans run as task grids of fv_fused.cuh's bodies:
+//    proj_tasks_kernel and scan_tasks_kernel, items 3-4)
 //   epilogue_dense_kernel / mask_epilogue_kernel                item 5 (repeat, skip, gate)
-// The work is HBM-streaming except the projection and the scan, which are small; none of it
-// is a dense contraction large enough for tensor cores (the x_proj GEMM has N = nd(R+2N) <= 192
-// columns and K = E, and must stay fp32 to meet the layer's tolerance).
+// The work here is HBM streaming.
 #pragma once
 
 #include "fv_common.cuh"
@@ -187,174 +184,6 @@ mask_pool_kernel(Shape sh, const float* __restrict__ x, const int32_t* __restric
             f4_add(a0, a1);
             out[slot] = f4_scale(a0, scale);
         }
-    }
-}
-
-// ------------------------------------------------------------------------------------------
-// x_proj: u[k][m][0:J] = W_x[k] . xbar[m] for the pooled tokens m = b*T + t (fp32 FFMA).
-// One CTA per 32 pooled tokens, all nd*J outputs; channels staged 32 at a time in shared memory.
-// ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads)
-proj_kernel(Shape sh, const float* __restrict__ xbar, const float* __restrict__ W_x, float* __restrict__ u) {
-    extern __shared__ float smem_f[];
-    float* xs = smem_f;                        // [32][33]
-    float* wsm = smem_f + kProjRows * 33;      // [NJ][33]
-    const int M = sh.B * sh.T, E = sh.E, NJ = sh.NJ, J = sh.J;
-    const int m0 = blockIdx.x * kProjRows;
-    const int ml = threadIdx.x & 31, jg = threadIdx.x >> 5;
-    float acc[kProjQ];
-#pragma unroll
-    for (int q = 0; q < kProjQ; ++q) acc[q] = 0.f;
-    for (int e0 = 0; e0 < E; e0 += kProjChunk) {
-        for (int i = threadIdx.x; i < kProjRows * kProjChunk; i += kThreads) {
-            const int r = i >> 5, c = i & 31;
-            const int m = m0 + r, e = e0 + c;
-            xs[r * 33 + c] = (m < M && e < E) ? xbar[(size_t)m * E + e] : 0.f;
-        }
-        for (int i = threadIdx.x; i < NJ * kProjChunk; i += kThreads) {
-            const int jj = i >> 5, c = i & 31;
-            const int e = e0 + c;
-            wsm[jj * 33 + c] = (e < E) ? W_x[(size_t)jj * E + e] : 0.f;
-        }
-        __syncthreads();
-#pragma unroll 4
-        for (int c = 0; c < kProjChunk; ++c) {
-            const float xv = xs[ml * 33 + c];
-#pragma unroll
-            for (int q = 0; q < kProjQ; ++q) {
-                const int jj = jg + 8 * q;
-                if (jj < NJ) acc[q] = fmaf(wsm[jj * 33 + c], xv, acc[q]);
-            }
-        }
-        __syncthreads();
-    }
-    const int m = m0 + ml;
-    if (m < M) {
-        const int bm = m / sh.T, tm = m - bm * sh.T;
-#pragma unroll
-        for (int q = 0; q < kProjQ; ++q) {
-            const int jj = jg + 8 * q;
-            if (jj < NJ) {
-                const int k = jj / J, j = jj - k * J;
-                u[u_offset(sh, k, bm, tm) + j] = acc[q];
-            }
-        }
-    }
-}
-
-// ------------------------------------------------------------------------------------------
-// dt_proj + softplus, ZOH and the forward/backward selective scans in one launch.
-// One CTA per (image b, tile of ECH channels).  Thread = (state group g, direction kd, channel c):
-// G lanes of 4 states each cover the N <= 16 states of one (kd, c), so the state lives in
-// registers and is never written; the G partial C.h sums meet through __shfl_xor, and the two
-// directions meet in a shared-memory accumulator (two fp32 adds onto zero commute exactly, so
-// the sum does not depend on their order).
-// ------------------------------------------------------------------------------------------
-template <int G, int ND>
-__host__ __device__ constexpr int scan_ech() { return kThreads / (G * ND); }
-
-__host__ __forceinline__ size_t scan_smem_floats(int T, int J, int R, int G, int ND) {
-    const int ech = kThreads / (G * ND);
-    return (size_t)ND * T * J + (size_t)T * ech + (size_t)ND * T * ech + (size_t)ND * ech * R +
-           (size_t)T * ech;
-}
-
-template <int G, int ND, bool ZOH_EXACT>
-__global__ void __launch_bounds__(kThreads)
-scan_kernel(Shape sh, const float* __restrict__ xbar, const float* __restrict__ u,
-            const float* __restrict__ A_log, const float* __restrict__ W_dt,
-            const float* __restrict__ b_dt, float* __restrict__ ys) {
-    constexpr int ECH = scan_ech<G, ND>();
-    extern __shared__ float smem_f[];
-    const int T = sh.T, J = sh.J, R = sh.R, N = sh.N, E = sh.E;
-    const int ntile = (E + ECH - 1) / ECH;
-    const int b = blockIdx.x / ntile;
-    const int e0 = (blockIdx.x - b * ntile) * ECH;
-    float* us = smem_f;                  // [ND][T][J]   projections of this image
-    float* xs = us + ND * T * J;         // [T][ECH]     pooled tokens, this channel tile
-    float* dts = xs + T * ECH;           // [ND][T][ECH] Delta
-    float* wdt = dts + ND * T * ECH;     // [ND][ECH][R] dt_proj rows of this tile
-    float* ysum = wdt + ND * ECH * R;    // [T][ECH]     output, summed over directions
-
-    for (int k = 0; k < ND; ++k) {
-        const float* src = u + u_offset(sh, k, b, 0);
-        for (int i = threadIdx.x; i < T * J; i += kThreads) us[k * T * J + i] = src[i];
-    }
-    for (int i = threadIdx.x; i < T * ECH; i += kThreads) {
-        const int t = i / ECH, c = i - t * ECH;
-        const int e = e0 + c;
-        xs[i] = (e < E) ? xbar[((size_t)b * T + t) * E + e] : 0.f;
-        ysum[i] = 0.f;
-    }
-    for (int i = threadIdx.x; i < ND * ECH * R; i += kThreads) {
-        const int k = i / (ECH * R);
-        const int rem = i - k * ECH * R;
-        const int c = rem / R, r = rem - c * R;
-        const int e = e0 + c;
-        wdt[i] = (e < E) ? W_dt[((size_t)k * E + e) * R + r] : 0.f;
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < ND * T * ECH; i += kThreads) {
-        const int k = i / (T * ECH);
-        const int rem = i - k * T * ECH;
-        const int t = rem / ECH, c = rem - t * ECH;
-        const int e = e0 + c;
-        float acc = (e < E) ? b_dt[(size_t)k * E + e] : 0.f;
-        const float* ur = us + (k * T + t) * J;
-        const float* wr = wdt + (k * ECH + c) * R;
-        for (int r = 0; r < R; ++r) acc = fmaf(wr[r], ur[r], acc);
-        dts[i] = softplus_f(acc);
-    }
-    __syncthreads();
-
-    const int g = threadIdx.x % G;
-    const int kd = (threadIdx.x / G) % ND;
-    const int c = threadIdx.x / (G * ND);
-    const int e = e0 + c;
-    const bool active = e < E;
-    const bool fwd = (ND == 2) ? (kd == 0) : ((sh.dir_flags & 1u) != 0);
-    constexpr float kLog2e = 1.4426950408889634f;
-    float An[4], A2[4], Ainv[4], hs[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int n = 4 * g + i;
-        const float A = (active && n < N) ? -expf(A_log[((size_t)kd * E + e) * N + n]) : -1.f;
-        An[i] = A;
-        A2[i] = A * kLog2e;
-        Ainv[i] = 1.f / A;
-        hs[i] = 0.f;
-    }
-    const float* ub = us + kd * T * J;
-    const float* dcol = dts + kd * T * ECH + c;
-    for (int step = 0; step < T; ++step) {
-        const int t = fwd ? step : T - 1 - step;
-        const float dt = dcol[t * ECH];
-        const float xv = xs[t * ECH + c];
-        const float dtx = dt * xv;
-        const float* Brow = ub + t * J + R;
-        const float* Crow = Brow + N;
-        float yp = 0.f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int n = 4 * g + i;
-            if (n < N) {
-                const float dA = exp2f(dt * A2[i]);
-                float bx;
-                if (ZOH_EXACT) bx = expm1f(dt * An[i]) * Ainv[i] * Brow[n] * xv;
-                else bx = dtx * Brow[n];
-                hs[i] = fmaf(dA, hs[i], bx);
-                yp = fmaf(Crow[n], hs[i], yp);
-            }
-        }
-        if (G >= 2) yp += __shfl_xor_sync(0xffffffffu, yp, 1);
-        if (G >= 4) yp += __shfl_xor_sync(0xffffffffu, yp, 2);
-        if (g == 0 && active) atomicAdd(&ysum[t * ECH + c], yp);
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < T * ECH; i += kThreads) {
-        const int t = i / ECH, cc = i - t * ECH;
-        const int ee = e0 + cc;
-        if (ee < E) ys[((size_t)b * T + t) * E + ee] = ysum[i];
     }
 }
 

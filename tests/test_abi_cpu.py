@@ -170,7 +170,7 @@ def test_workspace_layout(lib, pool_axis, K):
 
 
 @pytest.mark.parametrize("flags,want", [(0, ["fused_layer_kernel"]), (4, ["fused_layer_kernel"]),
-                                        (2, ["pool_dense_kernel", "proj_kernel", "scan_kernel",
+                                        (2, ["pool_dense_kernel", "proj_tasks_kernel", "scan_tasks_kernel",
                                              "epilogue_dense_kernel"])])
 def test_path_selection_is_host_side(lib, flags, want):
     a = good_args(h=128, w=128, B=4, flags=flags)  # 2048 px FastVim-T images: fused by default
