@@ -116,7 +116,7 @@ typedef struct {
 /* Byte offsets of the intermediates inside a workspace (for inspection and tests). */
 typedef struct {
     size_t total_bytes;  /* what fastvim_ssm_workspace_size returns                          */
-    size_t status;       /* uint32 device status word                                        */
+    size_t status;       /* uint32 device status word (+ one uint32 of scratch)              */
     size_t xbar;         /* fp32 [B][T][E] pooled tokens                                     */
     size_t u;            /* fp32 projections dt_low | B | C: [nd][B] blocks of [T][R+2N], each
                             block starting every ceil(T (R+2N) / 32) * 32 floats            */
@@ -178,7 +178,11 @@ FV_API fv_status fastvim_ssm_forward_events(const fv_ssm_args* args, void* ws, s
 /* End-to-end variant for host-resident data.  `host` names pinned HOST buffers for x, z,
  * the parameters, keep_idx and y; `dev` names DEVICE buffers of the same shapes (its sizes
  * and flags must equal host's).  Copies the inputs host -> device, runs the layer, copies y
- * device -> host and waits for the stream, so y is ready in host memory on return. */
+ * device -> host and waits for the stream, so y is ready in host memory on return.  The batch
+ * runs as chunks of whole images (about 64 MB of x each, at most 16 chunks) in a pipeline: the
+ * upload of one chunk, the layer on the previous one (on `stream`) and the download of the one
+ * before overlap, on two streams the call creates and destroys.  The device status word of ws
+ * reports the first device error of any chunk. */
 FV_API fv_status fastvim_ssm_forward_host(const fv_ssm_args* host, const fv_ssm_args* dev, void* ws,
                                    size_t ws_bytes, void* stream);
 

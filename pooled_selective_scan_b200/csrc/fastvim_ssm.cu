@@ -8,6 +8,8 @@
 #include <stdlib.h>
 
 #include <mutex>
+#include <vector>
+#include <algorithm>
 
 #include "fv_common.cuh"
 #include "fv_fused.cuh"
@@ -94,7 +96,8 @@ fv::FusedPlan plan_fused(const fv::Shape& sh);
 fv_status plan_layout(const fv::Shape& sh, fv_ws_layout* L) {
     memset(L, 0, sizeof *L);
     size_t off = 0;
-    L->status = off; off = round256(off + sizeof(unsigned));
+    // word 0: the call's device status; word 1: scratch of fastvim_ssm_forward_host
+    L->status = off; off = round256(off + 2 * sizeof(unsigned));
     L->xbar = off; off = round256(off + (size_t)sh.B * sh.T * sh.E * sizeof(float));
     L->u = off; off = round256(off + (size_t)sh.nd * sh.B * fv::u_block_stride(sh.T, sh.J) * sizeof(float));
     L->ys = off; off = round256(off + (size_t)sh.B * sh.T * sh.E * sizeof(float));
@@ -481,6 +484,32 @@ fv_status fastvim_ssm_forward_events(const fv_ssm_args* args, void* ws, size_t w
     return forward_impl(args, ws, ws_bytes, (cudaStream_t)stream, events, n_events);
 }
 
+namespace {
+// x bytes per chunk of images in fastvim_ssm_forward_host, and the most chunks it makes.
+constexpr size_t kHostChunkBytes = (size_t)64 << 20;
+constexpr int kHostMaxChunks = 16;
+
+// Streams and events of one fastvim_ssm_forward_host call, released on every exit path.
+struct HostPipe {
+    cudaStream_t up = nullptr, down = nullptr;
+    std::vector<cudaEvent_t> ev;
+    ~HostPipe() {
+        if (up) cudaStreamSynchronize(up);
+        if (down) cudaStreamSynchronize(down);
+        for (cudaEvent_t e : ev)
+            if (e) cudaEventDestroy(e);
+        if (up) cudaStreamDestroy(up);
+        if (down) cudaStreamDestroy(down);
+    }
+    cudaEvent_t make() {
+        cudaEvent_t e = nullptr;
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) e = nullptr;
+        ev.push_back(e);
+        return e;
+    }
+};
+}  // namespace
+
 fv_status fastvim_ssm_forward_host(const fv_ssm_args* host, const fv_ssm_args* dev, void* ws,
                                    size_t ws_bytes, void* stream) {
     if (!host || !dev) return FV_ERR_NULL;
@@ -494,13 +523,44 @@ fv_status fastvim_ssm_forward_host(const fv_ssm_args* host, const fv_ssm_args* d
         return FV_ERR_SHAPE;
     if ((s = check_pointers(host, sh)) != FV_OK) return s;
     if ((s = check_pointers(dev, shd)) != FV_OK) return s;
+    {
+        fv_ws_layout L;
+        plan_layout(sh, &L);
+        if (!ws || ws_bytes < L.total_bytes || ((uintptr_t)ws & 255u) != 0) return FV_ERR_WORKSPACE;
+        if ((s = check_limits(sh)) != FV_OK) return s;
+    }
     cudaStream_t st = (cudaStream_t)stream;
     const size_t tok = sh.K > 0 ? (size_t)sh.K : (size_t)sh.h * sh.w;
-    const size_t act = (size_t)sh.B * tok * sh.E * sizeof(float);
+    const size_t img = tok * sh.E * sizeof(float);  // bytes of one image's x, z or y
     const size_t nd = (size_t)sh.nd;
-    struct Copy { void* dst; const void* src; size_t bytes; } copies[] = {
-        {(void*)dev->x, host->x, act},
-        {(void*)dev->z, host->z, act},
+
+    // The images are independent, so the batch runs as chunks of images in a three-stage
+    // pipeline: chunk c's x and z go up on one stream while chunk c-1 is computed on the caller's
+    // stream and chunk c-2's y comes down on a third (the two copy directions run concurrently).
+    int chunks = 1;
+    if (sh.B > 1) {
+        const size_t want = ((size_t)sh.B * img + kHostChunkBytes - 1) / kHostChunkBytes;
+        chunks = (int)std::min<size_t>(std::min<size_t>(want, (size_t)kHostMaxChunks), (size_t)sh.B);
+        if (chunks < 1) chunks = 1;
+    }
+    const int per = sh.B > 0 ? (sh.B + chunks - 1) / chunks : 0;
+    chunks = per > 0 ? (sh.B + per - 1) / per : 1;
+
+    HostPipe pp;
+    auto cuda_fail = [&](cudaError_t e, const char* where) { note_cuda(e, where); return FV_ERR_CUDA; };
+    cudaError_t e = cudaStreamCreateWithFlags(&pp.up, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&pp.down, cudaStreamNonBlocking);
+    if (e != cudaSuccess) return cuda_fail(e, "host pipeline streams");
+    cudaEvent_t start = pp.make(), down_done = pp.make();
+    std::vector<cudaEvent_t> up_done(chunks), computed(chunks);
+    for (int c = 0; c < chunks; ++c) { up_done[c] = pp.make(); computed[c] = pp.make(); }
+    for (cudaEvent_t v : pp.ev)
+        if (!v) return cuda_fail(cudaErrorMemoryAllocation, "host pipeline events");
+
+    // the copies start after the work the caller queued before this call
+    if ((e = cudaEventRecord(start, st)) != cudaSuccess) return cuda_fail(e, "event record");
+    if ((e = cudaStreamWaitEvent(pp.up, start, 0)) != cudaSuccess) return cuda_fail(e, "stream wait");
+    struct Copy { void* dst; const void* src; size_t bytes; } params[] = {
         {(void*)dev->A_log, host->A_log, nd * sh.E * sh.N * sizeof(float)},
         {(void*)dev->D, host->D, nd * sh.E * sizeof(float)},
         {(void*)dev->W_x, host->W_x, nd * sh.J * sh.E * sizeof(float)},
@@ -508,18 +568,47 @@ fv_status fastvim_ssm_forward_host(const fv_ssm_args* host, const fv_ssm_args* d
         {(void*)dev->b_dt, host->b_dt, nd * sh.E * sizeof(float)},
         {(void*)dev->keep_idx, host->keep_idx, sh.K > 0 ? (size_t)sh.B * sh.K * sizeof(int32_t) : 0},
     };
-    for (const Copy& c : copies) {
+    for (const Copy& c : params) {
         if (c.bytes == 0 || !c.dst) continue;
-        cudaError_t e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, st);
-        if (e != cudaSuccess) { note_cuda(e, "host->device copy"); return FV_ERR_CUDA; }
+        if ((e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, pp.up)) != cudaSuccess)
+            return cuda_fail(e, "host->device copy");
     }
-    if ((s = forward_impl(dev, ws, ws_bytes, st)) != FV_OK) return s;
-    if (act > 0) {
-        cudaError_t e = cudaMemcpyAsync(host->y, dev->y, act, cudaMemcpyDeviceToHost, st);
-        if (e != cudaSuccess) { note_cuda(e, "device->host copy"); return FV_ERR_CUDA; }
+    unsigned* status = (unsigned*)ws;  // word 0 of the layout; word 1 keeps the first error
+    if (chunks > 1 && (e = cudaMemsetAsync(status + 1, 0, sizeof(unsigned), st)) != cudaSuccess)
+        return cuda_fail(e, "status reset");
+    for (int c = 0; c < chunks; ++c) {
+        const int b0 = c * per, nb = std::max(0, std::min(per, sh.B - b0));
+        const size_t off = (size_t)b0 * tok * sh.E;  // float offset of the chunk's first image
+        const size_t bytes = (size_t)nb * img;
+        if (bytes > 0) {
+            if ((e = cudaMemcpyAsync((void*)(dev->x + off), host->x + off, bytes, cudaMemcpyHostToDevice, pp.up)) != cudaSuccess ||
+                (e = cudaMemcpyAsync((void*)(dev->z + off), host->z + off, bytes, cudaMemcpyHostToDevice, pp.up)) != cudaSuccess)
+                return cuda_fail(e, "host->device copy");
+        }
+        if ((e = cudaEventRecord(up_done[c], pp.up)) != cudaSuccess) return cuda_fail(e, "event record");
+        if ((e = cudaStreamWaitEvent(st, up_done[c], 0)) != cudaSuccess) return cuda_fail(e, "stream wait");
+        fv_ssm_args a = *dev;
+        a.B = nb;
+        if (bytes > 0) { a.x = dev->x + off; a.z = dev->z + off; a.y = dev->y + off; }
+        if (sh.K > 0 && nb > 0) a.keep_idx = dev->keep_idx + (size_t)b0 * sh.K;
+        if ((s = forward_impl(&a, ws, ws_bytes, st)) != FV_OK) return s;
+        if (chunks > 1) {
+            fv::status_fold_kernel<<<1, 32, 0, st>>>(status + 1, status);
+            FV_LAUNCH_CHECK("status_fold_kernel");
+        }
+        if ((e = cudaEventRecord(computed[c], st)) != cudaSuccess) return cuda_fail(e, "event record");
+        if ((e = cudaStreamWaitEvent(pp.down, computed[c], 0)) != cudaSuccess) return cuda_fail(e, "stream wait");
+        if (bytes > 0 &&
+            (e = cudaMemcpyAsync(host->y + off, dev->y + off, bytes, cudaMemcpyDeviceToHost, pp.down)) != cudaSuccess)
+            return cuda_fail(e, "device->host copy");
     }
-    cudaError_t e = cudaStreamSynchronize(st);
-    if (e != cudaSuccess) { note_cuda(e, "stream synchronize"); return FV_ERR_CUDA; }
+    if (chunks > 1) {  // the call's status word reports the first error of any chunk
+        fv::status_fold_kernel<<<1, 32, 0, st>>>(status, status + 1);
+        FV_LAUNCH_CHECK("status_fold_kernel");
+    }
+    if ((e = cudaEventRecord(down_done, pp.down)) != cudaSuccess) return cuda_fail(e, "event record");
+    if ((e = cudaStreamWaitEvent(st, down_done, 0)) != cudaSuccess) return cuda_fail(e, "stream wait");
+    if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "stream synchronize");
     return FV_OK;
 }
 

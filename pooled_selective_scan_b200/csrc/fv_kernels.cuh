@@ -37,6 +37,11 @@ __device__ __forceinline__ float4 f4_scale(float4 v, float s) {
     return make_float4(v.x * s, v.y * s, v.z * s, v.w * s);
 }
 
+// Keeps the first device error of a sequence of calls: *dst = *dst ? *dst : *src.
+__global__ void status_fold_kernel(unsigned* dst, const unsigned* src) {
+    if (threadIdx.x == 0 && *dst == 0u) *dst = *src;
+}
+
 // One CTA per pooled token (b, t): mean of the S grid tokens of line t, 128-bit loads, no copy
 // or transpose of the grid (the pooled axis only changes the base/stride of the index map).
 __global__ void __launch_bounds__(kThreads)

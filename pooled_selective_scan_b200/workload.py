@@ -18,8 +18,18 @@ def params_tensors(cfg: LayerConfig, device) -> dict:
     return {k: torch.from_numpy(v).to(device) for k, v in p.items()}
 
 
-def activations(cfg: LayerConfig, device, pinned_host: bool = False) -> dict:
-    """x, z (and keep_idx) for every image of ``cfg`` on ``device`` (or in pinned host memory)."""
+def shard_images(cfg: LayerConfig, rank: int, world: int) -> range:
+    """Global image ids that rank ``rank`` of ``world`` processes: every rank holds its own batch of
+    ``cfg.B`` distinct images (the global batch is world * B; images are independent, so ranks
+    exchange nothing)."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError(f"rank {rank} of world {world}")
+    return range(rank * cfg.B, (rank + 1) * cfg.B)
+
+
+def activations(cfg: LayerConfig, device, pinned_host: bool = False, first_image: int = 0) -> dict:
+    """x, z (and keep_idx) for images first_image .. first_image + B - 1 of ``cfg``'s seeded
+    stream on ``device`` (or in pinned host memory)."""
     shp = inputs.token_shape(cfg)
     kw = dict(dtype=torch.float32)
     if pinned_host:
@@ -28,20 +38,21 @@ def activations(cfg: LayerConfig, device, pinned_host: bool = False) -> dict:
     else:
         x = torch.empty((cfg.B,) + shp, device=device, **kw)
         z = torch.empty((cfg.B,) + shp, device=device, **kw)
-    for b in range(cfg.B):
-        x[b].copy_(torch.from_numpy(inputs.image_x(cfg.seed, b, shp)), non_blocking=False)
-        z[b].copy_(torch.from_numpy(inputs.image_z(cfg.seed, b, shp)), non_blocking=False)
+    for i in range(cfg.B):
+        b = first_image + i
+        x[i].copy_(torch.from_numpy(inputs.image_x(cfg.seed, b, shp)), non_blocking=False)
+        z[i].copy_(torch.from_numpy(inputs.image_z(cfg.seed, b, shp)), non_blocking=False)
     out = dict(x=x, z=z)
     if cfg.masked:
-        idx = np.stack([inputs.image_keep_idx(cfg.seed, b, cfg.h, cfg.w, cfg.K) for b in range(cfg.B)])
+        idx = np.stack([inputs.image_keep_idx(cfg.seed, first_image + i, cfg.h, cfg.w, cfg.K) for i in range(cfg.B)])
         t = torch.from_numpy(idx)
         out["keep_idx"] = t.pin_memory() if pinned_host else t.to(device)
     return out
 
 
-def layer_tensors(cfg: LayerConfig, device, pinned_host: bool = False) -> dict:
+def layer_tensors(cfg: LayerConfig, device, pinned_host: bool = False, first_image: int = 0) -> dict:
     d = params_tensors(cfg, "cpu" if pinned_host else device)
     if pinned_host:
         d = {k: v.pin_memory() for k, v in d.items()}
-    d.update(activations(cfg, device, pinned_host))
+    d.update(activations(cfg, device, pinned_host, first_image))
     return d

@@ -165,6 +165,37 @@ def test_masked_permutation_covariance():
     assert_close(yp, ref[:, perm])
 
 
+@pytest.mark.parametrize("masked", [False, True])
+def test_host_entry_point_pipelines_chunks(masked):
+    """Over 64 MB of x, the host entry point runs the batch as chunks of images (here 3 + 2): y
+    equals the device entry point's bit for bit and the oracle within tolerance, and a bad keep
+    index in the first chunk is still reported after the last chunk ran clean."""
+    from pooled_selective_scan_b200 import ssm
+    if masked:
+        h = w = 64
+        p = rand_layer(181, B=5, h=h, w=w, E=1152, N=16, R=8, dir_flags=3, K=3000)
+    else:
+        h = w = None
+        p = rand_layer(182, B=5, h=48, w=48, E=1536, N=16, R=8, dir_flags=3)
+    assert p["x"].nbytes > 64 << 20
+    t = {k: torch.from_numpy(v).pin_memory() for k, v in p.items()}
+    shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], 0, 3, t.get("keep_idx"), h, w)
+    run = ssm.HostForward(shape)
+    y_host = torch.empty(t["x"].shape, dtype=torch.float32).pin_memory()
+    run(t, y_host)
+    assert ssm.device_status(run.workspace) == 0
+    ref = oracle.forward(p["x"], p["z"], p["A_log"], p["D"], p["W_x"], p["W_dt"], p["b_dt"], 0, 3,
+                         keep_idx=p.get("keep_idx"), h=h, w=w)
+    assert_close(y_host.numpy(), ref)
+    dev = gpu_forward(p, 0, 3, h=h, w=w, intermediates=False)["y"]
+    assert np.array_equal(dev, y_host.numpy())
+    if masked:
+        t["keep_idx"][0, 7] = h * w  # out of range, in image 0 (first chunk)
+        run(t, y_host)
+        assert ssm.device_status(run.workspace) == 4  # FV_ERR_INDEX
+        assert_close(y_host.numpy()[3:], ref[3:])  # the second chunk is untouched by it
+
+
 @pytest.mark.parametrize("bad", ["dup", "neg", "big"])
 def test_masked_bad_index_reported_on_device(bad):
     p = rand_layer(140, B=2, h=4, w=4, E=16, N=16, R=2, dir_flags=3, K=6)
