@@ -7,7 +7,8 @@ One step = one fastvim_ssm_forward call over the whole batch of the workload (po
 projections -> scans -> repeat/skip/gate), inputs resident in HBM.  The default workload is the
 FastVim-T layer at 2048 px: B = 128, a 128 x 128 token grid, E = 384, N = 16, R = 12, column
 pooling, forward + backward scans, fp32.  Its x, z and y take 9.7 GB, far above the 126 MB L2,
-so no L2 flush is needed between steps.
+so no L2 flush is needed between steps (workloads under twice the L2 size get one before every
+step, outside the step's timed span).
 
 Under torchrun (N > 1) every rank runs its own batch of B distinct images on its own GPU
 (images rank*B .. rank*B + B - 1 of the seeded stream; the images are independent, so there is
@@ -37,15 +38,31 @@ UNIT = "grid tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 REFERENCE_BUDGET_S = 150.0
 
-# Algorithmic bytes per processed token of each kernel, in units of E*4 bytes (fp32 channels):
-# what the kernel must move at minimum for its step of the layer.
-KERNEL_BYTES_PER_TOKEN_E4 = {
-    "pool_dense_kernel": 1,        # read x
-    "epilogue_dense_kernel": 3,    # read x, read z, write y
-    "mask_pool_kernel": 1,         # read kept x
-    "mask_epilogue_kernel": 3,     # read kept x and z, write y
-    "fused_layer_kernel": 3,       # the whole layer: x once, z, y
-}
+L2_BYTES = 126 * 1024 * 1024
+# Special-function (MUFU) lanes per SM per clock on sm_100: 4 per SM sub-partition.
+MUFU_PER_SM_CLK = 16
+
+
+def kernel_work(name: str, cfg, pool_axis: int):
+    """(bound, algorithmic amount per launch) of one launch of kernel `name` on workload `cfg`:
+    bytes for the streaming kernels (what the step must move at minimum), exp2 evaluations for
+    the scans (one per state, step, channel and direction), None for the rest."""
+    tok = cfg.tokens_per_call()                       # grid tokens, or kept tokens when masked
+    row = 4 * cfg.E                                   # one fp32 token row
+    T = cfg.h if pool_axis == 0 else cfg.w
+    if name in ("pool_dense_kernel", "mask_pool_kernel"):
+        return "hbm", row * tok                       # read x
+    if name in ("epilogue_dense_kernel", "mask_epilogue_kernel", "fused_layer_kernel"):
+        return "hbm", 3 * row * tok                   # read x and z, write y (the fused launch: the layer)
+    if name == "scan_seq_kernel":
+        return "alu", cfg.B * T * cfg.E * cfg.N * cfg.nd
+    return None, 0
+
+
+def mufu_peak_gops(device_index: int, sm_max_mhz) -> float:
+    import torch
+    sms = torch.cuda.get_device_properties(device_index).multi_processor_count
+    return sms * MUFU_PER_SM_CLK * float(sm_max_mhz or 1965) * 1e6 / 1e9
 
 
 def parse(argv=None):
@@ -343,6 +360,11 @@ def run_ours(a, cfg, pool_axis):
     torch.cuda.synchronize(dev)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
+    # Workloads whose inputs fit in L2 get an L2 flush (a write of 2x the L2 size) before every
+    # step; the step time is then the span of the step's own launches (first to last event).
+    alg_bytes_call = cfg.algorithmic_bytes_per_call()
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if alg_bytes_call < 2 * L2_BYTES else None
+
     clocks = ClockSampler(local)
     clocks.start()
     if world > 1:
@@ -350,13 +372,18 @@ def run_ours(a, cfg, pool_axis):
     torch.cuda.synchronize(dev)
     start.record(stream)
     for i in range(a.steps):
+        if flush is not None:
+            flush.fill_(float(i))
         fwd.run_events(events[i])
     end.record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     clocks.stop()
-    local_ms = start.elapsed_time(end)
+    if flush is None:
+        local_ms = start.elapsed_time(end)
+    else:
+        local_ms = sum(evs[0].elapsed_time(evs[nl]) for evs in events)
     max_ms = reduce_max(local_ms, dev)
     per_kernel = {n: [] for n in names}
     for evs in events:
@@ -369,26 +396,42 @@ def run_ours(a, cfg, pool_axis):
     ms_step = max_ms / a.steps
     value = weak_scaling_value(tokens * a.steps, world, max_ms / 1e3)
     peak, peak_src = load_peaks()
-    alg_bytes_call = cfg.algorithmic_bytes_per_call()
 
     total_k = sum(sum(v) for v in per_kernel.values())
-    kern = {n: {"launches": len(v), "avg_us": 1e3 * statistics.mean(v), "share": sum(v) / total_k}
-            for n, v in per_kernel.items()}
+    mufu_peak = mufu_peak_gops(local, clocks.summary().get("sm_max_mhz"))
+    kern = {}
+    for n, v in per_kernel.items():
+        avg_s = statistics.mean(v) / 1e3
+        bound, amount = kernel_work(n, cfg, pool_axis)
+        ent = {"launches": len(v), "avg_us": avg_s * 1e6, "share": sum(v) / total_k, "bound": bound}
+        if bound == "hbm":
+            ent.update(achieved=amount / avg_s / 1e9, unit="GB/s", frac=amount / avg_s / 1e9 / peak)
+        elif bound == "alu":
+            ent.update(achieved=amount / avg_s / 1e9, unit="G exp2/s", frac=amount / avg_s / 1e9 / mufu_peak)
+        kern[n] = ent
     dom = max(kern, key=lambda n: kern[n]["share"])
-    dom_alg = KERNEL_BYTES_PER_TOKEN_E4.get(dom, 0) * 4 * cfg.E * tokens
-    dom_s = kern[dom]["avg_us"] / 1e6
-    achieved = dom_alg / dom_s / 1e9 if dom_alg else None
-    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": (achieved / peak) if achieved else None, "traffic": recorded_traffic(dom, cfg.name),
-                "algorithmic_bytes_per_launch": dom_alg, "peak_source": peak_src,
-                "note": "achieved = algorithmic bytes per launch / mean CUDA-event duration of the launch"}
+    bound, amount = kernel_work(dom, cfg, pool_axis)
+    dk = kern[dom]
+    if bound == "alu":
+        roofline = {"bound": "alu", "kernel": dom, "achieved": dk["achieved"], "peak": mufu_peak,
+                    "unit": "G exp2/s", "frac": dk["frac"], "traffic": recorded_traffic(dom, cfg.name),
+                    "algorithmic_exp2_per_launch": amount,
+                    "peak_source": f"derived: SMs x {MUFU_PER_SM_CLK} MUFU lanes/clk x max SM clock",
+                    "note": "achieved = exp2 evaluations per launch / mean CUDA-event duration of the launch"}
+    else:
+        roofline = {"bound": "hbm", "kernel": dom, "achieved": dk.get("achieved"), "peak": peak, "unit": "GB/s",
+                    "frac": dk.get("frac"), "traffic": recorded_traffic(dom, cfg.name),
+                    "algorithmic_bytes_per_launch": amount, "peak_source": peak_src,
+                    "note": "achieved = algorithmic bytes per launch / mean CUDA-event duration of the launch"}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic (seeded N(0,1) x, z; Mamba-style parameter init)",
         "config": dict(workload_desc(cfg, pool_axis),
-                       l2=f"inputs {alg_bytes_call / 1e9:.2f} GB per step > 126 MB L2; no flush",
+                       l2=(f"inputs {alg_bytes_call / 1e9:.2f} GB per step > 126 MB L2; no flush" if flush is None
+                           else f"inputs {alg_bytes_call / 1e6:.1f} MB per step < 2 x L2: L2 flushed (256 MB write) "
+                                f"before every step, step time = span of the step's launches"),
                        global_batch=cfg.B * world,
                        parallelism=f"data parallel, no collective: each of {world} GPU(s) runs its own "
                                    f"{cfg.B} distinct images"),

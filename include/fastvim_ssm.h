@@ -131,8 +131,8 @@ typedef struct {
                             w1 = SM id << 32 | CTA id, w2 = start (ns, %globaltimer),
                             w3 = wait_ns << 40 | total_ns (from start to the task's end)        */
     size_t trace_records;  /* number of trace entries (tasks of the call), else 0               */
-    size_t scan_bc;      /* dense layers: fused launch's B | C rows in scan order, else 0        */
-    size_t scan_dt;      /* dense layers: fused launch's dt_low rows, else 0                     */
+    size_t scan_bc;      /* fused launch only: B | C rows in scan order, else 0              */
+    size_t scan_dt;      /* fused launch only: dt_low rows, else 0                             */
     int T, S, nd;        /* pooled length, pooled-over length, number of directions          */
 } fv_ws_layout;
 
@@ -213,6 +213,15 @@ FV_API fv_status fastvim_ssm_forward_noalloc(const fv_ssm_args* args, void* stre
  * it records FV_ERR_TIMEOUT in the status word of `ws` (>= 1 KB, 256-byte aligned) and exits.
  * fastvim_get_device_status(ws, stream) then returns FV_ERR_TIMEOUT; the context stays usable. */
 FV_API fv_status fastvim_selftest_bounded_wait(void* ws, size_t ws_bytes, unsigned limit_us, void* stream);
+
+/* Self-test of the device math the layer uses instead of CUDA's full-precision functions, for
+ * checking against a reference on the host: out[i] = f(in[i]) for i < n, with f chosen by `fn`:
+ *   0  softplus(v) = log(1 + e^v)   (SFU exp2/log2 and a Mercator series for small e^-|v|)
+ *   1  SiLU(v) = v / (1 + e^-v)      (SFU exp2 and reciprocal; the gate)
+ *   2  2^v                           (SFU exp2, inputs below -126 flush to 0; the ZOH exponential)
+ * in, out: DEVICE float arrays of n elements (16-byte aligned, not overlapping); queued on
+ * `stream`.  Returns FV_ERR_SHAPE for an unknown fn or n < 0, FV_ERR_NULL for a NULL array. */
+FV_API fv_status fastvim_selftest_math(int fn, const float* in, float* out, int n, void* stream);
 
 /* Waits for `stream`, then reads the device status word of a workspace used by the last
  * forward call: FV_OK, FV_ERR_INDEX or FV_ERR_TIMEOUT (or FV_ERR_CUDA if the read fails). */

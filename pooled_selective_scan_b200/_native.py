@@ -43,6 +43,7 @@ EXPORTS = (
     "fastvim_ssm_forward_host",
     "fastvim_ssm_forward_noalloc",
     "fastvim_selftest_bounded_wait",
+    "fastvim_selftest_math",
     "fastvim_get_device_status",
 )
 
@@ -127,6 +128,9 @@ def lib() -> ctypes.CDLL:
             L.fastvim_ssm_forward_noalloc.restype = ctypes.c_int
             L.fastvim_selftest_bounded_wait.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint, ctypes.c_void_p]
             L.fastvim_selftest_bounded_wait.restype = ctypes.c_int
+            L.fastvim_selftest_math.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                                ctypes.c_void_p]
+            L.fastvim_selftest_math.restype = ctypes.c_int
             L.fastvim_get_device_status.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
             L.fastvim_get_device_status.restype = ctypes.c_int
             _lib = L

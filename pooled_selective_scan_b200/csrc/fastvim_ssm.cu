@@ -101,9 +101,11 @@ fv_status plan_layout(const fv::Shape& sh, fv_ws_layout* L) {
     L->xbar = off; off = round256(off + (size_t)sh.B * sh.T * sh.E * sizeof(float));
     L->u = off; off = round256(off + (size_t)sh.nd * sh.B * fv::u_block_stride(sh.T, sh.J) * sizeof(float));
     L->ys = off; off = round256(off + (size_t)sh.B * sh.T * sh.E * sizeof(float));
-    // scan-ready copies of B | C (chunk-interleaved rows) and dt_low, written by the projections
-    L->scan_bc = off; off = round256(off + (size_t)sh.nd * sh.B * fv::fused_bcs_stride(sh.T) * sizeof(float));
-    L->scan_dt = off; off = round256(off + (size_t)sh.nd * sh.B * fv::fused_dts_stride(sh.T, sh.R) * sizeof(float));
+    if (choose_path(sh) == Path::Fused) {
+        // scan-ready copies of B | C (chunk-interleaved rows) and dt_low, written by the projections
+        L->scan_bc = off; off = round256(off + (size_t)sh.nd * sh.B * fv::fused_bcs_stride(sh.T) * sizeof(float));
+        L->scan_dt = off; off = round256(off + (size_t)sh.nd * sh.B * fv::fused_dts_stride(sh.T, sh.R) * sizeof(float));
+    }
     if (sh.K > 0) {
         L->row_of = off; off = round256(off + (size_t)sh.B * sh.K * sizeof(int32_t));
         L->row_off = off; off = round256(off + (size_t)sh.B * (sh.T + 1) * sizeof(int32_t));
@@ -129,7 +131,7 @@ constexpr size_t kMaxSmemOptin = 227 * 1024;
 constexpr double kChainLatencyUs = 60.0;
 
 fv_status check_limits(const fv::Shape& sh) {
-    if (fv::fused_scan_smem_floats(sh) * sizeof(float) > kMaxSmemOptin) return FV_ERR_UNSUPPORTED;
+    if (fv::seq_smem_floats(sh) * sizeof(float) > kMaxSmemOptin) return FV_ERR_UNSUPPORTED;
     if (fv::fused_proj_smem_floats(sh) * sizeof(float) > kMaxSmemOptin) return FV_ERR_UNSUPPORTED;
     if (sh.K > 0 && bucket_smem_bytes(sh) > kMaxSmemOptin) return FV_ERR_UNSUPPORTED;
     return FV_OK;
@@ -259,9 +261,9 @@ int launch_count_of(const fv::Shape& sh) {
 }
 
 const char* launch_name_of(const fv::Shape& sh, int i) {
-    static const char* dense[] = {"pool_dense_kernel", "proj_tasks_kernel", "scan_tasks_kernel",
+    static const char* dense[] = {"pool_dense_kernel", "proj_tasks_kernel", "scan_seq_kernel",
                                   "epilogue_dense_kernel"};
-    static const char* masked[] = {"mask_bucket_kernel", "mask_pool_kernel", "proj_tasks_kernel", "scan_tasks_kernel",
+    static const char* masked[] = {"mask_bucket_kernel", "mask_pool_kernel", "proj_tasks_kernel", "scan_seq_kernel",
                                    "mask_epilogue_kernel"};
     if (i < 0 || i >= launch_count_of(sh)) return "";
     if (choose_path(sh) == Path::Fused) return "fused_layer_kernel";
@@ -315,6 +317,8 @@ fv_status launch_proj_tasks(const fv::Shape& sh, const fv_ssm_args* a, const fv_
     const fv::FusedPlan pl = plan_fused(sh);
     fv::FusedPtrs p = fused_ptrs(a, L, ws);
     p.ctrl = nullptr;
+    p.bcs = nullptr;  // the staged scans read u directly
+    p.dts = nullptr;
     const size_t smem = fv::fused_proj_smem_floats(sh) * sizeof(float);
     cudaError_t e = ensure_smem(fv::proj_tasks_kernel, smem);
     if (e != cudaSuccess) { note_cuda(e, "proj smem attribute"); return FV_ERR_CUDA; }
@@ -323,24 +327,25 @@ fv_status launch_proj_tasks(const fv::Shape& sh, const fv_ssm_args* a, const fv_
     return FV_OK;
 }
 
-// Staged: scans of every channel tile of every image (one CTA per tile).
-template <int ND, bool Z>
-fv_status launch_scan_tasks_t(const fv::Shape& sh, const fv::FusedPlan& pl, const fv::FusedPtrs& p, cudaStream_t st) {
-    const size_t smem = fv::fused_scan_smem_floats(sh) * sizeof(float);
-    auto kern = fv::scan_tasks_kernel<ND, Z>;
-    cudaError_t e = ensure_smem(kern, smem);
-    if (e != cudaSuccess) { note_cuda(e, "scan smem attribute"); return FV_ERR_CUDA; }
-    kern<<<sh.B * pl.nS, fv::kFusedThreads, smem, st>>>(sh, pl, p);
-    FV_LAUNCH_CHECK("scan_tasks_kernel");
+// Staged: every (image, 128-channel tile, direction) recurrence, one thread each.  With both
+// directions the two add into ys, which is zeroed first.
+fv_status launch_scan_seq(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st) {
+    float* ys = (float*)(ws + L.ys);
+    cudaError_t e;
+    if (sh.nd == 2 && (e = cudaMemsetAsync(ys, 0, (size_t)sh.B * sh.T * sh.E * sizeof(float), st)) != cudaSuccess) {
+        note_cuda(e, "scan output reset");
+        return FV_ERR_CUDA;
+    }
+    const size_t smem = fv::seq_smem_floats(sh) * sizeof(float);
+    auto kern = sh.zoh_exact ? fv::scan_seq_kernel<true> : fv::scan_seq_kernel<false>;
+    if ((e = ensure_smem(kern, smem)) != cudaSuccess) { note_cuda(e, "scan smem attribute"); return FV_ERR_CUDA; }
+    const long long tiles = (sh.E + fv::kSeqThreads - 1) / fv::kSeqThreads;
+    const long long grid = (long long)sh.B * tiles * sh.nd;
+    if (grid >= (1ll << 31)) return FV_ERR_UNSUPPORTED;
+    kern<<<(unsigned)grid, fv::kSeqThreads, smem, st>>>(sh, (const float*)(ws + L.u), (const float*)(ws + L.xbar),
+                                                         a->A_log, a->W_dt, a->b_dt, ys);
+    FV_LAUNCH_CHECK("scan_seq_kernel");
     return FV_OK;
-}
-fv_status launch_scan_tasks(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st) {
-    const fv::FusedPlan pl = plan_fused(sh);
-    fv::FusedPtrs p = fused_ptrs(a, L, ws);
-    p.ctrl = nullptr;
-    if (sh.nd == 2)
-        return sh.zoh_exact ? launch_scan_tasks_t<2, true>(sh, pl, p, st) : launch_scan_tasks_t<2, false>(sh, pl, p, st);
-    return sh.zoh_exact ? launch_scan_tasks_t<1, true>(sh, pl, p, st) : launch_scan_tasks_t<1, false>(sh, pl, p, st);
 }
 
 fv_status forward_impl(const fv_ssm_args* a, void* ws_v, size_t ws_bytes, cudaStream_t st,
@@ -400,7 +405,7 @@ fv_status forward_impl(const fv_ssm_args* a, void* ws_v, size_t ws_bytes, cudaSt
     FV_MARK(marks, st);
     if ((s = launch_proj_tasks(sh, a, L, ws, st)) != FV_OK) return s;
     FV_MARK(marks, st);
-    if ((s = launch_scan_tasks(sh, a, L, ws, st)) != FV_OK) return s;
+    if ((s = launch_scan_seq(sh, a, L, ws, st)) != FV_OK) return s;
     FV_MARK(marks, st);
     if (sh.K == 0) {
         fv::epilogue_dense_kernel<<<M, fv::kThreads, 0, st>>>(sh, a->x, a->z, (const float*)(ws + L.ys), a->D, a->y);
@@ -623,6 +628,17 @@ fv_status fastvim_selftest_bounded_wait(void* ws, size_t ws_bytes, unsigned limi
     unsigned* ctrl = (unsigned*)((char*)ws + 256);
     fv::bounded_wait_selftest_kernel<<<1, 32, 0, st>>>(status, ctrl, (unsigned long long)limit_us * 1000ull);
     FV_LAUNCH_CHECK("bounded_wait_selftest_kernel");
+    return FV_OK;
+}
+
+fv_status fastvim_selftest_math(int fn, const float* in, float* out, int n, void* stream) {
+    if (fn < 0 || fn > 2 || n < 0) return FV_ERR_SHAPE;
+    if (n == 0) return FV_OK;
+    if (!in || !out) return FV_ERR_NULL;
+    if (((uintptr_t)in & 15u) || ((uintptr_t)out & 15u)) return FV_ERR_ALIGN;
+    if ((const char*)out < (const char*)(in + n) && (const char*)in < (const char*)(out + n)) return FV_ERR_ALIAS;
+    fv::math_selftest_kernel<<<(n + 255) / 256, 256, 0, (cudaStream_t)stream>>>(fn, in, out, n);
+    FV_LAUNCH_CHECK("math_selftest_kernel");
     return FV_OK;
 }
 

@@ -1,5 +1,5 @@
 // fv_fused.cuh -- the dense FastVim SSM layer as ONE persistent, image-pipelined launch (sm_100a),
-// and the task bodies that the staged launches reuse.
+// and the projection task body that the staged launches reuse.
 //
 // The layer's pooled tokens depend on ALL of an image's x, and every output token depends on the
 // whole image's scan, so x must be read once for pooling and once more for the D x skip.  One
@@ -473,6 +473,7 @@ __device__ __forceinline__ void fused_proj_t(const Shape& sh, const FusedPlan& p
                     const int t = tq0 + r;
                     const float v = acc[i][j];
                     p.u[u_offset(sh, k, b, t) + jc] = v;
+                    if (!p.bcs) continue;  // staged launches scan from u alone
                     if (jc < R) {
                         dtb[(size_t)t * R + jc] = v;
                     } else {
@@ -568,7 +569,7 @@ __device__ __forceinline__ void fused_scan(const Shape& sh, const FusedPlan& pl,
                 float a = wr[R];
 #pragma unroll 4
                 for (int r = 0; r < R; ++r) a = fmaf(wr[r], dl[r], a);
-                dx[(k * rows + post[t]) * XS + c] = live ? softplus_f(a) : 0.f;
+                dx[(k * rows + post[t]) * XS + c] = live ? softplus_fast(a) : 0.f;
             }
         }
     }
@@ -832,16 +833,11 @@ fused_layer_kernel(Shape sh, FusedPlan pl, FusedPtrs p) {
     }
 }
 
-// Staged launches of the same task bodies: one CTA per projection task / per scan task, ordered by
-// the launch boundaries instead of counters.
+// Staged launch of the projection task body: one CTA per task, ordered by the launch boundaries
+// instead of counters.
 __global__ void __launch_bounds__(kFusedThreads, 2) proj_tasks_kernel(Shape sh, FusedPlan pl, FusedPtrs p) {
     extern __shared__ __align__(128) float smem_f[];
     fused_proj(sh, pl, p, blockIdx.x / pl.nQ, blockIdx.x % pl.nQ, smem_f);
-}
-template <int ND, bool ZOH_EXACT>
-__global__ void __launch_bounds__(kFusedThreads, 2) scan_tasks_kernel(Shape sh, FusedPlan pl, FusedPtrs p) {
-    extern __shared__ __align__(128) float smem_f[];
-    fused_scan<ND, ZOH_EXACT>(sh, pl, p, blockIdx.x / pl.nS, blockIdx.x % pl.nS, smem_f);
 }
 
 // A single CTA that waits, with the layer's bounded wait, on a counter that nothing increments:

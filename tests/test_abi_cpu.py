@@ -170,7 +170,7 @@ def test_workspace_layout(lib, pool_axis, K):
 
 
 @pytest.mark.parametrize("flags,want", [(0, ["fused_layer_kernel"]), (4, ["fused_layer_kernel"]),
-                                        (2, ["pool_dense_kernel", "proj_tasks_kernel", "scan_tasks_kernel",
+                                        (2, ["pool_dense_kernel", "proj_tasks_kernel", "scan_seq_kernel",
                                              "epilogue_dense_kernel"])])
 def test_path_selection_is_host_side(lib, flags, want):
     a = good_args(h=128, w=128, B=4, flags=flags)  # 2048 px FastVim-T images: fused by default
@@ -185,3 +185,13 @@ def test_path_selection_is_host_side(lib, flags, want):
 def test_forced_fused_path_refuses_masked_layers(lib):
     a = good_args(K=49, keep_idx=FAKE + (9 << 32), flags=4)
     assert lib.fastvim_ssm_launch_count(ctypes.byref(a)) == 0
+
+
+def test_math_selftest_rejects_bad_arguments(lib):
+    f = lib.fastvim_selftest_math
+    assert f(3, ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE + (1 << 32)), 8, None) == nat.FV_ERR_SHAPE
+    assert f(0, ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE + (1 << 32)), -1, None) == nat.FV_ERR_SHAPE
+    assert f(0, None, ctypes.c_void_p(FAKE), 8, None) == nat.FV_ERR_NULL
+    assert f(0, ctypes.c_void_p(FAKE + 4), ctypes.c_void_p(FAKE + (1 << 32)), 8, None) == nat.FV_ERR_ALIGN
+    assert f(0, ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE + 16), 8, None) == nat.FV_ERR_ALIAS
+    assert f(1, None, None, 0, None) == nat.FV_OK  # nothing to do
