@@ -56,9 +56,9 @@ def _load():
                 "fvo_pool_masked": [P, P, P, I, I, I, I, I, Dbl, P],
                 "fvo_proj": [P, I, I, I, I, I, I, P, P, P, P, P],
                 "fvo_scan": [P, P, P, P, I, I, I, I, I, I, U, I, P],
-                "fvo_gate_dense": [P, P, P, P, I, I, I, I, I, I, P],
-                "fvo_gate_masked": [P, P, P, P, P, I, I, I, I, I, P],
-                "fvo_forward": [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, U, Dbl, I, I, P],
+                "fvo_gate_dense": [P, P, P, P, I, I, I, I, I, I, P, P, Dbl, P],
+                "fvo_gate_masked": [P, P, P, P, P, I, I, I, I, I, P, P, Dbl, P],
+                "fvo_forward": [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, U, Dbl, I, P, P, Dbl, I, P],
             }
             for name, argtypes in sigs.items():
                 fn = getattr(lib, name)
@@ -169,32 +169,48 @@ def scan(xbar, delta, u, A_log, R, N, dir_flags, zoh_exact=False):
     return ys
 
 
-def gate_dense(x, z, ys, D, pool_axis):
-    """Repeat + D x skip + SiLU(z) gate on the dense grid -> y [B,h,w,E]."""
+def _ln(ln_gamma, ln_beta, E):
+    """LayerNorm gamma and beta as fp32 [E] arrays (None stays None: the C side checks that both
+    or neither are given)."""
+    out = []
+    for v in (ln_gamma, ln_beta):
+        a = None if v is None else _f32(v)
+        assert a is None or a.shape == (E,)
+        out.append(a)
+    return out
+
+
+def gate_dense(x, z, ys, D, pool_axis, ln_gamma=None, ln_beta=None, ln_eps=1e-5):
+    """Repeat + D x skip (+ post-SSM LayerNorm) + SiLU(z) gate on the dense grid -> y [B,h,w,E]."""
     x, z, D = _f32(x), _f32(z), _f32(D)
     ys = _f64(ys)
     B, h, w, E = x.shape
+    g, b = _ln(ln_gamma, ln_beta, E)
     y = np.empty(x.shape, np.float64)
-    st = _load().fvo_gate_dense(_p(x), _p(z), _p(ys), _p(D), B, h, w, E, D.shape[0], pool_axis, _p(y))
+    st = _load().fvo_gate_dense(_p(x), _p(z), _p(ys), _p(D), B, h, w, E, D.shape[0], pool_axis, _p(g), _p(b),
+                                float(ln_eps), _p(y))
     _check(st, "gate_dense")
     return y
 
 
-def gate_masked(x, z, ys, D, row_of):
-    """Repeat to kept tokens + skip + gate -> y [B,K,E]."""
+def gate_masked(x, z, ys, D, row_of, ln_gamma=None, ln_beta=None, ln_eps=1e-5):
+    """Repeat to kept tokens + skip (+ post-SSM LayerNorm) + gate -> y [B,K,E]."""
     x, z, D = _f32(x), _f32(z), _f32(D)
     ys = _f64(ys)
     row_of = _i32(row_of)
     B, K, E = x.shape
     T = ys.shape[1]
+    g, b = _ln(ln_gamma, ln_beta, E)
     y = np.empty(x.shape, np.float64)
-    st = _load().fvo_gate_masked(_p(x), _p(z), _p(ys), _p(D), _p(row_of), B, K, T, E, D.shape[0], _p(y))
+    st = _load().fvo_gate_masked(_p(x), _p(z), _p(ys), _p(D), _p(row_of), B, K, T, E, D.shape[0], _p(g), _p(b),
+                                 float(ln_eps), _p(y))
     _check(st, "gate_masked")
     return y
 
 
 def forward(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis, dir_flags, keep_idx=None, h=None,
-            w=None, pool_scale=1.0, zoh_exact=False, nthreads=1, allow_bad_index=False):
+            w=None, pool_scale=1.0, zoh_exact=False, nthreads=1, allow_bad_index=False, ln_gamma=None,
+            ln_beta=None, ln_eps=1e-5):
     """The whole layer, image by image.
 
     Dense: x, z [B,h,w,E] -> y [B,h,w,E].  Masked: x, z [B,K,E], keep_idx [B,K] with the grid
@@ -214,16 +230,18 @@ def forward(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis, dir_flags, keep_idx=None
         idx = _i32(keep_idx)
         assert h is not None and w is not None and idx.shape == (B, K)
     assert E2 == E and z.shape == x.shape
+    g, b = _ln(ln_gamma, ln_beta, E)
     y = np.empty(x.shape, np.float64)
     st = _load().fvo_forward(_p(x), _p(z), _p(A_log), _p(D), _p(W_x), _p(W_dt), _p(b_dt), _p(idx),
                              B, h, w, E, N, R, K, pool_axis, int(dir_flags), float(pool_scale),
-                             int(bool(zoh_exact)), int(nthreads), _p(y))
+                             int(bool(zoh_exact)), _p(g), _p(b), float(ln_eps), int(nthreads), _p(y))
     _check(st, "forward", allow=(FVO_BAD_INDEX,) if allow_bad_index else ())
     return (y, st) if allow_bad_index else y
 
 
 def forward_intermediates(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis, dir_flags, keep_idx=None,
-                          h=None, w=None, pool_scale=1.0, zoh_exact=False):
+                          h=None, w=None, pool_scale=1.0, zoh_exact=False, ln_gamma=None, ln_beta=None,
+                          ln_eps=1e-5):
     """The same chain step by step, returning every intermediate as a dict (small sizes only)."""
     A_log, W_dt = _f32(A_log), _f32(W_dt)
     N = A_log.shape[2]
@@ -240,8 +258,8 @@ def forward_intermediates(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis, dir_flags,
     u, delta = proj(xbar, W_x, W_dt, b_dt, R, N)
     ys = scan(xbar, delta, u, A_log, R, N, dir_flags, zoh_exact)
     if keep_idx is None:
-        y = gate_dense(x, z, ys, D, pool_axis)
+        y = gate_dense(x, z, ys, D, pool_axis, ln_gamma, ln_beta, ln_eps)
     else:
-        y = gate_masked(x, z, ys, D, out["row_of"])
+        y = gate_masked(x, z, ys, D, out["row_of"], ln_gamma, ln_beta, ln_eps)
     out.update(xbar=xbar, u=u, delta=delta, ys=ys, y=y)
     return out

@@ -191,47 +191,94 @@ int fvo_scan(const double* xbar, const double* delta, const double* u, const flo
     return FVO_OK;
 }
 
+/* Post-SSM LayerNorm over the E channels of one token (gptget.net summary of 2502.00594,
+ * "方法详解" item 5: the repeated output goes through the skip connection and a LayerNorm;
+ * pith.science verdict, referee report: the post-SSM LayerNorm is the one VMamba adds before
+ * the gate).  Standard layer normalisation with the biased variance:
+ *   LN(s)_e = gamma_e (s_e - mu) / sqrt(var + eps) + beta_e,
+ *   mu = (1/E) sum_e s_e,  var = (1/E) sum_e (s_e - mu)^2. */
+static void layernorm_row(double* s, int E, const float* gamma, const float* beta, double eps)
+{
+    double mu = 0.0;
+    for (int e = 0; e < E; ++e) mu += s[e];
+    mu /= (double)E;
+    double var = 0.0;
+    for (int e = 0; e < E; ++e) {
+        const double d = s[e] - mu;
+        var += d * d;
+    }
+    var /= (double)E;
+    const double inv = 1.0 / sqrt(var + eps);
+    for (int e = 0; e < E; ++e) s[e] = (double)gamma[e] * ((s[e] - mu) * inv) + (double)beta[e];
+}
+
+static int ln_args_ok(const float* ln_gamma, const float* ln_beta, double ln_eps)
+{
+    if ((ln_gamma == NULL) != (ln_beta == NULL)) return 0;
+    return ln_gamma == NULL || (ln_eps >= 0.0 && isfinite(ln_eps));
+}
+
+/* One output token: s = ys row + (sum_k D[k]) x (the repeat and the skip), optionally
+ * LayerNorm(s), then y = SiLU(z) * s.  tmp: E doubles of scratch. */
+static void gate_token(const float* x, const float* z, const double* ysr, const float* D, int E, int nd,
+                       const float* ln_gamma, const float* ln_beta, double ln_eps, double* tmp, double* y)
+{
+    for (int e = 0; e < E; ++e) {
+        double Dsum = 0.0;
+        for (int k = 0; k < nd; ++k) Dsum += (double)D[(size_t)k * E + e];
+        tmp[e] = ysr[e] + Dsum * (double)x[e];
+    }
+    if (ln_gamma) layernorm_row(tmp, E, ln_gamma, ln_beta, ln_eps);
+    for (int e = 0; e < E; ++e) y[e] = silu((double)z[e]) * tmp[e];
+}
+
 /* Repeat, skip and gate (pith.science verdict, "key_machinery": the repeat restores the token
  * count before the D x skip; ijyty.com Vision Mamba article, section 2.1: gate(z, y_fwd + y_bwd)):
- *   y[b][i][j] = SiLU(z[b][i][j]) * (ys[b][t(i,j)] + (sum_k D[k]) * x[b][i][j]). */
+ *   y[b][i][j] = SiLU(z[b][i][j]) * N(ys[b][t(i,j)] + (sum_k D[k]) * x[b][i][j]),
+ * N = the post-SSM LayerNorm when ln_gamma is given, else the identity. */
 int fvo_gate_dense(const float* x, const float* z, const double* ys, const float* D, int B,
-                   int h, int w, int E, int nd, int pool_axis, double* y)
+                   int h, int w, int E, int nd, int pool_axis, const float* ln_gamma,
+                   const float* ln_beta, double ln_eps, double* y)
 {
     if (B < 0 || h <= 0 || w <= 0 || E <= 0 || nd < 1 || nd > 2) return FVO_BAD_SHAPE;
+    if (!ln_args_ok(ln_gamma, ln_beta, ln_eps)) return FVO_BAD_SHAPE;
     const int T = pooled_len(h, w, pool_axis);
+    double* tmp = (double*)malloc(sizeof(double) * (size_t)E);
+    if (!tmp) return FVO_NO_MEMORY;
     for (int b = 0; b < B; ++b)
         for (int i = 0; i < h; ++i)
             for (int j = 0; j < w; ++j) {
                 const int t = (pool_axis == FVO_POOL_W) ? i : j;
-                for (int e = 0; e < E; ++e) {
-                    const size_t g = (((size_t)b * h + i) * w + j) * E + e;
-                    double Dsum = 0.0;
-                    for (int k = 0; k < nd; ++k) Dsum += (double)D[(size_t)k * E + e];
-                    const double s = ys[((size_t)b * T + t) * E + e] + Dsum * (double)x[g];
-                    y[g] = silu((double)z[g]) * s;
-                }
+                const size_t g = (((size_t)b * h + i) * w + j) * E;
+                gate_token(x + g, z + g, ys + ((size_t)b * T + t) * E, D, E, nd, ln_gamma, ln_beta, ln_eps,
+                           tmp, y + g);
             }
+    free(tmp);
     return FVO_OK;
 }
 
 /* Masked form: each kept token takes the pooled output of its row (repeat only to kept
  * indices).  A token whose index was rejected (row_of < 0) gets 0. */
 int fvo_gate_masked(const float* x, const float* z, const double* ys, const float* D,
-                    const int32_t* row_of, int B, int K, int T, int E, int nd, double* y)
+                    const int32_t* row_of, int B, int K, int T, int E, int nd, const float* ln_gamma,
+                    const float* ln_beta, double ln_eps, double* y)
 {
     if (B < 0 || K < 0 || T <= 0 || E <= 0 || nd < 1 || nd > 2) return FVO_BAD_SHAPE;
+    if (!ln_args_ok(ln_gamma, ln_beta, ln_eps)) return FVO_BAD_SHAPE;
+    double* tmp = (double*)malloc(sizeof(double) * (size_t)E);
+    if (!tmp) return FVO_NO_MEMORY;
     for (int b = 0; b < B; ++b)
         for (int k = 0; k < K; ++k) {
             const int32_t t = row_of[(size_t)b * K + k];
-            for (int e = 0; e < E; ++e) {
-                const size_t g = ((size_t)b * K + k) * E + e;
-                if (t < 0) { y[g] = 0.0; continue; }
-                double Dsum = 0.0;
-                for (int d = 0; d < nd; ++d) Dsum += (double)D[(size_t)d * E + e];
-                const double s = ys[((size_t)b * T + t) * E + e] + Dsum * (double)x[g];
-                y[g] = silu((double)z[g]) * s;
+            const size_t g = ((size_t)b * K + k) * E;
+            if (t < 0) {
+                for (int e = 0; e < E; ++e) y[g + e] = 0.0;
+                continue;
             }
+            gate_token(x + g, z + g, ys + ((size_t)b * T + t) * E, D, E, nd, ln_gamma, ln_beta, ln_eps, tmp,
+                       y + g);
         }
+    free(tmp);
     return FVO_OK;
 }
 
@@ -240,6 +287,7 @@ static int forward_one(const float* x, const float* z, const float* A_log, const
                        const float* W_x, const float* W_dt, const float* b_dt,
                        const int32_t* keep_idx, int h, int w, int E, int N, int R, int K,
                        int pool_axis, unsigned dir_flags, double pool_scale, int zoh_exact,
+                       const float* ln_gamma, const float* ln_beta, double ln_eps,
                        double* y, double* xbar, double* u, double* delta, double* ys,
                        int32_t* row_of, int32_t* row_off, int32_t* row_tok)
 {
@@ -257,9 +305,9 @@ static int forward_one(const float* x, const float* z, const float* A_log, const
     if ((st = fvo_proj(xbar, 1, T, E, nd, R, N, W_x, W_dt, b_dt, u, delta))) return st;
     if ((st = fvo_scan(xbar, delta, u, A_log, 1, T, E, nd, R, N, dir_flags, zoh_exact, ys))) return st;
     if (keep_idx)
-        st = fvo_gate_masked(x, z, ys, D, row_of, 1, K, T, E, nd, y);
+        st = fvo_gate_masked(x, z, ys, D, row_of, 1, K, T, E, nd, ln_gamma, ln_beta, ln_eps, y);
     else
-        st = fvo_gate_dense(x, z, ys, D, 1, h, w, E, nd, pool_axis, y);
+        st = fvo_gate_dense(x, z, ys, D, 1, h, w, E, nd, pool_axis, ln_gamma, ln_beta, ln_eps, y);
     return st ? st : idx_status;
 }
 
@@ -267,12 +315,12 @@ int fvo_forward(const float* x, const float* z, const float* A_log, const float*
                 const float* W_x, const float* W_dt, const float* b_dt,
                 const int32_t* keep_idx, int B, int h, int w, int E, int N, int R, int K,
                 int pool_axis, unsigned dir_flags, double pool_scale, int zoh_exact,
-                int nthreads, double* y)
+                const float* ln_gamma, const float* ln_beta, double ln_eps, int nthreads, double* y)
 {
     const int nd = popcount2(dir_flags);
     if (B < 0 || h <= 0 || w <= 0 || E <= 0 || N <= 0 || R <= 0 || nd < 1 ||
         (dir_flags & ~3u) != 0 || (pool_axis != FVO_POOL_W && pool_axis != FVO_POOL_H) ||
-        (keep_idx && (K < 0 || K > h * w)))
+        (keep_idx && (K < 0 || K > h * w)) || !ln_args_ok(ln_gamma, ln_beta, ln_eps))
         return FVO_BAD_SHAPE;
     const int T = pooled_len(h, w, pool_axis);
     const int J = R + 2 * N;
@@ -294,8 +342,8 @@ int fvo_forward(const float* x, const float* z, const float* A_log, const float*
         if (xbar && u && delta && ys && row_of && row_off && row_tok)
             st = forward_one(x + (size_t)b * tok * E, z + (size_t)b * tok * E, A_log, D, W_x,
                              W_dt, b_dt, keep_idx ? keep_idx + (size_t)b * K : NULL, h, w, E, N,
-                             R, K, pool_axis, dir_flags, pool_scale, zoh_exact,
-                             y + (size_t)b * tok * E, xbar, u, delta, ys, row_of, row_off, row_tok);
+                             R, K, pool_axis, dir_flags, pool_scale, zoh_exact, ln_gamma, ln_beta,
+                             ln_eps, y + (size_t)b * tok * E, xbar, u, delta, ys, row_of, row_off, row_tok);
         free(xbar); free(u); free(delta); free(ys); free(row_of); free(row_off); free(row_tok);
         if (st != FVO_OK) {
 #ifdef _OPENMP

@@ -15,7 +15,9 @@
  *   - pith.science verdict on 2502.00594, field "key_machinery": the repeat restores the token
  *     count before the D x_t skip connection (so the skip uses full-resolution x);
  *   - ijyty.com Vision Mamba article, section 2.1 code: the block gates the sum of the forward
- *     and backward SSM outputs with z.
+ *     and backward SSM outputs with z;
+ *   - optional post-SSM LayerNorm after the skip and before the gate (summary page, "方法详解"
+ *     item 5; verdict page, referee report on the VMamba post-SSM LayerNorm).
  *
  * All arithmetic is fp64; inputs are fp32 arrays as the GPU library sees them.
  * Layouts (row-major, last index fastest):
@@ -63,13 +65,16 @@ int fvo_scan(const double* xbar, const double* delta, const double* u, const flo
              int B, int T, int E, int nd, int R, int N, unsigned dir_flags, int zoh_exact,
              double* ys);
 
-/* Repeat + D x skip + SiLU(z) gate on the dense grid. */
+/* Repeat + D x skip (+ the post-SSM LayerNorm over E when ln_gamma, ln_beta [E] are given,
+ * both or neither, ln_eps >= 0) + SiLU(z) gate on the dense grid. */
 int fvo_gate_dense(const float* x, const float* z, const double* ys, const float* D, int B,
-                   int h, int w, int E, int nd, int pool_axis, double* y);
+                   int h, int w, int E, int nd, int pool_axis, const float* ln_gamma,
+                   const float* ln_beta, double ln_eps, double* y);
 
 /* Same on the kept tokens, each taking the pooled output of its row. */
 int fvo_gate_masked(const float* x, const float* z, const double* ys, const float* D,
-                    const int32_t* row_of, int B, int K, int T, int E, int nd, double* y);
+                    const int32_t* row_of, int B, int K, int T, int E, int nd, const float* ln_gamma,
+                    const float* ln_beta, double ln_eps, double* y);
 
 /* The whole layer, one image at a time (OpenMP over images when nthreads > 1).
  * keep_idx == NULL: dense x, z, y [B][h][w][E]; otherwise masked [B][K][E]. */
@@ -77,7 +82,7 @@ int fvo_forward(const float* x, const float* z, const float* A_log, const float*
                 const float* W_x, const float* W_dt, const float* b_dt,
                 const int32_t* keep_idx, int B, int h, int w, int E, int N, int R, int K,
                 int pool_axis, unsigned dir_flags, double pool_scale, int zoh_exact,
-                int nthreads, double* y);
+                const float* ln_gamma, const float* ln_beta, double ln_eps, int nthreads, double* y);
 
 #ifdef __cplusplus
 }

@@ -35,6 +35,16 @@ MUTATIONS = {
     "masked pool divides by T": ("pool_scale * acc / (double)S;\n            }\n    return FVO_OK;\n}\n\n/* Input-dependent",
                                  "pool_scale * acc / (double)T;\n            }\n    return FVO_OK;\n}\n\n/* Input-dependent"),
     "duplicate ids accepted": ("if (g < 0 || g >= G || seen[g])", "if (g < 0 || g >= G)"),
+    "LayerNorm with the unbiased variance": ("var /= (double)E;", "var /= (double)(E - 1);"),
+    "LayerNorm eps outside the root": ("1.0 / sqrt(var + eps)", "1.0 / (sqrt(var) + eps)"),
+    "LayerNorm gamma and beta swapped": ("(double)gamma[e] * ((s[e] - mu) * inv) + (double)beta[e]",
+                                         "(double)beta[e] * ((s[e] - mu) * inv) + (double)gamma[e]"),
+    "LayerNorm before the skip": ("tmp[e] = ysr[e] + Dsum * (double)x[e];\n    }\n    if (ln_gamma) layernorm_row(tmp, E, ln_gamma, ln_beta, ln_eps);",
+                                  "tmp[e] = ysr[e];\n    }\n    if (ln_gamma) layernorm_row(tmp, E, ln_gamma, ln_beta, ln_eps);\n"
+                                  "    for (int e = 0; e < E; ++e) for (int k = 0; k < nd; ++k) tmp[e] += (double)D[(size_t)k * E + e] * (double)x[e];"),
+    "LayerNorm after the gate": ("    if (ln_gamma) layernorm_row(tmp, E, ln_gamma, ln_beta, ln_eps);\n    for (int e = 0; e < E; ++e) y[e] = silu((double)z[e]) * tmp[e];",
+                                 "    for (int e = 0; e < E; ++e) tmp[e] *= silu((double)z[e]);\n"
+                                 "    if (ln_gamma) layernorm_row(tmp, E, ln_gamma, ln_beta, ln_eps);\n    for (int e = 0; e < E; ++e) y[e] = tmp[e];"),
     "pool scale ignored": ("pool_scale * acc / (double)S;\n            }\n    return FVO_OK;\n}\n\n/* Row of",
                            "acc / (double)S;\n            }\n    return FVO_OK;\n}\n\n/* Row of"),
 }

@@ -445,3 +445,63 @@ def test_p8_bad_indices_are_reported(oracle_mod, bad):
     st, row_of, _, _ = oracle_mod.mask_rows(idx, h, w, 0)
     assert st == oracle_mod.FVO_BAD_INDEX
     assert (row_of < 0).sum() == 1
+
+
+# ---------------------------------------------------------------------------------------------
+# p9: the post-SSM LayerNorm (after the repeat and the skip, before the gate).
+# ---------------------------------------------------------------------------------------------
+def _silu(z):
+    return z * scipy.special.expit(z)
+
+
+def _ln_case(rng, masked, pool_axis):
+    B, h, w, E, N, R, nd = 2, 3, 5, 7, 4, 3, 2
+    A_log, D, W_x, W_dt, b_dt = _rand_params(rng, nd, E, N, R)
+    shp = (B, 6, E) if masked else (B, h, w, E)
+    x = rng.standard_normal(shp).astype(np.float32)
+    # |SiLU(z)| >= 0.27 everywhere, so the pre-gate value can be recovered by division
+    z = (np.sign(rng.standard_normal(shp)) * (1.0 + np.abs(rng.standard_normal(shp)))).astype(np.float32)
+    idx = np.stack([rng.permutation(h * w)[:6] for _ in range(B)]).astype(np.int32) if masked else None
+    gamma = rng.uniform(0.5, 1.5, E).astype(np.float32)
+    beta = (0.3 * rng.standard_normal(E)).astype(np.float32)
+    return dict(x=x, z=z, A_log=A_log, D=D, W_x=W_x, W_dt=W_dt, b_dt=b_dt, pool_axis=pool_axis, dir_flags=3,
+                keep_idx=idx, h=h, w=w), gamma, beta
+
+
+@pytest.mark.parametrize("masked,pool_axis", [(False, 0), (False, 1), (True, 0), (True, 1)])
+def test_p9_layernorm_is_torch_layer_norm_of_the_pre_gate_value(oracle_mod, masked, pool_axis):
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(950 + 2 * pool_axis + masked)
+    a, gamma, beta = _ln_case(rng, masked, pool_axis)
+    eps = 0.05  # large enough that its placement under the root matters
+    y0 = oracle_mod.forward(**a)
+    y1 = oracle_mod.forward(**a, ln_gamma=gamma, ln_beta=beta, ln_eps=eps)
+    s = _silu(a["z"].astype(np.float64))
+    pre = y0 / s  # the pre-gate value ys[t] + (sum D) x, pinned by p2-p8
+    ln = torch.nn.functional.layer_norm(torch.from_numpy(pre), (pre.shape[-1],),
+                                        torch.from_numpy(gamma.astype(np.float64)),
+                                        torch.from_numpy(beta.astype(np.float64)), eps).numpy()
+    np.testing.assert_allclose(y1, s * ln, rtol=1e-11, atol=1e-13)
+
+
+def test_p9_layernorm_standardises_each_token(oracle_mod):
+    rng = np.random.default_rng(960)
+    a, gamma, beta = _ln_case(rng, False, 0)
+    E = gamma.shape[0]
+    y = oracle_mod.forward(**a, ln_gamma=np.ones(E, np.float32), ln_beta=np.zeros(E, np.float32), ln_eps=0.0)
+    v = y / _silu(a["z"].astype(np.float64))
+    np.testing.assert_allclose(v.mean(axis=-1), 0.0, atol=1e-12)
+    np.testing.assert_allclose((v * v).mean(axis=-1), 1.0, rtol=1e-12)
+    # gamma scales and beta shifts the normalised value channel by channel
+    y2 = oracle_mod.forward(**a, ln_gamma=gamma, ln_beta=beta, ln_eps=0.0)
+    v2 = y2 / _silu(a["z"].astype(np.float64))
+    np.testing.assert_allclose(v2, gamma.astype(np.float64) * v + beta.astype(np.float64), rtol=1e-12, atol=1e-13)
+
+
+def test_p9_layernorm_arguments(oracle_mod):
+    rng = np.random.default_rng(970)
+    a, gamma, beta = _ln_case(rng, False, 1)
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.forward(**a, ln_gamma=gamma, ln_beta=None)
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.forward(**a, ln_gamma=gamma, ln_beta=beta, ln_eps=-1.0)
