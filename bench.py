@@ -52,7 +52,7 @@ def kernel_work(name: str, cfg, pool_axis: int):
     T = cfg.h if pool_axis == 0 else cfg.w
     if name in ("pool_dense_kernel", "mask_pool_kernel"):
         return "hbm", row * tok                       # read x
-    if name in ("epilogue_dense_kernel", "mask_epilogue_kernel", "fused_layer_kernel"):
+    if name in ("epilogue_dense_kernel", "mask_epilogue_kernel", "ln_epilogue_kernel", "fused_layer_kernel"):
         return "hbm", 3 * row * tok                   # read x and z, write y (the fused launch: the layer)
     if name == "scan_seq_kernel":
         return "alu", cfg.B * T * cfg.E * cfg.N * cfg.nd
@@ -77,6 +77,8 @@ def parse(argv=None):
                     help="override the batch (small cases for profiler captures; not a benchmark line)")
     ap.add_argument("--path", choices=["auto", "staged", "fused"], default="auto",
                     help="implementation of the layer (auto picks the fused launch for this workload)")
+    ap.add_argument("--ln", action="store_true",
+                    help="add the post-SSM LayerNorm before the gate (gamma = 1, beta = 0: the usual init)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -338,8 +340,11 @@ def run_ours(a, cfg, pool_axis):
 
     mine = workload.shard_images(cfg, rank, world)
     t = workload.layer_tensors(cfg, dev, first_image=mine.start)
+    if a.ln:
+        t.update(workload.ln_tensors(cfg, dev))
     keep = t.get("keep_idx")
-    shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, cfg.dir_flags, keep, cfg.h, cfg.w, path=a.path)
+    shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, cfg.dir_flags, keep, cfg.h, cfg.w, path=a.path,
+                            ln=a.ln)
     y = torch.empty_like(t["x"])
     ws = ssm.alloc_workspace(shape, dev)
     stream = torch.cuda.current_stream(dev)
@@ -429,6 +434,7 @@ def run_ours(a, cfg, pool_axis):
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic (seeded N(0,1) x, z; Mamba-style parameter init)",
         "config": dict(workload_desc(cfg, pool_axis),
+                       **({"post_ssm_layernorm": "gamma = 1, beta = 0, eps = 1e-5"} if a.ln else {}),
                        l2=(f"inputs {alg_bytes_call / 1e9:.2f} GB per step > 126 MB L2; no flush" if flush is None
                            else f"inputs {alg_bytes_call / 1e6:.1f} MB per step < 2 x L2: L2 flushed (256 MB write) "
                                 f"before every step, step time = span of the step's launches"),
@@ -452,6 +458,8 @@ def run_ours(a, cfg, pool_axis):
         del t, y
         torch.cuda.empty_cache()
         host = workload.layer_tensors(cfg, dev, pinned_host=True, first_image=mine.start)
+        if a.ln:
+            host.update({k: v.pin_memory() for k, v in workload.ln_tensors(cfg, "cpu").items()})
         run = ssm.HostForward(shape, dev)
         y_host = torch.empty(host["x"].shape, dtype=torch.float32).pin_memory()
         run(host, y_host)  # warm

@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define FASTVIM_SSM_ABI_VERSION 1
+#define FASTVIM_SSM_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define FV_API __attribute__((visibility("default")))
@@ -86,14 +86,15 @@ enum {
     FV_FLAG_PATH_STAGED = 2u, /* force the staged kernels (pool, proj, scan, epilogue launches)  */
     FV_FLAG_PATH_FUSED = 4u,  /* force the single persistent launch (dense layers only;
                                  FV_ERR_UNSUPPORTED when the layer does not fit it)             */
-    FV_FLAG_TRACE = 8u        /* fused launch: record one entry per task in the workspace
+    FV_FLAG_TRACE = 8u,       /* fused launch: record one entry per task in the workspace
                                  (fv_ws_layout.trace); costs a little time, for profiling      */
+    FV_FLAG_LAYERNORM = 16u   /* post-SSM LayerNorm before the gate (ln_gamma, ln_beta, ln_eps) */
 };
 /* Without a PATH flag a dense layer whose images hold >= 16 MiB of x runs the fused launch, every
- * other layer the staged kernels; both compute the same layer.  The fused launch keeps each
- * image's x in L2 between pooling and the epilogue; the environment variable FASTVIM_FUSED_LAG
- * (2..64, read per call) overrides how many images it lets lie between the two, and
- * FASTVIM_FUSED_LP (1..4) how many grid lines one streaming task covers (tuning only). */
+ * other layer the staged kernels; both compute the same layer.  The fused launch gates image b
+ * L rounds after it pools it; the environment variable FASTVIM_FUSED_LAG (3..64, read per call)
+ * overrides L, and FASTVIM_FUSED_LP (1..4) how many grid lines one streaming task covers (tuning
+ * only). */
 
 typedef struct {
     int B, h, w, E, N, R;    /* batch, grid height/width, channels, d_state, dt_rank        */
@@ -111,6 +112,17 @@ typedef struct {
     const float* b_dt;       /* [nd][E]                                                      */
     const int32_t* keep_idx; /* NULL (dense) or [B][K] grid ids r*w + c                      */
     float* y;                /* same shape as x; must not overlap x or z                     */
+    /* Post-SSM LayerNorm, with FV_FLAG_LAYERNORM (summary page, "方法详解" item 5: after the
+     * repeat and the skip; verdict page: VMamba's post-SSM LayerNorm), over the E channels of
+     * each token, before the gate:
+     *   y = SiLU(z) * (ln_gamma * (s - mean(s)) / sqrt(var(s) + ln_eps) + ln_beta),
+     *   s = ys[t] + (sum_k D[k]) * x,  var the biased variance over E.
+     * With the flag: ln_gamma and ln_beta [E] are required (FV_ERR_NULL), ln_eps must be > 0 and
+     * finite (FV_ERR_SHAPE), E <= 4096 (FV_ERR_UNSUPPORTED).  Without it both must be NULL
+     * (FV_ERR_SHAPE) and ln_eps is ignored. */
+    const float* ln_gamma;   /* NULL or [E]                                                  */
+    const float* ln_beta;    /* NULL or [E]                                                  */
+    float ln_eps;            /* LayerNorm epsilon (e.g. 1e-5)                                */
 } fv_ssm_args;
 
 /* Byte offsets of the intermediates inside a workspace (for inspection and tests). */
@@ -131,8 +143,8 @@ typedef struct {
                             w1 = SM id << 32 | CTA id, w2 = start (ns, %globaltimer),
                             w3 = wait_ns << 40 | total_ns (from start to the task's end)        */
     size_t trace_records;  /* number of trace entries (tasks of the call), else 0               */
-    size_t scan_bc;      /* fused launch only: B | C rows in scan order, else 0              */
-    size_t scan_dt;      /* fused launch only: dt_low rows, else 0                             */
+    size_t scan_bc;      /* reserved, 0                                                      */
+    size_t scan_dt;      /* reserved, 0                                                      */
     int T, S, nd;        /* pooled length, pooled-over length, number of directions          */
 } fv_ws_layout;
 

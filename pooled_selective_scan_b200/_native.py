@@ -27,6 +27,7 @@ FV_FLAG_ZOH_EXACT = 1
 FV_FLAG_PATH_STAGED = 2
 FV_FLAG_PATH_FUSED = 4
 FV_FLAG_TRACE = 8
+FV_FLAG_LAYERNORM = 16
 
 # Every exported symbol of the ABI, as the header declares it.
 EXPORTS = (
@@ -62,6 +63,7 @@ class FvSsmArgs(ctypes.Structure):
         ("W_dt", ctypes.c_void_p), ("b_dt", ctypes.c_void_p),
         ("keep_idx", ctypes.c_void_p),
         ("y", ctypes.c_void_p),
+        ("ln_gamma", ctypes.c_void_p), ("ln_beta", ctypes.c_void_p), ("ln_eps", ctypes.c_float),
     ]
 
 

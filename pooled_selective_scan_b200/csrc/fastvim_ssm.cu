@@ -29,6 +29,7 @@ size_t round256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 constexpr int kMaxT = 4096;
 constexpr long long kMaxMaskGrid = 1ll << 20;
+constexpr int kMaxLnE = 4096;  // channels of a LayerNorm row (shared-memory rows of the LN epilogue)
 
 size_t bucket_smem_bytes(const fv::Shape& sh) {
     const long long G = (long long)sh.h * sh.w;
@@ -41,7 +42,8 @@ fv_status make_shape(const fv_ssm_args* a, fv::Shape* sh) {
     if (a->B < 0 || a->h < 1 || a->w < 1 || a->E < 4 || a->N < 1 || a->R < 1) return FV_ERR_SHAPE;
     if (a->pool_axis != FV_POOL_W && a->pool_axis != FV_POOL_H) return FV_ERR_SHAPE;
     if (a->dir_flags == 0 || (a->dir_flags & ~3u) != 0) return FV_ERR_SHAPE;
-    if ((a->flags & ~(unsigned)(FV_FLAG_ZOH_EXACT | FV_FLAG_PATH_STAGED | FV_FLAG_PATH_FUSED | FV_FLAG_TRACE)) != 0)
+    if ((a->flags & ~(unsigned)(FV_FLAG_ZOH_EXACT | FV_FLAG_PATH_STAGED | FV_FLAG_PATH_FUSED | FV_FLAG_TRACE |
+                                FV_FLAG_LAYERNORM)) != 0)
         return FV_ERR_SHAPE;
     if ((a->flags & FV_FLAG_PATH_STAGED) && (a->flags & FV_FLAG_PATH_FUSED)) return FV_ERR_SHAPE;
     if (a->E % 4 != 0) return FV_ERR_SHAPE;
@@ -65,6 +67,10 @@ fv_status make_shape(const fv_ssm_args* a, fv::Shape* sh) {
     sh->trace = (a->flags & FV_FLAG_TRACE) ? 1 : 0;
     sh->pool_scale = a->pool_scale == 0.f ? 1.f : a->pool_scale;
     sh->SL = a->E / 4;
+    sh->ln = (a->flags & FV_FLAG_LAYERNORM) ? 1 : 0;
+    sh->ln_eps = sh->ln ? a->ln_eps : 0.f;
+    if (sh->ln && !(a->ln_eps > 0.f && a->ln_eps <= 3.0e38f)) return FV_ERR_SHAPE;
+    if (sh->ln && a->E > kMaxLnE) return FV_ERR_UNSUPPORTED;
     if (sh->T > kMaxT) return FV_ERR_UNSUPPORTED;
     if (a->K > 0 && (long long)a->h * a->w > kMaxMaskGrid) return FV_ERR_UNSUPPORTED;
     if ((long long)sh->B * sh->T >= (1ll << 31)) return FV_ERR_UNSUPPORTED;
@@ -76,7 +82,10 @@ fv_status check_pointers(const fv_ssm_args* a, const fv::Shape& sh) {
     if (sh.B > 0 && (!a->x || !a->z || !a->y)) return FV_ERR_NULL;
     if (sh.K > 0 && sh.B > 0 && !a->keep_idx) return FV_ERR_NULL;
     if (sh.K == 0 && a->keep_idx) return FV_ERR_SHAPE;  // a keep list needs K
-    const void* ps[] = {a->x, a->z, a->y, a->A_log, a->D, a->W_x, a->W_dt, a->b_dt, a->keep_idx};
+    if (sh.ln && (!a->ln_gamma || !a->ln_beta)) return FV_ERR_NULL;
+    if (!sh.ln && (a->ln_gamma || a->ln_beta)) return FV_ERR_SHAPE;  // LayerNorm weights need the flag
+    const void* ps[] = {a->x, a->z, a->y, a->A_log, a->D, a->W_x, a->W_dt, a->b_dt, a->keep_idx, a->ln_gamma,
+                        a->ln_beta};
     for (const void* p : ps)
         if (p && !aligned16(p)) return FV_ERR_ALIGN;
     if (sh.B > 0) {
@@ -101,11 +110,6 @@ fv_status plan_layout(const fv::Shape& sh, fv_ws_layout* L) {
     L->xbar = off; off = round256(off + (size_t)sh.B * sh.T * sh.E * sizeof(float));
     L->u = off; off = round256(off + (size_t)sh.nd * sh.B * fv::u_block_stride(sh.T, sh.J) * sizeof(float));
     L->ys = off; off = round256(off + (size_t)sh.B * sh.T * sh.E * sizeof(float));
-    if (choose_path(sh) == Path::Fused) {
-        // scan-ready copies of B | C (chunk-interleaved rows) and dt_low, written by the projections
-        L->scan_bc = off; off = round256(off + (size_t)sh.nd * sh.B * fv::fused_bcs_stride(sh.T) * sizeof(float));
-        L->scan_dt = off; off = round256(off + (size_t)sh.nd * sh.B * fv::fused_dts_stride(sh.T, sh.R) * sizeof(float));
-    }
     if (sh.K > 0) {
         L->row_of = off; off = round256(off + (size_t)sh.B * sh.K * sizeof(int32_t));
         L->row_off = off; off = round256(off + (size_t)sh.B * (sh.T + 1) * sizeof(int32_t));
@@ -127,8 +131,10 @@ fv_status plan_layout(const fv::Shape& sh, fv_ws_layout* L) {
 
 // The library is built for sm_100a only: 227 KB of opt-in shared memory per CTA.
 constexpr size_t kMaxSmemOptin = 227 * 1024;
-// Latency of one image's pool -> x_proj -> scan chain inside the fused launch (trace, B200).
-constexpr double kChainLatencyUs = 60.0;
+// Latency of one image's pool -> x_proj -> scan chain inside the fused launch: the scan task runs
+// the T steps of its recurrences in sequence (traces on B200: 55 us at T = 128, 36 us at T = 64),
+// the projection and the last pooling tasks add about 40 us.
+double chain_latency_us(const fv::Shape& sh) { return 40.0 + 0.5 * sh.T; }
 
 fv_status check_limits(const fv::Shape& sh) {
     if (fv::seq_smem_floats(sh) * sizeof(float) > kMaxSmemOptin) return FV_ERR_UNSUPPORTED;
@@ -183,15 +189,14 @@ fv::FusedPlan plan_fused(const fv::Shape& sh) {
     pl.nQ = (sh.T + fv::kQT - 1) / fv::kQT;
     pl.ECH = fv::fused_ech(sh.nd);
     pl.nS = (sh.E + pl.ECH - 1) / pl.ECH;
-    pl.CL = (sh.T + fv::kScanChunks - 1) / fv::kScanChunks;
     pl.ctP = fv::kStageBytes / (sh.E * (int)sizeof(float));
     pl.ctE = fv::kStageBytes / 2 / (sh.E * (int)sizeof(float));
-    // Lag: enough rounds to cover one image's pool -> proj -> scan chain (about 60 us measured on
-    // B200) at the rate one round streams (x twice, z and y once: 16 E bytes per grid token at
+    // Lag: enough rounds to cover one image's pool -> proj -> scan chain (chain_latency_us) at the
+    // rate one round streams (x twice, z and y once: 16 E bytes per grid token at
     // ~6.5 TB/s).  (Keeping x in L2 across that window does not happen: traffic of this size
     // evicts first-touch lines whatever their L2 eviction priority.)
     const double round_us = (double)sh.h * sh.w * sh.E * 16.0 / 6.5e6;
-    long long lag = (long long)(kChainLatencyUs / (round_us > 0.01 ? round_us : 0.01)) + 3;
+    long long lag = (long long)(chain_latency_us(sh) / (round_us > 0.01 ? round_us : 0.01)) + 3;
     if (const char* env = getenv("FASTVIM_FUSED_LAG")) {
         const long long v = atoll(env);
         if (v >= 3 && v <= 64) lag = v;
@@ -267,6 +272,7 @@ const char* launch_name_of(const fv::Shape& sh, int i) {
                                    "mask_epilogue_kernel"};
     if (i < 0 || i >= launch_count_of(sh)) return "";
     if (choose_path(sh) == Path::Fused) return "fused_layer_kernel";
+    if (sh.ln && i == launch_count_of(sh) - 1) return "ln_epilogue_kernel";
     return sh.K > 0 ? masked[i] : dense[i];
 }
 
@@ -294,11 +300,11 @@ fv::FusedPtrs fused_ptrs(const fv_ssm_args* a, const fv_ws_layout& L, char* ws) 
     fv::FusedPtrs p;
     p.x = a->x; p.z = a->z; p.A_log = a->A_log; p.D = a->D; p.W_x = a->W_x; p.W_dt = a->W_dt; p.b_dt = a->b_dt;
     p.y = a->y;
+    p.ln_gamma = a->ln_gamma;
+    p.ln_beta = a->ln_beta;
     p.xbar = (float*)(ws + L.xbar);
     p.u = (float*)(ws + L.u);
     p.ys = (float*)(ws + L.ys);
-    p.bcs = (float*)(ws + L.scan_bc);
-    p.dts = (float*)(ws + L.scan_dt);
     p.status = (unsigned*)(ws + L.status);
     p.ctrl = L.ctrl ? (unsigned*)(ws + L.ctrl) : nullptr;
     p.trace = L.trace_records ? (unsigned long long*)(ws + L.trace) : nullptr;
@@ -317,8 +323,6 @@ fv_status launch_proj_tasks(const fv::Shape& sh, const fv_ssm_args* a, const fv_
     const fv::FusedPlan pl = plan_fused(sh);
     fv::FusedPtrs p = fused_ptrs(a, L, ws);
     p.ctrl = nullptr;
-    p.bcs = nullptr;  // the staged scans read u directly
-    p.dts = nullptr;
     const size_t smem = fv::fused_proj_smem_floats(sh) * sizeof(float);
     cudaError_t e = ensure_smem(fv::proj_tasks_kernel, smem);
     if (e != cudaSuccess) { note_cuda(e, "proj smem attribute"); return FV_ERR_CUDA; }
@@ -407,7 +411,19 @@ fv_status forward_impl(const fv_ssm_args* a, void* ws_v, size_t ws_bytes, cudaSt
     FV_MARK(marks, st);
     if ((s = launch_scan_seq(sh, a, L, ws, st)) != FV_OK) return s;
     FV_MARK(marks, st);
-    if (sh.K == 0) {
+    if (sh.ln) {
+        const size_t smem = fv::ln_epilogue_smem_bytes(sh);
+        cudaError_t e = ensure_smem(fv::ln_epilogue_kernel, smem);
+        if (e != cudaSuccess) { note_cuda(e, "LayerNorm epilogue smem attribute"); return FV_ERR_CUDA; }
+        const long long ntok = (long long)sh.B * (sh.K > 0 ? (long long)sh.K : (long long)sh.h * sh.w);
+        const long long per = (long long)fv::kLnWarps * fv::kLnTokensPerWarp;
+        const long long grid = (ntok + per - 1) / per;
+        if (grid >= (1ll << 31)) return FV_ERR_UNSUPPORTED;
+        fv::ln_epilogue_kernel<<<(unsigned)grid, fv::kLnWarps * 32, smem, st>>>(
+            sh, a->x, a->z, (const float*)(ws + L.ys), a->D, a->ln_gamma, a->ln_beta,
+            sh.K > 0 ? (const int32_t*)(ws + L.row_of) : nullptr, a->y);
+        FV_LAUNCH_CHECK("ln_epilogue_kernel");
+    } else if (sh.K == 0) {
         fv::epilogue_dense_kernel<<<M, fv::kThreads, 0, st>>>(sh, a->x, a->z, (const float*)(ws + L.ys), a->D, a->y);
         FV_LAUNCH_CHECK("epilogue_dense_kernel");
     } else {
@@ -524,7 +540,8 @@ fv_status fastvim_ssm_forward_host(const fv_ssm_args* host, const fv_ssm_args* d
     if ((s = make_shape(dev, &shd)) != FV_OK) return s;
     if (host->B != dev->B || host->h != dev->h || host->w != dev->w || host->E != dev->E ||
         host->N != dev->N || host->R != dev->R || host->K != dev->K || host->pool_axis != dev->pool_axis ||
-        host->dir_flags != dev->dir_flags || host->flags != dev->flags || host->pool_scale != dev->pool_scale)
+        host->dir_flags != dev->dir_flags || host->flags != dev->flags || host->pool_scale != dev->pool_scale ||
+        ((host->flags & FV_FLAG_LAYERNORM) && host->ln_eps != dev->ln_eps))
         return FV_ERR_SHAPE;
     if ((s = check_pointers(host, sh)) != FV_OK) return s;
     if ((s = check_pointers(dev, shd)) != FV_OK) return s;
@@ -572,6 +589,8 @@ fv_status fastvim_ssm_forward_host(const fv_ssm_args* host, const fv_ssm_args* d
         {(void*)dev->W_dt, host->W_dt, nd * sh.E * sh.R * sizeof(float)},
         {(void*)dev->b_dt, host->b_dt, nd * sh.E * sizeof(float)},
         {(void*)dev->keep_idx, host->keep_idx, sh.K > 0 ? (size_t)sh.B * sh.K * sizeof(int32_t) : 0},
+        {(void*)dev->ln_gamma, host->ln_gamma, sh.ln ? (size_t)sh.E * sizeof(float) : 0},
+        {(void*)dev->ln_beta, host->ln_beta, sh.ln ? (size_t)sh.E * sizeof(float) : 0},
     };
     for (const Copy& c : params) {
         if (c.bytes == 0 || !c.dst) continue;

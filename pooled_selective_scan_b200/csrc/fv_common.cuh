@@ -27,6 +27,8 @@ struct Shape {
     int trace;            // FV_FLAG_TRACE: record one trace entry per fused task
     float pool_scale;
     int SL;            // float4 slots per token row: E / 4
+    int ln;            // FV_FLAG_LAYERNORM: post-SSM LayerNorm before the gate
+    float ln_eps;
 };
 
 // Projections u of (direction k, image b) are one block of T x J floats; blocks start every
@@ -189,6 +191,36 @@ __device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); 
 
 __device__ __forceinline__ void f4_add(float4& a, const float4& b) {
     a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+}
+
+// ---- post-SSM LayerNorm helpers (one warp per token row) ----
+__device__ __forceinline__ float4 f4_fma(const float4& a, const float4& b, const float4& c) {
+    return make_float4(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y), fmaf(a.z, b.z, c.z), fmaf(a.w, b.w, c.w));
+}
+// Adds the shifted first and second moments of v's four values to (m1, m2).
+__device__ __forceinline__ void ln_accum(const float4& v, float K, float& m1, float& m2) {
+    const float a = v.x - K, b = v.y - K, c = v.z - K, d = v.w - K;
+    m1 += (a + b) + (c + d);
+    m2 += (a * a + b * b) + (c * c + d * d);
+}
+// Warp totals of (m1, m2) -> mean and 1 / sqrt(var + eps).
+__device__ __forceinline__ void ln_stats(float m1, float m2, float K, float invE, float eps, float& mean,
+                                         float& rstd) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        m1 += __shfl_xor_sync(0xffffffffu, m1, o);
+        m2 += __shfl_xor_sync(0xffffffffu, m2, o);
+    }
+    const float d = m1 * invE;
+    mean = K + d;
+    rstd = rsqrtf(fmaxf(m2 * invE - d * d, 0.f) + eps);
+}
+__device__ __forceinline__ float4 ln_gate4(const float4& sv, const float4& zv, const float4& gv, const float4& bv,
+                                           float mean, float rstd) {
+    return make_float4(silu_fast(zv.x) * fmaf(gv.x, (sv.x - mean) * rstd, bv.x),
+                       silu_fast(zv.y) * fmaf(gv.y, (sv.y - mean) * rstd, bv.y),
+                       silu_fast(zv.z) * fmaf(gv.z, (sv.z - mean) * rstd, bv.z),
+                       silu_fast(zv.w) * fmaf(gv.w, (sv.w - mean) * rstd, bv.w));
 }
 
 // Record the first device-side error of a call; later ones keep the first code.

@@ -7,7 +7,7 @@
 //
 //   P(b, g)  pool LP grid lines of image b into pooled tokens     (TMA bulk-copy ring over x)
 //   Q(b, q)  x_proj of 16 pooled tokens of image b                (fp32 GEMM, cp.async pipeline)
-//   S(b, c)  dt_proj + softplus, ZOH and the forward/backward scans of a channel tile of image b
+//   S(b, c)  dt_proj + softplus, ZOH and the forward/backward scans of 128 channels of image b
 //   E(b, g)  repeat + D x skip + SiLU(z) gate for LP grid lines  (TMA ring over x and z; y stored)
 //
 // taken from a global ticket counter in the order  [Q_{r-1}][P_r][E_{r-L}][S_{r-2}]  for r = 0, 1,
@@ -25,26 +25,22 @@
 // the abort flag (which makes every other CTA stop taking work), lets its own copies in flight
 // land, and exits.
 //
-// The scan of one (direction, channel) is split into 8 time chunks held by 8 lanes.  Pass 1 runs
-// each chunk from a zero state, giving the chunk's affine map h -> P h + H (P = product of the
-// Abar, taken as one exp2 of the summed step sizes); a 3-step shuffle scan over the 8 lanes
-// composes the maps in scan order; pass 2 reruns each chunk from its true incoming state and
-// emits C_t . h_t.  All 16 states of a lane stay in registers; the sequential depth is ~2 T/8 + 3
-// instead of T.
+// An S task runs one recurrence per thread over the whole pooled sequence (fv_scan.cuh): 256
+// threads = 128 channels x 2 directions.  The image's P tasks zero its scan output, so both
+// directions add into it.
 #pragma once
 
 #include "fv_common.cuh"
+#include "fv_scan.cuh"
 
 namespace fv {
 
 constexpr int kFusedThreads = 256;       // two persistent CTAs per SM
-constexpr int kScanChunks = 8;           // time chunks (lanes) per (direction, channel)
-constexpr int kScanStates = 16;          // states per lane (N <= 16, unused ones are zero)
-constexpr int kBCStride = 2 * kScanStates + 4;  // floats per token row of B|C in shared memory
 constexpr int kMaxLP = 4;                // grid lines per P/E task at most
 constexpr int kRingStages = 4;           // TMA bulk-copy ring of the streaming tasks
 constexpr int kStageBytes = 24 * 1024;   // per stage: P tasks x only; E tasks x and z halves
 constexpr int kMaxSlots = 2;             // float4 slots per thread in P tasks: E <= 2048
+constexpr int kLnCache = 3;              // LayerNorm: float4 slots of s a lane keeps in registers
 constexpr int kQT = 16;                  // pooled tokens per projection task
 constexpr int kQK = 32;                  // channels per projection K-step
 constexpr int kQPad = kQK + 4;           // padded row of a projection tile (16-byte aligned)
@@ -65,8 +61,7 @@ struct FusedPlan {
     int nP;      // P tasks (and E tasks) per image
     int nQ;      // Q tasks per image
     int nS;      // S tasks per image
-    int ECH;     // channels per S task
-    int CL;      // time steps per scan chunk: ceil(T / 8)
+    int ECH;     // channels per S task (and direction)
     int L;       // E of image r - L is issued in round r
     int B;
     int ctP;     // tokens per ring chunk in P tasks
@@ -87,11 +82,11 @@ struct FusedPtrs {
     const float* W_dt;
     const float* b_dt;
     float* y;
+    const float* ln_gamma;  // [E] (FV_FLAG_LAYERNORM) or NULL
+    const float* ln_beta;
     float* xbar;   // [B][T][E]
     float* u;      // [nd][B] blocks of [T][J] (see u_offset)
     float* ys;     // [B][T][E]
-    float* bcs;    // [nd][B][8 CL][kBCStride]: B | C rows in the scan's chunk-interleaved order
-    float* dts;    // [nd][B][Tr]: dt_low rows [T][R], block padded to Tr = ceil(T R / 32) * 32
     unsigned* status;
     unsigned* ctrl;
     unsigned long long* trace;  // NULL, or 4 words per ticket
@@ -104,13 +99,8 @@ struct Ring {
     unsigned count;            // chunks issued (and consumed) by this CTA so far
 };
 
-__host__ __device__ __forceinline__ int fused_ech(int nd) { return kFusedThreads / (kScanChunks * nd); }
-// Per-(direction, image) block strides of the scan-ready copies, in floats.
-__host__ __device__ __forceinline__ size_t fused_bcs_stride(int T) {
-    return (size_t)kScanChunks * ((T + kScanChunks - 1) / kScanChunks) * kBCStride;
-}
-__host__ __device__ __forceinline__ size_t fused_dts_stride(int T, int R) { return (((size_t)T * R + 31) / 32) * 32; }
-__host__ __device__ __forceinline__ int fused_xstride(int nd) { return fused_ech(nd) + 4; }
+// Channels per S task: 256 threads cover 128 channels x 2 directions, or 256 channels x 1.
+__host__ __device__ __forceinline__ int fused_ech(int nd) { return kFusedThreads / nd; }
 
 // Dynamic shared memory (floats) per task kind; the fused launch takes the maximum.
 __host__ __device__ __forceinline__ size_t fused_proj_smem_floats(const Shape& sh) {
@@ -118,17 +108,12 @@ __host__ __device__ __forceinline__ size_t fused_proj_smem_floats(const Shape& s
     return (size_t)q_stages(tn) * ((size_t)kQT * kQPad + (size_t)32 * tn * kQPad);
 }
 __host__ __device__ __forceinline__ size_t fused_scan_smem_floats(const Shape& sh) {
-    const int CL = (sh.T + kScanChunks - 1) / kScanChunks;
-    const size_t rows = (size_t)kScanChunks * CL;
-    const int XS = fused_xstride(sh.nd);
-    return (size_t)sh.nd * rows * kBCStride + (size_t)(sh.nd + 1) * rows * XS +
-           (size_t)sh.nd * fused_dts_stride(sh.T, sh.R) + (size_t)sh.nd * fused_ech(sh.nd) * (sh.R + 1) +
-           (size_t)sh.T;
+    return seq_smem_floats(kFusedThreads, sh.nd, sh.R);
 }
 __host__ __device__ __forceinline__ size_t fused_smem_floats(const Shape& sh, int LP) {
     const size_t ring = (size_t)kRingStages * kStageBytes / 4;
     const size_t pool = ring + (size_t)kFusedThreads * 4;
-    const size_t gate = ring + (size_t)(LP + 1) * sh.E;
+    const size_t gate = ring + (size_t)(LP + 1 + (sh.ln ? 2 : 0)) * sh.E;
     const size_t proj = fused_proj_smem_floats(sh);
     const size_t scan = fused_scan_smem_floats(sh);
     size_t m = pool > gate ? pool : gate;
@@ -363,6 +348,9 @@ __device__ __forceinline__ bool fused_pool(const Shape& sh, const FusedPlan& pl,
                 for (int j = sm.g; j < n; j += sm.G) f4_add(acc[k], chunk[(size_t)j * SL + sm.slot[k]]);
         if (i == nch - 1) {
             float4* out = reinterpret_cast<float4*>(p.xbar + (m0 + q / nch) * E);
+            // the image's scan output starts at zero: both directions add into it
+            float4* yz = reinterpret_cast<float4*>(p.ys + (m0 + q / nch) * E);
+            const bool zero_ys = sh.nd == 2;
             if (SL <= kFusedThreads) {
                 part[threadIdx.x] = acc[0];
                 __syncthreads();
@@ -370,11 +358,15 @@ __device__ __forceinline__ bool fused_pool(const Shape& sh, const FusedPlan& pl,
                     float4 sum = part[threadIdx.x];
                     for (int qq = 1; qq < sm.G; ++qq) f4_add(sum, part[qq * SL + threadIdx.x]);
                     out[threadIdx.x] = f4_mul(sum, scale);
+                    if (zero_ys) yz[threadIdx.x] = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             } else {
 #pragma unroll
                 for (int k = 0; k < kMaxSlots; ++k)
-                    if (k < sm.nslot) out[sm.slot[k]] = f4_mul(acc[k], scale);
+                    if (k < sm.nslot) {
+                        out[sm.slot[k]] = f4_mul(acc[k], scale);
+                        if (zero_ys) yz[sm.slot[k]] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
             }
         }
         __syncthreads();  // everyone is done with stage st
@@ -457,36 +449,15 @@ __device__ __forceinline__ void fused_proj_t(const Shape& sh, const FusedPlan& p
         }
     }
     cp_async_wait<0>();
-    const int CL = pl.CL;
-    const size_t bstride = fused_bcs_stride(T), dstride = fused_dts_stride(T, R);
 #pragma unroll
     for (int j = 0; j < TN; ++j) {
         const int jj = cg + 32 * j;
         if (jj < NJ) {
             const int k = jj / J, jc = jj - k * J;
-            float* bcb = p.bcs + ((size_t)k * sh.B + b) * bstride;
-            float* dtb = p.dts + ((size_t)k * sh.B + b) * dstride;
 #pragma unroll
             for (int i = 0; i < TM; ++i) {
                 const int r = tg + 8 * i;
-                if (r < mt) {
-                    const int t = tq0 + r;
-                    const float v = acc[i][j];
-                    p.u[u_offset(sh, k, b, t) + jc] = v;
-                    if (!p.bcs) continue;  // staged launches scan from u alone
-                    if (jc < R) {
-                        dtb[(size_t)t * R + jc] = v;
-                    } else {
-                        const int nb = jc - R;
-                        float* row = bcb + (size_t)((t % CL) * kScanChunks + t / CL) * kBCStride;
-                        row[nb < N ? nb : kScanStates + (nb - N)] = v;
-                        if (nb == 0)  // unused state slots of this token read as zero
-                            for (int n = N; n < kScanStates; ++n) {
-                                row[n] = 0.f;
-                                row[kScanStates + n] = 0.f;
-                            }
-                    }
-                }
+                if (r < mt) p.u[u_offset(sh, k, b, tq0 + r) + jc] = acc[i][j];
             }
         }
     }
@@ -502,197 +473,13 @@ __device__ __forceinline__ void fused_proj(const Shape& sh, const FusedPlan& pl,
     }
 }
 
-// ---- S: dt_proj + softplus, ZOH and scans of channels [e0, e0 + ECH) of image b -----------------
-// Shared rows are stored in chunk-interleaved time order p(t) = (t % CL) * 8 + t / CL, so that at
-// any step the 8 chunk lanes read 8 consecutive rows (bank-conflict free with the paddings).
+// ---- S: dt_proj + softplus, ZOH and both scans of channels [e0, e0 + ECH) of image b -------------
+// 256 threads = ECH channels x ND directions, one recurrence each (fv_scan.cuh).  ys of image b
+// was zeroed by the image's P tasks when both directions add into it.
 template <int ND, bool ZOH_EXACT>
 __device__ __forceinline__ void fused_scan(const Shape& sh, const FusedPlan& pl, const FusedPtrs& p, int b, int tile,
                                            float* smem) {
-    constexpr int ECH = kFusedThreads / (kScanChunks * ND);
-    constexpr int XS = ECH + 4;
-    constexpr int NS = kScanStates;
-    const int T = sh.T, E = sh.E, N = sh.N, R = sh.R;
-    const int CL = pl.CL;
-    const int rows = kScanChunks * CL;
-    const int e0 = tile * ECH;
-    float* bc = smem;                          // [ND][rows][kBCStride]: B_0..B_15 | C_0..C_15
-    float* dx = bc + ND * rows * kBCStride;    // [ND][rows][XS]: Delta, then y of that direction
-    float* xsm = dx + ND * rows * XS;          // [rows][XS]: pooled tokens
-    const int DTS = (int)fused_dts_stride(T, R);
-    float* dtl = xsm + rows * XS;              // [ND][DTS]: dt_low rows [T][R]
-    float* wdt = dtl + ND * DTS;               // [ND][ECH][R+1]: dt_proj rows (+ bias)
-    int* post = reinterpret_cast<int*>(wdt + ND * ECH * (R + 1));  // [T]: p(t)
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    constexpr int kWarps = kFusedThreads / 32;
-    // Stage the tile's inputs with 16-byte asynchronous copies (all in flight together): the
-    // scan-ready B | C rows and dt_low rows written by the projection tasks, the pooled tokens of
-    // the tile's channels; and the tile's dt_proj rows and biases.
-    {
-        const int nbc = rows * kBCStride / 4, ndt = DTS / 4;
-        for (int k = 0; k < ND; ++k) {
-            const float* sb = p.bcs + ((size_t)k * sh.B + b) * fused_bcs_stride(T);
-            const float* sd = p.dts + ((size_t)k * sh.B + b) * DTS;
-            for (int v = threadIdx.x; v < nbc; v += kFusedThreads) cp_async16(bc + k * rows * kBCStride + 4 * v, sb + 4 * v, 16u);
-            for (int v = threadIdx.x; v < ndt; v += kFusedThreads) cp_async16(dtl + k * DTS + 4 * v, sd + 4 * v, 16u);
-        }
-        for (int t = threadIdx.x; t < T; t += kFusedThreads) post[t] = (t % CL) * kScanChunks + t / CL;
-        __syncthreads();
-        for (int v = threadIdx.x; v < T * (ECH / 4); v += kFusedThreads) {
-            const int t = v / (ECH / 4), c4 = (v % (ECH / 4)) * 4;
-            const bool ok = e0 + c4 < E;
-            cp_async16(xsm + post[t] * XS + c4, ok ? (const void*)(p.xbar + ((size_t)b * T + t) * E + e0 + c4)
-                                                   : (const void*)p.xbar, ok ? 16u : 0u);
-        }
-        cp_async_commit();
-        for (int i = threadIdx.x; i < ND * ECH * (R + 1); i += kFusedThreads) {
-            const int k = i / (ECH * (R + 1));
-            const int rem = i - k * ECH * (R + 1);
-            const int c = rem / (R + 1), r = rem - c * (R + 1);
-            const int e = e0 + c;
-            float v = 0.f;
-            if (e < E) v = r < R ? __ldg(p.W_dt + ((size_t)k * E + e) * R + r) : __ldg(p.b_dt + (size_t)k * E + e);
-            wdt[i] = v;
-        }
-        cp_async_wait<0>();
-        __syncthreads();
-    }
-    // Delta = softplus(W_dt . dt_low + b_dt) for this tile: lane -> channel, warps -> tokens
-    {
-        constexpr int kTPerWarpPass = 32 / ECH > 0 ? 32 / ECH : 1;
-        const int c = lane % ECH;
-        const int tsub = lane / ECH;
-        const bool live = e0 + c < E;
-        for (int k = 0; k < ND; ++k) {
-            const float* wr = wdt + (k * ECH + c) * (R + 1);
-            for (int t = warp * kTPerWarpPass + tsub; t < T; t += kWarps * kTPerWarpPass) {
-                const float* dl = dtl + k * DTS + t * R;
-                float a = wr[R];
-#pragma unroll 4
-                for (int r = 0; r < R; ++r) a = fmaf(wr[r], dl[r], a);
-                dx[(k * rows + post[t]) * XS + c] = live ? softplus_fast(a) : 0.f;
-            }
-        }
-    }
-    __syncthreads();
-
-    const int chunk = lane & 7;
-    constexpr int kWarpsPerDir = ECH / 4;
-    const int kd = warp / kWarpsPerDir;
-    const int ch = (warp - kd * kWarpsPerDir) * 4 + (lane >> 3);
-    const int e = e0 + ch;
-    const bool active = e < E;
-    const bool fwd = (ND == 2) ? (kd == 0) : ((sh.dir_flags & 1u) != 0);
-    constexpr float kLog2e = 1.4426950408889634f;
-    float A2[NS], h[NS];
-    float An[NS], Ainv[NS];  // used by the exact-ZOH input term only
-#pragma unroll
-    for (int n = 0; n < NS; ++n) {
-        const float A = (active && n < N) ? -expf(__ldg(p.A_log + ((size_t)kd * E + e) * N + n)) : 0.f;
-        A2[n] = A * kLog2e;
-        An[n] = A;
-        Ainv[n] = A != 0.f ? 1.f / A : 0.f;
-        h[n] = 0.f;
-    }
-    const int c_lo = chunk * CL;
-    const int c_hi = min(T, c_lo + CL);
-    const int len = c_hi > c_lo ? c_hi - c_lo : 0;
-    const float* bck = bc + kd * rows * kBCStride;
-    float* dxk = dx + kd * rows * XS;
-
-    // pass 1: this chunk from a zero state
-    float sdt = 0.f;
-    for (int s = 0; s < len; ++s) {
-        const int t = fwd ? c_lo + s : c_hi - 1 - s;
-        const int pos = (t - c_lo) * kScanChunks + chunk;
-        const float dt = dxk[pos * XS + ch];
-        const float xv = xsm[pos * XS + ch];
-        const float dtx = dt * xv;
-        sdt += dt;
-        const float4* Bq = reinterpret_cast<const float4*>(bck + pos * kBCStride);
-#pragma unroll
-        for (int q = 0; q < NS / 4; ++q) {
-            const float4 bv = Bq[q];
-            const float bb[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int n = 4 * q + i;
-                const float dA = ex2_approx(dt * A2[n]);
-                const float bx = ZOH_EXACT ? expm1f(dt * An[n]) * Ainv[n] * bb[i] * xv : dtx * bb[i];
-                h[n] = fmaf(dA, h[n], bx);
-            }
-        }
-    }
-    // compose the chunk maps h -> P h + H along the scan order (lanes 0..7 forward, 7..0 backward;
-    // the direction is uniform within a warp)
-    if (fwd) {
-#pragma unroll
-        for (int n = 0; n < NS; ++n) {
-            float P = ex2_approx(A2[n] * sdt), H = h[n];
-#pragma unroll
-            for (int d = 1; d < kScanChunks; d <<= 1) {
-                const float Pp = __shfl_up_sync(0xffffffffu, P, d, kScanChunks);
-                const float Hp = __shfl_up_sync(0xffffffffu, H, d, kScanChunks);
-                if (chunk >= d) {
-                    H = fmaf(P, Hp, H);
-                    P = P * Pp;
-                }
-            }
-            const float Hin = __shfl_up_sync(0xffffffffu, H, 1, kScanChunks);
-            h[n] = chunk == 0 ? 0.f : Hin;
-        }
-    } else {
-#pragma unroll
-        for (int n = 0; n < NS; ++n) {
-            float P = ex2_approx(A2[n] * sdt), H = h[n];
-#pragma unroll
-            for (int d = 1; d < kScanChunks; d <<= 1) {
-                const float Pp = __shfl_down_sync(0xffffffffu, P, d, kScanChunks);
-                const float Hp = __shfl_down_sync(0xffffffffu, H, d, kScanChunks);
-                if (chunk + d < kScanChunks) {
-                    H = fmaf(P, Hp, H);
-                    P = P * Pp;
-                }
-            }
-            const float Hin = __shfl_down_sync(0xffffffffu, H, 1, kScanChunks);
-            h[n] = chunk == kScanChunks - 1 ? 0.f : Hin;
-        }
-    }
-    // pass 2: rerun the chunk from its incoming state and emit C_t . h_t
-    for (int s = 0; s < len; ++s) {
-        const int t = fwd ? c_lo + s : c_hi - 1 - s;
-        const int pos = (t - c_lo) * kScanChunks + chunk;
-        const float dt = dxk[pos * XS + ch];
-        const float xv = xsm[pos * XS + ch];
-        const float dtx = dt * xv;
-        const float4* Bq = reinterpret_cast<const float4*>(bck + pos * kBCStride);
-        const float4* Cq = Bq + NS / 4;
-        float y = 0.f;
-#pragma unroll
-        for (int q = 0; q < NS / 4; ++q) {
-            const float4 bv = Bq[q], cv = Cq[q];
-            const float bb[4] = {bv.x, bv.y, bv.z, bv.w};
-            const float cc[4] = {cv.x, cv.y, cv.z, cv.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int n = 4 * q + i;
-                const float dA = ex2_approx(dt * A2[n]);
-                const float bx = ZOH_EXACT ? expm1f(dt * An[n]) * Ainv[n] * bb[i] * xv : dtx * bb[i];
-                h[n] = fmaf(dA, h[n], bx);
-                y = fmaf(cc[i], h[n], y);
-            }
-        }
-        dxk[pos * XS + ch] = y;  // the slot held this step's Delta, read above by this lane only
-    }
-    __syncthreads();
-    for (int t = warp; t < T; t += kWarps) {
-        const int pos = post[t];
-        for (int c = lane; c < ECH; c += 32) {
-            const int ee = e0 + c;
-            float sum = dx[pos * XS + c];
-            if (ND == 2) sum += dx[(rows + pos) * XS + c];
-            if (ee < E) p.ys[((size_t)b * T + t) * E + ee] = sum;
-        }
-    }
+    seq_scan<kFusedThreads, ND, ZOH_EXACT>(sh, p.u, p.xbar, p.A_log, p.W_dt, p.b_dt, p.ys, b, tile * pl.ECH, 0, smem);
     cta_signal(p.ctrl ? p.ctrl + kCtrlHeaderWords + 2 * sh.B + b : nullptr);
 }
 
@@ -728,6 +515,13 @@ __device__ __forceinline__ bool fused_gate(const Shape& sh, const FusedPlan& pl,
         const int l = i / E, e = i - l * E;
         ysl[i] = __ldcg(p.ys + ((size_t)b * sh.T + t0 + l) * E + e);
     }
+    float* gam = ysl + (size_t)pl.LP * E;  // [E], [E]: LayerNorm gamma, beta
+    float* bet = gam + E;
+    if (sh.ln)
+        for (int e = threadIdx.x; e < E; e += kFusedThreads) {
+            gam[e] = __ldg(p.ln_gamma + e);
+            bet[e] = __ldg(p.ln_beta + e);
+        }
     const float inv_sl = 1.f / (float)SL;
     for (int q = 0; q < nq; ++q) {
         const unsigned gg = g0 + q;
@@ -744,6 +538,43 @@ __device__ __forceinline__ bool fused_gate(const Shape& sh, const FusedPlan& pl,
         const float4* ys4 = reinterpret_cast<const float4*>(ysl + (size_t)l * E);
         const float4* d4 = reinterpret_cast<const float4*>(dsum);
         float4* y4 = reinterpret_cast<float4*>(p.y + dense_base(sh, b, t0 + l));
+        if (sh.ln) {
+            // post-SSM LayerNorm: one warp per token of the stage; s = ys + (sum D) x is kept in
+            // registers for the first kLnCache slots of each lane and recomputed from the stage
+            // beyond; mean and variance from one warp reduction of sums about the shift K = s[0]
+            const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+            const float4* g4 = reinterpret_cast<const float4*>(gam);
+            const float4* b4 = reinterpret_cast<const float4*>(bet);
+            const float invE = 1.f / (float)E;
+            for (int j = warp; j < n; j += kFusedThreads / 32) {
+                const float4* xr = xc + (size_t)j * SL;
+                const float4* zr = zc + (size_t)j * SL;
+                const float K = fmaf(dsum[0], xr[0].x, ysl[(size_t)l * E]);
+                float4 sc[kLnCache];
+                float m1 = 0.f, m2 = 0.f;
+#pragma unroll
+                for (int u = 0; u < kLnCache; ++u) {
+                    const int slot = lane + 32 * u;
+                    if (slot < SL) {
+                        sc[u] = f4_fma(d4[slot], xr[slot], ys4[slot]);
+                        ln_accum(sc[u], K, m1, m2);
+                    }
+                }
+                for (int slot = lane + 32 * kLnCache; slot < SL; slot += 32)
+                    ln_accum(f4_fma(d4[slot], xr[slot], ys4[slot]), K, m1, m2);
+                float mean, rstd;
+                ln_stats(m1, m2, K, invE, sh.ln_eps, mean, rstd);
+                float4* yrow = y4 + (size_t)(tok0 + j) * stride4;
+#pragma unroll
+                for (int u = 0; u < kLnCache; ++u) {
+                    const int slot = lane + 32 * u;
+                    if (slot < SL) st_hint(yrow + slot, ln_gate4(sc[u], zr[slot], g4[slot], b4[slot], mean, rstd), pol_stream);
+                }
+                for (int slot = lane + 32 * kLnCache; slot < SL; slot += 32)
+                    st_hint(yrow + slot, ln_gate4(f4_fma(d4[slot], xr[slot], ys4[slot]), zr[slot], g4[slot], b4[slot],
+                                                  mean, rstd), pol_stream);
+            }
+        } else
         for (int f = threadIdx.x; f < n * SL; f += kFusedThreads) {
             const int j = (int)(((float)f + 0.5f) * inv_sl);  // f / SL (exact for f < 2^16)
             const int slot = f - j * SL;

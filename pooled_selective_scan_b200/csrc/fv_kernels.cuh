@@ -9,6 +9,7 @@
 #pragma once
 
 #include "fv_common.cuh"
+#include "fv_scan.cuh"
 
 namespace fv {
 
@@ -276,200 +277,108 @@ mask_epilogue_kernel(Shape sh, const float* __restrict__ x, const float* __restr
     }
 }
 
-// ---- Staged scans: one thread per (image, channel, direction), all T steps in order -------------
-// The staged launches have every projection in HBM before the scans start, and 10^4 - 10^5
-// independent (image, channel, direction) recurrences, so each thread runs one recurrence
-// sequentially over the whole pooled sequence: one exp2 per state and step (no second pass).
-// The per-step inputs shared by a CTA's 128 channels (B, C and dt_low of the image and direction)
-// and the CTA's pooled tokens stream through shared memory in chunks of 16 steps, double-buffered
-// with cp.async.  A backward chunk is staged in reverse, so slot i is always the i-th step taken
-// and every shared-memory offset in the loops is a constant.  dt_proj for a chunk is computed up
-// front per thread (dt_low staged transposed, W_dt rows in shared memory), so the sequential loop
-// holds only the state update.  With both directions enabled each adds its output into ys, zeroed
-// beforehand: two float additions into +0 give the same sum in either order.
-constexpr int kSeqThreads = 128;   // channels per CTA
-constexpr int kSeqChunk = 16;      // steps per staged chunk
-constexpr int kSeqStates = 16;     // states per thread (N <= 16; unused ones stay zero)
+// ---- Staged epilogue with the post-SSM LayerNorm (dense and masked) ------------------------------
+// s = ys[t] + (sum_k D[k]) x;  y = SiLU(z) * (gamma * (s - mean) * rsqrt(var + eps) + beta), mean and
+// (biased) variance over the E channels of the token (summary page, "方法详解" item 5: repeat,
+// skip, LayerNorm; VMamba's post-SSM LayerNorm sits before the gate).  One warp per token: x and z
+// are streamed once (loads batched kLnBatch slots per lane) into shared-memory rows; the mean and
+// variance come from one warp reduction of sums about a shift K (the token's first s value), which
+// keeps var = E[(s-K)^2] - E[s-K]^2 free of cancellation when |mean| >> std.
+constexpr int kLnWarps = 4;
+constexpr int kLnTokensPerWarp = 4;
+constexpr int kLnBatch = 4;
 
-__host__ __device__ __forceinline__ int seq_r4(int R) { return (R + 3) & ~3; }
-// Row stride (floats) of the per-thread W_dt rows: a multiple of 4 whose quarter is odd, so the
-// 8 lanes of a 128-bit shared load hit 8 distinct bank quads.
-__host__ __device__ __forceinline__ int seq_wstride(int R) {
-    const int r4 = seq_r4(R);
-    return ((r4 / 4) & 1) ? r4 + 8 : r4 + 4;
-}
-__host__ __device__ __forceinline__ size_t seq_smem_floats(const Shape& sh) {
-    const int r4 = seq_r4(sh.R);
-    return (size_t)kSeqThreads * seq_wstride(sh.R)              // W_dt rows [128][WS]
-           + 2 * (size_t)kSeqChunk * 2 * kSeqStates             // B | C rows [2][16][32]
-           + 2 * (size_t)r4 * kSeqChunk                         // dt_low, transposed [2][R4][16]
-           + 2 * (size_t)kSeqChunk * kSeqThreads;               // pooled tokens [2][16][128]
+__host__ __forceinline__ size_t ln_epilogue_smem_bytes(const Shape& sh) {
+    return (size_t)(3 + 2 * kLnWarps) * sh.SL * sizeof(float4);  // sum D, gamma, beta; per warp s and z rows
 }
 
-struct SeqSmem {
-    float* w;    // [128][WS]
-    float* bc;   // [2][16][32]
-    float* dtT;  // [2][R4][16]
-    float* xs;   // [2][16][128]
-};
-
-// dt_proj + softplus and the recurrence over one staged chunk of `len` steps (LEN = 16 for a full
-// chunk, 0 for a shorter one).  Slot i holds the i-th step taken; y of slot i goes to yp + i * ystep.
-template <int LEN, bool ZOH_EXACT>
-__device__ __forceinline__ void seq_chunk(const float* __restrict__ bc, const float* __restrict__ dtT,
-                                          const float* __restrict__ xs, const float* __restrict__ wrow, int R4,
-                                          float bias, int len, const float (&A2)[kSeqStates],
-                                          const float (&An)[kSeqStates], const float (&Ainv)[kSeqStates],
-                                          float (&h)[kSeqStates], float* yp, ptrdiff_t ystep, bool live, bool add) {
-    constexpr int NS = kSeqStates;
-    const int n_steps = LEN ? LEN : len;
-    float dl[kSeqChunk];
-#pragma unroll
-    for (int i = 0; i < kSeqChunk; ++i) dl[i] = bias;
-    for (int r4 = 0; r4 < R4; r4 += 4) {
-        const float4 w = *reinterpret_cast<const float4*>(wrow + r4);
-        const float wq[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float4* d4 = reinterpret_cast<const float4*>(dtT + (r4 + q) * kSeqChunk);
-#pragma unroll
-            for (int i4 = 0; i4 < kSeqChunk / 4; ++i4) {
-                const float4 d = d4[i4];
-                dl[4 * i4 + 0] = fmaf(wq[q], d.x, dl[4 * i4 + 0]);
-                dl[4 * i4 + 1] = fmaf(wq[q], d.y, dl[4 * i4 + 1]);
-                dl[4 * i4 + 2] = fmaf(wq[q], d.z, dl[4 * i4 + 2]);
-                dl[4 * i4 + 3] = fmaf(wq[q], d.w, dl[4 * i4 + 3]);
-            }
-        }
+__global__ void __launch_bounds__(kLnWarps * 32)
+ln_epilogue_kernel(Shape sh, const float* __restrict__ x, const float* __restrict__ z,
+                   const float* __restrict__ ys, const float* __restrict__ D, const float* __restrict__ gamma,
+                   const float* __restrict__ beta, const int32_t* __restrict__ row_of, float* __restrict__ y) {
+    extern __shared__ float4 lsm[];
+    const int SL = sh.SL;
+    float4* dsum = lsm;
+    float4* g4 = dsum + SL;
+    float4* b4 = g4 + SL;
+    for (int slot = threadIdx.x; slot < SL; slot += kLnWarps * 32) {
+        dsum[slot] = dsum4(D, sh.nd, SL, slot);
+        g4[slot] = __ldg(reinterpret_cast<const float4*>(gamma) + slot);
+        b4[slot] = __ldg(reinterpret_cast<const float4*>(beta) + slot);
     }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float4* srow = b4 + SL + (size_t)warp * 2 * SL;
+    float4* zrow = srow + SL;
+    const long long per_img = sh.K > 0 ? (long long)sh.K : (long long)sh.h * sh.w;
+    const long long ntok = (long long)sh.B * per_img;
+    const long long tok0 = ((long long)blockIdx.x * kLnWarps + warp) * kLnTokensPerWarp;
+    const float invE = 1.f / (float)sh.E;
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    const float4* z4 = reinterpret_cast<const float4*>(z);
+    float4* y4 = reinterpret_cast<float4*>(y);
+    for (int q = 0; q < kLnTokensPerWarp; ++q) {
+        const long long tok = tok0 + q;
+        if (tok >= ntok) break;
+        const int b = (int)(tok / per_img);
+        const long long r = tok - (long long)b * per_img;
+        int t;
+        if (sh.K > 0) {
+            t = row_of[tok];  // < 0: a rejected id, output 0
+        } else {
+            const int i = (int)(r / sh.w), j = (int)(r - (long long)i * sh.w);
+            t = sh.pool_axis == 0 ? i : j;
+        }
+        const size_t o = (size_t)tok * SL;
+        if (t < 0) {
+            for (int slot = lane; slot < SL; slot += 32) st_stream(y4 + o + slot, make_float4(0.f, 0.f, 0.f, 0.f));
+            continue;
+        }
+        const float4* ys4 = reinterpret_cast<const float4*>(ys + ((size_t)b * sh.T + t) * sh.E);
+        // shift: the token's first s value (the same value in every lane)
+        const float K = fmaf(dsum[0].x, __ldcg(x + o * 4), __ldcg(ys + ((size_t)b * sh.T + t) * sh.E));
+        float m1 = 0.f, m2 = 0.f;
+        for (int base = lane; base < SL; base += 32 * kLnBatch) {
+            float4 xv[kLnBatch], zv[kLnBatch], yv[kLnBatch];
 #pragma unroll
-    for (int i = 0; i < kSeqChunk; ++i) {
-        if (LEN || i < n_steps) {
-            const float dt = softplus_fast(dl[i]);
-            const float xv = xs[i * kSeqThreads];
-            const float dtx = dt * xv;
-            const float4* Bq = reinterpret_cast<const float4*>(bc + i * 2 * NS);
-            const float4* Cq = Bq + NS / 4;
-            float y = 0.f;
-#pragma unroll
-            for (int q = 0; q < NS / 4; ++q) {
-                const float4 bv = Bq[q], cv = Cq[q];
-                const float bb[4] = {bv.x, bv.y, bv.z, bv.w};
-                const float cc[4] = {cv.x, cv.y, cv.z, cv.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int n = 4 * q + j;
-                    const float dA = ex2_approx(dt * A2[n]);
-                    const float bx = ZOH_EXACT ? expm1f(dt * An[n]) * Ainv[n] * bb[j] * xv : dtx * bb[j];
-                    h[n] = fmaf(dA, h[n], bx);
-                    y = fmaf(cc[j], h[n], y);
+            for (int u = 0; u < kLnBatch; ++u) {
+                const int slot = base + 32 * u;
+                if (slot < SL) {
+                    xv[u] = ld_stream(x4 + o + slot);
+                    zv[u] = ld_stream(z4 + o + slot);
+                    yv[u] = __ldcg(ys4 + slot);
                 }
             }
-            if (live) {
-                if (add) atomicAdd(yp, y);
-                else *yp = y;
+#pragma unroll
+            for (int u = 0; u < kLnBatch; ++u) {
+                const int slot = base + 32 * u;
+                if (slot < SL) {
+                    const float4 sv = f4_fma(dsum[slot], xv[u], yv[u]);
+                    srow[slot] = sv;
+                    zrow[slot] = zv[u];
+                    ln_accum(sv, K, m1, m2);
+                }
             }
-            yp += ystep;
         }
+        float mean, rstd;
+        ln_stats(m1, m2, K, invE, sh.ln_eps, mean, rstd);
+        for (int slot = lane; slot < SL; slot += 32)
+            st_stream(y4 + o + slot, ln_gate4(srow[slot], zrow[slot], g4[slot], b4[slot], mean, rstd));
     }
 }
 
+// ---- Staged scans: one CTA per (image, 128-channel tile, direction) ----------------------------
 template <bool ZOH_EXACT>
 __global__ void __launch_bounds__(kSeqThreads)
 scan_seq_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__ xbar,
                 const float* __restrict__ A_log, const float* __restrict__ W_dt, const float* __restrict__ b_dt,
                 float* __restrict__ ys) {
     extern __shared__ __align__(16) float smem[];
-    constexpr int NS = kSeqStates;
-    const int T = sh.T, E = sh.E, N = sh.N, R = sh.R, J = sh.J;
-    const int R4 = seq_r4(R), WS = seq_wstride(R);
-    const int tiles = (E + kSeqThreads - 1) / kSeqThreads;
-    const int k = blockIdx.x % sh.nd;                   // parameter slot
+    const int tiles = (sh.E + kSeqThreads - 1) / kSeqThreads;
+    const int k = blockIdx.x % sh.nd;
     const int tile = (blockIdx.x / sh.nd) % tiles;
     const int b = blockIdx.x / (sh.nd * tiles);
-    const bool fwd = (sh.nd == 2) ? (k == 0) : ((sh.dir_flags & 1u) != 0);
-    const int c = threadIdx.x, e0 = tile * kSeqThreads, e = e0 + c;
-    const bool live = e < E;
-    SeqSmem sm;
-    sm.w = smem;
-    sm.bc = sm.w + kSeqThreads * WS;
-    sm.dtT = sm.bc + 2 * kSeqChunk * 2 * NS;
-    sm.xs = sm.dtT + 2 * R4 * kSeqChunk;
-    const float* ub = u + u_offset(sh, k, b, 0);
-
-    // W_dt rows of the CTA's channels (coalesced global reads; padding columns zero)
-    for (int i = threadIdx.x; i < kSeqThreads * R4; i += kSeqThreads) {
-        const int cc = i / R4, r = i - cc * R4;
-        const int ee = e0 + cc;
-        sm.w[cc * WS + r] = (ee < E && r < R) ? __ldg(W_dt + ((size_t)k * E + ee) * R + r) : 0.f;
-    }
-    constexpr float kLog2e = 1.4426950408889634f;
-    float A2[NS], An[NS], Ainv[NS], h[NS];
-#pragma unroll
-    for (int n = 0; n < NS; ++n) {
-        const float A = (live && n < N) ? -expf(__ldg(A_log + ((size_t)k * E + e) * N + n)) : 0.f;
-        A2[n] = A * kLog2e;
-        An[n] = A;
-        Ainv[n] = A != 0.f ? 1.f / A : 0.f;
-        h[n] = 0.f;
-    }
-    const float bias = live ? __ldg(b_dt + (size_t)k * E + e) : 0.f;
-    const bool add = sh.nd == 2;
-
-    const int nchunks = (T + kSeqChunk - 1) / kSeqChunk;
-    // stage chunk ci into buffer buf; slot i <- step t0 + i (forward) or t0 + len - 1 - i (backward)
-    auto stage = [&](int ci, int buf) {
-        const int t0 = ci * kSeqChunk, len = min(kSeqChunk, T - t0);
-        float* bcb = sm.bc + buf * kSeqChunk * 2 * NS;
-        for (int i = threadIdx.x; i < kSeqChunk * 2 * NS; i += kSeqThreads) {
-            const int slot = i >> 5, j = i & 31, n = j & 15;
-            const int t = t0 + (fwd ? slot : len - 1 - slot);
-            const bool ok = slot < len && n < N;
-            cp_async4z(bcb + i, ok ? ub + (size_t)t * J + R + (j < NS ? n : N + n) : ub, ok);
-        }
-        float* dtb = sm.dtT + buf * R4 * kSeqChunk;
-        for (int i = threadIdx.x; i < R4 * kSeqChunk; i += kSeqThreads) {
-            const int r = i >> 4, slot = i & 15;
-            const int t = t0 + (fwd ? slot : len - 1 - slot);
-            const bool ok = slot < len && r < R;
-            cp_async4z(dtb + i, ok ? ub + (size_t)t * J + r : ub, ok);
-        }
-        float* xb = sm.xs + buf * kSeqChunk * kSeqThreads;
-        for (int v = threadIdx.x; v < kSeqChunk * (kSeqThreads / 4); v += kSeqThreads) {
-            const int slot = v >> 5, c4 = (v & 31) * 4;
-            const int t = t0 + (fwd ? slot : len - 1 - slot);
-            const bool ok = slot < len && e0 + c4 < E;
-            cp_async16(xb + slot * kSeqThreads + c4, ok ? (const void*)(xbar + ((size_t)b * T + t) * E + e0 + c4)
-                                                        : (const void*)xbar, ok ? 16u : 0u);
-        }
-        cp_async_commit();
-    };
-
-    stage(fwd ? 0 : nchunks - 1, 0);
-    for (int it = 0; it < nchunks; ++it) {
-        const int ci = fwd ? it : nchunks - 1 - it;
-        if (it + 1 < nchunks) {
-            stage(fwd ? it + 1 : nchunks - 2 - it, (it + 1) & 1);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncthreads();
-        const int buf = it & 1;
-        const int t0 = ci * kSeqChunk, len = min(kSeqChunk, T - t0);
-        const int tfirst = fwd ? t0 : t0 + len - 1;
-        float* yp = ys + ((size_t)b * T + tfirst) * E + e;
-        const ptrdiff_t ystep = fwd ? (ptrdiff_t)E : -(ptrdiff_t)E;
-        const float* bcb = sm.bc + buf * kSeqChunk * 2 * NS;
-        const float* dtb = sm.dtT + buf * R4 * kSeqChunk;
-        const float* xb = sm.xs + buf * kSeqChunk * kSeqThreads + c;
-        const float* wrow = sm.w + c * WS;
-        if (len == kSeqChunk)
-            seq_chunk<kSeqChunk, ZOH_EXACT>(bcb, dtb, xb, wrow, R4, bias, len, A2, An, Ainv, h, yp, ystep, live, add);
-        else
-            seq_chunk<0, ZOH_EXACT>(bcb, dtb, xb, wrow, R4, bias, len, A2, An, Ainv, h, yp, ystep, live, add);
-        __syncthreads();  // the buffer is refilled by the next iteration's stage()
-    }
+    seq_scan<kSeqThreads, 1, ZOH_EXACT>(sh, u, xbar, A_log, W_dt, b_dt, ys, b, tile * kSeqThreads, k, smem);
 }
 
 // Device math self-test: out[i] = f(in[i]) for the SFU-based helpers the layer uses

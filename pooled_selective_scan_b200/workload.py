@@ -50,6 +50,12 @@ def activations(cfg: LayerConfig, device, pinned_host: bool = False, first_image
     return out
 
 
+def ln_tensors(cfg: LayerConfig, device) -> dict:
+    """Post-SSM LayerNorm weights at their usual initialisation: gamma = 1, beta = 0."""
+    return dict(ln_gamma=torch.ones(cfg.E, dtype=torch.float32, device=device),
+                ln_beta=torch.zeros(cfg.E, dtype=torch.float32, device=device))
+
+
 def layer_tensors(cfg: LayerConfig, device, pinned_host: bool = False, first_image: int = 0) -> dict:
     d = params_tensors(cfg, "cpu" if pinned_host else device)
     if pinned_host:

@@ -39,8 +39,9 @@ def assert_close(got, ref, what="y"):
 
 
 def gpu_forward(inp: dict, pool_axis: int, dir_flags: int, h=None, w=None, pool_scale=1.0, zoh_exact=False,
-                intermediates=True, path="auto"):
-    """Run the CUDA layer on numpy inputs; return y (and workspace intermediates) as numpy."""
+                intermediates=True, path="auto", ln_eps=1e-5):
+    """Run the CUDA layer on numpy inputs; return y (and workspace intermediates) as numpy.  The
+    post-SSM LayerNorm runs when inp holds ln_gamma and ln_beta."""
     import torch
 
     from pooled_selective_scan_b200 import ssm
@@ -48,12 +49,14 @@ def gpu_forward(inp: dict, pool_axis: int, dir_flags: int, h=None, w=None, pool_
     dev = torch.device("cuda")
     t = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev) for k, v in inp.items() if v is not None}
     keep = t.get("keep_idx")
+    ln = "ln_gamma" in t
     shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, dir_flags, keep, h, w, pool_scale, zoh_exact,
-                            path)
+                            path, ln, ln_eps)
     ws = ssm.alloc_workspace(shape, dev)
     ws.fill_(0xFF)  # poison: every intermediate must be written before it is read
     y = ssm.forward(t["x"], t["z"], t["A_log"], t["D"], t["W_x"], t["W_dt"], t["b_dt"], pool_axis, dir_flags,
-                    keep_idx=keep, h=h, w=w, pool_scale=pool_scale, zoh_exact=zoh_exact, workspace=ws, path=path)
+                    keep_idx=keep, h=h, w=w, pool_scale=pool_scale, zoh_exact=zoh_exact, workspace=ws, path=path,
+                    ln_gamma=t.get("ln_gamma"), ln_beta=t.get("ln_beta"), ln_eps=ln_eps)
     status = ssm.device_status(ws)
     out = dict(y=y.cpu().numpy(), status=status, launches=ssm.launch_names(shape))
     if intermediates:

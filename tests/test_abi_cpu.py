@@ -67,7 +67,7 @@ def test_status_strings(lib):
     assert nat.status_string(0) == "FV_OK"
     for s in range(1, 10):
         assert nat.status_string(s).startswith("FV_ERR_")
-    assert lib.fastvim_abi_version() == 1
+    assert lib.fastvim_abi_version() == 2
 
 
 # ---------------------------------------------------------------------------------------------
@@ -195,3 +195,31 @@ def test_math_selftest_rejects_bad_arguments(lib):
     assert f(0, ctypes.c_void_p(FAKE + 4), ctypes.c_void_p(FAKE + (1 << 32)), 8, None) == nat.FV_ERR_ALIGN
     assert f(0, ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE + 16), 8, None) == nat.FV_ERR_ALIAS
     assert f(1, None, None, 0, None) == nat.FV_OK  # nothing to do
+
+
+def test_layernorm_arguments(lib):
+    LN = nat.FV_FLAG_LAYERNORM
+    g, b = FAKE + (10 << 32), FAKE + (11 << 32)
+    assert validate(good_args(flags=LN, ln_gamma=g, ln_beta=b, ln_eps=1e-5)) == nat.FV_OK
+    assert validate(good_args(flags=LN, ln_gamma=g, ln_beta=None, ln_eps=1e-5)) == nat.FV_ERR_NULL
+    assert validate(good_args(flags=LN, ln_gamma=None, ln_beta=None, ln_eps=1e-5)) == nat.FV_ERR_NULL
+    assert validate(good_args(ln_gamma=g, ln_beta=b)) == nat.FV_ERR_SHAPE  # weights without the flag
+    for eps in (0.0, -1e-5, float("nan"), float("inf")):
+        assert validate(good_args(flags=LN, ln_gamma=g, ln_beta=b, ln_eps=eps)) == nat.FV_ERR_SHAPE
+    assert validate(good_args(flags=LN, ln_gamma=g + 4, ln_beta=b, ln_eps=1e-5)) == nat.FV_ERR_ALIGN
+    assert validate(good_args(flags=LN, ln_gamma=g, ln_beta=b, ln_eps=1e-5, E=4100)) == nat.FV_ERR_UNSUPPORTED
+    assert lib.fastvim_abi_version() == 2
+
+
+def test_layernorm_launches(lib):
+    LN = nat.FV_FLAG_LAYERNORM
+    g, b = FAKE + (10 << 32), FAKE + (11 << 32)
+    small = good_args(flags=LN, ln_gamma=g, ln_beta=b, ln_eps=1e-5)
+    n = lib.fastvim_ssm_launch_count(ctypes.byref(small))
+    names = [lib.fastvim_ssm_launch_name(ctypes.byref(small), i).decode() for i in range(n)]
+    assert names == ["pool_dense_kernel", "proj_tasks_kernel", "scan_seq_kernel", "ln_epilogue_kernel"]
+    masked = good_args(flags=LN, ln_gamma=g, ln_beta=b, ln_eps=1e-5, K=49, keep_idx=FAKE + (9 << 32))
+    n = lib.fastvim_ssm_launch_count(ctypes.byref(masked))
+    assert lib.fastvim_ssm_launch_name(ctypes.byref(masked), n - 1).decode() == "ln_epilogue_kernel"
+    big = good_args(h=128, w=128, B=4, flags=LN, ln_gamma=g, ln_beta=b, ln_eps=1e-5)
+    assert lib.fastvim_ssm_launch_count(ctypes.byref(big)) == 1  # the fused launch does it in its gate tasks
