@@ -44,7 +44,8 @@ MUFU_PER_SM_CLK = 16
 
 
 def kernel_work(name: str, cfg, pool_axis: int):
-    """(bound, algorithmic amount per launch) of one launch of kernel `name` on workload `cfg`:
+    """(bound, algorithmic amount per step) of kernel `name` on workload `cfg` (all its launches in
+    one step; a staged layer launches a kernel once per chunk of images):
     bytes for the streaming kernels (what the step must move at minimum), exp2 evaluations for
     the scans (one per state, step, channel and direction), None for the rest."""
     tok = cfg.tokens_per_call()                       # grid tokens, or kept tokens when masked
@@ -358,7 +359,8 @@ def run_ours(a, cfg, pool_axis):
     if ssm.device_status(ws) != 0:
         raise SystemExit("device status reported an error during warm-up")
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nl + 1)] for _ in range(a.steps)]
+    # events[2j], events[2j+1] bracket launch j on the stream it runs on
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nl)] for _ in range(a.steps)]
     for evs in events:  # materialise the event handles outside the timed region
         for e in evs:
             e.record(stream)
@@ -388,12 +390,17 @@ def run_ours(a, cfg, pool_axis):
     if flush is None:
         local_ms = start.elapsed_time(end)
     else:
-        local_ms = sum(evs[0].elapsed_time(evs[nl]) for evs in events)
+        local_ms = sum(evs[0].elapsed_time(evs[2 * nl - 1]) for evs in events)  # first to last launch
     max_ms = reduce_max(local_ms, dev)
-    per_kernel = {n: [] for n in names}
+    # per kernel: its launches' device time in each step (a staged layer launches each kernel once
+    # per chunk of images; those launches run one after another)
+    per_kernel = {n: [] for n in dict.fromkeys(names)}
     for evs in events:
+        step = {n: 0.0 for n in per_kernel}
         for j, n in enumerate(names):
-            per_kernel[n].append(evs[j].elapsed_time(evs[j + 1]))
+            step[n] += evs[2 * j].elapsed_time(evs[2 * j + 1])
+        for n, v in step.items():
+            per_kernel[n].append(v)
     if ssm.device_status(ws) != 0:
         raise SystemExit("device status reported an error in the timed region")
 
@@ -408,7 +415,8 @@ def run_ours(a, cfg, pool_axis):
     for n, v in per_kernel.items():
         avg_s = statistics.mean(v) / 1e3
         bound, amount = kernel_work(n, cfg, pool_axis)
-        ent = {"launches": len(v), "avg_us": avg_s * 1e6, "share": sum(v) / total_k, "bound": bound}
+        ent = {"launches_per_step": names.count(n), "us_per_step": avg_s * 1e6, "share": sum(v) / total_k,
+               "bound": bound}
         if bound == "hbm":
             ent.update(achieved=amount / avg_s / 1e9, unit="GB/s", frac=amount / avg_s / 1e9 / peak)
         elif bound == "alu":
@@ -417,6 +425,7 @@ def run_ours(a, cfg, pool_axis):
     dom = max(kern, key=lambda n: kern[n]["share"])
     bound, amount = kernel_work(dom, cfg, pool_axis)
     dk = kern[dom]
+    amount //= max(1, dk["launches_per_step"])  # per launch: one chunk of the batch
     if bound == "alu":
         roofline = {"bound": "alu", "kernel": dom, "achieved": dk["achieved"], "peak": mufu_peak,
                     "unit": "G exp2/s", "frac": dk["frac"], "traffic": recorded_traffic(dom, cfg.name),

@@ -130,7 +130,7 @@ typedef struct {
     size_t total_bytes;  /* what fastvim_ssm_workspace_size returns                          */
     size_t status;       /* uint32 device status word (+ one uint32 of scratch)              */
     size_t xbar;         /* fp32 [B][T][E] pooled tokens                                     */
-    size_t u;            /* fp32 projections dt_low | B | C: [nd][B] blocks of [T][R+2N], each
+    size_t u;            /* fp32 projections dt_low | B | C: [B][nd] blocks of [T][R+2N], each
                             block starting every ceil(T (R+2N) / 32) * 32 floats            */
     size_t ys;           /* fp32 [B][T][E] scan output summed over directions                */
     size_t row_of;       /* int32 [B][K] pooled row of each kept token (masked), else 0      */
@@ -176,14 +176,19 @@ FV_API const char* fastvim_ssm_launch_name(const fv_ssm_args* args, int i);
 
 /* The layer: queue pool -> projections -> scans -> repeat/skip/gate on `stream`.
  * ws: device workspace of at least fastvim_ssm_workspace_size(args) bytes, 256-byte aligned,
- * no initial contents required, not shared with a concurrently running call. */
+ * no initial contents required, not shared with a concurrently running call.
+ * With FASTVIM_STAGED_CHUNKS = C > 1 (environment, tuning only; default 1) the staged kernels run
+ * as C chunks of images in a pipeline: the projections and scans of one chunk go to a
+ * high-priority stream the library keeps per device, in parallel with the pooling and epilogue
+ * of its neighbours on `stream`; every piece of the call is ordered before the call's last
+ * launch on `stream` (CUDA-graph capture follows the events). */
 FV_API fv_status fastvim_ssm_forward(const fv_ssm_args* args, void* ws, size_t ws_bytes, void* stream);
 
-/* fastvim_ssm_forward with timing marks: `events` holds n_events >= launch_count + 1 CUDA
- * events (cudaEvent_t, created by the caller); events[i] is recorded on `stream` just before
- * the i-th kernel launch and events[launch_count] after the last one, so the elapsed time
- * between events i and i+1 is the device duration of launch i.  Same results as
- * fastvim_ssm_forward. */
+/* fastvim_ssm_forward with timing marks: `events` holds n_events >= 2 * launch_count CUDA
+ * events (cudaEvent_t, created by the caller); events[2i] and events[2i+1] are recorded just
+ * before and just after the i-th kernel launch, on the stream that launch runs on, so their
+ * elapsed time is the device duration of launch i (launches of the staged kernels may overlap
+ * one another on two streams).  Same results as fastvim_ssm_forward. */
 FV_API fv_status fastvim_ssm_forward_events(const fv_ssm_args* args, void* ws, size_t ws_bytes,
                                             void* stream, void* const* events, int n_events);
 

@@ -237,32 +237,57 @@ cudaError_t ensure_smem(Kern kernel, size_t bytes) {
         }                                              \
     } while (0)
 
-// Records events[i] just before the i-th kernel launch and events[n] after the last one when an
-// event list is given (n = the call's launch count).
+// Records events[2i] just before and events[2i+1] just after the i-th kernel launch, on the
+// stream of that launch, when an event list is given.
 struct EventMarks {
     void* const* ev;
     int n, next;
-    cudaError_t mark(cudaStream_t st) {
-        if (!ev || next > n) return cudaSuccess;
-        return cudaEventRecord((cudaEvent_t)ev[next++], st);
+    cudaError_t before(cudaStream_t st) {
+        if (!ev || next >= n) return cudaSuccess;
+        return cudaEventRecord((cudaEvent_t)ev[2 * next], st);
+    }
+    cudaError_t after(cudaStream_t st) {
+        if (!ev || next >= n) return cudaSuccess;
+        return cudaEventRecord((cudaEvent_t)ev[2 * next++ + 1], st);
     }
 };
 
-#define FV_MARK(marks, st)                                   \
-    do {                                                     \
-        cudaError_t e_ = (marks).mark(st);                   \
-        if (e_ != cudaSuccess) {                             \
-            note_cuda(e_, "event record");                   \
-            return FV_ERR_CUDA;                              \
-        }                                                    \
+#define FV_MARK_CALL(marks, st, call)                          \
+    do {                                                       \
+        cudaError_t e_ = (marks).before(st);                   \
+        if (e_ != cudaSuccess) {                               \
+            note_cuda(e_, "event record");                     \
+            return FV_ERR_CUDA;                                \
+        }                                                      \
+        fv_status s_ = (call);                                 \
+        if (s_ != FV_OK) return s_;                            \
+        if ((e_ = (marks).after(st)) != cudaSuccess) {         \
+            note_cuda(e_, "event record");                     \
+            return FV_ERR_CUDA;                                \
+        }                                                      \
     } while (0)
+
+// Chunks of images the staged kernels run as (a pipeline over two streams, see forward_impl).
+// One by default: on B200 the overlap measured slower for every workload (e.g. the masked
+// 1024 px layer 0.58 -> 0.78 ms, the 1024 px layer 1.24 -> 1.37 ms with 4 chunks): the
+// long-lived projection and scan CTAs on the side stream hold SMs that the pooling and epilogue
+// kernels need to keep HBM saturated.  FASTVIM_STAGED_CHUNKS (1..8) sets it (tuning only).
+int staged_chunks(const fv::Shape& sh) {
+    int c = 1;
+    if (const char* env = getenv("FASTVIM_STAGED_CHUNKS")) {
+        const int v = atoi(env);
+        if (v >= 1 && v <= 8) c = v;
+    }
+    return sh.B < c ? (sh.B > 0 ? sh.B : 1) : c;
+}
+int staged_per_chunk(const fv::Shape& sh) { return sh.K > 0 ? 5 : 4; }
 
 int launch_count_of(const fv::Shape& sh) {
     if (sh.B == 0) return 0;
     const Path path = choose_path(sh);
     if (path == Path::Invalid) return 0;
     if (path == Path::Fused) return 1;
-    return sh.K > 0 ? 5 : 4;
+    return staged_chunks(sh) * staged_per_chunk(sh);
 }
 
 const char* launch_name_of(const fv::Shape& sh, int i) {
@@ -272,8 +297,22 @@ const char* launch_name_of(const fv::Shape& sh, int i) {
                                    "mask_epilogue_kernel"};
     if (i < 0 || i >= launch_count_of(sh)) return "";
     if (choose_path(sh) == Path::Fused) return "fused_layer_kernel";
-    if (sh.ln && i == launch_count_of(sh) - 1) return "ln_epilogue_kernel";
-    return sh.K > 0 ? masked[i] : dense[i];
+    // Issue order: the front (pool) and middle (proj, scan) launches of chunk 0; then for each
+    // chunk c >= 1 its front and middle launches followed by the back (epilogue) launch of chunk
+    // c - 1; last the back launch of the last chunk.  k = position in a chunk's own list.
+    const int per = staged_per_chunk(sh), head = per - 1;
+    int k;
+    if (i == launch_count_of(sh) - 1) {
+        k = per - 1;
+    } else if (i < head) {
+        k = i;
+    } else {
+        const int r = (i - head) % per;
+        k = r < head ? r : per - 1;
+    }
+    const char* name = sh.K > 0 ? masked[k] : dense[k];
+    if (sh.ln && k == per - 1) name = "ln_epilogue_kernel";
+    return name;
 }
 
 template <int ND, bool Z>
@@ -352,6 +391,145 @@ fv_status launch_scan_seq(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws
     return FV_OK;
 }
 
+// Workspace view of images [b0, ...) of a staged call: every per-image region is image-major.
+fv_ws_layout chunk_layout(const fv::Shape& sh, const fv_ws_layout& L, int b0) {
+    fv_ws_layout c = L;
+    c.xbar += (size_t)b0 * sh.T * sh.E * sizeof(float);
+    c.u += (size_t)b0 * sh.nd * fv::u_block_stride(sh.T, sh.J) * sizeof(float);
+    c.ys += (size_t)b0 * sh.T * sh.E * sizeof(float);
+    if (sh.K > 0) {
+        c.row_of += (size_t)b0 * sh.K * sizeof(int32_t);
+        c.row_off += (size_t)b0 * (sh.T + 1) * sizeof(int32_t);
+        c.row_tok += (size_t)b0 * sh.K * sizeof(int32_t);
+    }
+    return c;
+}
+
+// The high-priority stream on which the staged pipeline runs projections and scans, one per
+// device, created on first use and kept for the life of the process.
+cudaStream_t side_stream(fv_status* s) {
+    static std::mutex mu;
+    static cudaStream_t streams[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64) {
+        note_cuda(e != cudaSuccess ? e : cudaErrorInvalidDevice, "side stream device");
+        *s = FV_ERR_CUDA;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!streams[dev]) {
+        int lo = 0, hi = 0;
+        if ((e = cudaDeviceGetStreamPriorityRange(&lo, &hi)) == cudaSuccess)
+            e = cudaStreamCreateWithPriority(&streams[dev], cudaStreamNonBlocking, hi);
+        if (e != cudaSuccess) {
+            note_cuda(e, "side stream");
+            streams[dev] = nullptr;
+            *s = FV_ERR_CUDA;
+            return nullptr;
+        }
+    }
+    return streams[dev];
+}
+
+// One chunk of a staged call: its shape, arguments and workspace view.
+struct StagedChunk {
+    fv::Shape sh;
+    fv_ssm_args a;
+    fv_ws_layout L;
+};
+
+// Front of a chunk: pooling (masked: bucketing of the kept ids, then pooling).
+fv_status staged_front(const StagedChunk& c, char* ws, unsigned* status, cudaStream_t st, EventMarks& marks) {
+    const fv::Shape& sh = c.sh;
+    const int M = sh.B * sh.T;
+    float* xbar = (float*)(ws + c.L.xbar);
+    if (sh.K == 0) {
+        FV_MARK_CALL(marks, st, ([&]() -> fv_status {
+            fv::pool_dense_kernel<<<M, fv::kThreads, 0, st>>>(sh, c.a.x, xbar);
+            FV_LAUNCH_CHECK("pool_dense_kernel");
+            return FV_OK;
+        })());
+        return FV_OK;
+    }
+    const size_t bsm = bucket_smem_bytes(sh);
+    cudaError_t e = ensure_smem(fv::mask_bucket_kernel, bsm);
+    if (e != cudaSuccess) { note_cuda(e, "bucket smem attribute"); return FV_ERR_CUDA; }
+    FV_MARK_CALL(marks, st, ([&]() -> fv_status {
+        fv::mask_bucket_kernel<<<sh.B, fv::kThreads, bsm, st>>>(sh, c.a.keep_idx, (int32_t*)(ws + c.L.row_of),
+                                                                (int32_t*)(ws + c.L.row_off),
+                                                                (int32_t*)(ws + c.L.row_tok), status);
+        FV_LAUNCH_CHECK("mask_bucket_kernel");
+        return FV_OK;
+    })());
+    FV_MARK_CALL(marks, st, ([&]() -> fv_status {
+        fv::mask_pool_kernel<<<M, fv::kThreads, 0, st>>>(sh, c.a.x, (const int32_t*)(ws + c.L.row_off),
+                                                         (const int32_t*)(ws + c.L.row_tok), xbar);
+        FV_LAUNCH_CHECK("mask_pool_kernel");
+        return FV_OK;
+    })());
+    return FV_OK;
+}
+
+// Middle of a chunk: x_proj, then dt_proj + ZOH + scans.
+fv_status staged_middle(const StagedChunk& c, char* ws, cudaStream_t st, EventMarks& marks) {
+    FV_MARK_CALL(marks, st, launch_proj_tasks(c.sh, &c.a, c.L, ws, st));
+    FV_MARK_CALL(marks, st, launch_scan_seq(c.sh, &c.a, c.L, ws, st));
+    return FV_OK;
+}
+
+// Back of a chunk: repeat + skip (+ LayerNorm) + gate.
+fv_status staged_back(const StagedChunk& c, char* ws, cudaStream_t st, EventMarks& marks) {
+    const fv::Shape& sh = c.sh;
+    const float* ys = (const float*)(ws + c.L.ys);
+    if (sh.ln) {
+        const size_t smem = fv::ln_epilogue_smem_bytes(sh);
+        cudaError_t e = ensure_smem(fv::ln_epilogue_kernel, smem);
+        if (e != cudaSuccess) { note_cuda(e, "LayerNorm epilogue smem attribute"); return FV_ERR_CUDA; }
+        const long long ntok = (long long)sh.B * (sh.K > 0 ? (long long)sh.K : (long long)sh.h * sh.w);
+        const long long per = (long long)fv::kLnWarps * fv::kLnTokensPerWarp;
+        const long long grid = (ntok + per - 1) / per;
+        if (grid >= (1ll << 31)) return FV_ERR_UNSUPPORTED;
+        FV_MARK_CALL(marks, st, ([&]() -> fv_status {
+            fv::ln_epilogue_kernel<<<(unsigned)grid, fv::kLnWarps * 32, smem, st>>>(
+                sh, c.a.x, c.a.z, ys, c.a.D, c.a.ln_gamma, c.a.ln_beta,
+                sh.K > 0 ? (const int32_t*)(ws + c.L.row_of) : nullptr, c.a.y);
+            FV_LAUNCH_CHECK("ln_epilogue_kernel");
+            return FV_OK;
+        })());
+    } else if (sh.K == 0) {
+        FV_MARK_CALL(marks, st, ([&]() -> fv_status {
+            fv::epilogue_dense_kernel<<<sh.B * sh.T, fv::kThreads, 0, st>>>(sh, c.a.x, c.a.z, ys, c.a.D, c.a.y);
+            FV_LAUNCH_CHECK("epilogue_dense_kernel");
+            return FV_OK;
+        })());
+    } else {
+        const int nkb = (sh.K + fv::kMaskEpiTokens - 1) / fv::kMaskEpiTokens;
+        FV_MARK_CALL(marks, st, ([&]() -> fv_status {
+            fv::mask_epilogue_kernel<<<sh.B * nkb, fv::kThreads, 0, st>>>(sh, c.a.x, c.a.z, ys, c.a.D,
+                                                                         (const int32_t*)(ws + c.L.row_of), c.a.y);
+            FV_LAUNCH_CHECK("mask_epilogue_kernel");
+            return FV_OK;
+        })());
+    }
+    return FV_OK;
+}
+
+// Events of one staged call, destroyed when the call has queued its work.
+struct CallEvents {
+    std::vector<cudaEvent_t> ev;
+    ~CallEvents() {
+        for (cudaEvent_t e : ev)
+            if (e) cudaEventDestroy(e);
+    }
+    cudaEvent_t make() {
+        cudaEvent_t e = nullptr;
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) e = nullptr;
+        ev.push_back(e);
+        return e;
+    }
+};
+
 fv_status forward_impl(const fv_ssm_args* a, void* ws_v, size_t ws_bytes, cudaStream_t st,
                        void* const* events = nullptr, int n_events = 0) {
     fv::Shape sh;
@@ -362,78 +540,75 @@ fv_status forward_impl(const fv_ssm_args* a, void* ws_v, size_t ws_bytes, cudaSt
     plan_layout(sh, &L);
     if (!ws_v || ws_bytes < L.total_bytes || ((uintptr_t)ws_v & 255u) != 0) return FV_ERR_WORKSPACE;
     if ((s = check_limits(sh)) != FV_OK) return s;
-    if (events && n_events < launch_count_of(sh) + 1) return FV_ERR_SHAPE;
+    if (events && n_events < 2 * launch_count_of(sh)) return FV_ERR_SHAPE;
     EventMarks marks{events, launch_count_of(sh), 0};
     char* ws = (char*)ws_v;
     unsigned* status = (unsigned*)(ws + L.status);
-    if (sh.B == 0) {
-        cudaError_t e = cudaMemsetAsync(status, 0, sizeof(unsigned), st);
-        if (e != cudaSuccess) { note_cuda(e, "status reset"); return FV_ERR_CUDA; }
-        return FV_OK;
-    }
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(unsigned), st);
+    if (e != cudaSuccess) { note_cuda(e, "status reset"); return FV_ERR_CUDA; }
+    if (sh.B == 0) return FV_OK;
     const Path path = choose_path(sh);
     if (path == Path::Invalid) return FV_ERR_UNSUPPORTED;
     if (path == Path::Fused) {
-        // status word and control block (ticket, abort flag, per-image counters) start at zero
-        cudaError_t e = cudaMemsetAsync(status, 0, sizeof(unsigned), st);
-        if (e == cudaSuccess)
-            e = cudaMemsetAsync(ws + L.ctrl, 0, (fv::kCtrlHeaderWords + fv::kCtrlCounters * (size_t)sh.B) * sizeof(unsigned), st);
+        // control block (ticket, abort flag, per-image counters) starts at zero
+        e = cudaMemsetAsync(ws + L.ctrl, 0, (fv::kCtrlHeaderWords + fv::kCtrlCounters * (size_t)sh.B) * sizeof(unsigned), st);
         if (e != cudaSuccess) { note_cuda(e, "control reset"); return FV_ERR_CUDA; }
-        FV_MARK(marks, st);
-        if ((s = launch_fused(sh, a, L, ws, st)) != FV_OK) return s;
-        FV_MARK(marks, st);
+        FV_MARK_CALL(marks, st, launch_fused(sh, a, L, ws, st));
         return FV_OK;
     }
-    const int M = sh.B * sh.T;
-    float* xbar = (float*)(ws + L.xbar);
-    if (sh.K == 0) {
-        FV_MARK(marks, st);
-        fv::pool_dense_kernel<<<M, fv::kThreads, 0, st>>>(sh, a->x, xbar, status);
-        FV_LAUNCH_CHECK("pool_dense_kernel");
-    } else {
-        cudaError_t e = cudaMemsetAsync(status, 0, sizeof(unsigned), st);
-        if (e != cudaSuccess) { note_cuda(e, "status reset"); return FV_ERR_CUDA; }
-        const size_t bsm = bucket_smem_bytes(sh);
-        e = ensure_smem(fv::mask_bucket_kernel, bsm);
-        if (e != cudaSuccess) { note_cuda(e, "bucket smem attribute"); return FV_ERR_CUDA; }
-        FV_MARK(marks, st);
-        fv::mask_bucket_kernel<<<sh.B, fv::kThreads, bsm, st>>>(sh, a->keep_idx, (int32_t*)(ws + L.row_of),
-                                                                (int32_t*)(ws + L.row_off),
-                                                                (int32_t*)(ws + L.row_tok), status);
-        FV_LAUNCH_CHECK("mask_bucket_kernel");
-        FV_MARK(marks, st);
-        fv::mask_pool_kernel<<<M, fv::kThreads, 0, st>>>(sh, a->x, (const int32_t*)(ws + L.row_off),
-                                                         (const int32_t*)(ws + L.row_tok), xbar);
-        FV_LAUNCH_CHECK("mask_pool_kernel");
+
+    // Staged: chunks of images; front (pool) and back (epilogue) on the caller's stream in the
+    // order front 0, front 1, back 0, front 2, back 1, ..., back C-1, and each chunk's middle
+    // (projections, scans) on the side stream between its front and its back.
+    const int C = staged_chunks(sh);
+    const int per_img_tok = sh.K > 0 ? sh.K : sh.h * sh.w;
+    std::vector<StagedChunk> ch(C);
+    const int base = sh.B / C, extra = sh.B % C;
+    for (int c = 0, b0 = 0; c < C; ++c) {
+        const int nb = base + (c < extra ? 1 : 0);
+        StagedChunk& k = ch[c];
+        k.sh = sh;
+        k.sh.B = nb;
+        k.a = *a;
+        k.a.B = nb;
+        const size_t off = (size_t)b0 * per_img_tok * sh.E;
+        k.a.x = a->x + off;
+        k.a.z = a->z + off;
+        k.a.y = a->y + off;
+        if (sh.K > 0) k.a.keep_idx = a->keep_idx + (size_t)b0 * sh.K;
+        k.L = chunk_layout(sh, L, b0);
+        b0 += nb;
     }
-    FV_MARK(marks, st);
-    if ((s = launch_proj_tasks(sh, a, L, ws, st)) != FV_OK) return s;
-    FV_MARK(marks, st);
-    if ((s = launch_scan_seq(sh, a, L, ws, st)) != FV_OK) return s;
-    FV_MARK(marks, st);
-    if (sh.ln) {
-        const size_t smem = fv::ln_epilogue_smem_bytes(sh);
-        cudaError_t e = ensure_smem(fv::ln_epilogue_kernel, smem);
-        if (e != cudaSuccess) { note_cuda(e, "LayerNorm epilogue smem attribute"); return FV_ERR_CUDA; }
-        const long long ntok = (long long)sh.B * (sh.K > 0 ? (long long)sh.K : (long long)sh.h * sh.w);
-        const long long per = (long long)fv::kLnWarps * fv::kLnTokensPerWarp;
-        const long long grid = (ntok + per - 1) / per;
-        if (grid >= (1ll << 31)) return FV_ERR_UNSUPPORTED;
-        fv::ln_epilogue_kernel<<<(unsigned)grid, fv::kLnWarps * 32, smem, st>>>(
-            sh, a->x, a->z, (const float*)(ws + L.ys), a->D, a->ln_gamma, a->ln_beta,
-            sh.K > 0 ? (const int32_t*)(ws + L.row_of) : nullptr, a->y);
-        FV_LAUNCH_CHECK("ln_epilogue_kernel");
-    } else if (sh.K == 0) {
-        fv::epilogue_dense_kernel<<<M, fv::kThreads, 0, st>>>(sh, a->x, a->z, (const float*)(ws + L.ys), a->D, a->y);
-        FV_LAUNCH_CHECK("epilogue_dense_kernel");
-    } else {
-        const int nkb = (sh.K + fv::kMaskEpiTokens - 1) / fv::kMaskEpiTokens;
-        fv::mask_epilogue_kernel<<<sh.B * nkb, fv::kThreads, 0, st>>>(sh, a->x, a->z, (const float*)(ws + L.ys),
-                                                                     a->D, (const int32_t*)(ws + L.row_of), a->y);
-        FV_LAUNCH_CHECK("mask_epilogue_kernel");
+    if (C == 1) {
+        if ((s = staged_front(ch[0], ws, status, st, marks)) != FV_OK) return s;
+        if ((s = staged_middle(ch[0], ws, st, marks)) != FV_OK) return s;
+        return staged_back(ch[0], ws, st, marks);
     }
-    FV_MARK(marks, st);
-    return FV_OK;
+    cudaStream_t side = side_stream(&s);
+    if (!side) return s;
+    CallEvents evs;
+    std::vector<cudaEvent_t> front_done(C), middle_done(C);
+    for (int c = 0; c < C; ++c) {
+        front_done[c] = evs.make();
+        middle_done[c] = evs.make();
+        if (!front_done[c] || !middle_done[c]) { note_cuda(cudaErrorMemoryAllocation, "pipeline events"); return FV_ERR_CUDA; }
+    }
+    for (int c = 0; c < C; ++c) {
+        if ((s = staged_front(ch[c], ws, status, st, marks)) != FV_OK) return s;
+        if ((e = cudaEventRecord(front_done[c], st)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(side, front_done[c], 0)) != cudaSuccess) {
+            note_cuda(e, "pipeline fork");
+            return FV_ERR_CUDA;
+        }
+        if ((s = staged_middle(ch[c], ws, side, marks)) != FV_OK) return s;
+        if ((e = cudaEventRecord(middle_done[c], side)) != cudaSuccess) { note_cuda(e, "pipeline event"); return FV_ERR_CUDA; }
+        if (c >= 1) {
+            if ((e = cudaStreamWaitEvent(st, middle_done[c - 1], 0)) != cudaSuccess) { note_cuda(e, "pipeline join"); return FV_ERR_CUDA; }
+            if ((s = staged_back(ch[c - 1], ws, st, marks)) != FV_OK) return s;
+        }
+    }
+    if ((e = cudaStreamWaitEvent(st, middle_done[C - 1], 0)) != cudaSuccess) { note_cuda(e, "pipeline join"); return FV_ERR_CUDA; }
+    return staged_back(ch[C - 1], ws, st, marks);
 }
 
 }  // namespace

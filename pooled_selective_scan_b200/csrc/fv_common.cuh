@@ -31,12 +31,13 @@ struct Shape {
     float ln_eps;
 };
 
-// Projections u of (direction k, image b) are one block of T x J floats; blocks start every
+// Projections u of (image b, direction k) are one block of T x J floats, image-major (so the
+// blocks of a run of images are contiguous); blocks start every
 // u_block_stride floats (T J rounded up to 32 floats = 128 bytes), so no cache line holds
 // projections of two images.
 __host__ __device__ __forceinline__ size_t u_block_stride(int T, int J) { return (((size_t)T * J + 31) / 32) * 32; }
 __host__ __device__ __forceinline__ size_t u_offset(const Shape& sh, int k, int b, int t) {
-    return ((size_t)k * sh.B + b) * u_block_stride(sh.T, sh.J) + (size_t)t * sh.J;
+    return ((size_t)b * sh.nd + k) * u_block_stride(sh.T, sh.J) + (size_t)t * sh.J;
 }
 
 // Offset (in floats) of token s of pooled token (b, t) on the dense grid, and the stride

@@ -85,7 +85,7 @@ struct FusedPtrs {
     const float* ln_gamma;  // [E] (FV_FLAG_LAYERNORM) or NULL
     const float* ln_beta;
     float* xbar;   // [B][T][E]
-    float* u;      // [nd][B] blocks of [T][J] (see u_offset)
+    float* u;      // [B][nd] blocks of [T][J] (see u_offset)
     float* ys;     // [B][T][E]
     unsigned* status;
     unsigned* ctrl;

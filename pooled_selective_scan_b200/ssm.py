@@ -186,7 +186,7 @@ def forward(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis=POOL_W, dir_flags=DIR_FWD
 class BoundForward:
     """A forward call with its tensors, workspace and argument block bound once, for repeated
     launches (benchmark loops): ``run()`` queues the layer, ``run_events(evs)`` also records
-    ``evs[i]`` before the i-th kernel launch and ``evs[-1]`` after the last one."""
+    ``evs[2i]`` and ``evs[2i+1]`` just before and after the i-th kernel launch."""
 
     def __init__(self, shape: LayerShape, t: dict, y, workspace, stream=None):
         self.shape = shape
@@ -198,7 +198,7 @@ class BoundForward:
         self._ws = ctypes.c_void_p(workspace.data_ptr())
         self._wsn = ctypes.c_size_t(workspace.numel())
         self.n_launch = launch_count(shape)
-        self._evbuf = (ctypes.c_void_p * (self.n_launch + 1))()
+        self._evbuf = (ctypes.c_void_p * (2 * self.n_launch))()
         L = nat.lib()
         nat.check(L.fastvim_ssm_validate(ctypes.byref(self._args)), "fastvim_ssm_validate")
 
@@ -207,6 +207,10 @@ class BoundForward:
                   "fastvim_ssm_forward")
 
     def run_events(self, events):
+        """events: 2 * n_launch CUDA events; events[2i], events[2i+1] bracket launch i."""
+        for e in events:
+            if not e.cuda_event:  # torch creates the CUDA event on its first record
+                e.record()
         for i, e in enumerate(events):
             self._evbuf[i] = e.cuda_event
         nat.check(nat.lib().fastvim_ssm_forward_events(ctypes.byref(self._args), self._ws, self._wsn, self._stream,

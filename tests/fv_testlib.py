@@ -69,7 +69,8 @@ def gpu_forward(inp: dict, pool_axis: int, dir_flags: int, h=None, w=None, pool_
 
         out["xbar"] = view(L["xbar"], B * T * E, np.float32).reshape(B, T, E)
         ub = -(-T * J // 32) * 32  # per (direction, image) block stride, floats
-        out["u"] = view(L["u"], nd * B * ub, np.float32).reshape(nd, B, ub)[:, :, :T * J].reshape(nd, B, T, J)
+        out["u"] = (view(L["u"], nd * B * ub, np.float32).reshape(B, nd, ub)[:, :, :T * J].reshape(B, nd, T, J)
+                    .transpose(1, 0, 2, 3))
         out["ys"] = view(L["ys"], B * T * E, np.float32).reshape(B, T, E)
         if shape.K:
             out["row_of"] = view(L["row_of"], B * shape.K, np.int32).reshape(B, shape.K)

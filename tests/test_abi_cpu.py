@@ -223,3 +223,23 @@ def test_layernorm_launches(lib):
     assert lib.fastvim_ssm_launch_name(ctypes.byref(masked), n - 1).decode() == "ln_epilogue_kernel"
     big = good_args(h=128, w=128, B=4, flags=LN, ln_gamma=g, ln_beta=b, ln_eps=1e-5)
     assert lib.fastvim_ssm_launch_count(ctypes.byref(big)) == 1  # the fused launch does it in its gate tasks
+
+
+@pytest.mark.parametrize("chunks,masked,ln", [(1, False, False), (3, False, True), (4, True, False), (2, True, True)])
+def test_staged_chunk_launch_order(lib, monkeypatch, chunks, masked, ln):
+    monkeypatch.setenv("FASTVIM_STAGED_CHUNKS", str(chunks))
+    kw = dict(B=5, flags=2)
+    if masked:
+        kw.update(K=49, keep_idx=FAKE + (9 << 32))
+    if ln:
+        kw.update(flags=2 | nat.FV_FLAG_LAYERNORM, ln_gamma=FAKE + (10 << 32), ln_beta=FAKE + (11 << 32), ln_eps=1e-5)
+    a = good_args(**kw)
+    front = ["mask_bucket_kernel", "mask_pool_kernel"] if masked else ["pool_dense_kernel"]
+    middle = ["proj_tasks_kernel", "scan_seq_kernel"]
+    back = ["ln_epilogue_kernel" if ln else ("mask_epilogue_kernel" if masked else "epilogue_dense_kernel")]
+    want = front + middle
+    for c in range(1, chunks):
+        want += front + middle + back
+    want += back
+    n = lib.fastvim_ssm_launch_count(ctypes.byref(a))
+    assert [lib.fastvim_ssm_launch_name(ctypes.byref(a), i).decode() for i in range(n)] == want
