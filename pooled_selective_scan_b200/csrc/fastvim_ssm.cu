@@ -291,9 +291,9 @@ int launch_count_of(const fv::Shape& sh) {
 }
 
 const char* launch_name_of(const fv::Shape& sh, int i) {
-    static const char* dense[] = {"pool_dense_kernel", "proj_tasks_kernel", "scan_seq_kernel",
+    static const char* dense[] = {"pool_dense_kernel", "proj_gemm_kernel", "scan_seq_kernel",
                                   "epilogue_dense_kernel"};
-    static const char* masked[] = {"mask_bucket_kernel", "mask_pool_kernel", "proj_tasks_kernel", "scan_seq_kernel",
+    static const char* masked[] = {"mask_bucket_kernel", "mask_pool_kernel", "proj_gemm_kernel", "scan_seq_kernel",
                                    "mask_epilogue_kernel"};
     if (i < 0 || i >= launch_count_of(sh)) return "";
     if (choose_path(sh) == Path::Fused) return "fused_layer_kernel";
@@ -355,19 +355,6 @@ fv_status launch_fused(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_la
     const fv::FusedPtrs p = fused_ptrs(a, L, ws);
     if (sh.nd == 2) return sh.zoh_exact ? launch_fused_t<2, true>(sh, pl, p, st) : launch_fused_t<2, false>(sh, pl, p, st);
     return sh.zoh_exact ? launch_fused_t<1, true>(sh, pl, p, st) : launch_fused_t<1, false>(sh, pl, p, st);
-}
-
-// Staged: x_proj over every pooled token (one CTA per 16 tokens of an image).
-fv_status launch_proj_tasks(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st) {
-    const fv::FusedPlan pl = plan_fused(sh);
-    fv::FusedPtrs p = fused_ptrs(a, L, ws);
-    p.ctrl = nullptr;
-    const size_t smem = fv::fused_proj_smem_floats(sh) * sizeof(float);
-    cudaError_t e = ensure_smem(fv::proj_tasks_kernel, smem);
-    if (e != cudaSuccess) { note_cuda(e, "proj smem attribute"); return FV_ERR_CUDA; }
-    fv::proj_tasks_kernel<<<sh.B * pl.nQ, fv::kFusedThreads, smem, st>>>(sh, pl, p);
-    FV_LAUNCH_CHECK("proj_tasks_kernel");
-    return FV_OK;
 }
 
 // Staged: every (image, 128-channel tile, direction) recurrence, one thread each.  With both
@@ -471,9 +458,22 @@ fv_status staged_front(const StagedChunk& c, char* ws, unsigned* status, cudaStr
     return FV_OK;
 }
 
+// Staged x_proj: one GEMM over all pooled tokens of the chunk.
+fv_status launch_proj_gemm(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st) {
+    cudaError_t e = ensure_smem(fv::proj_gemm_kernel, fv::kPgSmemBytes);
+    if (e != cudaSuccess) { note_cuda(e, "proj smem attribute"); return FV_ERR_CUDA; }
+    const long long M = (long long)sh.B * sh.T;
+    const dim3 grid((unsigned)((M + fv::kPgM - 1) / fv::kPgM), (unsigned)((sh.NJ + fv::kPgN - 1) / fv::kPgN));
+    if (M >= (1ll << 31) / 2) return FV_ERR_UNSUPPORTED;
+    fv::proj_gemm_kernel<<<grid, fv::kPgThreads, fv::kPgSmemBytes, st>>>(sh, (const float*)(ws + L.xbar), a->W_x,
+                                                                        (float*)(ws + L.u));
+    FV_LAUNCH_CHECK("proj_gemm_kernel");
+    return FV_OK;
+}
+
 // Middle of a chunk: x_proj, then dt_proj + ZOH + scans.
 fv_status staged_middle(const StagedChunk& c, char* ws, cudaStream_t st, EventMarks& marks) {
-    FV_MARK_CALL(marks, st, launch_proj_tasks(c.sh, &c.a, c.L, ws, st));
+    FV_MARK_CALL(marks, st, launch_proj_gemm(c.sh, &c.a, c.L, ws, st));
     FV_MARK_CALL(marks, st, launch_scan_seq(c.sh, &c.a, c.L, ws, st));
     return FV_OK;
 }

@@ -1,5 +1,4 @@
-// fv_fused.cuh -- the dense FastVim SSM layer as ONE persistent, image-pipelined launch (sm_100a),
-// and the projection task body that the staged launches reuse.
+// fv_fused.cuh -- the dense FastVim SSM layer as ONE persistent, image-pipelined launch (sm_100a).
 //
 // The layer's pooled tokens depend on ALL of an image's x, and every output token depends on the
 // whole image's scan, so x must be read once for pooling and once more for the D x skip.  One
@@ -664,12 +663,6 @@ fused_layer_kernel(Shape sh, FusedPlan pl, FusedPtrs p) {
     }
 }
 
-// Staged launch of the projection task body: one CTA per task, ordered by the launch boundaries
-// instead of counters.
-__global__ void __launch_bounds__(kFusedThreads, 2) proj_tasks_kernel(Shape sh, FusedPlan pl, FusedPtrs p) {
-    extern __shared__ __align__(128) float smem_f[];
-    fused_proj(sh, pl, p, blockIdx.x / pl.nQ, blockIdx.x % pl.nQ, smem_f);
-}
 
 // A single CTA that waits, with the layer's bounded wait, on a counter that nothing increments:
 // exercises the timeout path (status FV_ERR_TIMEOUT, clean exit) without the layer.

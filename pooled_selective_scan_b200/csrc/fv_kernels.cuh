@@ -2,7 +2,7 @@
 //
 // Step map (FastVim, arXiv 2502.00594; gptget.net summary of the paper, section "方法详解"):
 //   pool_dense_kernel / mask_bucket_kernel + mask_pool_kernel   item 2 (and item 6, masked)
-//   proj_tasks_kernel (fv_fused.cuh's x_proj task body as a grid)  item 3
+//   proj_gemm_kernel (x_proj over every pooled token)            item 3
 //   scan_seq_kernel (dt_proj + softplus, ZOH, both scans)       items 3-4
 //   epilogue_dense_kernel / mask_epilogue_kernel                item 5 (repeat, skip, gate)
 // Pooling and the epilogues are HBM streaming; the scans are MUFU/issue bound.
@@ -363,6 +363,100 @@ ln_epilogue_kernel(Shape sh, const float* __restrict__ x, const float* __restric
         ln_stats(m1, m2, K, invE, sh.ln_eps, mean, rstd);
         for (int slot = lane; slot < SL; slot += 32)
             st_stream(y4 + o + slot, ln_gate4(srow[slot], zrow[slot], g4[slot], b4[slot], mean, rstd));
+    }
+}
+
+// ---- Staged x_proj: one fp32 GEMM over every pooled token of the batch ---------------------------
+// u[b][k][t][j] = sum_e W_x[k][j][e] * xbar[b][t][e]: C[m][n] = sum_e A[m][e] B[n][e] with M = B T
+// pooled tokens, N = nd (R + 2N) outputs, K = E; both operands E-contiguous.  A CTA of 256 threads
+// computes a 64 x 32 tile: two groups of 128 threads each sum half of every 32-channel operand
+// tile (more warps to hide latency), each thread 4 tokens x 4 outputs (rows tg + 16 i, columns
+// og + 8 j), so a warp's 128-bit shared loads touch 4 A rows (broadcast) and 8 B rows (padded rows
+// of 36 floats: conflict-free); the groups' partial sums meet in shared memory at the end, in a
+// fixed order.  Operand tiles stream through a 3-stage cp.async pipeline.
+constexpr int kPgM = 64, kPgN = 32, kPgK = 32, kPgPad = kPgK + 4, kPgStages = 3, kPgThreads = 256;
+constexpr size_t kPgSmemBytes = (size_t)kPgStages * (kPgM + kPgN) * kPgPad * sizeof(float);
+
+__global__ void __launch_bounds__(kPgThreads)
+proj_gemm_kernel(Shape sh, const float* __restrict__ xbar, const float* __restrict__ W_x, float* __restrict__ u) {
+    extern __shared__ __align__(16) float pg[];
+    const int M = sh.B * sh.T, N = sh.NJ, K = sh.E;
+    const int m0 = blockIdx.x * kPgM, n0 = blockIdx.y * kPgN;
+    const int tid = threadIdx.x, grp = tid >> 7, og = tid & 7, tg = (tid & 127) >> 3;
+    float* As = pg;                                   // [stages][64][36]
+    float* Bs = pg + kPgStages * kPgM * kPgPad;       // [stages][32][36]
+    const int nk = (K + kPgK - 1) / kPgK;
+    auto issue = [&](int kt) {
+        const int st = kt % kPgStages, k0 = kt * kPgK;
+        for (int c = tid; c < kPgM * (kPgK / 4); c += kPgThreads) {
+            const int r = c >> 3, k4 = (c & 7) * 4;
+            const bool ok = m0 + r < M && k0 + k4 < K;
+            cp_async16(As + (st * kPgM + r) * kPgPad + k4, ok ? (const void*)(xbar + (size_t)(m0 + r) * K + k0 + k4)
+                                                            : (const void*)xbar, ok ? 16u : 0u);
+        }
+        for (int c = tid; c < kPgN * (kPgK / 4); c += kPgThreads) {
+            const int r = c >> 3, k4 = (c & 7) * 4;
+            const bool ok = n0 + r < N && k0 + k4 < K;
+            cp_async16(Bs + (st * kPgN + r) * kPgPad + k4, ok ? (const void*)(W_x + (size_t)(n0 + r) * K + k0 + k4)
+                                                            : (const void*)W_x, ok ? 16u : 0u);
+        }
+    };
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll
+    for (int s = 0; s < kPgStages - 1; ++s) {
+        if (s < nk) issue(s);
+        cp_async_commit();
+    }
+    for (int kt = 0; kt < nk; ++kt) {
+        cp_async_wait<kPgStages - 2>();
+        __syncthreads();  // tile kt landed for everyone; the stage refilled below is no longer read
+        if (kt + kPgStages - 1 < nk) issue(kt + kPgStages - 1);
+        cp_async_commit();
+        const int st = kt % kPgStages;
+        const float* a = As + st * kPgM * kPgPad;
+        const float* bq = Bs + st * kPgN * kPgPad;
+#pragma unroll
+        for (int k = grp * (kPgK / 2); k < (grp + 1) * (kPgK / 2); k += 4) {
+            float4 av[4], bv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) av[i] = *reinterpret_cast<const float4*>(a + (tg + 16 * i) * kPgPad + k);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) bv[j] = *reinterpret_cast<const float4*>(bq + (og + 8 * j) * kPgPad + k);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    acc[i][j] = fmaf(av[i].w, bv[j].w,
+                                     fmaf(av[i].z, bv[j].z, fmaf(av[i].y, bv[j].y, fmaf(av[i].x, bv[j].x, acc[i][j]))));
+        }
+    }
+    cp_async_wait<0>();
+    __syncthreads();  // the operand tiles are free: reuse them for the second group's partial sums
+    float* part = pg;  // [128][16]
+    if (grp == 1)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) part[(tid - 128) * 16 + i * 4 + j] = acc[i][j];
+    __syncthreads();
+    if (grp == 1) return;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int m = m0 + tg + 16 * i;
+        if (m >= M) continue;
+        const int b = m / sh.T, t = m - b * sh.T;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int n = n0 + og + 8 * j;
+            if (n < N) {
+                const int k = n / sh.J, jc = n - k * sh.J;
+                u[u_offset(sh, k, b, t) + jc] = acc[i][j] + part[tid * 16 + i * 4 + j];
+            }
+        }
     }
 }
 

@@ -84,7 +84,7 @@ __device__ __forceinline__ void seq_chunk(const float* __restrict__ bc, const fl
             const float dtx = dt * xv;
             const float4* Bq = reinterpret_cast<const float4*>(bc + i * 2 * NS);
             const float4* Cq = Bq + NS / 4;
-            float y = 0.f;
+            float yp4[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums: short dependency chains
 #pragma unroll
             for (int q = 0; q < NS / 4; ++q) {
                 const float4 bv = Bq[q], cv = Cq[q];
@@ -96,9 +96,10 @@ __device__ __forceinline__ void seq_chunk(const float* __restrict__ bc, const fl
                     const float dA = ex2_approx(dt * A2[n]);
                     const float bx = ZOH_EXACT ? expm1f(dt * An[n]) * Ainv[n] * bb[j] * xv : dtx * bb[j];
                     h[n] = fmaf(dA, h[n], bx);
-                    y = fmaf(cc[j], h[n], y);
+                    yp4[j] = fmaf(cc[j], h[n], yp4[j]);
                 }
             }
+            const float y = (yp4[0] + yp4[1]) + (yp4[2] + yp4[3]);
             if (live) {
                 if (add) atomicAdd(yp, y);
                 else *yp = y;

@@ -170,7 +170,7 @@ def test_workspace_layout(lib, pool_axis, K):
 
 
 @pytest.mark.parametrize("flags,want", [(0, ["fused_layer_kernel"]), (4, ["fused_layer_kernel"]),
-                                        (2, ["pool_dense_kernel", "proj_tasks_kernel", "scan_seq_kernel",
+                                        (2, ["pool_dense_kernel", "proj_gemm_kernel", "scan_seq_kernel",
                                              "epilogue_dense_kernel"])])
 def test_path_selection_is_host_side(lib, flags, want):
     a = good_args(h=128, w=128, B=4, flags=flags)  # 2048 px FastVim-T images: fused by default
@@ -217,7 +217,7 @@ def test_layernorm_launches(lib):
     small = good_args(flags=LN, ln_gamma=g, ln_beta=b, ln_eps=1e-5)
     n = lib.fastvim_ssm_launch_count(ctypes.byref(small))
     names = [lib.fastvim_ssm_launch_name(ctypes.byref(small), i).decode() for i in range(n)]
-    assert names == ["pool_dense_kernel", "proj_tasks_kernel", "scan_seq_kernel", "ln_epilogue_kernel"]
+    assert names == ["pool_dense_kernel", "proj_gemm_kernel", "scan_seq_kernel", "ln_epilogue_kernel"]
     masked = good_args(flags=LN, ln_gamma=g, ln_beta=b, ln_eps=1e-5, K=49, keep_idx=FAKE + (9 << 32))
     n = lib.fastvim_ssm_launch_count(ctypes.byref(masked))
     assert lib.fastvim_ssm_launch_name(ctypes.byref(masked), n - 1).decode() == "ln_epilogue_kernel"
@@ -235,7 +235,7 @@ def test_staged_chunk_launch_order(lib, monkeypatch, chunks, masked, ln):
         kw.update(flags=2 | nat.FV_FLAG_LAYERNORM, ln_gamma=FAKE + (10 << 32), ln_beta=FAKE + (11 << 32), ln_eps=1e-5)
     a = good_args(**kw)
     front = ["mask_bucket_kernel", "mask_pool_kernel"] if masked else ["pool_dense_kernel"]
-    middle = ["proj_tasks_kernel", "scan_seq_kernel"]
+    middle = ["proj_gemm_kernel", "scan_seq_kernel"]
     back = ["ln_epilogue_kernel" if ln else ("mask_epilogue_kernel" if masked else "epilogue_dense_kernel")]
     want = front + middle
     for c in range(1, chunks):

@@ -135,7 +135,7 @@ def test_path_auto_choice():
     small = ssm.LayerShape(B=2, h=14, w=14, E=384, N=16, R=12, pool_axis=0, dir_flags=3)
     masked = ssm.LayerShape(B=2, h=64, w=64, E=384, N=16, R=12, pool_axis=0, dir_flags=3, K=100)
     assert ssm.launch_names(big) == ["fused_layer_kernel"]
-    assert ssm.launch_names(small) == ["pool_dense_kernel", "proj_tasks_kernel", "scan_seq_kernel", "epilogue_dense_kernel"]
+    assert ssm.launch_names(small) == ["pool_dense_kernel", "proj_gemm_kernel", "scan_seq_kernel", "epilogue_dense_kernel"]
     assert ssm.launch_names(masked)[0] == "mask_bucket_kernel"
 
 
