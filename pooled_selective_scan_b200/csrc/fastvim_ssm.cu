@@ -144,12 +144,14 @@ fv_status check_limits(const fv::Shape& sh) {
 }
 
 
-// Grid lines per P/E task: the fewest that give each task at least 96 KB of x (short tasks keep
-// the per-image dependency chain short).  FASTVIM_FUSED_LP (1..4) overrides it (tuning only).
+// Grid lines per P/E task: the fewest that give each task at least 384 KB of x.  Every task costs
+// a ticket (a contended atomic, ~1 us under full HBM load), so fewer, larger streaming tasks pay:
+// B200, 2048 px layer, 2.17 -> 2.13 ms going from one 196 KB line to two per task.
+// FASTVIM_FUSED_LP (1..4) overrides it (tuning only).
 int fused_lines_per_task(const fv::Shape& sh) {
     const size_t line = (size_t)sh.S * sh.E * sizeof(float);
     int lp = 1;
-    while (lp < fv::kMaxLP && lp < sh.T && (size_t)lp * line < ((size_t)96 << 10)) ++lp;
+    while (lp < fv::kMaxLP && lp < sh.T && (size_t)lp * line < ((size_t)384 << 10)) ++lp;
     if (const char* env = getenv("FASTVIM_FUSED_LP")) {
         const int v = atoi(env);
         if (v >= 1 && v <= fv::kMaxLP) lp = v < sh.T ? v : sh.T;

@@ -486,7 +486,8 @@ __device__ __forceinline__ void fused_scan(const Shape& sh, const FusedPlan& pl,
 // x and z stream through the ring (x mostly hits L2); every thread takes consecutive float4s of a
 // chunk (all 256 threads busy for any E), and y is stored straight from registers (evict-first).
 __device__ __forceinline__ bool fused_gate(const Shape& sh, const FusedPlan& pl, const FusedPtrs& p, int b, int g,
-                                           float* smem, Ring& rg, uint64_t pol_stream, int* s_flag) {
+                                           float* smem, Ring& rg, uint64_t pol_stream, const unsigned* scan_done,
+                                           unsigned* abort_flag, int* s_flag, unsigned long long* t_ready) {
     const int SL = sh.SL, E = sh.E;
     const int t0 = g * pl.LP;
     const int nl = min(sh.T, t0 + pl.LP) - t0;
@@ -510,6 +511,12 @@ __device__ __forceinline__ bool fused_gate(const Shape& sh, const FusedPlan& pl,
         if (sh.nd == 2) d += __ldg(p.D + E + e);
         dsum[e] = d;
     }
+    // x and z are on their way; now the image's scans must be done before its ys is read
+    if (!cta_wait(scan_done, (unsigned)pl.nS, p.status, abort_flag, pl.wait_limit_ns, s_flag)) {
+        ring_drain(rg, g0, g0 + min(kRingStages, nq), pl.wait_limit_ns);
+        return false;
+    }
+    if (t_ready && threadIdx.x == 0) *t_ready = globaltimer_ns();  // trace: when the scans were seen done
     for (int i = threadIdx.x; i < nl * E; i += kFusedThreads) {
         const int l = i / E, e = i - l * E;
         ysl[i] = __ldcg(p.ys + ((size_t)b * sh.T + t0 + l) * E + e);
@@ -617,12 +624,14 @@ fused_layer_kernel(Shape sh, FusedPlan pl, FusedPtrs p) {
         for (int i = 0; i < kRingStages; ++i) mbar_init(&s_full[i], 1);
         fence_mbar_init();
     }
+    // (Claiming the next ticket while a task runs would hide the atomic's latency, but a pooling
+    // ticket held behind a 60 us scan task stalls that image's whole chain: measured 3.5 ms.)
     for (;;) {
         __syncthreads();
         if (threadIdx.x == 0) {
             int kind = kTaskNone, b = 0, idx = 0;
             const unsigned tk = atomicAdd(p.ctrl, 1u);
-            if (tk < pl.total && ld_acquire_gpu(abort_flag) == 0u) fused_decode(pl, tk, kind, b, idx);
+            if (tk < pl.total && ld_relaxed_gpu(abort_flag) == 0u) fused_decode(pl, tk, kind, b, idx);
             s_task[0] = kind;
             s_task[1] = b;
             s_task[2] = idx;
@@ -644,9 +653,10 @@ fused_layer_kernel(Shape sh, FusedPlan pl, FusedPtrs p) {
             if (p.trace && threadIdx.x == 0) s_t1 = globaltimer_ns();
             fused_scan<ND, ZOH_EXACT>(sh, pl, p, b, idx, smem_f);
         } else {
-            if (!cta_wait(cnt_scan + b, (unsigned)pl.nS, p.status, abort_flag, pl.wait_limit_ns, &s_flag)) return;
-            if (p.trace && threadIdx.x == 0) s_t1 = globaltimer_ns();
-            if (!fused_gate(sh, pl, p, b, idx, smem_f, rg, pol_stream, &s_flag)) return;
+            // the gate waits for its scans inside, after its loads have started
+            if (!fused_gate(sh, pl, p, b, idx, smem_f, rg, pol_stream, cnt_scan + b, abort_flag, &s_flag,
+                            p.trace ? &s_t1 : nullptr))
+                return;
         }
         if (p.trace) {
             __syncthreads();
