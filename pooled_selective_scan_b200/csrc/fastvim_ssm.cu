@@ -194,11 +194,13 @@ fv::FusedPlan plan_fused(const fv::Shape& sh) {
     pl.ctP = fv::kStageBytes / (sh.E * (int)sizeof(float));
     pl.ctE = fv::kStageBytes / 2 / (sh.E * (int)sizeof(float));
     // Lag: enough rounds to cover one image's pool -> proj -> scan chain (chain_latency_us) at the
-    // rate one round streams (x twice, z and y once: 16 E bytes per grid token at
+    // rate one round streams, plus one (B200, 2048 px: L = 7 measured 2.14-2.16 ms, L = 9
+    // 2.22-2.23; holding the first gates back further, so that the start's pooling-only rounds
+    // cover the first chain, measured no better); it streams (x twice, z and y once: 16 E bytes per grid token at
     // ~6.5 TB/s).  (Keeping x in L2 across that window does not happen: traffic of this size
     // evicts first-touch lines whatever their L2 eviction priority.)
     const double round_us = (double)sh.h * sh.w * sh.E * 16.0 / 6.5e6;
-    long long lag = (long long)(chain_latency_us(sh) / (round_us > 0.01 ? round_us : 0.01)) + 3;
+    long long lag = (long long)(chain_latency_us(sh) / (round_us > 0.01 ? round_us : 0.01)) + 1;
     if (const char* env = getenv("FASTVIM_FUSED_LAG")) {
         const long long v = atoll(env);
         if (v >= 3 && v <= 64) lag = v;
