@@ -262,3 +262,35 @@ def test_host_entry_point_matches_device_entry_point():
     assert_close(y_host.numpy(), ref)
     dev = gpu_forward(p, 1, 3, intermediates=False)["y"]
     assert np.array_equal(dev, y_host.numpy())
+
+
+@pytest.mark.parametrize("path", ["staged", "fused"])
+def test_longest_pooled_sequence(path):
+    # T = 4096 pooled tokens (the largest the library takes): 256 scan chunks of 16 steps
+    p = rand_layer(500, B=1, h=4096, w=3, E=8, N=16, R=2, dir_flags=3)
+    got = gpu_forward(p, 0, 3, intermediates=False, path=path)
+    assert got["status"] == 0
+    ref = oracle.forward(p["x"], p["z"], p["A_log"], p["D"], p["W_x"], p["W_dt"], p["b_dt"], 0, 3)
+    assert_close(got["y"], ref)
+
+
+@pytest.mark.parametrize("h,w,E,N,R,pool_axis,dir_flags", [(1, 1, 4, 1, 1, 0, 3), (1, 7, 4, 1, 1, 1, 1),
+                                                          (9, 1, 8, 2, 1, 0, 2), (1, 9, 12, 3, 2, 0, 3)])
+def test_smallest_layers(h, w, E, N, R, pool_axis, dir_flags):
+    p = rand_layer(510 + h + w, B=3, h=h, w=w, E=E, N=N, R=R, dir_flags=dir_flags)
+    for path in ("staged", "fused"):
+        got = gpu_forward(p, pool_axis, dir_flags, intermediates=False, path=path)
+        assert got["status"] == 0
+        ref = oracle.forward(p["x"], p["z"], p["A_log"], p["D"], p["W_x"], p["W_dt"], p["b_dt"], pool_axis, dir_flags)
+        assert_close(got["y"], ref)
+
+
+def test_masked_largest_grid():
+    # a 1024 x 1024 grid (2^20 ids, the masked limit) with 300 kept tokens per sample
+    p = rand_layer(520, B=2, h=1024, w=1024, E=16, N=16, R=2, dir_flags=3, K=300)
+    got = gpu_forward(p, 1, 3, h=1024, w=1024)
+    assert got["status"] == 0
+    ref = oracle.forward_intermediates(p["x"], p["z"], p["A_log"], p["D"], p["W_x"], p["W_dt"], p["b_dt"], 1, 3,
+                                       keep_idx=p["keep_idx"], h=1024, w=1024)
+    assert np.array_equal(got["row_of"], ref["row_of"])
+    assert_close(got["y"], ref["y"])
