@@ -509,9 +509,12 @@ fv_status staged_back(const StagedChunk& c, char* ws, cudaStream_t st, EventMark
         })());
     } else {
         const int nkb = (sh.K + fv::kMaskEpiTokens - 1) / fv::kMaskEpiTokens;
+        const size_t msm = (size_t)sh.SL * sizeof(float4);
+        cudaError_t e = ensure_smem(fv::mask_epilogue_kernel, msm);
+        if (e != cudaSuccess) { note_cuda(e, "masked epilogue smem attribute"); return FV_ERR_CUDA; }
         FV_MARK_CALL(marks, st, ([&]() -> fv_status {
-            fv::mask_epilogue_kernel<<<sh.B * nkb, fv::kThreads, 0, st>>>(sh, c.a.x, c.a.z, ys, c.a.D,
-                                                                         (const int32_t*)(ws + c.L.row_of), c.a.y);
+            fv::mask_epilogue_kernel<<<sh.B * nkb, fv::kThreads, msm, st>>>(sh, c.a.x, c.a.z, ys, c.a.D,
+                                                                           (const int32_t*)(ws + c.L.row_of), c.a.y);
             FV_LAUNCH_CHECK("mask_epilogue_kernel");
             return FV_OK;
         })());

@@ -178,15 +178,17 @@ mask_pool_kernel(Shape sh, const float* __restrict__ x, const int32_t* __restric
         }
     } else {
         for (int slot = threadIdx.x; slot < SL; slot += kThreads) {
-            float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+            float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
             int p = p0;
-            for (; p + 1 < p1; p += 2) {
+            for (; p + 3 < p1; p += 4) {  // four kept tokens in flight
                 const float4 v0 = ld_stream(xb + (size_t)tok[p] * SL + slot);
                 const float4 v1 = ld_stream(xb + (size_t)tok[p + 1] * SL + slot);
-                f4_add(a0, v0); f4_add(a1, v1);
+                const float4 v2 = ld_stream(xb + (size_t)tok[p + 2] * SL + slot);
+                const float4 v3 = ld_stream(xb + (size_t)tok[p + 3] * SL + slot);
+                f4_add(a0, v0); f4_add(a1, v1); f4_add(a2, v2); f4_add(a3, v3);
             }
-            if (p < p1) f4_add(a0, ld_stream(xb + (size_t)tok[p] * SL + slot));
-            f4_add(a0, a1);
+            for (; p < p1; ++p) f4_add(a0, ld_stream(xb + (size_t)tok[p] * SL + slot));
+            f4_add(a0, a1); f4_add(a2, a3); f4_add(a0, a2);
             out[slot] = f4_scale(a0, scale);
         }
     }
@@ -195,9 +197,10 @@ mask_pool_kernel(Shape sh, const float* __restrict__ x, const int32_t* __restric
 // ------------------------------------------------------------------------------------------
 // Repeat + skip + gate: y = SiLU(z) * (ys[row] + (sum_k D_k) x), streamed with 128-bit accesses.
 // ------------------------------------------------------------------------------------------
+// SiLU(z) * (ys + (sum D) x) for four channels; SiLU with the SFU exp2 and reciprocal (silu_fast).
 __device__ __forceinline__ float4 gate4(const float4& xv, const float4& zv, const float4& ysv, const float4& dv) {
-    return make_float4(silu_f(zv.x) * fmaf(dv.x, xv.x, ysv.x), silu_f(zv.y) * fmaf(dv.y, xv.y, ysv.y),
-                       silu_f(zv.z) * fmaf(dv.z, xv.z, ysv.z), silu_f(zv.w) * fmaf(dv.w, xv.w, ysv.w));
+    return make_float4(silu_fast(zv.x) * fmaf(dv.x, xv.x, ysv.x), silu_fast(zv.y) * fmaf(dv.y, xv.y, ysv.y),
+                       silu_fast(zv.z) * fmaf(dv.z, xv.z, ysv.z), silu_fast(zv.w) * fmaf(dv.w, xv.w, ysv.w));
 }
 
 __device__ __forceinline__ float4 dsum4(const float* __restrict__ D, int nd, int SL, int slot) {
@@ -254,25 +257,49 @@ __global__ void __launch_bounds__(kThreads)
 mask_epilogue_kernel(Shape sh, const float* __restrict__ x, const float* __restrict__ z,
                      const float* __restrict__ ys, const float* __restrict__ D,
                      const int32_t* __restrict__ row_of, float* __restrict__ y) {
+    extern __shared__ float4 mdsum[];      // [SL] sum_k D_k
+    __shared__ int rows[kMaskEpiTokens];   // pooled row of each of the CTA's kept tokens
     const int nkb = (sh.K + kMaskEpiTokens - 1) / kMaskEpiTokens;
     const int b = blockIdx.x / nkb;
     const int k0 = (blockIdx.x - b * nkb) * kMaskEpiTokens;
     const int SL = sh.SL;
-    const float4* x4 = reinterpret_cast<const float4*>(x);
-    const float4* z4 = reinterpret_cast<const float4*>(z);
-    const float4* ys4 = reinterpret_cast<const float4*>(ys);
-    float4* y4 = reinterpret_cast<float4*>(y);
-    for (int f = threadIdx.x; f < kMaskEpiTokens * SL; f += kThreads) {
-        const int kk = f / SL, slot = f - kk * SL;
-        const int k = k0 + kk;
-        if (k >= sh.K) break;
-        const int r = row_of[(size_t)b * sh.K + k];
-        const size_t o = ((size_t)b * sh.K + k) * SL + slot;
-        float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (r >= 0)
-            res = gate4(ld_stream(x4 + o), ld_stream(z4 + o), ys4[((size_t)b * sh.T + r) * SL + slot],
-                        dsum4(D, sh.nd, SL, slot));
-        st_stream(y4 + o, res);
+    for (int slot = threadIdx.x; slot < SL; slot += kThreads) mdsum[slot] = dsum4(D, sh.nd, SL, slot);
+    if (threadIdx.x < kMaskEpiTokens) {
+        const int k = k0 + threadIdx.x;
+        rows[threadIdx.x] = k < sh.K ? row_of[(size_t)b * sh.K + k] : -1;
+    }
+    __syncthreads();
+    const int n = min(kMaskEpiTokens, sh.K - k0) * SL;  // float4 elements of the CTA's tokens
+    const float inv_sl = 1.f / (float)SL;
+    const size_t obase = ((size_t)b * sh.K + k0) * SL;  // the tokens are contiguous rows
+    const float4* x4 = reinterpret_cast<const float4*>(x) + obase;
+    const float4* z4 = reinterpret_cast<const float4*>(z) + obase;
+    const float4* ys4 = reinterpret_cast<const float4*>(ys) + (size_t)b * sh.T * SL;
+    float4* y4 = reinterpret_cast<float4*>(y) + obase;
+    const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int f0 = threadIdx.x; f0 < n; f0 += 2 * kThreads) {  // two elements per thread in flight
+        float4 xv[2], zv[2], yv[2];
+        int slot[2], r[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int f = f0 + u * kThreads;
+            r[u] = -1;
+            if (f < n) {
+                const int kk = (int)(((float)f + 0.5f) * inv_sl);  // f / SL (exact for f < 2^16)
+                slot[u] = f - kk * SL;
+                r[u] = rows[kk];
+                if (r[u] >= 0) {
+                    xv[u] = ld_stream(x4 + f);
+                    zv[u] = ld_stream(z4 + f);
+                    yv[u] = __ldcg(ys4 + (size_t)r[u] * SL + slot[u]);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int f = f0 + u * kThreads;
+            if (f < n) st_stream(y4 + f, r[u] >= 0 ? gate4(xv[u], zv[u], yv[u], mdsum[slot[u]]) : zero);
+        }
     }
 }
 
