@@ -437,7 +437,9 @@ fv_status staged_front(const StagedChunk& c, char* ws, unsigned* status, cudaStr
     float* xbar = (float*)(ws + c.L.xbar);
     if (sh.K == 0) {
         FV_MARK_CALL(marks, st, ([&]() -> fv_status {
-            fv::pool_dense_kernel<<<M, fv::kThreads, 0, st>>>(sh, c.a.x, xbar);
+            // a whole number of token groups of SL threads each (no idle threads)
+            const int threads = sh.SL <= fv::kThreads ? (fv::kThreads / sh.SL) * sh.SL : fv::kThreads;
+            fv::pool_dense_kernel<<<M, threads, 0, st>>>(sh, c.a.x, xbar);
             FV_LAUNCH_CHECK("pool_dense_kernel");
             return FV_OK;
         })());

@@ -20,17 +20,24 @@ namespace fv {
 // Sum of tokens s0, s0+G, s0+2G, ... < S of one float4 column; four loads in flight.
 __device__ __forceinline__ float4 sum_line(const float4* __restrict__ p, size_t st4, int s0, int G,
                                            int S) {
-    float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+    float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
     int s = s0;
-    for (; s + 3 * G < S; s += 4 * G) {
-        const float4 v0 = ld_stream(p + (size_t)s * st4);
-        const float4 v1 = ld_stream(p + (size_t)(s + G) * st4);
-        const float4 v2 = ld_stream(p + (size_t)(s + 2 * G) * st4);
-        const float4 v3 = ld_stream(p + (size_t)(s + 3 * G) * st4);
-        f4_add(a0, v0); f4_add(a1, v1); f4_add(a0, v2); f4_add(a1, v3);
+    for (; s + 7 * G < S; s += 8 * G) {  // eight tokens in flight
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = ld_stream(p + (size_t)(s + u * G) * st4);
+        f4_add(a0, v[0]); f4_add(a1, v[1]); f4_add(a2, v[2]); f4_add(a3, v[3]);
+        f4_add(a0, v[4]); f4_add(a1, v[5]); f4_add(a2, v[6]); f4_add(a3, v[7]);
+    }
+    if (s + 3 * G < S) {  // then four, for short lines
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = ld_stream(p + (size_t)(s + u * G) * st4);
+        f4_add(a0, v[0]); f4_add(a1, v[1]); f4_add(a2, v[2]); f4_add(a3, v[3]);
+        s += 4 * G;
     }
     for (; s < S; s += G) f4_add(a0, ld_stream(p + (size_t)s * st4));
-    f4_add(a0, a1);
+    f4_add(a0, a1); f4_add(a2, a3); f4_add(a0, a2);
     return a0;
 }
 
@@ -56,7 +63,7 @@ pool_dense_kernel(Shape sh, const float* __restrict__ x, float* __restrict__ xba
     float4* out = reinterpret_cast<float4*>(xbar + (size_t)bt * sh.E);
     const int SL = sh.SL;
     if (SL <= kThreads) {
-        const int G = kThreads / SL;
+        const int G = kThreads / SL;  // launched with G * SL threads
         const int slot = threadIdx.x % SL, g = threadIdx.x / SL;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         if (g < G) acc = sum_line(base + slot, st4, g, G, sh.S);
