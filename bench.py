@@ -41,13 +41,16 @@ REFERENCE_BUDGET_S = 150.0
 L2_BYTES = 126 * 1024 * 1024
 # Special-function (MUFU) lanes per SM per clock on sm_100: 4 per SM sub-partition.
 MUFU_PER_SM_CLK = 16
+# fp32 FMA lanes per SM per clock on sm_100 (4 sub-partitions x 32); 2 flops each.
+FFMA_PER_SM_CLK = 128
 
 
 def kernel_work(name: str, cfg, pool_axis: int):
     """(bound, algorithmic amount per step) of kernel `name` on workload `cfg` (all its launches in
     one step; a staged layer launches a kernel once per chunk of images):
     bytes for the streaming kernels (what the step must move at minimum), exp2 evaluations for
-    the scans (one per state, step, channel and direction), None for the rest."""
+    the scans (one per state, step, channel and direction), fp32 flops for the projection GEMM,
+    None for the rest."""
     tok = cfg.tokens_per_call()                       # grid tokens, or kept tokens when masked
     row = 4 * cfg.E                                   # one fp32 token row
     T = cfg.h if pool_axis == 0 else cfg.w
@@ -57,7 +60,15 @@ def kernel_work(name: str, cfg, pool_axis: int):
         return "hbm", 3 * row * tok                   # read x and z, write y (the fused launch: the layer)
     if name == "scan_seq_kernel":
         return "alu", cfg.B * T * cfg.E * cfg.N * cfg.nd
+    if name == "proj_gemm_kernel":
+        return "fma", 2 * cfg.B * T * cfg.E * cfg.nd * (cfg.R + 2 * cfg.N)
     return None, 0
+
+
+def ffma_peak_tflops(device_index: int, sm_max_mhz) -> float:
+    import torch
+    sms = torch.cuda.get_device_properties(device_index).multi_processor_count
+    return sms * FFMA_PER_SM_CLK * 2 * float(sm_max_mhz or 1965) * 1e6 / 1e12
 
 
 def mufu_peak_gops(device_index: int, sm_max_mhz) -> float:
@@ -411,6 +422,7 @@ def run_ours(a, cfg, pool_axis):
 
     total_k = sum(sum(v) for v in per_kernel.values())
     mufu_peak = mufu_peak_gops(local, clocks.summary().get("sm_max_mhz"))
+    fma_peak = ffma_peak_tflops(local, clocks.summary().get("sm_max_mhz"))
     kern = {}
     for n, v in per_kernel.items():
         avg_s = statistics.mean(v) / 1e3
@@ -421,6 +433,8 @@ def run_ours(a, cfg, pool_axis):
             ent.update(achieved=amount / avg_s / 1e9, unit="GB/s", frac=amount / avg_s / 1e9 / peak)
         elif bound == "alu":
             ent.update(achieved=amount / avg_s / 1e9, unit="G exp2/s", frac=amount / avg_s / 1e9 / mufu_peak)
+        elif bound == "fma":
+            ent.update(achieved=amount / avg_s / 1e12, unit="TFLOP/s fp32", frac=amount / avg_s / 1e12 / fma_peak)
         kern[n] = ent
     dom = max(kern, key=lambda n: kern[n]["share"])
     bound, amount = kernel_work(dom, cfg, pool_axis)
@@ -432,6 +446,12 @@ def run_ours(a, cfg, pool_axis):
                     "algorithmic_exp2_per_launch": amount,
                     "peak_source": f"derived: SMs x {MUFU_PER_SM_CLK} MUFU lanes/clk x max SM clock",
                     "note": "achieved = exp2 evaluations per launch / mean CUDA-event duration of the launch"}
+    elif bound == "fma":
+        roofline = {"bound": "alu", "kernel": dom, "achieved": dk["achieved"], "peak": fma_peak,
+                    "unit": "TFLOP/s fp32", "frac": dk["frac"], "traffic": recorded_traffic(dom, cfg.name),
+                    "algorithmic_flop_per_launch": amount,
+                    "peak_source": f"derived: SMs x {FFMA_PER_SM_CLK} FMA lanes/clk x 2 flop x max SM clock",
+                    "note": "achieved = flops per launch / mean CUDA-event duration of the launch"}
     else:
         roofline = {"bound": "hbm", "kernel": dom, "achieved": dk.get("achieved"), "peak": peak, "unit": "GB/s",
                     "frac": dk.get("frac"), "traffic": recorded_traffic(dom, cfg.name),
