@@ -381,12 +381,11 @@ __device__ __forceinline__ bool fused_pool(const Shape& sh, const FusedPlan& pl,
 // ---- Q: x_proj of pooled tokens [q*16, q*16+16) of image b ------------------------------------
 // u = W_x . xbar as a register-blocked fp32 GEMM (2 tokens x TN outputs per thread: TN = 3, 4 or
 // 6 for nd(R+2N) <= 96, 128 or 192 outputs; weight rows past nd(R+2N) are zero-filled), 32-channel
-// K-steps in a 5-, 4- or 3-stage cp.async pipeline.  Besides u, the task writes the scan-ready copies: B | C
-// of each token into its chunk-interleaved row, dt_low into a dense [T][R] block.
+// K-steps in a 5-, 4- or 3-stage cp.async pipeline.  The result goes to u (image-major blocks).
 template <int TN, int kQStages>
 __device__ __forceinline__ void fused_proj_t(const Shape& sh, const FusedPlan& pl, const FusedPtrs& p, int b, int q,
                                              float* smem) {
-    const int T = sh.T, E = sh.E, J = sh.J, NJ = sh.NJ, R = sh.R, N = sh.N;
+    const int T = sh.T, E = sh.E, J = sh.J, NJ = sh.NJ;
     constexpr int WROWS = 32 * TN;
     constexpr int TM = kQT / 8;
     const int tq0 = q * kQT;
