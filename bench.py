@@ -125,14 +125,20 @@ def load_peaks():
         return FALLBACK_HBM_GBS, "fallback (6.65 TB/s earlier pool measurement)"
 
 
-def kernel_source_hash():
+# Sources each recorded kernel is built from (the traffic record is void once any of them changes).
+KERNEL_SOURCES = {
+    "fused_layer_kernel": ("fastvim_ssm.cu", "fv_common.cuh", "fv_fused.cuh", "fv_scan.cuh"),
+}
+
+
+def kernel_source_hash(kernel=None):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "pooled_selective_scan_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode())
-                h.update(f.read())
+    names = KERNEL_SOURCES.get(kernel) or [n for n in os.listdir(csrc) if n.endswith((".cu", ".cuh"))]
+    for name in sorted(names):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -145,10 +151,8 @@ def recorded_traffic(kernel, cfg_name):
             j = json.load(f)
     except Exception:
         return None
-    if j.get("kernel_source_hash") != kernel_source_hash():
-        return None
     ent = j.get("kernels", {}).get(f"{cfg_name}/{kernel}")
-    if not ent:
+    if not ent or ent.get("kernel_source_hash") != kernel_source_hash(kernel):
         return None
     return ent.get("dram_bytes_per_full_launch")
 
