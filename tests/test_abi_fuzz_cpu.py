@@ -1,0 +1,165 @@
+"""Host-side fuzzing of the C ABI (no GPU; no pointer is ever dereferenced).
+
+Arguments are drawn as a layer the ABI accepts, then, in about half the draws, one field is
+broken in a way whose status the header fixes.  For accepted layers the workspace size equals the
+layout's total, every region is 256-byte aligned, disjoint from the others and large enough for
+what it holds, and the launch list matches the path the flags and the shape choose."""
+import ctypes
+
+import pytest
+
+pytest.importorskip("hypothesis")
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+from pooled_selective_scan_b200 import _native as nat  # noqa: E402
+from pooled_selective_scan_b200 import build as fvbuild  # noqa: E402
+from pooled_selective_scan_b200.ssm import POOL_H, POOL_W  # noqa: E402
+
+FAKE = 1 << 40          # fake device addresses, 16-byte aligned, never dereferenced
+SLOT = 1 << 50          # far apart: no two tensors alias at any drawn size
+MAX_N, MAX_J, MAX_T = 16, 96, 4096
+CTRL_WORDS = lambda B: 64 + 3 * B  # noqa: E731  header + 3 counters per image (fused control block)
+PTRS = ("x", "z", "A_log", "D", "W_x", "W_dt", "b_dt", "y")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    fvbuild.build()
+
+
+@st.composite
+def valid_layer(draw):
+    a = nat.FvSsmArgs()
+    a.B = draw(st.integers(0, 300))
+    a.h = draw(st.integers(1, 300))
+    a.w = draw(st.integers(1, 300))
+    a.E = draw(st.sampled_from([4, 8, 12, 64, 192, 384, 768, 1536, 4096]))
+    a.N = draw(st.integers(1, MAX_N))
+    a.R = draw(st.integers(1, MAX_J - 2 * a.N))
+    a.pool_axis = draw(st.sampled_from([POOL_W, POOL_H]))
+    a.dir_flags = draw(st.sampled_from([1, 2, 3]))
+    a.K = draw(st.integers(1, a.h * a.w)) if draw(st.booleans()) else 0
+    a.pool_scale = draw(st.sampled_from([0.0, 1.0, 0.25]))
+    a.flags = (draw(st.sampled_from([0, nat.FV_FLAG_PATH_STAGED, nat.FV_FLAG_PATH_FUSED]))
+               | draw(st.sampled_from([0, nat.FV_FLAG_ZOH_EXACT]))
+               | draw(st.sampled_from([0, nat.FV_FLAG_TRACE]))
+               | draw(st.sampled_from([0, nat.FV_FLAG_LAYERNORM])))
+    for i, name in enumerate(PTRS):
+        setattr(a, name, FAKE + i * SLOT)
+    if a.K:
+        a.keep_idx = FAKE + 9 * SLOT
+    if a.flags & nat.FV_FLAG_LAYERNORM:
+        a.ln_gamma, a.ln_beta, a.ln_eps = FAKE + 10 * SLOT, FAKE + 11 * SLOT, 1e-5
+    return a
+
+
+def _set(field, value):
+    return lambda a: setattr(a, field, value(a) if callable(value) else value)
+
+
+# (name, applies to, change, status the header gives)
+BREAKS = [
+    ("E not a multiple of 4", lambda a: True, _set("E", lambda a: a.E + 2), nat.FV_ERR_SHAPE),
+    ("no direction", lambda a: True, _set("dir_flags", 0), nat.FV_ERR_SHAPE),
+    ("unknown direction bit", lambda a: True, _set("dir_flags", lambda a: a.dir_flags | 4), nat.FV_ERR_SHAPE),
+    ("unknown pool axis", lambda a: True, _set("pool_axis", 2), nat.FV_ERR_SHAPE),
+    ("both paths forced", lambda a: True,
+     _set("flags", lambda a: a.flags | nat.FV_FLAG_PATH_STAGED | nat.FV_FLAG_PATH_FUSED), nat.FV_ERR_SHAPE),
+    ("unknown flag", lambda a: True, _set("flags", lambda a: a.flags | 32), nat.FV_ERR_SHAPE),
+    ("negative batch", lambda a: True, _set("B", -1), nat.FV_ERR_SHAPE),
+    ("K above the grid", lambda a: True, _set("K", lambda a: a.h * a.w + 1), nat.FV_ERR_SHAPE),
+    ("NaN pool scale", lambda a: True, _set("pool_scale", float("nan")), nat.FV_ERR_SHAPE),
+    ("d_state above the limit", lambda a: True, _set("N", MAX_N + 1), nat.FV_ERR_UNSUPPORTED),
+    ("R + 2N above the limit", lambda a: True, _set("R", lambda a: MAX_J - 2 * a.N + 1), nat.FV_ERR_UNSUPPORTED),
+    ("no A_log", lambda a: True, _set("A_log", None), nat.FV_ERR_NULL),
+    ("no x", lambda a: a.B > 0, _set("x", None), nat.FV_ERR_NULL),
+    ("no keep list", lambda a: a.K > 0 and a.B > 0, _set("keep_idx", None), nat.FV_ERR_NULL),
+    ("keep list without K", lambda a: a.K == 0, _set("keep_idx", FAKE + 9 * SLOT), nat.FV_ERR_SHAPE),
+    ("LayerNorm without gamma", lambda a: a.flags & nat.FV_FLAG_LAYERNORM, _set("ln_gamma", None), nat.FV_ERR_NULL),
+    ("LayerNorm eps 0", lambda a: a.flags & nat.FV_FLAG_LAYERNORM, _set("ln_eps", 0.0), nat.FV_ERR_SHAPE),
+    ("gamma without the flag", lambda a: not a.flags & nat.FV_FLAG_LAYERNORM,
+     _set("ln_gamma", FAKE + 10 * SLOT), nat.FV_ERR_SHAPE),
+    ("misaligned z", lambda a: True, _set("z", FAKE + 1 * SLOT + 4), nat.FV_ERR_ALIGN),
+    ("misaligned W_x", lambda a: True, _set("W_x", FAKE + 4 * SLOT + 8), nat.FV_ERR_ALIGN),
+    ("y aliases x", lambda a: a.B > 0, _set("y", FAKE), nat.FV_ERR_ALIAS),
+    ("y overlaps z", lambda a: a.B > 0, _set("y", FAKE + SLOT + 16), nat.FV_ERR_ALIAS),
+]
+
+
+def _check_layout(lib, a):
+    size = lib.fastvim_ssm_workspace_size(ctypes.byref(a))
+    L = nat.FvWsLayout()
+    assert lib.fastvim_ssm_workspace_layout(ctypes.byref(a), ctypes.byref(L)) == nat.FV_OK
+    assert size == L.total_bytes
+    B, E = a.B, a.E
+    T = a.h if a.pool_axis == POOL_W else a.w
+    assert (L.T, L.S, L.nd) == (T, a.w + a.h - T, bin(a.dir_flags).count("1"))
+    ub = -(-T * (a.R + 2 * a.N) // 32) * 32
+    regions = [(L.status, 8), (L.xbar, B * T * E * 4), (L.u, B * L.nd * ub * 4), (L.ys, B * T * E * 4)]
+    if a.K:
+        assert L.ctrl == 0 and L.trace == 0
+        regions += [(L.row_of, B * a.K * 4), (L.row_off, B * (T + 1) * 4), (L.row_tok, B * a.K * 4)]
+    else:
+        assert L.row_of == L.row_off == L.row_tok == 0
+        regions.append((L.ctrl, CTRL_WORDS(B) * 4))
+        if L.trace:
+            assert a.flags & nat.FV_FLAG_TRACE and L.trace_records > 0
+            regions.append((L.trace, L.trace_records * 32))
+    regions.sort()
+    end = 0
+    for off, n in regions:
+        assert off % 256 == 0 and off >= end, (off, end)
+        end = off + n
+    assert end <= L.total_bytes < end + 256 * len(regions)
+
+
+def _check_launches(lib, a):
+    n = lib.fastvim_ssm_launch_count(ctypes.byref(a))
+    names = [lib.fastvim_ssm_launch_name(ctypes.byref(a), i).decode() for i in range(n)]
+    assert lib.fastvim_ssm_launch_name(ctypes.byref(a), n).decode() == ""
+    if a.B == 0:
+        assert n == 0
+        return
+    if n == 0:
+        # only a forced fused path on a layer it cannot run (masked, or token rows wider than half
+        # a 24 KB ring stage) has no launches: the forward call refuses it with FV_ERR_UNSUPPORTED
+        assert a.flags & nat.FV_FLAG_PATH_FUSED
+        assert a.K > 0 or a.E * 4 > 12 * 1024
+        return
+    if names == ["fused_layer_kernel"]:
+        assert a.K == 0 and not a.flags & nat.FV_FLAG_PATH_STAGED
+        return
+    assert not a.flags & nat.FV_FLAG_PATH_FUSED
+    assert n >= 4 and "fused_layer_kernel" not in names
+    last = {True: "ln_epilogue_kernel", False: "mask_epilogue_kernel" if a.K else "epilogue_dense_kernel"}
+    assert names[-1] == last[bool(a.flags & nat.FV_FLAG_LAYERNORM)]
+    assert "proj_gemm_kernel" in names and any(k.startswith("scan") for k in names)
+    if a.K:
+        assert names[0].startswith("mask_")
+
+
+@settings(max_examples=600, deadline=None)
+@given(valid_layer(), st.integers(-len(BREAKS), len(BREAKS) - 1))
+def test_validation_layout_and_launch_list(a, pick):
+    lib = nat.lib()
+    base = lib.fastvim_ssm_validate(ctypes.byref(a))
+    T = a.h if a.pool_axis == POOL_W else a.w
+    limited = T > MAX_T or (a.K and a.h * a.w > (1 << 20))
+    assert base == (nat.FV_ERR_UNSUPPORTED if limited else nat.FV_OK)
+    if base != nat.FV_OK:
+        assert lib.fastvim_ssm_workspace_size(ctypes.byref(a)) == 0
+        return
+    if pick < 0:  # keep the layer as drawn
+        _check_layout(lib, a)
+        _check_launches(lib, a)
+        return
+    name, applies, change, want = BREAKS[pick]
+    if not applies(a):
+        return
+    change(a)
+    assert lib.fastvim_ssm_validate(ctypes.byref(a)) == want, name
+    if want in (nat.FV_ERR_SHAPE, nat.FV_ERR_UNSUPPORTED) and name not in (
+            "keep list without K", "gamma without the flag"):
+        # shape errors: no workspace, no launches
+        assert lib.fastvim_ssm_workspace_size(ctypes.byref(a)) == 0
+        assert lib.fastvim_ssm_launch_count(ctypes.byref(a)) == 0
