@@ -19,6 +19,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "fastvim_oracle.c")
+_GRAD_SRC = os.path.join(_HERE, "fastvim_oracle_grad.c")
 _HDR = os.path.join(_HERE, "fastvim_oracle.h")
 _LIB_PATH = os.path.join(_HERE, "libfastvim_oracle.so")
 
@@ -32,10 +33,11 @@ _lib = None
 
 def build(force: bool = False) -> str:
     """Compile the oracle into ``libfastvim_oracle.so`` (gcc, -O2, OpenMP over images)."""
-    newest_src = max(os.path.getmtime(_SRC), os.path.getmtime(_HDR))
+    srcs = [_SRC, _GRAD_SRC]
+    newest_src = max(os.path.getmtime(p) for p in srcs + [_HDR])
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < newest_src:
         tmp = _LIB_PATH + f".tmp{os.getpid()}"
-        cmd = ["gcc", "-std=c99", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"]
+        cmd = ["gcc", "-std=c99", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", tmp, *srcs, "-lm"]
         subprocess.run(cmd, check=True)
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
@@ -59,6 +61,8 @@ def _load():
                 "fvo_gate_dense": [P, P, P, P, I, I, I, I, I, I, P, P, Dbl, P],
                 "fvo_gate_masked": [P, P, P, P, P, I, I, I, I, I, P, P, Dbl, P],
                 "fvo_forward": [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, U, Dbl, I, P, P, Dbl, I, P],
+                "fvo_backward": [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, U, Dbl, I, P, I,
+                                 P, P, P, P, P, P, P],
             }
             for name, argtypes in sigs.items():
                 fn = getattr(lib, name)
@@ -262,4 +266,38 @@ def forward_intermediates(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis, dir_flags,
     else:
         y = gate_masked(x, z, ys, D, out["row_of"], ln_gamma, ln_beta, ln_eps)
     out.update(xbar=xbar, u=u, delta=delta, ys=ys, y=y)
+    return out
+
+
+def backward(x, z, A_log, D, W_x, W_dt, b_dt, dy, pool_axis, dir_flags, keep_idx=None, h=None, w=None,
+             pool_scale=1.0, zoh_exact=False, nthreads=1, allow_bad_index=False):
+    """The gradient of the layer for the upstream gradient dy (layout of y), image by image.
+
+    Returns a dict of fp64 arrays: dx, dz (layouts of x, z) and the parameter gradients summed
+    over the batch, dA_log, dD, dW_x, dW_dt, db_dt (layouts of the parameters); with
+    allow_bad_index, also the status under "status".
+    """
+    x, z, dy = _f32(x), _f32(z), _f32(dy)
+    A_log, D, W_x, W_dt, b_dt = map(_f32, (A_log, D, W_x, W_dt, b_dt))
+    nd, E, N = A_log.shape
+    R = W_dt.shape[2]
+    if keep_idx is None:
+        B, h, w, E2 = x.shape
+        K = 0
+        idx = None
+    else:
+        B, K, E2 = x.shape
+        idx = _i32(keep_idx)
+        assert h is not None and w is not None and idx.shape == (B, K)
+    assert E2 == E and z.shape == x.shape and dy.shape == x.shape and nd == nd_of(dir_flags)
+    out = {"dx": np.empty(x.shape), "dz": np.empty(x.shape), "dA_log": np.empty(A_log.shape),
+           "dD": np.empty(D.shape), "dW_x": np.empty(W_x.shape), "dW_dt": np.empty(W_dt.shape),
+           "db_dt": np.empty(b_dt.shape)}
+    st = _load().fvo_backward(_p(x), _p(z), _p(A_log), _p(D), _p(W_x), _p(W_dt), _p(b_dt), _p(idx), B, h, w, E,
+                              N, R, K, pool_axis, int(dir_flags), float(pool_scale), int(bool(zoh_exact)), _p(dy),
+                              int(nthreads), *(_p(out[k]) for k in ("dx", "dz", "dA_log", "dD", "dW_x", "dW_dt",
+                                                                    "db_dt")))
+    _check(st, "backward", allow=(FVO_BAD_INDEX,) if allow_bad_index else ())
+    if allow_bad_index:
+        out["status"] = st
     return out

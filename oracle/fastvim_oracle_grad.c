@@ -1,0 +1,290 @@
+/*
+ * fastvim_oracle_grad.c -- fp64 CPU oracle of the gradient of the FastVim SSM layer.
+ *
+ * TEST INFRASTRUCTURE, NOT PRODUCT CODE: only the test suite may call it.  The pages train
+ * FastVim end to end (gptget.net summary of 2502.00594, "实验结果": faster pre-training and
+ * fine-tuning) but state no backward rule, so this file takes the plainest one: the exact
+ * derivative of the forward definition in fastvim_oracle.c, by the chain rule, one forward step
+ * at a time in reverse order (gate, repeat + skip, scans, dt_proj + softplus, x_proj, pooling).
+ * Plain loops in fp64, every forward intermediate recomputed with the forward oracle's own
+ * functions.  The post-SSM LayerNorm is not covered (the GPU backward does not take it).
+ *
+ * Given dy = dL/dy for a scalar loss L, it returns dL/dx, dL/dz (same layout as x, z) and the
+ * parameter gradients summed over the batch: dA_log [nd][E][N], dD [nd][E], dW_x [nd][R+2N][E],
+ * dW_dt [nd][E][R], db_dt [nd][E].
+ *
+ * Adjoint of one scan (direction slot k, channel e, state n; "prev" and "next" are the
+ * neighbouring steps in that direction's scan order, h_prev = 0 at its first step):
+ *   forward   h_t = Abar_t h_prev + q_t,  Abar_t = exp(Delta_t A),  A = -exp(A_log)
+ *             q_t = Delta_t B_t xbar_t (Euler)  or  (Abar_t - 1)/A B_t xbar_t (exact ZOH)
+ *             ys_t += C_t h_t
+ *   adjoint   lam_t = C_t dys_t + Abar_next lam_next   (lam = dL/dh_t, zero past the last step)
+ *             dC_t += dys_t h_t,   dAbar_t = lam_t h_prev,   dq_t = lam_t
+ * and the chain rule through Abar_t and q_t gives dDelta_t, dA, dB_t and dxbar_t.
+ */
+#include "fastvim_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static int g_popcount2(unsigned f) { return (int)((f & 1u) != 0) + (int)((f & 2u) != 0); }
+
+static double sigmoid(double v) { return 1.0 / (1.0 + exp(-v)); }
+
+typedef struct {
+    int h, w, E, N, R, K, T, S, J, nd;
+    int pool_axis, zoh_exact;
+    unsigned dir_flags;
+    double pool_scale;
+} gshape;
+
+/* Parameter gradients of one image (added into the caller's sums afterwards). */
+typedef struct {
+    double *dA_log, *dD, *dW_x, *dW_dt, *db_dt;
+} gparams;
+
+/* Step 1 of the reverse pass, one token: y = SiLU(z) s with s = ys_row + (sum_k D[k]) x.
+ * dz = dy s SiLU'(z), SiLU'(z) = sig(z) (1 + z (1 - sig(z))); ds = dy SiLU(z);
+ * ds feeds dys (the repeat's adjoint sums over the repeated tokens), dx (skip) and dD. */
+static void gate_token_grad(const float* x, const float* z, const float* dy, const double* ysr, const float* D,
+                            const gshape* g, double* dysr, double* dx, double* dz, double* dD)
+{
+    for (int e = 0; e < g->E; ++e) {
+        double Dsum = 0.0;
+        for (int k = 0; k < g->nd; ++k) Dsum += (double)D[(size_t)k * g->E + e];
+        const double s = ysr[e] + Dsum * (double)x[e];
+        const double zz = (double)z[e], sg = sigmoid(zz);
+        const double ds = (double)dy[e] * zz * sg;
+        dz[e] = (double)dy[e] * s * sg * (1.0 + zz * (1.0 - sg));
+        dysr[e] += ds;
+        dx[e] = ds * Dsum;
+        for (int k = 0; k < g->nd; ++k) dD[(size_t)k * g->E + e] += ds * (double)x[e];
+    }
+}
+
+/* Step 2: the adjoint of every scan of one image.  Reads xbar [T][E], delta [nd][T][E],
+ * u [nd][T][J], dys [T][E]; adds into ddelta [nd][T][E], du [nd][T][J] (the B and C slots),
+ * dxbar [T][E] and gp->dA_log.  hist: T doubles of scratch. */
+static void scan_grad(const double* xbar, const double* delta, const double* u, const double* dys,
+                      const float* A_log, const gshape* g, double* ddelta, double* du, double* dxbar,
+                      gparams* gp, double* hist)
+{
+    const int T = g->T, E = g->E, N = g->N, R = g->R, J = g->J;
+    int k = 0;
+    for (unsigned dir = FVO_FWD; dir <= FVO_BWD; dir <<= 1) {
+        if (!(g->dir_flags & dir)) continue;
+        const double* dl = delta + (size_t)k * T * E;
+        const double* uk = u + (size_t)k * T * J;
+        double* ddl = ddelta + (size_t)k * T * E;
+        double* duk = du + (size_t)k * T * J;
+        for (int e = 0; e < E; ++e)
+            for (int n = 0; n < N; ++n) {
+                const double A = -exp((double)A_log[((size_t)k * E + e) * N + n]);
+                /* forward: the state after every step, stored at its own t */
+                double hs = 0.0;
+                for (int step = 0; step < T; ++step) {
+                    const int t = (dir == FVO_FWD) ? step : T - 1 - step;
+                    const double dt = dl[(size_t)t * E + e], Bn = uk[(size_t)t * J + R + n];
+                    const double Abar = exp(dt * A);
+                    const double q = (g->zoh_exact ? (Abar - 1.0) / A : dt) * Bn * xbar[(size_t)t * E + e];
+                    hs = Abar * hs + q;
+                    hist[t] = hs;
+                }
+                /* reverse */
+                double lam = 0.0, Abar_next = 0.0, dA = 0.0;
+                for (int step = T - 1; step >= 0; --step) {
+                    const int t = (dir == FVO_FWD) ? step : T - 1 - step;
+                    const int tp = (dir == FVO_FWD) ? t - 1 : t + 1;
+                    const double hprev = step > 0 ? hist[tp] : 0.0;
+                    const double dt = dl[(size_t)t * E + e];
+                    const double Bn = uk[(size_t)t * J + R + n], Cn = uk[(size_t)t * J + R + N + n];
+                    const double xb = xbar[(size_t)t * E + e], dyt = dys[(size_t)t * E + e];
+                    const double Abar = exp(dt * A);
+                    lam = Cn * dyt + Abar_next * lam;
+                    duk[(size_t)t * J + R + N + n] += dyt * hist[t];
+                    /* through Abar_t = exp(dt A): dAbar = lam hprev */
+                    double d_dt = lam * hprev * Abar * A;
+                    dA += lam * hprev * Abar * dt;
+                    if (g->zoh_exact) {
+                        /* q = (Abar - 1)/A B xb: dq/ddt = Abar B xb, dq/dA = B xb (dt Abar A - (Abar - 1)) / A^2 */
+                        const double c = (Abar - 1.0) / A;
+                        d_dt += lam * Abar * Bn * xb;
+                        dA += lam * Bn * xb * (dt * Abar * A - (Abar - 1.0)) / (A * A);
+                        duk[(size_t)t * J + R + n] += lam * c * xb;
+                        dxbar[(size_t)t * E + e] += lam * c * Bn;
+                    } else {
+                        /* q = dt B xb */
+                        d_dt += lam * Bn * xb;
+                        duk[(size_t)t * J + R + n] += lam * dt * xb;
+                        dxbar[(size_t)t * E + e] += lam * dt * Bn;
+                    }
+                    ddl[(size_t)t * E + e] += d_dt;
+                    Abar_next = Abar;
+                }
+                /* A = -exp(A_log): dA/dA_log = A */
+                gp->dA_log[((size_t)k * E + e) * N + n] += dA * A;
+            }
+        ++k;
+    }
+}
+
+/* Steps 3 and 4: Delta = softplus(v), v = b_dt + W_dt dt_low, so dv = dDelta sig(v); then
+ * u = W_x xbar.  Adds into du (the dt_low slots), dxbar, dW_dt, db_dt and dW_x. */
+static void proj_grad(const double* xbar, const double* u, const double* ddelta, const float* W_x,
+                      const float* W_dt, const float* b_dt, const gshape* g, double* du, double* dxbar,
+                      gparams* gp)
+{
+    const int T = g->T, E = g->E, R = g->R, J = g->J;
+    for (int k = 0; k < g->nd; ++k)
+        for (int t = 0; t < T; ++t) {
+            const double* um = u + ((size_t)k * T + t) * J;
+            double* dum = du + ((size_t)k * T + t) * J;
+            for (int e = 0; e < E; ++e) {
+                double v = (double)b_dt[(size_t)k * E + e];
+                for (int r = 0; r < R; ++r) v += (double)W_dt[((size_t)k * E + e) * R + r] * um[r];
+                const double dv = ddelta[((size_t)k * T + t) * E + e] * sigmoid(v);
+                gp->db_dt[(size_t)k * E + e] += dv;
+                for (int r = 0; r < R; ++r) {
+                    gp->dW_dt[((size_t)k * E + e) * R + r] += dv * um[r];
+                    dum[r] += (double)W_dt[((size_t)k * E + e) * R + r] * dv;
+                }
+            }
+            for (int j = 0; j < J; ++j)
+                for (int e = 0; e < E; ++e) {
+                    gp->dW_x[((size_t)k * J + j) * E + e] += dum[j] * xbar[(size_t)t * E + e];
+                    dxbar[(size_t)t * E + e] += (double)W_x[((size_t)k * J + j) * E + e] * dum[j];
+                }
+        }
+}
+
+/* One image.  x, z, dy, dx, dz point at the image; keep (masked) at its K ids. */
+static int backward_one(const float* x, const float* z, const float* dy, const float* A_log, const float* D,
+                        const float* W_x, const float* W_dt, const float* b_dt, const int32_t* keep,
+                        const gshape* g, double* dx, double* dz, gparams* gp)
+{
+    const int T = g->T, E = g->E, J = g->J, nd = g->nd, K = g->K;
+    const size_t tok = keep ? (size_t)K : (size_t)g->h * g->w;
+    double* xbar = (double*)calloc((size_t)T * E, sizeof(double));
+    double* u = (double*)calloc((size_t)nd * T * J, sizeof(double));
+    double* delta = (double*)calloc((size_t)nd * T * E, sizeof(double));
+    double* ys = (double*)calloc((size_t)T * E, sizeof(double));
+    double* dys = (double*)calloc((size_t)T * E, sizeof(double));
+    double* ddelta = (double*)calloc((size_t)nd * T * E, sizeof(double));
+    double* du = (double*)calloc((size_t)nd * T * J, sizeof(double));
+    double* dxbar = (double*)calloc((size_t)T * E, sizeof(double));
+    double* hist = (double*)calloc((size_t)T, sizeof(double));
+    int32_t* row_of = (int32_t*)calloc((size_t)(K > 0 ? K : 1), sizeof(int32_t));
+    int32_t* row_off = (int32_t*)calloc((size_t)T + 1, sizeof(int32_t));
+    int32_t* row_tok = (int32_t*)calloc((size_t)(K > 0 ? K : 1), sizeof(int32_t));
+    int st = FVO_NO_MEMORY, idx_status = FVO_OK;
+    if (!(xbar && u && delta && ys && dys && ddelta && du && dxbar && hist && row_of && row_off && row_tok))
+        goto done;
+    /* the forward intermediates */
+    if (keep) {
+        idx_status = fvo_mask_rows(keep, 1, K, g->h, g->w, g->pool_axis, row_of, row_off, row_tok);
+        if (idx_status != FVO_OK && idx_status != FVO_BAD_INDEX) { st = idx_status; goto done; }
+        st = fvo_pool_masked(x, row_off, row_tok, 1, K, T, g->S, E, g->pool_scale, xbar);
+    } else {
+        st = fvo_pool(x, 1, g->h, g->w, E, g->pool_axis, g->pool_scale, xbar);
+    }
+    if (st) goto done;
+    if ((st = fvo_proj(xbar, 1, T, E, nd, g->R, g->N, W_x, W_dt, b_dt, u, delta))) goto done;
+    if ((st = fvo_scan(xbar, delta, u, A_log, 1, T, E, nd, g->R, g->N, g->dir_flags, g->zoh_exact, ys))) goto done;
+    /* 1: gate, skip and the repeat (a token whose id was rejected has no output and no gradient) */
+    for (size_t m = 0; m < tok; ++m) {
+        int t;
+        if (keep) {
+            t = row_of[m];
+            if (t < 0) {
+                for (int e = 0; e < E; ++e) dx[m * E + e] = dz[m * E + e] = 0.0;
+                continue;
+            }
+        } else {
+            const int i = (int)(m / (size_t)g->w), j = (int)(m % (size_t)g->w);
+            t = g->pool_axis == FVO_POOL_W ? i : j;
+        }
+        gate_token_grad(x + m * E, z + m * E, dy + m * E, ys + (size_t)t * E, D, g, dys + (size_t)t * E,
+                        dx + m * E, dz + m * E, gp->dD);
+    }
+    /* 2: scans; 3, 4: projections */
+    scan_grad(xbar, delta, u, dys, A_log, g, ddelta, du, dxbar, gp, hist);
+    proj_grad(xbar, u, ddelta, W_x, W_dt, b_dt, g, du, dxbar, gp);
+    /* 5: pooling, xbar_t = pool_scale / S * (sum of the tokens of row t) */
+    for (size_t m = 0; m < tok; ++m) {
+        int t;
+        if (keep) {
+            t = row_of[m];
+            if (t < 0) continue;
+        } else {
+            const int i = (int)(m / (size_t)g->w), j = (int)(m % (size_t)g->w);
+            t = g->pool_axis == FVO_POOL_W ? i : j;
+        }
+        for (int e = 0; e < E; ++e) dx[m * E + e] += g->pool_scale / (double)g->S * dxbar[(size_t)t * E + e];
+    }
+    st = idx_status;
+done:
+    free(xbar); free(u); free(delta); free(ys); free(dys); free(ddelta); free(du); free(dxbar); free(hist);
+    free(row_of); free(row_off); free(row_tok);
+    return st;
+}
+
+int fvo_backward(const float* x, const float* z, const float* A_log, const float* D, const float* W_x,
+                 const float* W_dt, const float* b_dt, const int32_t* keep_idx, int B, int h, int w, int E,
+                 int N, int R, int K, int pool_axis, unsigned dir_flags, double pool_scale, int zoh_exact,
+                 const float* dy, int nthreads, double* dx, double* dz, double* dA_log, double* dD,
+                 double* dW_x, double* dW_dt, double* db_dt)
+{
+    const int nd = g_popcount2(dir_flags);
+    if (B < 0 || h <= 0 || w <= 0 || E <= 0 || N <= 0 || R <= 0 || nd < 1 || (dir_flags & ~3u) != 0 ||
+        (pool_axis != FVO_POOL_W && pool_axis != FVO_POOL_H) || (keep_idx && (K < 0 || K > h * w)))
+        return FVO_BAD_SHAPE;
+    gshape g;
+    g.h = h; g.w = w; g.E = E; g.N = N; g.R = R; g.K = keep_idx ? K : 0;
+    g.T = pool_axis == FVO_POOL_W ? h : w;
+    g.S = pool_axis == FVO_POOL_W ? w : h;
+    g.J = R + 2 * N; g.nd = nd; g.pool_axis = pool_axis; g.zoh_exact = zoh_exact;
+    g.dir_flags = dir_flags; g.pool_scale = pool_scale;
+    const size_t nA = (size_t)nd * E * N, nDv = (size_t)nd * E, nWx = (size_t)nd * g.J * E,
+                 nWdt = (size_t)nd * E * R;
+    memset(dA_log, 0, nA * sizeof(double));
+    memset(dD, 0, nDv * sizeof(double));
+    memset(dW_x, 0, nWx * sizeof(double));
+    memset(dW_dt, 0, nWdt * sizeof(double));
+    memset(db_dt, 0, nDv * sizeof(double));
+    const size_t tok = keep_idx ? (size_t)K : (size_t)h * w;
+    int status = FVO_OK;
+    if (nthreads < 1) nthreads = 1;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads) if (nthreads > 1)
+#endif
+    for (int b = 0; b < B; ++b) {
+        gparams gp;
+        double* buf = (double*)calloc(nA + 2 * nDv + nWx + nWdt, sizeof(double));
+        int st = FVO_NO_MEMORY;
+        if (buf) {
+            gp.dA_log = buf; gp.dD = buf + nA; gp.db_dt = gp.dD + nDv; gp.dW_x = gp.db_dt + nDv;
+            gp.dW_dt = gp.dW_x + nWx;
+            st = backward_one(x + (size_t)b * tok * E, z + (size_t)b * tok * E, dy + (size_t)b * tok * E, A_log, D,
+                              W_x, W_dt, b_dt, keep_idx ? keep_idx + (size_t)b * K : NULL, &g,
+                              dx + (size_t)b * tok * E, dz + (size_t)b * tok * E, &gp);
+        }
+#ifdef _OPENMP
+#pragma omp critical
+#endif
+        {
+            if (buf) {
+                for (size_t i = 0; i < nA; ++i) dA_log[i] += gp.dA_log[i];
+                for (size_t i = 0; i < nDv; ++i) { dD[i] += gp.dD[i]; db_dt[i] += gp.db_dt[i]; }
+                for (size_t i = 0; i < nWx; ++i) dW_x[i] += gp.dW_x[i];
+                for (size_t i = 0; i < nWdt; ++i) dW_dt[i] += gp.dW_dt[i];
+            }
+            if (st != FVO_OK && (status == FVO_OK || status == FVO_BAD_INDEX)) status = st;
+        }
+        free(buf);
+    }
+    return status;
+}
