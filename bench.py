@@ -17,6 +17,10 @@ CUDA-event time.  Rank 0 prints one JSON line.
 
 --impl reference times the fp64 CPU oracle on the host cores instead (rank 0 only), on a bounded
 sample of images of the same workload per step.
+
+--grad times a training step of the layer instead: the forward call and then the gradient call
+(fastvim_ssm_backward: dx, dz and the parameter gradients for a seeded upstream gradient dy) over
+the same batch, and prints its own line for that.
 """
 from __future__ import annotations
 
@@ -62,6 +66,23 @@ def kernel_work(name: str, cfg, pool_axis: int):
         return "alu", cfg.B * T * cfg.E * cfg.N * cfg.nd
     if name == "proj_gemm_kernel":
         return "fma", 2 * cfg.B * T * cfg.E * cfg.nd * (cfg.R + 2 * cfg.N)
+    # the gradient's kernels
+    if name in ("bwd_gate_dense_kernel", "bwd_gate_masked_kernel"):
+        return "hbm", 5 * row * tok                   # read x, z, dy; write dz and dx
+    if name == "bwd_pool_dense_kernel":
+        return "hbm", 2 * row * tok                   # dx read and written back (+ the pooled share)
+    if name == "bwd_pool_masked_kernel":
+        return "hbm", 2 * row * tok
+    if name == "bwd_scan_kernel":
+        return "alu", cfg.B * T * cfg.E * cfg.N * cfg.nd   # one exp2 per state and step (the minimum)
+    if name.startswith("bwd_gemm_kernel"):
+        J = cfg.R + 2 * cfg.N
+        M = cfg.B * T
+        flops = {"bwd_gemm_kernel:dt_low": 2 * M * cfg.E * cfg.R * cfg.nd,
+                 "bwd_gemm_kernel:W_dt": 2 * M * cfg.E * (cfg.R + 1) * cfg.nd,
+                 "bwd_gemm_kernel:W_x": 2 * M * cfg.E * J * cfg.nd,
+                 "bwd_gemm_kernel:xbar": 2 * M * cfg.E * J * cfg.nd}
+        return "fma", flops.get(name, 0)
     return None, 0
 
 
@@ -94,6 +115,8 @@ def parse(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--grad", action="store_true",
+                    help="time a training step: the forward call, then the gradient call on its workspace")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -520,6 +543,142 @@ def run_ours(a, cfg, pool_axis):
     return 0
 
 
+def run_grad(a, cfg, pool_axis):
+    """One step = the forward call + the gradient call over the batch (a training step of the
+    layer), inputs and dy resident in HBM; 1 GPU."""
+    import torch
+
+    from pooled_selective_scan_b200 import build as fvbuild
+    from pooled_selective_scan_b200 import ssm, workload
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the layer has no CPU path)")
+    world, rank, local = dist_env()
+    if world > 1:
+        raise SystemExit("--grad runs on one GPU")
+    if not os.path.exists(os.path.join(ROOT, "pooled_selective_scan_b200", "libfastvim_ssm.so")):
+        fvbuild.build()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    t = workload.layer_tensors(cfg, dev)
+    dy = workload.upstream_grad(cfg, dev)
+    keep = t.get("keep_idx")
+    shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, cfg.dir_flags, keep, cfg.h, cfg.w, path=a.path)
+    y = torch.empty_like(t["x"])
+    fws = ssm.alloc_workspace(shape, dev)
+    bws = torch.empty(ssm.backward_workspace_size(shape), dtype=torch.uint8, device=dev)
+    grads = {"dx": torch.empty_like(t["x"]), "dz": torch.empty_like(t["z"])}
+    for n in ("A_log", "D", "W_x", "W_dt", "b_dt"):
+        grads["d" + n] = torch.empty_like(t[n])
+    stream = torch.cuda.current_stream(dev)
+    fwd = ssm.BoundForward(shape, t, y, fws, stream)
+    bwd = ssm.BoundBackward(shape, t, dy, grads, fws, bws, stream)
+    names = ssm.launch_names(shape) + bwd.names
+    nf, nl = fwd.n_launch, len(names)
+    for _ in range(a.warmup):
+        fwd.run()
+        bwd.run()
+    torch.cuda.synchronize(dev)
+    if ssm.device_status(fws) != 0:
+        raise SystemExit("device status reported an error during warm-up")
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nl)] for _ in range(a.steps)]
+    for evs in events:
+        for e in evs:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
+    alg_bytes = cfg.algorithmic_bytes_per_call()
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if alg_bytes < 2 * L2_BYTES else None
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for i in range(a.steps):
+        if flush is not None:
+            flush.fill_(float(i))
+        fwd.run_events(events[i][:2 * nf])
+        bwd.run_events(events[i][2 * nf:])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.stop()
+    if flush is None:
+        ms = start.elapsed_time(end)
+    else:
+        ms = sum(evs[0].elapsed_time(evs[2 * nl - 1]) for evs in events)
+    per_kernel = {n: [] for n in dict.fromkeys(names)}
+    for evs in events:
+        step = {n: 0.0 for n in per_kernel}
+        for j, n in enumerate(names):
+            step[n] += evs[2 * j].elapsed_time(evs[2 * j + 1])
+        for n, v in step.items():
+            per_kernel[n].append(v)
+    tokens = cfg.tokens_per_call()
+    peak, peak_src = load_peaks()
+    mufu_peak = mufu_peak_gops(local, clocks.summary().get("sm_max_mhz"))
+    fma_peak = ffma_peak_tflops(local, clocks.summary().get("sm_max_mhz"))
+    total_k = sum(sum(v) for v in per_kernel.values())
+    kern = {}
+    for n, v in per_kernel.items():
+        avg_s = statistics.mean(v) / 1e3
+        bound, amount = kernel_work(n, cfg, pool_axis)
+        ent = {"launches_per_step": names.count(n), "us_per_step": avg_s * 1e6, "share": sum(v) / total_k,
+               "bound": bound}
+        if bound == "hbm":
+            ent.update(achieved=amount / avg_s / 1e9, unit="GB/s", frac=amount / avg_s / 1e9 / peak)
+        elif bound == "alu":
+            ent.update(achieved=amount / avg_s / 1e9, unit="G exp2/s", frac=amount / avg_s / 1e9 / mufu_peak)
+        elif bound == "fma":
+            ent.update(achieved=amount / avg_s / 1e12, unit="TFLOP/s fp32", frac=amount / avg_s / 1e12 / fma_peak)
+        kern[n] = ent
+    dom = max((n for n in kern if n.startswith("bwd_")), key=lambda n: kern[n]["share"])
+    dk = kern[dom]
+    bound, amount = kernel_work(dom, cfg, pool_axis)
+    roofline = {"bound": bound if bound == "hbm" else "alu", "kernel": dom, "achieved": dk.get("achieved"),
+                "peak": peak if bound == "hbm" else (mufu_peak if bound == "alu" else fma_peak), "unit": dk.get("unit"),
+                "frac": dk.get("frac"), "traffic": None,
+                "algorithmic_per_launch": amount, "peak_source": peak_src if bound == "hbm" else "derived",
+                "note": "dominant kernel of the gradient; achieved = algorithmic amount per launch / mean "
+                        "CUDA-event duration of the launch; no ncu capture of the gradient kernels yet"}
+    # the gradient's own HBM floor: read x, z, dy, write dx, dz (5 rows per token)
+    bwd_ms = sum(statistics.mean(per_kernel[n]) for n in dict.fromkeys(bwd.names))
+    line = {
+        "metric": "SSM-layer training step (forward + gradient) grid tokens/s at " + cfg.name + " (fp32)",
+        "value": tokens * a.steps / (ms / 1e3), "unit": UNIT, "n_gpus": 1, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": ms / a.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic (seeded N(0,1) x, z, dy; Mamba-style parameter init)",
+        "config": dict(workload_desc(cfg, pool_axis), step="forward call + gradient call",
+                       l2=("no flush (inputs > 2 x L2)" if flush is None else "L2 flushed before every step")),
+        "gradient": {"ms": bwd_ms, "hbm_floor_ms": 5 * 4 * cfg.E * tokens / (peak * 1e9) * 1e3,
+                     "floor_note": "x, z, dy read once, dx, dz written once at the measured copy rate"},
+        "roofline": roofline,
+        "kernels": kern,
+        "gpu_launches": nl * a.steps,
+        "clocks": clocks.summary(),
+        "e2e": None,
+    }
+    if not a.no_cpu_baseline:
+        import oracle
+        from pooled_selective_scan_b200 import inputs
+        cores = host_cores()
+        which = list(range(min(cfg.B, max(1, cores), 16)))
+        d = inputs.layer_inputs(cfg, which=which)
+        shp = inputs.token_shape(cfg)
+        dyh = __import__("numpy").stack([inputs.image_dy(cfg.seed, b, shp) for b in which])
+        oracle.build()
+        t0 = time.perf_counter()
+        oracle.forward(d["x"], d["z"], d["A_log"], d["D"], d["W_x"], d["W_dt"], d["b_dt"], pool_axis, cfg.dir_flags,
+                       keep_idx=d.get("keep_idx"), h=cfg.h, w=cfg.w, nthreads=len(which))
+        oracle.backward(d["x"], d["z"], d["A_log"], d["D"], d["W_x"], d["W_dt"], d["b_dt"], dyh, pool_axis,
+                        cfg.dir_flags, keep_idx=d.get("keep_idx"), h=cfg.h, w=cfg.w, nthreads=len(which))
+        el = time.perf_counter() - t0
+        tok = len(which) * (cfg.K if cfg.masked else cfg.h * cfg.w)
+        line["cpu_baseline"] = {"value": tok / el, "unit": UNIT, "cores": len(which), "kind": "oracle",
+                                "sample": f"{len(which)} images of {cfg.name}: fp64 oracle forward + gradient, "
+                                          f"OpenMP over images ({el:.1f} s wall)"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     a = parse(argv)
     from pooled_selective_scan_b200.configs import by_name
@@ -530,6 +689,8 @@ def main(argv=None):
     pool_axis = cfg.pool_axes[0] if a.pool_axis is None else a.pool_axis
     if a.impl == "reference":
         return run_reference(a, cfg, pool_axis)
+    if a.grad:
+        return run_grad(a, cfg, pool_axis)
     return run_ours(a, cfg, pool_axis)
 
 

@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define FASTVIM_SSM_ABI_VERSION 2
+#define FASTVIM_SSM_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define FV_API __attribute__((visibility("default")))
@@ -233,7 +233,7 @@ FV_API fv_status fastvim_selftest_bounded_wait(void* ws, size_t ws_bytes, unsign
 
 /* Self-test of the device math the layer uses instead of CUDA's full-precision functions, for
  * checking against a reference on the host: out[i] = f(in[i]) for i < n, with f chosen by `fn`:
- *   0  softplus(v) = log(1 + e^v)   (SFU exp2/log2 and a Mercator series for small e^-|v|)
+ *   0  softplus(v) = log(1 + e^v)   (SFU exp2 and reciprocal, an odd series of atanh)
  *   1  SiLU(v) = v / (1 + e^-v)      (SFU exp2 and reciprocal; the gate)
  *   2  2^v                           (SFU exp2, inputs below -126 flush to 0; the ZOH exponential)
  * in, out: DEVICE float arrays of n elements (16-byte aligned, not overlapping); queued on
@@ -243,6 +243,64 @@ FV_API fv_status fastvim_selftest_math(int fn, const float* in, float* out, int 
 /* Waits for `stream`, then reads the device status word of a workspace used by the last
  * forward call: FV_OK, FV_ERR_INDEX or FV_ERR_TIMEOUT (or FV_ERR_CUDA if the read fails). */
 FV_API fv_status fastvim_get_device_status(const void* ws, void* stream);
+
+/* ---- Gradient (training) ---------------------------------------------------------------------
+ * FastVim is trained end to end (summary page, "实验结果": faster pre-training and fine-tuning);
+ * the pages give no backward rule, so this is the exact derivative of the layer above, by the
+ * chain rule in reverse step order: for an upstream gradient dy = dL/dy of a scalar loss L it
+ * returns dx = dL/dx, dz = dL/dz and the parameter gradients summed over the batch.  Dense and
+ * masked layers, both pool axes, one or two directions, pool_scale and FV_FLAG_ZOH_EXACT; not
+ * the post-SSM LayerNorm (FV_FLAG_LAYERNORM gives FV_ERR_UNSUPPORTED).  Masked tokens whose id
+ * the forward rejected (FV_ERR_INDEX) get dx = dz = 0. */
+typedef struct {
+    const float* dy;  /* dL/dy, the shape of y (dense [B][h][w][E] | masked [B][K][E])         */
+    float* dx;        /* dL/dx, the shape of x (written)                                      */
+    float* dz;        /* dL/dz, the shape of z (written)                                      */
+    float* dA_log;    /* [nd][E][N]      } parameter gradients, summed over the batch;          */
+    float* dD;        /* [nd][E]         } written (not accumulated into): the call zeroes     */
+    float* dW_x;      /* [nd][R+2N][E]   } them first.  The sums run in fp32 with atomic       */
+    float* dW_dt;     /* [nd][E][R]      } additions, so their last bits may differ between    */
+    float* db_dt;     /* [nd][E]         } runs.                                               */
+} fv_ssm_grads;
+
+/* Byte offsets of the gradient's intermediates inside its workspace. */
+typedef struct {
+    size_t total_bytes;  /* what fastvim_ssm_backward_workspace_size returns                 */
+    size_t dys;          /* float [B][T][E]   dL/dys: ds summed over each pooled row's tokens  */
+    size_t dxbar;        /* float [B][T][E]   dL/dxbar                                         */
+    size_t du;           /* float, the layout of the forward's u: d dt_low | dB | dC           */
+    size_t dv;           /* float [B][nd][T][E]  dL/dv, v = the softplus input of Delta         */
+    size_t dxs;          /* float [B][nd][T][E]  the scans' share of dL/dxbar per direction     */
+    size_t ckpt;         /* float [B][nd][ceil(T/16)][E][16]  scan state entering each 16-step chunk */
+} fv_bwd_ws_layout;
+
+/* Workspace bytes a gradient call needs (0 when the arguments are invalid). */
+FV_API size_t fastvim_ssm_backward_workspace_size(const fv_ssm_args* args);
+FV_API fv_status fastvim_ssm_backward_workspace_layout(const fv_ssm_args* args, fv_bwd_ws_layout* out);
+
+/* Kernel launches of one gradient call (0 when invalid or B == 0) and the name of the i-th. */
+FV_API int fastvim_ssm_backward_launch_count(const fv_ssm_args* args);
+FV_API const char* fastvim_ssm_backward_launch_name(const fv_ssm_args* args, int i);
+
+/* Queue the gradient on `stream`.
+ * args: the forward call's arguments (the same tensors; y is not read and may be NULL).
+ * fwd_ws: the workspace of a fastvim_ssm_forward (or _events) call with these args that is
+ *   complete or queued earlier on `stream`: the gradient reads its pooled tokens, projections,
+ *   scan outputs and (masked) row lists.  fwd_ws_bytes >= fastvim_ssm_workspace_size(args).
+ * ws: the gradient's own workspace, >= fastvim_ssm_backward_workspace_size(args) bytes, 256-byte
+ *   aligned, no initial contents; fwd_ws and ws must not overlap.
+ * grads: device arrays, 16-byte aligned; dx and dz must not overlap each other, x, z or dy.
+ * Errors: as fastvim_ssm_forward for args; FV_ERR_NULL for a missing grads array (dy, dx, dz may
+ * be NULL when B == 0); FV_ERR_ALIGN, FV_ERR_ALIAS as above; FV_ERR_WORKSPACE for a missing,
+ * short or misaligned fwd_ws or ws; FV_ERR_UNSUPPORTED with FV_FLAG_LAYERNORM. */
+FV_API fv_status fastvim_ssm_backward(const fv_ssm_args* args, const fv_ssm_grads* grads, const void* fwd_ws,
+                                      size_t fwd_ws_bytes, void* ws, size_t ws_bytes, void* stream);
+
+/* fastvim_ssm_backward with timing marks, as fastvim_ssm_forward_events:
+ * n_events >= 2 * fastvim_ssm_backward_launch_count(args). */
+FV_API fv_status fastvim_ssm_backward_events(const fv_ssm_args* args, const fv_ssm_grads* grads,
+                                             const void* fwd_ws, size_t fwd_ws_bytes, void* ws, size_t ws_bytes,
+                                             void* stream, void* const* events, int n_events);
 
 #ifdef __cplusplus
 }

@@ -46,6 +46,12 @@ EXPORTS = (
     "fastvim_selftest_bounded_wait",
     "fastvim_selftest_math",
     "fastvim_get_device_status",
+    "fastvim_ssm_backward_workspace_size",
+    "fastvim_ssm_backward_workspace_layout",
+    "fastvim_ssm_backward_launch_count",
+    "fastvim_ssm_backward_launch_name",
+    "fastvim_ssm_backward",
+    "fastvim_ssm_backward_events",
 )
 
 
@@ -76,6 +82,14 @@ class FvWsLayout(ctypes.Structure):
         ("trace_records", ctypes.c_size_t), ("scan_bc", ctypes.c_size_t), ("scan_dt", ctypes.c_size_t),
         ("T", ctypes.c_int), ("S", ctypes.c_int), ("nd", ctypes.c_int),
     ]
+
+
+class FvSsmGrads(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in ("dy", "dx", "dz", "dA_log", "dD", "dW_x", "dW_dt", "db_dt")]
+
+
+class FvBwdWsLayout(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_size_t) for name in ("total_bytes", "dys", "dxbar", "du", "dv", "dxs", "ckpt")]
 
 
 class FastvimError(RuntimeError):
@@ -135,6 +149,21 @@ def lib() -> ctypes.CDLL:
             L.fastvim_selftest_math.restype = ctypes.c_int
             L.fastvim_get_device_status.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
             L.fastvim_get_device_status.restype = ctypes.c_int
+            L.fastvim_ssm_backward_workspace_size.argtypes = [P(FvSsmArgs)]
+            L.fastvim_ssm_backward_workspace_size.restype = ctypes.c_size_t
+            L.fastvim_ssm_backward_workspace_layout.argtypes = [P(FvSsmArgs), P(FvBwdWsLayout)]
+            L.fastvim_ssm_backward_workspace_layout.restype = ctypes.c_int
+            L.fastvim_ssm_backward_launch_count.argtypes = [P(FvSsmArgs)]
+            L.fastvim_ssm_backward_launch_count.restype = ctypes.c_int
+            L.fastvim_ssm_backward_launch_name.argtypes = [P(FvSsmArgs), ctypes.c_int]
+            L.fastvim_ssm_backward_launch_name.restype = ctypes.c_char_p
+            L.fastvim_ssm_backward.argtypes = [P(FvSsmArgs), P(FvSsmGrads), ctypes.c_void_p, ctypes.c_size_t,
+                                               ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+            L.fastvim_ssm_backward.restype = ctypes.c_int
+            L.fastvim_ssm_backward_events.argtypes = [P(FvSsmArgs), P(FvSsmGrads), ctypes.c_void_p, ctypes.c_size_t,
+                                                      ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                                      P(ctypes.c_void_p), ctypes.c_int]
+            L.fastvim_ssm_backward_events.restype = ctypes.c_int
             _lib = L
     return _lib
 

@@ -14,6 +14,7 @@
 #include "fv_common.cuh"
 #include "fv_fused.cuh"
 #include "fv_kernels.cuh"
+#include "fv_backward.cuh"
 
 namespace {
 
@@ -915,3 +916,286 @@ extern "C" fv_status fastvim_ssm_forward_noalloc(const fv_ssm_args* args, void* 
     // resets the status word itself, so the contents left by an earlier call need no clearing.
     return forward_impl(args, scratch, kStaticScratchBytes, (cudaStream_t)stream);
 }
+
+// ------------------------------------------------------------------------------------------------
+// Gradient of the layer.
+// ------------------------------------------------------------------------------------------------
+namespace {
+
+struct BwdLayout {
+    size_t dys, dxbar, du, dv, dxs, ckpt, total;
+};
+
+BwdLayout plan_bwd(const fv::Shape& sh) {
+    BwdLayout L{};
+    size_t off = 0;
+    const size_t bte = (size_t)sh.B * sh.T * sh.E * sizeof(float);
+    L.dys = off; off = round256(off + bte);
+    L.dxbar = off; off = round256(off + bte);
+    L.du = off; off = round256(off + (size_t)sh.nd * sh.B * fv::u_block_stride(sh.T, sh.J) * sizeof(float));
+    L.dv = off; off = round256(off + (size_t)sh.nd * bte);
+    L.dxs = off; off = round256(off + (size_t)sh.nd * bte);
+    L.ckpt = off;
+    off = round256(off + (size_t)sh.B * sh.nd * fv::bs_nchunks(sh.T) * sh.E * 16 * sizeof(float));
+    L.total = off;
+    return L;
+}
+
+// Launch order of a gradient call: gate, scans, d dt_low, dW_dt | db_dt, dW_x, dxbar, pooling.
+const char* bwd_launch_name_of(const fv::Shape& sh, int i) {
+    static const char* dense[] = {"bwd_gate_dense_kernel", "bwd_scan_kernel", "bwd_gemm_kernel:dt_low",
+                                  "bwd_gemm_kernel:W_dt", "bwd_gemm_kernel:W_x", "bwd_gemm_kernel:xbar",
+                                  "bwd_pool_dense_kernel"};
+    static const char* masked[] = {"bwd_gate_masked_kernel", "bwd_scan_kernel", "bwd_gemm_kernel:dt_low",
+                                   "bwd_gemm_kernel:W_dt", "bwd_gemm_kernel:W_x", "bwd_gemm_kernel:xbar",
+                                   "bwd_pool_masked_kernel"};
+    if (sh.B == 0 || i < 0 || i >= 7) return "";
+    return sh.K > 0 ? masked[i] : dense[i];
+}
+int bwd_launch_count_of(const fv::Shape& sh) { return sh.B == 0 ? 0 : 7; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t a0 = (uintptr_t)a, b0 = (uintptr_t)b;
+    return a && b && a0 < b0 + nb && b0 < a0 + na;
+}
+
+fv_status check_grads(const fv_ssm_args* a, const fv::Shape& sh, const fv_ssm_grads* g) {
+    if (!g) return FV_ERR_NULL;
+    if (!g->dA_log || !g->dD || !g->dW_x || !g->dW_dt || !g->db_dt) return FV_ERR_NULL;
+    if (sh.B > 0 && (!g->dy || !g->dx || !g->dz)) return FV_ERR_NULL;
+    const void* ps[] = {g->dy, g->dx, g->dz, g->dA_log, g->dD, g->dW_x, g->dW_dt, g->db_dt};
+    for (const void* p : ps)
+        if (p && !aligned16(p)) return FV_ERR_ALIGN;
+    if (sh.B > 0) {
+        const size_t tok = sh.K > 0 ? (size_t)sh.K : (size_t)sh.h * sh.w;
+        const size_t n = (size_t)sh.B * tok * sh.E * sizeof(float);
+        if (overlaps(g->dx, n, g->dz, n) || overlaps(g->dx, n, g->dy, n) || overlaps(g->dz, n, g->dy, n) ||
+            overlaps(g->dx, n, a->x, n) || overlaps(g->dx, n, a->z, n) || overlaps(g->dz, n, a->x, n) ||
+            overlaps(g->dz, n, a->z, n))
+            return FV_ERR_ALIAS;
+    }
+    return FV_OK;
+}
+
+int device_sm_count() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        sms <= 0)
+        return 148;
+    return sms;
+}
+
+template <class AOp, class BOp, class COp>
+fv_status launch_bwd_gemm(int M, int Nc, int Kd, int nz, int splits, AOp A, BOp Bm, COp C, cudaStream_t st,
+                          const char* where) {
+    if (M <= 0 || Nc <= 0 || Kd <= 0) return FV_OK;
+    int kchunk = (Kd + splits - 1) / splits;
+    kchunk = (kchunk + fv::kBgK - 1) / fv::kBgK * fv::kBgK;
+    splits = (Kd + kchunk - 1) / kchunk;
+    const dim3 grid((M + fv::kBgTile - 1) / fv::kBgTile, (Nc + fv::kBgTile - 1) / fv::kBgTile, nz * splits);
+    fv::bwd_gemm_kernel<<<grid, fv::kThreads, 0, st>>>(M, Nc, Kd, splits, kchunk, A, Bm, C);
+    FV_LAUNCH_CHECK(where);
+    return FV_OK;
+}
+
+// Splits of a reduction over the M = B T pooled tokens: about 4 blocks per SM in all.
+int bwd_splits(int M, int tiles, int sms) {
+    int s = (4 * sms + tiles - 1) / tiles;
+    const int most = (M + 255) / 256;  // at least 256 tokens per split
+    if (s > most) s = most;
+    return s < 1 ? 1 : s;
+}
+
+fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const void* fwd_v, size_t fwd_bytes,
+                        void* ws_v, size_t ws_bytes, cudaStream_t st, void* const* events = nullptr, int n_events = 0) {
+    fv::Shape sh;
+    fv_status s = make_shape(args, &sh);
+    if (s != FV_OK) return s;
+    // y is not read: a NULL y stands for "no output", checked as dx (which must not overlap x, z)
+    fv_ssm_args ac = *args;
+    if (!ac.y && g) ac.y = g->dx;
+    const fv_ssm_args* a = &ac;
+    if ((s = check_pointers(a, sh)) != FV_OK) return s;
+    if (sh.ln) return FV_ERR_UNSUPPORTED;
+    if ((s = check_grads(a, sh, g)) != FV_OK) return s;
+    fv_ws_layout FL;
+    plan_layout(sh, &FL);
+    const BwdLayout L = plan_bwd(sh);
+    if (!fwd_v || fwd_bytes < FL.total_bytes || ((uintptr_t)fwd_v & 255u)) return FV_ERR_WORKSPACE;
+    if (!ws_v || ws_bytes < L.total || ((uintptr_t)ws_v & 255u)) return FV_ERR_WORKSPACE;
+    if (overlaps(fwd_v, FL.total_bytes, ws_v, L.total)) return FV_ERR_WORKSPACE;
+    const size_t scan_smem = fv::bs_smem_floats(sh.R) * sizeof(float);
+    if (scan_smem > kMaxSmemOptin) return FV_ERR_UNSUPPORTED;
+    if (events && n_events < 2 * bwd_launch_count_of(sh)) return FV_ERR_SHAPE;
+    EventMarks marks{events, bwd_launch_count_of(sh), 0};
+
+    // parameter gradients are sums (atomic additions): start from zero
+    const size_t nA = (size_t)sh.nd * sh.E * sh.N, nE = (size_t)sh.nd * sh.E, nWx = (size_t)sh.nd * sh.J * sh.E,
+                 nWdt = (size_t)sh.nd * sh.E * sh.R;
+    cudaError_t e = cudaSuccess;
+    if ((e = cudaMemsetAsync(g->dA_log, 0, nA * sizeof(float), st)) != cudaSuccess ||
+        (e = cudaMemsetAsync(g->dD, 0, nE * sizeof(float), st)) != cudaSuccess ||
+        (e = cudaMemsetAsync(g->dW_x, 0, nWx * sizeof(float), st)) != cudaSuccess ||
+        (e = cudaMemsetAsync(g->dW_dt, 0, nWdt * sizeof(float), st)) != cudaSuccess ||
+        (e = cudaMemsetAsync(g->db_dt, 0, nE * sizeof(float), st)) != cudaSuccess) {
+        note_cuda(e, "gradient reset");
+        return FV_ERR_CUDA;
+    }
+    if (sh.B == 0) return FV_OK;
+    const char* fw = (const char*)fwd_v;
+    char* ws = (char*)ws_v;
+    const float* xbar = (const float*)(fw + FL.xbar);
+    const float* u = (const float*)(fw + FL.u);
+    const float* ys = (const float*)(fw + FL.ys);
+    float* dys = (float*)(ws + L.dys);
+    float* dxbar = (float*)(ws + L.dxbar);
+    float* du = (float*)(ws + L.du);
+    float* dv = (float*)(ws + L.dv);
+    float* dxs = (float*)(ws + L.dxs);
+    float* ckpt = (float*)(ws + L.ckpt);
+    // the scans add dB and dC into du
+    if ((e = cudaMemsetAsync(du, 0, (size_t)sh.nd * sh.B * fv::u_block_stride(sh.T, sh.J) * sizeof(float), st)) !=
+        cudaSuccess) {
+        note_cuda(e, "du reset");
+        return FV_ERR_CUDA;
+    }
+    const int sms = device_sm_count();
+    const int M = sh.B * sh.T;
+
+    // 1. gate, skip and repeat
+    // the gate kernels are persistent over pooled rows: one wave of resident blocks
+    auto resident = [&](auto kern, int threads) {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0) != cudaSuccess || per_sm < 1)
+            per_sm = 1;
+        return std::min(M, per_sm * sms);
+    };
+    if (sh.K == 0) {
+        const int threads = fv::bwd_groups(sh.SL) * fv::bwd_slot_width(sh.SL);
+        const int grid = resident(fv::bwd_gate_dense_kernel, threads);
+        FV_MARK_CALL(marks, st, ([&]() -> fv_status {
+            fv::bwd_gate_dense_kernel<<<grid, threads, 0, st>>>(sh, a->x, a->z, g->dy, ys, a->D, g->dx, g->dz, dys,
+                                                                  g->dD);
+            FV_LAUNCH_CHECK("bwd_gate_dense_kernel");
+            return FV_OK;
+        })());
+    } else {
+        const int32_t* row_off = (const int32_t*)(fw + FL.row_off);
+        const int32_t* row_tok = (const int32_t*)(fw + FL.row_tok);
+        const int grid = resident(fv::bwd_gate_masked_kernel, fv::kThreads);
+        FV_MARK_CALL(marks, st, ([&]() -> fv_status {
+            fv::bwd_gate_masked_kernel<<<grid, fv::kThreads, 0, st>>>(sh, a->x, a->z, g->dy, ys, a->D, row_off, row_tok,
+                                                                       g->dx, g->dz, dys, g->dD);
+            FV_LAUNCH_CHECK("bwd_gate_masked_kernel");
+            return FV_OK;
+        })());
+    }
+    // 2. adjoint of the scans
+    FV_MARK_CALL(marks, st, ([&]() -> fv_status {
+        const dim3 grid(sh.B, sh.nd, (sh.E + fv::kBsCh - 1) / fv::kBsCh);
+        if (sh.zoh_exact) {
+            if ((e = ensure_smem(fv::bwd_scan_kernel<true>, scan_smem)) != cudaSuccess) {
+                note_cuda(e, "scan gradient smem attribute");
+                return FV_ERR_CUDA;
+            }
+            fv::bwd_scan_kernel<true><<<grid, fv::kBsThreads, scan_smem, st>>>(sh, u, xbar, dys, a->A_log, a->W_dt, a->b_dt,
+                                                                              ckpt, dv, dxs, du, g->dA_log);
+        } else {
+            if ((e = ensure_smem(fv::bwd_scan_kernel<false>, scan_smem)) != cudaSuccess) {
+                note_cuda(e, "scan gradient smem attribute");
+                return FV_ERR_CUDA;
+            }
+            fv::bwd_scan_kernel<false><<<grid, fv::kBsThreads, scan_smem, st>>>(sh, u, xbar, dys, a->A_log, a->W_dt,
+                                                                               a->b_dt, ckpt, dv, dxs, du, g->dA_log);
+        }
+        FV_LAUNCH_CHECK("bwd_scan_kernel");
+        return FV_OK;
+    })());
+    // 3. dt_proj: d dt_low = dv W_dt (into du), then dW_dt | db_dt = dv^T [dt_low | 1]
+    FV_MARK_CALL(marks, st, launch_bwd_gemm(M, sh.R, sh.E, sh.nd, 1, fv::OpDvMK{dv, sh.T, sh.E, sh.nd},
+                                            fv::OpWdt{a->W_dt, sh.E, sh.R}, fv::OutDtl{du, sh}, st,
+                                            "bwd_gemm_kernel (dt_low)"));
+    {
+        const int tiles = ((sh.E + 63) / 64) * ((sh.R + 1 + 63) / 64) * sh.nd;
+        FV_MARK_CALL(marks, st, launch_bwd_gemm(sh.E, sh.R + 1, M, sh.nd, bwd_splits(M, tiles, sms),
+                                                fv::OpDvEM{dv, sh.T, sh.E, sh.nd}, fv::OpDtlOne{u, sh},
+                                                fv::OutWdtBdt{g->dW_dt, g->db_dt, sh.E, sh.R}, st,
+                                                "bwd_gemm_kernel (W_dt)"));
+    }
+    // 4. x_proj: dW_x = du^T xbar, dxbar = the scans' share + sum_k du[k] W_x[k]
+    {
+        const int tiles = ((sh.J + 63) / 64) * ((sh.E + 63) / 64) * sh.nd;
+        FV_MARK_CALL(marks, st, launch_bwd_gemm(sh.J, sh.E, M, sh.nd, bwd_splits(M, tiles, sms), fv::OpDuJM{du, sh},
+                                                fv::OpXbar{xbar, sh.E}, fv::OutWx{g->dW_x, sh.J, sh.E}, st,
+                                                "bwd_gemm_kernel (W_x)"));
+    }
+    FV_MARK_CALL(marks, st, launch_bwd_gemm(M, sh.E, sh.nd * sh.J, 1, 1, fv::OpDuMK{du, sh}, fv::OpWx{a->W_x, sh.E},
+                                            fv::OutDxbar{dxbar, dxs, sh.T, sh.E, sh.nd}, st,
+                                            "bwd_gemm_kernel (xbar)"));
+    // 5. pooling
+    if (sh.K == 0) {
+        const int threads = fv::bwd_groups(sh.SL) * fv::bwd_slot_width(sh.SL);
+        FV_MARK_CALL(marks, st, ([&]() -> fv_status {
+            fv::bwd_pool_dense_kernel<<<M, threads, 0, st>>>(sh, dxbar, g->dx);
+            FV_LAUNCH_CHECK("bwd_pool_dense_kernel");
+            return FV_OK;
+        })());
+    } else {
+        const int32_t* row_of = (const int32_t*)(fw + FL.row_of);
+        const long long ntok = (long long)sh.B * sh.K;
+        if (ntok >= (1ll << 31)) return FV_ERR_UNSUPPORTED;
+        FV_MARK_CALL(marks, st, ([&]() -> fv_status {
+            fv::bwd_pool_masked_kernel<<<(unsigned)ntok, 128, 0, st>>>(sh, row_of, dxbar, g->dx, g->dz);
+            FV_LAUNCH_CHECK("bwd_pool_masked_kernel");
+            return FV_OK;
+        })());
+    }
+    return FV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fastvim_ssm_backward_workspace_size(const fv_ssm_args* args) {
+    fv::Shape sh;
+    if (make_shape(args, &sh) != FV_OK) return 0;
+    return plan_bwd(sh).total;
+}
+
+fv_status fastvim_ssm_backward_workspace_layout(const fv_ssm_args* args, fv_bwd_ws_layout* out) {
+    if (!out) return FV_ERR_NULL;
+    fv::Shape sh;
+    fv_status s = make_shape(args, &sh);
+    if (s != FV_OK) return s;
+    const BwdLayout L = plan_bwd(sh);
+    out->total_bytes = L.total;
+    out->dys = L.dys; out->dxbar = L.dxbar; out->du = L.du; out->dv = L.dv; out->dxs = L.dxs; out->ckpt = L.ckpt;
+    return FV_OK;
+}
+
+int fastvim_ssm_backward_launch_count(const fv_ssm_args* args) {
+    fv::Shape sh;
+    if (make_shape(args, &sh) != FV_OK || sh.ln) return 0;
+    return bwd_launch_count_of(sh);
+}
+
+const char* fastvim_ssm_backward_launch_name(const fv_ssm_args* args, int i) {
+    fv::Shape sh;
+    if (make_shape(args, &sh) != FV_OK || sh.ln) return "";
+    return bwd_launch_name_of(sh, i);
+}
+
+fv_status fastvim_ssm_backward(const fv_ssm_args* args, const fv_ssm_grads* grads, const void* fwd_ws,
+                               size_t fwd_ws_bytes, void* ws, size_t ws_bytes, void* stream) {
+    return backward_impl(args, grads, fwd_ws, fwd_ws_bytes, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+fv_status fastvim_ssm_backward_events(const fv_ssm_args* args, const fv_ssm_grads* grads, const void* fwd_ws,
+                                      size_t fwd_ws_bytes, void* ws, size_t ws_bytes, void* stream,
+                                      void* const* events, int n_events) {
+    if (!events) return FV_ERR_NULL;
+    return backward_impl(args, grads, fwd_ws, fwd_ws_bytes, ws, ws_bytes, (cudaStream_t)stream, events, n_events);
+}
+
+}  // extern "C"

@@ -1,0 +1,690 @@
+// fv_backward.cuh -- the gradient of the FastVim SSM layer (sm_100a, fp32).
+//
+// FastVim is trained end to end (gptget.net summary of arXiv 2502.00594, "实验结果": faster
+// pre-training and fine-tuning); the pages give no backward rule, so these kernels compute the
+// exact derivative of the forward definition (fv_scan.cuh, fv_kernels.cuh), by the chain rule in
+// reverse step order:
+//   bwd_gate_dense_kernel / bwd_gate_masked_kernel   gate, skip and repeat: dz, the skip part of
+//                                                    dx, dD, and dys = the sum of ds over the
+//                                                    tokens of each pooled row
+//   bwd_scan_kernel                                  adjoint of both scans: dDelta (as dv = dDelta
+//                                                    sig(v) for dt_proj), dB, dC, dA_log and the
+//                                                    scans' share of dxbar
+//   bwd_gemm_kernel (4 launches)                     dt_proj and x_proj: d dt_low, dW_dt | db_dt,
+//                                                    dW_x, dxbar
+//   bwd_pool_dense_kernel / bwd_pool_masked_kernel   pooling: dx += pool_scale / S dxbar of the
+//                                                    token's row
+// Inputs of the forward that the gradient reuses (xbar, the projections u, ys and, masked, the
+// row lists) are read from the forward call's workspace.  The gate and pooling kernels stream the
+// grid (HBM bound); the scan is SFU/issue bound; the GEMMs are small (< 1 GFLOP).
+#pragma once
+
+#include "fv_common.cuh"
+#include "fv_kernels.cuh"
+
+namespace fv {
+
+constexpr int kBsCh = 64;        // channels per scan-gradient CTA
+constexpr int kBsThreads = 256;  // 4 lanes per channel, 4 states per lane
+constexpr int kBsChunk = 16;     // steps per checkpointed chunk
+
+__host__ __device__ __forceinline__ int bs_nchunks(int T) { return (T + kBsChunk - 1) / kBsChunk; }
+// Row stride of the W_dt rows in shared memory: odd, so lanes reading 32 different rows at the
+// same column hit 32 different banks.
+__host__ __device__ __forceinline__ int bs_wstride(int R) { return R | 1; }
+__host__ __device__ __forceinline__ size_t bs_smem_floats(int R) {
+    return (size_t)kBsCh * bs_wstride(R)      // W_dt rows of the CTA's channels
+           + (size_t)kBsChunk * R             // dt_low of the chunk's steps
+           + (size_t)kBsChunk * 32            // B | C of the chunk's steps
+           + 6 * (size_t)kBsChunk * kBsCh     // xbar, dys, Delta, sig(v), dv, dxbar (scan share)
+           + (size_t)kBsChunk * 32            // dB | dC sums of the chunk
+           + kBsCh;                           // b_dt of the CTA's channels
+}
+
+// sigmoid(v) = 1 / (1 + e^-v) on the SFU (v -> -inf gives 0, v -> +inf gives 1).
+__device__ __forceinline__ float sigmoid_fast(float v) {
+    return rcp_approx(1.f + ex2_approx(v * -1.4426950408889634f));
+}
+
+// ------------------------------------------------------------------------------------------
+// Gate, skip and repeat
+// ------------------------------------------------------------------------------------------
+
+// One channel of one token.  y = SiLU(z) s, s = ys + Dsum x:
+//   dz = dy s SiLU'(z),  SiLU'(z) = sig(z) (1 + z (1 - sig(z))),  ds = dy SiLU(z),
+//   dx (skip part) = ds Dsum,  dD += ds x,  dys += ds.
+__device__ __forceinline__ void gate_grad1(float x, float z, float g, float ys, float Ds, float& dz, float& dx,
+                                           float& acc, float& dDa) {
+    const float sg = sigmoid_fast(z);
+    const float s = fmaf(Ds, x, ys);
+    const float ds = g * z * sg;
+    dz = g * s * sg * fmaf(z, 1.f - sg, 1.f);
+    dx = ds * Ds;
+    acc += ds;
+    dDa = fmaf(ds, x, dDa);
+}
+
+__device__ __forceinline__ void gate_grad4(const float4& x, const float4& z, const float4& g, const float4& ys,
+                                           const float4& Ds, float4& dz, float4& dx, float4& acc, float4& dDa) {
+    gate_grad1(x.x, z.x, g.x, ys.x, Ds.x, dz.x, dx.x, acc.x, dDa.x);
+    gate_grad1(x.y, z.y, g.y, ys.y, Ds.y, dz.y, dx.y, acc.y, dDa.y);
+    gate_grad1(x.z, z.z, g.z, ys.z, Ds.z, dz.z, dx.z, acc.z, dDa.z);
+    gate_grad1(x.w, z.w, g.w, ys.w, Ds.w, dz.w, dx.w, acc.w, dDa.w);
+}
+
+__device__ __forceinline__ float4 f4_zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+
+__device__ __forceinline__ float4 bwd_dsum4(const float* __restrict__ D, int nd, int SL, int slot) {
+    const float4* D4 = reinterpret_cast<const float4*>(D);
+    float4 dv = D4[slot];
+    if (nd == 2) f4_add(dv, D4[SL + slot]);
+    return dv;
+}
+
+// Slots (float4 columns) a thread block covers per pass and the token groups that share a slot:
+// SL <= 256: one pass over all SL slots, 256 / SL groups; otherwise passes of 256 slots, one group.
+__host__ __device__ __forceinline__ int bwd_slot_width(int SL) { return SL <= kThreads ? SL : kThreads; }
+__host__ __device__ __forceinline__ int bwd_groups(int SL) { return kThreads / bwd_slot_width(SL); }
+
+// Dense gate gradient, persistent over pooled rows (b, t) (grid-stride), launched with
+// bwd_groups(SL) * bwd_slot_width(SL) threads.  Writes dz and the skip part of dx for every token
+// of the row, dys[b][t] (the sum of ds over the row's S tokens), and adds the block's dD sums.
+__global__ void __launch_bounds__(kThreads)
+bwd_gate_dense_kernel(Shape sh, const float* __restrict__ x, const float* __restrict__ z,
+                      const float* __restrict__ dy, const float* __restrict__ ys, const float* __restrict__ D,
+                      float* __restrict__ dx, float* __restrict__ dz, float* __restrict__ dys,
+                      float* __restrict__ dD) {
+    __shared__ float4 part[kThreads];
+    const int SL = sh.SL, SW = bwd_slot_width(SL), G = bwd_groups(SL);
+    const int ls = threadIdx.x % SW, g = threadIdx.x / SW;
+    const int rows = sh.B * sh.T, S = sh.S;
+    const size_t st4 = dense_stride(sh) >> 2;
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    const float4* z4 = reinterpret_cast<const float4*>(z);
+    const float4* g4 = reinterpret_cast<const float4*>(dy);
+    float4* dx4 = reinterpret_cast<float4*>(dx);
+    float4* dz4 = reinterpret_cast<float4*>(dz);
+    for (int s0 = 0; s0 < SL; s0 += SW) {
+        const int slot = s0 + ls;
+        const bool act = g < G && slot < SL;
+        const float4 Ds = act ? bwd_dsum4(D, sh.nd, SL, slot) : f4_zero();
+        float4 dDa = f4_zero();
+        for (int bt = blockIdx.x; bt < rows; bt += gridDim.x) {
+            const int b = bt / sh.T, t = bt - b * sh.T;
+            float4 acc = f4_zero();
+            if (act) {
+                const size_t base = (dense_base(sh, b, t) >> 2) + slot;
+                const float4 yv = reinterpret_cast<const float4*>(ys + (size_t)bt * sh.E)[slot];
+                int s = g;
+                for (; s + 3 * G < S; s += 4 * G) {  // four tokens, twelve loads in flight
+                    float4 xv[4], zv[4], gv[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const size_t o = base + (size_t)(s + u * G) * st4;
+                        xv[u] = ld_stream(x4 + o);
+                        zv[u] = ld_stream(z4 + o);
+                        gv[u] = ld_stream(g4 + o);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const size_t o = base + (size_t)(s + u * G) * st4;
+                        float4 dzv, dxv;
+                        gate_grad4(xv[u], zv[u], gv[u], yv, Ds, dzv, dxv, acc, dDa);
+                        st_stream(dz4 + o, dzv);
+                        st_stream(dx4 + o, dxv);
+                    }
+                }
+                for (; s < S; s += G) {
+                    const size_t o = base + (size_t)s * st4;
+                    float4 dzv, dxv;
+                    gate_grad4(ld_stream(x4 + o), ld_stream(z4 + o), ld_stream(g4 + o), yv, Ds, dzv, dxv, acc, dDa);
+                    st_stream(dz4 + o, dzv);
+                    st_stream(dx4 + o, dxv);
+                }
+            }
+            part[threadIdx.x] = acc;
+            __syncthreads();
+            if (g == 0 && slot < SL) {
+                float4 sum = part[ls];
+                for (int q = 1; q < G; ++q) f4_add(sum, part[q * SW + ls]);
+                reinterpret_cast<float4*>(dys + (size_t)bt * sh.E)[slot] = sum;
+            }
+            __syncthreads();
+        }
+        part[threadIdx.x] = dDa;
+        __syncthreads();
+        if (g == 0 && slot < SL) {
+            float4 sum = part[ls];
+            for (int q = 1; q < G; ++q) f4_add(sum, part[q * SW + ls]);
+            for (int k = 0; k < sh.nd; ++k) {
+                float* d = dD + (size_t)k * sh.E + 4 * slot;
+                atomicAdd(d + 0, sum.x); atomicAdd(d + 1, sum.y); atomicAdd(d + 2, sum.z); atomicAdd(d + 3, sum.w);
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// Masked gate gradient, persistent over pooled rows (b, t): the row's kept tokens come from the
+// forward's row lists (row_off, row_tok).  A row without tokens gets dys = 0.  Tokens whose id was
+// rejected are in no row; bwd_pool_masked_kernel zeroes their dx and dz.
+__global__ void __launch_bounds__(kThreads)
+bwd_gate_masked_kernel(Shape sh, const float* __restrict__ x, const float* __restrict__ z,
+                       const float* __restrict__ dy, const float* __restrict__ ys, const float* __restrict__ D,
+                       const int32_t* __restrict__ row_off, const int32_t* __restrict__ row_tok,
+                       float* __restrict__ dx, float* __restrict__ dz, float* __restrict__ dys,
+                       float* __restrict__ dD) {
+    const int SL = sh.SL, K = sh.K, T = sh.T;
+    const int rows = sh.B * T;
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    const float4* z4 = reinterpret_cast<const float4*>(z);
+    const float4* g4 = reinterpret_cast<const float4*>(dy);
+    float4* dx4 = reinterpret_cast<float4*>(dx);
+    float4* dz4 = reinterpret_cast<float4*>(dz);
+    for (int s0 = 0; s0 < SL; s0 += kThreads) {
+        const int slot = s0 + threadIdx.x;
+        const bool act = slot < SL;
+        const float4 Ds = act ? bwd_dsum4(D, sh.nd, SL, slot) : f4_zero();
+        float4 dDa = f4_zero();
+        for (int bt = blockIdx.x; bt < rows; bt += gridDim.x) {
+            if (!act) continue;
+            const int b = bt / T, t = bt - b * T;
+            const int p0 = row_off[(size_t)b * (T + 1) + t], p1 = row_off[(size_t)b * (T + 1) + t + 1];
+            const int32_t* tok = row_tok + (size_t)b * K;
+            const float4 yv = reinterpret_cast<const float4*>(ys + (size_t)bt * sh.E)[slot];
+            float4 acc = f4_zero();
+            int p = p0;
+            for (; p + 1 < p1; p += 2) {  // two tokens, six loads in flight
+                const size_t o0 = ((size_t)b * K + tok[p]) * SL + slot;
+                const size_t o1 = ((size_t)b * K + tok[p + 1]) * SL + slot;
+                const float4 xa = ld_stream(x4 + o0), za = ld_stream(z4 + o0), ga = ld_stream(g4 + o0);
+                const float4 xb = ld_stream(x4 + o1), zb = ld_stream(z4 + o1), gb = ld_stream(g4 + o1);
+                float4 dzv, dxv;
+                gate_grad4(xa, za, ga, yv, Ds, dzv, dxv, acc, dDa);
+                st_stream(dz4 + o0, dzv);
+                st_stream(dx4 + o0, dxv);
+                gate_grad4(xb, zb, gb, yv, Ds, dzv, dxv, acc, dDa);
+                st_stream(dz4 + o1, dzv);
+                st_stream(dx4 + o1, dxv);
+            }
+            if (p < p1) {
+                const size_t o = ((size_t)b * K + tok[p]) * SL + slot;
+                float4 dzv, dxv;
+                gate_grad4(ld_stream(x4 + o), ld_stream(z4 + o), ld_stream(g4 + o), yv, Ds, dzv, dxv, acc, dDa);
+                st_stream(dz4 + o, dzv);
+                st_stream(dx4 + o, dxv);
+            }
+            reinterpret_cast<float4*>(dys + (size_t)bt * sh.E)[slot] = acc;
+        }
+        if (act) {
+            for (int k = 0; k < sh.nd; ++k) {
+                float* d = dD + (size_t)k * sh.E + 4 * slot;
+                atomicAdd(d + 0, dDa.x); atomicAdd(d + 1, dDa.y); atomicAdd(d + 2, dDa.z); atomicAdd(d + 3, dDa.w);
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// Adjoint of the scans
+// ------------------------------------------------------------------------------------------
+
+// Grid (B, nd, ceil(E / 64)), 256 threads: thread (channel c = tid / 4, lane q = tid % 4) holds
+// states n = 4q .. 4q + 3 of channel e0 + c.  For direction slot k with scan order t_0, t_1, ...
+// (forward t = 0..T-1, backward t = T-1..0), h_{-1} = 0:
+//   forward   h_i = Abar_i h_{i-1} + q_i,  Abar_i = exp(Delta_i A),  q_i = Delta_i B_i xbar_i (Euler)
+//             or (Abar_i - 1) / A B_i xbar_i (exact ZOH);  ys += C_i . h_i
+//   adjoint   lam_i = C_i dys_i + Abar_{i+1} lam_{i+1}  (lam = 0 past the last step)
+//             dC_i += dys_i h_i;  dAbar_i = lam_i h_{i-1};  dq_i = lam_i
+// Pass 1 runs the recurrence in scan order and stores the state entering every 16-step chunk
+// (ckpt [B][nd][nchunks][E][16]).  Pass 2 walks the chunks in reverse: it recomputes the chunk's
+// states from its checkpoint (16 steps x 4 states in registers) and steps the adjoint back through
+// them.  Per step: dDelta and the scans' dxbar are summed over the 4 lanes of a channel (written as
+// dv = dDelta sig(v) and dxs [B][nd][T][E]); dB and dC are summed over the warp's 8 channels by a
+// transposing butterfly, over the block's 8 warps in shared memory, and over the E / 64 blocks of
+// an image with global atomics into du (zeroed by the caller).  dA_log (= dA A) sums in registers
+// over all steps, then one atomic per state.
+template <bool ZOH_EXACT>
+__global__ void __launch_bounds__(kBsThreads, 1)
+bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__ xbar, const float* __restrict__ dys,
+                const float* __restrict__ A_log, const float* __restrict__ W_dt, const float* __restrict__ b_dt,
+                float* __restrict__ ckpt, float* __restrict__ dv, float* __restrict__ dxs, float* __restrict__ du,
+                float* __restrict__ dA_log) {
+    extern __shared__ float bsm[];
+    const int b = blockIdx.x, k = blockIdx.y, e0 = blockIdx.z * kBsCh;
+    const int T = sh.T, E = sh.E, N = sh.N, R = sh.R, J = sh.J;
+    const int WS = bs_wstride(R);
+    float* sw = bsm;                          // [64][WS]
+    float* sdtl = sw + kBsCh * WS;            // [16][R]
+    float* sbc = sdtl + kBsChunk * R;         // [16][32]
+    float* sx = sbc + kBsChunk * 32;          // [16][64]
+    float* sdy = sx + kBsChunk * kBsCh;       // [16][64]
+    float* sdl = sdy + kBsChunk * kBsCh;      // [16][64]
+    float* ssg = sdl + kBsChunk * kBsCh;      // [16][64]
+    float* sdv = ssg + kBsChunk * kBsCh;      // [16][64]
+    float* sdx = sdv + kBsChunk * kBsCh;      // [16][64]
+    float* sred = sdx + kBsChunk * kBsCh;     // [16][32]
+    float* sbias = sred + kBsChunk * 32;      // [64]
+    const int tid = threadIdx.x;
+    const int c = tid >> 2, q = tid & 3, lane = tid & 31;
+    const int e = e0 + c;
+    const bool live = e < E;
+    const bool fwd = sh.nd == 2 ? k == 0 : (sh.dir_flags & 1u) != 0;
+    const int nchunks = bs_nchunks(T);
+    const float* ub = u + u_offset(sh, k, b, 0);
+
+    for (int i = tid; i < kBsCh * R; i += kBsThreads) {
+        const int row = i / R, r = i - row * R;
+        sw[row * WS + r] = (e0 + row < E) ? __ldg(W_dt + ((size_t)k * E + e0 + row) * R + r) : 0.f;
+    }
+    for (int i = tid; i < kBsCh; i += kBsThreads) sbias[i] = (e0 + i < E) ? __ldg(b_dt + (size_t)k * E + e0 + i) : 0.f;
+
+    constexpr float kLog2e = 1.4426950408889634f;
+    float A2[4], An[4], Ainv[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int n = 4 * q + j;
+        const float A = (live && n < N) ? -expf(__ldg(A_log + ((size_t)k * E + e) * N + n)) : 0.f;
+        An[j] = A;
+        A2[j] = A * kLog2e;
+        Ainv[j] = A != 0.f ? 1.f / A : 0.f;
+    }
+
+    // chunk `it` in scan order: first pooled token and length; slot i <-> step t_of(i)
+    auto chunk_t0 = [&](int it) { return (fwd ? it : nchunks - 1 - it) * kBsChunk; };
+    auto chunk_len = [&](int it) { return min(kBsChunk, T - chunk_t0(it)); };
+    auto t_of = [&](int it, int i) { return fwd ? chunk_t0(it) + i : chunk_t0(it) + chunk_len(it) - 1 - i; };
+
+    // stage a chunk's per-step inputs and compute Delta (and sig(v) in pass 2)
+    auto stage = [&](int it, bool pass2) {
+        const int len = chunk_len(it);
+        for (int i = tid; i < kBsChunk * R; i += kBsThreads) {
+            const int s = i / R, r = i - s * R;
+            sdtl[i] = s < len ? ub[(size_t)t_of(it, s) * J + r] : 0.f;
+        }
+        for (int i = tid; i < kBsChunk * 32; i += kBsThreads) {
+            const int s = i >> 5, j = i & 31, n = j & 15;
+            sbc[i] = (s < len && n < N) ? ub[(size_t)t_of(it, s) * J + R + (j < 16 ? n : N + n)] : 0.f;
+            if (pass2) sred[i] = 0.f;
+        }
+        for (int i = tid; i < kBsChunk * kBsCh; i += kBsThreads) {
+            const int s = i / kBsCh, cc = i - s * kBsCh;
+            const bool ok = s < len && e0 + cc < E;
+            const size_t o = ((size_t)b * T + (ok ? t_of(it, s) : 0)) * E + e0 + cc;
+            sx[i] = ok ? xbar[o] : 0.f;
+            if (pass2) sdy[i] = ok ? dys[o] : 0.f;
+        }
+        __syncthreads();
+        for (int i = tid; i < kBsChunk * kBsCh; i += kBsThreads) {
+            const int s = i / kBsCh, cc = i - s * kBsCh;
+            float v = sbias[cc];
+            const float* wr = sw + cc * WS;
+            const float* dr = sdtl + s * R;
+            for (int r = 0; r < R; ++r) v = fmaf(wr[r], dr[r], v);
+            sdl[i] = softplus_fast(v);
+            if (pass2) ssg[i] = sigmoid_fast(v);
+        }
+        __syncthreads();
+    };
+
+    // the input term of one step and state
+    auto qterm = [&](float dt, float Bn, float xv, int j) {
+        return ZOH_EXACT ? expm1f(dt * An[j]) * Ainv[j] * Bn * xv : dt * Bn * xv;
+    };
+
+    // ---- pass 1: states entering each chunk ----
+    float h[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int it = 0; it < nchunks; ++it) {
+        stage(it, false);
+        if (live)
+            *reinterpret_cast<float4*>(ckpt + ((((size_t)b * sh.nd + k) * nchunks + it) * E + e) * 16 + 4 * q) =
+                make_float4(h[0], h[1], h[2], h[3]);
+        const int len = chunk_len(it);
+        for (int i = 0; i < len; ++i) {
+            const float dt = sdl[i * kBsCh + c], xv = sx[i * kBsCh + c];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float Bn = sbc[i * 32 + 4 * q + j];
+                h[j] = fmaf(ex2_approx(dt * A2[j]), h[j], qterm(dt, Bn, xv, j));
+            }
+        }
+        __syncthreads();  // the buffers are refilled by the next stage()
+    }
+
+    // ---- pass 2: the adjoint, chunks in reverse scan order ----
+    float lam[4] = {0.f, 0.f, 0.f, 0.f}, Anext[4] = {0.f, 0.f, 0.f, 0.f}, gA[4] = {0.f, 0.f, 0.f, 0.f};
+    const bool b2 = lane & 4, b3 = lane & 8, b4 = lane & 16;
+    const int v_idx = (b2 ? 1 : 0) + (b3 ? 2 : 0) + (b4 ? 4 : 0);  // value this lane ends up holding
+    const int red_n = 4 * q + (v_idx & 3), red_w = v_idx >> 2;       // state, and 0 = dB / 1 = dC
+    for (int it = nchunks - 1; it >= 0; --it) {
+        stage(it, true);
+        const int len = chunk_len(it);
+        float hin[4] = {0.f, 0.f, 0.f, 0.f};
+        if (live) {
+            const float4 v = *reinterpret_cast<const float4*>(
+                ckpt + ((((size_t)b * sh.nd + k) * nchunks + it) * E + e) * 16 + 4 * q);
+            hin[0] = v.x; hin[1] = v.y; hin[2] = v.z; hin[3] = v.w;
+        }
+        float hist[kBsChunk][4];
+        {
+            float hc[4] = {hin[0], hin[1], hin[2], hin[3]};
+#pragma unroll
+            for (int i = 0; i < kBsChunk; ++i) {
+                if (i < len) {
+                    const float dt = sdl[i * kBsCh + c], xv = sx[i * kBsCh + c];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float Bn = sbc[i * 32 + 4 * q + j];
+                        hc[j] = fmaf(ex2_approx(dt * A2[j]), hc[j], qterm(dt, Bn, xv, j));
+                        hist[i][j] = hc[j];
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) hist[i][j] = 0.f;
+                }
+            }
+        }
+#pragma unroll
+        for (int ii = 0; ii < kBsChunk; ++ii) {
+            const int i = kBsChunk - 1 - ii;
+            if (i < len) {
+                const float dt = sdl[i * kBsCh + c], xv = sx[i * kBsCh + c], gy = sdy[i * kBsCh + c];
+                float ddt = 0.f, dxb = 0.f, vals[8];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float Bn = sbc[i * 32 + 4 * q + j], Cn = sbc[i * 32 + 16 + 4 * q + j];
+                    const float Ab = ex2_approx(dt * A2[j]);
+                    const float hp = i > 0 ? hist[i > 0 ? i - 1 : 0][j] : hin[j];
+                    lam[j] = fmaf(Anext[j], lam[j], Cn * gy);
+                    vals[4 + j] = gy * hist[i][j];
+                    const float t1 = lam[j] * hp * Ab;
+                    ddt = fmaf(t1, An[j], ddt);
+                    gA[j] = fmaf(t1, dt, gA[j]);
+                    if (ZOH_EXACT) {
+                        const float em = expm1f(dt * An[j]);
+                        const float cf = em * Ainv[j];
+                        ddt = fmaf(lam[j] * Ab, Bn * xv, ddt);
+                        gA[j] = fmaf(lam[j] * Bn * xv, (dt * Ab * An[j] - em) * Ainv[j] * Ainv[j], gA[j]);
+                        vals[j] = lam[j] * cf * xv;
+                        dxb = fmaf(lam[j] * cf, Bn, dxb);
+                    } else {
+                        ddt = fmaf(lam[j], Bn * xv, ddt);
+                        vals[j] = lam[j] * dt * xv;
+                        dxb = fmaf(lam[j] * dt, Bn, dxb);
+                    }
+                    Anext[j] = Ab;
+                }
+                ddt += __shfl_xor_sync(0xffffffffu, ddt, 1);
+                ddt += __shfl_xor_sync(0xffffffffu, ddt, 2);
+                dxb += __shfl_xor_sync(0xffffffffu, dxb, 1);
+                dxb += __shfl_xor_sync(0xffffffffu, dxb, 2);
+                if (q == 0) {
+                    sdv[i * kBsCh + c] = ddt * ssg[i * kBsCh + c];
+                    sdx[i * kBsCh + c] = dxb;
+                }
+                // sum the 8 values over the warp's 8 channels (lane bits 2..4); each lane keeps one
+                float r1[4], r2[2];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float send = b4 ? vals[j] : vals[j + 4];
+                    const float keep = b4 ? vals[j + 4] : vals[j];
+                    r1[j] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+                }
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const float send = b3 ? r1[j] : r1[j + 2];
+                    const float keep = b3 ? r1[j + 2] : r1[j];
+                    r2[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+                }
+                const float send = b2 ? r2[0] : r2[1];
+                const float keep = b2 ? r2[1] : r2[0];
+                const float fin = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+                if (red_n < N) atomicAdd(&sred[i * 32 + red_w * 16 + red_n], fin);
+            }
+        }
+        __syncthreads();
+        for (int i = tid; i < len * kBsCh; i += kBsThreads) {
+            const int s = i / kBsCh, cc = i - s * kBsCh;
+            if (e0 + cc < E) {
+                const size_t o = (((size_t)b * sh.nd + k) * T + t_of(it, s)) * E + e0 + cc;
+                dv[o] = sdv[i];
+                dxs[o] = sdx[i];
+            }
+        }
+        for (int i = tid; i < len * 32; i += kBsThreads) {
+            const int s = i >> 5, j = i & 31, n = j & 15;
+            if (n < N) atomicAdd(du + u_offset(sh, k, b, t_of(it, s)) + R + (j < 16 ? n : N + n), sred[i]);
+        }
+        __syncthreads();  // the buffers are refilled by the next stage()
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int n = 4 * q + j;
+        if (live && n < N) atomicAdd(dA_log + ((size_t)k * E + e) * N + n, gA[j] * An[j]);
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// Projection gradients: small GEMMs out[i][j] = sum_kk A(i, kk) B(kk, j)
+// ------------------------------------------------------------------------------------------
+
+constexpr int kBgTile = 64, kBgK = 16, kBgPad = kBgTile + 4;
+
+// Operand accessors.  kContig: the operand is contiguous along kk (A) or along j (B), which picks
+// the coalesced loading order.  k is the direction slot of the launch (blockIdx.z / splits).
+
+// A = dv[k][m][e] as (i = m, kk = e), for d dt_low = dv W_dt[k]
+struct OpDvMK {
+    static constexpr bool kContig = true;
+    const float* dv; int T, E, nd;
+    __device__ float operator()(int k, int i, int kk) const {
+        const int b = i / T, t = i - b * T;
+        return dv[(((size_t)b * nd + k) * T + t) * E + kk];
+    }
+};
+// A = dv[k][m][e] as (i = e, kk = m), for dW_dt = dv^T dt_low and db_dt = dv^T 1
+struct OpDvEM {
+    static constexpr bool kContig = false;
+    const float* dv; int T, E, nd;
+    __device__ float operator()(int k, int i, int kk) const {
+        const int b = kk / T, t = kk - b * T;
+        return dv[(((size_t)b * nd + k) * T + t) * E + i];
+    }
+};
+// B = W_dt[k][e][r] as (kk = e, j = r)
+struct OpWdt {
+    static constexpr bool kContig = true;
+    const float* W_dt; int E, R;
+    __device__ float operator()(int k, int kk, int j) const { return W_dt[((size_t)k * E + kk) * R + j]; }
+};
+// B = [dt_low | 1] as (kk = m, j = r <= R): column R is ones (gives db_dt)
+struct OpDtlOne {
+    static constexpr bool kContig = true;
+    const float* u; Shape sh;
+    __device__ float operator()(int k, int kk, int j) const {
+        if (j == sh.R) return 1.f;
+        const int b = kk / sh.T, t = kk - b * sh.T;
+        return u[u_offset(sh, k, b, t) + j];
+    }
+};
+// A = du[k][m][jj] as (i = jj, kk = m), for dW_x = du^T xbar
+struct OpDuJM {
+    static constexpr bool kContig = false;
+    const float* du; Shape sh;
+    __device__ float operator()(int k, int i, int kk) const {
+        const int b = kk / sh.T, t = kk - b * sh.T;
+        return du[u_offset(sh, k, b, t) + i];
+    }
+};
+// B = xbar[m][e] as (kk = m, j = e)
+struct OpXbar {
+    static constexpr bool kContig = true;
+    const float* xbar; int E;
+    __device__ float operator()(int, int kk, int j) const { return xbar[(size_t)kk * E + j]; }
+};
+// A = du[k'][m][jj] as (i = m, kk = k' J + jj), for dxbar = sum_k' du[k'] W_x[k']
+struct OpDuMK {
+    static constexpr bool kContig = true;
+    const float* du; Shape sh;
+    __device__ float operator()(int, int i, int kk) const {
+        const int kd = kk / sh.J, jj = kk - kd * sh.J;
+        const int b = i / sh.T, t = i - b * sh.T;
+        return du[u_offset(sh, kd, b, t) + jj];
+    }
+};
+// B = W_x[k'][jj][e] as (kk = k' J + jj, j = e)
+struct OpWx {
+    static constexpr bool kContig = true;
+    const float* W_x; int E;
+    __device__ float operator()(int, int kk, int j) const { return W_x[(size_t)kk * E + j]; }
+};
+
+// Outputs.
+struct OutDtl {  // d dt_low into du (stored; the B and C slots hold the scans' sums)
+    float* du; Shape sh;
+    __device__ void operator()(int k, int i, int j, float v) const {
+        const int b = i / sh.T, t = i - b * sh.T;
+        du[u_offset(sh, k, b, t) + j] = v;
+    }
+};
+struct OutWdtBdt {  // split-K partial sums of dW_dt (j < R) and db_dt (j == R)
+    float* dW_dt; float* db_dt; int E, R;
+    __device__ void operator()(int k, int i, int j, float v) const {
+        atomicAdd(j < R ? dW_dt + ((size_t)k * E + i) * R + j : db_dt + (size_t)k * E + i, v);
+    }
+};
+struct OutWx {  // split-K partial sums of dW_x
+    float* dW_x; int J, E;
+    __device__ void operator()(int k, int i, int j, float v) const {
+        atomicAdd(dW_x + ((size_t)k * J + i) * E + j, v);
+    }
+};
+struct OutDxbar {  // dxbar = the scans' share (summed over directions) + the projections' share
+    float* dxbar; const float* dxs; int T, E, nd;
+    __device__ void operator()(int, int i, int j, float v) const {
+        const int b = i / T, t = i - b * T;
+        for (int k = 0; k < nd; ++k) v += dxs[(((size_t)b * nd + k) * T + t) * E + j];
+        dxbar[(size_t)i * E + j] = v;
+    }
+};
+
+// 64 x 64 output tile per block of 256 threads (4 x 4 per thread), k-steps of 16 through shared
+// memory.  Grid (ceil(M / 64), ceil(Nc / 64), nd * splits); split s of direction k covers
+// kk in [s * kchunk, min(Kd, (s + 1) * kchunk)).
+template <class AOp, class BOp, class COp>
+__global__ void __launch_bounds__(kThreads)
+bwd_gemm_kernel(int M, int Nc, int Kd, int splits, int kchunk, AOp A, BOp Bm, COp C) {
+    __shared__ __align__(16) float As[kBgK][kBgPad];
+    __shared__ __align__(16) float Bs[kBgK][kBgPad];
+    const int k = blockIdx.z / splits, s = blockIdx.z - k * splits;
+    const int i0 = blockIdx.x * kBgTile, j0 = blockIdx.y * kBgTile;
+    const int kbeg = s * kchunk, kend = min(Kd, kbeg + kchunk);
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int bq = 0; bq < 4; ++bq) acc[a][bq] = 0.f;
+    for (int kk0 = kbeg; kk0 < kend; kk0 += kBgK) {
+#pragma unroll
+        for (int l = 0; l < 4; ++l) {
+            const int idx = threadIdx.x + l * kThreads;
+            int ii, kk;
+            if (AOp::kContig) { kk = idx & 15; ii = idx >> 4; }
+            else { ii = idx & 63; kk = idx >> 6; }
+            const int gi = i0 + ii, gk = kk0 + kk;
+            As[kk][ii] = (gi < M && gk < kend) ? A(k, gi, gk) : 0.f;
+            int jj;
+            if (BOp::kContig) { jj = idx & 63; kk = idx >> 6; }
+            else { kk = idx & 15; jj = idx >> 4; }
+            const int gj = j0 + jj, gk2 = kk0 + kk;
+            Bs[kk][jj] = (gj < Nc && gk2 < kend) ? Bm(k, gk2, gj) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < kBgK; ++kk) {
+            const float4 a = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
+            const float4 bv = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
+            const float av[4] = {a.x, a.y, a.z, a.w}, bw[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) acc[p][r] = fmaf(av[p], bw[r], acc[p][r]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int gi = i0 + ty * 4 + p, gj = j0 + tx * 4 + r;
+            if (gi < M && gj < Nc) C(k, gi, gj, acc[p][r]);
+        }
+}
+
+// ------------------------------------------------------------------------------------------
+// Pooling
+// ------------------------------------------------------------------------------------------
+
+// One block per pooled row (b, t), launched with bwd_groups(SL) * bwd_slot_width(SL) threads:
+// every token of the row gets dx += pool_scale / S * dxbar[b][t].
+__global__ void __launch_bounds__(kThreads)
+bwd_pool_dense_kernel(Shape sh, const float* __restrict__ dxbar, float* __restrict__ dx) {
+    const int SL = sh.SL, SW = bwd_slot_width(SL), G = bwd_groups(SL);
+    const int ls = threadIdx.x % SW, g = threadIdx.x / SW;
+    const int bt = blockIdx.x, b = bt / sh.T, t = bt - b * sh.T;
+    const int S = sh.S;
+    const size_t st4 = dense_stride(sh) >> 2;
+    const float scale = sh.pool_scale / (float)S;
+    float4* dx4 = reinterpret_cast<float4*>(dx);
+    for (int s0 = 0; s0 < SL; s0 += SW) {
+        const int slot = s0 + ls;
+        if (g >= G || slot >= SL) continue;
+        const float4 a = f4_scale(reinterpret_cast<const float4*>(dxbar + (size_t)bt * sh.E)[slot], scale);
+        const size_t base = (dense_base(sh, b, t) >> 2) + slot;
+        int s = g;
+        for (; s + 3 * G < S; s += 4 * G) {
+            float4 v[4];
+#pragma unroll
+            for (int uu = 0; uu < 4; ++uu) v[uu] = ld_stream(dx4 + base + (size_t)(s + uu * G) * st4);
+#pragma unroll
+            for (int uu = 0; uu < 4; ++uu) {
+                f4_add(v[uu], a);
+                st_stream(dx4 + base + (size_t)(s + uu * G) * st4, v[uu]);
+            }
+        }
+        for (; s < S; s += G) {
+            float4 v = ld_stream(dx4 + base + (size_t)s * st4);
+            f4_add(v, a);
+            st_stream(dx4 + base + (size_t)s * st4, v);
+        }
+    }
+}
+
+// One block per kept token (b, k): dx += pool_scale / S * dxbar of its row; a token whose id was
+// rejected (row_of < 0) gets dx = dz = 0.
+__global__ void __launch_bounds__(kThreads)
+bwd_pool_masked_kernel(Shape sh, const int32_t* __restrict__ row_of, const float* __restrict__ dxbar,
+                       float* __restrict__ dx, float* __restrict__ dz) {
+    const size_t bk = blockIdx.x;
+    const int b = (int)(bk / sh.K);
+    const int r = row_of[bk];
+    const float scale = sh.pool_scale / (float)sh.S;
+    float4* dx4 = reinterpret_cast<float4*>(dx) + bk * sh.SL;
+    float4* dz4 = reinterpret_cast<float4*>(dz) + bk * sh.SL;
+    if (r < 0) {
+        for (int slot = threadIdx.x; slot < sh.SL; slot += blockDim.x) {
+            dx4[slot] = f4_zero();
+            dz4[slot] = f4_zero();
+        }
+        return;
+    }
+    const float4* a4 = reinterpret_cast<const float4*>(dxbar + ((size_t)b * sh.T + r) * sh.E);
+    for (int slot = threadIdx.x; slot < sh.SL; slot += blockDim.x) {
+        float4 v = ld_stream(dx4 + slot);
+        f4_add(v, f4_scale(a4[slot], scale));
+        st_stream(dx4 + slot, v);
+    }
+}
+
+}  // namespace fv

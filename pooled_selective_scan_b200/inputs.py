@@ -12,7 +12,8 @@ follow the usual Mamba/Vim initialisation that the layer is specified with:
            Delta0 ~ exp(U(ln 1e-3, ln 0.1))  [E],  b_dt = Delta0 + log(-expm1(-Delta0)),
            i.e. the value whose softplus is Delta0 (the initial step sizes are log-uniform);
   keep_idx[b] = default_rng([seed, 3, b]).permutation(h*w)[:K] (int32, unsorted) for a masked
-           layer at keep ratio K / (h*w).
+           layer at keep ratio K / (h*w);
+  dy     ~ N(0, 1) fp32, the upstream gradient of a training step, default_rng([seed, 4, b]).
 """
 from __future__ import annotations
 
@@ -45,6 +46,10 @@ def image_x(seed: int, b: int, shape) -> np.ndarray:
 
 def image_z(seed: int, b: int, shape) -> np.ndarray:
     return np.random.default_rng([seed, 2, b]).standard_normal(shape, dtype=np.float32)
+
+
+def image_dy(seed: int, b: int, shape) -> np.ndarray:
+    return np.random.default_rng([seed, 4, b]).standard_normal(shape, dtype=np.float32)
 
 
 def image_keep_idx(seed: int, b: int, h: int, w: int, K: int) -> np.ndarray:

@@ -217,6 +217,89 @@ class BoundForward:
                                                        self._evbuf, len(events)), "fastvim_ssm_forward_events")
 
 
+def backward_workspace_size(shape: LayerShape) -> int:
+    a = shape.args()
+    n = nat.lib().fastvim_ssm_backward_workspace_size(ctypes.byref(a))
+    if n == 0:
+        nat.check(nat.lib().fastvim_ssm_validate(ctypes.byref(a)), "fastvim_ssm_backward_workspace_size")
+    return int(n)
+
+
+def backward_launch_names(shape: LayerShape) -> list:
+    a = shape.args()
+    n = nat.lib().fastvim_ssm_backward_launch_count(ctypes.byref(a))
+    return [nat.lib().fastvim_ssm_backward_launch_name(ctypes.byref(a), i).decode() for i in range(n)]
+
+
+def _grads(dy, grads: dict) -> nat.FvSsmGrads:
+    g = nat.FvSsmGrads()
+    g.dy = _ptr(dy)
+    for name in ("dx", "dz", "dA_log", "dD", "dW_x", "dW_dt", "db_dt"):
+        setattr(g, name, _ptr(grads[name]))
+    return g
+
+
+def backward(x, z, A_log, D, W_x, W_dt, b_dt, dy, fwd_workspace, pool_axis=POOL_W, dir_flags=DIR_FWD | DIR_BWD,
+             keep_idx=None, h=None, w=None, pool_scale=1.0, zoh_exact=False, path="auto", grads=None,
+             workspace=None, stream=None) -> dict:
+    """Queue the gradient of the layer for the upstream gradient dy on ``stream`` and return the
+    dict {dx, dz, dA_log, dD, dW_x, dW_dt, db_dt}.  fwd_workspace is the workspace of a forward
+    call with the same tensors and options, queued earlier on the same stream."""
+    dev = x.device
+    for name, t in (("x", x), ("z", z), ("A_log", A_log), ("D", D), ("W_x", W_x), ("W_dt", W_dt), ("b_dt", b_dt),
+                    ("dy", dy)):
+        _check_tensor(name, t, torch.float32, dev)
+    if keep_idx is not None:
+        _check_tensor("keep_idx", keep_idx, torch.int32, dev)
+    shape = infer_shape(x, A_log, W_dt, pool_axis, dir_flags, keep_idx, h, w, pool_scale, zoh_exact, path)
+    if z.shape != x.shape or dy.shape != x.shape:
+        raise ValueError("z and dy must have the shape of x")
+    if grads is None:
+        grads = {"dx": torch.empty_like(x), "dz": torch.empty_like(z)}
+        for name, p in (("dA_log", A_log), ("dD", D), ("dW_x", W_x), ("dW_dt", W_dt), ("db_dt", b_dt)):
+            grads[name] = torch.empty_like(p)
+    if workspace is None:
+        workspace = torch.empty(max(backward_workspace_size(shape), 256), dtype=torch.uint8, device=dev)
+    a = shape.args(x, z, A_log, D, W_x, W_dt, b_dt, keep_idx)  # y is not read by the gradient
+    g = _grads(dy, grads)
+    st = nat.lib().fastvim_ssm_backward(ctypes.byref(a), ctypes.byref(g), ctypes.c_void_p(fwd_workspace.data_ptr()),
+                                        ctypes.c_size_t(fwd_workspace.numel()), ctypes.c_void_p(workspace.data_ptr()),
+                                        ctypes.c_size_t(workspace.numel()), _stream_handle(stream))
+    nat.check(st, "fastvim_ssm_backward")
+    return grads
+
+
+class BoundBackward:
+    """A gradient call with its tensors and workspaces bound once, for repeated launches:
+    ``run()`` queues it, ``run_events(evs)`` also brackets each of its kernel launches."""
+
+    def __init__(self, shape: LayerShape, t: dict, dy, grads: dict, fwd_workspace, workspace, stream=None):
+        self.shape = shape
+        self._keep = (t, dy, grads, fwd_workspace, workspace)
+        self._args = shape.args(t["x"], t["z"], t["A_log"], t["D"], t["W_x"], t["W_dt"], t["b_dt"], t.get("keep_idx"))
+        self._g = _grads(dy, grads)
+        self._fw = (ctypes.c_void_p(fwd_workspace.data_ptr()), ctypes.c_size_t(fwd_workspace.numel()))
+        self._ws = (ctypes.c_void_p(workspace.data_ptr()), ctypes.c_size_t(workspace.numel()))
+        self._stream = _stream_handle(stream)
+        self.names = backward_launch_names(shape)
+        self.n_launch = len(self.names)
+        self._evbuf = (ctypes.c_void_p * (2 * self.n_launch))()
+
+    def run(self):
+        nat.check(nat.lib().fastvim_ssm_backward(ctypes.byref(self._args), ctypes.byref(self._g), *self._fw, *self._ws,
+                                                 self._stream), "fastvim_ssm_backward")
+
+    def run_events(self, events):
+        for e in events:
+            if not e.cuda_event:
+                e.record()
+        for i, e in enumerate(events):
+            self._evbuf[i] = e.cuda_event
+        nat.check(nat.lib().fastvim_ssm_backward_events(ctypes.byref(self._args), ctypes.byref(self._g), *self._fw,
+                                                        *self._ws, self._stream, self._evbuf, len(events)),
+                  "fastvim_ssm_backward_events")
+
+
 def device_status(workspace, stream=None) -> int:
     """Wait for the stream and return the device status word of the last call (0 = FV_OK)."""
     return int(nat.lib().fastvim_get_device_status(ctypes.c_void_p(workspace.data_ptr()), _stream_handle(stream)))

@@ -50,6 +50,18 @@ def activations(cfg: LayerConfig, device, pinned_host: bool = False, first_image
     return out
 
 
+def upstream_grad(cfg: LayerConfig, device, pinned_host: bool = False, first_image: int = 0) -> torch.Tensor:
+    """dy (the gradient arriving at the layer's output in a training step) for the same images."""
+    shp = inputs.token_shape(cfg)
+    if pinned_host:
+        dy = torch.empty((cfg.B,) + shp, dtype=torch.float32, pin_memory=True)
+    else:
+        dy = torch.empty((cfg.B,) + shp, dtype=torch.float32, device=device)
+    for i in range(cfg.B):
+        dy[i].copy_(torch.from_numpy(inputs.image_dy(cfg.seed, first_image + i, shp)))
+    return dy
+
+
 def ln_tensors(cfg: LayerConfig, device) -> dict:
     """Post-SSM LayerNorm weights at their usual initialisation: gamma = 1, beta = 0."""
     return dict(ln_gamma=torch.ones(cfg.E, dtype=torch.float32, device=device),

@@ -1,0 +1,164 @@
+"""Parity of the layer's gradient (CUDA, through the C ABI) with the fp64 gradient oracle.
+
+Each case runs the forward call, then the gradient call on its workspace, with every workspace
+and output poisoned beforehand (NaN bytes), and compares dx, dz and the five parameter gradients
+element by element: dx and dz at the layer's tolerance, the batch-summed parameter gradients at
+the gradient tolerance (fv_testlib).  Shapes cover ragged channel blocks (E not a multiple of
+64), partial state groups (N < 16), pooled lengths below, at and across the 16-step checkpoint
+chunks, one or two directions, exact ZOH, pool_scale, the fused forward's workspace, masked
+layers with empty rows and a rejected id, and the empty batch."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle  # noqa: E402
+from fv_testlib import GRAD_PARAM_ABS_RMS, assert_close  # noqa: E402
+from pooled_selective_scan_b200 import inputs, ssm  # noqa: E402
+
+pytestmark = [pytest.mark.gpu, pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+PARAMS = ("A_log", "D", "W_x", "W_dt", "b_dt")
+
+
+def make_inputs(seed, B, h, w, E, N, R, nd, K=0, drop_row=None, pool_axis=0):
+    d = inputs.params(E, N, R, nd, seed)
+    rng = np.random.default_rng([seed, 99])
+    # spread A and D so that every parameter gradient has structure to check
+    d["A_log"] = (d["A_log"] + rng.uniform(-0.3, 0.3, d["A_log"].shape)).astype(np.float32)
+    d["D"] = rng.uniform(0.5, 1.5, d["D"].shape).astype(np.float32)
+    shp = (K, E) if K else (h, w, E)
+    d["x"] = np.stack([inputs.image_x(seed, b, shp) for b in range(B)]) if B else np.empty((0,) + shp, np.float32)
+    d["z"] = np.stack([inputs.image_z(seed, b, shp) for b in range(B)]) if B else np.empty((0,) + shp, np.float32)
+    d["dy"] = np.stack([inputs.image_dy(seed, b, shp) for b in range(B)]) if B else np.empty((0,) + shp, np.float32)
+    if K:
+        ids = []
+        for b in range(B):
+            pool = np.arange(h * w)
+            if drop_row is not None:  # leave one pooled row (grid row, or column under POOL_H) empty
+                pool = pool[(pool // w if pool_axis == 0 else pool % w) != drop_row]
+            ids.append(np.random.default_rng([seed, 3, b]).permutation(pool)[:K])
+        d["keep_idx"] = np.stack(ids).astype(np.int32)
+    return d
+
+
+def gpu_grads(d, pool_axis, dir_flags, h, w, pool_scale=1.0, zoh_exact=False, path="auto"):
+    dev = torch.device("cuda")
+    t = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev) for k, v in d.items()}
+    keep = t.get("keep_idx")
+    shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, dir_flags, keep, h, w, pool_scale, zoh_exact,
+                            path)
+    fws = ssm.alloc_workspace(shape, dev)
+    fws.fill_(0xFF)
+    ssm.forward(t["x"], t["z"], t["A_log"], t["D"], t["W_x"], t["W_dt"], t["b_dt"], pool_axis, dir_flags,
+                keep_idx=keep, h=h, w=w, pool_scale=pool_scale, zoh_exact=zoh_exact, workspace=fws, path=path)
+    fstatus = ssm.device_status(fws)
+    bws = torch.full((max(ssm.backward_workspace_size(shape), 256),), 0xFF, dtype=torch.uint8, device=dev)
+    grads = {"dx": torch.full_like(t["x"], float("nan")), "dz": torch.full_like(t["z"], float("nan"))}
+    for name in PARAMS:
+        grads["d" + name] = torch.full_like(t[name], float("nan"))
+    ssm.backward(t["x"], t["z"], t["A_log"], t["D"], t["W_x"], t["W_dt"], t["b_dt"], t["dy"], fws, pool_axis,
+                 dir_flags, keep_idx=keep, h=h, w=w, pool_scale=pool_scale, zoh_exact=zoh_exact, path=path,
+                 grads=grads, workspace=bws)
+    torch.cuda.synchronize()
+    return {k: v.cpu().numpy() for k, v in grads.items()}, fstatus, ssm.backward_launch_names(shape)
+
+
+def oracle_grads(d, pool_axis, dir_flags, h, w, pool_scale=1.0, zoh_exact=False, allow_bad_index=False):
+    return oracle.backward(d["x"], d["z"], d["A_log"], d["D"], d["W_x"], d["W_dt"], d["b_dt"], d["dy"], pool_axis,
+                           dir_flags, keep_idx=d.get("keep_idx"), h=h, w=w, pool_scale=pool_scale, zoh_exact=zoh_exact,
+                           nthreads=8, allow_bad_index=allow_bad_index)
+
+
+def compare(got, ref, what):
+    reps = {}
+    for k in ("dx", "dz"):
+        reps[k] = assert_close(got[k], ref[k], f"{what} {k}")
+    for name in PARAMS:
+        reps["d" + name] = assert_close(got["d" + name], ref["d" + name], f"{what} d{name}", GRAD_PARAM_ABS_RMS)
+    print(what, {k: (round(v["max_abs_over_rms"], 9), round(v["max_err_over_bound"], 4)) for k, v in reps.items()})
+    return reps
+
+
+DENSE = [
+    # B, h, w, E, N, R, pool_axis, dir_flags, zoh_exact, pool_scale, path
+    (2, 14, 14, 384, 16, 12, 0, 3, False, 1.0, "auto"),
+    (2, 14, 14, 384, 16, 12, 1, 3, False, 1.0, "auto"),
+    (3, 13, 7, 68, 5, 3, 0, 1, False, 1.0, "staged"),
+    (3, 13, 7, 68, 5, 3, 1, 2, True, 0.25, "staged"),
+    (2, 40, 3, 132, 16, 7, 0, 3, False, 1.0, "staged"),
+    (2, 5, 37, 64, 16, 4, 1, 3, True, 1.0, "staged"),
+    (2, 16, 9, 256, 16, 16, 0, 3, False, 1.0, "staged"),
+    (1, 1, 1, 4, 1, 1, 0, 3, False, 1.0, "staged"),
+    (2, 64, 64, 1024, 16, 64, 0, 3, False, 1.0, "fused"),
+    (2, 64, 64, 1024, 16, 64, 0, 3, False, 1.0, "staged"),
+]
+
+
+@pytest.mark.parametrize("case", DENSE, ids=lambda c: "x".join(map(str, c[:6])) + f"-a{c[6]}d{c[7]}z{int(c[8])}{c[10]}")
+def test_dense_gradient(case):
+    B, h, w, E, N, R, axis, dirs, zoh, scale, path = case
+    nd = bin(dirs).count("1")
+    d = make_inputs(7, B, h, w, E, N, R, nd)
+    got, fst, names = gpu_grads(d, axis, dirs, h, w, scale, zoh, path)
+    assert fst == 0
+    assert names[0] == "bwd_gate_dense_kernel" and len(names) == 7
+    ref = oracle_grads(d, axis, dirs, h, w, scale, zoh)
+    compare(got, ref, f"dense {case}")
+
+
+@pytest.mark.parametrize("pool_axis", [0, 1])
+@pytest.mark.parametrize("zoh", [False, True])
+def test_masked_gradient_with_an_empty_row(pool_axis, zoh):
+    h, w, E, N, R, K = 16, 16, 132, 16, 8, 100
+    d = make_inputs(11, 2, h, w, E, N, R, 2, K=K, drop_row=3, pool_axis=pool_axis)
+    got, fst, names = gpu_grads(d, pool_axis, 3, h, w, 1.0, zoh)
+    assert fst == 0 and names[0] == "bwd_gate_masked_kernel"
+    ref = oracle_grads(d, pool_axis, 3, h, w, 1.0, zoh)
+    compare(got, ref, f"masked axis {pool_axis} zoh {zoh}")
+
+
+def test_masked_gradient_rejected_id():
+    """A repeated id: one copy is rejected (the forward reports FV_ERR_INDEX) and gets zero
+    gradients.  Both copies carry the same x, z and dy, so the result is the same whichever copy
+    the device keeps; compare the pair as a set and everything else element by element."""
+    h, w, E, N, R, K = 8, 8, 64, 16, 4, 20
+    d = make_inputs(13, 2, h, w, E, N, R, 2, K=K)
+    k1, k2 = 2, 9
+    d["keep_idx"][0, k2] = d["keep_idx"][0, k1]
+    for key in ("x", "z", "dy"):
+        d[key][0, k2] = d[key][0, k1]
+    got, fst, _ = gpu_grads(d, 0, 3, h, w)
+    assert fst == 4  # FV_ERR_INDEX
+    ref = oracle_grads(d, 0, 3, h, w, allow_bad_index=True)
+    assert ref["status"] == oracle.FVO_BAD_INDEX
+    for key in ("dx", "dz"):
+        g, r = got[key][0], ref[key][0]
+        pair_g = sorted([g[k1], g[k2]], key=lambda v: float(np.abs(v).sum()))
+        pair_r = sorted([r[k1], r[k2]], key=lambda v: float(np.abs(v).sum()))
+        assert not pair_g[0].any() and not pair_r[0].any()
+        assert_close(pair_g[1], pair_r[1], f"kept copy {key}")
+        rest = [k for k in range(K) if k not in (k1, k2)]
+        assert_close(g[rest], r[rest], f"other tokens {key}")
+        assert_close(got[key][1], ref[key][1], f"clean sample {key}")
+    for name in PARAMS:
+        assert_close(got["d" + name], ref["d" + name], f"d{name}", GRAD_PARAM_ABS_RMS)
+
+
+def test_empty_batch_zeroes_the_parameter_gradients():
+    d = make_inputs(3, 0, 4, 4, 8, 2, 1, 2)
+    got, fst, names = gpu_grads(d, 0, 3, 4, 4)
+    assert names == []
+    for name in PARAMS:
+        assert got["d" + name].shape == d[name].shape and not got["d" + name].any()
+
+
+def test_gradient_is_reproducible_up_to_atomic_order():
+    d = make_inputs(5, 2, 16, 16, 128, 16, 8, 2)
+    a, _, _ = gpu_grads(d, 0, 3, 16, 16)
+    b, _, _ = gpu_grads(d, 0, 3, 16, 16)
+    # dz depends on the forward's ys only (order-independent): identical; dx and the parameter
+    # gradients go through atomic sums and may differ in the last bits
+    np.testing.assert_array_equal(a["dz"], b["dz"])
+    for name in PARAMS:
+        np.testing.assert_allclose(a["d" + name], b["d" + name], rtol=1e-5, atol=1e-6 * np.abs(b["d" + name]).max())
