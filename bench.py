@@ -151,6 +151,8 @@ def load_peaks():
 # Sources each recorded kernel is built from (the traffic record is void once any of them changes).
 KERNEL_SOURCES = {
     "fused_layer_kernel": ("fastvim_ssm.cu", "fv_common.cuh", "fv_fused.cuh", "fv_scan.cuh"),
+    "bwd_gate_dense_kernel": ("fastvim_ssm.cu", "fv_common.cuh", "fv_kernels.cuh", "fv_backward.cuh"),
+    "bwd_pool_dense_kernel": ("fastvim_ssm.cu", "fv_common.cuh", "fv_kernels.cuh", "fv_backward.cuh"),
 }
 
 
@@ -635,10 +637,10 @@ def run_grad(a, cfg, pool_axis):
     bound, amount = kernel_work(dom, cfg, pool_axis)
     roofline = {"bound": bound if bound == "hbm" else "alu", "kernel": dom, "achieved": dk.get("achieved"),
                 "peak": peak if bound == "hbm" else (mufu_peak if bound == "alu" else fma_peak), "unit": dk.get("unit"),
-                "frac": dk.get("frac"), "traffic": None,
+                "frac": dk.get("frac"), "traffic": recorded_traffic(dom, cfg.name) if cfg.B == 128 else None,
                 "algorithmic_per_launch": amount, "peak_source": peak_src if bound == "hbm" else "derived",
                 "note": "dominant kernel of the gradient; achieved = algorithmic amount per launch / mean "
-                        "CUDA-event duration of the launch; no ncu capture of the gradient kernels yet"}
+                        "CUDA-event duration of the launch"}
     # the gradient's own HBM floor: read x, z, dy, write dx, dz (5 rows per token)
     bwd_ms = sum(statistics.mean(per_kernel[n]) for n in dict.fromkeys(bwd.names))
     line = {

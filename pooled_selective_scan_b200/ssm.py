@@ -220,8 +220,10 @@ class BoundForward:
 def backward_workspace_size(shape: LayerShape) -> int:
     a = shape.args()
     n = nat.lib().fastvim_ssm_backward_workspace_size(ctypes.byref(a))
-    if n == 0:
-        nat.check(nat.lib().fastvim_ssm_validate(ctypes.byref(a)), "fastvim_ssm_backward_workspace_size")
+    if n == 0:  # an empty batch needs none; otherwise the shape is invalid
+        L = nat.FvBwdWsLayout()
+        nat.check(nat.lib().fastvim_ssm_backward_workspace_layout(ctypes.byref(a), ctypes.byref(L)),
+                  "fastvim_ssm_backward_workspace_size")
     return int(n)
 
 
