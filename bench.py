@@ -78,9 +78,7 @@ def kernel_work(name: str, cfg, pool_axis: int):
     if name.startswith("bwd_gemm_kernel"):
         J = cfg.R + 2 * cfg.N
         M = cfg.B * T
-        flops = {"bwd_gemm_kernel:dt_low": 2 * M * cfg.E * cfg.R * cfg.nd,
-                 "bwd_gemm_kernel:W_dt": 2 * M * cfg.E * (cfg.R + 1) * cfg.nd,
-                 "bwd_gemm_kernel:W_x": 2 * M * cfg.E * J * cfg.nd,
+        flops = {"bwd_gemm_kernel:W_x": 2 * M * cfg.E * J * cfg.nd,
                  "bwd_gemm_kernel:xbar": 2 * M * cfg.E * J * cfg.nd}
         return "fma", flops.get(name, 0)
     return None, 0

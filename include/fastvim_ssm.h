@@ -269,9 +269,8 @@ typedef struct {
     size_t dys;          /* float [B][T][E]   dL/dys: ds summed over each pooled row's tokens  */
     size_t dxbar;        /* float [B][T][E]   dL/dxbar                                         */
     size_t du;           /* float, the layout of the forward's u: d dt_low | dB | dC           */
-    size_t dv;           /* float [B][nd][T][E]  dL/dv, v = the softplus input of Delta         */
     size_t dxs;          /* float [B][nd][T][E]  the scans' share of dL/dxbar per direction     */
-    size_t ckpt;         /* float [B][nd][ceil(T/16)][E][16]  scan state entering each 16-step chunk */
+    size_t ckpt;         /* float [B][nd][2 ceil(T/16)][E][16]  scan state entering every 8 steps */
 } fv_bwd_ws_layout;
 
 /* Workspace bytes a gradient call needs (0 when the arguments are invalid). */

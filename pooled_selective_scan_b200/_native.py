@@ -89,7 +89,7 @@ class FvSsmGrads(ctypes.Structure):
 
 
 class FvBwdWsLayout(ctypes.Structure):
-    _fields_ = [(name, ctypes.c_size_t) for name in ("total_bytes", "dys", "dxbar", "du", "dv", "dxs", "ckpt")]
+    _fields_ = [(name, ctypes.c_size_t) for name in ("total_bytes", "dys", "dxbar", "du", "dxs", "ckpt")]
 
 
 class FastvimError(RuntimeError):

@@ -923,7 +923,7 @@ extern "C" fv_status fastvim_ssm_forward_noalloc(const fv_ssm_args* args, void* 
 namespace {
 
 struct BwdLayout {
-    size_t dys, dxbar, du, dv, dxs, ckpt, total;
+    size_t dys, dxbar, du, dxs, ckpt, total;
 };
 
 BwdLayout plan_bwd(const fv::Shape& sh) {
@@ -933,26 +933,23 @@ BwdLayout plan_bwd(const fv::Shape& sh) {
     L.dys = off; off = round256(off + bte);
     L.dxbar = off; off = round256(off + bte);
     L.du = off; off = round256(off + (size_t)sh.nd * sh.B * fv::u_block_stride(sh.T, sh.J) * sizeof(float));
-    L.dv = off; off = round256(off + (size_t)sh.nd * bte);
     L.dxs = off; off = round256(off + (size_t)sh.nd * bte);
     L.ckpt = off;
-    off = round256(off + (size_t)sh.B * sh.nd * fv::bs_nchunks(sh.T) * sh.E * 16 * sizeof(float));
+    off = round256(off + (size_t)sh.B * sh.nd * fv::bs_nckpt(sh.T) * sh.E * 16 * sizeof(float));
     L.total = off;
     return L;
 }
 
-// Launch order of a gradient call: gate, scans, d dt_low, dW_dt | db_dt, dW_x, dxbar, pooling.
+// Launch order of a gradient call: gate, scans (with dt_proj), dW_x, dxbar, pooling.
 const char* bwd_launch_name_of(const fv::Shape& sh, int i) {
-    static const char* dense[] = {"bwd_gate_dense_kernel", "bwd_scan_kernel", "bwd_gemm_kernel:dt_low",
-                                  "bwd_gemm_kernel:W_dt", "bwd_gemm_kernel:W_x", "bwd_gemm_kernel:xbar",
-                                  "bwd_pool_dense_kernel"};
-    static const char* masked[] = {"bwd_gate_masked_kernel", "bwd_scan_kernel", "bwd_gemm_kernel:dt_low",
-                                   "bwd_gemm_kernel:W_dt", "bwd_gemm_kernel:W_x", "bwd_gemm_kernel:xbar",
-                                   "bwd_pool_masked_kernel"};
-    if (sh.B == 0 || i < 0 || i >= 7) return "";
+    static const char* dense[] = {"bwd_gate_dense_kernel", "bwd_scan_kernel", "bwd_gemm_kernel:W_x",
+                                  "bwd_gemm_kernel:xbar", "bwd_pool_dense_kernel"};
+    static const char* masked[] = {"bwd_gate_masked_kernel", "bwd_scan_kernel", "bwd_gemm_kernel:W_x",
+                                   "bwd_gemm_kernel:xbar", "bwd_pool_masked_kernel"};
+    if (sh.B == 0 || i < 0 || i >= 5) return "";
     return sh.K > 0 ? masked[i] : dense[i];
 }
-int bwd_launch_count_of(const fv::Shape& sh) { return sh.B == 0 ? 0 : 7; }
+int bwd_launch_count_of(const fv::Shape& sh) { return sh.B == 0 ? 0 : 5; }
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     const uintptr_t a0 = (uintptr_t)a, b0 = (uintptr_t)b;
@@ -1050,7 +1047,6 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
     float* dys = (float*)(ws + L.dys);
     float* dxbar = (float*)(ws + L.dxbar);
     float* du = (float*)(ws + L.du);
-    float* dv = (float*)(ws + L.dv);
     float* dxs = (float*)(ws + L.dxs);
     float* ckpt = (float*)(ws + L.ckpt);
     // the scans add dB and dC into du
@@ -1099,30 +1095,21 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
                 return FV_ERR_CUDA;
             }
             fv::bwd_scan_kernel<true><<<grid, fv::kBsThreads, scan_smem, st>>>(sh, u, xbar, dys, a->A_log, a->W_dt, a->b_dt,
-                                                                              ckpt, dv, dxs, du, g->dA_log);
+                                                                              ckpt, dxs, du, g->dA_log, g->dW_dt,
+                                                                              g->db_dt);
         } else {
             if ((e = ensure_smem(fv::bwd_scan_kernel<false>, scan_smem)) != cudaSuccess) {
                 note_cuda(e, "scan gradient smem attribute");
                 return FV_ERR_CUDA;
             }
             fv::bwd_scan_kernel<false><<<grid, fv::kBsThreads, scan_smem, st>>>(sh, u, xbar, dys, a->A_log, a->W_dt,
-                                                                               a->b_dt, ckpt, dv, dxs, du, g->dA_log);
+                                                                               a->b_dt, ckpt, dxs, du, g->dA_log,
+                                                                               g->dW_dt, g->db_dt);
         }
         FV_LAUNCH_CHECK("bwd_scan_kernel");
         return FV_OK;
     })());
-    // 3. dt_proj: d dt_low = dv W_dt (into du), then dW_dt | db_dt = dv^T [dt_low | 1]
-    FV_MARK_CALL(marks, st, launch_bwd_gemm(M, sh.R, sh.E, sh.nd, 1, fv::OpDvMK{dv, sh.T, sh.E, sh.nd},
-                                            fv::OpWdt{a->W_dt, sh.E, sh.R}, fv::OutDtl{du, sh}, st,
-                                            "bwd_gemm_kernel (dt_low)"));
-    {
-        const int tiles = ((sh.E + 63) / 64) * ((sh.R + 1 + 63) / 64) * sh.nd;
-        FV_MARK_CALL(marks, st, launch_bwd_gemm(sh.E, sh.R + 1, M, sh.nd, bwd_splits(M, tiles, sms),
-                                                fv::OpDvEM{dv, sh.T, sh.E, sh.nd}, fv::OpDtlOne{u, sh},
-                                                fv::OutWdtBdt{g->dW_dt, g->db_dt, sh.E, sh.R}, st,
-                                                "bwd_gemm_kernel (W_dt)"));
-    }
-    // 4. x_proj: dW_x = du^T xbar, dxbar = the scans' share + sum_k du[k] W_x[k]
+    // 3. x_proj: dW_x = du^T xbar, dxbar = the scans' share + sum_k du[k] W_x[k]
     {
         const int tiles = ((sh.J + 63) / 64) * ((sh.E + 63) / 64) * sh.nd;
         FV_MARK_CALL(marks, st, launch_bwd_gemm(sh.J, sh.E, M, sh.nd, bwd_splits(M, tiles, sms), fv::OpDuJM{du, sh},
@@ -1132,7 +1119,7 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
     FV_MARK_CALL(marks, st, launch_bwd_gemm(M, sh.E, sh.nd * sh.J, 1, 1, fv::OpDuMK{du, sh}, fv::OpWx{a->W_x, sh.E},
                                             fv::OutDxbar{dxbar, dxs, sh.T, sh.E, sh.nd}, st,
                                             "bwd_gemm_kernel (xbar)"));
-    // 5. pooling
+    // 4. pooling
     if (sh.K == 0) {
         const int threads = fv::bwd_groups(sh.SL) * fv::bwd_slot_width(sh.SL);
         FV_MARK_CALL(marks, st, ([&]() -> fv_status {
@@ -1170,7 +1157,7 @@ fv_status fastvim_ssm_backward_workspace_layout(const fv_ssm_args* args, fv_bwd_
     if (s != FV_OK) return s;
     const BwdLayout L = plan_bwd(sh);
     out->total_bytes = L.total;
-    out->dys = L.dys; out->dxbar = L.dxbar; out->du = L.du; out->dv = L.dv; out->dxs = L.dxs; out->ckpt = L.ckpt;
+    out->dys = L.dys; out->dxbar = L.dxbar; out->du = L.du; out->dxs = L.dxs; out->ckpt = L.ckpt;
     return FV_OK;
 }
 

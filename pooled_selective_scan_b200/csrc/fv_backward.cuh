@@ -7,11 +7,10 @@
 //   bwd_gate_dense_kernel / bwd_gate_masked_kernel   gate, skip and repeat: dz, the skip part of
 //                                                    dx, dD, and dys = the sum of ds over the
 //                                                    tokens of each pooled row
-//   bwd_scan_kernel                                  adjoint of both scans: dDelta (as dv = dDelta
-//                                                    sig(v) for dt_proj), dB, dC, dA_log and the
-//                                                    scans' share of dxbar
-//   bwd_gemm_kernel (4 launches)                     dt_proj and x_proj: d dt_low, dW_dt | db_dt,
-//                                                    dW_x, dxbar
+//   bwd_scan_kernel                                  adjoint of both scans: dDelta, and through
+//                                                    dt_proj + softplus d dt_low, dW_dt, db_dt; dB,
+//                                                    dC, dA_log and the scans' share of dxbar
+//   bwd_gemm_kernel (2 launches)                     x_proj: dW_x, dxbar
 //   bwd_pool_dense_kernel / bwd_pool_masked_kernel   pooling: dx += pool_scale / S dxbar of the
 //                                                    token's row
 // Inputs of the forward that the gradient reuses (xbar, the projections u, ys and, masked, the
@@ -26,9 +25,12 @@ namespace fv {
 
 constexpr int kBsCh = 64;        // channels per scan-gradient CTA
 constexpr int kBsThreads = 256;  // 4 lanes per channel, 4 states per lane
-constexpr int kBsChunk = 16;     // steps per checkpointed chunk
+constexpr int kBsChunk = 16;     // steps per staged chunk
+constexpr int kBsHalf = 8;       // steps per checkpoint (two per staged chunk)
 
 __host__ __device__ __forceinline__ int bs_nchunks(int T) { return (T + kBsChunk - 1) / kBsChunk; }
+// checkpoints per scan: one every 8 steps of the scan order
+__host__ __device__ __forceinline__ int bs_nckpt(int T) { return 2 * bs_nchunks(T); }
 // Row stride of the W_dt rows in shared memory: odd, so lanes reading 32 different rows at the
 // same column hit 32 different banks.
 __host__ __device__ __forceinline__ int bs_wstride(int R) { return R | 1; }
@@ -38,7 +40,8 @@ __host__ __device__ __forceinline__ size_t bs_smem_floats(int R) {
            + (size_t)kBsChunk * 32            // B | C of the chunk's steps
            + 6 * (size_t)kBsChunk * kBsCh     // xbar, dys, Delta, sig(v), dv, dxbar (scan share)
            + (size_t)kBsChunk * 32            // dB | dC sums of the chunk
-           + kBsCh;                           // b_dt of the CTA's channels
+           + kBsCh                            // b_dt of the CTA's channels
+           + (size_t)kBsCh * (R + 1);         // dW_dt | db_dt sums of the CTA's channels
 }
 
 // sigmoid(v) = 1 / (1 + e^-v) on the SFU (v -> -inf gives 0, v -> +inf gives 1).
@@ -236,20 +239,24 @@ bwd_gate_masked_kernel(Shape sh, const float* __restrict__ x, const float* __res
 //             or (Abar_i - 1) / A B_i xbar_i (exact ZOH);  ys += C_i . h_i
 //   adjoint   lam_i = C_i dys_i + Abar_{i+1} lam_{i+1}  (lam = 0 past the last step)
 //             dC_i += dys_i h_i;  dAbar_i = lam_i h_{i-1};  dq_i = lam_i
-// Pass 1 runs the recurrence in scan order and stores the state entering every 16-step chunk
-// (ckpt [B][nd][nchunks][E][16]).  Pass 2 walks the chunks in reverse: it recomputes the chunk's
-// states from its checkpoint (16 steps x 4 states in registers) and steps the adjoint back through
-// them.  Per step: dDelta and the scans' dxbar are summed over the 4 lanes of a channel (written as
+// Pass 1 runs the recurrence in scan order and stores the state entering every 8 steps
+// (ckpt [B][nd][2 nchunks][E][16]).  Pass 2 walks the 16-step staged chunks in reverse, each as two
+// halves of 8 steps, last half first: it recomputes the half's states from its checkpoint (8 steps
+// x 4 states in registers, which keeps the kernel at two resident blocks per SM) and steps the
+// adjoint back through them.  Per step: dDelta and the scans' dxbar are summed over the 4 lanes of a channel (written as
 // dv = dDelta sig(v) and dxs [B][nd][T][E]); dB and dC are summed over the warp's 8 channels by a
 // transposing butterfly, over the block's 8 warps in shared memory, and over the E / 64 blocks of
 // an image with global atomics into du (zeroed by the caller).  dA_log (= dA A) sums in registers
-// over all steps, then one atomic per state.
+// over all steps, then one atomic per state.  dt_proj (v = W_dt dt_low + b_dt) is differentiated
+// here too, from the chunk's dv and dt_low already in shared memory: d dt_low[t] = sum over the
+// block's channels of W_dt[e] dv[t][e] (atomics into du's dt_low slots), dW_dt[e] and db_dt[e] =
+// sums over the steps of dv[t][e] [dt_low[t] | 1] (shared memory, one atomic each at the end).
 template <bool ZOH_EXACT>
-__global__ void __launch_bounds__(kBsThreads, 1)
+__global__ void __launch_bounds__(kBsThreads, 2)
 bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__ xbar, const float* __restrict__ dys,
                 const float* __restrict__ A_log, const float* __restrict__ W_dt, const float* __restrict__ b_dt,
-                float* __restrict__ ckpt, float* __restrict__ dv, float* __restrict__ dxs, float* __restrict__ du,
-                float* __restrict__ dA_log) {
+                float* __restrict__ ckpt, float* __restrict__ dxs, float* __restrict__ du,
+                float* __restrict__ dA_log, float* __restrict__ dW_dt, float* __restrict__ db_dt) {
     extern __shared__ float bsm[];
     const int b = blockIdx.x, k = blockIdx.y, e0 = blockIdx.z * kBsCh;
     const int T = sh.T, E = sh.E, N = sh.N, R = sh.R, J = sh.J;
@@ -265,19 +272,22 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
     float* sdx = sdv + kBsChunk * kBsCh;      // [16][64]
     float* sred = sdx + kBsChunk * kBsCh;     // [16][32]
     float* sbias = sred + kBsChunk * 32;      // [64]
+    float* swacc = sbias + kBsCh;             // [64][R + 1]
     const int tid = threadIdx.x;
     const int c = tid >> 2, q = tid & 3, lane = tid & 31;
     const int e = e0 + c;
     const bool live = e < E;
     const bool fwd = sh.nd == 2 ? k == 0 : (sh.dir_flags & 1u) != 0;
-    const int nchunks = bs_nchunks(T);
+    const int nchunks = bs_nchunks(T), nckpt = bs_nckpt(T);
     const float* ub = u + u_offset(sh, k, b, 0);
+    auto ckpt_at = [&](int c) { return ckpt + ((((size_t)b * sh.nd + k) * nckpt + c) * E + e) * 16 + 4 * q; };
 
     for (int i = tid; i < kBsCh * R; i += kBsThreads) {
         const int row = i / R, r = i - row * R;
         sw[row * WS + r] = (e0 + row < E) ? __ldg(W_dt + ((size_t)k * E + e0 + row) * R + r) : 0.f;
     }
     for (int i = tid; i < kBsCh; i += kBsThreads) sbias[i] = (e0 + i < E) ? __ldg(b_dt + (size_t)k * E + e0 + i) : 0.f;
+    for (int i = tid; i < kBsCh * (R + 1); i += kBsThreads) swacc[i] = 0.f;
 
     constexpr float kLog2e = 1.4426950408889634f;
     float A2[4], An[4], Ainv[4];
@@ -336,11 +346,10 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
     float h[4] = {0.f, 0.f, 0.f, 0.f};
     for (int it = 0; it < nchunks; ++it) {
         stage(it, false);
-        if (live)
-            *reinterpret_cast<float4*>(ckpt + ((((size_t)b * sh.nd + k) * nchunks + it) * E + e) * 16 + 4 * q) =
-                make_float4(h[0], h[1], h[2], h[3]);
         const int len = chunk_len(it);
         for (int i = 0; i < len; ++i) {
+            if (live && (i == 0 || i == kBsHalf))
+                *reinterpret_cast<float4*>(ckpt_at(2 * it + i / kBsHalf)) = make_float4(h[0], h[1], h[2], h[3]);
             const float dt = sdl[i * kBsCh + c], xv = sx[i * kBsCh + c];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -359,103 +368,121 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
     for (int it = nchunks - 1; it >= 0; --it) {
         stage(it, true);
         const int len = chunk_len(it);
-        float hin[4] = {0.f, 0.f, 0.f, 0.f};
-        if (live) {
-            const float4 v = *reinterpret_cast<const float4*>(
-                ckpt + ((((size_t)b * sh.nd + k) * nchunks + it) * E + e) * 16 + 4 * q);
-            hin[0] = v.x; hin[1] = v.y; hin[2] = v.z; hin[3] = v.w;
-        }
-        float hist[kBsChunk][4];
-        {
-            float hc[4] = {hin[0], hin[1], hin[2], hin[3]};
+        for (int half = (len - 1) / kBsHalf; half >= 0; --half) {
+            const int i0 = half * kBsHalf, hl = min(kBsHalf, len - i0);
+            float hin[4] = {0.f, 0.f, 0.f, 0.f};
+            if (live) {
+                const float4 v = *reinterpret_cast<const float4*>(ckpt_at(2 * it + half));
+                hin[0] = v.x; hin[1] = v.y; hin[2] = v.z; hin[3] = v.w;
+            }
+            float hist[kBsHalf][4];
+            {
+                float hc[4] = {hin[0], hin[1], hin[2], hin[3]};
 #pragma unroll
-            for (int i = 0; i < kBsChunk; ++i) {
-                if (i < len) {
-                    const float dt = sdl[i * kBsCh + c], xv = sx[i * kBsCh + c];
+                for (int ii = 0; ii < kBsHalf; ++ii) {
+                    const int i = i0 + ii;
+                    if (ii < hl) {
+                        const float dt = sdl[i * kBsCh + c], xv = sx[i * kBsCh + c];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float Bn = sbc[i * 32 + 4 * q + j];
-                        hc[j] = fmaf(ex2_approx(dt * A2[j]), hc[j], qterm(dt, Bn, xv, j));
-                        hist[i][j] = hc[j];
+                        for (int j = 0; j < 4; ++j) {
+                            const float Bn = sbc[i * 32 + 4 * q + j];
+                            hc[j] = fmaf(ex2_approx(dt * A2[j]), hc[j], qterm(dt, Bn, xv, j));
+                            hist[ii][j] = hc[j];
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) hist[ii][j] = 0.f;
                     }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) hist[i][j] = 0.f;
                 }
             }
-        }
 #pragma unroll
-        for (int ii = 0; ii < kBsChunk; ++ii) {
-            const int i = kBsChunk - 1 - ii;
-            if (i < len) {
-                const float dt = sdl[i * kBsCh + c], xv = sx[i * kBsCh + c], gy = sdy[i * kBsCh + c];
-                float ddt = 0.f, dxb = 0.f, vals[8];
+            for (int r = 0; r < kBsHalf; ++r) {
+                const int ii = kBsHalf - 1 - r;
+                const int i = i0 + ii;
+                if (ii < hl) {
+                    const float dt = sdl[i * kBsCh + c], xv = sx[i * kBsCh + c], gy = sdy[i * kBsCh + c];
+                    float ddt = 0.f, dxb = 0.f, vals[8];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float Bn = sbc[i * 32 + 4 * q + j], Cn = sbc[i * 32 + 16 + 4 * q + j];
-                    const float Ab = ex2_approx(dt * A2[j]);
-                    const float hp = i > 0 ? hist[i > 0 ? i - 1 : 0][j] : hin[j];
-                    lam[j] = fmaf(Anext[j], lam[j], Cn * gy);
-                    vals[4 + j] = gy * hist[i][j];
-                    const float t1 = lam[j] * hp * Ab;
-                    ddt = fmaf(t1, An[j], ddt);
-                    gA[j] = fmaf(t1, dt, gA[j]);
-                    if (ZOH_EXACT) {
-                        const float em = expm1f(dt * An[j]);
-                        const float cf = em * Ainv[j];
-                        ddt = fmaf(lam[j] * Ab, Bn * xv, ddt);
-                        gA[j] = fmaf(lam[j] * Bn * xv, (dt * Ab * An[j] - em) * Ainv[j] * Ainv[j], gA[j]);
-                        vals[j] = lam[j] * cf * xv;
-                        dxb = fmaf(lam[j] * cf, Bn, dxb);
-                    } else {
-                        ddt = fmaf(lam[j], Bn * xv, ddt);
-                        vals[j] = lam[j] * dt * xv;
-                        dxb = fmaf(lam[j] * dt, Bn, dxb);
+                    for (int j = 0; j < 4; ++j) {
+                        const float Bn = sbc[i * 32 + 4 * q + j], Cn = sbc[i * 32 + 16 + 4 * q + j];
+                        const float Ab = ex2_approx(dt * A2[j]);
+                        const float hp = ii > 0 ? hist[ii > 0 ? ii - 1 : 0][j] : hin[j];
+                        lam[j] = fmaf(Anext[j], lam[j], Cn * gy);
+                        vals[4 + j] = gy * hist[ii][j];
+                        const float t1 = lam[j] * hp * Ab;
+                        ddt = fmaf(t1, An[j], ddt);
+                        gA[j] = fmaf(t1, dt, gA[j]);
+                        if (ZOH_EXACT) {
+                            const float em = expm1f(dt * An[j]);
+                            const float cf = em * Ainv[j];
+                            ddt = fmaf(lam[j] * Ab, Bn * xv, ddt);
+                            gA[j] = fmaf(lam[j] * Bn * xv, (dt * Ab * An[j] - em) * Ainv[j] * Ainv[j], gA[j]);
+                            vals[j] = lam[j] * cf * xv;
+                            dxb = fmaf(lam[j] * cf, Bn, dxb);
+                        } else {
+                            ddt = fmaf(lam[j], Bn * xv, ddt);
+                            vals[j] = lam[j] * dt * xv;
+                            dxb = fmaf(lam[j] * dt, Bn, dxb);
+                        }
+                        Anext[j] = Ab;
                     }
-                    Anext[j] = Ab;
-                }
-                ddt += __shfl_xor_sync(0xffffffffu, ddt, 1);
-                ddt += __shfl_xor_sync(0xffffffffu, ddt, 2);
-                dxb += __shfl_xor_sync(0xffffffffu, dxb, 1);
-                dxb += __shfl_xor_sync(0xffffffffu, dxb, 2);
-                if (q == 0) {
-                    sdv[i * kBsCh + c] = ddt * ssg[i * kBsCh + c];
-                    sdx[i * kBsCh + c] = dxb;
-                }
-                // sum the 8 values over the warp's 8 channels (lane bits 2..4); each lane keeps one
-                float r1[4], r2[2];
+                    ddt += __shfl_xor_sync(0xffffffffu, ddt, 1);
+                    ddt += __shfl_xor_sync(0xffffffffu, ddt, 2);
+                    dxb += __shfl_xor_sync(0xffffffffu, dxb, 1);
+                    dxb += __shfl_xor_sync(0xffffffffu, dxb, 2);
+                    if (q == 0) {
+                        sdv[i * kBsCh + c] = ddt * ssg[i * kBsCh + c];
+                        sdx[i * kBsCh + c] = dxb;
+                    }
+                    // sum the 8 values over the warp's 8 channels (lane bits 2..4); each lane keeps one
+                    float r1[4], r2[2];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float send = b4 ? vals[j] : vals[j + 4];
-                    const float keep = b4 ? vals[j + 4] : vals[j];
-                    r1[j] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-                }
+                    for (int j = 0; j < 4; ++j) {
+                        const float send = b4 ? vals[j] : vals[j + 4];
+                        const float keep = b4 ? vals[j + 4] : vals[j];
+                        r1[j] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+                    }
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const float send = b3 ? r1[j] : r1[j + 2];
-                    const float keep = b3 ? r1[j + 2] : r1[j];
-                    r2[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+                    for (int j = 0; j < 2; ++j) {
+                        const float send = b3 ? r1[j] : r1[j + 2];
+                        const float keep = b3 ? r1[j + 2] : r1[j];
+                        r2[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+                    }
+                    const float send = b2 ? r2[0] : r2[1];
+                    const float keep = b2 ? r2[1] : r2[0];
+                    const float fin = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+                    if (red_n < N) atomicAdd(&sred[i * 32 + red_w * 16 + red_n], fin);
                 }
-                const float send = b2 ? r2[0] : r2[1];
-                const float keep = b2 ? r2[1] : r2[0];
-                const float fin = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-                if (red_n < N) atomicAdd(&sred[i * 32 + red_w * 16 + red_n], fin);
             }
         }
         __syncthreads();
         for (int i = tid; i < len * kBsCh; i += kBsThreads) {
             const int s = i / kBsCh, cc = i - s * kBsCh;
-            if (e0 + cc < E) {
-                const size_t o = (((size_t)b * sh.nd + k) * T + t_of(it, s)) * E + e0 + cc;
-                dv[o] = sdv[i];
-                dxs[o] = sdx[i];
-            }
+            if (e0 + cc < E) dxs[(((size_t)b * sh.nd + k) * T + t_of(it, s)) * E + e0 + cc] = sdx[i];
         }
         for (int i = tid; i < len * 32; i += kBsThreads) {
             const int s = i >> 5, j = i & 31, n = j & 15;
             if (n < N) atomicAdd(du + u_offset(sh, k, b, t_of(it, s)) + R + (j < 16 ? n : N + n), sred[i]);
         }
+        // dt_proj: d dt_low of the chunk's steps (this block's channels), dW_dt | db_dt partial sums
+        for (int i = tid; i < len * R; i += kBsThreads) {
+            const int s = i / R, r = i - s * R;
+            float acc = 0.f;
+            for (int cc = 0; cc < kBsCh; ++cc) acc = fmaf(sw[cc * WS + r], sdv[s * kBsCh + cc], acc);
+            atomicAdd(du + u_offset(sh, k, b, t_of(it, s)) + r, acc);
+        }
+        for (int i = tid; i < kBsCh * (R + 1); i += kBsThreads) {
+            const int cc = i / (R + 1), r = i - cc * (R + 1);
+            float acc = swacc[i];
+            for (int s = 0; s < len; ++s) acc = fmaf(sdv[s * kBsCh + cc], r < R ? sdtl[s * R + r] : 1.f, acc);
+            swacc[i] = acc;
+        }
         __syncthreads();  // the buffers are refilled by the next stage()
+    }
+    for (int i = tid; i < kBsCh * (R + 1); i += kBsThreads) {  // each entry was summed by this thread
+        const int cc = i / (R + 1), r = i - cc * (R + 1);
+        if (e0 + cc < E) atomicAdd(r < R ? dW_dt + ((size_t)k * E + e0 + cc) * R + r : db_dt + (size_t)k * E + e0 + cc,
+                                   swacc[i]);
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -473,40 +500,6 @@ constexpr int kBgTile = 64, kBgK = 16, kBgPad = kBgTile + 4;
 // Operand accessors.  kContig: the operand is contiguous along kk (A) or along j (B), which picks
 // the coalesced loading order.  k is the direction slot of the launch (blockIdx.z / splits).
 
-// A = dv[k][m][e] as (i = m, kk = e), for d dt_low = dv W_dt[k]
-struct OpDvMK {
-    static constexpr bool kContig = true;
-    const float* dv; int T, E, nd;
-    __device__ float operator()(int k, int i, int kk) const {
-        const int b = i / T, t = i - b * T;
-        return dv[(((size_t)b * nd + k) * T + t) * E + kk];
-    }
-};
-// A = dv[k][m][e] as (i = e, kk = m), for dW_dt = dv^T dt_low and db_dt = dv^T 1
-struct OpDvEM {
-    static constexpr bool kContig = false;
-    const float* dv; int T, E, nd;
-    __device__ float operator()(int k, int i, int kk) const {
-        const int b = kk / T, t = kk - b * T;
-        return dv[(((size_t)b * nd + k) * T + t) * E + i];
-    }
-};
-// B = W_dt[k][e][r] as (kk = e, j = r)
-struct OpWdt {
-    static constexpr bool kContig = true;
-    const float* W_dt; int E, R;
-    __device__ float operator()(int k, int kk, int j) const { return W_dt[((size_t)k * E + kk) * R + j]; }
-};
-// B = [dt_low | 1] as (kk = m, j = r <= R): column R is ones (gives db_dt)
-struct OpDtlOne {
-    static constexpr bool kContig = true;
-    const float* u; Shape sh;
-    __device__ float operator()(int k, int kk, int j) const {
-        if (j == sh.R) return 1.f;
-        const int b = kk / sh.T, t = kk - b * sh.T;
-        return u[u_offset(sh, k, b, t) + j];
-    }
-};
 // A = du[k][m][jj] as (i = jj, kk = m), for dW_x = du^T xbar
 struct OpDuJM {
     static constexpr bool kContig = false;
@@ -540,19 +533,6 @@ struct OpWx {
 };
 
 // Outputs.
-struct OutDtl {  // d dt_low into du (stored; the B and C slots hold the scans' sums)
-    float* du; Shape sh;
-    __device__ void operator()(int k, int i, int j, float v) const {
-        const int b = i / sh.T, t = i - b * sh.T;
-        du[u_offset(sh, k, b, t) + j] = v;
-    }
-};
-struct OutWdtBdt {  // split-K partial sums of dW_dt (j < R) and db_dt (j == R)
-    float* dW_dt; float* db_dt; int E, R;
-    __device__ void operator()(int k, int i, int j, float v) const {
-        atomicAdd(j < R ? dW_dt + ((size_t)k * E + i) * R + j : db_dt + (size_t)k * E + i, v);
-    }
-};
 struct OutWx {  // split-K partial sums of dW_x
     float* dW_x; int J, E;
     __device__ void operator()(int k, int i, int j, float v) const {

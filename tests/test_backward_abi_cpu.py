@@ -67,8 +67,8 @@ def test_workspace_plan(lib, pool_axis, K, dirs):
     J = 3 + 2 * 5
     ub = -(-T * J // 32) * 32
     regions = sorted([(L.dys, 3 * T * 68 * 4), (L.dxbar, 3 * T * 68 * 4), (L.du, nd * 3 * ub * 4),
-                      (L.dv, nd * 3 * T * 68 * 4), (L.dxs, nd * 3 * T * 68 * 4),
-                      (L.ckpt, 3 * nd * -(-T // 16) * 68 * 16 * 4)])
+                      (L.dxs, nd * 3 * T * 68 * 4),
+                      (L.ckpt, 3 * nd * 2 * -(-T // 16) * 68 * 16 * 4)])
     end = 0
     for off, n in regions:
         assert off % 256 == 0 and off >= end
@@ -77,15 +77,14 @@ def test_workspace_plan(lib, pool_axis, K, dirs):
 
 
 def test_launch_lists(lib):
-    dense = [lib.fastvim_ssm_backward_launch_name(ctypes.byref(args()), i).decode() for i in range(7)]
-    assert lib.fastvim_ssm_backward_launch_count(ctypes.byref(args())) == 7
-    assert dense[0] == "bwd_gate_dense_kernel" and dense[1] == "bwd_scan_kernel"
-    assert dense[-1] == "bwd_pool_dense_kernel"
-    assert all(n.startswith("bwd_gemm_kernel") for n in dense[2:6])
+    dense = [lib.fastvim_ssm_backward_launch_name(ctypes.byref(args()), i).decode() for i in range(5)]
+    assert lib.fastvim_ssm_backward_launch_count(ctypes.byref(args())) == 5
+    assert dense == ["bwd_gate_dense_kernel", "bwd_scan_kernel", "bwd_gemm_kernel:W_x", "bwd_gemm_kernel:xbar",
+                     "bwd_pool_dense_kernel"]
     m = args(K=49, keep_idx=FAKE + 9 * SLOT)
-    masked = [lib.fastvim_ssm_backward_launch_name(ctypes.byref(m), i).decode() for i in range(7)]
+    masked = [lib.fastvim_ssm_backward_launch_name(ctypes.byref(m), i).decode() for i in range(5)]
     assert masked[0] == "bwd_gate_masked_kernel" and masked[-1] == "bwd_pool_masked_kernel"
-    assert lib.fastvim_ssm_backward_launch_name(ctypes.byref(args()), 7) == b""
+    assert lib.fastvim_ssm_backward_launch_name(ctypes.byref(args()), 5) == b""
     assert lib.fastvim_ssm_backward_launch_count(ctypes.byref(args(B=0, x=None, z=None, y=None))) == 0
     ln = args(flags=nat.FV_FLAG_LAYERNORM, ln_gamma=FAKE + 10 * SLOT, ln_beta=FAKE + 11 * SLOT, ln_eps=1e-5)
     assert lib.fastvim_ssm_backward_launch_count(ctypes.byref(ln)) == 0
@@ -128,7 +127,7 @@ def test_rejections_before_any_launch(lib):
     # y is not read: NULL is accepted up to the first check it does not take part in
     assert _bwd(lib, args(y=None), grads(), ws=0) == nat.FV_ERR_WORKSPACE
     # too few events
-    ev = (ctypes.c_void_p * 4)()
+    ev = (ctypes.c_void_p * 4)()  # 5 launches need 10
     need_f = lib.fastvim_ssm_workspace_size(ctypes.byref(a))
     need_b = lib.fastvim_ssm_backward_workspace_size(ctypes.byref(a))
     assert lib.fastvim_ssm_backward_events(ctypes.byref(a), ctypes.byref(grads()), ctypes.c_void_p(FAKE + 20 * SLOT),
