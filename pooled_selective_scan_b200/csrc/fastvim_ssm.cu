@@ -974,6 +974,17 @@ fv_status check_grads(const fv_ssm_args* a, const fv::Shape& sh, const fv_ssm_gr
     return FV_OK;
 }
 
+// Tokens in flight per thread of the dense gate gradient: 2 (default) or 4; FASTVIM_BWD_GATE_UNROLL
+// overrides it (tuning only).  B200, 2048 px layer: 2 tokens (64 registers, 30 warps per SM)
+// stream at 0.945 of the copy rate, 4 tokens (99 registers, 18 warps) at 0.79.
+int bwd_gate_unroll() {
+    if (const char* env = getenv("FASTVIM_BWD_GATE_UNROLL")) {
+        const int v = atoi(env);
+        if (v == 2 || v == 4) return v;
+    }
+    return 2;
+}
+
 int device_sm_count() {
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
@@ -1068,10 +1079,15 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
     };
     if (sh.K == 0) {
         const int threads = fv::bwd_groups(sh.SL) * fv::bwd_slot_width(sh.SL);
-        const int grid = resident(fv::bwd_gate_dense_kernel, threads);
+        const bool u4 = bwd_gate_unroll() == 4;
+        const int grid = u4 ? resident(fv::bwd_gate_dense_kernel<4>, threads) : resident(fv::bwd_gate_dense_kernel<2>, threads);
         FV_MARK_CALL(marks, st, ([&]() -> fv_status {
-            fv::bwd_gate_dense_kernel<<<grid, threads, 0, st>>>(sh, a->x, a->z, g->dy, ys, a->D, g->dx, g->dz, dys,
-                                                                  g->dD);
+            if (u4)
+                fv::bwd_gate_dense_kernel<4><<<grid, threads, 0, st>>>(sh, a->x, a->z, g->dy, ys, a->D, g->dx, g->dz,
+                                                                         dys, g->dD);
+            else
+                fv::bwd_gate_dense_kernel<2><<<grid, threads, 0, st>>>(sh, a->x, a->z, g->dy, ys, a->D, g->dx, g->dz,
+                                                                         dys, g->dD);
             FV_LAUNCH_CHECK("bwd_gate_dense_kernel");
             return FV_OK;
         })());

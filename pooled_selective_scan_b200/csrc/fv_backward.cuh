@@ -92,6 +92,8 @@ __host__ __device__ __forceinline__ int bwd_groups(int SL) { return kThreads / b
 // Dense gate gradient, persistent over pooled rows (b, t) (grid-stride), launched with
 // bwd_groups(SL) * bwd_slot_width(SL) threads.  Writes dz and the skip part of dx for every token
 // of the row, dys[b][t] (the sum of ds over the row's S tokens), and adds the block's dD sums.
+// U tokens per thread in flight (3 U 128-bit loads).
+template <int U>
 __global__ void __launch_bounds__(kThreads)
 bwd_gate_dense_kernel(Shape sh, const float* __restrict__ x, const float* __restrict__ z,
                       const float* __restrict__ dy, const float* __restrict__ ys, const float* __restrict__ D,
@@ -119,17 +121,17 @@ bwd_gate_dense_kernel(Shape sh, const float* __restrict__ x, const float* __rest
                 const size_t base = (dense_base(sh, b, t) >> 2) + slot;
                 const float4 yv = reinterpret_cast<const float4*>(ys + (size_t)bt * sh.E)[slot];
                 int s = g;
-                for (; s + 3 * G < S; s += 4 * G) {  // four tokens, twelve loads in flight
-                    float4 xv[4], zv[4], gv[4];
+                for (; s + (U - 1) * G < S; s += U * G) {  // U tokens, 3 U loads in flight
+                    float4 xv[U], zv[U], gv[U];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
+                    for (int u = 0; u < U; ++u) {
                         const size_t o = base + (size_t)(s + u * G) * st4;
                         xv[u] = ld_stream(x4 + o);
                         zv[u] = ld_stream(z4 + o);
                         gv[u] = ld_stream(g4 + o);
                     }
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
+                    for (int u = 0; u < U; ++u) {
                         const size_t o = base + (size_t)(s + u * G) * st4;
                         float4 dzv, dxv;
                         gate_grad4(xv[u], zv[u], gv[u], yv, Ds, dzv, dxv, acc, dDa);
