@@ -61,8 +61,8 @@ def _load():
                 "fvo_gate_dense": [P, P, P, P, I, I, I, I, I, I, P, P, Dbl, P],
                 "fvo_gate_masked": [P, P, P, P, P, I, I, I, I, I, P, P, Dbl, P],
                 "fvo_forward": [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, U, Dbl, I, P, P, Dbl, I, P],
-                "fvo_backward": [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, U, Dbl, I, P, I,
-                                 P, P, P, P, P, P, P],
+                "fvo_backward": [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, U, Dbl, I, P, P, Dbl, P, I,
+                                 P, P, P, P, P, P, P, P, P],
             }
             for name, argtypes in sigs.items():
                 fn = getattr(lib, name)
@@ -270,12 +270,14 @@ def forward_intermediates(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis, dir_flags,
 
 
 def backward(x, z, A_log, D, W_x, W_dt, b_dt, dy, pool_axis, dir_flags, keep_idx=None, h=None, w=None,
-             pool_scale=1.0, zoh_exact=False, nthreads=1, allow_bad_index=False):
+             pool_scale=1.0, zoh_exact=False, nthreads=1, allow_bad_index=False, ln_gamma=None, ln_beta=None,
+             ln_eps=1e-5):
     """The gradient of the layer for the upstream gradient dy (layout of y), image by image.
 
     Returns a dict of fp64 arrays: dx, dz (layouts of x, z) and the parameter gradients summed
-    over the batch, dA_log, dD, dW_x, dW_dt, db_dt (layouts of the parameters); with
-    allow_bad_index, also the status under "status".
+    over the batch, dA_log, dD, dW_x, dW_dt, db_dt (layouts of the parameters), plus dln_gamma,
+    dln_beta when the post-SSM LayerNorm is given; with allow_bad_index, also the status under
+    "status".
     """
     x, z, dy = _f32(x), _f32(z), _f32(dy)
     A_log, D, W_x, W_dt, b_dt = map(_f32, (A_log, D, W_x, W_dt, b_dt))
@@ -290,13 +292,17 @@ def backward(x, z, A_log, D, W_x, W_dt, b_dt, dy, pool_axis, dir_flags, keep_idx
         idx = _i32(keep_idx)
         assert h is not None and w is not None and idx.shape == (B, K)
     assert E2 == E and z.shape == x.shape and dy.shape == x.shape and nd == nd_of(dir_flags)
+    g, b = _ln(ln_gamma, ln_beta, E)
     out = {"dx": np.empty(x.shape), "dz": np.empty(x.shape), "dA_log": np.empty(A_log.shape),
            "dD": np.empty(D.shape), "dW_x": np.empty(W_x.shape), "dW_dt": np.empty(W_dt.shape),
            "db_dt": np.empty(b_dt.shape)}
+    if g is not None:
+        out["dln_gamma"], out["dln_beta"] = np.empty(E), np.empty(E)
     st = _load().fvo_backward(_p(x), _p(z), _p(A_log), _p(D), _p(W_x), _p(W_dt), _p(b_dt), _p(idx), B, h, w, E,
-                              N, R, K, pool_axis, int(dir_flags), float(pool_scale), int(bool(zoh_exact)), _p(dy),
-                              int(nthreads), *(_p(out[k]) for k in ("dx", "dz", "dA_log", "dD", "dW_x", "dW_dt",
-                                                                    "db_dt")))
+                              N, R, K, pool_axis, int(dir_flags), float(pool_scale), int(bool(zoh_exact)), _p(g),
+                              _p(b), float(ln_eps), _p(dy), int(nthreads),
+                              *(_p(out[k]) for k in ("dx", "dz", "dA_log", "dD", "dW_x", "dW_dt", "db_dt")),
+                              _p(out.get("dln_gamma")), _p(out.get("dln_beta")))
     _check(st, "backward", allow=(FVO_BAD_INDEX,) if allow_bad_index else ())
     if allow_bad_index:
         out["status"] = st

@@ -86,13 +86,15 @@ int fvo_forward(const float* x, const float* z, const float* A_log, const float*
 
 /* The gradient of the layer (fastvim_oracle_grad.c): given dy = dL/dy (layout of y), writes
  * dx, dz (layouts of x, z) and the parameter gradients summed over the batch, dA_log [nd][E][N],
- * dD [nd][E], dW_x [nd][R+2N][E], dW_dt [nd][E][R], db_dt [nd][E].  No post-SSM LayerNorm.
+ * dD [nd][E], dW_x [nd][R+2N][E], dW_dt [nd][E][R], db_dt [nd][E]; with the post-SSM LayerNorm
+ * (ln_gamma, ln_beta [E], both or neither) also dln_gamma, dln_beta [E].
  * Tokens whose id is rejected (masked) get dx = dz = 0 and the call returns FVO_BAD_INDEX. */
 int fvo_backward(const float* x, const float* z, const float* A_log, const float* D, const float* W_x,
                  const float* W_dt, const float* b_dt, const int32_t* keep_idx, int B, int h, int w, int E,
                  int N, int R, int K, int pool_axis, unsigned dir_flags, double pool_scale, int zoh_exact,
-                 const float* dy, int nthreads, double* dx, double* dz, double* dA_log, double* dD,
-                 double* dW_x, double* dW_dt, double* db_dt);
+                 const float* ln_gamma, const float* ln_beta, double ln_eps, const float* dy, int nthreads,
+                 double* dx, double* dz, double* dA_log, double* dD, double* dW_x, double* dW_dt, double* db_dt,
+                 double* dln_gamma, double* dln_beta);
 
 #ifdef __cplusplus
 }

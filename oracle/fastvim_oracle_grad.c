@@ -7,7 +7,8 @@
  * derivative of the forward definition in fastvim_oracle.c, by the chain rule, one forward step
  * at a time in reverse order (gate, repeat + skip, scans, dt_proj + softplus, x_proj, pooling).
  * Plain loops in fp64, every forward intermediate recomputed with the forward oracle's own
- * functions.  The post-SSM LayerNorm is not covered (the GPU backward does not take it).
+ * functions.  With the post-SSM LayerNorm (ln_gamma, ln_beta given) the gate's adjoint goes
+ * through the normalisation of each token and also returns dln_gamma, dln_beta [E].
  *
  * Given dy = dL/dy for a scalar loss L, it returns dL/dx, dL/dz (same layout as x, z) and the
  * parameter gradients summed over the batch: dA_log [nd][E][N], dD [nd][E], dW_x [nd][R+2N][E],
@@ -44,15 +45,74 @@ typedef struct {
 
 /* Parameter gradients of one image (added into the caller's sums afterwards). */
 typedef struct {
-    double *dA_log, *dD, *dW_x, *dW_dt, *db_dt;
+    double *dA_log, *dD, *dW_x, *dW_dt, *db_dt, *dln_gamma, *dln_beta;
 } gparams;
+
+typedef struct {
+    const float *gamma, *beta;
+    double eps;
+} glnorm;
+
+/* Step 1 with the post-SSM LayerNorm, one token: s = ys_row + (sum_k D[k]) x,
+ * sh = (s - mu) / sqrt(var + eps) (mu, var: mean and biased variance over E), n = gamma sh + beta,
+ * y = SiLU(z) n.  Reverse: dz = dy n SiLU'(z); dn = dy SiLU(z); dgamma += dn sh; dbeta += dn;
+ * with gs = dn gamma, the normalisation's adjoint ds = (gs - mean(gs) - sh mean(gs sh)) / sqrt(var + eps);
+ * then ds feeds dys, dx (skip) and dD as without the norm.  tmp: 3 E doubles of scratch. */
+static void ln_token_grad(const float* x, const float* z, const float* dy, const double* ysr, const float* D,
+                          const gshape* g, const glnorm* ln, double* tmp, double* dysr, double* dx, double* dz,
+                          gparams* gp)
+{
+    const int E = g->E;
+    double *s = tmp, *sh = tmp + E, *gs = tmp + 2 * E;
+    double mu = 0.0;
+    for (int e = 0; e < E; ++e) {
+        double Dsum = 0.0;
+        for (int k = 0; k < g->nd; ++k) Dsum += (double)D[(size_t)k * E + e];
+        s[e] = ysr[e] + Dsum * (double)x[e];
+        mu += s[e];
+    }
+    mu /= (double)E;
+    double var = 0.0;
+    for (int e = 0; e < E; ++e) var += (s[e] - mu) * (s[e] - mu);
+    var /= (double)E;
+    const double inv = 1.0 / sqrt(var + ln->eps);
+    double mean_gs = 0.0, mean_gs_sh = 0.0;
+    for (int e = 0; e < E; ++e) {
+        sh[e] = (s[e] - mu) * inv;
+        const double zz = (double)z[e], sg = sigmoid(zz);
+        const double n = (double)ln->gamma[e] * sh[e] + (double)ln->beta[e];
+        const double dn = (double)dy[e] * zz * sg;
+        dz[e] = (double)dy[e] * n * sg * (1.0 + zz * (1.0 - sg));
+        gp->dln_gamma[e] += dn * sh[e];
+        gp->dln_beta[e] += dn;
+        gs[e] = dn * (double)ln->gamma[e];
+        mean_gs += gs[e];
+        mean_gs_sh += gs[e] * sh[e];
+    }
+    mean_gs /= (double)E;
+    mean_gs_sh /= (double)E;
+    for (int e = 0; e < E; ++e) {
+        double Dsum = 0.0;
+        for (int k = 0; k < g->nd; ++k) Dsum += (double)D[(size_t)k * E + e];
+        const double ds = (gs[e] - mean_gs - sh[e] * mean_gs_sh) * inv;
+        dysr[e] += ds;
+        dx[e] = ds * Dsum;
+        for (int k = 0; k < g->nd; ++k) gp->dD[(size_t)k * E + e] += ds * (double)x[e];
+    }
+}
 
 /* Step 1 of the reverse pass, one token: y = SiLU(z) s with s = ys_row + (sum_k D[k]) x.
  * dz = dy s SiLU'(z), SiLU'(z) = sig(z) (1 + z (1 - sig(z))); ds = dy SiLU(z);
  * ds feeds dys (the repeat's adjoint sums over the repeated tokens), dx (skip) and dD. */
 static void gate_token_grad(const float* x, const float* z, const float* dy, const double* ysr, const float* D,
-                            const gshape* g, double* dysr, double* dx, double* dz, double* dD)
+                            const gshape* g, const glnorm* ln, double* tmp, double* dysr, double* dx, double* dz,
+                            gparams* gp)
 {
+    double* dD = gp->dD;
+    if (ln->gamma) {
+        ln_token_grad(x, z, dy, ysr, D, g, ln, tmp, dysr, dx, dz, gp);
+        return;
+    }
     for (int e = 0; e < g->E; ++e) {
         double Dsum = 0.0;
         for (int k = 0; k < g->nd; ++k) Dsum += (double)D[(size_t)k * g->E + e];
@@ -164,7 +224,7 @@ static void proj_grad(const double* xbar, const double* u, const double* ddelta,
 /* One image.  x, z, dy, dx, dz point at the image; keep (masked) at its K ids. */
 static int backward_one(const float* x, const float* z, const float* dy, const float* A_log, const float* D,
                         const float* W_x, const float* W_dt, const float* b_dt, const int32_t* keep,
-                        const gshape* g, double* dx, double* dz, gparams* gp)
+                        const gshape* g, const glnorm* ln, double* dx, double* dz, gparams* gp)
 {
     const int T = g->T, E = g->E, J = g->J, nd = g->nd, K = g->K;
     const size_t tok = keep ? (size_t)K : (size_t)g->h * g->w;
@@ -176,7 +236,7 @@ static int backward_one(const float* x, const float* z, const float* dy, const f
     double* ddelta = (double*)calloc((size_t)nd * T * E, sizeof(double));
     double* du = (double*)calloc((size_t)nd * T * J, sizeof(double));
     double* dxbar = (double*)calloc((size_t)T * E, sizeof(double));
-    double* hist = (double*)calloc((size_t)T, sizeof(double));
+    double* hist = (double*)calloc((size_t)(T > 3 * E ? T : 3 * E), sizeof(double));
     int32_t* row_of = (int32_t*)calloc((size_t)(K > 0 ? K : 1), sizeof(int32_t));
     int32_t* row_off = (int32_t*)calloc((size_t)T + 1, sizeof(int32_t));
     int32_t* row_tok = (int32_t*)calloc((size_t)(K > 0 ? K : 1), sizeof(int32_t));
@@ -207,8 +267,8 @@ static int backward_one(const float* x, const float* z, const float* dy, const f
             const int i = (int)(m / (size_t)g->w), j = (int)(m % (size_t)g->w);
             t = g->pool_axis == FVO_POOL_W ? i : j;
         }
-        gate_token_grad(x + m * E, z + m * E, dy + m * E, ys + (size_t)t * E, D, g, dys + (size_t)t * E,
-                        dx + m * E, dz + m * E, gp->dD);
+        gate_token_grad(x + m * E, z + m * E, dy + m * E, ys + (size_t)t * E, D, g, ln, hist, dys + (size_t)t * E,
+                        dx + m * E, dz + m * E, gp);
     }
     /* 2: scans; 3, 4: projections */
     scan_grad(xbar, delta, u, dys, A_log, g, ddelta, du, dxbar, gp, hist);
@@ -235,13 +295,18 @@ done:
 int fvo_backward(const float* x, const float* z, const float* A_log, const float* D, const float* W_x,
                  const float* W_dt, const float* b_dt, const int32_t* keep_idx, int B, int h, int w, int E,
                  int N, int R, int K, int pool_axis, unsigned dir_flags, double pool_scale, int zoh_exact,
-                 const float* dy, int nthreads, double* dx, double* dz, double* dA_log, double* dD,
-                 double* dW_x, double* dW_dt, double* db_dt)
+                 const float* ln_gamma, const float* ln_beta, double ln_eps, const float* dy, int nthreads,
+                 double* dx, double* dz, double* dA_log, double* dD, double* dW_x, double* dW_dt, double* db_dt,
+                 double* dln_gamma, double* dln_beta)
 {
     const int nd = g_popcount2(dir_flags);
     if (B < 0 || h <= 0 || w <= 0 || E <= 0 || N <= 0 || R <= 0 || nd < 1 || (dir_flags & ~3u) != 0 ||
         (pool_axis != FVO_POOL_W && pool_axis != FVO_POOL_H) || (keep_idx && (K < 0 || K > h * w)))
         return FVO_BAD_SHAPE;
+    if ((ln_gamma == NULL) != (ln_beta == NULL) || (ln_gamma && (!(ln_eps >= 0.0) || !dln_gamma || !dln_beta)))
+        return FVO_BAD_SHAPE;
+    glnorm ln;
+    ln.gamma = ln_gamma; ln.beta = ln_beta; ln.eps = ln_eps;
     gshape g;
     g.h = h; g.w = w; g.E = E; g.N = N; g.R = R; g.K = keep_idx ? K : 0;
     g.T = pool_axis == FVO_POOL_W ? h : w;
@@ -255,6 +320,11 @@ int fvo_backward(const float* x, const float* z, const float* A_log, const float
     memset(dW_x, 0, nWx * sizeof(double));
     memset(dW_dt, 0, nWdt * sizeof(double));
     memset(db_dt, 0, nDv * sizeof(double));
+    const size_t nL = ln_gamma ? (size_t)E : 0;
+    if (nL) {
+        memset(dln_gamma, 0, nL * sizeof(double));
+        memset(dln_beta, 0, nL * sizeof(double));
+    }
     const size_t tok = keep_idx ? (size_t)K : (size_t)h * w;
     int status = FVO_OK;
     if (nthreads < 1) nthreads = 1;
@@ -263,13 +333,14 @@ int fvo_backward(const float* x, const float* z, const float* A_log, const float
 #endif
     for (int b = 0; b < B; ++b) {
         gparams gp;
-        double* buf = (double*)calloc(nA + 2 * nDv + nWx + nWdt, sizeof(double));
+        double* buf = (double*)calloc(nA + 2 * nDv + nWx + nWdt + 2 * nL, sizeof(double));
         int st = FVO_NO_MEMORY;
         if (buf) {
             gp.dA_log = buf; gp.dD = buf + nA; gp.db_dt = gp.dD + nDv; gp.dW_x = gp.db_dt + nDv;
             gp.dW_dt = gp.dW_x + nWx;
+            gp.dln_gamma = gp.dW_dt + nWdt; gp.dln_beta = gp.dln_gamma + nL;
             st = backward_one(x + (size_t)b * tok * E, z + (size_t)b * tok * E, dy + (size_t)b * tok * E, A_log, D,
-                              W_x, W_dt, b_dt, keep_idx ? keep_idx + (size_t)b * K : NULL, &g,
+                              W_x, W_dt, b_dt, keep_idx ? keep_idx + (size_t)b * K : NULL, &g, &ln,
                               dx + (size_t)b * tok * E, dz + (size_t)b * tok * E, &gp);
         }
 #ifdef _OPENMP
@@ -281,6 +352,7 @@ int fvo_backward(const float* x, const float* z, const float* A_log, const float
                 for (size_t i = 0; i < nDv; ++i) { dD[i] += gp.dD[i]; db_dt[i] += gp.db_dt[i]; }
                 for (size_t i = 0; i < nWx; ++i) dW_x[i] += gp.dW_x[i];
                 for (size_t i = 0; i < nWdt; ++i) dW_dt[i] += gp.dW_dt[i];
+                for (size_t i = 0; i < nL; ++i) { dln_gamma[i] += gp.dln_gamma[i]; dln_beta[i] += gp.dln_beta[i]; }
             }
             if (st != FVO_OK && (status == FVO_OK || status == FVO_BAD_INDEX)) status = st;
         }

@@ -19,7 +19,12 @@ ORACLE_DIR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file
 
 MUTATIONS = {
     "SiLU derivative taken as the sigmoid": ("s * sg * (1.0 + zz * (1.0 - sg))", "s * sg"),
-    "skip gradient from one direction": ("dx[e] = ds * Dsum;", "dx[e] = ds * (double)D[e];"),
+    "skip gradient from one direction": ("        dysr[e] += ds;\n        dx[e] = ds * Dsum;\n        for (int k = 0; k < g->nd; ++k) dD[",
+                                         "        dysr[e] += ds;\n        dx[e] = ds * (double)D[e];\n        for (int k = 0; k < g->nd; ++k) dD["),
+    "LayerNorm adjoint without the mean term": ("(gs[e] - mean_gs - sh[e] * mean_gs_sh) * inv", "(gs[e] - sh[e] * mean_gs_sh) * inv"),
+    "LayerNorm adjoint without the projection term": ("(gs[e] - mean_gs - sh[e] * mean_gs_sh) * inv", "(gs[e] - mean_gs) * inv"),
+    "LayerNorm dgamma without the normalised value": ("gp->dln_gamma[e] += dn * sh[e];", "gp->dln_gamma[e] += dn;"),
+    "LayerNorm dz from the pre-norm value": ("dz[e] = (double)dy[e] * n * sg", "dz[e] = (double)dy[e] * s[e] * sg"),
     "adjoint decays with the current step": ("lam = Cn * dyt + Abar_next * lam;", "lam = Cn * dyt + Abar * lam;"),
     "dC from the previous state": ("+= dyt * hist[t];", "+= dyt * hprev;"),
     "Abar term of dDelta dropped": ("double d_dt = lam * hprev * Abar * A;", "double d_dt = 0.0;"),

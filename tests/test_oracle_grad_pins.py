@@ -39,18 +39,24 @@ def _case(rng, masked, B=2, h=3, w=4, E=4, N=3, R=2, K=7, nd=2):
     return x, z, dy, P, kw
 
 
-def _fd_check(oracle_mod, rng, x, z, dy, P, kw, pool_axis, dir_flags, zoh, scale, per_array=6):
+def _fd_check(oracle_mod, rng, x, z, dy, P, kw, pool_axis, dir_flags, zoh, scale, per_array=6, ln=None):
+    """ln: None, or (gamma, beta, eps) for the post-SSM LayerNorm (then its gradients are checked too)."""
+    lnkw = {} if ln is None else {"ln_gamma": ln[0], "ln_beta": ln[1], "ln_eps": ln[2]}
     g = oracle_mod.backward(x, z, P["A_log"], P["D"], P["W_x"], P["W_dt"], P["b_dt"], dy, pool_axis, dir_flags,
-                            pool_scale=scale, zoh_exact=zoh, **kw)
+                            pool_scale=scale, zoh_exact=zoh, **kw, **lnkw)
     dy64 = dy.astype(np.float64)
 
     def loss(**over):
-        a = {"x": x, "z": z, **P, **over}
+        a = {"x": x, "z": z, **P, **lnkw, **over}
+        extra = {} if ln is None else {"ln_gamma": a["ln_gamma"], "ln_beta": a["ln_beta"], "ln_eps": a["ln_eps"]}
         y = oracle_mod.forward(a["x"], a["z"], a["A_log"], a["D"], a["W_x"], a["W_dt"], a["b_dt"], pool_axis,
-                               dir_flags, pool_scale=scale, zoh_exact=zoh, **kw)
+                               dir_flags, pool_scale=scale, zoh_exact=zoh, **kw, **extra)
         return float(np.sum(dy64 * y))
 
-    for name, arr in [("x", x), ("z", z)] + [(k, P[k]) for k in PARAMS]:
+    arrays = [("x", x), ("z", z)] + [(k, P[k]) for k in PARAMS]
+    if ln is not None:
+        arrays += [("ln_gamma", ln[0]), ("ln_beta", ln[1])]
+    for name, arr in arrays:
         grad = g["d" + name]
         assert grad.shape == arr.shape
         scale_ref = np.abs(grad).max()
@@ -84,6 +90,20 @@ def test_masked_gradient_equals_finite_differences(pool_axis, zoh, oracle_mod=No
     rng = np.random.default_rng(200 + pool_axis + 2 * zoh)
     x, z, dy, P, kw = _case(rng, True)
     _fd_check(oracle_mod, rng, x, z, dy, P, kw, pool_axis, 3, zoh, 1.0)
+
+
+@pytest.mark.parametrize("masked", [False, True])
+@pytest.mark.parametrize("pool_axis", [0, 1])
+def test_layernorm_gradient_equals_finite_differences(masked, pool_axis, oracle_mod=None):
+    """With the post-SSM LayerNorm: every gradient, dgamma and dbeta included (E = 6 channels, so
+    the normalisation's mean and projection terms are far from negligible)."""
+    import oracle
+    oracle_mod = oracle_mod or oracle
+    rng = np.random.default_rng(600 + 2 * masked + pool_axis)
+    x, z, dy, P, kw = _case(rng, masked, E=6)
+    gamma = rng.uniform(0.5, 1.5, 6).astype(np.float32)
+    beta = rng.uniform(-0.5, 0.5, 6).astype(np.float32)
+    _fd_check(oracle_mod, rng, x, z, dy, P, kw, pool_axis, 3, False, 1.0, ln=(gamma, beta, 1e-5))
 
 
 def test_longer_sequence_gradient_equals_finite_differences(oracle_mod=None):
