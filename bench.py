@@ -67,7 +67,7 @@ def kernel_work(name: str, cfg, pool_axis: int):
     if name == "proj_gemm_kernel":
         return "fma", 2 * cfg.B * T * cfg.E * cfg.nd * (cfg.R + 2 * cfg.N)
     # the gradient's kernels
-    if name in ("bwd_gate_dense_kernel", "bwd_gate_masked_kernel"):
+    if name in ("bwd_gate_dense_kernel", "bwd_gate_masked_kernel", "bwd_ln_gate_kernel"):
         return "hbm", 5 * row * tok                   # read x, z, dy; write dz and dx
     if name == "bwd_pool_dense_kernel":
         return "hbm", 2 * row * tok                   # dx read and written back (+ the pooled share)
@@ -561,14 +561,17 @@ def run_grad(a, cfg, pool_axis):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     t = workload.layer_tensors(cfg, dev)
+    if a.ln:
+        t.update(workload.ln_tensors(cfg, dev))
     dy = workload.upstream_grad(cfg, dev)
     keep = t.get("keep_idx")
-    shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, cfg.dir_flags, keep, cfg.h, cfg.w, path=a.path)
+    shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, cfg.dir_flags, keep, cfg.h, cfg.w, path=a.path,
+                            ln=a.ln)
     y = torch.empty_like(t["x"])
     fws = ssm.alloc_workspace(shape, dev)
-    bws = torch.empty(ssm.backward_workspace_size(shape), dtype=torch.uint8, device=dev)
+    bws = torch.empty(max(ssm.backward_workspace_size(shape), 256), dtype=torch.uint8, device=dev)
     grads = {"dx": torch.empty_like(t["x"]), "dz": torch.empty_like(t["z"])}
-    for n in ("A_log", "D", "W_x", "W_dt", "b_dt"):
+    for n in ("A_log", "D", "W_x", "W_dt", "b_dt") + (("ln_gamma", "ln_beta") if a.ln else ()):
         grads["d" + n] = torch.empty_like(t[n])
     stream = torch.cuda.current_stream(dev)
     fwd = ssm.BoundForward(shape, t, y, fws, stream)
@@ -642,7 +645,8 @@ def run_grad(a, cfg, pool_axis):
     # the gradient's own HBM floor: read x, z, dy, write dx, dz (5 rows per token)
     bwd_ms = sum(statistics.mean(per_kernel[n]) for n in dict.fromkeys(bwd.names))
     line = {
-        "metric": "SSM-layer training step (forward + gradient) grid tokens/s at " + cfg.name + " (fp32)",
+        "metric": "SSM-layer training step (forward + gradient) grid tokens/s at " + cfg.name +
+                  (" with the post-SSM LayerNorm" if a.ln else "") + " (fp32)",
         "value": tokens * a.steps / (ms / 1e3), "unit": UNIT, "n_gpus": 1, "steps": a.steps, "warmup": a.warmup,
         "ms_per_step": ms / a.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic (seeded N(0,1) x, z, dy; Mamba-style parameter init)",
@@ -657,19 +661,24 @@ def run_grad(a, cfg, pool_axis):
         "e2e": None,
     }
     if not a.no_cpu_baseline:
+        import numpy as np
+
         import oracle
         from pooled_selective_scan_b200 import inputs
         cores = host_cores()
         which = list(range(min(cfg.B, max(1, cores), 16)))
         d = inputs.layer_inputs(cfg, which=which)
         shp = inputs.token_shape(cfg)
-        dyh = __import__("numpy").stack([inputs.image_dy(cfg.seed, b, shp) for b in which])
+        dyh = np.stack([inputs.image_dy(cfg.seed, b, shp) for b in which])
         oracle.build()
+        lnkw = {}
+        if a.ln:
+            lnkw = dict(ln_gamma=np.ones(cfg.E, np.float32), ln_beta=np.zeros(cfg.E, np.float32), ln_eps=1e-5)
         t0 = time.perf_counter()
         oracle.forward(d["x"], d["z"], d["A_log"], d["D"], d["W_x"], d["W_dt"], d["b_dt"], pool_axis, cfg.dir_flags,
-                       keep_idx=d.get("keep_idx"), h=cfg.h, w=cfg.w, nthreads=len(which))
+                       keep_idx=d.get("keep_idx"), h=cfg.h, w=cfg.w, nthreads=len(which), **lnkw)
         oracle.backward(d["x"], d["z"], d["A_log"], d["D"], d["W_x"], d["W_dt"], d["b_dt"], dyh, pool_axis,
-                        cfg.dir_flags, keep_idx=d.get("keep_idx"), h=cfg.h, w=cfg.w, nthreads=len(which))
+                        cfg.dir_flags, keep_idx=d.get("keep_idx"), h=cfg.h, w=cfg.w, nthreads=len(which), **lnkw)
         el = time.perf_counter() - t0
         tok = len(which) * (cfg.K if cfg.masked else cfg.h * cfg.w)
         line["cpu_baseline"] = {"value": tok / el, "unit": UNIT, "cores": len(which), "kind": "oracle",

@@ -249,9 +249,9 @@ FV_API fv_status fastvim_get_device_status(const void* ws, void* stream);
  * the pages give no backward rule, so this is the exact derivative of the layer above, by the
  * chain rule in reverse step order: for an upstream gradient dy = dL/dy of a scalar loss L it
  * returns dx = dL/dx, dz = dL/dz and the parameter gradients summed over the batch.  Dense and
- * masked layers, both pool axes, one or two directions, pool_scale and FV_FLAG_ZOH_EXACT; not
- * the post-SSM LayerNorm (FV_FLAG_LAYERNORM gives FV_ERR_UNSUPPORTED).  Masked tokens whose id
- * the forward rejected (FV_ERR_INDEX) get dx = dz = 0. */
+ * masked layers, both pool axes, one or two directions, pool_scale, FV_FLAG_ZOH_EXACT and the
+ * post-SSM LayerNorm (FV_FLAG_LAYERNORM: also dln_gamma, dln_beta).  Masked tokens whose id the
+ * forward rejected (FV_ERR_INDEX) get dx = dz = 0. */
 typedef struct {
     const float* dy;  /* dL/dy, the shape of y (dense [B][h][w][E] | masked [B][K][E])         */
     float* dx;        /* dL/dx, the shape of x (written)                                      */
@@ -261,6 +261,8 @@ typedef struct {
     float* dW_x;      /* [nd][R+2N][E]   } them first.  The sums run in fp32 with atomic       */
     float* dW_dt;     /* [nd][E][R]      } additions, so their last bits may differ between    */
     float* db_dt;     /* [nd][E]         } runs.                                               */
+    float* dln_gamma; /* [E] with FV_FLAG_LAYERNORM (written, like the above), else NULL          */
+    float* dln_beta;  /* [E] with FV_FLAG_LAYERNORM, else NULL                                    */
 } fv_ssm_grads;
 
 /* Byte offsets of the gradient's intermediates inside its workspace. */
@@ -290,8 +292,9 @@ FV_API const char* fastvim_ssm_backward_launch_name(const fv_ssm_args* args, int
  *   aligned, no initial contents; fwd_ws and ws must not overlap.
  * grads: device arrays, 16-byte aligned; dx and dz must not overlap each other, x, z or dy.
  * Errors: as fastvim_ssm_forward for args; FV_ERR_NULL for a missing grads array (dy, dx, dz may
- * be NULL when B == 0); FV_ERR_ALIGN, FV_ERR_ALIAS as above; FV_ERR_WORKSPACE for a missing,
- * short or misaligned fwd_ws or ws; FV_ERR_UNSUPPORTED with FV_FLAG_LAYERNORM. */
+ * be NULL when B == 0; dln_gamma, dln_beta are required with FV_FLAG_LAYERNORM); FV_ERR_SHAPE
+ * for dln_gamma or dln_beta without the flag; FV_ERR_ALIGN, FV_ERR_ALIAS as above;
+ * FV_ERR_WORKSPACE for a missing, short or misaligned fwd_ws or ws. */
 FV_API fv_status fastvim_ssm_backward(const fv_ssm_args* args, const fv_ssm_grads* grads, const void* fwd_ws,
                                       size_t fwd_ws_bytes, void* ws, size_t ws_bytes, void* stream);
 

@@ -85,7 +85,8 @@ class FvWsLayout(ctypes.Structure):
 
 
 class FvSsmGrads(ctypes.Structure):
-    _fields_ = [(name, ctypes.c_void_p) for name in ("dy", "dx", "dz", "dA_log", "dD", "dW_x", "dW_dt", "db_dt")]
+    _fields_ = [(name, ctypes.c_void_p) for name in ("dy", "dx", "dz", "dA_log", "dD", "dW_x", "dW_dt", "db_dt",
+                                                     "dln_gamma", "dln_beta")]
 
 
 class FvBwdWsLayout(ctypes.Structure):

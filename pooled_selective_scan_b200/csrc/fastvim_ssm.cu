@@ -940,13 +940,15 @@ BwdLayout plan_bwd(const fv::Shape& sh) {
     return L;
 }
 
-// Launch order of a gradient call: gate, scans (with dt_proj), dW_x, dxbar, pooling.
+// Launch order of a gradient call: gate (through the LayerNorm with FV_FLAG_LAYERNORM), scans (with
+// dt_proj), dW_x, dxbar, pooling.
 const char* bwd_launch_name_of(const fv::Shape& sh, int i) {
     static const char* dense[] = {"bwd_gate_dense_kernel", "bwd_scan_kernel", "bwd_gemm_kernel:W_x",
                                   "bwd_gemm_kernel:xbar", "bwd_pool_dense_kernel"};
     static const char* masked[] = {"bwd_gate_masked_kernel", "bwd_scan_kernel", "bwd_gemm_kernel:W_x",
                                    "bwd_gemm_kernel:xbar", "bwd_pool_masked_kernel"};
     if (sh.B == 0 || i < 0 || i >= 5) return "";
+    if (i == 0 && sh.ln) return "bwd_ln_gate_kernel";
     return sh.K > 0 ? masked[i] : dense[i];
 }
 int bwd_launch_count_of(const fv::Shape& sh) { return sh.B == 0 ? 0 : 5; }
@@ -960,7 +962,9 @@ fv_status check_grads(const fv_ssm_args* a, const fv::Shape& sh, const fv_ssm_gr
     if (!g) return FV_ERR_NULL;
     if (!g->dA_log || !g->dD || !g->dW_x || !g->dW_dt || !g->db_dt) return FV_ERR_NULL;
     if (sh.B > 0 && (!g->dy || !g->dx || !g->dz)) return FV_ERR_NULL;
-    const void* ps[] = {g->dy, g->dx, g->dz, g->dA_log, g->dD, g->dW_x, g->dW_dt, g->db_dt};
+    if (sh.ln && (!g->dln_gamma || !g->dln_beta)) return FV_ERR_NULL;
+    if (!sh.ln && (g->dln_gamma || g->dln_beta)) return FV_ERR_SHAPE;  // LayerNorm gradients need the flag
+    const void* ps[] = {g->dy, g->dx, g->dz, g->dA_log, g->dD, g->dW_x, g->dW_dt, g->db_dt, g->dln_gamma, g->dln_beta};
     for (const void* p : ps)
         if (p && !aligned16(p)) return FV_ERR_ALIGN;
     if (sh.B > 0) {
@@ -1024,7 +1028,6 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
     if (!ac.y && g) ac.y = g->dx;
     const fv_ssm_args* a = &ac;
     if ((s = check_pointers(a, sh)) != FV_OK) return s;
-    if (sh.ln) return FV_ERR_UNSUPPORTED;
     if ((s = check_grads(a, sh, g)) != FV_OK) return s;
     fv_ws_layout FL;
     plan_layout(sh, &FL);
@@ -1045,7 +1048,9 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
         (e = cudaMemsetAsync(g->dD, 0, nE * sizeof(float), st)) != cudaSuccess ||
         (e = cudaMemsetAsync(g->dW_x, 0, nWx * sizeof(float), st)) != cudaSuccess ||
         (e = cudaMemsetAsync(g->dW_dt, 0, nWdt * sizeof(float), st)) != cudaSuccess ||
-        (e = cudaMemsetAsync(g->db_dt, 0, nE * sizeof(float), st)) != cudaSuccess) {
+        (e = cudaMemsetAsync(g->db_dt, 0, nE * sizeof(float), st)) != cudaSuccess ||
+        (sh.ln && (e = cudaMemsetAsync(g->dln_gamma, 0, (size_t)sh.E * sizeof(float), st)) != cudaSuccess) ||
+        (sh.ln && (e = cudaMemsetAsync(g->dln_beta, 0, (size_t)sh.E * sizeof(float), st)) != cudaSuccess)) {
         note_cuda(e, "gradient reset");
         return FV_ERR_CUDA;
     }
@@ -1071,13 +1076,43 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
 
     // 1. gate, skip and repeat
     // the gate kernels are persistent over pooled rows: one wave of resident blocks
-    auto resident = [&](auto kern, int threads) {
+    auto resident = [&](auto kern, int threads, size_t smem = 0) {
         int per_sm = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0) != cudaSuccess || per_sm < 1)
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess || per_sm < 1)
             per_sm = 1;
         return std::min(M, per_sm * sms);
     };
-    if (sh.K == 0) {
+    if (sh.ln) {
+        const int warps = fv::bwd_ln_warps(sh.SL);
+        const size_t smem = fv::bwd_ln_smem_bytes(sh.SL, warps);
+        const int32_t* row_off = sh.K > 0 ? (const int32_t*)(fw + FL.row_off) : nullptr;
+        const int32_t* row_tok = sh.K > 0 ? (const int32_t*)(fw + FL.row_tok) : nullptr;
+        FV_MARK_CALL(marks, st, ([&]() -> fv_status {
+            if (sh.K > 0) {
+                if ((e = ensure_smem(fv::bwd_ln_gate_kernel<true>, smem)) != cudaSuccess) {
+                    note_cuda(e, "LayerNorm gradient smem attribute");
+                    return FV_ERR_CUDA;
+                }
+                const int grid = resident(fv::bwd_ln_gate_kernel<true>, 32 * warps, smem);
+                fv::bwd_ln_gate_kernel<true><<<grid, 32 * warps, smem, st>>>(sh, a->x, a->z, g->dy, ys, a->D,
+                                                                             a->ln_gamma, a->ln_beta, row_off, row_tok,
+                                                                             g->dx, g->dz, dys, g->dD, g->dln_gamma,
+                                                                             g->dln_beta);
+            } else {
+                if ((e = ensure_smem(fv::bwd_ln_gate_kernel<false>, smem)) != cudaSuccess) {
+                    note_cuda(e, "LayerNorm gradient smem attribute");
+                    return FV_ERR_CUDA;
+                }
+                const int grid = resident(fv::bwd_ln_gate_kernel<false>, 32 * warps, smem);
+                fv::bwd_ln_gate_kernel<false><<<grid, 32 * warps, smem, st>>>(sh, a->x, a->z, g->dy, ys, a->D,
+                                                                              a->ln_gamma, a->ln_beta, row_off,
+                                                                              row_tok, g->dx, g->dz, dys, g->dD,
+                                                                              g->dln_gamma, g->dln_beta);
+            }
+            FV_LAUNCH_CHECK("bwd_ln_gate_kernel");
+            return FV_OK;
+        })());
+    } else if (sh.K == 0) {
         const int threads = fv::bwd_groups(sh.SL) * fv::bwd_slot_width(sh.SL);
         const bool u4 = bwd_gate_unroll() == 4;
         const int grid = u4 ? resident(fv::bwd_gate_dense_kernel<4>, threads) : resident(fv::bwd_gate_dense_kernel<2>, threads);
@@ -1179,13 +1214,13 @@ fv_status fastvim_ssm_backward_workspace_layout(const fv_ssm_args* args, fv_bwd_
 
 int fastvim_ssm_backward_launch_count(const fv_ssm_args* args) {
     fv::Shape sh;
-    if (make_shape(args, &sh) != FV_OK || sh.ln) return 0;
+    if (make_shape(args, &sh) != FV_OK) return 0;
     return bwd_launch_count_of(sh);
 }
 
 const char* fastvim_ssm_backward_launch_name(const fv_ssm_args* args, int i) {
     fv::Shape sh;
-    if (make_shape(args, &sh) != FV_OK || sh.ln) return "";
+    if (make_shape(args, &sh) != FV_OK) return "";
     return bwd_launch_name_of(sh, i);
 }
 

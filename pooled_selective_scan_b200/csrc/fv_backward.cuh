@@ -7,6 +7,8 @@
 //   bwd_gate_dense_kernel / bwd_gate_masked_kernel   gate, skip and repeat: dz, the skip part of
 //                                                    dx, dD, and dys = the sum of ds over the
 //                                                    tokens of each pooled row
+//   bwd_ln_gate_kernel                               the same through the post-SSM LayerNorm,
+//                                                    plus dln_gamma, dln_beta
 //   bwd_scan_kernel                                  adjoint of both scans: dDelta, and through
 //                                                    dt_proj + softplus d dt_low, dW_dt, db_dt; dB,
 //                                                    dC, dA_log and the scans' share of dxbar
@@ -226,6 +228,173 @@ bwd_gate_masked_kernel(Shape sh, const float* __restrict__ x, const float* __res
                 float* d = dD + (size_t)k * sh.E + 4 * slot;
                 atomicAdd(d + 0, dDa.x); atomicAdd(d + 1, dDa.y); atomicAdd(d + 2, dDa.z); atomicAdd(d + 3, dDa.w);
             }
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// Gate, skip and repeat through the post-SSM LayerNorm
+// ------------------------------------------------------------------------------------------
+
+// Warps per block of the LayerNorm gate gradient: as many (up to 4) as keep its shared memory
+// ((3 + 4 W) E floats) within about 100 KB.
+__host__ __forceinline__ int bwd_ln_warps(int SL) {
+    for (int w = 4; w > 1; w >>= 1)
+        if ((size_t)(3 + 4 * w) * SL * sizeof(float4) <= (size_t)100 * 1024) return w;
+    return 1;
+}
+__host__ __forceinline__ size_t bwd_ln_smem_bytes(int SL, int warps) {
+    return (size_t)(3 + 4 * warps) * SL * sizeof(float4);
+}
+
+// Persistent over pooled rows (b, t) (grid-stride); the block's warps take the row's tokens in
+// turn, one token per warp at a time.  Per token, with s = ys[t] + (sum_k D[k]) x over its E
+// channels, sh = (s - mean) rstd, n = gamma sh + beta, y = SiLU(z) n:
+//   dz = dy n SiLU'(z);  dn = dy SiLU(z);  gs = dn gamma;
+//   ds = rstd (gs - mean(gs) - sh mean(gs sh));  dx (skip part) = ds sum_k D[k];
+//   dys[t] += ds;  dgamma += dn sh;  dbeta += dn;  dD += ds x.
+// Three passes over the token's channels: the statistics of s, the two means of gs, the outputs;
+// the first pass reads x and the second z and dy from HBM, the repeats hit L1.  Every lane owns
+// the same float4 slots in every pass, so each warp sums dys, dgamma, dbeta and dD into private
+// shared-memory rows with no atomics; the rows meet at the end of each pooled row (dys) and of
+// the kernel (one global atomic per channel per block for the batch sums).  Masked layers take a
+// row's kept tokens from the forward's row lists; a rejected id is in no row (dx, dz zeroed by
+// bwd_pool_masked_kernel).
+template <bool MASKED>
+__global__ void __launch_bounds__(128)
+bwd_ln_gate_kernel(Shape sh, const float* __restrict__ x, const float* __restrict__ z, const float* __restrict__ dy,
+                   const float* __restrict__ ys, const float* __restrict__ D, const float* __restrict__ gamma,
+                   const float* __restrict__ beta, const int32_t* __restrict__ row_off,
+                   const int32_t* __restrict__ row_tok, float* __restrict__ dx, float* __restrict__ dz,
+                   float* __restrict__ dys, float* __restrict__ dD, float* __restrict__ dgamma,
+                   float* __restrict__ dbeta) {
+    extern __shared__ float4 lgs[];
+    const int SL = sh.SL, W = blockDim.x >> 5;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float4* dsum = lgs;
+    float4* g4 = dsum + SL;
+    float4* be4 = g4 + SL;
+    float4* prow = be4 + SL;  // [W][4][SL]: dys, dgamma, dbeta, dD of each warp
+    float4* pdys = prow + (size_t)warp * 4 * SL;
+    float4* pdg = pdys + SL;
+    float4* pdb = pdg + SL;
+    float4* pdD = pdb + SL;
+    for (int slot = threadIdx.x; slot < SL; slot += blockDim.x) {
+        dsum[slot] = bwd_dsum4(D, sh.nd, SL, slot);
+        g4[slot] = __ldg(reinterpret_cast<const float4*>(gamma) + slot);
+        be4[slot] = __ldg(reinterpret_cast<const float4*>(beta) + slot);
+    }
+    for (int i = threadIdx.x; i < 4 * W * SL; i += blockDim.x) prow[i] = f4_zero();
+    __syncthreads();
+    const int T = sh.T, K = sh.K;
+    const int rows = sh.B * T;
+    const size_t st4 = dense_stride(sh) >> 2;
+    const float invE = 1.f / (float)sh.E, eps = sh.ln_eps;
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    const float4* z4 = reinterpret_cast<const float4*>(z);
+    const float4* gy4 = reinterpret_cast<const float4*>(dy);
+    float4* dx4 = reinterpret_cast<float4*>(dx);
+    float4* dz4 = reinterpret_cast<float4*>(dz);
+    for (int bt = blockIdx.x; bt < rows; bt += gridDim.x) {
+        const int b = bt / T, t = bt - b * T;
+        int p0 = 0, ntok = sh.S;
+        if (MASKED) {
+            p0 = row_off[(size_t)b * (T + 1) + t];
+            ntok = row_off[(size_t)b * (T + 1) + t + 1] - p0;
+        }
+        const float4* ys4 = reinterpret_cast<const float4*>(ys + (size_t)bt * sh.E);
+        for (int i = warp; i < ntok; i += W) {
+            const size_t o = MASKED ? ((size_t)b * K + row_tok[(size_t)b * K + p0 + i]) * SL
+                                    : (dense_base(sh, b, t) >> 2) + (size_t)i * st4;
+            // statistics of s (moments shifted by the token's first s value, the same in every lane)
+            const float Ks = fmaf(dsum[0].x, __ldg(x + o * 4), __ldg(ys + (size_t)bt * sh.E));
+            float m1 = 0.f, m2 = 0.f;
+#pragma unroll 4
+            for (int slot = lane; slot < SL; slot += 32)
+                ln_accum(f4_fma(dsum[slot], __ldg(x4 + o + slot), ys4[slot]), Ks, m1, m2);
+            float mean, rstd;
+            ln_stats(m1, m2, Ks, invE, eps, mean, rstd);
+            // the two means of gs = dy SiLU(z) gamma
+            float a1 = 0.f, a2 = 0.f;
+#pragma unroll 4
+            for (int slot = lane; slot < SL; slot += 32) {
+                const float4 sv = f4_fma(dsum[slot], __ldg(x4 + o + slot), ys4[slot]);
+                const float4 zv = __ldg(z4 + o + slot), gv = __ldg(gy4 + o + slot), gm = g4[slot];
+                const float sa[4] = {sv.x, sv.y, sv.z, sv.w}, za[4] = {zv.x, zv.y, zv.z, zv.w};
+                const float ga[4] = {gv.x, gv.y, gv.z, gv.w}, gma[4] = {gm.x, gm.y, gm.z, gm.w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float shv = (sa[c] - mean) * rstd;
+                    const float gs = ga[c] * za[c] * sigmoid_fast(za[c]) * gma[c];
+                    a1 += gs;
+                    a2 = fmaf(gs, shv, a2);
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                a1 += __shfl_xor_sync(0xffffffffu, a1, off);
+                a2 += __shfl_xor_sync(0xffffffffu, a2, off);
+            }
+            const float mgs = a1 * invE, mgss = a2 * invE;
+            // outputs
+#pragma unroll 2
+            for (int slot = lane; slot < SL; slot += 32) {
+                const float4 xv = __ldg(x4 + o + slot), zv = __ldg(z4 + o + slot), gv = __ldg(gy4 + o + slot);
+                const float4 ds4 = dsum[slot], gm = g4[slot], bm = be4[slot];
+                const float4 sv = f4_fma(ds4, xv, ys4[slot]);
+                const float sa[4] = {sv.x, sv.y, sv.z, sv.w}, za[4] = {zv.x, zv.y, zv.z, zv.w};
+                const float ga[4] = {gv.x, gv.y, gv.z, gv.w}, xa[4] = {xv.x, xv.y, xv.z, xv.w};
+                const float gma[4] = {gm.x, gm.y, gm.z, gm.w}, bma[4] = {bm.x, bm.y, bm.z, bm.w};
+                const float dsa[4] = {ds4.x, ds4.y, ds4.z, ds4.w};
+                float dzo[4], dxo[4], dso[4], dno[4], sho[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float shv = (sa[c] - mean) * rstd;
+                    const float sg = sigmoid_fast(za[c]);
+                    const float dn = ga[c] * za[c] * sg;
+                    const float n = fmaf(gma[c], shv, bma[c]);
+                    dzo[c] = ga[c] * n * sg * fmaf(za[c], 1.f - sg, 1.f);
+                    const float ds = (fmaf(dn, gma[c], -mgs) - shv * mgss) * rstd;
+                    dxo[c] = ds * dsa[c];
+                    dso[c] = ds;
+                    dno[c] = dn;
+                    sho[c] = shv;
+                }
+                st_stream(dz4 + o + slot, make_float4(dzo[0], dzo[1], dzo[2], dzo[3]));
+                st_stream(dx4 + o + slot, make_float4(dxo[0], dxo[1], dxo[2], dxo[3]));
+                f4_add(pdys[slot], make_float4(dso[0], dso[1], dso[2], dso[3]));
+                f4_add(pdg[slot], make_float4(dno[0] * sho[0], dno[1] * sho[1], dno[2] * sho[2], dno[3] * sho[3]));
+                f4_add(pdb[slot], make_float4(dno[0], dno[1], dno[2], dno[3]));
+                f4_add(pdD[slot], make_float4(dso[0] * xa[0], dso[1] * xa[1], dso[2] * xa[2], dso[3] * xa[3]));
+            }
+        }
+        __syncthreads();
+        for (int slot = threadIdx.x; slot < SL; slot += blockDim.x) {
+            float4 acc = f4_zero();
+            for (int w = 0; w < W; ++w) {
+                float4* r = prow + (size_t)w * 4 * SL + slot;
+                f4_add(acc, *r);
+                *r = f4_zero();
+            }
+            reinterpret_cast<float4*>(dys)[(size_t)bt * SL + slot] = acc;
+        }
+        __syncthreads();
+    }
+    for (int slot = threadIdx.x; slot < SL; slot += blockDim.x) {
+        float4 sg = f4_zero(), sb = f4_zero(), sd = f4_zero();
+        for (int w = 0; w < W; ++w) {
+            const float4* r = prow + (size_t)w * 4 * SL;
+            f4_add(sg, r[SL + slot]);
+            f4_add(sb, r[2 * SL + slot]);
+            f4_add(sd, r[3 * SL + slot]);
+        }
+        float* pg = dgamma + 4 * slot;
+        float* pb = dbeta + 4 * slot;
+        atomicAdd(pg + 0, sg.x); atomicAdd(pg + 1, sg.y); atomicAdd(pg + 2, sg.z); atomicAdd(pg + 3, sg.w);
+        atomicAdd(pb + 0, sb.x); atomicAdd(pb + 1, sb.y); atomicAdd(pb + 2, sb.z); atomicAdd(pb + 3, sb.w);
+        for (int k = 0; k < sh.nd; ++k) {
+            float* d = dD + (size_t)k * sh.E + 4 * slot;
+            atomicAdd(d + 0, sd.x); atomicAdd(d + 1, sd.y); atomicAdd(d + 2, sd.z); atomicAdd(d + 3, sd.w);
         }
     }
 }

@@ -238,31 +238,42 @@ def _grads(dy, grads: dict) -> nat.FvSsmGrads:
     g.dy = _ptr(dy)
     for name in ("dx", "dz", "dA_log", "dD", "dW_x", "dW_dt", "db_dt"):
         setattr(g, name, _ptr(grads[name]))
+    g.dln_gamma, g.dln_beta = _ptr(grads.get("dln_gamma")), _ptr(grads.get("dln_beta"))
     return g
 
 
 def backward(x, z, A_log, D, W_x, W_dt, b_dt, dy, fwd_workspace, pool_axis=POOL_W, dir_flags=DIR_FWD | DIR_BWD,
              keep_idx=None, h=None, w=None, pool_scale=1.0, zoh_exact=False, path="auto", grads=None,
-             workspace=None, stream=None) -> dict:
+             workspace=None, stream=None, ln_gamma=None, ln_beta=None, ln_eps=1e-5) -> dict:
     """Queue the gradient of the layer for the upstream gradient dy on ``stream`` and return the
-    dict {dx, dz, dA_log, dD, dW_x, dW_dt, db_dt}.  fwd_workspace is the workspace of a forward
-    call with the same tensors and options, queued earlier on the same stream."""
+    dict {dx, dz, dA_log, dD, dW_x, dW_dt, db_dt} (+ dln_gamma, dln_beta with the post-SSM
+    LayerNorm).  fwd_workspace is the workspace of a forward call with the same tensors and
+    options, queued earlier on the same stream."""
     dev = x.device
     for name, t in (("x", x), ("z", z), ("A_log", A_log), ("D", D), ("W_x", W_x), ("W_dt", W_dt), ("b_dt", b_dt),
                     ("dy", dy)):
         _check_tensor(name, t, torch.float32, dev)
     if keep_idx is not None:
         _check_tensor("keep_idx", keep_idx, torch.int32, dev)
-    shape = infer_shape(x, A_log, W_dt, pool_axis, dir_flags, keep_idx, h, w, pool_scale, zoh_exact, path)
+    ln = ln_gamma is not None or ln_beta is not None
+    if ln:
+        if ln_gamma is None or ln_beta is None:
+            raise ValueError("the LayerNorm needs both ln_gamma and ln_beta")
+        _check_tensor("ln_gamma", ln_gamma, torch.float32, dev)
+        _check_tensor("ln_beta", ln_beta, torch.float32, dev)
+    shape = infer_shape(x, A_log, W_dt, pool_axis, dir_flags, keep_idx, h, w, pool_scale, zoh_exact, path, ln, ln_eps)
     if z.shape != x.shape or dy.shape != x.shape:
         raise ValueError("z and dy must have the shape of x")
     if grads is None:
         grads = {"dx": torch.empty_like(x), "dz": torch.empty_like(z)}
         for name, p in (("dA_log", A_log), ("dD", D), ("dW_x", W_x), ("dW_dt", W_dt), ("db_dt", b_dt)):
             grads[name] = torch.empty_like(p)
+        if ln:
+            grads["dln_gamma"], grads["dln_beta"] = torch.empty_like(ln_gamma), torch.empty_like(ln_beta)
     if workspace is None:
         workspace = torch.empty(max(backward_workspace_size(shape), 256), dtype=torch.uint8, device=dev)
-    a = shape.args(x, z, A_log, D, W_x, W_dt, b_dt, keep_idx)  # y is not read by the gradient
+    # y is not read by the gradient
+    a = shape.args(x, z, A_log, D, W_x, W_dt, b_dt, keep_idx, None, ln_gamma, ln_beta)
     g = _grads(dy, grads)
     st = nat.lib().fastvim_ssm_backward(ctypes.byref(a), ctypes.byref(g), ctypes.c_void_p(fwd_workspace.data_ptr()),
                                         ctypes.c_size_t(fwd_workspace.numel()), ctypes.c_void_p(workspace.data_ptr()),
@@ -278,7 +289,8 @@ class BoundBackward:
     def __init__(self, shape: LayerShape, t: dict, dy, grads: dict, fwd_workspace, workspace, stream=None):
         self.shape = shape
         self._keep = (t, dy, grads, fwd_workspace, workspace)
-        self._args = shape.args(t["x"], t["z"], t["A_log"], t["D"], t["W_x"], t["W_dt"], t["b_dt"], t.get("keep_idx"))
+        self._args = shape.args(t["x"], t["z"], t["A_log"], t["D"], t["W_x"], t["W_dt"], t["b_dt"], t.get("keep_idx"),
+                                None, t.get("ln_gamma"), t.get("ln_beta"))
         self._g = _grads(dy, grads)
         self._fw = (ctypes.c_void_p(fwd_workspace.data_ptr()), ctypes.c_size_t(fwd_workspace.numel()))
         self._ws = (ctypes.c_void_p(workspace.data_ptr()), ctypes.c_size_t(workspace.numel()))

@@ -32,10 +32,12 @@ def args(**kw):
     return a
 
 
-def grads(**kw):
+def grads(ln=False, **kw):
     g = nat.FvSsmGrads()
     for i, name in enumerate(("dy", "dx", "dz", "dA_log", "dD", "dW_x", "dW_dt", "db_dt")):
         setattr(g, name, FAKE + (12 + i) * SLOT)
+    if ln:
+        g.dln_gamma, g.dln_beta = FAKE + 30 * SLOT, FAKE + 31 * SLOT
     for k, v in kw.items():
         setattr(g, k, v)
     return g
@@ -87,7 +89,9 @@ def test_launch_lists(lib):
     assert lib.fastvim_ssm_backward_launch_name(ctypes.byref(args()), 5) == b""
     assert lib.fastvim_ssm_backward_launch_count(ctypes.byref(args(B=0, x=None, z=None, y=None))) == 0
     ln = args(flags=nat.FV_FLAG_LAYERNORM, ln_gamma=FAKE + 10 * SLOT, ln_beta=FAKE + 11 * SLOT, ln_eps=1e-5)
-    assert lib.fastvim_ssm_backward_launch_count(ctypes.byref(ln)) == 0
+    names = [lib.fastvim_ssm_backward_launch_name(ctypes.byref(ln), i).decode() for i in range(5)]
+    assert lib.fastvim_ssm_backward_launch_count(ctypes.byref(ln)) == 5
+    assert names[0] == "bwd_ln_gate_kernel" and names[1:] == dense[1:]
 
 
 def _bwd(lib, a, g, fwd=FAKE + 20 * SLOT, fwd_n=None, ws=FAKE + 22 * SLOT, ws_n=None):
@@ -105,7 +109,10 @@ def test_rejections_before_any_launch(lib):
     assert _bwd(lib, args(E=382), grads()) == nat.FV_ERR_SHAPE
     assert _bwd(lib, args(W_x=None), grads()) == nat.FV_ERR_NULL
     ln = args(flags=nat.FV_FLAG_LAYERNORM, ln_gamma=FAKE + 10 * SLOT, ln_beta=FAKE + 11 * SLOT, ln_eps=1e-5)
-    assert _bwd(lib, ln, grads()) == nat.FV_ERR_UNSUPPORTED
+    assert _bwd(lib, ln, grads()) == nat.FV_ERR_NULL  # the LayerNorm's gradients are required
+    assert _bwd(lib, ln, grads(ln=True, dln_beta=FAKE + 31 * SLOT + 4)) == nat.FV_ERR_ALIGN
+    assert _bwd(lib, ln, grads(ln=True), ws=0) == nat.FV_ERR_WORKSPACE  # accepted up to the workspace check
+    assert _bwd(lib, a, grads(ln=True)) == nat.FV_ERR_SHAPE  # LayerNorm gradients without the flag
     # gradient arrays
     assert _bwd(lib, a, None) == nat.FV_ERR_NULL
     for name in ("dy", "dx", "dz", "dA_log", "dD", "dW_x", "dW_dt", "db_dt"):

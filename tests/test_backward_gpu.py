@@ -42,39 +42,43 @@ def make_inputs(seed, B, h, w, E, N, R, nd, K=0, drop_row=None, pool_axis=0):
     return d
 
 
-def gpu_grads(d, pool_axis, dir_flags, h, w, pool_scale=1.0, zoh_exact=False, path="auto"):
+def gpu_grads(d, pool_axis, dir_flags, h, w, pool_scale=1.0, zoh_exact=False, path="auto", ln_eps=1e-5):
+    """d may hold ln_gamma and ln_beta: then the layer has the post-SSM LayerNorm."""
     dev = torch.device("cuda")
     t = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev) for k, v in d.items()}
     keep = t.get("keep_idx")
+    ln = "ln_gamma" in t
     shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, dir_flags, keep, h, w, pool_scale, zoh_exact,
-                            path)
+                            path, ln, ln_eps)
+    lnkw = dict(ln_gamma=t.get("ln_gamma"), ln_beta=t.get("ln_beta"), ln_eps=ln_eps)
     fws = ssm.alloc_workspace(shape, dev)
     fws.fill_(0xFF)
     ssm.forward(t["x"], t["z"], t["A_log"], t["D"], t["W_x"], t["W_dt"], t["b_dt"], pool_axis, dir_flags,
-                keep_idx=keep, h=h, w=w, pool_scale=pool_scale, zoh_exact=zoh_exact, workspace=fws, path=path)
+                keep_idx=keep, h=h, w=w, pool_scale=pool_scale, zoh_exact=zoh_exact, workspace=fws, path=path, **lnkw)
     fstatus = ssm.device_status(fws)
     bws = torch.full((max(ssm.backward_workspace_size(shape), 256),), 0xFF, dtype=torch.uint8, device=dev)
     grads = {"dx": torch.full_like(t["x"], float("nan")), "dz": torch.full_like(t["z"], float("nan"))}
-    for name in PARAMS:
+    for name in PARAMS + (("ln_gamma", "ln_beta") if ln else ()):
         grads["d" + name] = torch.full_like(t[name], float("nan"))
     ssm.backward(t["x"], t["z"], t["A_log"], t["D"], t["W_x"], t["W_dt"], t["b_dt"], t["dy"], fws, pool_axis,
                  dir_flags, keep_idx=keep, h=h, w=w, pool_scale=pool_scale, zoh_exact=zoh_exact, path=path,
-                 grads=grads, workspace=bws)
+                 grads=grads, workspace=bws, **lnkw)
     torch.cuda.synchronize()
     return {k: v.cpu().numpy() for k, v in grads.items()}, fstatus, ssm.backward_launch_names(shape)
 
 
-def oracle_grads(d, pool_axis, dir_flags, h, w, pool_scale=1.0, zoh_exact=False, allow_bad_index=False):
+def oracle_grads(d, pool_axis, dir_flags, h, w, pool_scale=1.0, zoh_exact=False, allow_bad_index=False, ln_eps=1e-5):
     return oracle.backward(d["x"], d["z"], d["A_log"], d["D"], d["W_x"], d["W_dt"], d["b_dt"], d["dy"], pool_axis,
                            dir_flags, keep_idx=d.get("keep_idx"), h=h, w=w, pool_scale=pool_scale, zoh_exact=zoh_exact,
-                           nthreads=8, allow_bad_index=allow_bad_index)
+                           nthreads=8, allow_bad_index=allow_bad_index, ln_gamma=d.get("ln_gamma"),
+                           ln_beta=d.get("ln_beta"), ln_eps=ln_eps)
 
 
 def compare(got, ref, what):
     reps = {}
     for k in ("dx", "dz"):
         reps[k] = assert_close(got[k], ref[k], f"{what} {k}")
-    for name in PARAMS:
+    for name in PARAMS + (("ln_gamma", "ln_beta") if "dln_gamma" in ref else ()):
         reps["d" + name] = assert_close(got["d" + name], ref["d" + name], f"{what} d{name}", GRAD_PARAM_ABS_RMS)
     print(what, {k: (round(v["max_abs_over_rms"], 9), round(v["max_err_over_bound"], 4)) for k, v in reps.items()})
     return reps
@@ -162,3 +166,31 @@ def test_gradient_is_reproducible_up_to_atomic_order():
     np.testing.assert_array_equal(a["dz"], b["dz"])
     for name in PARAMS:
         np.testing.assert_allclose(a["d" + name], b["d" + name], rtol=1e-5, atol=1e-6 * np.abs(b["d" + name]).max())
+
+
+LN_CASES = [
+    # B, h, w, E, N, R, pool_axis, K, path   (K > 0: masked, 75 % of the grid kept)
+    (2, 14, 14, 384, 16, 12, 0, 0, "staged"),
+    (2, 14, 14, 384, 16, 12, 1, 0, "staged"),
+    (2, 64, 64, 1024, 16, 64, 0, 0, "fused"),
+    (3, 13, 7, 68, 5, 3, 1, 0, "staged"),
+    (2, 8, 8, 1536, 16, 48, 0, 48, "auto"),
+    (1, 3, 5, 4096, 16, 8, 0, 0, "staged"),
+    (2, 16, 16, 132, 16, 8, 1, 100, "auto"),
+]
+
+
+@pytest.mark.parametrize("case", LN_CASES, ids=lambda c: "x".join(map(str, c[:6])) + f"-a{c[6]}K{c[7]}{c[8]}")
+def test_layernorm_gradient(case):
+    """The gradient through the post-SSM LayerNorm (gamma, beta drawn around their init), the
+    three warp counts its kernel picks by E (4 up to E = 1316, 2 up to 2272, then 1), dense on
+    either forward path and masked."""
+    B, h, w, E, N, R, axis, K, path = case
+    d = make_inputs(17, B, h, w, E, N, R, 2, K=K)
+    rng = np.random.default_rng([17, 5])
+    d["ln_gamma"] = rng.uniform(0.5, 1.5, E).astype(np.float32)
+    d["ln_beta"] = rng.uniform(-0.5, 0.5, E).astype(np.float32)
+    got, fst, names = gpu_grads(d, axis, 3, h, w, path=path)
+    assert fst == 0 and names[0] == "bwd_ln_gate_kernel"
+    ref = oracle_grads(d, axis, 3, h, w)
+    compare(got, ref, f"layernorm {case}")

@@ -33,6 +33,7 @@ def test_every_launched_kernel_has_a_bound(cfg):
             names |= set(ssm.launch_names(_shape(cfg, axis, path)))
         names |= set(ssm.launch_names(_shape(cfg, axis, "auto", ln=True)))
         names |= set(ssm.backward_launch_names(_shape(cfg, axis)))
+        names |= set(ssm.backward_launch_names(_shape(cfg, axis, ln=True)))
         for n in names:
             bound, amount = bench.kernel_work(n, cfg, axis)
             if n == "mask_bucket_kernel":  # integer bucketing: no roofline of its own
