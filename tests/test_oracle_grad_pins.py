@@ -146,3 +146,50 @@ def test_rejected_id_gets_no_gradient(oracle_mod=None):
     assert g["status"] == oracle_mod.FVO_BAD_INDEX
     assert not g["dx"][0, 3].any() and not g["dz"][0, 3].any()
     assert g["dx"][0, 1].any() and g["dz"][0, 1].any()
+
+
+def test_gradient_axis_and_direction_symmetries(oracle_mod=None):
+    """Pooling over h is pooling over w of the transposed grid, and a backward-only scan is a
+    forward-only scan of the sequence read in reverse: the gradients must map the same way."""
+    import oracle
+    oracle_mod = oracle_mod or oracle
+    rng = np.random.default_rng(700)
+    B, h, w, E, N, R = 2, 3, 5, 4, 3, 2
+    x, z, dy, P, _ = _case(rng, False, B=B, h=h, w=w, E=E, N=N, R=R)
+    args = (P["A_log"], P["D"], P["W_x"], P["W_dt"], P["b_dt"])
+    tr = lambda a: np.ascontiguousarray(a.transpose(0, 2, 1, 3))  # noqa: E731
+    gh = oracle_mod.backward(x, z, *args, dy, 1, 3)
+    gw = oracle_mod.backward(tr(x), tr(z), *args, tr(dy), 0, 3)
+    np.testing.assert_allclose(gh["dx"], tr(gw["dx"]), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(gh["dz"], tr(gw["dz"]), rtol=1e-12, atol=1e-13)
+    for k in PARAMS:
+        np.testing.assert_allclose(gh["d" + k], gw["d" + k], rtol=1e-11, atol=1e-13)
+    # backward-only on x == forward-only on x flipped along the scan axis (POOL_W: axis h)
+    one = {k: v[:1].copy() for k, v in P.items()}
+    a1 = (one["A_log"], one["D"], one["W_x"], one["W_dt"], one["b_dt"])
+    fl = lambda a: np.ascontiguousarray(a[:, ::-1])  # noqa: E731
+    gb = oracle_mod.backward(x, z, *a1, dy, 0, 2)
+    gf = oracle_mod.backward(fl(x), fl(z), *a1, fl(dy), 0, 1)
+    np.testing.assert_allclose(gb["dx"], fl(gf["dx"]), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(gb["dz"], fl(gf["dz"]), rtol=1e-12, atol=1e-13)
+    for k in PARAMS:
+        np.testing.assert_allclose(gb["d" + k], gf["d" + k], rtol=1e-11, atol=1e-13)
+
+
+def test_masked_gradient_follows_a_permutation_of_the_kept_ids(oracle_mod=None):
+    """Listing the kept tokens in another order permutes dx and dz the same way and leaves the
+    parameter gradients unchanged."""
+    import oracle
+    oracle_mod = oracle_mod or oracle
+    rng = np.random.default_rng(800)
+    x, z, dy, P, kw = _case(rng, True)
+    args = (P["A_log"], P["D"], P["W_x"], P["W_dt"], P["b_dt"])
+    g0 = oracle_mod.backward(x, z, *args, dy, 0, 3, **kw)
+    perm = rng.permutation(x.shape[1])
+    kw2 = dict(kw, keep_idx=np.ascontiguousarray(kw["keep_idx"][:, perm]))
+    g1 = oracle_mod.backward(np.ascontiguousarray(x[:, perm]), np.ascontiguousarray(z[:, perm]), *args,
+                             np.ascontiguousarray(dy[:, perm]), 0, 3, **kw2)
+    np.testing.assert_allclose(g1["dx"], g0["dx"][:, perm], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(g1["dz"], g0["dz"][:, perm], rtol=1e-12, atol=1e-13)
+    for k in PARAMS:
+        np.testing.assert_allclose(g1["d" + k], g0["d" + k], rtol=1e-11, atol=1e-13)
