@@ -163,3 +163,78 @@ def test_validation_layout_and_launch_list(a, pick):
         # shape errors: no workspace, no launches
         assert lib.fastvim_ssm_workspace_size(ctypes.byref(a)) == 0
         assert lib.fastvim_ssm_launch_count(ctypes.byref(a)) == 0
+
+
+GRAD_NAMES = ("dy", "dx", "dz", "dA_log", "dD", "dW_x", "dW_dt", "db_dt")
+
+
+def _grads_for(a):
+    g = nat.FvSsmGrads()
+    for i, name in enumerate(GRAD_NAMES):
+        setattr(g, name, FAKE + (12 + i) * SLOT)
+    if a.flags & nat.FV_FLAG_LAYERNORM:
+        g.dln_gamma, g.dln_beta = FAKE + 20 * SLOT, FAKE + 21 * SLOT
+    return g
+
+
+GRAD_BREAKS = [
+    ("no grads block", lambda a, g: True, None, nat.FV_ERR_NULL),
+    ("no dA_log", lambda a, g: True, ("dA_log", None), nat.FV_ERR_NULL),
+    ("no dx", lambda a, g: a.B > 0, ("dx", None), nat.FV_ERR_NULL),
+    ("no dy", lambda a, g: a.B > 0, ("dy", None), nat.FV_ERR_NULL),
+    ("misaligned dW_x", lambda a, g: True, ("dW_x", FAKE + 17 * SLOT + 4), nat.FV_ERR_ALIGN),
+    ("dx aliases x", lambda a, g: a.B > 0, ("dx", FAKE), nat.FV_ERR_ALIAS),
+    ("dz aliases dy", lambda a, g: a.B > 0, ("dz", FAKE + 12 * SLOT), nat.FV_ERR_ALIAS),
+    ("LayerNorm gradient missing", lambda a, g: a.flags & nat.FV_FLAG_LAYERNORM, ("dln_beta", None),
+     nat.FV_ERR_NULL),
+    ("LayerNorm gradient without the flag", lambda a, g: not a.flags & nat.FV_FLAG_LAYERNORM,
+     ("dln_gamma", FAKE + 20 * SLOT), nat.FV_ERR_SHAPE),
+]
+
+
+@settings(max_examples=300, deadline=None)
+@given(valid_layer(), st.integers(-len(GRAD_BREAKS), len(GRAD_BREAKS) - 1))
+def test_gradient_validation_and_plan(a, pick):
+    lib = nat.lib()
+    if lib.fastvim_ssm_validate(ctypes.byref(a)) != nat.FV_OK:
+        return
+    L = nat.FvBwdWsLayout()
+    assert lib.fastvim_ssm_backward_workspace_layout(ctypes.byref(a), ctypes.byref(L)) == nat.FV_OK
+    assert lib.fastvim_ssm_backward_workspace_size(ctypes.byref(a)) == L.total_bytes
+    T = a.h if a.pool_axis == POOL_W else a.w
+    nd = bin(a.dir_flags).count("1")
+    ub = -(-T * (a.R + 2 * a.N) // 32) * 32
+    bte = a.B * T * a.E * 4
+    regions = sorted([(L.dys, bte), (L.dxbar, bte), (L.du, nd * a.B * ub * 4), (L.dxs, nd * bte),
+                      (L.ckpt, a.B * nd * 2 * -(-T // 16) * a.E * 16 * 4)])
+    end = 0
+    for off, n in regions:
+        assert off % 256 == 0 and off >= end
+        end = off + n
+    assert end <= L.total_bytes < end + 256 * len(regions)
+    n = lib.fastvim_ssm_backward_launch_count(ctypes.byref(a))
+    names = [lib.fastvim_ssm_backward_launch_name(ctypes.byref(a), i).decode() for i in range(n)]
+    if a.B == 0:
+        assert n == 0
+    else:
+        first = ("bwd_ln_gate_kernel" if a.flags & nat.FV_FLAG_LAYERNORM else
+                 "bwd_gate_masked_kernel" if a.K else "bwd_gate_dense_kernel")
+        assert names[0] == first and names[1] == "bwd_scan_kernel" and len(names) == 5
+    g = _grads_for(a)
+    fws = lib.fastvim_ssm_workspace_size(ctypes.byref(a))
+
+    def call(gp):
+        # a NULL gradient workspace: every argument check runs, nothing is queued
+        return lib.fastvim_ssm_backward(ctypes.byref(a), gp, ctypes.c_void_p(FAKE + 40 * SLOT), fws, None, 0, None)
+
+    if pick < 0:
+        assert call(ctypes.byref(g)) == nat.FV_ERR_WORKSPACE
+        return
+    name, applies, change, want = GRAD_BREAKS[pick]
+    if not applies(a, g):
+        return
+    if change is None:
+        assert call(None) == want, name
+        return
+    setattr(g, change[0], change[1])
+    assert call(ctypes.byref(g)) == want, name
