@@ -1,9 +1,9 @@
-"""Full-size parity of the gradient: the 2048 px FastVim-T layer (B = 128, 128 x 128 grid,
-E = 384, column pooling, both directions) in the launch configuration the benchmark's gradient
-leg times (one forward call over the batch, then one gradient call on its workspace).  The
-parameter gradients, sums over all 128 images, are compared in full with the oracle's sum
-(computed image by image from each image's seeded stream); dx and dz on sampled images (first,
-middle, last)."""
+"""Full-size parity of the gradient in the launch configuration the benchmark's gradient leg
+times (one forward call over the batch, then one gradient call on its workspace): the 2048 px
+FastVim-T layer (B = 128, 128 x 128 grid, E = 384) and the masked FastMaskVim-B layer (B = 64,
+1,024 of 4,096 tokens kept, E = 1536).  The parameter gradients, sums over the whole batch, are
+compared in full with the oracle's sum (computed image by image from each image's seeded
+stream); dx and dz on sampled images (first, middle, last)."""
 import numpy as np
 import pytest
 
@@ -20,17 +20,23 @@ pytestmark = [pytest.mark.gpu, pytest.mark.slow,
 PARAMS = ("A_log", "D", "W_x", "W_dt", "b_dt")
 
 
-def test_full_size_gradient_fastvim_t_2048():
-    cfg = CONFIGS[3]
+@pytest.mark.parametrize("ci", [3, 4])
+def test_full_size_gradient(ci):
+    """ci 3: the 2048 px FastVim-T layer (fused forward); ci 4: the 75 %-masked FastMaskVim-B layer
+    (E = 1536, staged forward)."""
+    cfg = CONFIGS[ci]
     axis = cfg.pool_axes[0]
     dev = torch.device("cuda")
     t = workload.layer_tensors(cfg, dev)
     dy = workload.upstream_grad(cfg, dev)
-    shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], axis, cfg.dir_flags)
+    keep = t.get("keep_idx")
+    shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], axis, cfg.dir_flags, keep, cfg.h, cfg.w)
     fws = ssm.alloc_workspace(shape, dev)
-    ssm.forward(t["x"], t["z"], t["A_log"], t["D"], t["W_x"], t["W_dt"], t["b_dt"], axis, cfg.dir_flags, workspace=fws)
+    ssm.forward(t["x"], t["z"], t["A_log"], t["D"], t["W_x"], t["W_dt"], t["b_dt"], axis, cfg.dir_flags, keep_idx=keep,
+                h=cfg.h, w=cfg.w, workspace=fws)
     assert ssm.device_status(fws) == 0
-    g = ssm.backward(t["x"], t["z"], t["A_log"], t["D"], t["W_x"], t["W_dt"], t["b_dt"], dy, fws, axis, cfg.dir_flags)
+    g = ssm.backward(t["x"], t["z"], t["A_log"], t["D"], t["W_x"], t["W_dt"], t["b_dt"], dy, fws, axis, cfg.dir_flags,
+                     keep_idx=keep, h=cfg.h, w=cfg.w)
     torch.cuda.synchronize()
     samples = [0, cfg.B // 2, cfg.B - 1]
     got = {k: g[k][samples].cpu().numpy() for k in ("dx", "dz")}
@@ -48,8 +54,12 @@ def test_full_size_gradient_fastvim_t_2048():
         x = np.stack([inputs.image_x(cfg.seed, b, shp) for b in ids])
         z = np.stack([inputs.image_z(cfg.seed, b, shp) for b in ids])
         dyi = np.stack([inputs.image_dy(cfg.seed, b, shp) for b in ids])
+        kw = {}
+        if cfg.masked:
+            kw = dict(keep_idx=np.stack([inputs.image_keep_idx(cfg.seed, b, cfg.h, cfg.w, cfg.K) for b in ids]),
+                      h=cfg.h, w=cfg.w)
         r = oracle.backward(x, z, p["A_log"], p["D"], p["W_x"], p["W_dt"], p["b_dt"], dyi, axis, cfg.dir_flags,
-                            nthreads=chunk)
+                            nthreads=chunk, **kw)
         for n in PARAMS:
             sums["d" + n] += r["d" + n]
         for b in ids:

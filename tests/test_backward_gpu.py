@@ -94,6 +94,7 @@ DENSE = [
     (2, 5, 37, 64, 16, 4, 1, 3, True, 1.0, "staged"),
     (2, 16, 9, 256, 16, 16, 0, 3, False, 1.0, "staged"),
     (1, 1, 1, 4, 1, 1, 0, 3, False, 1.0, "staged"),
+    (1, 6, 5, 2048, 16, 8, 1, 3, False, 1.0, "staged"),
     (2, 64, 64, 1024, 16, 64, 0, 3, False, 1.0, "fused"),
     (2, 64, 64, 1024, 16, 64, 0, 3, False, 1.0, "staged"),
 ]
