@@ -41,6 +41,7 @@ METRIC = "SSM-layer grid tokens/s at 2048² FastVim-T (fp32, B=128); HBM GB/s vs
 UNIT = "grid tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 REFERENCE_BUDGET_S = 150.0
+HEADLINE_NAME = "fastvim_t_2048"
 
 L2_BYTES = 126 * 1024 * 1024
 # Special-function (MUFU) lanes per SM per clock on sm_100: 4 per SM sub-partition.
@@ -113,6 +114,9 @@ def parse(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-configs", action="store_true",
+                    help="time only the chosen workload (by default the headline run also times the other "
+                         "workloads and reports them under 'configs')")
     ap.add_argument("--grad", action="store_true",
                     help="time a training step: the forward call, then the gradient call on its workspace")
     a = ap.parse_args(argv)
@@ -356,29 +360,68 @@ def run_reference(a, cfg, pool_axis):
 # ------------------------------------------------------------------------------------------------
 # Our arm
 # ------------------------------------------------------------------------------------------------
-def run_ours(a, cfg, pool_axis):
+# The other workloads of the method's efficiency study, timed in the same default run after the
+# headline (one GPU): (config name, pool axis).  The 224 px layer runs both axes (alternating
+# blocks); its inputs fit in L2, so each of its steps starts after an L2 flush.
+SECONDARY = (("fastvim_t_224_tiny", 0), ("fastvim_t_224", 0), ("fastvim_t_224", 1), ("fastvim_s_1024", 1),
+             ("fastmaskvim_b_1024_mask75", 0))
+
+
+def summarize_kernels(per_kernel, names, cfg, pool_axis, peak, mufu_peak, fma_peak):
+    """Per kernel: launches per step, mean device time per step, share of the step's kernel time,
+    and achieved work rate against the bound of kernel_work."""
+    total_k = sum(sum(v) for v in per_kernel.values())
+    kern = {}
+    for n, v in per_kernel.items():
+        avg_s = statistics.mean(v) / 1e3
+        bound, amount = kernel_work(n, cfg, pool_axis)
+        ent = {"launches_per_step": names.count(n), "us_per_step": avg_s * 1e6,
+               "share": sum(v) / total_k if total_k > 0 else 0.0, "bound": bound}
+        if bound == "hbm":
+            ent.update(achieved=amount / avg_s / 1e9, unit="GB/s", frac=amount / avg_s / 1e9 / peak)
+        elif bound == "alu":
+            ent.update(achieved=amount / avg_s / 1e9, unit="G exp2/s", frac=amount / avg_s / 1e9 / mufu_peak)
+        elif bound == "fma":
+            ent.update(achieved=amount / avg_s / 1e12, unit="TFLOP/s fp32", frac=amount / avg_s / 1e12 / fma_peak)
+        kern[n] = ent
+    return kern
+
+
+def roofline_of(kern, dom, cfg, pool_axis, peak, peak_src, mufu_peak, fma_peak):
+    """The roofline object of the dominant kernel `dom` (algorithmic amount per launch over the mean
+    CUDA-event duration of its launches)."""
+    bound, amount = kernel_work(dom, cfg, pool_axis)
+    dk = kern[dom]
+    amount //= max(1, dk["launches_per_step"])
+    if bound == "alu":
+        return {"bound": "alu", "kernel": dom, "achieved": dk["achieved"], "peak": mufu_peak,
+                "unit": "G exp2/s", "frac": dk["frac"], "traffic": recorded_traffic(dom, cfg.name),
+                "algorithmic_exp2_per_launch": amount,
+                "peak_source": f"derived: SMs x {MUFU_PER_SM_CLK} MUFU lanes/clk x max SM clock",
+                "note": "achieved = exp2 evaluations per launch / mean CUDA-event duration of the launch"}
+    if bound == "fma":
+        return {"bound": "alu", "kernel": dom, "achieved": dk["achieved"], "peak": fma_peak,
+                "unit": "TFLOP/s fp32", "frac": dk["frac"], "traffic": recorded_traffic(dom, cfg.name),
+                "algorithmic_flop_per_launch": amount,
+                "peak_source": f"derived: SMs x {FFMA_PER_SM_CLK} FMA lanes/clk x 2 flop x max SM clock",
+                "note": "achieved = flops per launch / mean CUDA-event duration of the launch"}
+    return {"bound": "hbm", "kernel": dom, "achieved": dk.get("achieved"), "peak": peak, "unit": "GB/s",
+            "frac": dk.get("frac"), "traffic": recorded_traffic(dom, cfg.name),
+            "algorithmic_bytes_per_launch": amount, "peak_source": peak_src,
+            "note": "achieved = algorithmic bytes per launch / mean CUDA-event duration of the launch"}
+
+
+def time_layer(a, cfg, pool_axis, dev, world=1, first_image=0, clocks=None):
+    """Device-timed forward calls of one workload (inputs resident in HBM): `a.warmup` untimed calls,
+    then `a.steps` timed ones between CUDA events on the launching stream, each launch bracketed by
+    its own pair of events.  Returns the step time (max over ranks), the per-kernel table and the
+    roofline of the dominant kernel, plus the shape (for the end-to-end leg)."""
     import torch
     import torch.distributed as dist
 
-    from pooled_selective_scan_b200 import build as fvbuild
     from pooled_selective_scan_b200 import ssm, workload
 
-    world, rank, local = dist_env()
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device (the layer has no CPU path)")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
-    if not os.path.exists(os.path.join(ROOT, "pooled_selective_scan_b200", "libfastvim_ssm.so")):
-        if rank == 0:
-            fvbuild.build()
-        if world > 1:
-            dist.barrier()
-
-    mine = workload.shard_images(cfg, rank, world)
-    t = workload.layer_tensors(cfg, dev, first_image=mine.start)
+    t = workload.layer_tensors(cfg, dev, first_image=first_image)
     if a.ln:
         t.update(workload.ln_tensors(cfg, dev))
     keep = t.get("keep_idx")
@@ -395,7 +438,7 @@ def run_ours(a, cfg, pool_axis):
         fwd.run()
     torch.cuda.synchronize(dev)
     if ssm.device_status(ws) != 0:
-        raise SystemExit("device status reported an error during warm-up")
+        raise SystemExit(f"{cfg.name}: device status reported an error during warm-up")
 
     # events[2j], events[2j+1] bracket launch j on the stream it runs on
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nl)] for _ in range(a.steps)]
@@ -410,8 +453,10 @@ def run_ours(a, cfg, pool_axis):
     alg_bytes_call = cfg.algorithmic_bytes_per_call()
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if alg_bytes_call < 2 * L2_BYTES else None
 
-    clocks = ClockSampler(local)
-    clocks.start()
+    own_clocks = clocks is None
+    if own_clocks:
+        clocks = ClockSampler(dev.index or 0)
+        clocks.start()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -424,14 +469,14 @@ def run_ours(a, cfg, pool_axis):
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    clocks.stop()
+    if own_clocks:
+        clocks.stop()
     if flush is None:
         local_ms = start.elapsed_time(end)
     else:
         local_ms = sum(evs[0].elapsed_time(evs[2 * nl - 1]) for evs in events)  # first to last launch
     max_ms = reduce_max(local_ms, dev)
-    # per kernel: its launches' device time in each step (a staged layer launches each kernel once
-    # per chunk of images; those launches run one after another)
+    # per kernel: its launches' device time in each step
     per_kernel = {n: [] for n in dict.fromkeys(names)}
     for evs in events:
         step = {n: 0.0 for n in per_kernel}
@@ -440,101 +485,153 @@ def run_ours(a, cfg, pool_axis):
         for n, v in step.items():
             per_kernel[n].append(v)
     if ssm.device_status(ws) != 0:
-        raise SystemExit("device status reported an error in the timed region")
+        raise SystemExit(f"{cfg.name}: device status reported an error in the timed region")
 
     tokens = cfg.tokens_per_call()
     ms_step = max_ms / a.steps
-    value = weak_scaling_value(tokens * a.steps, world, max_ms / 1e3)
     peak, peak_src = load_peaks()
-
-    total_k = sum(sum(v) for v in per_kernel.values())
-    mufu_peak = mufu_peak_gops(local, clocks.summary().get("sm_max_mhz"))
-    fma_peak = ffma_peak_tflops(local, clocks.summary().get("sm_max_mhz"))
-    kern = {}
-    for n, v in per_kernel.items():
-        avg_s = statistics.mean(v) / 1e3
-        bound, amount = kernel_work(n, cfg, pool_axis)
-        ent = {"launches_per_step": names.count(n), "us_per_step": avg_s * 1e6, "share": sum(v) / total_k,
-               "bound": bound}
-        if bound == "hbm":
-            ent.update(achieved=amount / avg_s / 1e9, unit="GB/s", frac=amount / avg_s / 1e9 / peak)
-        elif bound == "alu":
-            ent.update(achieved=amount / avg_s / 1e9, unit="G exp2/s", frac=amount / avg_s / 1e9 / mufu_peak)
-        elif bound == "fma":
-            ent.update(achieved=amount / avg_s / 1e12, unit="TFLOP/s fp32", frac=amount / avg_s / 1e12 / fma_peak)
-        kern[n] = ent
+    summ = clocks.summary()
+    mufu_peak = mufu_peak_gops(dev.index or 0, summ.get("sm_max_mhz"))
+    fma_peak = ffma_peak_tflops(dev.index or 0, summ.get("sm_max_mhz"))
+    kern = summarize_kernels(per_kernel, names, cfg, pool_axis, peak, mufu_peak, fma_peak)
     dom = max(kern, key=lambda n: kern[n]["share"])
-    bound, amount = kernel_work(dom, cfg, pool_axis)
-    dk = kern[dom]
-    amount //= max(1, dk["launches_per_step"])  # per launch: one chunk of the batch
-    if bound == "alu":
-        roofline = {"bound": "alu", "kernel": dom, "achieved": dk["achieved"], "peak": mufu_peak,
-                    "unit": "G exp2/s", "frac": dk["frac"], "traffic": recorded_traffic(dom, cfg.name),
-                    "algorithmic_exp2_per_launch": amount,
-                    "peak_source": f"derived: SMs x {MUFU_PER_SM_CLK} MUFU lanes/clk x max SM clock",
-                    "note": "achieved = exp2 evaluations per launch / mean CUDA-event duration of the launch"}
-    elif bound == "fma":
-        roofline = {"bound": "alu", "kernel": dom, "achieved": dk["achieved"], "peak": fma_peak,
-                    "unit": "TFLOP/s fp32", "frac": dk["frac"], "traffic": recorded_traffic(dom, cfg.name),
-                    "algorithmic_flop_per_launch": amount,
-                    "peak_source": f"derived: SMs x {FFMA_PER_SM_CLK} FMA lanes/clk x 2 flop x max SM clock",
-                    "note": "achieved = flops per launch / mean CUDA-event duration of the launch"}
-    else:
-        roofline = {"bound": "hbm", "kernel": dom, "achieved": dk.get("achieved"), "peak": peak, "unit": "GB/s",
-                    "frac": dk.get("frac"), "traffic": recorded_traffic(dom, cfg.name),
-                    "algorithmic_bytes_per_launch": amount, "peak_source": peak_src,
-                    "note": "achieved = algorithmic bytes per launch / mean CUDA-event duration of the launch"}
-
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
-        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32", "data": "synthetic (seeded N(0,1) x, z; Mamba-style parameter init)",
-        "config": dict(workload_desc(cfg, pool_axis),
-                       **({"post_ssm_layernorm": "gamma = 1, beta = 0, eps = 1e-5"} if a.ln else {}),
-                       l2=(f"inputs {alg_bytes_call / 1e9:.2f} GB per step > 126 MB L2; no flush" if flush is None
-                           else f"inputs {alg_bytes_call / 1e6:.1f} MB per step < 2 x L2: L2 flushed (256 MB write) "
-                                f"before every step, step time = span of the step's launches"),
-                       global_batch=cfg.B * world,
-                       parallelism=f"data parallel, no collective: each of {world} GPU(s) runs its own "
-                                   f"{cfg.B} distinct images"),
+    res = {
+        "ms_per_step": ms_step,
+        "value": weak_scaling_value(tokens * a.steps, world, max_ms / 1e3),
         "layer_hbm": {"achieved_gbs": alg_bytes_call / (ms_step / 1e3) / 1e9, "peak_gbs": peak,
                       "frac": alg_bytes_call / (ms_step / 1e3) / 1e9 / peak,
                       "algorithmic_bytes_per_step": alg_bytes_call},
-        "roofline": roofline,
+        "roofline": roofline_of(kern, dom, cfg, pool_axis, peak, peak_src, mufu_peak, fma_peak),
         "kernels": kern,
         "gpu_launches": nl * a.steps,
-        "clocks": clocks.summary(),
+        "l2": (f"inputs {alg_bytes_call / 1e9:.2f} GB per step > 126 MB L2; no flush" if flush is None
+               else f"inputs {alg_bytes_call / 1e6:.1f} MB per step < 2 x L2: L2 flushed (256 MB write) "
+                    f"before every step, step time = span of the step's launches"),
+        "shape": shape,
     }
+    if own_clocks:
+        res["clocks"] = summ
+    del fwd, t, y, ws, events, flush
+    torch.cuda.empty_cache()
+    return res
 
-    del events
-    # end-to-end leg: host buffers through fastvim_ssm_forward_host (every rank runs it; max over ranks)
-    if not a.no_e2e:
-        del fwd
-        dev_keep = None
-        del t, y
-        torch.cuda.empty_cache()
-        host = workload.layer_tensors(cfg, dev, pinned_host=True, first_image=mine.start)
-        if a.ln:
-            host.update({k: v.pin_memory() for k, v in workload.ln_tensors(cfg, "cpu").items()})
-        run = ssm.HostForward(shape, dev)
-        y_host = torch.empty(host["x"].shape, dtype=torch.float32).pin_memory()
-        run(host, y_host)  # warm
+
+def link_copy_rates(dev, nbytes=1 << 30, reps=3):
+    """Measured pinned-host <-> device copy rates (GB/s) over one direction at a time: the host
+    link's own ceiling for the end-to-end leg."""
+    import torch
+    h = torch.empty(nbytes // 4, dtype=torch.float32).pin_memory()
+    d = torch.empty(nbytes // 4, dtype=torch.float32, device=dev)
+    rates = {}
+    for name, (dst, src) in (("h2d", (d, h)), ("d2h", (h, d))):
+        best = float("inf")
+        for _ in range(reps):
+            torch.cuda.synchronize(dev)
+            t0 = time.perf_counter()
+            dst.copy_(src, non_blocking=True)
+            torch.cuda.synchronize(dev)
+            best = min(best, time.perf_counter() - t0)
+        rates[name] = nbytes / best / 1e9
+    del h, d
+    return rates
+
+
+def time_e2e(a, cfg, shape, dev, world=1, first_image=0):
+    """End-to-end calls through fastvim_ssm_forward_host on pinned host buffers (every rank; max
+    over ranks), with the host link's measured copy rates as its ceiling."""
+    import torch
+    import torch.distributed as dist
+
+    from pooled_selective_scan_b200 import ssm, workload
+
+    host = workload.layer_tensors(cfg, dev, pinned_host=True, first_image=first_image)
+    if a.ln:
+        host.update({k: v.pin_memory() for k, v in workload.ln_tensors(cfg, "cpu").items()})
+    run = ssm.HostForward(shape, dev)
+    y_host = torch.empty(host["x"].shape, dtype=torch.float32).pin_memory()
+    run(host, y_host)  # warm
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for _ in range(a.e2e_steps):
+        run(host, y_host)
+    el = reduce_max(time.perf_counter() - t0, dev)
+    tokens = cfg.tokens_per_call()
+    bi, bo = run.h2d_bytes(), run.d2h_bytes()
+    del run, host, y_host
+    torch.cuda.empty_cache()
+    rates = link_copy_rates(dev)
+    step_s = el / a.e2e_steps
+    # the two directions run on separate copy engines: the slower one bounds a step
+    bound_s = max(bi / (rates["h2d"] * 1e9), bo / (rates["d2h"] * 1e9))
+    return {"value": weak_scaling_value(tokens * a.e2e_steps, world, el), "unit": UNIT,
+            "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": a.e2e_steps,
+            "link": {"h2d_gbs": bi / step_s / 1e9, "d2h_gbs": bo / step_s / 1e9,
+                     "h2d_copy_gbs_measured": rates["h2d"], "d2h_copy_gbs_measured": rates["d2h"],
+                     "bound_ms": bound_s * 1e3, "frac": bound_s / step_s,
+                     "note": "frac = the step time that one-way pinned copies at the measured rates would take, "
+                             "over the measured step time"},
+            "note": "pinned host x, z, params -> device, layer, y -> pinned host; per-step wall time"}
+
+
+def run_ours(a, cfg, pool_axis):
+    import torch
+    import torch.distributed as dist
+
+    from pooled_selective_scan_b200 import build as fvbuild
+    from pooled_selective_scan_b200 import workload
+    from pooled_selective_scan_b200.configs import by_name
+
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the layer has no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    if not os.path.exists(os.path.join(ROOT, "pooled_selective_scan_b200", "libfastvim_ssm.so")):
+        if rank == 0:
+            fvbuild.build()
         if world > 1:
             dist.barrier()
-        t0 = time.perf_counter()
-        for _ in range(a.e2e_steps):
-            run(host, y_host)
-        el = reduce_max(time.perf_counter() - t0, dev)
-        line["e2e"] = {"value": weak_scaling_value(tokens * a.e2e_steps, world, el), "unit": UNIT,
-                       "h2d_bytes_per_step": run.h2d_bytes(), "d2h_bytes_per_step": run.d2h_bytes(),
-                       "steps": a.e2e_steps,
-                       "note": "pinned host x, z, params -> device, layer, y -> pinned host; per-step wall time"}
-        del run, host, y_host, dev_keep
-    else:
-        line["e2e"] = None
+
+    mine = workload.shard_images(cfg, rank, world)
+    r = time_layer(a, cfg, pool_axis, dev, world, first_image=mine.start)
+    line = {
+        "metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic (seeded N(0,1) x, z; Mamba-style parameter init)",
+        "config": dict(workload_desc(cfg, pool_axis),
+                       **({"post_ssm_layernorm": "gamma = 1, beta = 0, eps = 1e-5"} if a.ln else {}),
+                       l2=r["l2"], global_batch=cfg.B * world,
+                       parallelism=f"data parallel, no collective: each of {world} GPU(s) runs its own "
+                                   f"{cfg.B} distinct images"),
+        "layer_hbm": r["layer_hbm"],
+        "roofline": r["roofline"],
+        "kernels": r["kernels"],
+        "gpu_launches": r["gpu_launches"],
+        "clocks": r["clocks"],
+    }
+    line["e2e"] = None if a.no_e2e else time_e2e(a, cfg, r["shape"], dev, world, first_image=mine.start)
 
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, pool_axis)
+
+    # the other workloads of the efficiency study, one GPU, default run only
+    if world == 1 and not a.no_configs and a.batch is None and cfg.name == HEADLINE_NAME:
+        configs = {}
+        for name, axis in SECONDARY:
+            c = by_name(name)
+            sub = time_layer(a, c, axis, dev)
+            ent = {"workload": workload_desc(c, axis), "ms_per_step": sub["ms_per_step"], "value": sub["value"],
+                   "unit": UNIT + (" (kept tokens)" if c.masked else ""), "steps": a.steps, "warmup": a.warmup,
+                   "l2": sub["l2"], "layer_hbm": sub["layer_hbm"], "roofline": sub["roofline"],
+                   "kernels": sub["kernels"], "gpu_launches": sub["gpu_launches"], "clocks": sub["clocks"]}
+            if not a.no_cpu_baseline:
+                ent["cpu_baseline"] = cpu_baseline(c, axis, min_seconds=5.0)
+            configs[f"{name}/{'pool_w' if axis == 0 else 'pool_h'}"] = ent
+        line["configs"] = configs
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -619,20 +716,7 @@ def run_grad(a, cfg, pool_axis):
     peak, peak_src = load_peaks()
     mufu_peak = mufu_peak_gops(local, clocks.summary().get("sm_max_mhz"))
     fma_peak = ffma_peak_tflops(local, clocks.summary().get("sm_max_mhz"))
-    total_k = sum(sum(v) for v in per_kernel.values())
-    kern = {}
-    for n, v in per_kernel.items():
-        avg_s = statistics.mean(v) / 1e3
-        bound, amount = kernel_work(n, cfg, pool_axis)
-        ent = {"launches_per_step": names.count(n), "us_per_step": avg_s * 1e6, "share": sum(v) / total_k,
-               "bound": bound}
-        if bound == "hbm":
-            ent.update(achieved=amount / avg_s / 1e9, unit="GB/s", frac=amount / avg_s / 1e9 / peak)
-        elif bound == "alu":
-            ent.update(achieved=amount / avg_s / 1e9, unit="G exp2/s", frac=amount / avg_s / 1e9 / mufu_peak)
-        elif bound == "fma":
-            ent.update(achieved=amount / avg_s / 1e12, unit="TFLOP/s fp32", frac=amount / avg_s / 1e12 / fma_peak)
-        kern[n] = ent
+    kern = summarize_kernels(per_kernel, names, cfg, pool_axis, peak, mufu_peak, fma_peak)
     dom = max((n for n in kern if n.startswith("bwd_")), key=lambda n: kern[n]["share"])
     dk = kern[dom]
     bound, amount = kernel_work(dom, cfg, pool_axis)

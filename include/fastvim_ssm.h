@@ -92,9 +92,10 @@ enum {
 };
 /* Without a PATH flag a dense layer whose images hold >= 16 MiB of x runs the fused launch, every
  * other layer the staged kernels; both compute the same layer.  The fused launch gates image b
- * L rounds after it pools it; the environment variable FASTVIM_FUSED_LAG (3..64, read per call)
- * overrides L, and FASTVIM_FUSED_LP (1..4) how many grid lines one streaming task covers (tuning
- * only). */
+ * L rounds after it pools it, L chosen from the layer's shape; the environment variable
+ * FASTVIM_FUSED_LAG (an integer 3..64, read by every call that takes the fused launch) replaces
+ * that choice.  It is a test hook: the tests run the schedule at its smallest safe lag (3) and at
+ * large ones; results do not depend on it.  No other environment variable is read. */
 
 typedef struct {
     int B, h, w, E, N, R;    /* batch, grid height/width, channels, d_state, dt_rank        */
@@ -176,19 +177,14 @@ FV_API const char* fastvim_ssm_launch_name(const fv_ssm_args* args, int i);
 
 /* The layer: queue pool -> projections -> scans -> repeat/skip/gate on `stream`.
  * ws: device workspace of at least fastvim_ssm_workspace_size(args) bytes, 256-byte aligned,
- * no initial contents required, not shared with a concurrently running call.
- * With FASTVIM_STAGED_CHUNKS = C > 1 (environment, tuning only; default 1) the staged kernels run
- * as C chunks of images in a pipeline: the projections and scans of one chunk go to a
- * high-priority stream the library keeps per device, in parallel with the pooling and epilogue
- * of its neighbours on `stream`; every piece of the call is ordered before the call's last
- * launch on `stream` (CUDA-graph capture follows the events). */
+ * no initial contents required, not shared with a concurrently running call.  Every launch of
+ * the call goes to `stream`, in order. */
 FV_API fv_status fastvim_ssm_forward(const fv_ssm_args* args, void* ws, size_t ws_bytes, void* stream);
 
 /* fastvim_ssm_forward with timing marks: `events` holds n_events >= 2 * launch_count CUDA
  * events (cudaEvent_t, created by the caller); events[2i] and events[2i+1] are recorded just
  * before and just after the i-th kernel launch, on the stream that launch runs on, so their
- * elapsed time is the device duration of launch i (launches of the staged kernels may overlap
- * one another on two streams).  Same results as fastvim_ssm_forward. */
+ * elapsed time is the device duration of launch i.  Same results as fastvim_ssm_forward. */
 FV_API fv_status fastvim_ssm_forward_events(const fv_ssm_args* args, void* ws, size_t ws_bytes,
                                             void* stream, void* const* events, int n_events);
 
@@ -208,20 +204,27 @@ FV_API fv_status fastvim_ssm_forward_host(const fv_ssm_args* host, const fv_ssm_
  * buffers for their inputs and outputs from a host framework that owns all device memory and
  * offers them no allocator, or must not call cudaMalloc/cudaFree because those calls can stall
  * the whole device.  This entry point needs no workspace argument: its scratch is a fixed
- * 16 MiB array in device memory that the library reserves on every GPU that loads it, held
- * until the process exits.
+ * 16 MiB array in device memory, part of this library's device code, held until the process
+ * exits.
  *   - Limit: fastvim_ssm_workspace_size(args) must be <= 16 MiB (e.g. the 224 px FastVim-T
- *     layer at batch 128: about 12 MiB); larger layers return FV_ERR_UNSUPPORTED with a message
- *     in fastvim_last_error() and queue nothing; split the batch or use fastvim_ssm_forward.
+ *     layer at batch 128 needs about 6 MiB); larger layers return FV_ERR_UNSUPPORTED with a
+ *     message in fastvim_last_error() and queue nothing; split the batch or use
+ *     fastvim_ssm_forward.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  *   - The first call on a device looks up that device's scratch address (with the device
- *     current); make that first call before any stream capture begins.
+ *     current).  CUDA loads the library's device code lazily, so this first call is also
+ *     where the 16 MiB are committed on that device: it can fail with FV_ERR_CUDA when the
+ *     device is out of memory.  Make that first call before any stream capture begins.
  *   - All calls on a device share the one scratch array: calls that may overlap on the GPU
- *     (different streams, no ordering between them) race and give wrong results.  Calls
- *     queued on one stream are ordered and safe.  The contents left by a previous call need
- *     no clearing.
+ *     (different streams, no ordering between them) race and give wrong results; on the
+ *     single-launch path one call's reset of the shared control block can also leave the
+ *     other call's blocks waiting until their bounded wait (1 s) runs out, and that timeout
+ *     is not reported (see below).  Calls queued on one stream are ordered and safe.  Each
+ *     call resets what must start at zero; the contents left by a previous call need no
+ *     clearing.
  *   - The device status word lives in the shared scratch and is not readable through this
- *     entry point; use fastvim_ssm_forward with a workspace where FV_ERR_INDEX must be seen.
+ *     entry point; use fastvim_ssm_forward with a workspace where FV_ERR_INDEX or
+ *     FV_ERR_TIMEOUT must be seen.
  * Inputs, outputs and the returned status are as for fastvim_ssm_forward. */
 FV_API fv_status fastvim_ssm_forward_noalloc(const fv_ssm_args* args, void* stream);
 

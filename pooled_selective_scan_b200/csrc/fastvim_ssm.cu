@@ -148,15 +148,10 @@ fv_status check_limits(const fv::Shape& sh) {
 // Grid lines per P/E task: the fewest that give each task at least 384 KB of x.  Every task costs
 // a ticket (a contended atomic, ~1 us under full HBM load), so fewer, larger streaming tasks pay:
 // B200, 2048 px layer, 2.17 -> 2.13 ms going from one 196 KB line to two per task.
-// FASTVIM_FUSED_LP (1..4) overrides it (tuning only).
 int fused_lines_per_task(const fv::Shape& sh) {
     const size_t line = (size_t)sh.S * sh.E * sizeof(float);
     int lp = 1;
     while (lp < fv::kMaxLP && lp < sh.T && (size_t)lp * line < ((size_t)384 << 10)) ++lp;
-    if (const char* env = getenv("FASTVIM_FUSED_LP")) {
-        const int v = atoi(env);
-        if (v >= 1 && v <= fv::kMaxLP) lp = v < sh.T ? v : sh.T;
-    }
     return lp;
 }
 
@@ -202,6 +197,8 @@ fv::FusedPlan plan_fused(const fv::Shape& sh) {
     // evicts first-touch lines whatever their L2 eviction priority.)
     const double round_us = (double)sh.h * sh.w * sh.E * 16.0 / 6.5e6;
     long long lag = (long long)(chain_latency_us(sh) / (round_us > 0.01 ? round_us : 0.01)) + 1;
+    // FASTVIM_FUSED_LAG replaces the choice (a test hook, declared in the header: the tests run
+    // the schedule at its smallest safe lag and at large ones)
     if (const char* env = getenv("FASTVIM_FUSED_LAG")) {
         const long long v = atoll(env);
         if (v >= 3 && v <= 64) lag = v;
@@ -272,27 +269,13 @@ struct EventMarks {
         }                                                      \
     } while (0)
 
-// Chunks of images the staged kernels run as (a pipeline over two streams, see forward_impl).
-// One by default: on B200 the overlap measured slower for every workload (e.g. the masked
-// 1024 px layer 0.58 -> 0.78 ms, the 1024 px layer 1.24 -> 1.37 ms with 4 chunks): the
-// long-lived projection and scan CTAs on the side stream hold SMs that the pooling and epilogue
-// kernels need to keep HBM saturated.  FASTVIM_STAGED_CHUNKS (1..8) sets it (tuning only).
-int staged_chunks(const fv::Shape& sh) {
-    int c = 1;
-    if (const char* env = getenv("FASTVIM_STAGED_CHUNKS")) {
-        const int v = atoi(env);
-        if (v >= 1 && v <= 8) c = v;
-    }
-    return sh.B < c ? (sh.B > 0 ? sh.B : 1) : c;
-}
-int staged_per_chunk(const fv::Shape& sh) { return sh.K > 0 ? 5 : 4; }
-
+// Launches of a staged call: pool (masked: bucket, pool), x_proj, scans, epilogue.
 int launch_count_of(const fv::Shape& sh) {
     if (sh.B == 0) return 0;
     const Path path = choose_path(sh);
     if (path == Path::Invalid) return 0;
     if (path == Path::Fused) return 1;
-    return staged_chunks(sh) * staged_per_chunk(sh);
+    return sh.K > 0 ? 5 : 4;
 }
 
 const char* launch_name_of(const fv::Shape& sh, int i) {
@@ -300,24 +283,11 @@ const char* launch_name_of(const fv::Shape& sh, int i) {
                                   "epilogue_dense_kernel"};
     static const char* masked[] = {"mask_bucket_kernel", "mask_pool_kernel", "proj_gemm_kernel", "scan_seq_kernel",
                                    "mask_epilogue_kernel"};
-    if (i < 0 || i >= launch_count_of(sh)) return "";
+    const int n = launch_count_of(sh);
+    if (i < 0 || i >= n) return "";
     if (choose_path(sh) == Path::Fused) return "fused_layer_kernel";
-    // Issue order: the front (pool) and middle (proj, scan) launches of chunk 0; then for each
-    // chunk c >= 1 its front and middle launches followed by the back (epilogue) launch of chunk
-    // c - 1; last the back launch of the last chunk.  k = position in a chunk's own list.
-    const int per = staged_per_chunk(sh), head = per - 1;
-    int k;
-    if (i == launch_count_of(sh) - 1) {
-        k = per - 1;
-    } else if (i < head) {
-        k = i;
-    } else {
-        const int r = (i - head) % per;
-        k = r < head ? r : per - 1;
-    }
-    const char* name = sh.K > 0 ? masked[k] : dense[k];
-    if (sh.ln && k == per - 1) name = "ln_epilogue_kernel";
-    return name;
+    if (sh.ln && i == n - 1) return "ln_epilogue_kernel";
+    return sh.K > 0 ? masked[i] : dense[i];
 }
 
 template <int ND, bool Z>
@@ -383,64 +353,16 @@ fv_status launch_scan_seq(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws
     return FV_OK;
 }
 
-// Workspace view of images [b0, ...) of a staged call: every per-image region is image-major.
-fv_ws_layout chunk_layout(const fv::Shape& sh, const fv_ws_layout& L, int b0) {
-    fv_ws_layout c = L;
-    c.xbar += (size_t)b0 * sh.T * sh.E * sizeof(float);
-    c.u += (size_t)b0 * sh.nd * fv::u_block_stride(sh.T, sh.J) * sizeof(float);
-    c.ys += (size_t)b0 * sh.T * sh.E * sizeof(float);
-    if (sh.K > 0) {
-        c.row_of += (size_t)b0 * sh.K * sizeof(int32_t);
-        c.row_off += (size_t)b0 * (sh.T + 1) * sizeof(int32_t);
-        c.row_tok += (size_t)b0 * sh.K * sizeof(int32_t);
-    }
-    return c;
-}
-
-// The high-priority stream on which the staged pipeline runs projections and scans, one per
-// device, created on first use and kept for the life of the process.
-cudaStream_t side_stream(fv_status* s) {
-    static std::mutex mu;
-    static cudaStream_t streams[64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess || dev < 0 || dev >= 64) {
-        note_cuda(e != cudaSuccess ? e : cudaErrorInvalidDevice, "side stream device");
-        *s = FV_ERR_CUDA;
-        return nullptr;
-    }
-    std::lock_guard<std::mutex> lock(mu);
-    if (!streams[dev]) {
-        int lo = 0, hi = 0;
-        if ((e = cudaDeviceGetStreamPriorityRange(&lo, &hi)) == cudaSuccess)
-            e = cudaStreamCreateWithPriority(&streams[dev], cudaStreamNonBlocking, hi);
-        if (e != cudaSuccess) {
-            note_cuda(e, "side stream");
-            streams[dev] = nullptr;
-            *s = FV_ERR_CUDA;
-            return nullptr;
-        }
-    }
-    return streams[dev];
-}
-
-// One chunk of a staged call: its shape, arguments and workspace view.
-struct StagedChunk {
-    fv::Shape sh;
-    fv_ssm_args a;
-    fv_ws_layout L;
-};
-
-// Front of a chunk: pooling (masked: bucketing of the kept ids, then pooling).
-fv_status staged_front(const StagedChunk& c, char* ws, unsigned* status, cudaStream_t st, EventMarks& marks) {
-    const fv::Shape& sh = c.sh;
+// Staged pooling (masked: bucketing of the kept ids, then pooling).
+fv_status staged_front(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, unsigned* status,
+                       cudaStream_t st, EventMarks& marks) {
     const int M = sh.B * sh.T;
-    float* xbar = (float*)(ws + c.L.xbar);
+    float* xbar = (float*)(ws + L.xbar);
     if (sh.K == 0) {
         FV_MARK_CALL(marks, st, ([&]() -> fv_status {
             // a whole number of token groups of SL threads each (no idle threads)
             const int threads = sh.SL <= fv::kThreads ? (fv::kThreads / sh.SL) * sh.SL : fv::kThreads;
-            fv::pool_dense_kernel<<<M, threads, 0, st>>>(sh, c.a.x, xbar);
+            fv::pool_dense_kernel<<<M, threads, 0, st>>>(sh, a->x, xbar);
             FV_LAUNCH_CHECK("pool_dense_kernel");
             return FV_OK;
         })());
@@ -450,15 +372,15 @@ fv_status staged_front(const StagedChunk& c, char* ws, unsigned* status, cudaStr
     cudaError_t e = ensure_smem(fv::mask_bucket_kernel, bsm);
     if (e != cudaSuccess) { note_cuda(e, "bucket smem attribute"); return FV_ERR_CUDA; }
     FV_MARK_CALL(marks, st, ([&]() -> fv_status {
-        fv::mask_bucket_kernel<<<sh.B, fv::kThreads, bsm, st>>>(sh, c.a.keep_idx, (int32_t*)(ws + c.L.row_of),
-                                                                (int32_t*)(ws + c.L.row_off),
-                                                                (int32_t*)(ws + c.L.row_tok), status);
+        fv::mask_bucket_kernel<<<sh.B, fv::kThreads, bsm, st>>>(sh, a->keep_idx, (int32_t*)(ws + L.row_of),
+                                                                (int32_t*)(ws + L.row_off),
+                                                                (int32_t*)(ws + L.row_tok), status);
         FV_LAUNCH_CHECK("mask_bucket_kernel");
         return FV_OK;
     })());
     FV_MARK_CALL(marks, st, ([&]() -> fv_status {
-        fv::mask_pool_kernel<<<M, fv::kThreads, 0, st>>>(sh, c.a.x, (const int32_t*)(ws + c.L.row_off),
-                                                         (const int32_t*)(ws + c.L.row_tok), xbar);
+        fv::mask_pool_kernel<<<M, fv::kThreads, 0, st>>>(sh, a->x, (const int32_t*)(ws + L.row_off),
+                                                         (const int32_t*)(ws + L.row_tok), xbar);
         FV_LAUNCH_CHECK("mask_pool_kernel");
         return FV_OK;
     })());
@@ -478,17 +400,18 @@ fv_status launch_proj_gemm(const fv::Shape& sh, const fv_ssm_args* a, const fv_w
     return FV_OK;
 }
 
-// Middle of a chunk: x_proj, then dt_proj + ZOH + scans.
-fv_status staged_middle(const StagedChunk& c, char* ws, cudaStream_t st, EventMarks& marks) {
-    FV_MARK_CALL(marks, st, launch_proj_gemm(c.sh, &c.a, c.L, ws, st));
-    FV_MARK_CALL(marks, st, launch_scan_seq(c.sh, &c.a, c.L, ws, st));
+// Staged x_proj, then dt_proj + ZOH + scans.
+fv_status staged_middle(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st,
+                        EventMarks& marks) {
+    FV_MARK_CALL(marks, st, launch_proj_gemm(sh, a, L, ws, st));
+    FV_MARK_CALL(marks, st, launch_scan_seq(sh, a, L, ws, st));
     return FV_OK;
 }
 
-// Back of a chunk: repeat + skip (+ LayerNorm) + gate.
-fv_status staged_back(const StagedChunk& c, char* ws, cudaStream_t st, EventMarks& marks) {
-    const fv::Shape& sh = c.sh;
-    const float* ys = (const float*)(ws + c.L.ys);
+// Staged repeat + skip (+ LayerNorm) + gate.
+fv_status staged_back(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st,
+                      EventMarks& marks) {
+    const float* ys = (const float*)(ws + L.ys);
     if (sh.ln) {
         const size_t smem = fv::ln_epilogue_smem_bytes(sh);
         cudaError_t e = ensure_smem(fv::ln_epilogue_kernel, smem);
@@ -499,14 +422,14 @@ fv_status staged_back(const StagedChunk& c, char* ws, cudaStream_t st, EventMark
         if (grid >= (1ll << 31)) return FV_ERR_UNSUPPORTED;
         FV_MARK_CALL(marks, st, ([&]() -> fv_status {
             fv::ln_epilogue_kernel<<<(unsigned)grid, fv::kLnWarps * 32, smem, st>>>(
-                sh, c.a.x, c.a.z, ys, c.a.D, c.a.ln_gamma, c.a.ln_beta,
-                sh.K > 0 ? (const int32_t*)(ws + c.L.row_of) : nullptr, c.a.y);
+                sh, a->x, a->z, ys, a->D, a->ln_gamma, a->ln_beta,
+                sh.K > 0 ? (const int32_t*)(ws + L.row_of) : nullptr, a->y);
             FV_LAUNCH_CHECK("ln_epilogue_kernel");
             return FV_OK;
         })());
     } else if (sh.K == 0) {
         FV_MARK_CALL(marks, st, ([&]() -> fv_status {
-            fv::epilogue_dense_kernel<<<sh.B * sh.T, fv::kThreads, 0, st>>>(sh, c.a.x, c.a.z, ys, c.a.D, c.a.y);
+            fv::epilogue_dense_kernel<<<sh.B * sh.T, fv::kThreads, 0, st>>>(sh, a->x, a->z, ys, a->D, a->y);
             FV_LAUNCH_CHECK("epilogue_dense_kernel");
             return FV_OK;
         })());
@@ -516,29 +439,14 @@ fv_status staged_back(const StagedChunk& c, char* ws, cudaStream_t st, EventMark
         cudaError_t e = ensure_smem(fv::mask_epilogue_kernel, msm);
         if (e != cudaSuccess) { note_cuda(e, "masked epilogue smem attribute"); return FV_ERR_CUDA; }
         FV_MARK_CALL(marks, st, ([&]() -> fv_status {
-            fv::mask_epilogue_kernel<<<sh.B * nkb, fv::kThreads, msm, st>>>(sh, c.a.x, c.a.z, ys, c.a.D,
-                                                                           (const int32_t*)(ws + c.L.row_of), c.a.y);
+            fv::mask_epilogue_kernel<<<sh.B * nkb, fv::kThreads, msm, st>>>(sh, a->x, a->z, ys, a->D,
+                                                                           (const int32_t*)(ws + L.row_of), a->y);
             FV_LAUNCH_CHECK("mask_epilogue_kernel");
             return FV_OK;
         })());
     }
     return FV_OK;
 }
-
-// Events of one staged call, destroyed when the call has queued its work.
-struct CallEvents {
-    std::vector<cudaEvent_t> ev;
-    ~CallEvents() {
-        for (cudaEvent_t e : ev)
-            if (e) cudaEventDestroy(e);
-    }
-    cudaEvent_t make() {
-        cudaEvent_t e = nullptr;
-        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) e = nullptr;
-        ev.push_back(e);
-        return e;
-    }
-};
 
 fv_status forward_impl(const fv_ssm_args* a, void* ws_v, size_t ws_bytes, cudaStream_t st,
                        void* const* events = nullptr, int n_events = 0) {
@@ -567,58 +475,9 @@ fv_status forward_impl(const fv_ssm_args* a, void* ws_v, size_t ws_bytes, cudaSt
         return FV_OK;
     }
 
-    // Staged: chunks of images; front (pool) and back (epilogue) on the caller's stream in the
-    // order front 0, front 1, back 0, front 2, back 1, ..., back C-1, and each chunk's middle
-    // (projections, scans) on the side stream between its front and its back.
-    const int C = staged_chunks(sh);
-    const int per_img_tok = sh.K > 0 ? sh.K : sh.h * sh.w;
-    std::vector<StagedChunk> ch(C);
-    const int base = sh.B / C, extra = sh.B % C;
-    for (int c = 0, b0 = 0; c < C; ++c) {
-        const int nb = base + (c < extra ? 1 : 0);
-        StagedChunk& k = ch[c];
-        k.sh = sh;
-        k.sh.B = nb;
-        k.a = *a;
-        k.a.B = nb;
-        const size_t off = (size_t)b0 * per_img_tok * sh.E;
-        k.a.x = a->x + off;
-        k.a.z = a->z + off;
-        k.a.y = a->y + off;
-        if (sh.K > 0) k.a.keep_idx = a->keep_idx + (size_t)b0 * sh.K;
-        k.L = chunk_layout(sh, L, b0);
-        b0 += nb;
-    }
-    if (C == 1) {
-        if ((s = staged_front(ch[0], ws, status, st, marks)) != FV_OK) return s;
-        if ((s = staged_middle(ch[0], ws, st, marks)) != FV_OK) return s;
-        return staged_back(ch[0], ws, st, marks);
-    }
-    cudaStream_t side = side_stream(&s);
-    if (!side) return s;
-    CallEvents evs;
-    std::vector<cudaEvent_t> front_done(C), middle_done(C);
-    for (int c = 0; c < C; ++c) {
-        front_done[c] = evs.make();
-        middle_done[c] = evs.make();
-        if (!front_done[c] || !middle_done[c]) { note_cuda(cudaErrorMemoryAllocation, "pipeline events"); return FV_ERR_CUDA; }
-    }
-    for (int c = 0; c < C; ++c) {
-        if ((s = staged_front(ch[c], ws, status, st, marks)) != FV_OK) return s;
-        if ((e = cudaEventRecord(front_done[c], st)) != cudaSuccess ||
-            (e = cudaStreamWaitEvent(side, front_done[c], 0)) != cudaSuccess) {
-            note_cuda(e, "pipeline fork");
-            return FV_ERR_CUDA;
-        }
-        if ((s = staged_middle(ch[c], ws, side, marks)) != FV_OK) return s;
-        if ((e = cudaEventRecord(middle_done[c], side)) != cudaSuccess) { note_cuda(e, "pipeline event"); return FV_ERR_CUDA; }
-        if (c >= 1) {
-            if ((e = cudaStreamWaitEvent(st, middle_done[c - 1], 0)) != cudaSuccess) { note_cuda(e, "pipeline join"); return FV_ERR_CUDA; }
-            if ((s = staged_back(ch[c - 1], ws, st, marks)) != FV_OK) return s;
-        }
-    }
-    if ((e = cudaStreamWaitEvent(st, middle_done[C - 1], 0)) != cudaSuccess) { note_cuda(e, "pipeline join"); return FV_ERR_CUDA; }
-    return staged_back(ch[C - 1], ws, st, marks);
+    if ((s = staged_front(sh, a, L, ws, status, st, marks)) != FV_OK) return s;
+    if ((s = staged_middle(sh, a, L, ws, st, marks)) != FV_OK) return s;
+    return staged_back(sh, a, L, ws, st, marks);
 }
 
 }  // namespace
@@ -864,7 +723,8 @@ fv_status fastvim_get_device_status(const void* ws, void* stream) {
 // ------------------------------------------------------------------------------------------------
 namespace {
 
-// 16 MiB, reserved on every GPU that loads this library, for as long as the process lives.
+// 16 MiB of device memory on every GPU where this library's device code is loaded (CUDA loads it
+// lazily, at the first symbol lookup or launch on that device), held until the process exits.
 constexpr size_t kStaticScratchBytes = (size_t)16 << 20;
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
@@ -978,16 +838,10 @@ fv_status check_grads(const fv_ssm_args* a, const fv::Shape& sh, const fv_ssm_gr
     return FV_OK;
 }
 
-// Tokens in flight per thread of the dense gate gradient: 2 (default) or 4; FASTVIM_BWD_GATE_UNROLL
-// overrides it (tuning only).  B200, 2048 px layer: 2 tokens (64 registers, 30 warps per SM)
-// stream at 0.945 of the copy rate, 4 tokens (99 registers, 18 warps) at 0.79.
-int bwd_gate_unroll() {
-    if (const char* env = getenv("FASTVIM_BWD_GATE_UNROLL")) {
-        const int v = atoi(env);
-        if (v == 2 || v == 4) return v;
-    }
-    return 2;
-}
+// Tokens in flight per thread of the dense gate gradient.  B200, 2048 px layer: 2 tokens (64
+// registers, 30 warps per SM) stream at 0.945 of the copy rate, 4 tokens (99 registers, 18 warps)
+// at 0.79.
+constexpr int kBwdGateTokens = 2;
 
 int device_sm_count() {
     int dev = 0, sms = 0;
@@ -1114,15 +968,10 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
         })());
     } else if (sh.K == 0) {
         const int threads = fv::bwd_groups(sh.SL) * fv::bwd_slot_width(sh.SL);
-        const bool u4 = bwd_gate_unroll() == 4;
-        const int grid = u4 ? resident(fv::bwd_gate_dense_kernel<4>, threads) : resident(fv::bwd_gate_dense_kernel<2>, threads);
+        auto kern = fv::bwd_gate_dense_kernel<kBwdGateTokens>;
+        const int grid = resident(kern, threads);
         FV_MARK_CALL(marks, st, ([&]() -> fv_status {
-            if (u4)
-                fv::bwd_gate_dense_kernel<4><<<grid, threads, 0, st>>>(sh, a->x, a->z, g->dy, ys, a->D, g->dx, g->dz,
-                                                                         dys, g->dD);
-            else
-                fv::bwd_gate_dense_kernel<2><<<grid, threads, 0, st>>>(sh, a->x, a->z, g->dy, ys, a->D, g->dx, g->dz,
-                                                                         dys, g->dD);
+            kern<<<grid, threads, 0, st>>>(sh, a->x, a->z, g->dy, ys, a->D, g->dx, g->dz, dys, g->dD);
             FV_LAUNCH_CHECK("bwd_gate_dense_kernel");
             return FV_OK;
         })());

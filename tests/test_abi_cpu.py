@@ -225,9 +225,8 @@ def test_layernorm_launches(lib):
     assert lib.fastvim_ssm_launch_count(ctypes.byref(big)) == 1  # the fused launch does it in its gate tasks
 
 
-@pytest.mark.parametrize("chunks,masked,ln", [(1, False, False), (3, False, True), (4, True, False), (2, True, True)])
-def test_staged_chunk_launch_order(lib, monkeypatch, chunks, masked, ln):
-    monkeypatch.setenv("FASTVIM_STAGED_CHUNKS", str(chunks))
+@pytest.mark.parametrize("masked,ln", [(False, False), (False, True), (True, False), (True, True)])
+def test_staged_launch_order(lib, masked, ln):
     kw = dict(B=5, flags=2)
     if masked:
         kw.update(K=49, keep_idx=FAKE + (9 << 32))
@@ -237,9 +236,6 @@ def test_staged_chunk_launch_order(lib, monkeypatch, chunks, masked, ln):
     front = ["mask_bucket_kernel", "mask_pool_kernel"] if masked else ["pool_dense_kernel"]
     middle = ["proj_gemm_kernel", "scan_seq_kernel"]
     back = ["ln_epilogue_kernel" if ln else ("mask_epilogue_kernel" if masked else "epilogue_dense_kernel")]
-    want = front + middle
-    for c in range(1, chunks):
-        want += front + middle + back
-    want += back
+    want = front + middle + back
     n = lib.fastvim_ssm_launch_count(ctypes.byref(a))
     assert [lib.fastvim_ssm_launch_name(ctypes.byref(a), i).decode() for i in range(n)] == want

@@ -82,3 +82,15 @@ def test_flags():
         bench.parse(["--warmup", "2"])
     with pytest.raises(SystemExit):
         bench.parse(["--steps", "0"])
+
+
+def test_secondary_workloads_cover_every_config_and_axis():
+    """The default run times every workload of the efficiency study: the headline and, under
+    'configs', each other config on each of its pool axes."""
+    from pooled_selective_scan_b200.configs import by_name
+    want = {(c.name, ax) for c in CONFIGS for ax in c.pool_axes} - {(bench.HEADLINE_NAME, 0)}
+    assert set(bench.SECONDARY) == want
+    for name, axis in bench.SECONDARY:
+        assert axis in by_name(name).pool_axes
+    assert bench.parse(["--no-configs"]).no_configs
+    assert not bench.parse([]).no_configs

@@ -294,3 +294,28 @@ def test_masked_largest_grid():
                                        keep_idx=p["keep_idx"], h=1024, w=1024)
     assert np.array_equal(got["row_of"], ref["row_of"])
     assert_close(got["y"], ref["y"])
+
+
+def test_events_bracket_every_staged_launch():
+    """fastvim_ssm_forward_events records a start and an end event around each launch; every
+    bracket has a positive duration and the result still matches the oracle."""
+    from pooled_selective_scan_b200 import ssm, workload
+    from pooled_selective_scan_b200.configs import by_name
+    cfg = by_name("fastvim_t_224")
+    dev = torch.device("cuda")
+    t = workload.layer_tensors(cfg, dev)
+    shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], 0, 3, path="staged")
+    y = torch.empty_like(t["x"])
+    ws = ssm.alloc_workspace(shape, dev)
+    fwd = ssm.BoundForward(shape, t, y, ws)
+    n = fwd.n_launch
+    assert n == 4
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n)]
+    fwd.run_events(evs)
+    torch.cuda.synchronize()
+    assert ssm.device_status(ws) == 0
+    d = [evs[2 * i].elapsed_time(evs[2 * i + 1]) for i in range(n)]
+    assert all(v > 0 for v in d)
+    ref = oracle.forward(*(t[k][:4].cpu().numpy() if k in ("x", "z") else t[k].cpu().numpy()
+                           for k in ("x", "z", "A_log", "D", "W_x", "W_dt", "b_dt")), 0, 3)
+    assert_close(y[:4].cpu().numpy(), ref)

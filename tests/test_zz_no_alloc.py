@@ -3,10 +3,12 @@ their input and output buffers by a host framework and have no way to allocate d
 (or must not, since cudaMalloc/cudaFree can stall the device).  It runs the same layer with its
 scratch in a fixed 16 MiB static device array instead of a caller workspace.
 
-Checked through the C ABI: two calls in a row (different layers, so the second runs on the
-scratch the first left behind) each match fastvim_ssm_forward with a caller workspace, within
-the layer's tolerance; a layer whose scratch would exceed 16 MiB is refused with
-FV_ERR_UNSUPPORTED and queues nothing.  This file is collected last on purpose."""
+Checked through the C ABI: three calls in a row (different layers, so each later call runs on
+the scratch the one before left behind: the staged kernels on a dense layer, then on a masked
+layer, then the single persistent launch, whose control block must be reset by the call itself)
+each match fastvim_ssm_forward with a caller workspace and the fp64 oracle, within the layer's
+tolerance; a layer whose scratch would exceed 16 MiB is refused with FV_ERR_UNSUPPORTED and
+queues nothing.  This file is collected last on purpose."""
 import ctypes
 
 import numpy as np
@@ -14,6 +16,7 @@ import pytest
 
 torch = pytest.importorskip("torch")
 
+import oracle  # noqa: E402
 from fv_testlib import assert_close  # noqa: E402
 from pooled_selective_scan_b200 import _native as nat  # noqa: E402
 from pooled_selective_scan_b200 import inputs, ssm  # noqa: E402
@@ -37,9 +40,9 @@ def _layer(seed, B, h, w, E, R, K=0):
     return {k: torch.from_numpy(v).to(dev) for k, v in d.items()}
 
 
-def _both_entry_points(t, pool_axis, h, w):
+def _both_entry_points(t, pool_axis, h, w, path="auto"):
     keep = t.get("keep_idx")
-    shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, 3, keep, h, w)
+    shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, 3, keep, h, w, path=path)
     assert ssm.workspace_size(shape) <= STATIC_SCRATCH_BYTES
     y_ref = torch.full_like(t["x"], float("nan"))
     y_new = torch.full_like(t["x"], float("nan"))
@@ -52,19 +55,40 @@ def _both_entry_points(t, pool_axis, h, w):
                                       ctypes.c_size_t(ws.numel()), stream), "fastvim_ssm_forward")
     nat.check(lib.fastvim_ssm_forward_noalloc(ctypes.byref(a_new), stream), "fastvim_ssm_forward_noalloc")
     torch.cuda.synchronize()
-    return y_new.cpu().numpy(), y_ref.cpu().numpy()
+    assert ssm.device_status(ws) == 0
+    return y_new.cpu().numpy(), y_ref.cpu().numpy(), ssm.launch_names(shape)
 
 
-def test_noalloc_matches_workspace_entry_point_twice_in_a_row():
+def _oracle(t, pool_axis, h, w, images):
+    """The fp64 oracle on the given images of the layer (inputs copied back from the device)."""
+    g = {k: v.cpu().numpy() for k, v in t.items()}
+    keep = g.get("keep_idx")
+    return oracle.forward(g["x"][images], g["z"][images], g["A_log"], g["D"], g["W_x"], g["W_dt"], g["b_dt"],
+                          pool_axis, 3, keep_idx=None if keep is None else keep[images], h=h, w=w,
+                          nthreads=len(images))
+
+
+def test_noalloc_matches_workspace_entry_point_and_oracle_three_times_in_a_row():
     cfg = CONFIGS[1]  # FastVim-T layer, 224 px, batch 128 (about 6 MiB of scratch)
     first = _layer(1, B=cfg.B, h=cfg.h, w=cfg.w, E=cfg.E, R=cfg.R)
     second = _layer(2, B=8, h=12, w=10, E=96, R=6, K=70)  # a masked layer of another shape
-    y_new, y_ref = _both_entry_points(first, 1, cfg.h, cfg.w)
+    third = _layer(5, B=3, h=40, w=36, E=136, R=6)  # dense, forced onto the single persistent launch
+    y_new, y_ref, names = _both_entry_points(first, 1, cfg.h, cfg.w)
+    assert names[0] == "pool_dense_kernel"
     assert np.isfinite(y_new).all()
     assert_close(y_new, y_ref, "first call")
-    y_new, y_ref = _both_entry_points(second, 0, 12, 10)
+    sample = [0, cfg.B // 2, cfg.B - 1]
+    assert_close(y_new[sample], _oracle(first, 1, cfg.h, cfg.w, sample), "first call vs oracle")
+    y_new, y_ref, names = _both_entry_points(second, 0, 12, 10)
+    assert names[0] == "mask_bucket_kernel"
     assert np.isfinite(y_new).all()
     assert_close(y_new, y_ref, "second call")
+    assert_close(y_new, _oracle(second, 0, 12, 10, list(range(8))), "second call vs oracle")
+    y_new, y_ref, names = _both_entry_points(third, 0, 40, 36, path="fused")
+    assert names == ["fused_layer_kernel"]
+    assert np.isfinite(y_new).all()
+    assert_close(y_new, y_ref, "third call")
+    assert_close(y_new, _oracle(third, 0, 40, 36, [0, 1, 2]), "third call vs oracle")
 
 
 def test_noalloc_refuses_layers_beyond_the_static_scratch():
