@@ -63,6 +63,11 @@ def _load():
                 "fvo_forward": [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, U, Dbl, I, P, P, Dbl, I, P],
                 "fvo_backward": [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, U, Dbl, I, P, P, Dbl, P, I,
                                  P, P, P, P, P, P, P, P, P],
+                "fvo_conv": [P, I, I, I, I, I, U, I, P, P, I, P],
+                "fvo_pool_d": [P, I, I, I, I, I, Dbl, P],
+                "fvo_gate_dense_conv": [P, P, P, P, I, I, I, I, I, I, P, P, Dbl, P],
+                "fvo_forward_conv": [P, P, P, P, P, P, P, I, I, I, I, I, I, I, U, Dbl, I, I, P, P, I, P, P, Dbl, I,
+                                     P],
             }
             for name, argtypes in sigs.items():
                 fn = getattr(lib, name)
@@ -212,19 +217,69 @@ def gate_masked(x, z, ys, D, row_of, ln_gamma=None, ln_beta=None, ln_eps=1e-5):
     return y
 
 
+def conv(x, conv_w, conv_b, pool_axis, dir_flags, conv_silu=False):
+    """The block's Conv1D, one filter per direction slot: x [B,h,w,E], conv_w [nd,E,dc],
+    conv_b [nd,E] -> xc [nd,B,h,w,E] (fp64)."""
+    x, conv_w, conv_b = _f32(x), _f32(conv_w), _f32(conv_b)
+    B, h, w, E = x.shape
+    nd, E2, dc = conv_w.shape
+    assert E2 == E and conv_b.shape == (nd, E) and nd == nd_of(dir_flags)
+    xc = np.empty((nd, B, h, w, E), np.float64)
+    st = _load().fvo_conv(_p(x), B, h, w, E, pool_axis, int(dir_flags), dc, _p(conv_w), _p(conv_b),
+                          int(bool(conv_silu)), _p(xc))
+    _check(st, "conv")
+    return xc
+
+
+def pool_d(x, pool_axis, pool_scale=1.0):
+    """Mean pooling of an fp64 grid x [B,h,w,E] -> xbar [B,T,E]."""
+    x = _f64(x)
+    B, h, w, E = x.shape
+    out = np.empty((B, pooled_len(h, w, pool_axis), E), np.float64)
+    _check(_load().fvo_pool_d(_p(x), B, h, w, E, pool_axis, float(pool_scale), _p(out)), "pool_d")
+    return out
+
+
+def gate_dense_conv(xc, z, ys, D, pool_axis, ln_gamma=None, ln_beta=None, ln_eps=1e-5):
+    """Repeat + skip with each direction's convolved input (+ LayerNorm) + gate -> y [B,h,w,E]."""
+    xc, ys = _f64(xc), _f64(ys)
+    z, D = _f32(z), _f32(D)
+    nd, B, h, w, E = xc.shape
+    g, b = _ln(ln_gamma, ln_beta, E)
+    y = np.empty(z.shape, np.float64)
+    st = _load().fvo_gate_dense_conv(_p(xc), _p(z), _p(ys), _p(D), B, h, w, E, nd, pool_axis, _p(g), _p(b),
+                                     float(ln_eps), _p(y))
+    _check(st, "gate_dense_conv")
+    return y
+
+
 def forward(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis, dir_flags, keep_idx=None, h=None,
             w=None, pool_scale=1.0, zoh_exact=False, nthreads=1, allow_bad_index=False, ln_gamma=None,
-            ln_beta=None, ln_eps=1e-5):
+            ln_beta=None, ln_eps=1e-5, conv_w=None, conv_b=None, conv_silu=False):
     """The whole layer, image by image.
 
     Dense: x, z [B,h,w,E] -> y [B,h,w,E].  Masked: x, z [B,K,E], keep_idx [B,K] with the grid
     given by h, w -> y [B,K,E].  Returns fp64 y (and the status when allow_bad_index is set).
+    With conv_w [nd,E,dc] and conv_b [nd,E] (dense only) x is the input of the block's Conv1D.
     """
     x, z = _f32(x), _f32(z)
     A_log, D, W_x, W_dt, b_dt = map(_f32, (A_log, D, W_x, W_dt, b_dt))
     N = A_log.shape[2]
     E = A_log.shape[1]
     R = W_dt.shape[2]
+    if conv_w is not None or conv_b is not None:
+        assert keep_idx is None and conv_w is not None and conv_b is not None
+        cw, cb = _f32(conv_w), _f32(conv_b)
+        B, h, w, E2 = x.shape
+        assert E2 == E and z.shape == x.shape and cw.shape[:2] == (nd_of(dir_flags), E)
+        g, b = _ln(ln_gamma, ln_beta, E)
+        y = np.empty(x.shape, np.float64)
+        st = _load().fvo_forward_conv(_p(x), _p(z), _p(A_log), _p(D), _p(W_x), _p(W_dt), _p(b_dt), B, h, w, E, N, R,
+                                      pool_axis, int(dir_flags), float(pool_scale), int(bool(zoh_exact)),
+                                      cw.shape[2], _p(cw), _p(cb), int(bool(conv_silu)), _p(g), _p(b), float(ln_eps),
+                                      int(nthreads), _p(y))
+        _check(st, "forward_conv")
+        return (y, st) if allow_bad_index else y
     if keep_idx is None:
         B, h, w, E2 = x.shape
         K = 0
@@ -245,12 +300,32 @@ def forward(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis, dir_flags, keep_idx=None
 
 def forward_intermediates(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis, dir_flags, keep_idx=None,
                           h=None, w=None, pool_scale=1.0, zoh_exact=False, ln_gamma=None, ln_beta=None,
-                          ln_eps=1e-5):
-    """The same chain step by step, returning every intermediate as a dict (small sizes only)."""
+                          ln_eps=1e-5, conv_w=None, conv_b=None, conv_silu=False):
+    """The same chain step by step, returning every intermediate as a dict (small sizes only).
+    With the Conv1D (conv_w, conv_b) the per-direction intermediates are stacked: xc [nd,B,h,w,E],
+    xbar [B,nd,T,E] (each direction pools its own convolved tokens), u [nd,B,T,J], delta
+    [nd,B,T,E]."""
     A_log, W_dt = _f32(A_log), _f32(W_dt)
     N = A_log.shape[2]
     R = W_dt.shape[2]
     out = {}
+    if conv_w is not None:
+        assert keep_idx is None
+        W_x, b_dt = _f32(W_x), _f32(b_dt)
+        xc = conv(x, conv_w, conv_b, pool_axis, dir_flags, conv_silu)
+        dirs = [d for d in (FWD, BWD) if dir_flags & d]
+        xbars, us, deltas = [], [], []
+        ys = 0.0
+        for k, d in enumerate(dirs):
+            xb = pool_d(xc[k], pool_axis, pool_scale)
+            u, delta = proj(xb, W_x[k:k + 1], W_dt[k:k + 1], b_dt[k:k + 1], R, N)
+            ys = ys + scan(xb, delta, u, A_log[k:k + 1], R, N, d, zoh_exact)
+            xbars.append(xb)
+            us.append(u[0])
+            deltas.append(delta[0])
+        y = gate_dense_conv(xc, z, ys, D, pool_axis, ln_gamma, ln_beta, ln_eps)
+        out.update(xc=xc, xbar=np.stack(xbars, axis=1), u=np.stack(us), delta=np.stack(deltas), ys=ys, y=y)
+        return out
     if keep_idx is None:
         xbar = pool(x, pool_axis, pool_scale)
     else:

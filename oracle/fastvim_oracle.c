@@ -282,6 +282,189 @@ int fvo_gate_masked(const float* x, const float* z, const double* ys, const floa
     return FVO_OK;
 }
 
+/* ---- The block's Conv1D in front of the layer -------------------------------------------------
+ * gptget.net summary of 2502.00594, "方法详解" item 2: the tokens go through Norm, the expansion
+ * layer and a Conv1D, and the layer pools the Conv1D's output; ijyty.com Vision Mamba article,
+ * section 2.1 code: the forward and the backward SSM each take the output of their own Conv1D
+ * of the expanded tokens, the backward one run over the reversed sequence.
+ * Readings taken (the pages give no more):
+ *   - depthwise (one filter of dc taps and a bias per channel and direction), zero padding;
+ *   - the block's token sequence runs line by line along the pooled-over axis: position
+ *     p = t * S + s holds token (i, j) = (t, s) under POOL_W and (s, t) under POOL_H (the
+ *     transposed grid of an alternate block, flattened row by row), L = h * w positions;
+ *   - forward slot:  xc[p] = act(b + sum_{q<dc} w[q] x[p - (dc-1) + q])  (x = 0 before p = 0)
+ *     backward slot: xc[p] = act(b + sum_{q<dc} w[q] x[p + (dc-1) - q])  (x = 0 past L - 1),
+ *     i.e. the same causal filter run over the reversed sequence and reversed back;
+ *   - act is the identity, or SiLU when conv_silu is set (Mamba-family blocks follow the
+ *     Conv1D with SiLU; the pages do not say).
+ * Layouts: conv_w [nd][E][dc], conv_b [nd][E]; xc [nd][B][h][w][E] (the grid layout of x). */
+static void seq_token(int p, int h, int w, int pool_axis, int* i, int* j)
+{
+    const int S = pooled_over(h, w, pool_axis);
+    const int t = p / S, s = p % S;
+    *i = (pool_axis == FVO_POOL_W) ? t : s;
+    *j = (pool_axis == FVO_POOL_W) ? s : t;
+}
+
+int fvo_conv(const float* x, int B, int h, int w, int E, int pool_axis, unsigned dir_flags, int dc,
+             const float* conv_w, const float* conv_b, int conv_silu, double* xc)
+{
+    if (B < 0 || h <= 0 || w <= 0 || E <= 0 || dc < 1 || (dir_flags & ~3u) != 0 || dir_flags == 0 ||
+        (pool_axis != FVO_POOL_W && pool_axis != FVO_POOL_H))
+        return FVO_BAD_SHAPE;
+    const int L = h * w;
+    const size_t img = (size_t)L * E;
+    int k = 0;
+    for (unsigned dir = FVO_FWD; dir <= FVO_BWD; dir <<= 1) {
+        if (!(dir_flags & dir)) continue;
+        for (int b = 0; b < B; ++b)
+            for (int p = 0; p < L; ++p) {
+                int i, j;
+                seq_token(p, h, w, pool_axis, &i, &j);
+                for (int e = 0; e < E; ++e) {
+                    double acc = (double)conv_b[(size_t)k * E + e];
+                    for (int q = 0; q < dc; ++q) {
+                        const int pp = (dir == FVO_FWD) ? p - (dc - 1) + q : p + (dc - 1) - q;
+                        if (pp < 0 || pp >= L) continue;
+                        int ii, jj;
+                        seq_token(pp, h, w, pool_axis, &ii, &jj);
+                        acc += (double)conv_w[((size_t)k * E + e) * dc + q] *
+                               (double)x[(size_t)b * img + ((size_t)ii * w + jj) * E + e];
+                    }
+                    xc[((size_t)k * B + b) * img + ((size_t)i * w + j) * E + e] = conv_silu ? silu(acc) : acc;
+                }
+            }
+        ++k;
+    }
+    return FVO_OK;
+}
+
+/* Mean pooling (as fvo_pool) of a grid held in fp64: the convolved tokens. */
+int fvo_pool_d(const double* x, int B, int h, int w, int E, int pool_axis, double pool_scale, double* xbar)
+{
+    if (B < 0 || h <= 0 || w <= 0 || E <= 0 || (pool_axis != FVO_POOL_W && pool_axis != FVO_POOL_H))
+        return FVO_BAD_SHAPE;
+    const int T = pooled_len(h, w, pool_axis), S = pooled_over(h, w, pool_axis);
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t)
+            for (int e = 0; e < E; ++e) {
+                double acc = 0.0;
+                for (int s = 0; s < S; ++s) {
+                    const int i = (pool_axis == FVO_POOL_W) ? t : s;
+                    const int j = (pool_axis == FVO_POOL_W) ? s : t;
+                    acc += x[(((size_t)b * h + i) * w + j) * E + e];
+                }
+                xbar[((size_t)b * T + t) * E + e] = pool_scale * acc / (double)S;
+            }
+    return FVO_OK;
+}
+
+/* Repeat + skip (+ LayerNorm) + gate when every direction has its own convolved input:
+ *   y[b][i][j] = SiLU(z[b][i][j]) * N(ys[b][t(i,j)] + sum_k D[k] * xc[k][b][i][j]). */
+int fvo_gate_dense_conv(const double* xc, const float* z, const double* ys, const float* D, int B, int h,
+                        int w, int E, int nd, int pool_axis, const float* ln_gamma, const float* ln_beta,
+                        double ln_eps, double* y)
+{
+    if (B < 0 || h <= 0 || w <= 0 || E <= 0 || nd < 1 || nd > 2) return FVO_BAD_SHAPE;
+    if (!ln_args_ok(ln_gamma, ln_beta, ln_eps)) return FVO_BAD_SHAPE;
+    const int T = pooled_len(h, w, pool_axis);
+    const size_t all = (size_t)B * h * w * E;
+    double* tmp = (double*)malloc(sizeof(double) * (size_t)E);
+    if (!tmp) return FVO_NO_MEMORY;
+    for (int b = 0; b < B; ++b)
+        for (int i = 0; i < h; ++i)
+            for (int j = 0; j < w; ++j) {
+                const int t = (pool_axis == FVO_POOL_W) ? i : j;
+                const size_t g = (((size_t)b * h + i) * w + j) * E;
+                for (int e = 0; e < E; ++e) {
+                    double v = ys[((size_t)b * T + t) * E + e];
+                    for (int k = 0; k < nd; ++k) v += (double)D[(size_t)k * E + e] * xc[(size_t)k * all + g + e];
+                    tmp[e] = v;
+                }
+                if (ln_gamma) layernorm_row(tmp, E, ln_gamma, ln_beta, ln_eps);
+                for (int e = 0; e < E; ++e) y[g + e] = silu((double)z[g + e]) * tmp[e];
+            }
+    free(tmp);
+    return FVO_OK;
+}
+
+/* One image of the layer with the Conv1D in front: each direction slot k convolves x with its
+ * own filter, pools its own convolved tokens, projects and scans them with its own parameters;
+ * the scan outputs are summed and the skip adds each direction's D times its own convolved
+ * input.  Scratch: xc [nd][h][w][E], xbar [T][E], u [T][J], delta [T][E], ys and ysk [T][E]. */
+static int forward_one_conv(const float* x, const float* z, const float* A_log, const float* D,
+                            const float* W_x, const float* W_dt, const float* b_dt, int h, int w, int E,
+                            int N, int R, int pool_axis, unsigned dir_flags, double pool_scale, int zoh_exact,
+                            int dc, const float* conv_w, const float* conv_b, int conv_silu,
+                            const float* ln_gamma, const float* ln_beta, double ln_eps, double* y,
+                            double* xc, double* xbar, double* u, double* delta, double* ys, double* ysk)
+{
+    const int nd = popcount2(dir_flags);
+    const int T = pooled_len(h, w, pool_axis);
+    const int J = R + 2 * N;
+    const size_t img = (size_t)h * w * E;
+    int st = fvo_conv(x, 1, h, w, E, pool_axis, dir_flags, dc, conv_w, conv_b, conv_silu, xc);
+    if (st) return st;
+    for (size_t m = 0; m < (size_t)T * E; ++m) ys[m] = 0.0;
+    int k = 0;
+    for (unsigned dir = FVO_FWD; dir <= FVO_BWD; dir <<= 1) {
+        if (!(dir_flags & dir)) continue;
+        if ((st = fvo_pool_d(xc + (size_t)k * img, 1, h, w, E, pool_axis, pool_scale, xbar))) return st;
+        if ((st = fvo_proj(xbar, 1, T, E, 1, R, N, W_x + (size_t)k * J * E, W_dt + (size_t)k * E * R,
+                           b_dt + (size_t)k * E, u, delta)))
+            return st;
+        if ((st = fvo_scan(xbar, delta, u, A_log + (size_t)k * E * N, 1, T, E, 1, R, N, dir, zoh_exact, ysk)))
+            return st;
+        for (size_t m = 0; m < (size_t)T * E; ++m) ys[m] += ysk[m];
+        ++k;
+    }
+    return fvo_gate_dense_conv(xc, z, ys, D, 1, h, w, E, nd, pool_axis, ln_gamma, ln_beta, ln_eps, y);
+}
+
+int fvo_forward_conv(const float* x, const float* z, const float* A_log, const float* D,
+                     const float* W_x, const float* W_dt, const float* b_dt, int B, int h, int w, int E,
+                     int N, int R, int pool_axis, unsigned dir_flags, double pool_scale, int zoh_exact, int dc,
+                     const float* conv_w, const float* conv_b, int conv_silu, const float* ln_gamma,
+                     const float* ln_beta, double ln_eps, int nthreads, double* y)
+{
+    const int nd = popcount2(dir_flags);
+    if (B < 0 || h <= 0 || w <= 0 || E <= 0 || N <= 0 || R <= 0 || nd < 1 || dc < 1 ||
+        (dir_flags & ~3u) != 0 || (pool_axis != FVO_POOL_W && pool_axis != FVO_POOL_H) || !conv_w ||
+        !conv_b || !ln_args_ok(ln_gamma, ln_beta, ln_eps))
+        return FVO_BAD_SHAPE;
+    const int T = pooled_len(h, w, pool_axis);
+    const int J = R + 2 * N;
+    const size_t img = (size_t)h * w * E;
+    int status = FVO_OK;
+    if (nthreads < 1) nthreads = 1;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads) if (nthreads > 1)
+#endif
+    for (int b = 0; b < B; ++b) {
+        double* xc = (double*)malloc(sizeof(double) * (size_t)nd * img);
+        double* xbar = (double*)malloc(sizeof(double) * (size_t)T * E);
+        double* u = (double*)malloc(sizeof(double) * (size_t)T * J);
+        double* delta = (double*)malloc(sizeof(double) * (size_t)T * E);
+        double* ys = (double*)malloc(sizeof(double) * (size_t)T * E);
+        double* ysk = (double*)malloc(sizeof(double) * (size_t)T * E);
+        int st = FVO_NO_MEMORY;
+        if (xc && xbar && u && delta && ys && ysk)
+            st = forward_one_conv(x + (size_t)b * img, z + (size_t)b * img, A_log, D, W_x, W_dt, b_dt, h, w, E, N,
+                                  R, pool_axis, dir_flags, pool_scale, zoh_exact, dc, conv_w, conv_b, conv_silu,
+                                  ln_gamma, ln_beta, ln_eps, y + (size_t)b * img, xc, xbar, u, delta, ys, ysk);
+        free(xc); free(xbar); free(u); free(delta); free(ys); free(ysk);
+        if (st != FVO_OK) {
+#ifdef _OPENMP
+#pragma omp critical
+#endif
+            {
+                if (status == FVO_OK) status = st;
+            }
+        }
+    }
+    return status;
+}
+
 /* One image through the whole chain; scratch is owned by the caller. */
 static int forward_one(const float* x, const float* z, const float* A_log, const float* D,
                        const float* W_x, const float* W_dt, const float* b_dt,

@@ -84,6 +84,31 @@ int fvo_forward(const float* x, const float* z, const float* A_log, const float*
                 int pool_axis, unsigned dir_flags, double pool_scale, int zoh_exact,
                 const float* ln_gamma, const float* ln_beta, double ln_eps, int nthreads, double* y);
 
+/* The block's Conv1D in front of the layer (depthwise, dc taps, zero padding), one filter per
+ * direction slot: conv_w [nd][E][dc], conv_b [nd][E]; the sequence runs line by line along the
+ * pooled-over axis (position t*S + s); the forward slot's filter is causal, the backward slot's
+ * runs over the reversed sequence; SiLU after it when conv_silu.  xc [nd][B][h][w][E]. */
+int fvo_conv(const float* x, int B, int h, int w, int E, int pool_axis, unsigned dir_flags, int dc,
+             const float* conv_w, const float* conv_b, int conv_silu, double* xc);
+
+/* Mean pooling of an fp64 grid [B][h][w][E] (the convolved tokens of one direction). */
+int fvo_pool_d(const double* x, int B, int h, int w, int E, int pool_axis, double pool_scale, double* xbar);
+
+/* Repeat + skip (+ LayerNorm) + gate with a convolved input per direction:
+ * y = SiLU(z) * N(ys[t] + sum_k D[k] * xc[k]), xc [nd][B][h][w][E]. */
+int fvo_gate_dense_conv(const double* xc, const float* z, const double* ys, const float* D, int B, int h,
+                        int w, int E, int nd, int pool_axis, const float* ln_gamma, const float* ln_beta,
+                        double ln_eps, double* y);
+
+/* The whole dense layer with the Conv1D in front: x is the Conv1D's input; each direction
+ * pools, projects and scans its own convolved tokens, and the skip adds each direction's D
+ * times its own convolved input (OpenMP over images when nthreads > 1). */
+int fvo_forward_conv(const float* x, const float* z, const float* A_log, const float* D,
+                     const float* W_x, const float* W_dt, const float* b_dt, int B, int h, int w, int E,
+                     int N, int R, int pool_axis, unsigned dir_flags, double pool_scale, int zoh_exact, int dc,
+                     const float* conv_w, const float* conv_b, int conv_silu, const float* ln_gamma,
+                     const float* ln_beta, double ln_eps, int nthreads, double* y);
+
 /* The gradient of the layer (fastvim_oracle_grad.c): given dy = dL/dy (layout of y), writes
  * dx, dz (layouts of x, z) and the parameter gradients summed over the batch, dA_log [nd][E][N],
  * dD [nd][E], dW_x [nd][R+2N][E], dW_dt [nd][E][R], db_dt [nd][E]; with the post-SSM LayerNorm

@@ -45,6 +45,18 @@ MUTATIONS = {
     "LayerNorm after the gate": ("    if (ln_gamma) layernorm_row(tmp, E, ln_gamma, ln_beta, ln_eps);\n    for (int e = 0; e < E; ++e) y[e] = silu((double)z[e]) * tmp[e];",
                                  "    for (int e = 0; e < E; ++e) tmp[e] *= silu((double)z[e]);\n"
                                  "    if (ln_gamma) layernorm_row(tmp, E, ln_gamma, ln_beta, ln_eps);\n    for (int e = 0; e < E; ++e) y[e] = tmp[e];"),
+    "conv taps reversed": ("(double)conv_w[((size_t)k * E + e) * dc + q]", "(double)conv_w[((size_t)k * E + e) * dc + (dc - 1 - q)]"),
+    "conv filter of slot 0 for both directions": ("(double)conv_w[((size_t)k * E + e) * dc + q]",
+                                                  "(double)conv_w[((size_t)0 * E + e) * dc + q]"),
+    "backward conv causal too": ("(dir == FVO_FWD) ? p - (dc - 1) + q : p + (dc - 1) - q", "p - (dc - 1) + q"),
+    "conv sequence row-major on both axes": ("const int t = p / S, s = p % S;\n    *i = (pool_axis == FVO_POOL_W) ? t : s;\n    *j = (pool_axis == FVO_POOL_W) ? s : t;",
+                                             "(void)S;\n    *i = p / w;\n    *j = p % w;"),
+    "conv bias dropped": ("double acc = (double)conv_b[(size_t)k * E + e];", "double acc = 0.0;"),
+    "conv padding wraps around": ("const int pp = (dir == FVO_FWD) ? p - (dc - 1) + q : p + (dc - 1) - q;",
+                                  "const int pp = (((dir == FVO_FWD) ? p - (dc - 1) + q : p + (dc - 1) - q) + L) % L;"),
+    "conv skip from the forward slot only": ("v += (double)D[(size_t)k * E + e] * xc[(size_t)k * all + g + e];",
+                                             "v += (double)D[(size_t)k * E + e] * xc[g + e];"),
+    "both directions pool the forward convolved tokens": ("fvo_pool_d(xc + (size_t)k * img, 1,", "fvo_pool_d(xc, 1,"),
     "pool scale ignored": ("pool_scale * acc / (double)S;\n            }\n    return FVO_OK;\n}\n\n/* Row of",
                            "acc / (double)S;\n            }\n    return FVO_OK;\n}\n\n/* Row of"),
 }

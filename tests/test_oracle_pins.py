@@ -505,3 +505,157 @@ def test_p9_layernorm_arguments(oracle_mod):
         oracle_mod.forward(**a, ln_gamma=gamma, ln_beta=None)
     with pytest.raises(oracle_mod.OracleError):
         oracle_mod.forward(**a, ln_gamma=gamma, ln_beta=beta, ln_eps=-1.0)
+
+
+# ---------------------------------------------------------------------------------------------
+# p10: the block's Conv1D in front of the layer (per-direction depthwise filters along the
+# block's sequence, which runs line by line along the pooled-over axis).
+# ---------------------------------------------------------------------------------------------
+def _seq(x, pool_axis):
+    """Grid [B,h,w,E] -> the block's sequence [B,L,E]: lines t in order, tokens s along each line."""
+    return (x if pool_axis == 0 else x.transpose(0, 2, 1, 3)).reshape(x.shape[0], -1, x.shape[-1])
+
+
+def _unseq(s, h, w, pool_axis):
+    B, L, E = s.shape
+    return s.reshape(B, h, w, E) if pool_axis == 0 else s.reshape(B, w, h, E).transpose(0, 2, 1, 3)
+
+
+def _torch_conv(x, conv_w, conv_b, pool_axis, dir_flags, silu):
+    """Reference Conv1D through torch.nn.functional.conv1d (fp64, groups = E, zero padding, the
+    first L outputs: causal); the backward slot runs the same filter on the reversed sequence."""
+    torch = pytest.importorskip("torch")
+    B, h, w, E = x.shape
+    dc = conv_w.shape[2]
+    seq = torch.from_numpy(_seq(x.astype(np.float64), pool_axis)).permute(0, 2, 1)  # [B,E,L]
+    outs = []
+    dirs = [d for d in (1, 2) if dir_flags & d]
+    for k, d in enumerate(dirs):
+        wt = torch.from_numpy(conv_w[k].astype(np.float64))[:, None, :]
+        bt = torch.from_numpy(conv_b[k].astype(np.float64))
+        inp = seq if d == 1 else seq.flip(-1)
+        o = torch.nn.functional.conv1d(inp, wt, bt, padding=dc - 1, groups=E)[..., :h * w]
+        if d == 2:
+            o = o.flip(-1)
+        if silu:
+            o = torch.nn.functional.silu(o)
+        outs.append(_unseq(o.permute(0, 2, 1).numpy(), h, w, pool_axis))
+    return np.stack(outs)
+
+
+def _conv_case(rng, B=2, h=3, w=5, E=6, dc=4, nd=2):
+    x = rng.standard_normal((B, h, w, E)).astype(np.float32)
+    cw = rng.uniform(-1, 1, size=(nd, E, dc)).astype(np.float32)
+    cb = rng.uniform(-0.5, 0.5, size=(nd, E)).astype(np.float32)
+    return x, cw, cb
+
+
+@pytest.mark.parametrize("pool_axis", [0, 1])
+@pytest.mark.parametrize("dc,silu", [(1, False), (2, False), (4, False), (4, True), (3, True)])
+def test_p10_conv_matches_torch_conv1d(oracle_mod, pool_axis, dc, silu):
+    rng = np.random.default_rng(1000 + 10 * dc + 2 * pool_axis + silu)
+    x, cw, cb = _conv_case(rng, dc=dc)
+    got = oracle_mod.conv(x, cw, cb, pool_axis, 3, silu)
+    ref = _torch_conv(x, cw, cb, pool_axis, 3, silu)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-13)
+    # one direction alone takes its own filter slot 0
+    got_b = oracle_mod.conv(x, cw[1:], cb[1:], pool_axis, 2, silu)
+    np.testing.assert_allclose(got_b[0], ref[1], rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("pool_axis", [0, 1])
+def test_p10_conv_identity_and_one_step_shift(oracle_mod, pool_axis):
+    rng = np.random.default_rng(1100 + pool_axis)
+    B, h, w, E, dc = 2, 4, 3, 5, 4
+    x, _, _ = _conv_case(rng, B, h, w, E, dc)
+    zero_b = np.zeros((2, E), np.float32)
+    ident = np.zeros((2, E, dc), np.float32)
+    ident[..., dc - 1] = 1.0
+    np.testing.assert_array_equal(oracle_mod.conv(x, ident, zero_b, pool_axis, 3), np.stack([x, x]).astype(np.float64))
+    shift = np.zeros((2, E, dc), np.float32)
+    shift[..., dc - 2] = 1.0
+    xc = oracle_mod.conv(x, shift, zero_b, pool_axis, 3)
+    s = _seq(x.astype(np.float64), pool_axis)
+    prev = np.concatenate([np.zeros_like(s[:, :1]), s[:, :-1]], axis=1)  # forward: the token one step back
+    nxt = np.concatenate([s[:, 1:], np.zeros_like(s[:, :1])], axis=1)    # backward: one step ahead
+    np.testing.assert_array_equal(xc[0], _unseq(prev, h, w, pool_axis))
+    np.testing.assert_array_equal(xc[1], _unseq(nxt, h, w, pool_axis))
+    # bias only: a constant (SiLU of it) everywhere
+    xb = oracle_mod.conv(np.zeros_like(x), shift, np.full((2, E), 0.75, np.float32), pool_axis, 3, True)
+    np.testing.assert_allclose(xb, 0.75 / (1 + math.exp(-0.75)), rtol=1e-15)
+
+
+@pytest.mark.parametrize("pool_axis", [0, 1])
+@pytest.mark.parametrize("dir_flags", [1, 2, 3])
+def test_p10_identity_conv_layer_is_the_plain_layer(oracle_mod, pool_axis, dir_flags):
+    rng = np.random.default_rng(1200 + 3 * pool_axis + dir_flags)
+    B, h, w, E, N, R = 2, 3, 4, 5, 3, 2
+    nd = oracle_mod.nd_of(dir_flags)
+    A_log, D, W_x, W_dt, b_dt = _rand_params(rng, nd, E, N, R)
+    x = rng.standard_normal((B, h, w, E)).astype(np.float32)
+    z = rng.standard_normal((B, h, w, E)).astype(np.float32)
+    ident = np.zeros((nd, E, 4), np.float32)
+    ident[..., 3] = 1.0
+    plain = oracle_mod.forward(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis, dir_flags)
+    conv = oracle_mod.forward(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis, dir_flags, conv_w=ident,
+                              conv_b=np.zeros((nd, E), np.float32))
+    np.testing.assert_allclose(conv, plain, rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("pool_axis", [0, 1])
+@pytest.mark.parametrize("d", [1, 2])
+def test_p10_one_direction_pools_scans_and_skips_its_own_convolved_input(oracle_mod, pool_axis, d):
+    """With one direction the layer is the plain layer of that direction's convolved tokens: their
+    explicit numpy mean pooled, the pinned projection and scan, and the skip D * xc."""
+    rng = np.random.default_rng(1300 + 2 * pool_axis + d)
+    B, h, w, E, N, R = 2, 4, 3, 5, 3, 2
+    A_log, D, W_x, W_dt, b_dt = _rand_params(rng, 1, E, N, R)
+    x, cw, cb = _conv_case(rng, B, h, w, E, 3, 1)
+    z = rng.standard_normal((B, h, w, E)).astype(np.float32)
+    y = oracle_mod.forward(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis, d, conv_w=cw, conv_b=cb, conv_silu=True)
+    xc = _torch_conv(x, cw, cb, pool_axis, d, True)[0]
+    xbar = xc.mean(axis=2 if pool_axis == 0 else 1)
+    u, delta = oracle_mod.proj(xbar, W_x, W_dt, b_dt, R, N)
+    ys = oracle_mod.scan(xbar, delta, u, A_log, R, N, d)
+    rep = ys[:, :, None, :] if pool_axis == 0 else ys[:, None, :, :]
+    ref = _silu(z.astype(np.float64)) * (rep + D[0].astype(np.float64) * xc)
+    np.testing.assert_allclose(y, ref, rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("pool_axis", [0, 1])
+def test_p10_two_directions_add(oracle_mod, pool_axis):
+    """The gate is linear in the summed directions, so the two-direction layer equals the sum of
+    the single-direction layers built from each slot's own filter and parameters."""
+    rng = np.random.default_rng(1400 + pool_axis)
+    B, h, w, E, N, R = 2, 3, 4, 5, 3, 2
+    A_log, D, W_x, W_dt, b_dt = _rand_params(rng, 2, E, N, R)
+    x, cw, cb = _conv_case(rng, B, h, w, E, 4, 2)
+    z = rng.standard_normal((B, h, w, E)).astype(np.float32)
+    both = oracle_mod.forward(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis, 3, conv_w=cw, conv_b=cb)
+    parts = 0.0
+    for k, d in enumerate((1, 2)):
+        sl = slice(k, k + 1)
+        parts = parts + oracle_mod.forward(x, z, A_log[sl], D[sl], W_x[sl], W_dt[sl], b_dt[sl], pool_axis, d,
+                                           conv_w=cw[sl], conv_b=cb[sl])
+    np.testing.assert_allclose(both, parts, rtol=1e-12, atol=1e-13)
+
+
+def test_p10_golden_hand_worked_conv_example(oracle_mod):
+    with open(os.path.join(GOLDEN, "conv_1x3_hand.json")) as f:
+        g = json.load(f)
+    inp = {k: np.array(v, np.float32) for k, v in g["inputs"].items()}
+    ln2 = math.log(2.0)
+    for x, axis in ((inp["x"], g["pool_axis"]), (inp["x"].transpose(0, 2, 1, 3), 0)):  # and its 3x1 transpose
+        inter = oracle_mod.forward_intermediates(x, inp["z"].reshape(x.shape), inp["A_log"], inp["D"], inp["W_x"],
+                                                 inp["W_dt"], inp["b_dt"], axis, g["dir_flags"],
+                                                 conv_w=inp["conv_w"], conv_b=inp["conv_b"])
+        np.testing.assert_array_equal(inter["xc"][0].ravel(), g["expected"]["xc_fwd"])
+        np.testing.assert_array_equal(inter["xc"][1].ravel(), g["expected"]["xc_bwd"])
+        ys = np.array(g["expected"]["ys_over_ln2"]) * ln2
+        np.testing.assert_allclose(inter["ys"].ravel(), ys, rtol=1e-14)
+        z = inp["z"].astype(np.float64).ravel()
+        y = z / (1 + np.exp(-z)) * (ys + np.array(g["expected"]["skip"]))
+        np.testing.assert_allclose(inter["y"].ravel(), y, rtol=1e-14)
+        full = oracle_mod.forward(x, inp["z"].reshape(x.shape), inp["A_log"], inp["D"], inp["W_x"], inp["W_dt"],
+                                  inp["b_dt"], axis, g["dir_flags"], conv_w=inp["conv_w"], conv_b=inp["conv_b"])
+        np.testing.assert_allclose(full.ravel(), y, rtol=1e-14)
