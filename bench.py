@@ -59,9 +59,10 @@ def kernel_work(name: str, cfg, pool_axis: int):
     tok = cfg.tokens_per_call()                       # grid tokens, or kept tokens when masked
     row = 4 * cfg.E                                   # one fp32 token row
     T = cfg.h if pool_axis == 0 else cfg.w
-    if name in ("pool_dense_kernel", "mask_pool_kernel"):
-        return "hbm", row * tok                       # read x
-    if name in ("epilogue_dense_kernel", "mask_epilogue_kernel", "ln_epilogue_kernel", "fused_layer_kernel"):
+    if name in ("pool_dense_kernel", "mask_pool_kernel", "pool_conv_kernel"):
+        return "hbm", row * tok                       # read x (with the Conv1D: its input)
+    if name in ("epilogue_dense_kernel", "mask_epilogue_kernel", "ln_epilogue_kernel", "fused_layer_kernel",
+                "epilogue_conv_kernel"):
         return "hbm", 3 * row * tok                   # read x and z, write y (the fused launch: the layer)
     if name == "scan_seq_kernel":
         return "alu", cfg.B * T * cfg.E * cfg.N * cfg.nd
@@ -114,6 +115,8 @@ def parse(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--conv", type=int, default=0, choices=range(0, 5), metavar="TAPS",
+                    help="put the block's Conv1D (TAPS taps per direction, SiLU after it) in front of the layer")
     ap.add_argument("--no-configs", action="store_true",
                     help="time only the chosen workload (by default the headline run also times the other "
                          "workloads and reports them under 'configs')")
@@ -365,6 +368,11 @@ def run_reference(a, cfg, pool_axis):
 # blocks); its inputs fit in L2, so each of its steps starts after an L2 flush.
 SECONDARY = (("fastvim_t_224_tiny", 0), ("fastvim_t_224", 0), ("fastvim_t_224", 1), ("fastvim_s_1024", 1),
              ("fastmaskvim_b_1024_mask75", 0))
+# Variants timed beside them: (config, pool axis, Conv1D taps, path).  The headline layer with the
+# block's Conv1D in front (4 taps per direction, SiLU after it: x is the Conv1D's input, so the
+# layer's algorithmic bytes are unchanged), and the small 224 px layer on the single persistent
+# launch (the automatic choice takes the staged kernels there).
+SECONDARY_VARIANTS = (("fastvim_t_2048", 0, 4, "auto"), ("fastvim_t_224", 0, 0, "fused"))
 
 
 def summarize_kernels(per_kernel, names, cfg, pool_axis, peak, mufu_peak, fma_peak):
@@ -411,7 +419,7 @@ def roofline_of(kern, dom, cfg, pool_axis, peak, peak_src, mufu_peak, fma_peak):
             "note": "achieved = algorithmic bytes per launch / mean CUDA-event duration of the launch"}
 
 
-def time_layer(a, cfg, pool_axis, dev, world=1, first_image=0, clocks=None):
+def time_layer(a, cfg, pool_axis, dev, world=1, first_image=0, clocks=None, conv=None, path=None):
     """Device-timed forward calls of one workload (inputs resident in HBM): `a.warmup` untimed calls,
     then `a.steps` timed ones between CUDA events on the launching stream, each launch bracketed by
     its own pair of events.  Returns the step time (max over ranks), the per-kernel table and the
@@ -421,12 +429,16 @@ def time_layer(a, cfg, pool_axis, dev, world=1, first_image=0, clocks=None):
 
     from pooled_selective_scan_b200 import ssm, workload
 
+    conv = a.conv if conv is None else conv
+    path = a.path if path is None else path
     t = workload.layer_tensors(cfg, dev, first_image=first_image)
     if a.ln:
         t.update(workload.ln_tensors(cfg, dev))
+    if conv:
+        t.update(workload.conv_tensors(cfg, dev, conv))
     keep = t.get("keep_idx")
-    shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, cfg.dir_flags, keep, cfg.h, cfg.w, path=a.path,
-                            ln=a.ln)
+    shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, cfg.dir_flags, keep, cfg.h, cfg.w, path=path,
+                            ln=a.ln, d_conv=conv, conv_silu=bool(conv))
     y = torch.empty_like(t["x"])
     ws = ssm.alloc_workspace(shape, dev)
     stream = torch.cuda.current_stream(dev)
@@ -547,6 +559,8 @@ def time_e2e(a, cfg, shape, dev, world=1, first_image=0):
     host = workload.layer_tensors(cfg, dev, pinned_host=True, first_image=first_image)
     if a.ln:
         host.update({k: v.pin_memory() for k, v in workload.ln_tensors(cfg, "cpu").items()})
+    if a.conv:
+        host.update({k: v.pin_memory() for k, v in workload.conv_tensors(cfg, "cpu", a.conv).items()})
     run = ssm.HostForward(shape, dev)
     y_host = torch.empty(host["x"].shape, dtype=torch.float32).pin_memory()
     run(host, y_host)  # warm
@@ -604,6 +618,7 @@ def run_ours(a, cfg, pool_axis):
         "dtype": "f32", "data": "synthetic (seeded N(0,1) x, z; Mamba-style parameter init)",
         "config": dict(workload_desc(cfg, pool_axis),
                        **({"post_ssm_layernorm": "gamma = 1, beta = 0, eps = 1e-5"} if a.ln else {}),
+                       **({"conv1d": f"{a.conv} taps per direction + SiLU in front; x is its input"} if a.conv else {}),
                        l2=r["l2"], global_batch=cfg.B * world,
                        parallelism=f"data parallel, no collective: each of {world} GPU(s) runs its own "
                                    f"{cfg.B} distinct images"),
@@ -619,7 +634,7 @@ def run_ours(a, cfg, pool_axis):
         line["cpu_baseline"] = cpu_baseline(cfg, pool_axis)
 
     # the other workloads of the efficiency study, one GPU, default run only
-    if world == 1 and not a.no_configs and a.batch is None and cfg.name == HEADLINE_NAME:
+    if world == 1 and not a.no_configs and a.batch is None and cfg.name == HEADLINE_NAME and not a.conv and not a.ln:
         configs = {}
         for name, axis in SECONDARY:
             c = by_name(name)
@@ -631,6 +646,20 @@ def run_ours(a, cfg, pool_axis):
             if not a.no_cpu_baseline:
                 ent["cpu_baseline"] = cpu_baseline(c, axis, min_seconds=5.0)
             configs[f"{name}/{'pool_w' if axis == 0 else 'pool_h'}"] = ent
+        for name, axis, taps, path in SECONDARY_VARIANTS:
+            c = by_name(name)
+            sub = time_layer(a, c, axis, dev, conv=taps, path=path)
+            desc = workload_desc(c, axis)
+            if taps:
+                desc["conv1d"] = f"{taps} taps per direction + SiLU in front; x is its input"
+            if path != "auto":
+                desc["path"] = path
+            ent = {"workload": desc, "ms_per_step": sub["ms_per_step"], "value": sub["value"], "unit": UNIT,
+                   "steps": a.steps, "warmup": a.warmup, "l2": sub["l2"], "layer_hbm": sub["layer_hbm"],
+                   "roofline": sub["roofline"], "kernels": sub["kernels"], "gpu_launches": sub["gpu_launches"],
+                   "clocks": sub["clocks"]}
+            key = name + (f"+conv{taps}" if taps else "") + ("" if path == "auto" else f"+{path}")
+            configs[f"{key}/{'pool_w' if axis == 0 else 'pool_h'}"] = ent
         line["configs"] = configs
     if world > 1:
         dist.barrier()
@@ -653,6 +682,8 @@ def run_grad(a, cfg, pool_axis):
     world, rank, local = dist_env()
     if world > 1:
         raise SystemExit("--grad runs on one GPU")
+    if a.conv:
+        raise SystemExit("--grad: the gradient through the Conv1D is not built")
     if not os.path.exists(os.path.join(ROOT, "pooled_selective_scan_b200", "libfastvim_ssm.so")):
         fvbuild.build()
     dev = torch.device("cuda", local)

@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define FASTVIM_SSM_ABI_VERSION 3
+#define FASTVIM_SSM_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define FV_API __attribute__((visibility("default")))
@@ -88,7 +88,8 @@ enum {
                                  FV_ERR_UNSUPPORTED when the layer does not fit it)             */
     FV_FLAG_TRACE = 8u,       /* fused launch: record one entry per task in the workspace
                                  (fv_ws_layout.trace); costs a little time, for profiling      */
-    FV_FLAG_LAYERNORM = 16u   /* post-SSM LayerNorm before the gate (ln_gamma, ln_beta, ln_eps) */
+    FV_FLAG_LAYERNORM = 16u,  /* post-SSM LayerNorm before the gate (ln_gamma, ln_beta, ln_eps) */
+    FV_FLAG_CONV_SILU = 32u   /* SiLU after the block's Conv1D (needs d_conv > 0)               */
 };
 /* Without a PATH flag a dense layer whose images hold >= 16 MiB of x runs the fused launch, every
  * other layer the staged kernels; both compute the same layer.  The fused launch gates image b
@@ -124,13 +125,33 @@ typedef struct {
     const float* ln_gamma;   /* NULL or [E]                                                  */
     const float* ln_beta;    /* NULL or [E]                                                  */
     float ln_eps;            /* LayerNorm epsilon (e.g. 1e-5)                                */
+    /* The block's Conv1D in front of the layer, with d_conv > 0 (dense layers).  The summary
+     * page ("方法详解" item 2) pools the output of the block's Conv1D; the Vim article's code
+     * (section 2.1) gives each direction its own Conv1D of the expanded tokens, the backward one
+     * run over the reversed sequence.  With d_conv > 0, x is the Conv1D's INPUT (the x half of
+     * the expansion layer's output) and, per channel, for direction slot k
+     *   forward slot:  xc_k[p] = act(conv_b[k] + sum_{q<d_conv} conv_w[k][q] x[p - (d_conv-1) + q])
+     *   backward slot: xc_k[p] = act(conv_b[k] + sum_{q<d_conv} conv_w[k][q] x[p + (d_conv-1) - q])
+     * with x = 0 outside the sequence and act = SiLU under FV_FLAG_CONV_SILU, else the identity.
+     * The sequence is the block's token order p = t * S + s: the pooled lines t in order and the
+     * tokens s along each line (row-major for POOL_W, column-major for POOL_H), so a line's first
+     * tokens see the end of the line before.  Each direction then pools, projects and scans its
+     * own xc_k, and the skip is sum_k D[k] * xc_k.  xc is never written to memory.
+     * d_conv: 0 (no Conv1D: x is its output) or 1..4 (> 4: FV_ERR_UNSUPPORTED); conv_w
+     * [nd][E][d_conv] and conv_b [nd][E] are required with d_conv > 0 (FV_ERR_NULL) and must be
+     * NULL without (FV_ERR_SHAPE), as must FV_FLAG_CONV_SILU; masked layers, the single
+     * persistent launch (FV_FLAG_PATH_FUSED) and the gradient return FV_ERR_UNSUPPORTED with it. */
+    int d_conv;              /* taps of the depthwise Conv1D, 0 = none                        */
+    const float* conv_w;     /* NULL or [nd][E][d_conv]                                      */
+    const float* conv_b;     /* NULL or [nd][E]                                              */
 } fv_ssm_args;
 
 /* Byte offsets of the intermediates inside a workspace (for inspection and tests). */
 typedef struct {
     size_t total_bytes;  /* what fastvim_ssm_workspace_size returns                          */
     size_t status;       /* uint32 device status word (+ one uint32 of scratch)              */
-    size_t xbar;         /* fp32 [B][T][E] pooled tokens                                     */
+    size_t xbar;         /* fp32 [B][nx][T][E] pooled tokens; nx = nd with the Conv1D (each
+                            direction pools its own convolved tokens), else 1              */
     size_t u;            /* fp32 projections dt_low | B | C: [B][nd] blocks of [T][R+2N], each
                             block starting every ceil(T (R+2N) / 32) * 32 floats            */
     size_t ys;           /* fp32 [B][T][E] scan output summed over directions                */

@@ -28,6 +28,7 @@ FV_FLAG_PATH_STAGED = 2
 FV_FLAG_PATH_FUSED = 4
 FV_FLAG_TRACE = 8
 FV_FLAG_LAYERNORM = 16
+FV_FLAG_CONV_SILU = 32
 
 # Every exported symbol of the ABI, as the header declares it.
 EXPORTS = (
@@ -70,6 +71,7 @@ class FvSsmArgs(ctypes.Structure):
         ("keep_idx", ctypes.c_void_p),
         ("y", ctypes.c_void_p),
         ("ln_gamma", ctypes.c_void_p), ("ln_beta", ctypes.c_void_p), ("ln_eps", ctypes.c_float),
+        ("d_conv", ctypes.c_int), ("conv_w", ctypes.c_void_p), ("conv_b", ctypes.c_void_p),
     ]
 
 

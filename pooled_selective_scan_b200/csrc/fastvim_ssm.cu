@@ -44,8 +44,10 @@ fv_status make_shape(const fv_ssm_args* a, fv::Shape* sh) {
     if (a->pool_axis != FV_POOL_W && a->pool_axis != FV_POOL_H) return FV_ERR_SHAPE;
     if (a->dir_flags == 0 || (a->dir_flags & ~3u) != 0) return FV_ERR_SHAPE;
     if ((a->flags & ~(unsigned)(FV_FLAG_ZOH_EXACT | FV_FLAG_PATH_STAGED | FV_FLAG_PATH_FUSED | FV_FLAG_TRACE |
-                                FV_FLAG_LAYERNORM)) != 0)
+                                FV_FLAG_LAYERNORM | FV_FLAG_CONV_SILU)) != 0)
         return FV_ERR_SHAPE;
+    if (a->d_conv < 0) return FV_ERR_SHAPE;
+    if (a->d_conv == 0 && (a->flags & FV_FLAG_CONV_SILU)) return FV_ERR_SHAPE;  // SiLU of no Conv1D
     if ((a->flags & FV_FLAG_PATH_STAGED) && (a->flags & FV_FLAG_PATH_FUSED)) return FV_ERR_SHAPE;
     if (a->E % 4 != 0) return FV_ERR_SHAPE;
     if (a->K < 0 || (long long)a->K > (long long)a->h * a->w) return FV_ERR_SHAPE;
@@ -72,6 +74,11 @@ fv_status make_shape(const fv_ssm_args* a, fv::Shape* sh) {
     sh->ln_eps = sh->ln ? a->ln_eps : 0.f;
     if (sh->ln && !(a->ln_eps > 0.f && a->ln_eps <= 3.0e38f)) return FV_ERR_SHAPE;
     if (sh->ln && a->E > kMaxLnE) return FV_ERR_UNSUPPORTED;
+    sh->dc = a->d_conv;
+    sh->conv_silu = (a->flags & FV_FLAG_CONV_SILU) ? 1 : 0;
+    sh->nx = a->d_conv > 0 ? sh->nd : 1;
+    if (a->d_conv > fv::kMaxConv) return FV_ERR_UNSUPPORTED;
+    if (a->d_conv > 0 && a->K > 0) return FV_ERR_UNSUPPORTED;  // the Conv1D is for dense grids
     if (sh->T > kMaxT) return FV_ERR_UNSUPPORTED;
     if (a->K > 0 && (long long)a->h * a->w > kMaxMaskGrid) return FV_ERR_UNSUPPORTED;
     if ((long long)sh->B * sh->T >= (1ll << 31)) return FV_ERR_UNSUPPORTED;
@@ -85,8 +92,10 @@ fv_status check_pointers(const fv_ssm_args* a, const fv::Shape& sh) {
     if (sh.K == 0 && a->keep_idx) return FV_ERR_SHAPE;  // a keep list needs K
     if (sh.ln && (!a->ln_gamma || !a->ln_beta)) return FV_ERR_NULL;
     if (!sh.ln && (a->ln_gamma || a->ln_beta)) return FV_ERR_SHAPE;  // LayerNorm weights need the flag
+    if (sh.dc > 0 && (!a->conv_w || !a->conv_b)) return FV_ERR_NULL;
+    if (sh.dc == 0 && (a->conv_w || a->conv_b)) return FV_ERR_SHAPE;  // Conv1D weights need d_conv
     const void* ps[] = {a->x, a->z, a->y, a->A_log, a->D, a->W_x, a->W_dt, a->b_dt, a->keep_idx, a->ln_gamma,
-                        a->ln_beta};
+                        a->ln_beta, a->conv_w, a->conv_b};
     for (const void* p : ps)
         if (p && !aligned16(p)) return FV_ERR_ALIGN;
     if (sh.B > 0) {
@@ -108,7 +117,7 @@ fv_status plan_layout(const fv::Shape& sh, fv_ws_layout* L) {
     size_t off = 0;
     // word 0: the call's device status; word 1: scratch of fastvim_ssm_forward_host
     L->status = off; off = round256(off + 2 * sizeof(unsigned));
-    L->xbar = off; off = round256(off + (size_t)sh.B * sh.T * sh.E * sizeof(float));
+    L->xbar = off; off = round256(off + (size_t)sh.B * sh.nx * sh.T * sh.E * sizeof(float));
     L->u = off; off = round256(off + (size_t)sh.nd * sh.B * fv::u_block_stride(sh.T, sh.J) * sizeof(float));
     L->ys = off; off = round256(off + (size_t)sh.B * sh.T * sh.E * sizeof(float));
     if (sh.K > 0) {
@@ -156,7 +165,7 @@ int fused_lines_per_task(const fv::Shape& sh) {
 }
 
 bool fused_possible(const fv::Shape& sh) {
-    if (sh.K > 0 || sh.B < 1) return false;
+    if (sh.K > 0 || sh.B < 1 || sh.dc > 0) return false;
     // a token row of x (and of z) must fit half a ring stage; a thread holds at most 2 float4 slots
     if ((size_t)sh.E * sizeof(float) > (size_t)fv::kStageBytes / 2) return false;
     if (sh.SL > fv::kMaxSlots * fv::kFusedThreads) return false;
@@ -281,13 +290,14 @@ int launch_count_of(const fv::Shape& sh) {
 const char* launch_name_of(const fv::Shape& sh, int i) {
     static const char* dense[] = {"pool_dense_kernel", "proj_gemm_kernel", "scan_seq_kernel",
                                   "epilogue_dense_kernel"};
+    static const char* conv[] = {"pool_conv_kernel", "proj_gemm_kernel", "scan_seq_kernel", "epilogue_conv_kernel"};
     static const char* masked[] = {"mask_bucket_kernel", "mask_pool_kernel", "proj_gemm_kernel", "scan_seq_kernel",
                                    "mask_epilogue_kernel"};
     const int n = launch_count_of(sh);
     if (i < 0 || i >= n) return "";
     if (choose_path(sh) == Path::Fused) return "fused_layer_kernel";
     if (sh.ln && i == n - 1) return "ln_epilogue_kernel";
-    return sh.K > 0 ? masked[i] : dense[i];
+    return sh.K > 0 ? masked[i] : (sh.dc > 0 ? conv[i] : dense[i]);
 }
 
 template <int ND, bool Z>
@@ -362,8 +372,13 @@ fv_status staged_front(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_la
         FV_MARK_CALL(marks, st, ([&]() -> fv_status {
             // a whole number of token groups of SL threads each (no idle threads)
             const int threads = sh.SL <= fv::kThreads ? (fv::kThreads / sh.SL) * sh.SL : fv::kThreads;
-            fv::pool_dense_kernel<<<M, threads, 0, st>>>(sh, a->x, xbar);
-            FV_LAUNCH_CHECK("pool_dense_kernel");
+            if (sh.dc > 0) {
+                fv::pool_conv_kernel<<<M, threads, 0, st>>>(sh, a->x, a->conv_w, a->conv_b, xbar);
+                FV_LAUNCH_CHECK("pool_conv_kernel");
+            } else {
+                fv::pool_dense_kernel<<<M, threads, 0, st>>>(sh, a->x, xbar);
+                FV_LAUNCH_CHECK("pool_dense_kernel");
+            }
             return FV_OK;
         })());
         return FV_OK;
@@ -379,7 +394,9 @@ fv_status staged_front(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_la
         return FV_OK;
     })());
     FV_MARK_CALL(marks, st, ([&]() -> fv_status {
-        fv::mask_pool_kernel<<<M, fv::kThreads, 0, st>>>(sh, a->x, (const int32_t*)(ws + L.row_off),
+        const int threads = sh.SL <= fv::kThreads ? fv::kThreads
+                                                  : std::min(fv::kMaskPoolMaxThreads, (sh.SL + 31) / 32 * 32);
+        fv::mask_pool_kernel<<<M, threads, 0, st>>>(sh, a->x, (const int32_t*)(ws + L.row_off),
                                                          (const int32_t*)(ws + L.row_tok), xbar);
         FV_LAUNCH_CHECK("mask_pool_kernel");
         return FV_OK;
@@ -392,7 +409,9 @@ fv_status launch_proj_gemm(const fv::Shape& sh, const fv_ssm_args* a, const fv_w
     cudaError_t e = ensure_smem(fv::proj_gemm_kernel, fv::kPgSmemBytes);
     if (e != cudaSuccess) { note_cuda(e, "proj smem attribute"); return FV_ERR_CUDA; }
     const long long M = (long long)sh.B * sh.T;
-    const dim3 grid((unsigned)((M + fv::kPgM - 1) / fv::kPgM), (unsigned)((sh.NJ + fv::kPgN - 1) / fv::kPgN));
+    const int nz = sh.NJ / sh.nx;  // outputs per pooled-token set
+    const dim3 grid((unsigned)((M + fv::kPgM - 1) / fv::kPgM), (unsigned)((nz + fv::kPgN - 1) / fv::kPgN),
+                    (unsigned)sh.nx);
     if (M >= (1ll << 31) / 2) return FV_ERR_UNSUPPORTED;
     fv::proj_gemm_kernel<<<grid, fv::kPgThreads, fv::kPgSmemBytes, st>>>(sh, (const float*)(ws + L.xbar), a->W_x,
                                                                         (float*)(ws + L.u));
@@ -414,17 +433,26 @@ fv_status staged_back(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_lay
     const float* ys = (const float*)(ws + L.ys);
     if (sh.ln) {
         const size_t smem = fv::ln_epilogue_smem_bytes(sh);
-        cudaError_t e = ensure_smem(fv::ln_epilogue_kernel, smem);
+        auto kern = sh.dc > 0 ? fv::ln_epilogue_kernel<true> : fv::ln_epilogue_kernel<false>;
+        cudaError_t e = ensure_smem(kern, smem);
         if (e != cudaSuccess) { note_cuda(e, "LayerNorm epilogue smem attribute"); return FV_ERR_CUDA; }
         const long long ntok = (long long)sh.B * (sh.K > 0 ? (long long)sh.K : (long long)sh.h * sh.w);
         const long long per = (long long)fv::kLnWarps * fv::kLnTokensPerWarp;
         const long long grid = (ntok + per - 1) / per;
         if (grid >= (1ll << 31)) return FV_ERR_UNSUPPORTED;
         FV_MARK_CALL(marks, st, ([&]() -> fv_status {
-            fv::ln_epilogue_kernel<<<(unsigned)grid, fv::kLnWarps * 32, smem, st>>>(
+            kern<<<(unsigned)grid, fv::kLnWarps * 32, smem, st>>>(
                 sh, a->x, a->z, ys, a->D, a->ln_gamma, a->ln_beta,
-                sh.K > 0 ? (const int32_t*)(ws + L.row_of) : nullptr, a->y);
+                sh.K > 0 ? (const int32_t*)(ws + L.row_of) : nullptr, a->conv_w, a->conv_b, a->y);
             FV_LAUNCH_CHECK("ln_epilogue_kernel");
+            return FV_OK;
+        })());
+    } else if (sh.K == 0 && sh.dc > 0) {
+        FV_MARK_CALL(marks, st, ([&]() -> fv_status {
+            const int threads = sh.SL <= fv::kThreads ? (fv::kThreads / sh.SL) * sh.SL : fv::kThreads;
+            fv::epilogue_conv_kernel<<<sh.B * sh.T, threads, 0, st>>>(sh, a->x, a->z, ys, a->D, a->conv_w, a->conv_b,
+                                                                       a->y);
+            FV_LAUNCH_CHECK("epilogue_conv_kernel");
             return FV_OK;
         })());
     } else if (sh.K == 0) {
@@ -585,6 +613,7 @@ fv_status fastvim_ssm_forward_host(const fv_ssm_args* host, const fv_ssm_args* d
     if (host->B != dev->B || host->h != dev->h || host->w != dev->w || host->E != dev->E ||
         host->N != dev->N || host->R != dev->R || host->K != dev->K || host->pool_axis != dev->pool_axis ||
         host->dir_flags != dev->dir_flags || host->flags != dev->flags || host->pool_scale != dev->pool_scale ||
+        host->d_conv != dev->d_conv ||
         ((host->flags & FV_FLAG_LAYERNORM) && host->ln_eps != dev->ln_eps))
         return FV_ERR_SHAPE;
     if ((s = check_pointers(host, sh)) != FV_OK) return s;
@@ -635,6 +664,8 @@ fv_status fastvim_ssm_forward_host(const fv_ssm_args* host, const fv_ssm_args* d
         {(void*)dev->keep_idx, host->keep_idx, sh.K > 0 ? (size_t)sh.B * sh.K * sizeof(int32_t) : 0},
         {(void*)dev->ln_gamma, host->ln_gamma, sh.ln ? (size_t)sh.E * sizeof(float) : 0},
         {(void*)dev->ln_beta, host->ln_beta, sh.ln ? (size_t)sh.E * sizeof(float) : 0},
+        {(void*)dev->conv_w, host->conv_w, nd * sh.E * (size_t)sh.dc * sizeof(float)},
+        {(void*)dev->conv_b, host->conv_b, sh.dc > 0 ? nd * sh.E * sizeof(float) : 0},
     };
     for (const Copy& c : params) {
         if (c.bytes == 0 || !c.dst) continue;
@@ -883,6 +914,7 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
     const fv_ssm_args* a = &ac;
     if ((s = check_pointers(a, sh)) != FV_OK) return s;
     if ((s = check_grads(a, sh, g)) != FV_OK) return s;
+    if (sh.dc > 0) return FV_ERR_UNSUPPORTED;  // the gradient through the Conv1D is not built
     fv_ws_layout FL;
     plan_layout(sh, &FL);
     const BwdLayout L = plan_bwd(sh);

@@ -29,7 +29,17 @@ struct Shape {
     int SL;            // float4 slots per token row: E / 4
     int ln;            // FV_FLAG_LAYERNORM: post-SSM LayerNorm before the gate
     float ln_eps;
+    int dc;            // taps of the block's Conv1D in front of the layer (0: x is its output)
+    int conv_silu;     // FV_FLAG_CONV_SILU: SiLU after the Conv1D
+    int nx;            // pooled-token sets: nd with the Conv1D (one per direction), else 1
 };
+
+constexpr int kMaxConv = 4;  // Conv1D taps at most
+
+// Pooled tokens of image b, set kx (the direction's own with the Conv1D, else 0): [T][E] rows.
+__host__ __device__ __forceinline__ size_t xbar_offset(const Shape& sh, int b, int kx, int t) {
+    return (((size_t)b * sh.nx + kx) * sh.T + t) * (size_t)sh.E;
+}
 
 // Projections u of (image b, direction k) are one block of T x J floats, image-major (so the
 // blocks of a run of images are contiguous); blocks start every

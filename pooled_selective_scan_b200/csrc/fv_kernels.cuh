@@ -156,8 +156,11 @@ mask_bucket_kernel(Shape sh, const int32_t* __restrict__ keep_idx, int32_t* row_
 }
 
 // One CTA per pooled row (b, t) of a masked sample: sum of the row's kept tokens divided by the
-// fixed full length S (an empty row pools to 0).
-__global__ void __launch_bounds__(kThreads)
+// fixed full length S (an empty row pools to 0).  Up to 256 float4 slots per token: groups of SL
+// threads split the row's tokens; wider rows: one thread per slot (launched with SL threads
+// rounded up to whole warps, up to 1024), so no thread takes two slots while others take one.
+constexpr int kMaskPoolMaxThreads = 1024;
+__global__ void __launch_bounds__(kMaskPoolMaxThreads)
 mask_pool_kernel(Shape sh, const float* __restrict__ x, const int32_t* __restrict__ row_off,
                  const int32_t* __restrict__ row_tok, float* __restrict__ xbar) {
     __shared__ float4 part[kThreads];
@@ -184,7 +187,7 @@ mask_pool_kernel(Shape sh, const float* __restrict__ x, const int32_t* __restric
             out[threadIdx.x] = f4_scale(s, scale);
         }
     } else {
-        for (int slot = threadIdx.x; slot < SL; slot += kThreads) {
+        for (int slot = threadIdx.x; slot < SL; slot += blockDim.x) {
             float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
             int p = p0;
             for (; p + 3 < p1; p += 4) {  // four kept tokens in flight
@@ -310,6 +313,247 @@ mask_epilogue_kernel(Shape sh, const float* __restrict__ x, const float* __restr
     }
 }
 
+// ---- The block's Conv1D in front of the layer (dense layers, staged kernels) ---------------------
+// Summary page, "方法详解" item 2 (the layer pools the output of the block's Conv1D) and the Vim
+// article's section 2.1 code (one Conv1D per direction, the backward one over the reversed
+// sequence).  Depthwise, d_conv <= 4 taps, zero padding, along the block's sequence p = t S + s.
+// Nothing convolved is stored: the pooling and the epilogue recompute it from x as they stream it,
+// each thread sliding a window of 7 tokens (p - 3 .. p + 3) of one float4 slot along a run of
+// consecutive sequence positions, so every token row is loaded once per run (plus 6 halo rows).
+struct ConvSlot {
+    float4 w[2][kMaxConv];  // taps of direction slots 0, 1, right-aligned in a 4-wide window (zero-padded)
+    float4 b[2];            // biases
+};
+
+// Filters of float4 slot `slot` (channels 4 slot .. 4 slot + 3).  conv_w [nd][E][dc], conv_b [nd][E].
+__device__ __forceinline__ ConvSlot conv_slot(const Shape& sh, const float* __restrict__ conv_w,
+                                              const float* __restrict__ conv_b, int slot) {
+    ConvSlot c;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        c.b[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < kMaxConv; ++q) c.w[k][q] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (k < sh.nd) {
+            c.b[k] = __ldg(reinterpret_cast<const float4*>(conv_b + (size_t)k * sh.E) + slot);
+            const float* wk = conv_w + ((size_t)k * sh.E + 4 * slot) * sh.dc;
+#pragma unroll
+            for (int qq = 0; qq < kMaxConv; ++qq) {  // window tap qq holds filter tap qq - (4 - dc)
+                const int q = qq - (kMaxConv - sh.dc);
+                if (q >= 0)
+                    c.w[k][qq] = make_float4(__ldg(wk + q), __ldg(wk + sh.dc + q), __ldg(wk + 2 * sh.dc + q),
+                                             __ldg(wk + 3 * sh.dc + q));
+            }
+        }
+    }
+    return c;
+}
+
+__device__ __forceinline__ float4 f4_silu(const float4& v) {
+    return make_float4(silu_fast(v.x), silu_fast(v.y), silu_fast(v.z), silu_fast(v.w));
+}
+
+// The convolved value of direction slot k at the window's centre: a forward slot reads the window
+// tokens p - 3 .. p (taps in order), a backward slot p + 3 .. p (the same filter on the reversed
+// sequence).
+__device__ __forceinline__ float4 conv_at(const Shape& sh, const ConvSlot& c, int k, bool fwd, const float4 (&win)[7]) {
+    float4 a = c.b[k];
+#pragma unroll
+    for (int q = 0; q < kMaxConv; ++q) a = f4_fma(c.w[k][q], fwd ? win[q] : win[6 - q], a);
+    return sh.conv_silu ? f4_silu(a) : a;
+}
+
+// Sequence cursor of image b: position (t, s), t = line, s = token along it.
+struct SeqPos {
+    int t, s;
+};
+__device__ __forceinline__ void seq_step(const Shape& sh, SeqPos& p) {
+    if (++p.s == sh.S) { p.s = 0; ++p.t; }
+}
+__device__ __forceinline__ SeqPos seq_back(const Shape& sh, SeqPos p, int n) {
+    p.s -= n;
+    while (p.s < 0) { p.s += sh.S; --p.t; }
+    return p;
+}
+// Slot `slot` of the token at position p of image b (zero outside the sequence).
+__device__ __forceinline__ float4 seq_load(const Shape& sh, const float4* __restrict__ x4, int b, const SeqPos& p,
+                                           int slot) {
+    if (p.t < 0 || p.t >= sh.T) return make_float4(0.f, 0.f, 0.f, 0.f);
+    return ld_stream(x4 + ((dense_base(sh, b, p.t) + (size_t)p.s * dense_stride(sh)) >> 2) + slot);
+}
+
+// Runs `emit(s, xc0, xc1, zv)` for the tokens s in [s0, s1) of line t of image b, xc0 and xc1
+// the convolved values of direction slots 0 and 1 (xc1 unused with one direction), zv the token's
+// z (with WITH_Z).  Loads run one batch of kU tokens ahead of the arithmetic, so 2 kU tokens are
+// in flight (kU = 4 for the pooling, 2 for the epilogue, whose registers also hold z); tokens inside line t are addressed from the line's base, the halo beyond it through
+// the sequence cursor.
+template <bool WITH_Z, int kU, class Emit>
+__device__ __forceinline__ void conv_line_run(const Shape& sh, const float* __restrict__ x, const float* __restrict__ z,
+                                              const ConvSlot& c, int b, int t, int s0, int s1, int slot, Emit&& emit) {
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    const size_t line4 = (dense_base(sh, b, t) >> 2) + slot;
+    const size_t st4 = dense_stride(sh) >> 2;
+    const int S = sh.S;
+    const bool fwd0 = (sh.dir_flags & 1u) != 0;  // slot 0 is the forward direction when it is enabled
+    auto load_x = [&](int s) -> float4 {
+        if (s >= 0 && s < S) return ld_stream(x4 + line4 + (size_t)s * st4);
+        SeqPos p{t, s};
+        while (p.s < 0) { p.s += S; --p.t; }
+        while (p.s >= S) { p.s -= S; ++p.t; }
+        return seq_load(sh, x4, b, p, slot);
+    };
+    auto load_z = [&](int s) -> float4 {
+        return (WITH_Z && s < s1) ? ld_stream(reinterpret_cast<const float4*>(z) + line4 + (size_t)s * st4)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+    };
+    float4 win[7];
+#pragma unroll
+    for (int i = 0; i < 6; ++i) win[i + 1] = load_x(s0 - 3 + i);  // positions s0 - 3 .. s0 + 2
+    float4 nx[kU], nz[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+        nx[u] = load_x(s0 + 3 + u);
+        nz[u] = load_z(s0 + u);
+    }
+    for (int s = s0; s < s1; s += kU) {
+        float4 cx[kU], cz[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            cx[u] = nx[u];
+            cz[u] = nz[u];
+        }
+        if (s + kU < s1) {
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                nx[u] = load_x(s + kU + 3 + u);
+                nz[u] = load_z(s + kU + u);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+#pragma unroll
+            for (int i = 0; i < 6; ++i) win[i] = win[i + 1];
+            win[6] = cx[u];
+            if (s + u < s1) {
+                const float4 a = conv_at(sh, c, 0, fwd0, win);
+                const float4 bb = sh.nd == 2 ? conv_at(sh, c, 1, false, win) : a;
+                emit(s + u, a, bb, cz[u]);
+            }
+        }
+    }
+}
+
+// Thread layout of the conv kernels: G groups of SL threads (one float4 slot each) per CTA, group
+// g taking a contiguous run of the line's tokens; above 256 slots one group loops over the slots.
+__device__ __forceinline__ void conv_groups(const Shape& sh, int& G, int& g, int& slot0, int& slot_step) {
+    if (sh.SL <= kThreads) {
+        G = kThreads / sh.SL;
+        g = threadIdx.x / sh.SL;
+        slot0 = threadIdx.x - g * sh.SL;
+        slot_step = sh.SL;  // one slot
+    } else {
+        G = 1;
+        g = 0;
+        slot0 = threadIdx.x;
+        slot_step = kThreads;
+    }
+}
+
+// One CTA per pooled token (b, t): each direction slot pools its own convolved tokens of line t,
+// xbar[b][k][t] = pool_scale / S * sum_s xc_k(t, s).
+__global__ void __launch_bounds__(kThreads, 2)
+pool_conv_kernel(Shape sh, const float* __restrict__ x, const float* __restrict__ conv_w,
+                 const float* __restrict__ conv_b, float* __restrict__ xbar) {
+    __shared__ float4 part[2][kThreads];
+    const int bt = blockIdx.x;
+    const int b = bt / sh.T, t = bt - b * sh.T;
+    const float scale = sh.pool_scale / (float)sh.S;
+    int G, g, slot0, sstep;
+    conv_groups(sh, G, g, slot0, sstep);
+    const int run = (sh.S + G - 1) / G;
+    const int s0 = g * run, s1 = min(sh.S, s0 + run);
+    for (int slot = slot0; slot < sh.SL; slot += sstep) {
+        float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+        if (g < G && s0 < s1) {
+            const ConvSlot c = conv_slot(sh, conv_w, conv_b, slot);
+            conv_line_run<false, 4>(sh, x, nullptr, c, b, t, s0, s1, slot,
+                                 [&](int, const float4& a, const float4& bb, const float4&) {
+                                     f4_add(acc0, a);
+                                     f4_add(acc1, bb);
+                                 });
+        }
+        if (G == 1) {
+            reinterpret_cast<float4*>(xbar + xbar_offset(sh, b, 0, t))[slot] = f4_scale(acc0, scale);
+            if (sh.nd == 2) reinterpret_cast<float4*>(xbar + xbar_offset(sh, b, 1, t))[slot] = f4_scale(acc1, scale);
+        } else {
+            part[0][threadIdx.x] = acc0;
+            part[1][threadIdx.x] = acc1;
+            __syncthreads();
+            if (threadIdx.x < sh.SL) {
+                for (int k = 0; k < sh.nd; ++k) {
+                    float4 v = part[k][threadIdx.x];
+                    for (int q = 1; q < G; ++q) f4_add(v, part[k][q * sh.SL + threadIdx.x]);
+                    reinterpret_cast<float4*>(xbar + xbar_offset(sh, b, k, t))[threadIdx.x] = f4_scale(v, scale);
+                }
+            }
+        }
+    }
+}
+
+// One CTA per pooled token (b, t): y = SiLU(z) * (ys[b][t] + sum_k D[k] * xc_k) for the tokens of
+// line t, the convolved values recomputed from x.
+__global__ void __launch_bounds__(kThreads, 2)
+epilogue_conv_kernel(Shape sh, const float* __restrict__ x, const float* __restrict__ z,
+                     const float* __restrict__ ys, const float* __restrict__ D, const float* __restrict__ conv_w,
+                     const float* __restrict__ conv_b, float* __restrict__ y) {
+    const int bt = blockIdx.x;
+    const int b = bt / sh.T, t = bt - b * sh.T;
+    const size_t base4 = dense_base(sh, b, t) >> 2;
+    const size_t st4 = dense_stride(sh) >> 2;
+    float4* y4 = reinterpret_cast<float4*>(y) + base4;
+    int G, g, slot0, sstep;
+    conv_groups(sh, G, g, slot0, sstep);
+    if (g >= G) return;
+    const int run = (sh.S + G - 1) / G;
+    const int s0 = g * run, s1 = min(sh.S, s0 + run);
+    if (s0 >= s1) return;
+    for (int slot = slot0; slot < sh.SL; slot += sstep) {
+        const ConvSlot c = conv_slot(sh, conv_w, conv_b, slot);
+        const float4 ysv = __ldcg(reinterpret_cast<const float4*>(ys + ((size_t)b * sh.T + t) * sh.E) + slot);
+        const float4 d0 = __ldg(reinterpret_cast<const float4*>(D) + slot);
+        const float4 d1 = sh.nd == 2 ? __ldg(reinterpret_cast<const float4*>(D + sh.E) + slot)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+        conv_line_run<true, 2>(sh, x, z, c, b, t, s0, s1, slot, [&](int s, const float4& a, const float4& bb,
+                                                                 const float4& zv) {
+            const size_t o = (size_t)s * st4 + slot;
+            const float4 sv = f4_fma(d1, bb, f4_fma(d0, a, ysv));
+            st_stream(y4 + o, make_float4(silu_fast(zv.x) * sv.x, silu_fast(zv.y) * sv.y, silu_fast(zv.z) * sv.z,
+                                          silu_fast(zv.w) * sv.w));
+        });
+    }
+}
+
+// The skip term sum_k D[k] * xc_k of one float4 slot of one token (i, j) of image b, loading the
+// token's sequence neighbours directly (the LayerNorm epilogue, which walks tokens, not runs).
+__device__ __forceinline__ float4 conv_skip_at(const Shape& sh, const float* __restrict__ x,
+                                               const float* __restrict__ conv_w, const float* __restrict__ conv_b,
+                                               const float* __restrict__ D, int b, int i, int j, int slot) {
+    const ConvSlot c = conv_slot(sh, conv_w, conv_b, slot);
+    const SeqPos p = sh.pool_axis == 0 ? SeqPos{i, j} : SeqPos{j, i};
+    SeqPos q = seq_back(sh, p, 3);
+    float4 win[7];
+#pragma unroll
+    for (int u = 0; u < 7; ++u) {
+        win[u] = seq_load(sh, reinterpret_cast<const float4*>(x), b, q, slot);
+        seq_step(sh, q);
+    }
+    const bool fwd0 = (sh.dir_flags & 1u) != 0;
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    s = f4_fma(__ldg(reinterpret_cast<const float4*>(D) + slot), conv_at(sh, c, 0, fwd0, win), s);
+    if (sh.nd == 2) s = f4_fma(__ldg(reinterpret_cast<const float4*>(D + sh.E) + slot), conv_at(sh, c, 1, false, win), s);
+    return s;
+}
+
 // ---- Staged epilogue with the post-SSM LayerNorm (dense and masked) ------------------------------
 // s = ys[t] + (sum_k D[k]) x;  y = SiLU(z) * (gamma * (s - mean) * rsqrt(var + eps) + beta), mean and
 // (biased) variance over the E channels of the token (summary page, "方法详解" item 5: repeat,
@@ -325,10 +569,12 @@ __host__ __forceinline__ size_t ln_epilogue_smem_bytes(const Shape& sh) {
     return (size_t)(3 + 2 * kLnWarps) * sh.SL * sizeof(float4);  // sum D, gamma, beta; per warp s and z rows
 }
 
+template <bool CONV>
 __global__ void __launch_bounds__(kLnWarps * 32)
 ln_epilogue_kernel(Shape sh, const float* __restrict__ x, const float* __restrict__ z,
                    const float* __restrict__ ys, const float* __restrict__ D, const float* __restrict__ gamma,
-                   const float* __restrict__ beta, const int32_t* __restrict__ row_of, float* __restrict__ y) {
+                   const float* __restrict__ beta, const int32_t* __restrict__ row_of,
+                   const float* __restrict__ conv_w, const float* __restrict__ conv_b, float* __restrict__ y) {
     extern __shared__ float4 lsm[];
     const int SL = sh.SL;
     float4* dsum = lsm;
@@ -368,8 +614,10 @@ ln_epilogue_kernel(Shape sh, const float* __restrict__ x, const float* __restric
             continue;
         }
         const float4* ys4 = reinterpret_cast<const float4*>(ys + ((size_t)b * sh.T + t) * sh.E);
-        // shift: the token's first s value (the same value in every lane)
-        const float K = fmaf(dsum[0].x, __ldcg(x + o * 4), __ldcg(ys + ((size_t)b * sh.T + t) * sh.E));
+        // shift: the token's first s value (the same value in every lane; with the Conv1D the
+        // first scan output, any value near the data will do)
+        const float K = CONV ? __ldcg(ys + ((size_t)b * sh.T + t) * sh.E)
+                                  : fmaf(dsum[0].x, __ldcg(x + o * 4), __ldcg(ys + ((size_t)b * sh.T + t) * sh.E));
         float m1 = 0.f, m2 = 0.f;
         for (int base = lane; base < SL; base += 32 * kLnBatch) {
             float4 xv[kLnBatch], zv[kLnBatch], yv[kLnBatch];
@@ -377,16 +625,26 @@ ln_epilogue_kernel(Shape sh, const float* __restrict__ x, const float* __restric
             for (int u = 0; u < kLnBatch; ++u) {
                 const int slot = base + 32 * u;
                 if (slot < SL) {
-                    xv[u] = ld_stream(x4 + o + slot);
+                    if (!CONV) xv[u] = ld_stream(x4 + o + slot);
                     zv[u] = ld_stream(z4 + o + slot);
                     yv[u] = __ldcg(ys4 + slot);
+                }
+            }
+            if (CONV) {  // the skip from each direction's convolved tokens, loaded by sequence position
+                const int i = (int)(r / sh.w), j = (int)(r - (long long)i * sh.w);
+#pragma unroll
+                for (int u = 0; u < kLnBatch; ++u) {
+                    const int slot = base + 32 * u;
+                    if (slot < SL) xv[u] = conv_skip_at(sh, x, conv_w, conv_b, D, b, i, j, slot);
                 }
             }
 #pragma unroll
             for (int u = 0; u < kLnBatch; ++u) {
                 const int slot = base + 32 * u;
                 if (slot < SL) {
-                    const float4 sv = f4_fma(dsum[slot], xv[u], yv[u]);
+                    const float4 sv = CONV ? make_float4(yv[u].x + xv[u].x, yv[u].y + xv[u].y, yv[u].z + xv[u].z,
+                                                              yv[u].w + xv[u].w)
+                                                : f4_fma(dsum[slot], xv[u], yv[u]);
                     srow[slot] = sv;
                     zrow[slot] = zv[u];
                     ln_accum(sv, K, m1, m2);
@@ -402,38 +660,51 @@ ln_epilogue_kernel(Shape sh, const float* __restrict__ x, const float* __restric
 
 // ---- Staged x_proj: one fp32 GEMM over every pooled token of the batch ---------------------------
 // u[b][k][t][j] = sum_e W_x[k][j][e] * xbar[b][t][e]: C[m][n] = sum_e A[m][e] B[n][e] with M = B T
-// pooled tokens, N = nd (R + 2N) outputs, K = E; both operands E-contiguous.  A CTA of 256 threads
-// computes a 64 x 32 tile: two groups of 128 threads each sum half of every 32-channel operand
-// tile (more warps to hide latency), each thread 4 tokens x 4 outputs (rows tg + 16 i, columns
-// og + 8 j), so a warp's 128-bit shared loads touch 4 A rows (broadcast) and 8 B rows (padded rows
-// of 36 floats: conflict-free); the groups' partial sums meet in shared memory at the end, in a
-// fixed order.  Operand tiles stream through a 3-stage cp.async pipeline.
+// pooled tokens, N = nd (R + 2N) outputs, K = E; both operands E-contiguous.  With the Conv1D each
+// direction has its own pooled tokens: blockIdx.z picks the set, and the set's GEMM covers only its
+// direction's R + 2N outputs.  A CTA of 256 threads computes a 64 x 32 tile: two groups of 128
+// threads each sum half of every 32-channel operand tile (more warps to hide latency), each thread
+// 4 tokens x 4 outputs (rows tg + 16 i, columns og + 8 j), so a warp's 128-bit shared loads touch 4
+// A rows (broadcast) and 8 B rows (padded rows of 36 floats: conflict-free); the groups' partial
+// sums meet in shared memory at the end, in a fixed order.  Operand tiles stream through a 3-stage
+// cp.async pipeline.
 constexpr int kPgM = 64, kPgN = 32, kPgK = 32, kPgPad = kPgK + 4, kPgStages = 3, kPgThreads = 256;
 constexpr size_t kPgSmemBytes = (size_t)kPgStages * (kPgM + kPgN) * kPgPad * sizeof(float);
 
 __global__ void __launch_bounds__(kPgThreads)
 proj_gemm_kernel(Shape sh, const float* __restrict__ xbar, const float* __restrict__ W_x, float* __restrict__ u) {
     extern __shared__ __align__(16) float pg[];
-    const int M = sh.B * sh.T, N = sh.NJ, K = sh.E;
+    const int kz = blockIdx.z;                        // pooled-token set
+    const int NZ = sh.NJ / sh.nx;                     // outputs of one set
+    const int M = sh.B * sh.T, N = NZ, K = sh.E;
     const int m0 = blockIdx.x * kPgM, n0 = blockIdx.y * kPgN;
     const int tid = threadIdx.x, grp = tid >> 7, og = tid & 7, tg = (tid & 127) >> 3;
     float* As = pg;                                   // [stages][64][36]
     float* Bs = pg + kPgStages * kPgM * kPgPad;       // [stages][32][36]
     const int nk = (K + kPgK - 1) / kPgK;
+    // the operand rows this thread copies: A rows ar and ar + 32, B row ar, channels k4 .. k4 + 3
+    const int ar = tid >> 3, k4 = (tid & 7) * 4;
+    const float* arow[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int m = m0 + ar + 32 * i;
+        const int mm = m < M ? m : 0;
+        const int b = mm / sh.T, t = mm - b * sh.T;
+        arow[i] = m < M ? xbar + xbar_offset(sh, b, kz, t) : nullptr;
+    }
+    const float* brow = n0 + ar < N ? W_x + (size_t)(kz * NZ + n0 + ar) * K : nullptr;
     auto issue = [&](int kt) {
         const int st = kt % kPgStages, k0 = kt * kPgK;
-        for (int c = tid; c < kPgM * (kPgK / 4); c += kPgThreads) {
-            const int r = c >> 3, k4 = (c & 7) * 4;
-            const bool ok = m0 + r < M && k0 + k4 < K;
-            cp_async16(As + (st * kPgM + r) * kPgPad + k4, ok ? (const void*)(xbar + (size_t)(m0 + r) * K + k0 + k4)
-                                                            : (const void*)xbar, ok ? 16u : 0u);
+        const bool kok = k0 + k4 < K;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const bool ok = arow[i] && kok;
+            cp_async16(As + (st * kPgM + ar + 32 * i) * kPgPad + k4, ok ? (const void*)(arow[i] + k0 + k4)
+                                                                        : (const void*)xbar, ok ? 16u : 0u);
         }
-        for (int c = tid; c < kPgN * (kPgK / 4); c += kPgThreads) {
-            const int r = c >> 3, k4 = (c & 7) * 4;
-            const bool ok = n0 + r < N && k0 + k4 < K;
-            cp_async16(Bs + (st * kPgN + r) * kPgPad + k4, ok ? (const void*)(W_x + (size_t)(n0 + r) * K + k0 + k4)
-                                                            : (const void*)W_x, ok ? 16u : 0u);
-        }
+        const bool ok = brow && kok;
+        cp_async16(Bs + (st * kPgN + ar) * kPgPad + k4, ok ? (const void*)(brow + k0 + k4) : (const void*)W_x,
+                   ok ? 16u : 0u);
     };
     float acc[4][4];
 #pragma unroll
@@ -487,7 +758,8 @@ proj_gemm_kernel(Shape sh, const float* __restrict__ xbar, const float* __restri
         for (int j = 0; j < 4; ++j) {
             const int n = n0 + og + 8 * j;
             if (n < N) {
-                const int k = n / sh.J, jc = n - k * sh.J;
+                const int ng = kz * NZ + n;
+                const int k = ng / sh.J, jc = ng - k * sh.J;
                 u[u_offset(sh, k, b, t) + jc] = acc[i][j] + part[tid * 16 + i * 4 + j];
             }
         }
@@ -505,7 +777,9 @@ scan_seq_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
     const int k = blockIdx.x % sh.nd;
     const int tile = (blockIdx.x / sh.nd) % tiles;
     const int b = blockIdx.x / (sh.nd * tiles);
-    seq_scan<kSeqThreads, 1, ZOH_EXACT>(sh, u, xbar, A_log, W_dt, b_dt, ys, b, tile * kSeqThreads, k, smem);
+    const int e0 = tile * kSeqThreads;
+    seq_scan<kSeqThreads, 1, ZOH_EXACT>(sh, u, xbar, A_log, W_dt, b_dt, ys + (size_t)b * sh.T * sh.E + e0, sh.E, b, e0,
+                                        k, smem);
 }
 
 // Device math self-test: out[i] = f(in[i]) for the SFU-based helpers the layer uses

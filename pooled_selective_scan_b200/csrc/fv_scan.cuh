@@ -110,27 +110,29 @@ __device__ __forceinline__ void seq_chunk(const float* __restrict__ bc, const fl
     }
 }
 
-// The scans of image b, channels [e0, e0 + NT / NDC), parameter slots k0 .. k0 + NDC - 1, by a
-// block of NT threads: thread (slot kk, channel c) = (threadIdx.x / (NT/NDC), threadIdx.x % (NT/NDC)).
-// u: projections (u_offset layout), xbar: pooled tokens [B][T][E], ys: [B][T][E] output, zeroed by
-// the caller when both directions are enabled.  smem: seq_smem_floats(NT, NDC, R) floats.
+// The scans of image b, channels [e0, e0 + NT / NDC), parameter slots k0 .. k0 + NDC - 1, by
+// threads 0 .. NT-1 of the CTA: thread (slot kk, channel c) = (threadIdx.x / (NT/NDC),
+// threadIdx.x % (NT/NDC)).  u: projections (u_offset layout), xbar: pooled tokens (xbar_offset:
+// with the Conv1D each direction reads its own).  The output of step t, channel e0 + c goes to
+// ys0[t * ys_stride + c] ([T][E] rows: ys0 = ys + b T E + e0), zeroed by the caller when both
+// directions add into it.  smem: seq_smem_floats(NT, NDC, R) floats.
 template <int NT, int NDC, bool ZOH_EXACT>
 __device__ __forceinline__ void seq_scan(const Shape& sh, const float* __restrict__ u, const float* __restrict__ xbar,
                                          const float* __restrict__ A_log, const float* __restrict__ W_dt,
-                                         const float* __restrict__ b_dt, float* __restrict__ ys, int b, int e0,
-                                         int k0, float* smem) {
+                                         const float* __restrict__ b_dt, float* __restrict__ ys0, int ys_stride, int b,
+                                         int e0, int k0, float* smem) {
     constexpr int NS = kSeqStates;
-    constexpr int ECH = NT / NDC;          // channels per direction
+    constexpr int ECH = NT / NDC;             // channels per direction
     const int T = sh.T, E = sh.E, N = sh.N, R = sh.R, J = sh.J;
     const int R4 = seq_r4(R), WS = seq_wstride(R);
     const int kk = threadIdx.x / ECH, c = threadIdx.x - kk * ECH;
     const int k = k0 + kk;
     const int e = e0 + c;
     const bool live = e < E;
-    float* sw = smem;                                       // [NT][WS]
-    float* sbc = sw + NT * WS;                              // [2][NDC][16][32]
-    float* sdt = sbc + 2 * NDC * kSeqChunk * 2 * NS;        // [2][NDC][R4][16]
-    float* sxs = sdt + 2 * NDC * R4 * kSeqChunk;            // [2][NDC][16][ECH]
+    float* sw = smem;                                            // [NT][WS]
+    float* sbc = sw + NT * WS;                                   // [2][NDC][16][32]
+    float* sdt = sbc + 2 * NDC * kSeqChunk * 2 * kSeqStates;     // [2][NDC][R4][16]
+    float* sxs = sdt + 2 * NDC * R4 * kSeqChunk;                 // [2][NDC][16][ECH]
     auto dir_fwd = [&](int kd) { return sh.nd == 2 ? kd == 0 : (sh.dir_flags & 1u) != 0; };
     const bool fwd = dir_fwd(k);
 
@@ -162,12 +164,12 @@ __device__ __forceinline__ void seq_scan(const Shape& sh, const float* __restric
             const int ci = f ? it : nchunks - 1 - it;
             const int t0 = ci * kSeqChunk, len = min(kSeqChunk, T - t0);
             const float* ub = u + u_offset(sh, k0 + kd, b, 0);
-            float* bcb = sbc + (buf * NDC + kd) * kSeqChunk * 2 * NS;
-            for (int i = threadIdx.x; i < kSeqChunk * 2 * NS; i += NT) {
+            float* bcb = sbc + (buf * NDC + kd) * kSeqChunk * 2 * kSeqStates;
+            for (int i = threadIdx.x; i < kSeqChunk * 2 * kSeqStates; i += NT) {
                 const int slot = i >> 5, j = i & 31, n = j & 15;
                 const int t = t0 + (f ? slot : len - 1 - slot);
                 const bool ok = slot < len && n < N;
-                cp_async4z(bcb + i, ok ? ub + (size_t)t * J + R + (j < NS ? n : N + n) : ub, ok);
+                cp_async4z(bcb + i, ok ? ub + (size_t)t * J + R + (j < kSeqStates ? n : N + n) : ub, ok);
             }
             float* dtb = sdt + (buf * NDC + kd) * R4 * kSeqChunk;
             for (int i = threadIdx.x; i < R4 * kSeqChunk; i += NT) {
@@ -181,8 +183,10 @@ __device__ __forceinline__ void seq_scan(const Shape& sh, const float* __restric
                 const int slot = v / (ECH / 4), c4 = (v - slot * (ECH / 4)) * 4;
                 const int t = t0 + (f ? slot : len - 1 - slot);
                 const bool ok = slot < len && e0 + c4 < E;
-                cp_async16(xb + slot * ECH + c4, ok ? (const void*)(xbar + ((size_t)b * T + t) * E + e0 + c4)
-                                                    : (const void*)xbar, ok ? 16u : 0u);
+                cp_async16(xb + slot * ECH + c4,
+                           ok ? (const void*)(xbar + xbar_offset(sh, b, sh.nx > 1 ? k0 + kd : 0, t) + e0 + c4)
+                              : (const void*)xbar,
+                           ok ? 16u : 0u);
             }
         }
         cp_async_commit();
@@ -201,9 +205,9 @@ __device__ __forceinline__ void seq_scan(const Shape& sh, const float* __restric
         const int ci = fwd ? it : nchunks - 1 - it;
         const int t0 = ci * kSeqChunk, len = min(kSeqChunk, T - t0);
         const int tfirst = fwd ? t0 : t0 + len - 1;
-        float* yp = ys + ((size_t)b * T + tfirst) * E + e;
-        const ptrdiff_t ystep = fwd ? (ptrdiff_t)E : -(ptrdiff_t)E;
-        const float* bcb = sbc + (buf * NDC + kk) * kSeqChunk * 2 * NS;
+        float* yp = ys0 + (size_t)tfirst * ys_stride + c;
+        const ptrdiff_t ystep = fwd ? (ptrdiff_t)ys_stride : -(ptrdiff_t)ys_stride;
+        const float* bcb = sbc + (buf * NDC + kk) * kSeqChunk * 2 * kSeqStates;
         const float* dtb = sdt + (buf * NDC + kk) * R4 * kSeqChunk;
         const float* xb = sxs + (buf * NDC + kk) * kSeqChunk * ECH + c;
         const float* wrow = sw + threadIdx.x * WS;

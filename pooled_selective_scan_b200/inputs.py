@@ -13,7 +13,10 @@ follow the usual Mamba/Vim initialisation that the layer is specified with:
            i.e. the value whose softplus is Delta0 (the initial step sizes are log-uniform);
   keep_idx[b] = default_rng([seed, 3, b]).permutation(h*w)[:K] (int32, unsorted) for a masked
            layer at keep ratio K / (h*w);
-  dy     ~ N(0, 1) fp32, the upstream gradient of a training step, default_rng([seed, 4, b]).
+  dy     ~ N(0, 1) fp32, the upstream gradient of a training step, default_rng([seed, 4, b]);
+  the block's Conv1D (per direction slot, stream default_rng([seed, 5])): taps and bias
+           ~ U(-1/sqrt(d_conv), 1/sqrt(d_conv)), the default initialisation of a depthwise
+           torch Conv1d (fan-in d_conv).
 """
 from __future__ import annotations
 
@@ -80,3 +83,12 @@ def layer_inputs(cfg: LayerConfig, which=None) -> dict:
     d = params(cfg.E, cfg.N, cfg.R, cfg.nd, cfg.seed)
     d.update(images(cfg, which))
     return d
+
+
+def conv_params(E: int, d_conv: int, nd: int, seed: int) -> dict:
+    """Weights of the block's Conv1D: conv_w [nd, E, d_conv], conv_b [nd, E]."""
+    rng = np.random.default_rng([seed, 5])
+    bound = 1.0 / np.sqrt(d_conv)
+    w = rng.uniform(-bound, bound, size=(nd, E, d_conv)).astype(np.float32)
+    b = rng.uniform(-bound, bound, size=(nd, E)).astype(np.float32)
+    return dict(conv_w=w, conv_b=b)

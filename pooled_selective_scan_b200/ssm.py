@@ -8,6 +8,8 @@ CUDA device; parameters are stacked per enabled direction (slot 0 = forward when
 
 Dense layer:  x, z [B,h,w,E] -> y [B,h,w,E].
 Masked layer: x, z [B,K,E] with keep_idx [B,K] (grid ids r*w + c of an h x w grid) -> y [B,K,E].
+With the block's Conv1D (dense layers): conv_w [nd,E,d_conv], conv_b [nd,E]; x is then the Conv1D's
+input.
 """
 from __future__ import annotations
 
@@ -66,6 +68,8 @@ class LayerShape:
     path: str = "auto"  # "auto", "staged" or "fused" (FV_FLAG_PATH_*)
     ln: bool = False    # post-SSM LayerNorm before the gate (FV_FLAG_LAYERNORM)
     ln_eps: float = 1e-5
+    d_conv: int = 0     # taps of the block's Conv1D in front of the layer (0: none)
+    conv_silu: bool = False  # SiLU after the Conv1D (FV_FLAG_CONV_SILU)
 
     @property
     def nd(self) -> int:
@@ -79,7 +83,7 @@ class LayerShape:
         return (self.B, self.K, self.E) if self.K else (self.B, self.h, self.w, self.E)
 
     def args(self, x=None, z=None, A_log=None, D=None, W_x=None, W_dt=None, b_dt=None, keep_idx=None,
-             y=None, ln_gamma=None, ln_beta=None) -> nat.FvSsmArgs:
+             y=None, ln_gamma=None, ln_beta=None, conv_w=None, conv_b=None) -> nat.FvSsmArgs:
         a = nat.FvSsmArgs()
         a.B, a.h, a.w, a.E, a.N, a.R = self.B, self.h, self.w, self.E, self.N, self.R
         a.pool_axis = self.pool_axis
@@ -87,16 +91,18 @@ class LayerShape:
         a.K = self.K
         a.pool_scale = float(self.pool_scale)
         a.flags = ((nat.FV_FLAG_ZOH_EXACT if self.zoh_exact else 0) | _PATH_FLAGS[self.path] |
-                   (nat.FV_FLAG_LAYERNORM if self.ln else 0))
+                   (nat.FV_FLAG_LAYERNORM if self.ln else 0) | (nat.FV_FLAG_CONV_SILU if self.conv_silu else 0))
         a.x, a.z, a.A_log, a.D, a.W_x, a.W_dt, a.b_dt, a.keep_idx, a.y = (
             _ptr(x), _ptr(z), _ptr(A_log), _ptr(D), _ptr(W_x), _ptr(W_dt), _ptr(b_dt), _ptr(keep_idx), _ptr(y))
         a.ln_gamma, a.ln_beta = _ptr(ln_gamma), _ptr(ln_beta)
         a.ln_eps = float(self.ln_eps)
+        a.d_conv = int(self.d_conv)
+        a.conv_w, a.conv_b = _ptr(conv_w), _ptr(conv_b)
         return a
 
 
 def infer_shape(x, A_log, W_dt, pool_axis, dir_flags, keep_idx=None, h=None, w=None, pool_scale=1.0,
-                zoh_exact=False, path="auto", ln=False, ln_eps=1e-5) -> LayerShape:
+                zoh_exact=False, path="auto", ln=False, ln_eps=1e-5, d_conv=0, conv_silu=False) -> LayerShape:
     nd, E, N = A_log.shape
     R = W_dt.shape[2]
     if keep_idx is None:
@@ -114,7 +120,8 @@ def infer_shape(x, A_log, W_dt, pool_axis, dir_flags, keep_idx=None, h=None, w=N
         raise ValueError(f"x has E={E2}, parameters have E={E}")
     if path not in _PATH_FLAGS:
         raise ValueError(f"path must be one of {sorted(_PATH_FLAGS)}")
-    s = LayerShape(B, h, w, E, N, R, pool_axis, dir_flags, K, pool_scale, zoh_exact, path, bool(ln), float(ln_eps))
+    s = LayerShape(B, h, w, E, N, R, pool_axis, dir_flags, K, pool_scale, zoh_exact, path, bool(ln), float(ln_eps),
+                   int(d_conv), bool(conv_silu))
     if s.nd != nd:
         raise ValueError(f"dir_flags={dir_flags} enables {s.nd} directions, parameters stack {nd}")
     return s
@@ -151,9 +158,10 @@ def alloc_workspace(shape: LayerShape, device=None) -> torch.Tensor:
 
 def forward(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis=POOL_W, dir_flags=DIR_FWD | DIR_BWD, keep_idx=None,
             h=None, w=None, pool_scale=1.0, zoh_exact=False, y=None, workspace=None, stream=None, path="auto",
-            ln_gamma=None, ln_beta=None, ln_eps=1e-5):
+            ln_gamma=None, ln_beta=None, ln_eps=1e-5, conv_w=None, conv_b=None, conv_silu=False):
     """Queue the layer on ``stream`` (default: the current stream) and return y.  Passing
-    ln_gamma and ln_beta ([E]) adds the post-SSM LayerNorm before the gate."""
+    ln_gamma and ln_beta ([E]) adds the post-SSM LayerNorm before the gate; conv_w [nd,E,d_conv]
+    and conv_b [nd,E] put the block's Conv1D in front (x is then the Conv1D's input)."""
     dev = x.device
     for name, t in (("x", x), ("z", z), ("A_log", A_log), ("D", D), ("W_x", W_x), ("W_dt", W_dt), ("b_dt", b_dt)):
         _check_tensor(name, t, torch.float32, dev)
@@ -165,7 +173,15 @@ def forward(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis=POOL_W, dir_flags=DIR_FWD
             raise ValueError("the LayerNorm needs both ln_gamma and ln_beta")
         _check_tensor("ln_gamma", ln_gamma, torch.float32, dev)
         _check_tensor("ln_beta", ln_beta, torch.float32, dev)
-    shape = infer_shape(x, A_log, W_dt, pool_axis, dir_flags, keep_idx, h, w, pool_scale, zoh_exact, path, ln, ln_eps)
+    d_conv = 0
+    if conv_w is not None or conv_b is not None:
+        if conv_w is None or conv_b is None:
+            raise ValueError("the Conv1D needs both conv_w and conv_b")
+        _check_tensor("conv_w", conv_w, torch.float32, dev)
+        _check_tensor("conv_b", conv_b, torch.float32, dev)
+        d_conv = conv_w.shape[-1]
+    shape = infer_shape(x, A_log, W_dt, pool_axis, dir_flags, keep_idx, h, w, pool_scale, zoh_exact, path, ln, ln_eps,
+                        d_conv, conv_silu)
     if z.shape != x.shape:
         raise ValueError("z must have the shape of x")
     if y is None:
@@ -176,7 +192,7 @@ def forward(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis=POOL_W, dir_flags=DIR_FWD
             raise ValueError("y must have the shape of x")
     if workspace is None:
         workspace = alloc_workspace(shape, dev)
-    a = shape.args(x, z, A_log, D, W_x, W_dt, b_dt, keep_idx, y, ln_gamma, ln_beta)
+    a = shape.args(x, z, A_log, D, W_x, W_dt, b_dt, keep_idx, y, ln_gamma, ln_beta, conv_w, conv_b)
     st = nat.lib().fastvim_ssm_forward(ctypes.byref(a), ctypes.c_void_p(workspace.data_ptr()),
                                        ctypes.c_size_t(workspace.numel()), _stream_handle(stream))
     nat.check(st, "fastvim_ssm_forward")
@@ -193,7 +209,7 @@ class BoundForward:
         self.workspace = workspace
         self._keep = (t, y, workspace)
         self._args = shape.args(t["x"], t["z"], t["A_log"], t["D"], t["W_x"], t["W_dt"], t["b_dt"], t.get("keep_idx"), y,
-                                t.get("ln_gamma"), t.get("ln_beta"))
+                                t.get("ln_gamma"), t.get("ln_beta"), t.get("conv_w"), t.get("conv_b"))
         self._stream = _stream_handle(stream)
         self._ws = ctypes.c_void_p(workspace.data_ptr())
         self._wsn = ctypes.c_size_t(workspace.numel())
@@ -334,13 +350,16 @@ class HostForward:
         self.dev["keep_idx"] = (torch.empty((shape.B, shape.K), dtype=torch.int32, device=dev) if shape.K else None)
         self.dev["ln_gamma"] = mk(E) if shape.ln else None
         self.dev["ln_beta"] = mk(E) if shape.ln else None
+        self.dev["conv_w"] = mk(nd, E, shape.d_conv) if shape.d_conv else None
+        self.dev["conv_b"] = mk(nd, E) if shape.d_conv else None
         self.workspace = alloc_workspace(shape, dev)
 
     def h2d_bytes(self) -> int:
         s = self.shape
         act = 2 * s.B * (s.K if s.K else s.h * s.w) * s.E * 4
         par = s.nd * (s.E * s.N + 2 * s.E + (s.R + 2 * s.N) * s.E + s.E * s.R) * 4
-        return act + par + (s.B * s.K * 4 if s.K else 0) + (2 * s.E * 4 if s.ln else 0)
+        conv = s.nd * s.E * (s.d_conv + 1) * 4 if s.d_conv else 0
+        return act + par + (s.B * s.K * 4 if s.K else 0) + (2 * s.E * 4 if s.ln else 0) + conv
 
     def d2h_bytes(self) -> int:
         s = self.shape
@@ -352,9 +371,10 @@ class HostForward:
         _check_tensor("y", y_host, torch.float32, host=True)
         d = self.dev
         ha = self.shape.args(host["x"], host["z"], host["A_log"], host["D"], host["W_x"], host["W_dt"], host["b_dt"],
-                             host.get("keep_idx"), y_host, host.get("ln_gamma"), host.get("ln_beta"))
+                             host.get("keep_idx"), y_host, host.get("ln_gamma"), host.get("ln_beta"),
+                             host.get("conv_w"), host.get("conv_b"))
         da = self.shape.args(d["x"], d["z"], d["A_log"], d["D"], d["W_x"], d["W_dt"], d["b_dt"], d["keep_idx"], d["y"],
-                             d["ln_gamma"], d["ln_beta"])
+                             d["ln_gamma"], d["ln_beta"], d["conv_w"], d["conv_b"])
         st = nat.lib().fastvim_ssm_forward_host(ctypes.byref(ha), ctypes.byref(da),
                                                 ctypes.c_void_p(self.workspace.data_ptr()),
                                                 ctypes.c_size_t(self.workspace.numel()), _stream_handle(stream))

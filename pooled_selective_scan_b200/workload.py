@@ -68,6 +68,12 @@ def ln_tensors(cfg: LayerConfig, device) -> dict:
                 ln_beta=torch.zeros(cfg.E, dtype=torch.float32, device=device))
 
 
+def conv_tensors(cfg: LayerConfig, device, d_conv: int = 4) -> dict:
+    """The block's Conv1D weights (seeded, default depthwise Conv1d initialisation)."""
+    c = inputs.conv_params(cfg.E, d_conv, cfg.nd, cfg.seed)
+    return {k: torch.from_numpy(v).to(device) for k, v in c.items()}
+
+
 def layer_tensors(cfg: LayerConfig, device, pinned_host: bool = False, first_image: int = 0) -> dict:
     d = params_tensors(cfg, "cpu" if pinned_host else device)
     if pinned_host:

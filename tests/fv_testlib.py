@@ -50,22 +50,27 @@ def assert_close(got, ref, what="y", abs_rms=ABS_RMS):
 def gpu_forward(inp: dict, pool_axis: int, dir_flags: int, h=None, w=None, pool_scale=1.0, zoh_exact=False,
                 intermediates=True, path="auto", ln_eps=1e-5):
     """Run the CUDA layer on numpy inputs; return y (and workspace intermediates) as numpy.  The
-    post-SSM LayerNorm runs when inp holds ln_gamma and ln_beta."""
+    post-SSM LayerNorm runs when inp holds ln_gamma and ln_beta, the block's Conv1D when it holds
+    conv_w and conv_b (conv_silu: a bool entry)."""
     import torch
 
     from pooled_selective_scan_b200 import ssm
 
     dev = torch.device("cuda")
-    t = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev) for k, v in inp.items() if v is not None}
+    conv_silu = bool(inp.get("conv_silu", False))
+    t = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev) for k, v in inp.items()
+         if v is not None and k != "conv_silu"}
     keep = t.get("keep_idx")
     ln = "ln_gamma" in t
+    d_conv = t["conv_w"].shape[-1] if "conv_w" in t else 0
     shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, dir_flags, keep, h, w, pool_scale, zoh_exact,
-                            path, ln, ln_eps)
+                            path, ln, ln_eps, d_conv, conv_silu)
     ws = ssm.alloc_workspace(shape, dev)
     ws.fill_(0xFF)  # poison: every intermediate must be written before it is read
     y = ssm.forward(t["x"], t["z"], t["A_log"], t["D"], t["W_x"], t["W_dt"], t["b_dt"], pool_axis, dir_flags,
                     keep_idx=keep, h=h, w=w, pool_scale=pool_scale, zoh_exact=zoh_exact, workspace=ws, path=path,
-                    ln_gamma=t.get("ln_gamma"), ln_beta=t.get("ln_beta"), ln_eps=ln_eps)
+                    ln_gamma=t.get("ln_gamma"), ln_beta=t.get("ln_beta"), ln_eps=ln_eps, conv_w=t.get("conv_w"),
+                    conv_b=t.get("conv_b"), conv_silu=conv_silu)
     status = ssm.device_status(ws)
     out = dict(y=y.cpu().numpy(), status=status, launches=ssm.launch_names(shape))
     if intermediates:
@@ -76,7 +81,9 @@ def gpu_forward(inp: dict, pool_axis: int, dir_flags: int, h=None, w=None, pool_
             nbytes = count * np.dtype(dtype).itemsize
             return ws[off:off + nbytes].cpu().numpy().view(dtype).copy()
 
-        out["xbar"] = view(L["xbar"], B * T * E, np.float32).reshape(B, T, E)
+        nx = nd if d_conv else 1
+        xb = view(L["xbar"], B * nx * T * E, np.float32).reshape(B, nx, T, E)
+        out["xbar"] = xb if d_conv else xb[:, 0]
         ub = -(-T * J // 32) * 32  # per (direction, image) block stride, floats
         out["u"] = (view(L["u"], nd * B * ub, np.float32).reshape(B, nd, ub)[:, :, :T * J].reshape(B, nd, T, J)
                     .transpose(1, 0, 2, 3))

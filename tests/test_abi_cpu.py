@@ -52,14 +52,16 @@ def test_header_compiles_as_plain_c(tmp_path):
 def test_struct_layout_matches_header(tmp_path):
     src = tmp_path / "off.c"
     src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "fastvim_ssm.h"\n'
-                   'int main(void){printf("%zu %zu %zu %zu %zu\\n", sizeof(fv_ssm_args), '
+                   'int main(void){printf("%zu %zu %zu %zu %zu %zu %zu %zu\\n", sizeof(fv_ssm_args), '
                    'offsetof(fv_ssm_args, pool_scale), offsetof(fv_ssm_args, x), offsetof(fv_ssm_args, y), '
-                   'sizeof(fv_ws_layout)); return 0;}\n')
+                   'sizeof(fv_ws_layout), offsetof(fv_ssm_args, d_conv), offsetof(fv_ssm_args, conv_w), '
+                   'offsetof(fv_ssm_args, conv_b)); return 0;}\n')
     exe = tmp_path / "off"
     subprocess.run(["gcc", "-std=c99", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)], check=True)
     got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
     want = [ctypes.sizeof(nat.FvSsmArgs), nat.FvSsmArgs.pool_scale.offset, nat.FvSsmArgs.x.offset,
-            nat.FvSsmArgs.y.offset, ctypes.sizeof(nat.FvWsLayout)]
+            nat.FvSsmArgs.y.offset, ctypes.sizeof(nat.FvWsLayout), nat.FvSsmArgs.d_conv.offset,
+            nat.FvSsmArgs.conv_w.offset, nat.FvSsmArgs.conv_b.offset]
     assert got == want
 
 
@@ -67,7 +69,7 @@ def test_status_strings(lib):
     assert nat.status_string(0) == "FV_OK"
     for s in range(1, 10):
         assert nat.status_string(s).startswith("FV_ERR_")
-    assert lib.fastvim_abi_version() == 3
+    assert lib.fastvim_abi_version() == 4
 
 
 # ---------------------------------------------------------------------------------------------
@@ -208,7 +210,7 @@ def test_layernorm_arguments(lib):
         assert validate(good_args(flags=LN, ln_gamma=g, ln_beta=b, ln_eps=eps)) == nat.FV_ERR_SHAPE
     assert validate(good_args(flags=LN, ln_gamma=g + 4, ln_beta=b, ln_eps=1e-5)) == nat.FV_ERR_ALIGN
     assert validate(good_args(flags=LN, ln_gamma=g, ln_beta=b, ln_eps=1e-5, E=4100)) == nat.FV_ERR_UNSUPPORTED
-    assert lib.fastvim_abi_version() == 3
+    assert lib.fastvim_abi_version() == 4
 
 
 def test_layernorm_launches(lib):
@@ -239,3 +241,57 @@ def test_staged_launch_order(lib, masked, ln):
     want = front + middle + back
     n = lib.fastvim_ssm_launch_count(ctypes.byref(a))
     assert [lib.fastvim_ssm_launch_name(ctypes.byref(a), i).decode() for i in range(n)] == want
+
+
+# ---------------------------------------------------------------------------------------------
+# The block's Conv1D in front of the layer (d_conv, conv_w, conv_b, FV_FLAG_CONV_SILU).
+# ---------------------------------------------------------------------------------------------
+CW, CB = FAKE + (12 << 32), FAKE + (13 << 32)
+
+
+def test_conv_arguments(lib):
+    assert validate(good_args(d_conv=4, conv_w=CW, conv_b=CB)) == nat.FV_OK
+    assert validate(good_args(d_conv=1, conv_w=CW, conv_b=CB, flags=nat.FV_FLAG_CONV_SILU)) == nat.FV_OK
+    assert validate(good_args(d_conv=4, conv_w=None, conv_b=CB)) == nat.FV_ERR_NULL
+    assert validate(good_args(d_conv=4, conv_w=CW, conv_b=None)) == nat.FV_ERR_NULL
+    assert validate(good_args(conv_w=CW, conv_b=CB)) == nat.FV_ERR_SHAPE          # weights without taps
+    assert validate(good_args(flags=nat.FV_FLAG_CONV_SILU)) == nat.FV_ERR_SHAPE   # SiLU of no Conv1D
+    assert validate(good_args(d_conv=-1)) == nat.FV_ERR_SHAPE
+    assert validate(good_args(d_conv=5, conv_w=CW, conv_b=CB)) == nat.FV_ERR_UNSUPPORTED
+    assert validate(good_args(d_conv=4, conv_w=CW + 4, conv_b=CB)) == nat.FV_ERR_ALIGN
+    masked = good_args(d_conv=4, conv_w=CW, conv_b=CB, K=49, keep_idx=FAKE + (9 << 32))
+    assert validate(masked) == nat.FV_ERR_UNSUPPORTED
+
+
+def test_conv_launches_and_workspace(lib):
+    a = good_args(d_conv=4, conv_w=CW, conv_b=CB)
+    n = lib.fastvim_ssm_launch_count(ctypes.byref(a))
+    names = [lib.fastvim_ssm_launch_name(ctypes.byref(a), i).decode() for i in range(n)]
+    assert names == ["pool_conv_kernel", "proj_gemm_kernel", "scan_seq_kernel", "epilogue_conv_kernel"]
+    ln = good_args(d_conv=4, conv_w=CW, conv_b=CB, flags=nat.FV_FLAG_LAYERNORM, ln_gamma=FAKE + (10 << 32),
+                   ln_beta=FAKE + (11 << 32), ln_eps=1e-5)
+    assert lib.fastvim_ssm_launch_name(ctypes.byref(ln), 3).decode() == "ln_epilogue_kernel"
+    # large images take the staged kernels with the Conv1D; forcing the single launch is refused
+    big = good_args(h=128, w=128, d_conv=4, conv_w=CW, conv_b=CB)
+    assert lib.fastvim_ssm_launch_name(ctypes.byref(big), 0).decode() == "pool_conv_kernel"
+    assert lib.fastvim_ssm_launch_count(ctypes.byref(good_args(h=128, w=128, d_conv=4, conv_w=CW, conv_b=CB,
+                                                                flags=nat.FV_FLAG_PATH_FUSED))) == 0
+    # each direction pools its own convolved tokens: two sets of pooled tokens
+    L0, L1 = nat.FvWsLayout(), nat.FvWsLayout()
+    assert lib.fastvim_ssm_workspace_layout(ctypes.byref(good_args()), ctypes.byref(L0)) == nat.FV_OK
+    assert lib.fastvim_ssm_workspace_layout(ctypes.byref(a), ctypes.byref(L1)) == nat.FV_OK
+    assert L1.u - L1.xbar == 2 * (L0.u - L0.xbar)
+    one = good_args(dir_flags=2, d_conv=2, conv_w=CW, conv_b=CB)
+    assert lib.fastvim_ssm_workspace_layout(ctypes.byref(one), ctypes.byref(L1)) == nat.FV_OK
+    assert L1.u - L1.xbar == L0.u - L0.xbar
+
+
+def test_conv_gradient_not_built(lib):
+    a = good_args(d_conv=4, conv_w=CW, conv_b=CB)
+    g = nat.FvSsmGrads()
+    for i, name in enumerate(("dy", "dx", "dz", "dA_log", "dD", "dW_x", "dW_dt", "db_dt")):
+        setattr(g, name, FAKE + ((20 + i) << 32))
+    st = lib.fastvim_ssm_backward(ctypes.byref(a), ctypes.byref(g), ctypes.c_void_p(FAKE + (40 << 32)),
+                                  ctypes.c_size_t(1 << 30), ctypes.c_void_p(FAKE + (41 << 32)), ctypes.c_size_t(1 << 30),
+                                  None)
+    assert st == nat.FV_ERR_UNSUPPORTED

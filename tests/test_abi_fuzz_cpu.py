@@ -130,9 +130,12 @@ def _check_launches(lib, a):
         assert a.K == 0 and not a.flags & nat.FV_FLAG_PATH_STAGED
         return
     assert not a.flags & nat.FV_FLAG_PATH_FUSED
-    assert n >= 4 and "fused_layer_kernel" not in names
-    last = {True: "ln_epilogue_kernel", False: "mask_epilogue_kernel" if a.K else "epilogue_dense_kernel"}
-    assert names[-1] == last[bool(a.flags & nat.FV_FLAG_LAYERNORM)]
+    assert "fused_layer_kernel" not in names
+    full = 5 if a.K else 4  # pooling (masked: bucketing, pooling), x_proj, scans, epilogue
+    if a.flags & nat.FV_FLAG_LAYERNORM:
+        assert n == full and names[-1] == "ln_epilogue_kernel"
+    else:
+        assert n == full and names[-1] == ("mask_epilogue_kernel" if a.K else "epilogue_dense_kernel")
     assert "proj_gemm_kernel" in names and any(k.startswith("scan") for k in names)
     if a.K:
         assert names[0].startswith("mask_")

@@ -32,6 +32,10 @@ def test_every_launched_kernel_has_a_bound(cfg):
         for path in (("auto", "staged", "fused") if not cfg.masked else ("auto",)):
             names |= set(ssm.launch_names(_shape(cfg, axis, path)))
         names |= set(ssm.launch_names(_shape(cfg, axis, "auto", ln=True)))
+        if not cfg.masked:
+            conv = _shape(cfg, axis)
+            conv.d_conv = 4
+            names |= set(ssm.launch_names(conv))
         names |= set(ssm.backward_launch_names(_shape(cfg, axis)))
         names |= set(ssm.backward_launch_names(_shape(cfg, axis, ln=True)))
         for n in names:
@@ -90,6 +94,9 @@ def test_secondary_workloads_cover_every_config_and_axis():
     from pooled_selective_scan_b200.configs import by_name
     want = {(c.name, ax) for c in CONFIGS for ax in c.pool_axes} - {(bench.HEADLINE_NAME, 0)}
     assert set(bench.SECONDARY) == want
+    assert (bench.HEADLINE_NAME, 0, 4, "auto") in bench.SECONDARY_VARIANTS
+    for name, axis, taps, path in bench.SECONDARY_VARIANTS:
+        assert axis in by_name(name).pool_axes and path in ("auto", "staged", "fused")
     for name, axis in bench.SECONDARY:
         assert axis in by_name(name).pool_axes
     assert bench.parse(["--no-configs"]).no_configs

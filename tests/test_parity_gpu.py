@@ -39,8 +39,8 @@ def rand_layer(seed, B, h, w, E, N, R, dir_flags, K=0, dt_hi=0.1):
 
 
 def check_layer(p, pool_axis, dir_flags, h=None, w=None, pool_scale=1.0, zoh_exact=False):
-    """Both implementations of a dense layer (staged kernels and the fused launch), or the staged
-    masked one, against the oracle: intermediates and output."""
+    """Every implementation of the layer against the oracle, intermediates and output: the staged
+    kernels and (dense) the single persistent launch."""
     keep = p.get("keep_idx")
     ref = oracle.forward_intermediates(p["x"], p["z"], p["A_log"], p["D"], p["W_x"], p["W_dt"], p["b_dt"],
                                        pool_axis, dir_flags, keep_idx=keep, h=h, w=w, pool_scale=pool_scale,
