@@ -61,8 +61,8 @@ def kernel_work(name: str, cfg, pool_axis: int):
     T = cfg.h if pool_axis == 0 else cfg.w
     if name in ("pool_dense_kernel", "mask_pool_kernel", "pool_conv_kernel"):
         return "hbm", row * tok                       # read x (with the Conv1D: its input)
-    if name in ("epilogue_dense_kernel", "mask_epilogue_kernel", "ln_epilogue_kernel", "fused_layer_kernel",
-                "epilogue_conv_kernel"):
+    if name in ("epilogue_dense_kernel", "mask_epilogue_kernel", "ln_epilogue_kernel", "ln_epilogue_reg_kernel",
+                "fused_layer_kernel", "epilogue_conv_kernel"):
         return "hbm", 3 * row * tok                   # read x and z, write y (the fused launch: the layer)
     if name == "scan_seq_kernel":
         return "alu", cfg.B * T * cfg.E * cfg.N * cfg.nd

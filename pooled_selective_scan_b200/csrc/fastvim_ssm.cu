@@ -109,6 +109,7 @@ fv_status check_pointers(const fv_ssm_args* a, const fv::Shape& sh) {
 }
 
 enum class Path { Staged, Fused, Invalid };
+int device_sm_count();
 Path choose_path(const fv::Shape& sh);
 fv::FusedPlan plan_fused(const fv::Shape& sh);
 
@@ -278,6 +279,10 @@ struct EventMarks {
         }                                                      \
     } while (0)
 
+// The post-SSM LayerNorm epilogue keeps each lane's share of a token in registers up to 1536
+// channels (without the Conv1D, whose skip needs each token's sequence neighbours).
+bool ln_uses_reg_kernel(const fv::Shape& sh) { return sh.dc == 0 && fv::ln_reg_nsl(sh.SL) > 0; }
+
 // Launches of a staged call: pool (masked: bucket, pool), x_proj, scans, epilogue.
 int launch_count_of(const fv::Shape& sh) {
     if (sh.B == 0) return 0;
@@ -296,7 +301,7 @@ const char* launch_name_of(const fv::Shape& sh, int i) {
     const int n = launch_count_of(sh);
     if (i < 0 || i >= n) return "";
     if (choose_path(sh) == Path::Fused) return "fused_layer_kernel";
-    if (sh.ln && i == n - 1) return "ln_epilogue_kernel";
+    if (sh.ln && i == n - 1) return ln_uses_reg_kernel(sh) ? "ln_epilogue_reg_kernel" : "ln_epilogue_kernel";
     return sh.K > 0 ? masked[i] : (sh.dc > 0 ? conv[i] : dense[i]);
 }
 
@@ -431,7 +436,35 @@ fv_status staged_middle(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_l
 fv_status staged_back(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st,
                       EventMarks& marks) {
     const float* ys = (const float*)(ws + L.ys);
-    if (sh.ln) {
+    if (sh.ln && ln_uses_reg_kernel(sh)) {
+        const size_t smem = (size_t)3 * sh.SL * sizeof(float4);
+        const int nsl = fv::ln_reg_nsl(sh.SL);
+        auto kern = nsl == 1 ? fv::ln_epilogue_reg_kernel<1> : nsl == 2 ? fv::ln_epilogue_reg_kernel<2>
+                  : nsl == 3 ? fv::ln_epilogue_reg_kernel<3> : nsl == 4 ? fv::ln_epilogue_reg_kernel<4>
+                  : nsl == 6 ? fv::ln_epilogue_reg_kernel<6> : nsl == 8 ? fv::ln_epilogue_reg_kernel<8>
+                  : fv::ln_epilogue_reg_kernel<12>;
+        cudaError_t e = ensure_smem(kern, smem);
+        if (e != cudaSuccess) { note_cuda(e, "LayerNorm epilogue smem attribute"); return FV_ERR_CUDA; }
+        int per_sm = 0;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, fv::kLnRegWarps * 32, smem)) !=
+            cudaSuccess) {
+            note_cuda(e, "LayerNorm epilogue occupancy");
+            return FV_ERR_CUDA;
+        }
+        const long long ntok = (long long)sh.B * (sh.K > 0 ? (long long)sh.K : (long long)sh.h * sh.w);
+        // persistent over tokens: four waves of resident blocks, a warp per token at a time
+        long long grid = (long long)std::max(per_sm, 1) * device_sm_count() * 4;
+        const long long need = (ntok + fv::kLnRegWarps - 1) / fv::kLnRegWarps;
+        if (grid > need) grid = need;
+        FV_MARK_CALL(marks, st, ([&]() -> fv_status {
+            kern<<<(unsigned)grid, fv::kLnRegWarps * 32, smem, st>>>(sh, a->x, a->z, ys, a->D, a->ln_gamma, a->ln_beta,
+                                                                     sh.K > 0 ? (const int32_t*)(ws + L.row_of)
+                                                                              : nullptr,
+                                                                     a->y);
+            FV_LAUNCH_CHECK("ln_epilogue_reg_kernel");
+            return FV_OK;
+        })());
+    } else if (sh.ln) {
         const size_t smem = fv::ln_epilogue_smem_bytes(sh);
         auto kern = sh.dc > 0 ? fv::ln_epilogue_kernel<true> : fv::ln_epilogue_kernel<false>;
         cudaError_t e = ensure_smem(kern, smem);

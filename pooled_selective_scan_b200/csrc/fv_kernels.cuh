@@ -658,6 +658,83 @@ ln_epilogue_kernel(Shape sh, const float* __restrict__ x, const float* __restric
     }
 }
 
+// The same epilogue for rows of up to 1536 channels (without the Conv1D), with each lane's share of
+// the token's s = ys[t] + (sum D) x held in registers (NSL float4 slots per lane) instead of
+// shared-memory rows: eight warps per CTA and no per-warp shared memory, so occupancy is set by
+// registers alone.  Per token: x and ys are loaded, s and its shifted moments formed, the warp
+// reduction gives the mean and 1/sqrt(var + eps); then z is loaded and y stored.
+constexpr int kLnRegWarps = 8;
+__host__ __device__ __forceinline__ int ln_reg_nsl(int SL) {
+    const int need = (SL + 31) / 32;
+    return need <= 4 ? need : (need <= 6 ? 6 : (need <= 8 ? 8 : (need <= 12 ? 12 : 0)));
+}
+
+template <int NSL>
+__global__ void __launch_bounds__(kLnRegWarps * 32)
+ln_epilogue_reg_kernel(Shape sh, const float* __restrict__ x, const float* __restrict__ z,
+                       const float* __restrict__ ys, const float* __restrict__ D, const float* __restrict__ gamma,
+                       const float* __restrict__ beta, const int32_t* __restrict__ row_of, float* __restrict__ y) {
+    extern __shared__ float4 lrs[];
+    const int SL = sh.SL;
+    float4* dsum = lrs;
+    float4* g4 = dsum + SL;
+    float4* b4 = g4 + SL;
+    for (int slot = threadIdx.x; slot < SL; slot += kLnRegWarps * 32) {
+        dsum[slot] = dsum4(D, sh.nd, SL, slot);
+        g4[slot] = __ldg(reinterpret_cast<const float4*>(gamma) + slot);
+        b4[slot] = __ldg(reinterpret_cast<const float4*>(beta) + slot);
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long per_img = sh.K > 0 ? (long long)sh.K : (long long)sh.h * sh.w;
+    const long long ntok = (long long)sh.B * per_img;
+    const float invE = 1.f / (float)sh.E;
+    // this lane's slots are lane + 32 u: one base pointer per tensor, constant offsets per slot
+    const int nsl = (SL - lane + 31) >> 5;  // slots of this lane
+    const float4* dl = dsum + lane;
+    const float4* gl = g4 + lane;
+    const float4* bl = b4 + lane;
+    for (long long tok = (long long)blockIdx.x * kLnRegWarps + warp; tok < ntok;
+         tok += (long long)gridDim.x * kLnRegWarps) {
+        const int b = (int)(tok / per_img);
+        const long long r = tok - (long long)b * per_img;
+        int t;
+        if (sh.K > 0) {
+            t = row_of[tok];  // < 0: a rejected id, output 0
+        } else {
+            const int i = (int)(r / sh.w), j = (int)(r - (long long)i * sh.w);
+            t = sh.pool_axis == 0 ? i : j;
+        }
+        const size_t o = (size_t)tok * SL + lane;
+        float4* yl = reinterpret_cast<float4*>(y) + o;
+        if (t < 0) {
+#pragma unroll
+            for (int u = 0; u < NSL; ++u)
+                if (u < nsl) st_stream(yl + 32 * u, make_float4(0.f, 0.f, 0.f, 0.f));
+            continue;
+        }
+        const float4* xl = reinterpret_cast<const float4*>(x) + o;
+        const float4* yl4 = reinterpret_cast<const float4*>(ys + ((size_t)b * sh.T + t) * sh.E) + lane;
+        float4 sv[NSL];
+#pragma unroll
+        for (int u = 0; u < NSL; ++u)
+            sv[u] = u < nsl ? f4_fma(dl[32 * u], ld_stream(xl + 32 * u), __ldcg(yl4 + 32 * u))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        // shift: the token's first s value, from lane 0
+        const float K = __shfl_sync(0xffffffffu, sv[0].x, 0);
+        float m1 = 0.f, m2 = 0.f;
+#pragma unroll
+        for (int u = 0; u < NSL; ++u)
+            if (u < nsl) ln_accum(sv[u], K, m1, m2);
+        float mean, rstd;
+        ln_stats(m1, m2, K, invE, sh.ln_eps, mean, rstd);
+        const float4* zl = reinterpret_cast<const float4*>(z) + o;
+#pragma unroll
+        for (int u = 0; u < NSL; ++u)
+            if (u < nsl) st_stream(yl + 32 * u, ln_gate4(sv[u], ld_stream(zl + 32 * u), gl[32 * u], bl[32 * u], mean, rstd));
+    }
+}
+
 // ---- Staged x_proj: one fp32 GEMM over every pooled token of the batch ---------------------------
 // u[b][k][t][j] = sum_e W_x[k][j][e] * xbar[b][t][e]: C[m][n] = sum_e A[m][e] B[n][e] with M = B T
 // pooled tokens, N = nd (R + 2N) outputs, K = E; both operands E-contiguous.  With the Conv1D each

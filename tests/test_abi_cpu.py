@@ -219,10 +219,18 @@ def test_layernorm_launches(lib):
     small = good_args(flags=LN, ln_gamma=g, ln_beta=b, ln_eps=1e-5)
     n = lib.fastvim_ssm_launch_count(ctypes.byref(small))
     names = [lib.fastvim_ssm_launch_name(ctypes.byref(small), i).decode() for i in range(n)]
-    assert names == ["pool_dense_kernel", "proj_gemm_kernel", "scan_seq_kernel", "ln_epilogue_kernel"]
+    # rows of up to 1536 channels keep each lane's share of a token in registers, wider ones in shared memory
+    assert names == ["pool_dense_kernel", "proj_gemm_kernel", "scan_seq_kernel", "ln_epilogue_reg_kernel"]
     masked = good_args(flags=LN, ln_gamma=g, ln_beta=b, ln_eps=1e-5, K=49, keep_idx=FAKE + (9 << 32))
     n = lib.fastvim_ssm_launch_count(ctypes.byref(masked))
-    assert lib.fastvim_ssm_launch_name(ctypes.byref(masked), n - 1).decode() == "ln_epilogue_kernel"
+    assert lib.fastvim_ssm_launch_name(ctypes.byref(masked), n - 1).decode() == "ln_epilogue_reg_kernel"
+    wide = good_args(flags=LN, ln_gamma=g, ln_beta=b, ln_eps=1e-5, E=2048, R=12)
+    n = lib.fastvim_ssm_launch_count(ctypes.byref(wide))
+    assert lib.fastvim_ssm_launch_name(ctypes.byref(wide), n - 1).decode() == "ln_epilogue_kernel"
+    conv = good_args(flags=LN, ln_gamma=g, ln_beta=b, ln_eps=1e-5, d_conv=4, conv_w=FAKE + (12 << 32),
+                     conv_b=FAKE + (13 << 32))
+    n = lib.fastvim_ssm_launch_count(ctypes.byref(conv))
+    assert lib.fastvim_ssm_launch_name(ctypes.byref(conv), n - 1).decode() == "ln_epilogue_kernel"
     big = good_args(h=128, w=128, B=4, flags=LN, ln_gamma=g, ln_beta=b, ln_eps=1e-5)
     assert lib.fastvim_ssm_launch_count(ctypes.byref(big)) == 1  # the fused launch does it in its gate tasks
 
@@ -237,7 +245,7 @@ def test_staged_launch_order(lib, masked, ln):
     a = good_args(**kw)
     front = ["mask_bucket_kernel", "mask_pool_kernel"] if masked else ["pool_dense_kernel"]
     middle = ["proj_gemm_kernel", "scan_seq_kernel"]
-    back = ["ln_epilogue_kernel" if ln else ("mask_epilogue_kernel" if masked else "epilogue_dense_kernel")]
+    back = ["ln_epilogue_reg_kernel" if ln else ("mask_epilogue_kernel" if masked else "epilogue_dense_kernel")]
     want = front + middle + back
     n = lib.fastvim_ssm_launch_count(ctypes.byref(a))
     assert [lib.fastvim_ssm_launch_name(ctypes.byref(a), i).decode() for i in range(n)] == want
@@ -270,7 +278,7 @@ def test_conv_launches_and_workspace(lib):
     assert names == ["pool_conv_kernel", "proj_gemm_kernel", "scan_seq_kernel", "epilogue_conv_kernel"]
     ln = good_args(d_conv=4, conv_w=CW, conv_b=CB, flags=nat.FV_FLAG_LAYERNORM, ln_gamma=FAKE + (10 << 32),
                    ln_beta=FAKE + (11 << 32), ln_eps=1e-5)
-    assert lib.fastvim_ssm_launch_name(ctypes.byref(ln), 3).decode() == "ln_epilogue_kernel"
+    assert lib.fastvim_ssm_launch_name(ctypes.byref(ln), 3).decode() == "ln_epilogue_kernel"  # neighbours: rows
     # large images take the staged kernels with the Conv1D; forcing the single launch is refused
     big = good_args(h=128, w=128, d_conv=4, conv_w=CW, conv_b=CB)
     assert lib.fastvim_ssm_launch_name(ctypes.byref(big), 0).decode() == "pool_conv_kernel"

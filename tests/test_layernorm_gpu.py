@@ -1,6 +1,7 @@
 """Parity of the post-SSM LayerNorm variant (FV_FLAG_LAYERNORM) with the fp64 oracle: the
-staged LayerNorm epilogue (dense and masked) and the fused launch's gate tasks, over ragged
-channel counts, both pool axes, one and two directions, a large epsilon, rejected keep ids and
+staged LayerNorm epilogues (a token's share per lane in registers up to 1536 channels, shared-memory
+rows above; dense and masked) and the fused launch's gate tasks, over ragged channel counts
+(every register-slot count: 1-4, 6, 8, 12 float4 slots per lane), both pool axes, one and two directions, a large epsilon, rejected keep ids and
 the host entry point."""
 import numpy as np
 import pytest
@@ -28,8 +29,8 @@ def ref_of(q, pool_axis, dir_flags, h=None, w=None, eps=1e-5):
                           ln_eps=eps)
 
 
-@pytest.mark.parametrize("E,pool_axis,dir_flags", [(52, 0, 3), (52, 1, 3), (384, 0, 3), (388, 1, 1), (1540, 0, 2),
-                                                   (4096, 1, 3)])
+@pytest.mark.parametrize("E,pool_axis,dir_flags", [(52, 0, 3), (52, 1, 3), (384, 0, 3), (388, 1, 1), (704, 1, 3), (772, 0, 3),
+                                                   (1024, 1, 3), (1536, 0, 3), (1540, 0, 2), (4096, 1, 3)])
 @pytest.mark.parametrize("path", ["staged", "fused"])
 def test_layernorm_dense(E, pool_axis, dir_flags, path):
     if path == "fused" and E > 2048:
@@ -37,7 +38,8 @@ def test_layernorm_dense(E, pool_axis, dir_flags, path):
     p = with_ln(rand_layer(300 + E + pool_axis, B=2, h=5, w=7, E=E, N=16, R=6, dir_flags=dir_flags), 1 + E, E)
     got = gpu_forward(p, pool_axis, dir_flags, intermediates=False, path=path)
     assert got["status"] == 0
-    assert got["launches"][-1] == ("fused_layer_kernel" if path == "fused" else "ln_epilogue_kernel")
+    staged = "ln_epilogue_reg_kernel" if E <= 1536 else "ln_epilogue_kernel"  # registers / shared-memory rows
+    assert got["launches"][-1] == ("fused_layer_kernel" if path == "fused" else staged)
     assert_close(got["y"], ref_of(p, pool_axis, dir_flags))
 
 
