@@ -54,8 +54,9 @@ def kernel_work(name: str, cfg, pool_axis: int):
     """(bound, algorithmic amount per step) of kernel `name` on workload `cfg` (all its launches in
     one step; a staged layer launches a kernel once per chunk of images):
     bytes for the streaming kernels (what the step must move at minimum), exp2 evaluations for
-    the scans (one per state, step, channel and direction), fp32 flops for the projection GEMM,
-    None for the rest."""
+    the scans (one per state, step, channel and direction), fp32 flops for the x_proj GEMM, the
+    step sizes written for dt_proj (a K = R tensor-core GEMM whose output is the cost), None for the
+    rest."""
     tok = cfg.tokens_per_call()                       # grid tokens, or kept tokens when masked
     row = 4 * cfg.E                                   # one fp32 token row
     T = cfg.h if pool_axis == 0 else cfg.w
@@ -68,6 +69,8 @@ def kernel_work(name: str, cfg, pool_axis: int):
         return "alu", cfg.B * T * cfg.E * cfg.N * cfg.nd
     if name == "proj_gemm_kernel":
         return "fma", 2 * cfg.B * T * cfg.E * cfg.nd * (cfg.R + 2 * cfg.N)
+    if name == "dt_proj_kernel":
+        return "hbm", 4 * cfg.B * T * cfg.E * cfg.nd          # Delta written (tensor-core GEMM, K = R)
     # the gradient's kernels
     if name in ("bwd_gate_dense_kernel", "bwd_gate_masked_kernel", "bwd_ln_gate_kernel"):
         return "hbm", 5 * row * tok                   # read x, z, dy; write dz and dx

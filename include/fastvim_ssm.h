@@ -158,7 +158,8 @@ typedef struct {
     size_t row_of;       /* int32 [B][K] pooled row of each kept token (masked), else 0      */
     size_t row_off;      /* int32 [B][T+1] CSR row offsets (masked), else 0                  */
     size_t row_tok;      /* int32 [B][K] kept-token ordinals grouped by row, ascending       */
-    size_t delta;        /* reserved (0): step sizes stay on chip                            */
+    size_t delta;        /* fp32 [nd][B][T][E] step sizes Delta = softplus(dt_proj) of the
+                            staged kernels; 0 on the fused launch (they stay on chip)       */
     size_t ctrl;         /* uint32 control block of the fused launch (dense layers), else 0  */
     size_t trace;        /* FV_FLAG_TRACE on the fused launch: uint64 [trace_records][4]:
                             w0 = kind << 60 | image << 32 | index (kind 0 pool, 1 scan, 2 gate, 3 x_proj),
@@ -228,7 +229,7 @@ FV_API fv_status fastvim_ssm_forward_host(const fv_ssm_args* host, const fv_ssm_
  * 16 MiB array in device memory, part of this library's device code, held until the process
  * exits.
  *   - Limit: fastvim_ssm_workspace_size(args) must be <= 16 MiB (e.g. the 224 px FastVim-T
- *     layer at batch 128 needs about 6 MiB); larger layers return FV_ERR_UNSUPPORTED with a
+ *     layer at batch 128 needs about 11 MiB); larger layers return FV_ERR_UNSUPPORTED with a
  *     message in fastvim_last_error() and queue nothing; split the batch or use
  *     fastvim_ssm_forward.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.

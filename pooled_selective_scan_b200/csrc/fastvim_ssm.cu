@@ -13,6 +13,7 @@
 
 #include "fv_common.cuh"
 #include "fv_fused.cuh"
+#include "fv_dt_tc.cuh"
 #include "fv_kernels.cuh"
 #include "fv_backward.cuh"
 
@@ -121,6 +122,9 @@ fv_status plan_layout(const fv::Shape& sh, fv_ws_layout* L) {
     L->xbar = off; off = round256(off + (size_t)sh.B * sh.nx * sh.T * sh.E * sizeof(float));
     L->u = off; off = round256(off + (size_t)sh.nd * sh.B * fv::u_block_stride(sh.T, sh.J) * sizeof(float));
     L->ys = off; off = round256(off + (size_t)sh.B * sh.T * sh.E * sizeof(float));
+    if (choose_path(sh) != Path::Fused && fv::staged_delta_kernel(sh)) {  // step sizes of the staged dt_proj kernel
+        L->delta = off; off = round256(off + (size_t)sh.nd * sh.B * sh.T * sh.E * sizeof(float));
+    }
     if (sh.K > 0) {
         L->row_of = off; off = round256(off + (size_t)sh.B * sh.K * sizeof(int32_t));
         L->row_off = off; off = round256(off + (size_t)sh.B * (sh.T + 1) * sizeof(int32_t));
@@ -289,20 +293,23 @@ int launch_count_of(const fv::Shape& sh) {
     const Path path = choose_path(sh);
     if (path == Path::Invalid) return 0;
     if (path == Path::Fused) return 1;
-    return sh.K > 0 ? 5 : 4;
+    return (sh.K > 0 ? 5 : 4) + (fv::staged_delta_kernel(sh) ? 1 : 0);
 }
 
 const char* launch_name_of(const fv::Shape& sh, int i) {
-    static const char* dense[] = {"pool_dense_kernel", "proj_gemm_kernel", "scan_seq_kernel",
+    static const char* dense[] = {"pool_dense_kernel", "proj_gemm_kernel", "dt_proj_kernel", "scan_seq_kernel",
                                   "epilogue_dense_kernel"};
-    static const char* conv[] = {"pool_conv_kernel", "proj_gemm_kernel", "scan_seq_kernel", "epilogue_conv_kernel"};
-    static const char* masked[] = {"mask_bucket_kernel", "mask_pool_kernel", "proj_gemm_kernel", "scan_seq_kernel",
-                                   "mask_epilogue_kernel"};
+    static const char* conv[] = {"pool_conv_kernel", "proj_gemm_kernel", "dt_proj_kernel", "scan_seq_kernel",
+                                 "epilogue_conv_kernel"};
+    static const char* masked[] = {"mask_bucket_kernel", "mask_pool_kernel", "proj_gemm_kernel", "dt_proj_kernel",
+                                   "scan_seq_kernel", "mask_epilogue_kernel"};
     const int n = launch_count_of(sh);
     if (i < 0 || i >= n) return "";
     if (choose_path(sh) == Path::Fused) return "fused_layer_kernel";
     if (sh.ln && i == n - 1) return ln_uses_reg_kernel(sh) ? "ln_epilogue_reg_kernel" : "ln_epilogue_kernel";
-    return sh.K > 0 ? masked[i] : (sh.dc > 0 ? conv[i] : dense[i]);
+    const int first_scan = sh.K > 0 ? 3 : 2;  // without the dt_proj kernel the later launches move up one
+    const int j = (!fv::staged_delta_kernel(sh) && i >= first_scan) ? i + 1 : i;
+    return sh.K > 0 ? masked[j] : (sh.dc > 0 ? conv[j] : dense[j]);
 }
 
 template <int ND, bool Z>
@@ -357,13 +364,16 @@ fv_status launch_scan_seq(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws
         return FV_ERR_CUDA;
     }
     const size_t smem = fv::seq_smem_floats(sh) * sizeof(float);
-    auto kern = sh.zoh_exact ? fv::scan_seq_kernel<true> : fv::scan_seq_kernel<false>;
+    const bool din = fv::staged_delta_kernel(sh);
+    auto kern = sh.zoh_exact ? (din ? fv::scan_seq_kernel<true, true> : fv::scan_seq_kernel<true, false>)
+                             : (din ? fv::scan_seq_kernel<false, true> : fv::scan_seq_kernel<false, false>);
     if ((e = ensure_smem(kern, smem)) != cudaSuccess) { note_cuda(e, "scan smem attribute"); return FV_ERR_CUDA; }
     const long long tiles = (sh.E + fv::kSeqThreads - 1) / fv::kSeqThreads;
     const long long grid = (long long)sh.B * tiles * sh.nd;
     if (grid >= (1ll << 31)) return FV_ERR_UNSUPPORTED;
     kern<<<(unsigned)grid, fv::kSeqThreads, smem, st>>>(sh, (const float*)(ws + L.u), (const float*)(ws + L.xbar),
-                                                         a->A_log, a->W_dt, a->b_dt, ys);
+                                                         a->A_log, a->W_dt, a->b_dt,
+                                                         din ? (const float*)(ws + L.delta) : nullptr, ys);
     FV_LAUNCH_CHECK("scan_seq_kernel");
     return FV_OK;
 }
@@ -424,10 +434,28 @@ fv_status launch_proj_gemm(const fv::Shape& sh, const fv_ssm_args* a, const fv_w
     return FV_OK;
 }
 
-// Staged x_proj, then dt_proj + ZOH + scans.
+// Staged dt_proj + softplus: Delta for every pooled token of the batch and direction, on the
+// tensor cores (fv_dt_tc.cuh), one CTA per 128 tokens x 128 channels of a direction.
+fv_status launch_dt_proj(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st) {
+    const long long M = (long long)sh.B * sh.T;
+    if (M >= (1ll << 31) / 2) return FV_ERR_UNSUPPORTED;
+    cudaError_t e = ensure_smem(fv::dt_proj_kernel, fv::kDtSmemBytes);
+    if (e != cudaSuccess) { note_cuda(e, "dt_proj smem attribute"); return FV_ERR_CUDA; }
+    const dim3 grid((unsigned)((M + fv::kDtM - 1) / fv::kDtM), (unsigned)((sh.E + fv::kDtN - 1) / fv::kDtN),
+                    (unsigned)sh.nd);
+    fv::dt_proj_kernel<<<grid, fv::kDtThreads, fv::kDtSmemBytes, st>>>(sh, (const float*)(ws + L.u), a->W_dt,
+                                                                        a->b_dt, (float*)(ws + L.delta),
+                                                                        (unsigned*)(ws + L.status));
+    FV_LAUNCH_CHECK("dt_proj_kernel");
+    return FV_OK;
+}
+
+// Staged x_proj, dt_proj + softplus as its own GEMM from dt_rank 32 (else inside the scans), then
+// ZOH + scans.
 fv_status staged_middle(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st,
                         EventMarks& marks) {
     FV_MARK_CALL(marks, st, launch_proj_gemm(sh, a, L, ws, st));
+    if (fv::staged_delta_kernel(sh)) FV_MARK_CALL(marks, st, launch_dt_proj(sh, a, L, ws, st));
     FV_MARK_CALL(marks, st, launch_scan_seq(sh, a, L, ws, st));
     return FV_OK;
 }

@@ -50,6 +50,12 @@ __host__ __device__ __forceinline__ size_t u_offset(const Shape& sh, int k, int 
     return ((size_t)b * sh.nd + k) * u_block_stride(sh.T, sh.J) + (size_t)t * sh.J;
 }
 
+// Offset (in floats) of step size row (direction k, image b, pooled token t) in the staged path's
+// Delta buffer, fp32 [nd][B][T][E].
+__host__ __device__ __forceinline__ size_t delta_offset(const Shape& sh, int k, int b, int t) {
+    return (((size_t)k * sh.B + b) * sh.T + t) * (size_t)sh.E;
+}
+
 // Offset (in floats) of token s of pooled token (b, t) on the dense grid, and the stride
 // between consecutive s.  POOL_W: token (t, s); POOL_H: token (s, t).
 __host__ __device__ __forceinline__ size_t dense_base(const Shape& sh, int b, int t) {

@@ -478,7 +478,7 @@ template <int ND, bool ZOH_EXACT>
 __device__ __forceinline__ void fused_scan(const Shape& sh, const FusedPlan& pl, const FusedPtrs& p, int b, int tile,
                                            float* smem) {
     const int e0 = tile * pl.ECH;
-    seq_scan<kFusedThreads, ND, ZOH_EXACT>(sh, p.u, p.xbar, p.A_log, p.W_dt, p.b_dt, p.ys + (size_t)b * sh.T * sh.E + e0,
+    seq_scan<kFusedThreads, ND, ZOH_EXACT>(sh, p.u, p.xbar, p.A_log, p.W_dt, p.b_dt, nullptr, p.ys + (size_t)b * sh.T * sh.E + e0,
                                            sh.E, b, e0, 0, smem);
     cta_signal(p.ctrl ? p.ctrl + kCtrlHeaderWords + 2 * sh.B + b : nullptr);
 }

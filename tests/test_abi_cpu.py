@@ -158,6 +158,7 @@ def test_workspace_layout(lib, pool_axis, K):
     assert (L.T, L.S, L.nd) == (T, 15 - T, 2)
     ub = -(-T * 36 // 32) * 32
     regions = [(L.status, 4), (L.xbar, 3 * T * 64 * 4), (L.u, 2 * 3 * ub * 4), (L.ys, 3 * T * 64 * 4)]
+    assert L.delta == 0  # dt_rank 4: the scans compute their step sizes themselves
     if K:
         regions += [(L.row_of, 3 * K * 4), (L.row_off, 3 * (T + 1) * 4), (L.row_tok, 3 * K * 4)]
     else:
@@ -249,6 +250,30 @@ def test_staged_launch_order(lib, masked, ln):
     want = front + middle + back
     n = lib.fastvim_ssm_launch_count(ctypes.byref(a))
     assert [lib.fastvim_ssm_launch_name(ctypes.byref(a), i).decode() for i in range(n)] == want
+
+
+@pytest.mark.parametrize("masked", [False, True])
+@pytest.mark.parametrize("R", [31, 32, 48])
+def test_delta_kernel_from_dt_rank_32(lib, masked, R):
+    """With dt_rank >= 32 the staged path computes the step sizes in their own (tensor-core) GEMM
+    launch between x_proj and the scans and keeps them in the workspace; below, the scans compute
+    them."""
+    kw = dict(B=3, h=6, w=9, E=64, R=R, flags=2)
+    if masked:
+        kw.update(K=37, keep_idx=FAKE + (9 << 32))
+    a = good_args(**kw)
+    n = lib.fastvim_ssm_launch_count(ctypes.byref(a))
+    names = [lib.fastvim_ssm_launch_name(ctypes.byref(a), i).decode() for i in range(n)]
+    front = ["mask_bucket_kernel", "mask_pool_kernel"] if masked else ["pool_dense_kernel"]
+    mid = ["proj_gemm_kernel"] + (["dt_proj_kernel"] if R >= 32 else []) + ["scan_seq_kernel"]
+    assert names == front + mid + ["mask_epilogue_kernel" if masked else "epilogue_dense_kernel"]
+    L = nat.FvWsLayout()
+    assert lib.fastvim_ssm_workspace_layout(ctypes.byref(a), ctypes.byref(L)) == nat.FV_OK
+    if R >= 32:  # [nd][B][T][E] fp32 after ys, inside the workspace
+        assert L.delta % 256 == 0 and L.delta >= L.ys + 3 * 6 * 64 * 4
+        assert L.total_bytes >= L.delta + 2 * 3 * 6 * 64 * 4
+    else:
+        assert L.delta == 0
 
 
 # ---------------------------------------------------------------------------------------------

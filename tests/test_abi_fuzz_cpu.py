@@ -131,12 +131,14 @@ def _check_launches(lib, a):
         return
     assert not a.flags & nat.FV_FLAG_PATH_FUSED
     assert "fused_layer_kernel" not in names
-    full = 5 if a.K else 4  # pooling (masked: bucketing, pooling), x_proj, scans, epilogue
+    # pooling (masked: bucketing, pooling), x_proj, (dt_proj from dt_rank 32), scans, epilogue
+    full = (5 if a.K else 4) + (1 if a.R >= 32 else 0)
     if a.flags & nat.FV_FLAG_LAYERNORM:  # registers up to 1536 channels, shared-memory rows above
         assert n == full and names[-1] == ("ln_epilogue_reg_kernel" if a.E <= 1536 else "ln_epilogue_kernel")
     else:
         assert n == full and names[-1] == ("mask_epilogue_kernel" if a.K else "epilogue_dense_kernel")
     assert "proj_gemm_kernel" in names and any(k.startswith("scan") for k in names)
+    assert ("dt_proj_kernel" in names) == (a.R >= 32)
     if a.K:
         assert names[0].startswith("mask_")
 

@@ -81,6 +81,15 @@ def test_state_counts(N):
     check_layer(p, 0, 3)
 
 
+@pytest.mark.parametrize("R,N", [(32, 3), (36, 6), (33, 16), (64, 16), (61, 16)])
+def test_dt_proj_copy_paths(R, N):
+    """The step-size GEMM (dt_rank >= 32) copies its operands 16 bytes at a time when every row of u
+    (R + 2N floats) and of W_dt (R floats) starts on 16 bytes, 4 bytes at a time otherwise; R above
+    32 takes two or more slices of the tensor-core K loop."""
+    p = rand_layer(70 + R + N, B=3, h=11, w=5, E=136, N=N, R=R, dir_flags=3)
+    check_layer(p, 0, 3)
+
+
 @pytest.mark.parametrize("E,R", [(4, 1), (100, 7), (1032, 40), (1536, 48)])
 def test_channel_counts(E, R):
     p = rand_layer(60 + E, B=2, h=3, w=6, E=E, N=16, R=R, dir_flags=3)
