@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define FASTVIM_SSM_ABI_VERSION 4
+#define FASTVIM_SSM_ABI_VERSION 5
 
 #if defined(__GNUC__)
 #define FV_API __attribute__((visibility("default")))
@@ -298,6 +298,11 @@ typedef struct {
     size_t du;           /* float, the layout of the forward's u: d dt_low | dB | dC           */
     size_t dxs;          /* float [B][nd][T][E]  the scans' share of dL/dxbar per direction     */
     size_t ckpt;         /* float [B][nd][2 ceil(T/16)][E][16]  scan state entering every 8 steps */
+    size_t status;       /* uint32 device status word (FV_ERR_TIMEOUT from a bounded wait), read
+                            by fastvim_get_device_status(ws, stream); the call clears it       */
+    size_t delta;        /* float [nd][B][T][E] step sizes Delta, computed by the gradient call
+                            when the forward workspace holds none (fv_ws_layout.delta == 0),
+                            else 0 (the forward's are read)                                   */
 } fv_bwd_ws_layout;
 
 /* Workspace bytes a gradient call needs (0 when the arguments are invalid). */

@@ -92,7 +92,8 @@ class FvSsmGrads(ctypes.Structure):
 
 
 class FvBwdWsLayout(ctypes.Structure):
-    _fields_ = [(name, ctypes.c_size_t) for name in ("total_bytes", "dys", "dxbar", "du", "dxs", "ckpt")]
+    _fields_ = [(name, ctypes.c_size_t) for name in ("total_bytes", "dys", "dxbar", "du", "dxs", "ckpt", "status",
+                                                     "delta")]
 
 
 class FastvimError(RuntimeError):

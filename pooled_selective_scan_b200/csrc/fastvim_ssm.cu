@@ -434,22 +434,24 @@ fv_status launch_proj_gemm(const fv::Shape& sh, const fv_ssm_args* a, const fv_w
     return FV_OK;
 }
 
-// Staged dt_proj + softplus: Delta for every pooled token of the batch and direction, on the
-// tensor cores (fv_dt_tc.cuh), one CTA per 128 tokens x 128 channels of a direction.
-fv_status launch_dt_proj(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st) {
+// dt_proj + softplus: Delta for every pooled token of the batch and direction, on the tensor
+// cores (fv_dt_tc.cuh), one CTA per 128 tokens x 128 channels of a direction.
+fv_status launch_dt_proj_to(const fv::Shape& sh, const float* u, const float* W_dt, const float* b_dt, float* delta,
+                            unsigned* status, cudaStream_t st) {
     const long long M = (long long)sh.B * sh.T;
     if (M >= (1ll << 31) / 2) return FV_ERR_UNSUPPORTED;
     cudaError_t e = ensure_smem(fv::dt_proj_kernel, fv::kDtSmemBytes);
     if (e != cudaSuccess) { note_cuda(e, "dt_proj smem attribute"); return FV_ERR_CUDA; }
     const dim3 grid((unsigned)((M + fv::kDtM - 1) / fv::kDtM), (unsigned)((sh.E + fv::kDtN - 1) / fv::kDtN),
                     (unsigned)sh.nd);
-    fv::dt_proj_kernel<<<grid, fv::kDtThreads, fv::kDtSmemBytes, st>>>(sh, (const float*)(ws + L.u), a->W_dt,
-                                                                        a->b_dt, (float*)(ws + L.delta),
-                                                                        (unsigned*)(ws + L.status));
+    fv::dt_proj_kernel<<<grid, fv::kDtThreads, fv::kDtSmemBytes, st>>>(sh, u, W_dt, b_dt, delta, status);
     FV_LAUNCH_CHECK("dt_proj_kernel");
     return FV_OK;
 }
-
+fv_status launch_dt_proj(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st) {
+    return launch_dt_proj_to(sh, (const float*)(ws + L.u), a->W_dt, a->b_dt, (float*)(ws + L.delta),
+                             (unsigned*)(ws + L.status), st);
+}
 // Staged x_proj, dt_proj + softplus as its own GEMM from dt_rank 32 (else inside the scans), then
 // ZOH + scans.
 fv_status staged_middle(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_layout& L, char* ws, cudaStream_t st,
@@ -875,35 +877,51 @@ extern "C" fv_status fastvim_ssm_forward_noalloc(const fv_ssm_args* args, void* 
 namespace {
 
 struct BwdLayout {
-    size_t dys, dxbar, du, dxs, ckpt, total;
+    size_t status, dys, dxbar, du, dxs, ckpt, delta, total;
 };
+
+// Whether the forward call's workspace holds the step sizes Delta (staged path, dt_rank >= 32);
+// otherwise the gradient computes them into its own workspace first.
+bool fwd_has_delta(const fv::Shape& sh) {
+    fv_ws_layout FL;
+    plan_layout(sh, &FL);
+    return FL.delta != 0;
+}
 
 BwdLayout plan_bwd(const fv::Shape& sh) {
     BwdLayout L{};
     size_t off = 0;
     const size_t bte = (size_t)sh.B * sh.T * sh.E * sizeof(float);
+    L.status = off; off = round256(off + 2 * sizeof(unsigned));
     L.dys = off; off = round256(off + bte);
     L.dxbar = off; off = round256(off + bte);
     L.du = off; off = round256(off + (size_t)sh.nd * sh.B * fv::u_block_stride(sh.T, sh.J) * sizeof(float));
     L.dxs = off; off = round256(off + (size_t)sh.nd * bte);
     L.ckpt = off;
     off = round256(off + (size_t)sh.B * sh.nd * fv::bs_nckpt(sh.T) * sh.E * 16 * sizeof(float));
+    if (!fwd_has_delta(sh)) {
+        L.delta = off;
+        off = round256(off + (size_t)sh.nd * sh.B * sh.T * sh.E * sizeof(float));
+    }
     L.total = off;
     return L;
 }
 
-// Launch order of a gradient call: gate (through the LayerNorm with FV_FLAG_LAYERNORM), scans (with
-// dt_proj), dW_x, dxbar, pooling.
+// Launch order of a gradient call: gate (through the LayerNorm with FV_FLAG_LAYERNORM), dt_proj
+// (when the forward workspace holds no step sizes), scans (with dt_proj's gradient), dW_x, dxbar,
+// pooling.
+int bwd_launch_count_of(const fv::Shape& sh) { return sh.B == 0 ? 0 : (fwd_has_delta(sh) ? 5 : 6); }
 const char* bwd_launch_name_of(const fv::Shape& sh, int i) {
-    static const char* dense[] = {"bwd_gate_dense_kernel", "bwd_scan_kernel", "bwd_gemm_kernel:W_x",
+    static const char* dense[] = {"bwd_gate_dense_kernel", "dt_proj_kernel", "bwd_scan_kernel", "bwd_gemm_kernel:W_x",
                                   "bwd_gemm_kernel:xbar", "bwd_pool_dense_kernel"};
-    static const char* masked[] = {"bwd_gate_masked_kernel", "bwd_scan_kernel", "bwd_gemm_kernel:W_x",
+    static const char* masked[] = {"bwd_gate_masked_kernel", "dt_proj_kernel", "bwd_scan_kernel", "bwd_gemm_kernel:W_x",
                                    "bwd_gemm_kernel:xbar", "bwd_pool_masked_kernel"};
-    if (sh.B == 0 || i < 0 || i >= 5) return "";
+    const int n = bwd_launch_count_of(sh);
+    if (i < 0 || i >= n) return "";
     if (i == 0 && sh.ln) return "bwd_ln_gate_kernel";
-    return sh.K > 0 ? masked[i] : dense[i];
+    const int j = (n == 5 && i >= 1) ? i + 1 : i;
+    return sh.K > 0 ? masked[j] : dense[j];
 }
-int bwd_launch_count_of(const fv::Shape& sh) { return sh.B == 0 ? 0 : 5; }
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     const uintptr_t a0 = (uintptr_t)a, b0 = (uintptr_t)b;
@@ -1012,9 +1030,12 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
     float* du = (float*)(ws + L.du);
     float* dxs = (float*)(ws + L.dxs);
     float* ckpt = (float*)(ws + L.ckpt);
-    // the scans add dB and dC into du
+    // the step sizes: the forward's (staged, dt_rank >= 32), else computed below into ws
+    const float* delta = L.delta ? (const float*)(ws + L.delta) : (const float*)(fw + FL.delta);
+    // the scans add dB and dC into du; the status word starts clear
     if ((e = cudaMemsetAsync(du, 0, (size_t)sh.nd * sh.B * fv::u_block_stride(sh.T, sh.J) * sizeof(float), st)) !=
-        cudaSuccess) {
+            cudaSuccess ||
+        (e = cudaMemsetAsync(ws + L.status, 0, 2 * sizeof(unsigned), st)) != cudaSuccess) {
         note_cuda(e, "du reset");
         return FV_ERR_CUDA;
     }
@@ -1079,7 +1100,10 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
             return FV_OK;
         })());
     }
-    // 2. adjoint of the scans
+    // 2. the step sizes (when the forward kept none), then the adjoint of the scans
+    if (L.delta)
+        FV_MARK_CALL(marks, st, launch_dt_proj_to(sh, u, a->W_dt, a->b_dt, (float*)(ws + L.delta),
+                                                  (unsigned*)(ws + L.status), st));
     FV_MARK_CALL(marks, st, ([&]() -> fv_status {
         const dim3 grid(sh.B, sh.nd, (sh.E + fv::kBsCh - 1) / fv::kBsCh);
         if (sh.zoh_exact) {
@@ -1087,7 +1111,7 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
                 note_cuda(e, "scan gradient smem attribute");
                 return FV_ERR_CUDA;
             }
-            fv::bwd_scan_kernel<true><<<grid, fv::kBsThreads, scan_smem, st>>>(sh, u, xbar, dys, a->A_log, a->W_dt, a->b_dt,
+            fv::bwd_scan_kernel<true><<<grid, fv::kBsThreads, scan_smem, st>>>(sh, u, xbar, dys, a->A_log, a->W_dt, delta,
                                                                               ckpt, dxs, du, g->dA_log, g->dW_dt,
                                                                               g->db_dt);
         } else {
@@ -1096,7 +1120,7 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
                 return FV_ERR_CUDA;
             }
             fv::bwd_scan_kernel<false><<<grid, fv::kBsThreads, scan_smem, st>>>(sh, u, xbar, dys, a->A_log, a->W_dt,
-                                                                               a->b_dt, ckpt, dxs, du, g->dA_log,
+                                                                               delta, ckpt, dxs, du, g->dA_log,
                                                                                g->dW_dt, g->db_dt);
         }
         FV_LAUNCH_CHECK("bwd_scan_kernel");
@@ -1151,6 +1175,7 @@ fv_status fastvim_ssm_backward_workspace_layout(const fv_ssm_args* args, fv_bwd_
     const BwdLayout L = plan_bwd(sh);
     out->total_bytes = L.total;
     out->dys = L.dys; out->dxbar = L.dxbar; out->du = L.du; out->dxs = L.dxs; out->ckpt = L.ckpt;
+    out->status = L.status; out->delta = L.delta;
     return FV_OK;
 }
 

@@ -42,7 +42,6 @@ __host__ __device__ __forceinline__ size_t bs_smem_floats(int R) {
            + (size_t)kBsChunk * 32            // B | C of the chunk's steps
            + 6 * (size_t)kBsChunk * kBsCh     // xbar, dys, Delta, sig(v), dv, dxbar (scan share)
            + (size_t)kBsChunk * 32            // dB | dC sums of the chunk
-           + kBsCh                            // b_dt of the CTA's channels
            + (size_t)kBsCh * (R + 1);         // dW_dt | db_dt sums of the CTA's channels
 }
 
@@ -410,6 +409,8 @@ bwd_ln_gate_kernel(Shape sh, const float* __restrict__ x, const float* __restric
 //             or (Abar_i - 1) / A B_i xbar_i (exact ZOH);  ys += C_i . h_i
 //   adjoint   lam_i = C_i dys_i + Abar_{i+1} lam_{i+1}  (lam = 0 past the last step)
 //             dC_i += dys_i h_i;  dAbar_i = lam_i h_{i-1};  dq_i = lam_i
+// Delta comes from a buffer: the forward's (staged path, dt_rank >= 32) or the one the gradient call
+// fills first with dt_proj_kernel; sig(v) = softplus'(v) = 1 - e^-Delta.
 // Pass 1 runs the recurrence in scan order and stores the state entering every 8 steps
 // (ckpt [B][nd][2 nchunks][E][16]).  Pass 2 walks the 16-step staged chunks in reverse, each as two
 // halves of 8 steps, last half first: it recomputes the half's states from its checkpoint (8 steps
@@ -425,7 +426,7 @@ bwd_ln_gate_kernel(Shape sh, const float* __restrict__ x, const float* __restric
 template <bool ZOH_EXACT>
 __global__ void __launch_bounds__(kBsThreads, 2)
 bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__ xbar, const float* __restrict__ dys,
-                const float* __restrict__ A_log, const float* __restrict__ W_dt, const float* __restrict__ b_dt,
+                const float* __restrict__ A_log, const float* __restrict__ W_dt, const float* __restrict__ delta,
                 float* __restrict__ ckpt, float* __restrict__ dxs, float* __restrict__ du,
                 float* __restrict__ dA_log, float* __restrict__ dW_dt, float* __restrict__ db_dt) {
     extern __shared__ float bsm[];
@@ -442,8 +443,7 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
     float* sdv = ssg + kBsChunk * kBsCh;      // [16][64]
     float* sdx = sdv + kBsChunk * kBsCh;      // [16][64]
     float* sred = sdx + kBsChunk * kBsCh;     // [16][32]
-    float* sbias = sred + kBsChunk * 32;      // [64]
-    float* swacc = sbias + kBsCh;             // [64][R + 1]
+    float* swacc = sred + kBsChunk * 32;      // [64][R + 1]
     const int tid = threadIdx.x;
     const int c = tid >> 2, q = tid & 3, lane = tid & 31;
     const int e = e0 + c;
@@ -457,7 +457,6 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
         const int row = i / R, r = i - row * R;
         sw[row * WS + r] = (e0 + row < E) ? __ldg(W_dt + ((size_t)k * E + e0 + row) * R + r) : 0.f;
     }
-    for (int i = tid; i < kBsCh; i += kBsThreads) sbias[i] = (e0 + i < E) ? __ldg(b_dt + (size_t)k * E + e0 + i) : 0.f;
     for (int i = tid; i < kBsCh * (R + 1); i += kBsThreads) swacc[i] = 0.f;
 
     constexpr float kLog2e = 1.4426950408889634f;
@@ -476,13 +475,16 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
     auto chunk_len = [&](int it) { return min(kBsChunk, T - chunk_t0(it)); };
     auto t_of = [&](int it, int i) { return fwd ? chunk_t0(it) + i : chunk_t0(it) + chunk_len(it) - 1 - i; };
 
-    // stage a chunk's per-step inputs and compute Delta (and sig(v) in pass 2)
+    // stage a chunk's per-step inputs: Delta (written by the forward's or this call's dt_proj
+    // kernel), and in pass 2 dt_low, dys and softplus'(v) = sigmoid(v) = 1 - e^-Delta (as -expm1,
+    // exact for small Delta)
     auto stage = [&](int it, bool pass2) {
         const int len = chunk_len(it);
-        for (int i = tid; i < kBsChunk * R; i += kBsThreads) {
-            const int s = i / R, r = i - s * R;
-            sdtl[i] = s < len ? ub[(size_t)t_of(it, s) * J + r] : 0.f;
-        }
+        if (pass2)
+            for (int i = tid; i < kBsChunk * R; i += kBsThreads) {
+                const int s = i / R, r = i - s * R;
+                sdtl[i] = s < len ? ub[(size_t)t_of(it, s) * J + r] : 0.f;
+            }
         for (int i = tid; i < kBsChunk * 32; i += kBsThreads) {
             const int s = i >> 5, j = i & 31, n = j & 15;
             sbc[i] = (s < len && n < N) ? ub[(size_t)t_of(it, s) * J + R + (j < 16 ? n : N + n)] : 0.f;
@@ -491,19 +493,15 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
         for (int i = tid; i < kBsChunk * kBsCh; i += kBsThreads) {
             const int s = i / kBsCh, cc = i - s * kBsCh;
             const bool ok = s < len && e0 + cc < E;
-            const size_t o = ((size_t)b * T + (ok ? t_of(it, s) : 0)) * E + e0 + cc;
+            const int t = ok ? t_of(it, s) : 0;
+            const size_t o = ((size_t)b * T + t) * E + e0 + cc;
             sx[i] = ok ? xbar[o] : 0.f;
-            if (pass2) sdy[i] = ok ? dys[o] : 0.f;
-        }
-        __syncthreads();
-        for (int i = tid; i < kBsChunk * kBsCh; i += kBsThreads) {
-            const int s = i / kBsCh, cc = i - s * kBsCh;
-            float v = sbias[cc];
-            const float* wr = sw + cc * WS;
-            const float* dr = sdtl + s * R;
-            for (int r = 0; r < R; ++r) v = fmaf(wr[r], dr[r], v);
-            sdl[i] = softplus_fast(v);
-            if (pass2) ssg[i] = sigmoid_fast(v);
+            const float dl = ok ? delta[delta_offset(sh, k, b, t) + e0 + cc] : 0.f;
+            sdl[i] = dl;
+            if (pass2) {
+                sdy[i] = ok ? dys[o] : 0.f;
+                ssg[i] = -expm1f(-dl);
+            }
         }
         __syncthreads();
     };

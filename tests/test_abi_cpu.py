@@ -69,7 +69,7 @@ def test_status_strings(lib):
     assert nat.status_string(0) == "FV_OK"
     for s in range(1, 10):
         assert nat.status_string(s).startswith("FV_ERR_")
-    assert lib.fastvim_abi_version() == 4
+    assert lib.fastvim_abi_version() == 5
 
 
 # ---------------------------------------------------------------------------------------------
@@ -211,7 +211,7 @@ def test_layernorm_arguments(lib):
         assert validate(good_args(flags=LN, ln_gamma=g, ln_beta=b, ln_eps=eps)) == nat.FV_ERR_SHAPE
     assert validate(good_args(flags=LN, ln_gamma=g + 4, ln_beta=b, ln_eps=1e-5)) == nat.FV_ERR_ALIGN
     assert validate(good_args(flags=LN, ln_gamma=g, ln_beta=b, ln_eps=1e-5, E=4100)) == nat.FV_ERR_UNSUPPORTED
-    assert lib.fastvim_abi_version() == 4
+    assert lib.fastvim_abi_version() == 5
 
 
 def test_layernorm_launches(lib):

@@ -210,8 +210,14 @@ def test_gradient_validation_and_plan(a, pick):
     nd = bin(a.dir_flags).count("1")
     ub = -(-T * (a.R + 2 * a.N) // 32) * 32
     bte = a.B * T * a.E * 4
-    regions = sorted([(L.dys, bte), (L.dxbar, bte), (L.du, nd * a.B * ub * 4), (L.dxs, nd * bte),
-                      (L.ckpt, a.B * nd * 2 * -(-T // 16) * a.E * 16 * 4)])
+    regions = [(L.status, 8), (L.dys, bte), (L.dxbar, bte), (L.du, nd * a.B * ub * 4), (L.dxs, nd * bte),
+               (L.ckpt, a.B * nd * 2 * -(-T // 16) * a.E * 16 * 4)]
+    FL = nat.FvWsLayout()
+    assert lib.fastvim_ssm_workspace_layout(ctypes.byref(a), ctypes.byref(FL)) == nat.FV_OK
+    assert (L.delta == 0) == (FL.delta != 0)  # the step sizes live in exactly one of the workspaces
+    if L.delta:
+        regions.append((L.delta, nd * bte))
+    regions = sorted(regions)
     end = 0
     for off, n in regions:
         assert off % 256 == 0 and off >= end
@@ -224,7 +230,8 @@ def test_gradient_validation_and_plan(a, pick):
     else:
         first = ("bwd_ln_gate_kernel" if a.flags & nat.FV_FLAG_LAYERNORM else
                  "bwd_gate_masked_kernel" if a.K else "bwd_gate_dense_kernel")
-        assert names[0] == first and names[1] == "bwd_scan_kernel" and len(names) == 5
+        mid = ["bwd_scan_kernel"] if FL.delta else ["dt_proj_kernel", "bwd_scan_kernel"]
+        assert names[0] == first and names[1:1 + len(mid)] == mid and len(names) == 4 + len(mid)
     g = _grads_for(a)
     fws = lib.fastvim_ssm_workspace_size(ctypes.byref(a))
 
