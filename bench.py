@@ -80,6 +80,10 @@ def kernel_work(name: str, cfg, pool_axis: int):
         return "hbm", 2 * row * tok
     if name == "bwd_scan_kernel":
         return "alu", cfg.B * T * cfg.E * cfg.N * cfg.nd   # one exp2 per state and step (the minimum)
+    if name == "bwd_reduce_kernel:du":                # the 64-channel tiles' du shares read, du written
+        return "hbm", 4 * (-(-cfg.E // 64) + 1) * cfg.nd * cfg.B * T * (cfg.R + 2 * cfg.N)
+    if name == "bwd_reduce_kernel:params":            # per-image partials of dA_log, dW_dt, db_dt read
+        return "hbm", 4 * cfg.B * cfg.nd * cfg.E * (cfg.N + cfg.R + 1)
     if name.startswith("bwd_gemm_kernel"):
         J = cfg.R + 2 * cfg.N
         M = cfg.B * T

@@ -283,9 +283,9 @@ typedef struct {
     float* dz;        /* dL/dz, the shape of z (written)                                      */
     float* dA_log;    /* [nd][E][N]      } parameter gradients, summed over the batch;          */
     float* dD;        /* [nd][E]         } written (not accumulated into): the call zeroes     */
-    float* dW_x;      /* [nd][R+2N][E]   } them first.  The sums run in fp32 with atomic       */
-    float* dW_dt;     /* [nd][E][R]      } additions, so their last bits may differ between    */
-    float* db_dt;     /* [nd][E]         } runs.                                               */
+    float* dW_x;      /* [nd][R+2N][E]   } them.  The sums run in fp32 over per-block partial  */
+    float* dW_dt;     /* [nd][E][R]      } sums added in a fixed order (no atomics), so two    */
+    float* db_dt;     /* [nd][E]         } calls on one GPU give the same bits.                */
     float* dln_gamma; /* [E] with FV_FLAG_LAYERNORM (written, like the above), else NULL          */
     float* dln_beta;  /* [E] with FV_FLAG_LAYERNORM, else NULL                                    */
 } fv_ssm_grads;
@@ -303,6 +303,8 @@ typedef struct {
     size_t delta;        /* float [nd][B][T][E] step sizes Delta, computed by the gradient call
                             when the forward workspace holds none (fv_ws_layout.delta == 0),
                             else 0 (the forward's are read)                                   */
+    size_t partials;     /* float scratch from here to the end: per-block partial sums of du and
+                            of the parameter gradients, added in a fixed order                 */
 } fv_bwd_ws_layout;
 
 /* Workspace bytes a gradient call needs (0 when the arguments are invalid). */

@@ -93,7 +93,7 @@ class FvSsmGrads(ctypes.Structure):
 
 class FvBwdWsLayout(ctypes.Structure):
     _fields_ = [(name, ctypes.c_size_t) for name in ("total_bytes", "dys", "dxbar", "du", "dxs", "ckpt", "status",
-                                                     "delta")]
+                                                     "delta", "partials")]
 
 
 class FastvimError(RuntimeError):

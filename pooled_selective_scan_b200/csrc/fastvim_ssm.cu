@@ -877,8 +877,16 @@ extern "C" fv_status fastvim_ssm_forward_noalloc(const fv_ssm_args* args, void* 
 namespace {
 
 struct BwdLayout {
-    size_t status, dys, dxbar, du, dxs, ckpt, delta, total;
+    size_t status, dys, dxbar, du, dxs, ckpt, delta;
+    // per-block partial sums, added in a fixed order by bwd_reduce_kernel
+    size_t partials, part_du, part_dA, part_wdt, part_bdt, part_wx, part_gate;
+    size_t total;
 };
+
+// Caps that size the partial-sum scratch independently of the GPU: blocks of the persistent gate
+// gradient, and K splits of the dW_x GEMM.
+constexpr int kMaxGateBlocks = 2048;
+constexpr int kMaxWxSplits = 64;
 
 // Whether the forward call's workspace holds the step sizes Delta (staged path, dt_rank >= 32);
 // otherwise the gradient computes them into its own workspace first.
@@ -903,6 +911,15 @@ BwdLayout plan_bwd(const fv::Shape& sh) {
         L.delta = off;
         off = round256(off + (size_t)sh.nd * sh.B * sh.T * sh.E * sizeof(float));
     }
+    const size_t f = sizeof(float), ne = (size_t)sh.nd * sh.B * sh.E;
+    L.partials = off;
+    L.part_du = off;
+    off = round256(off + (size_t)((sh.E + fv::kBsCh - 1) / fv::kBsCh) * sh.nd * sh.B * fv::u_block_stride(sh.T, sh.J) * f);
+    L.part_dA = off; off = round256(off + ne * sh.N * f);
+    L.part_wdt = off; off = round256(off + ne * sh.R * f);
+    L.part_bdt = off; off = round256(off + ne * f);
+    L.part_wx = off; off = round256(off + (size_t)kMaxWxSplits * sh.nd * sh.J * sh.E * f);
+    L.part_gate = off; off = round256(off + (size_t)kMaxGateBlocks * (sh.ln ? 3 : 1) * sh.E * f);
     L.total = off;
     return L;
 }
@@ -910,16 +927,18 @@ BwdLayout plan_bwd(const fv::Shape& sh) {
 // Launch order of a gradient call: gate (through the LayerNorm with FV_FLAG_LAYERNORM), dt_proj
 // (when the forward workspace holds no step sizes), scans (with dt_proj's gradient), dW_x, dxbar,
 // pooling.
-int bwd_launch_count_of(const fv::Shape& sh) { return sh.B == 0 ? 0 : (fwd_has_delta(sh) ? 5 : 6); }
+int bwd_launch_count_of(const fv::Shape& sh) { return sh.B == 0 ? 0 : (fwd_has_delta(sh) ? 7 : 8); }
 const char* bwd_launch_name_of(const fv::Shape& sh, int i) {
-    static const char* dense[] = {"bwd_gate_dense_kernel", "dt_proj_kernel", "bwd_scan_kernel", "bwd_gemm_kernel:W_x",
-                                  "bwd_gemm_kernel:xbar", "bwd_pool_dense_kernel"};
-    static const char* masked[] = {"bwd_gate_masked_kernel", "dt_proj_kernel", "bwd_scan_kernel", "bwd_gemm_kernel:W_x",
-                                   "bwd_gemm_kernel:xbar", "bwd_pool_masked_kernel"};
+    static const char* dense[] = {"bwd_gate_dense_kernel", "dt_proj_kernel", "bwd_scan_kernel", "bwd_reduce_kernel:du",
+                                  "bwd_gemm_kernel:W_x", "bwd_gemm_kernel:xbar", "bwd_pool_dense_kernel",
+                                  "bwd_reduce_kernel:params"};
+    static const char* masked[] = {"bwd_gate_masked_kernel", "dt_proj_kernel", "bwd_scan_kernel", "bwd_reduce_kernel:du",
+                                   "bwd_gemm_kernel:W_x", "bwd_gemm_kernel:xbar", "bwd_pool_masked_kernel",
+                                   "bwd_reduce_kernel:params"};
     const int n = bwd_launch_count_of(sh);
     if (i < 0 || i >= n) return "";
     if (i == 0 && sh.ln) return "bwd_ln_gate_kernel";
-    const int j = (n == 5 && i >= 1) ? i + 1 : i;
+    const int j = (n == 7 && i >= 1) ? i + 1 : i;
     return sh.K > 0 ? masked[j] : dense[j];
 }
 
@@ -961,12 +980,18 @@ int device_sm_count() {
     return sms;
 }
 
+// K per split (a multiple of the GEMM's k-step) for about `splits` splits of Kd; the splits that
+// result are ceil(Kd / chunk).
+int bwd_kchunk(int Kd, int splits) {
+    const int kchunk = (Kd + splits - 1) / splits;
+    return (kchunk + fv::kBgK - 1) / fv::kBgK * fv::kBgK;
+}
+
 template <class AOp, class BOp, class COp>
 fv_status launch_bwd_gemm(int M, int Nc, int Kd, int nz, int splits, AOp A, BOp Bm, COp C, cudaStream_t st,
                           const char* where) {
     if (M <= 0 || Nc <= 0 || Kd <= 0) return FV_OK;
-    int kchunk = (Kd + splits - 1) / splits;
-    kchunk = (kchunk + fv::kBgK - 1) / fv::kBgK * fv::kBgK;
+    const int kchunk = bwd_kchunk(Kd, splits);
     splits = (Kd + kchunk - 1) / kchunk;
     const dim3 grid((M + fv::kBgTile - 1) / fv::kBgTile, (Nc + fv::kBgTile - 1) / fv::kBgTile, nz * splits);
     fv::bwd_gemm_kernel<<<grid, fv::kThreads, 0, st>>>(M, Nc, Kd, splits, kchunk, A, Bm, C);
@@ -1005,17 +1030,17 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
     if (events && n_events < 2 * bwd_launch_count_of(sh)) return FV_ERR_SHAPE;
     EventMarks marks{events, bwd_launch_count_of(sh), 0};
 
-    // parameter gradients are sums (atomic additions): start from zero
+    // parameter gradients: written by the final fixed-order reduction; an empty batch sums to zero
     const size_t nA = (size_t)sh.nd * sh.E * sh.N, nE = (size_t)sh.nd * sh.E, nWx = (size_t)sh.nd * sh.J * sh.E,
                  nWdt = (size_t)sh.nd * sh.E * sh.R;
     cudaError_t e = cudaSuccess;
-    if ((e = cudaMemsetAsync(g->dA_log, 0, nA * sizeof(float), st)) != cudaSuccess ||
+    if (sh.B == 0 && ((e = cudaMemsetAsync(g->dA_log, 0, nA * sizeof(float), st)) != cudaSuccess ||
         (e = cudaMemsetAsync(g->dD, 0, nE * sizeof(float), st)) != cudaSuccess ||
         (e = cudaMemsetAsync(g->dW_x, 0, nWx * sizeof(float), st)) != cudaSuccess ||
         (e = cudaMemsetAsync(g->dW_dt, 0, nWdt * sizeof(float), st)) != cudaSuccess ||
         (e = cudaMemsetAsync(g->db_dt, 0, nE * sizeof(float), st)) != cudaSuccess ||
         (sh.ln && (e = cudaMemsetAsync(g->dln_gamma, 0, (size_t)sh.E * sizeof(float), st)) != cudaSuccess) ||
-        (sh.ln && (e = cudaMemsetAsync(g->dln_beta, 0, (size_t)sh.E * sizeof(float), st)) != cudaSuccess)) {
+        (sh.ln && (e = cudaMemsetAsync(g->dln_beta, 0, (size_t)sh.E * sizeof(float), st)) != cudaSuccess))) {
         note_cuda(e, "gradient reset");
         return FV_ERR_CUDA;
     }
@@ -1032,15 +1057,28 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
     float* ckpt = (float*)(ws + L.ckpt);
     // the step sizes: the forward's (staged, dt_rank >= 32), else computed below into ws
     const float* delta = L.delta ? (const float*)(ws + L.delta) : (const float*)(fw + FL.delta);
-    // the scans add dB and dC into du; the status word starts clear
-    if ((e = cudaMemsetAsync(du, 0, (size_t)sh.nd * sh.B * fv::u_block_stride(sh.T, sh.J) * sizeof(float), st)) !=
-            cudaSuccess ||
-        (e = cudaMemsetAsync(ws + L.status, 0, 2 * sizeof(unsigned), st)) != cudaSuccess) {
-        note_cuda(e, "du reset");
+    float* part_du = (float*)(ws + L.part_du);
+    float* part_dA = (float*)(ws + L.part_dA);
+    float* part_wdt = (float*)(ws + L.part_wdt);
+    float* part_bdt = (float*)(ws + L.part_bdt);
+    float* part_gate = (float*)(ws + L.part_gate);
+    // the status word starts clear
+    if ((e = cudaMemsetAsync(ws + L.status, 0, 2 * sizeof(unsigned), st)) != cudaSuccess) {
+        note_cuda(e, "status reset");
         return FV_ERR_CUDA;
     }
     const int sms = device_sm_count();
     const int M = sh.B * sh.T;
+    // one pass of bwd_reduce_kernel over `n` segments
+    auto reduce = [&](const fv::RedSegs& segs, int n, const char* where) -> fv_status {
+        long long most = 1;
+        for (int i = 0; i < n; ++i) most = std::max(most, segs.seg[i].L);
+        const long long want = (most + 31) / 32;  // 32 outputs per block at a time
+        const dim3 grid((unsigned)std::min<long long>(want, 8ll * sms), (unsigned)n);
+        fv::bwd_reduce_kernel<<<grid, fv::kRedWarps * 32, 0, st>>>(segs);
+        FV_LAUNCH_CHECK(where);
+        return FV_OK;
+    };
 
     // 1. gate, skip and repeat
     // the gate kernels are persistent over pooled rows: one wave of resident blocks
@@ -1048,8 +1086,9 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
         int per_sm = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess || per_sm < 1)
             per_sm = 1;
-        return std::min(M, per_sm * sms);
+        return std::min(std::min(M, per_sm * sms), kMaxGateBlocks);
     };
+    int gate_blocks = 0;  // rows of part_gate the gate kernel fills
     if (sh.ln) {
         const int warps = fv::bwd_ln_warps(sh.SL);
         const size_t smem = fv::bwd_ln_smem_bytes(sh.SL, warps);
@@ -1061,21 +1100,19 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
                     note_cuda(e, "LayerNorm gradient smem attribute");
                     return FV_ERR_CUDA;
                 }
-                const int grid = resident(fv::bwd_ln_gate_kernel<true>, 32 * warps, smem);
+                const int grid = gate_blocks = resident(fv::bwd_ln_gate_kernel<true>, 32 * warps, smem);
                 fv::bwd_ln_gate_kernel<true><<<grid, 32 * warps, smem, st>>>(sh, a->x, a->z, g->dy, ys, a->D,
                                                                              a->ln_gamma, a->ln_beta, row_off, row_tok,
-                                                                             g->dx, g->dz, dys, g->dD, g->dln_gamma,
-                                                                             g->dln_beta);
+                                                                             g->dx, g->dz, dys, part_gate);
             } else {
                 if ((e = ensure_smem(fv::bwd_ln_gate_kernel<false>, smem)) != cudaSuccess) {
                     note_cuda(e, "LayerNorm gradient smem attribute");
                     return FV_ERR_CUDA;
                 }
-                const int grid = resident(fv::bwd_ln_gate_kernel<false>, 32 * warps, smem);
+                const int grid = gate_blocks = resident(fv::bwd_ln_gate_kernel<false>, 32 * warps, smem);
                 fv::bwd_ln_gate_kernel<false><<<grid, 32 * warps, smem, st>>>(sh, a->x, a->z, g->dy, ys, a->D,
                                                                               a->ln_gamma, a->ln_beta, row_off,
-                                                                              row_tok, g->dx, g->dz, dys, g->dD,
-                                                                              g->dln_gamma, g->dln_beta);
+                                                                              row_tok, g->dx, g->dz, dys, part_gate);
             }
             FV_LAUNCH_CHECK("bwd_ln_gate_kernel");
             return FV_OK;
@@ -1083,19 +1120,19 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
     } else if (sh.K == 0) {
         const int threads = fv::bwd_groups(sh.SL) * fv::bwd_slot_width(sh.SL);
         auto kern = fv::bwd_gate_dense_kernel<kBwdGateTokens>;
-        const int grid = resident(kern, threads);
+        const int grid = gate_blocks = resident(kern, threads);
         FV_MARK_CALL(marks, st, ([&]() -> fv_status {
-            kern<<<grid, threads, 0, st>>>(sh, a->x, a->z, g->dy, ys, a->D, g->dx, g->dz, dys, g->dD);
+            kern<<<grid, threads, 0, st>>>(sh, a->x, a->z, g->dy, ys, a->D, g->dx, g->dz, dys, part_gate);
             FV_LAUNCH_CHECK("bwd_gate_dense_kernel");
             return FV_OK;
         })());
     } else {
         const int32_t* row_off = (const int32_t*)(fw + FL.row_off);
         const int32_t* row_tok = (const int32_t*)(fw + FL.row_tok);
-        const int grid = resident(fv::bwd_gate_masked_kernel, fv::kThreads);
+        const int grid = gate_blocks = resident(fv::bwd_gate_masked_kernel, fv::kThreads);
         FV_MARK_CALL(marks, st, ([&]() -> fv_status {
             fv::bwd_gate_masked_kernel<<<grid, fv::kThreads, 0, st>>>(sh, a->x, a->z, g->dy, ys, a->D, row_off, row_tok,
-                                                                       g->dx, g->dz, dys, g->dD);
+                                                                       g->dx, g->dz, dys, part_gate);
             FV_LAUNCH_CHECK("bwd_gate_masked_kernel");
             return FV_OK;
         })());
@@ -1112,27 +1149,36 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
                 return FV_ERR_CUDA;
             }
             fv::bwd_scan_kernel<true><<<grid, fv::kBsThreads, scan_smem, st>>>(sh, u, xbar, dys, a->A_log, a->W_dt, delta,
-                                                                              ckpt, dxs, du, g->dA_log, g->dW_dt,
-                                                                              g->db_dt);
+                                                                              ckpt, dxs, part_du, part_dA, part_wdt,
+                                                                              part_bdt);
         } else {
             if ((e = ensure_smem(fv::bwd_scan_kernel<false>, scan_smem)) != cudaSuccess) {
                 note_cuda(e, "scan gradient smem attribute");
                 return FV_ERR_CUDA;
             }
             fv::bwd_scan_kernel<false><<<grid, fv::kBsThreads, scan_smem, st>>>(sh, u, xbar, dys, a->A_log, a->W_dt,
-                                                                               delta, ckpt, dxs, du, g->dA_log,
-                                                                               g->dW_dt, g->db_dt);
+                                                                               delta, ckpt, dxs, part_du, part_dA,
+                                                                               part_wdt, part_bdt);
         }
         FV_LAUNCH_CHECK("bwd_scan_kernel");
         return FV_OK;
     })());
-    // 3. x_proj: dW_x = du^T xbar, dxbar = the scans' share + sum_k du[k] W_x[k]
+    // du = the sum of the 64-channel tiles' shares, in tile order
     {
-        const int tiles = ((sh.J + 63) / 64) * ((sh.E + 63) / 64) * sh.nd;
-        FV_MARK_CALL(marks, st, launch_bwd_gemm(sh.J, sh.E, M, sh.nd, bwd_splits(M, tiles, sms), fv::OpDuJM{du, sh},
-                                                fv::OpXbar{xbar, sh.E}, fv::OutWx{g->dW_x, sh.J, sh.E}, st,
-                                                "bwd_gemm_kernel (W_x)"));
+        const int tiles = (sh.E + fv::kBsCh - 1) / fv::kBsCh;
+        const long long ub = (long long)fv::u_block_stride(sh.T, sh.J), L_du = (long long)sh.nd * sh.B * ub;
+        fv::RedSegs segs{};
+        segs.seg[0] = fv::RedSeg{part_du, du, L_du, L_du, 0, ub, (long long)sh.T * sh.J, tiles, 1};
+        FV_MARK_CALL(marks, st, reduce(segs, 1, "bwd_reduce_kernel (du)"));
     }
+    // 3. x_proj: dW_x = du^T xbar (split-K partials), dxbar = the scans' share + sum_k du[k] W_x[k]
+    const int wx_tiles = ((sh.J + 63) / 64) * ((sh.E + 63) / 64) * sh.nd;
+    const int wx_chunk = bwd_kchunk(M, std::min(bwd_splits(M, wx_tiles, sms), kMaxWxSplits));
+    const int wx_splits = (M + wx_chunk - 1) / wx_chunk;
+    FV_MARK_CALL(marks, st, launch_bwd_gemm(sh.J, sh.E, M, sh.nd, wx_splits, fv::OpDuJM{du, sh},
+                                            fv::OpXbar{xbar, sh.E},
+                                            fv::OutWx{(float*)(ws + L.part_wx), sh.J, sh.E, sh.nd, wx_splits}, st,
+                                            "bwd_gemm_kernel (W_x)"));
     FV_MARK_CALL(marks, st, launch_bwd_gemm(M, sh.E, sh.nd * sh.J, 1, 1, fv::OpDuMK{du, sh}, fv::OpWx{a->W_x, sh.E},
                                             fv::OutDxbar{dxbar, dxs, sh.T, sh.E, sh.nd}, st,
                                             "bwd_gemm_kernel (xbar)"));
@@ -1153,6 +1199,26 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
             FV_LAUNCH_CHECK("bwd_pool_masked_kernel");
             return FV_OK;
         })());
+    }
+    // 5. the batch sums of the parameter gradients, each added in a fixed order (images, K splits,
+    // gate blocks), so that every run gives the same bits
+    {
+        const long long E = sh.E, nd = sh.nd, ne = nd * E;
+        fv::RedSegs segs{};
+        int n = 0;
+        segs.seg[n++] = fv::RedSeg{part_dA, g->dA_log, ne * sh.N, ne * sh.N, 0, 0, 0, sh.B, 1};
+        segs.seg[n++] = fv::RedSeg{part_wdt, g->dW_dt, ne * sh.R, ne * sh.R, 0, 0, 0, sh.B, 1};
+        segs.seg[n++] = fv::RedSeg{part_bdt, g->db_dt, ne, ne, 0, 0, 0, sh.B, 1};
+        segs.seg[n++] = fv::RedSeg{(const float*)(ws + L.part_wx), g->dW_x, (long long)nWx, (long long)nWx, 0, 0, 0,
+                                   wx_splits, 1};
+        if (sh.ln) {  // part_gate rows: dgamma | dbeta | dD per gate block
+            segs.seg[n++] = fv::RedSeg{part_gate, g->dln_gamma, E, 3 * E, 0, 0, 0, gate_blocks, 1};
+            segs.seg[n++] = fv::RedSeg{part_gate + E, g->dln_beta, E, 3 * E, 0, 0, 0, gate_blocks, 1};
+            segs.seg[n++] = fv::RedSeg{part_gate + 2 * E, g->dD, E, 3 * E, E, 0, 0, gate_blocks, (int)nd};
+        } else {  // dD is the same sum for every direction
+            segs.seg[n++] = fv::RedSeg{part_gate, g->dD, E, E, E, 0, 0, gate_blocks, (int)nd};
+        }
+        FV_MARK_CALL(marks, st, reduce(segs, n, "bwd_reduce_kernel (params)"));
     }
     return FV_OK;
 }
@@ -1175,7 +1241,7 @@ fv_status fastvim_ssm_backward_workspace_layout(const fv_ssm_args* args, fv_bwd_
     const BwdLayout L = plan_bwd(sh);
     out->total_bytes = L.total;
     out->dys = L.dys; out->dxbar = L.dxbar; out->du = L.du; out->dxs = L.dxs; out->ckpt = L.ckpt;
-    out->status = L.status; out->delta = L.delta;
+    out->status = L.status; out->delta = L.delta; out->partials = L.partials;
     return FV_OK;
 }
 

@@ -41,7 +41,7 @@ __host__ __device__ __forceinline__ size_t bs_smem_floats(int R) {
            + (size_t)kBsChunk * R             // dt_low of the chunk's steps
            + (size_t)kBsChunk * 32            // B | C of the chunk's steps
            + 6 * (size_t)kBsChunk * kBsCh     // xbar, dys, Delta, sig(v), dv, dxbar (scan share)
-           + (size_t)kBsChunk * 32            // dB | dC sums of the chunk
+           + (size_t)(kBsThreads / 32) * kBsChunk * 32  // dB | dC sums of the chunk, one row per warp
            + (size_t)kBsCh * (R + 1);         // dW_dt | db_dt sums of the CTA's channels
 }
 
@@ -92,14 +92,15 @@ __host__ __device__ __forceinline__ int bwd_groups(int SL) { return kThreads / b
 
 // Dense gate gradient, persistent over pooled rows (b, t) (grid-stride), launched with
 // bwd_groups(SL) * bwd_slot_width(SL) threads.  Writes dz and the skip part of dx for every token
-// of the row, dys[b][t] (the sum of ds over the row's S tokens), and adds the block's dD sums.
+// of the row, dys[b][t] (the sum of ds over the row's S tokens), and the block's dD sums into row
+// blockIdx.x of part_dD ([gridDim.x][E]; bwd_reduce_kernel adds the rows in block order).
 // U tokens per thread in flight (3 U 128-bit loads).
 template <int U>
 __global__ void __launch_bounds__(kThreads)
 bwd_gate_dense_kernel(Shape sh, const float* __restrict__ x, const float* __restrict__ z,
                       const float* __restrict__ dy, const float* __restrict__ ys, const float* __restrict__ D,
                       float* __restrict__ dx, float* __restrict__ dz, float* __restrict__ dys,
-                      float* __restrict__ dD) {
+                      float* __restrict__ part_dD) {
     __shared__ float4 part[kThreads];
     const int SL = sh.SL, SW = bwd_slot_width(SL), G = bwd_groups(SL);
     const int ls = threadIdx.x % SW, g = threadIdx.x / SW;
@@ -159,13 +160,10 @@ bwd_gate_dense_kernel(Shape sh, const float* __restrict__ x, const float* __rest
         }
         part[threadIdx.x] = dDa;
         __syncthreads();
-        if (g == 0 && slot < SL) {
+        if (g == 0 && slot < SL) {  // this block's dD sums (the same for every direction)
             float4 sum = part[ls];
             for (int q = 1; q < G; ++q) f4_add(sum, part[q * SW + ls]);
-            for (int k = 0; k < sh.nd; ++k) {
-                float* d = dD + (size_t)k * sh.E + 4 * slot;
-                atomicAdd(d + 0, sum.x); atomicAdd(d + 1, sum.y); atomicAdd(d + 2, sum.z); atomicAdd(d + 3, sum.w);
-            }
+            reinterpret_cast<float4*>(part_dD + (size_t)blockIdx.x * sh.E)[slot] = sum;
         }
         __syncthreads();
     }
@@ -179,7 +177,7 @@ bwd_gate_masked_kernel(Shape sh, const float* __restrict__ x, const float* __res
                        const float* __restrict__ dy, const float* __restrict__ ys, const float* __restrict__ D,
                        const int32_t* __restrict__ row_off, const int32_t* __restrict__ row_tok,
                        float* __restrict__ dx, float* __restrict__ dz, float* __restrict__ dys,
-                       float* __restrict__ dD) {
+                       float* __restrict__ part_dD) {
     const int SL = sh.SL, K = sh.K, T = sh.T;
     const int rows = sh.B * T;
     const float4* x4 = reinterpret_cast<const float4*>(x);
@@ -222,12 +220,7 @@ bwd_gate_masked_kernel(Shape sh, const float* __restrict__ x, const float* __res
             }
             reinterpret_cast<float4*>(dys + (size_t)bt * sh.E)[slot] = acc;
         }
-        if (act) {
-            for (int k = 0; k < sh.nd; ++k) {
-                float* d = dD + (size_t)k * sh.E + 4 * slot;
-                atomicAdd(d + 0, dDa.x); atomicAdd(d + 1, dDa.y); atomicAdd(d + 2, dDa.z); atomicAdd(d + 3, dDa.w);
-            }
-        }
+        if (act) reinterpret_cast<float4*>(part_dD + (size_t)blockIdx.x * sh.E)[slot] = dDa;  // this block's sums
     }
 }
 
@@ -255,9 +248,10 @@ __host__ __forceinline__ size_t bwd_ln_smem_bytes(int SL, int warps) {
 // Three passes over the token's channels: the statistics of s, the two means of gs, the outputs;
 // the first pass reads x and the second z and dy from HBM, the repeats hit L1.  Every lane owns
 // the same float4 slots in every pass, so each warp sums dys, dgamma, dbeta and dD into private
-// shared-memory rows with no atomics; the rows meet at the end of each pooled row (dys) and of
-// the kernel (one global atomic per channel per block for the batch sums).  Masked layers take a
-// row's kept tokens from the forward's row lists; a rejected id is in no row (dx, dz zeroed by
+// shared-memory rows with no atomics; the rows meet, in warp order, at the end of each pooled row
+// (dys) and of the kernel (the block's batch sums: row blockIdx.x of part_ln, [gridDim.x][3][E] =
+// dgamma | dbeta | dD, added in block order by bwd_reduce_kernel).  Masked layers take a row's kept
+// tokens from the forward's row lists; a rejected id is in no row (dx, dz zeroed by
 // bwd_pool_masked_kernel).
 template <bool MASKED>
 __global__ void __launch_bounds__(128)
@@ -265,8 +259,7 @@ bwd_ln_gate_kernel(Shape sh, const float* __restrict__ x, const float* __restric
                    const float* __restrict__ ys, const float* __restrict__ D, const float* __restrict__ gamma,
                    const float* __restrict__ beta, const int32_t* __restrict__ row_off,
                    const int32_t* __restrict__ row_tok, float* __restrict__ dx, float* __restrict__ dz,
-                   float* __restrict__ dys, float* __restrict__ dD, float* __restrict__ dgamma,
-                   float* __restrict__ dbeta) {
+                   float* __restrict__ dys, float* __restrict__ part_ln) {
     extern __shared__ float4 lgs[];
     const int SL = sh.SL, W = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -387,14 +380,10 @@ bwd_ln_gate_kernel(Shape sh, const float* __restrict__ x, const float* __restric
             f4_add(sb, r[2 * SL + slot]);
             f4_add(sd, r[3 * SL + slot]);
         }
-        float* pg = dgamma + 4 * slot;
-        float* pb = dbeta + 4 * slot;
-        atomicAdd(pg + 0, sg.x); atomicAdd(pg + 1, sg.y); atomicAdd(pg + 2, sg.z); atomicAdd(pg + 3, sg.w);
-        atomicAdd(pb + 0, sb.x); atomicAdd(pb + 1, sb.y); atomicAdd(pb + 2, sb.z); atomicAdd(pb + 3, sb.w);
-        for (int k = 0; k < sh.nd; ++k) {
-            float* d = dD + (size_t)k * sh.E + 4 * slot;
-            atomicAdd(d + 0, sd.x); atomicAdd(d + 1, sd.y); atomicAdd(d + 2, sd.z); atomicAdd(d + 3, sd.w);
-        }
+        float4* row = reinterpret_cast<float4*>(part_ln + (size_t)blockIdx.x * 3 * sh.E);
+        row[slot] = sg;
+        row[SL + slot] = sb;
+        row[2 * SL + slot] = sd;
     }
 }
 
@@ -415,20 +404,22 @@ bwd_ln_gate_kernel(Shape sh, const float* __restrict__ x, const float* __restric
 // (ckpt [B][nd][2 nchunks][E][16]).  Pass 2 walks the 16-step staged chunks in reverse, each as two
 // halves of 8 steps, last half first: it recomputes the half's states from its checkpoint (8 steps
 // x 4 states in registers, which keeps the kernel at two resident blocks per SM) and steps the
-// adjoint back through them.  Per step: dDelta and the scans' dxbar are summed over the 4 lanes of a channel (written as
-// dv = dDelta sig(v) and dxs [B][nd][T][E]); dB and dC are summed over the warp's 8 channels by a
-// transposing butterfly, over the block's 8 warps in shared memory, and over the E / 64 blocks of
-// an image with global atomics into du (zeroed by the caller).  dA_log (= dA A) sums in registers
-// over all steps, then one atomic per state.  dt_proj (v = W_dt dt_low + b_dt) is differentiated
-// here too, from the chunk's dv and dt_low already in shared memory: d dt_low[t] = sum over the
-// block's channels of W_dt[e] dv[t][e] (atomics into du's dt_low slots), dW_dt[e] and db_dt[e] =
-// sums over the steps of dv[t][e] [dt_low[t] | 1] (shared memory, one atomic each at the end).
+// adjoint back through them.  Per step: dDelta and the scans' dxbar are summed over the 4 lanes of
+// a channel (written as dv = dDelta sig(v) and dxs [B][nd][T][E]); dB and dC are summed over the
+// warp's 8 channels by a transposing butterfly, then over the block's 8 warps (one shared row per
+// warp, added in warp order).  dA_log (= dA A) sums in registers over all steps.  dt_proj
+// (v = W_dt dt_low + b_dt) is differentiated here too, from the chunk's dv and dt_low already in
+// shared memory: d dt_low[t] = sum over the block's channels of W_dt[e] dv[t][e], dW_dt[e] and
+// db_dt[e] = sums over the steps of dv[t][e] [dt_low[t] | 1].  No atomics: the block's du terms go
+// to its own copy of du's layout in part_du (one per 64-channel tile) and its parameter terms to
+// per-image slots; bwd_reduce_kernel adds tiles and images in a fixed order, so the sums are the
+// same in every run.
 template <bool ZOH_EXACT>
 __global__ void __launch_bounds__(kBsThreads, 2)
 bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__ xbar, const float* __restrict__ dys,
                 const float* __restrict__ A_log, const float* __restrict__ W_dt, const float* __restrict__ delta,
-                float* __restrict__ ckpt, float* __restrict__ dxs, float* __restrict__ du,
-                float* __restrict__ dA_log, float* __restrict__ dW_dt, float* __restrict__ db_dt) {
+                float* __restrict__ ckpt, float* __restrict__ dxs, float* __restrict__ part_du,
+                float* __restrict__ part_dA, float* __restrict__ part_wdt, float* __restrict__ part_bdt) {
     extern __shared__ float bsm[];
     const int b = blockIdx.x, k = blockIdx.y, e0 = blockIdx.z * kBsCh;
     const int T = sh.T, E = sh.E, N = sh.N, R = sh.R, J = sh.J;
@@ -442,8 +433,8 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
     float* ssg = sdl + kBsChunk * kBsCh;      // [16][64]
     float* sdv = ssg + kBsChunk * kBsCh;      // [16][64]
     float* sdx = sdv + kBsChunk * kBsCh;      // [16][64]
-    float* sred = sdx + kBsChunk * kBsCh;     // [16][32]
-    float* swacc = sred + kBsChunk * 32;      // [64][R + 1]
+    float* sred = sdx + kBsChunk * kBsCh;     // [8 warps][16][32]
+    float* swacc = sred + (kBsThreads / 32) * kBsChunk * 32;  // [64][R + 1]
     const int tid = threadIdx.x;
     const int c = tid >> 2, q = tid & 3, lane = tid & 31;
     const int e = e0 + c;
@@ -451,6 +442,9 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
     const bool fwd = sh.nd == 2 ? k == 0 : (sh.dir_flags & 1u) != 0;
     const int nchunks = bs_nchunks(T), nckpt = bs_nckpt(T);
     const float* ub = u + u_offset(sh, k, b, 0);
+    // this CTA's share of du (dB, dC and d dt_low summed over its 64 channels): part_du holds one
+    // copy of du's layout per 64-channel tile
+    float* pdu = part_du + (size_t)blockIdx.z * sh.nd * sh.B * u_block_stride(T, J);
     auto ckpt_at = [&](int c) { return ckpt + ((((size_t)b * sh.nd + k) * nckpt + c) * E + e) * 16 + 4 * q; };
 
     for (int i = tid; i < kBsCh * R; i += kBsThreads) {
@@ -488,7 +482,6 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
         for (int i = tid; i < kBsChunk * 32; i += kBsThreads) {
             const int s = i >> 5, j = i & 31, n = j & 15;
             sbc[i] = (s < len && n < N) ? ub[(size_t)t_of(it, s) * J + R + (j < 16 ? n : N + n)] : 0.f;
-            if (pass2) sred[i] = 0.f;
         }
         for (int i = tid; i < kBsChunk * kBsCh; i += kBsThreads) {
             const int s = i / kBsCh, cc = i - s * kBsCh;
@@ -620,7 +613,7 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
                     const float send = b2 ? r2[0] : r2[1];
                     const float keep = b2 ? r2[1] : r2[0];
                     const float fin = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-                    if (red_n < N) atomicAdd(&sred[i * 32 + red_w * 16 + red_n], fin);
+                    if (red_n < N) sred[((tid >> 5) * kBsChunk + i) * 32 + red_w * 16 + red_n] = fin;
                 }
             }
         }
@@ -629,16 +622,20 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
             const int s = i / kBsCh, cc = i - s * kBsCh;
             if (e0 + cc < E) dxs[(((size_t)b * sh.nd + k) * T + t_of(it, s)) * E + e0 + cc] = sdx[i];
         }
-        for (int i = tid; i < len * 32; i += kBsThreads) {
+        for (int i = tid; i < len * 32; i += kBsThreads) {  // the warps' dB | dC rows, in warp order
             const int s = i >> 5, j = i & 31, n = j & 15;
-            if (n < N) atomicAdd(du + u_offset(sh, k, b, t_of(it, s)) + R + (j < 16 ? n : N + n), sred[i]);
+            if (n < N) {
+                float acc = sred[i];
+                for (int w = 1; w < kBsThreads / 32; ++w) acc += sred[w * kBsChunk * 32 + i];
+                pdu[u_offset(sh, k, b, t_of(it, s)) + R + (j < 16 ? n : N + n)] = acc;
+            }
         }
         // dt_proj: d dt_low of the chunk's steps (this block's channels), dW_dt | db_dt partial sums
         for (int i = tid; i < len * R; i += kBsThreads) {
             const int s = i / R, r = i - s * R;
             float acc = 0.f;
             for (int cc = 0; cc < kBsCh; ++cc) acc = fmaf(sw[cc * WS + r], sdv[s * kBsCh + cc], acc);
-            atomicAdd(du + u_offset(sh, k, b, t_of(it, s)) + r, acc);
+            pdu[u_offset(sh, k, b, t_of(it, s)) + r] = acc;
         }
         for (int i = tid; i < kBsCh * (R + 1); i += kBsThreads) {
             const int cc = i / (R + 1), r = i - cc * (R + 1);
@@ -648,15 +645,20 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
         }
         __syncthreads();  // the buffers are refilled by the next stage()
     }
+    // this image's dW_dt | db_dt and dA_log terms (part_wdt [B][nd][E][R], part_bdt [B][nd][E],
+    // part_dA [B][nd][E][N]; bwd_reduce_kernel adds the images in order)
+    const size_t img = (size_t)b * sh.nd + k;
     for (int i = tid; i < kBsCh * (R + 1); i += kBsThreads) {  // each entry was summed by this thread
         const int cc = i / (R + 1), r = i - cc * (R + 1);
-        if (e0 + cc < E) atomicAdd(r < R ? dW_dt + ((size_t)k * E + e0 + cc) * R + r : db_dt + (size_t)k * E + e0 + cc,
-                                   swacc[i]);
+        if (e0 + cc < E) {
+            if (r < R) part_wdt[(img * E + e0 + cc) * R + r] = swacc[i];
+            else part_bdt[img * E + e0 + cc] = swacc[i];
+        }
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int n = 4 * q + j;
-        if (live && n < N) atomicAdd(dA_log + ((size_t)k * E + e) * N + n, gA[j] * An[j]);
+        if (live && n < N) part_dA[(img * E + e) * N + n] = gA[j] * An[j];
     }
 }
 
@@ -702,13 +704,18 @@ struct OpWx {
 };
 
 // Outputs.
-struct OutWx {  // split-K partial sums of dW_x
-    float* dW_x; int J, E;
-    __device__ void operator()(int k, int i, int j, float v) const {
-        atomicAdd(dW_x + ((size_t)k * J + i) * E + j, v);
+struct OutWx {  // split-K partial sums of dW_x: part [splits][nd][J][E], added in split order later
+    static constexpr bool kVec4 = true;  // 4 consecutive j at once (E is a multiple of 4)
+    float* part; int J, E, nd, splits;
+    __device__ float* at(int k, int i, int j) const {
+        const int s = (int)blockIdx.z % splits;  // the GEMM's grid z is (direction, split)
+        return part + (((size_t)s * nd + k) * J + i) * E + j;
     }
+    __device__ void operator()(int k, int i, int j, float v) const { *at(k, i, j) = v; }
+    __device__ void store4(int k, int i, int j, float4 v) const { *reinterpret_cast<float4*>(at(k, i, j)) = v; }
 };
 struct OutDxbar {  // dxbar = the scans' share (summed over directions) + the projections' share
+    static constexpr bool kVec4 = false;
     float* dxbar; const float* dxs; int T, E, nd;
     __device__ void operator()(int, int i, int j, float v) const {
         const int b = i / T, t = i - b * T;
@@ -763,12 +770,74 @@ bwd_gemm_kernel(int M, int Nc, int Kd, int splits, int kchunk, AOp A, BOp Bm, CO
         __syncthreads();
     }
 #pragma unroll
-    for (int p = 0; p < 4; ++p)
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int gi = i0 + ty * 4 + p, gj = j0 + tx * 4 + r;
-            if (gi < M && gj < Nc) C(k, gi, gj, acc[p][r]);
+    for (int p = 0; p < 4; ++p) {
+        const int gi = i0 + ty * 4 + p, gj = j0 + tx * 4;
+        if constexpr (COp::kVec4) {
+            if (gi < M && gj + 3 < Nc) {
+                C.store4(k, gi, gj, make_float4(acc[p][0], acc[p][1], acc[p][2], acc[p][3]));
+                continue;
+            }
         }
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+            if (gi < M && gj + r < Nc) C(k, gi, gj + r, acc[p][r]);
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// Fixed-order sums of per-block partials (reproducible batch sums)
+// ------------------------------------------------------------------------------------------
+
+// out[c * out_stride + i] = the sum over p < P of part[p][i] (partial p starts at
+// part + p * part_stride) for i < L and c < copies; with blk > 0 entries whose i % blk >= valid are
+// padding and get 0.
+struct RedSeg {
+    const float* part;
+    float* out;
+    long long L, part_stride, out_stride, blk, valid;
+    int P, copies;
+};
+constexpr int kMaxRedSegs = 8;
+struct RedSegs {
+    RedSeg seg[kMaxRedSegs];
+};
+// Grid (x, number of segments): blockIdx.y picks the segment.  Few partials (P <= 32): one
+// thread per output adds them in order.  Many: a block takes 32 consecutive outputs at a time (one
+// per lane: coalesced loads) and splits the P partials over its 8 warps (warp w adds partials
+// w, w + 8, ... in order); the 8 warp sums are then added in warp order.  Either grouping depends
+// on nothing but P, so the result is the same in every run.
+constexpr int kRedWarps = 8;
+__global__ void __launch_bounds__(kRedWarps * 32)
+bwd_reduce_kernel(RedSegs segs) {
+    __shared__ float wsum[kRedWarps][32];
+    const RedSeg g = segs.seg[blockIdx.y];
+    if (g.P <= 32) {
+        for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < g.L;
+             i += (long long)gridDim.x * blockDim.x) {
+            float acc = 0.f;
+            if (g.blk == 0 || i % g.blk < g.valid)
+                for (int p = 0; p < g.P; ++p) acc += g.part[(size_t)p * g.part_stride + i];
+            for (int c = 0; c < g.copies; ++c) g.out[(size_t)c * g.out_stride + i] = acc;
+        }
+        return;
+    }
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    for (long long i0 = (long long)blockIdx.x * 32; i0 < g.L; i0 += (long long)gridDim.x * 32) {
+        const long long i = i0 + lane;
+        float acc = 0.f;
+        if (i < g.L && (g.blk == 0 || i % g.blk < g.valid)) {
+#pragma unroll 4
+            for (int p = w; p < g.P; p += kRedWarps) acc += g.part[(size_t)p * g.part_stride + i];
+        }
+        wsum[w][lane] = acc;
+        __syncthreads();
+        if (w == 0 && i < g.L) {
+            float sum = wsum[0][lane];
+            for (int q = 1; q < kRedWarps; ++q) sum += wsum[q][lane];
+            for (int c = 0; c < g.copies; ++c) g.out[(size_t)c * g.out_stride + i] = sum;
+        }
+        __syncthreads();
+    }
 }
 
 // ------------------------------------------------------------------------------------------

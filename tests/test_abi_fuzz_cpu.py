@@ -105,6 +105,9 @@ def _check_layout(lib, a):
         if L.trace:
             assert a.flags & nat.FV_FLAG_TRACE and L.trace_records > 0
             regions.append((L.trace, L.trace_records * 32))
+    if L.delta:  # the staged path's step sizes (dt_rank >= 32)
+        assert a.R >= 32
+        regions.append((L.delta, L.nd * B * T * E * 4))
     regions.sort()
     end = 0
     for off, n in regions:
@@ -222,7 +225,7 @@ def test_gradient_validation_and_plan(a, pick):
     for off, n in regions:
         assert off % 256 == 0 and off >= end
         end = off + n
-    assert end <= L.total_bytes < end + 256 * len(regions)
+    assert end <= L.partials < L.total_bytes  # then the partial sums of the fixed-order reductions
     n = lib.fastvim_ssm_backward_launch_count(ctypes.byref(a))
     names = [lib.fastvim_ssm_backward_launch_name(ctypes.byref(a), i).decode() for i in range(n)]
     if a.B == 0:
@@ -231,7 +234,8 @@ def test_gradient_validation_and_plan(a, pick):
         first = ("bwd_ln_gate_kernel" if a.flags & nat.FV_FLAG_LAYERNORM else
                  "bwd_gate_masked_kernel" if a.K else "bwd_gate_dense_kernel")
         mid = ["bwd_scan_kernel"] if FL.delta else ["dt_proj_kernel", "bwd_scan_kernel"]
-        assert names[0] == first and names[1:1 + len(mid)] == mid and len(names) == 4 + len(mid)
+        assert names[0] == first and names[1:1 + len(mid)] == mid and len(names) == 6 + len(mid)
+        assert names[-1] == "bwd_reduce_kernel:params"
     g = _grads_for(a)
     fws = lib.fastvim_ssm_workspace_size(ctypes.byref(a))
 

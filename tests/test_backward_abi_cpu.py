@@ -47,12 +47,12 @@ def test_struct_layouts_match_header(tmp_path):
     src = tmp_path / "off.c"
     src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "fastvim_ssm.h"\n'
                    'int main(void){printf("%zu %zu %zu %zu\\n", sizeof(fv_ssm_grads), offsetof(fv_ssm_grads, db_dt), '
-                   'sizeof(fv_bwd_ws_layout), offsetof(fv_bwd_ws_layout, delta)); return 0;}\n')
+                   'sizeof(fv_bwd_ws_layout), offsetof(fv_bwd_ws_layout, partials)); return 0;}\n')
     exe = tmp_path / "off"
     subprocess.run(["gcc", "-std=c99", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)], check=True)
     got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
     assert got == [ctypes.sizeof(nat.FvSsmGrads), nat.FvSsmGrads.db_dt.offset, ctypes.sizeof(nat.FvBwdWsLayout),
-                   nat.FvBwdWsLayout.delta.offset]
+                   nat.FvBwdWsLayout.partials.offset]
 
 
 @pytest.mark.parametrize("pool_axis,K,dirs", [(0, 0, 3), (1, 0, 1), (0, 37, 3), (1, 37, 2)])
@@ -77,28 +77,29 @@ def test_workspace_plan(lib, pool_axis, K, dirs):
     for off, n in regions:
         assert off % 256 == 0 and off >= end
         end = off + n
-    assert end <= L.total_bytes < end + 256
+    assert end <= L.partials < L.total_bytes  # then the partial sums of the fixed-order reductions
 
 
 def test_launch_lists(lib):
     # dt_rank 12: the forward workspace holds no step sizes, so the gradient computes them first
-    dense = [lib.fastvim_ssm_backward_launch_name(ctypes.byref(args()), i).decode() for i in range(6)]
-    assert lib.fastvim_ssm_backward_launch_count(ctypes.byref(args())) == 6
-    assert dense == ["bwd_gate_dense_kernel", "dt_proj_kernel", "bwd_scan_kernel", "bwd_gemm_kernel:W_x",
-                     "bwd_gemm_kernel:xbar", "bwd_pool_dense_kernel"]
+    dense = [lib.fastvim_ssm_backward_launch_name(ctypes.byref(args()), i).decode() for i in range(8)]
+    assert lib.fastvim_ssm_backward_launch_count(ctypes.byref(args())) == 8
+    assert dense == ["bwd_gate_dense_kernel", "dt_proj_kernel", "bwd_scan_kernel", "bwd_reduce_kernel:du",
+                     "bwd_gemm_kernel:W_x", "bwd_gemm_kernel:xbar", "bwd_pool_dense_kernel",
+                     "bwd_reduce_kernel:params"]
     m = args(K=49, keep_idx=FAKE + 9 * SLOT)
-    masked = [lib.fastvim_ssm_backward_launch_name(ctypes.byref(m), i).decode() for i in range(6)]
-    assert masked[0] == "bwd_gate_masked_kernel" and masked[-1] == "bwd_pool_masked_kernel"
-    assert lib.fastvim_ssm_backward_launch_name(ctypes.byref(args()), 6) == b""
+    masked = [lib.fastvim_ssm_backward_launch_name(ctypes.byref(m), i).decode() for i in range(8)]
+    assert masked[0] == "bwd_gate_masked_kernel" and masked[-2] == "bwd_pool_masked_kernel"
+    assert lib.fastvim_ssm_backward_launch_name(ctypes.byref(args()), 8) == b""
     assert lib.fastvim_ssm_backward_launch_count(ctypes.byref(args(B=0, x=None, z=None, y=None))) == 0
     ln = args(flags=nat.FV_FLAG_LAYERNORM, ln_gamma=FAKE + 10 * SLOT, ln_beta=FAKE + 11 * SLOT, ln_eps=1e-5)
-    names = [lib.fastvim_ssm_backward_launch_name(ctypes.byref(ln), i).decode() for i in range(6)]
-    assert lib.fastvim_ssm_backward_launch_count(ctypes.byref(ln)) == 6
+    names = [lib.fastvim_ssm_backward_launch_name(ctypes.byref(ln), i).decode() for i in range(8)]
+    assert lib.fastvim_ssm_backward_launch_count(ctypes.byref(ln)) == 8
     assert names[0] == "bwd_ln_gate_kernel" and names[1:] == dense[1:]
     # dt_rank 48 on the staged path: the forward's step sizes are read, no dt_proj launch
     big = args(h=64, w=64, E=1536, R=48, K=1024, keep_idx=FAKE + 9 * SLOT)
     n = lib.fastvim_ssm_backward_launch_count(ctypes.byref(big))
-    assert n == 5 and "dt_proj_kernel" not in [lib.fastvim_ssm_backward_launch_name(ctypes.byref(big), i).decode()
+    assert n == 7 and "dt_proj_kernel" not in [lib.fastvim_ssm_backward_launch_name(ctypes.byref(big), i).decode()
                                                for i in range(n)]
     L = nat.FvBwdWsLayout()
     assert lib.fastvim_ssm_backward_workspace_layout(ctypes.byref(big), ctypes.byref(L)) == nat.FV_OK
