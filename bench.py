@@ -72,7 +72,7 @@ def kernel_work(name: str, cfg, pool_axis: int):
     if name == "dt_proj_kernel":
         return "hbm", 4 * cfg.B * T * cfg.E * cfg.nd          # Delta written (tensor-core GEMM, K = R)
     # the gradient's kernels
-    if name in ("bwd_gate_dense_kernel", "bwd_gate_masked_kernel", "bwd_ln_gate_kernel"):
+    if name in ("bwd_gate_dense_kernel", "bwd_gate_masked_kernel", "bwd_ln_gate_kernel", "bwd_ln_gate_reg_kernel"):
         return "hbm", 5 * row * tok                   # read x, z, dy; write dz and dx
     if name == "bwd_pool_dense_kernel":
         return "hbm", 2 * row * tok                   # dx read and written back (+ the pooled share)

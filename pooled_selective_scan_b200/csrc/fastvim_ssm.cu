@@ -927,6 +927,9 @@ BwdLayout plan_bwd(const fv::Shape& sh) {
 // Launch order of a gradient call: gate (through the LayerNorm with FV_FLAG_LAYERNORM), dt_proj
 // (when the forward workspace holds no step sizes), scans (with dt_proj's gradient), dW_x, dxbar,
 // pooling.
+// The LayerNorm gate gradient keeps each token in registers across groups of up to 8 warps
+// (E <= 2048); wider rows take the shared-memory-row kernel.
+bool bwd_ln_uses_reg(const fv::Shape& sh) { return fv::bwd_lnr_wpt(sh.SL) <= 8; }
 int bwd_launch_count_of(const fv::Shape& sh) { return sh.B == 0 ? 0 : (fwd_has_delta(sh) ? 7 : 8); }
 const char* bwd_launch_name_of(const fv::Shape& sh, int i) {
     static const char* dense[] = {"bwd_gate_dense_kernel", "dt_proj_kernel", "bwd_scan_kernel", "bwd_reduce_kernel:du",
@@ -937,7 +940,7 @@ const char* bwd_launch_name_of(const fv::Shape& sh, int i) {
                                    "bwd_reduce_kernel:params"};
     const int n = bwd_launch_count_of(sh);
     if (i < 0 || i >= n) return "";
-    if (i == 0 && sh.ln) return "bwd_ln_gate_kernel";
+    if (i == 0 && sh.ln) return bwd_ln_uses_reg(sh) ? "bwd_ln_gate_reg_kernel" : "bwd_ln_gate_kernel";
     const int j = (n == 7 && i >= 1) ? i + 1 : i;
     return sh.K > 0 ? masked[j] : dense[j];
 }
@@ -1089,7 +1092,24 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
         return std::min(std::min(M, per_sm * sms), kMaxGateBlocks);
     };
     int gate_blocks = 0;  // rows of part_gate the gate kernel fills
-    if (sh.ln) {
+    if (sh.ln && bwd_ln_uses_reg(sh)) {
+        const int threads = 32 * fv::bwd_lnr_wpt(sh.SL) * fv::bwd_lnr_groups(sh.SL);
+        const size_t smem = fv::bwd_lnr_smem_bytes(sh.SL);
+        const int32_t* row_off = sh.K > 0 ? (const int32_t*)(fw + FL.row_off) : nullptr;
+        const int32_t* row_tok = sh.K > 0 ? (const int32_t*)(fw + FL.row_tok) : nullptr;
+        auto kern = sh.K > 0 ? fv::bwd_ln_gate_reg_kernel<true> : fv::bwd_ln_gate_reg_kernel<false>;
+        if ((e = ensure_smem(kern, smem)) != cudaSuccess) {
+            note_cuda(e, "LayerNorm gradient smem attribute");
+            return FV_ERR_CUDA;
+        }
+        const int grid = gate_blocks = resident(kern, threads, smem);
+        FV_MARK_CALL(marks, st, ([&]() -> fv_status {
+            kern<<<grid, threads, smem, st>>>(sh, a->x, a->z, g->dy, ys, a->D, a->ln_gamma, a->ln_beta, row_off, row_tok,
+                                              g->dx, g->dz, dys, part_gate);
+            FV_LAUNCH_CHECK("bwd_ln_gate_reg_kernel");
+            return FV_OK;
+        })());
+    } else if (sh.ln) {
         const int warps = fv::bwd_ln_warps(sh.SL);
         const size_t smem = fv::bwd_ln_smem_bytes(sh.SL, warps);
         const int32_t* row_off = sh.K > 0 ? (const int32_t*)(fw + FL.row_off) : nullptr;

@@ -387,6 +387,214 @@ bwd_ln_gate_kernel(Shape sh, const float* __restrict__ x, const float* __restric
     }
 }
 
+// The same gradient with each token's values in registers.  A group of WPT warps takes one token
+// (thread gt of the group owns float4 slots gt + 32 WPT u, u < 2: E <= 256 WPT); a
+// block of NG groups is persistent over pooled rows, its groups taking the row's tokens in turn.
+// Per token: x, z and dy are loaded at once; pass 1 forms s and its shifted moments, pass 2 the
+// two means of gs, pass 3 writes dz, dx from the registers.  The group's sums (moments, means) go
+// through a shared-memory slot per warp, added in warp order behind a named barrier of the group.
+// dys of the current row and the batch sums of dgamma, dbeta, dD stay in each thread's registers;
+// the groups' dys meet in shared memory at the end of each row, the batch sums at the end of the
+// kernel (row blockIdx.x of part_ln, in group order).  No per-warp shared rows: occupancy is set
+// by registers, and the group spans any E up to 2 x 32 x WPT x 4 channels.
+constexpr int kBlrNsl = 2;  // float4 slots per thread
+__host__ __device__ __forceinline__ int bwd_lnr_wpt(int SL) { return (SL + 32 * kBlrNsl - 1) / (32 * kBlrNsl); }
+// groups per block: about 8 warps, at most 15 (named barrier ids 1..15)
+__host__ __device__ __forceinline__ int bwd_lnr_groups(int SL) {
+    const int w = bwd_lnr_wpt(SL);
+    const int ng = w >= 8 ? 1 : 8 / w;
+    return ng > 15 ? 15 : ng;
+}
+__host__ __device__ __forceinline__ size_t bwd_lnr_smem_bytes(int SL) {
+    const int ng = bwd_lnr_groups(SL), wpt = bwd_lnr_wpt(SL);
+    return (size_t)(3 + ng) * SL * sizeof(float4)                // sum D, gamma, beta; the groups' rows
+           + (size_t)ng * wpt * 4 * sizeof(float);               // the warps' partial sums
+}
+__device__ __forceinline__ void group_bar(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" : : "r"(id), "r"(threads) : "memory");
+}
+
+template <bool MASKED>
+__global__ void __launch_bounds__(256, 2)
+bwd_ln_gate_reg_kernel(Shape sh, const float* __restrict__ x, const float* __restrict__ z,
+                       const float* __restrict__ dy, const float* __restrict__ ys, const float* __restrict__ D,
+                       const float* __restrict__ gamma, const float* __restrict__ beta,
+                       const int32_t* __restrict__ row_off, const int32_t* __restrict__ row_tok,
+                       float* __restrict__ dx, float* __restrict__ dz, float* __restrict__ dys,
+                       float* __restrict__ part_ln) {
+    constexpr int U = kBlrNsl;
+    extern __shared__ float4 lrs[];
+    const int SL = sh.SL, WPT = bwd_lnr_wpt(SL), NG = bwd_lnr_groups(SL), G = 32 * WPT;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int grp = warp / WPT, wig = warp - grp * WPT, gt = wig * 32 + lane;
+    float4* dsum = lrs;
+    float4* g4 = dsum + SL;
+    float4* be4 = g4 + SL;
+    float4* rows = be4 + SL;                                    // [NG][SL]
+    float* red = reinterpret_cast<float*>(rows + (size_t)NG * SL) + (size_t)grp * WPT * 4;  // [WPT][4]
+    for (int slot = threadIdx.x; slot < SL; slot += blockDim.x) {
+        dsum[slot] = bwd_dsum4(D, sh.nd, SL, slot);
+        g4[slot] = __ldg(reinterpret_cast<const float4*>(gamma) + slot);
+        be4[slot] = __ldg(reinterpret_cast<const float4*>(beta) + slot);
+    }
+    __syncthreads();
+    const bool live = grp < NG;  // warps past the last whole group only help with the row sums
+    const int T = sh.T, K = sh.K, rows_n = sh.B * T;
+    const size_t st4 = dense_stride(sh) >> 2;
+    const float invE = 1.f / (float)sh.E, eps = sh.ln_eps;
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    const float4* z4 = reinterpret_cast<const float4*>(z);
+    const float4* gy4 = reinterpret_cast<const float4*>(dy);
+    float4* dx4 = reinterpret_cast<float4*>(dx);
+    float4* dz4 = reinterpret_cast<float4*>(dz);
+    bool own[U];
+    float4 acc_g[U], acc_b[U], acc_d[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        own[u] = live && gt + G * u < SL;
+        acc_g[u] = acc_b[u] = acc_d[u] = f4_zero();
+    }
+    // sum D, gamma, beta of the thread's slots, from shared memory
+    auto ds4 = [&](int u) { return own[u] ? dsum[gt + G * u] : f4_zero(); };
+    auto gm = [&](int u) { return own[u] ? g4[gt + G * u] : f4_zero(); };
+    auto bm = [&](int u) { return own[u] ? be4[gt + G * u] : f4_zero(); };
+    // the group's sum of (a, b) over its WPT warps, in warp order; `phase` picks one of two slots
+    auto group_sum2 = [&](float& a, float& b, int phase) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            a += __shfl_xor_sync(0xffffffffu, a, off);
+            b += __shfl_xor_sync(0xffffffffu, b, off);
+        }
+        if (WPT == 1) return;
+        if (lane == 0) {
+            red[wig * 4 + 2 * phase] = a;
+            red[wig * 4 + 2 * phase + 1] = b;
+        }
+        group_bar(1 + grp, G);
+        a = red[2 * phase];
+        b = red[2 * phase + 1];
+        for (int w = 1; w < WPT; ++w) {
+            a += red[w * 4 + 2 * phase];
+            b += red[w * 4 + 2 * phase + 1];
+        }
+    };
+    for (int bt = blockIdx.x; bt < rows_n; bt += gridDim.x) {
+        const int b = bt / T, t = bt - b * T;
+        int p0 = 0, ntok = sh.S;
+        if (MASKED) {
+            p0 = row_off[(size_t)b * (T + 1) + t];
+            ntok = row_off[(size_t)b * (T + 1) + t + 1] - p0;
+        }
+        const float4* ys4 = reinterpret_cast<const float4*>(ys + (size_t)bt * sh.E);
+        float4 yv[U], acc_y[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            yv[u] = own[u] ? ys4[gt + G * u] : f4_zero();
+            acc_y[u] = f4_zero();
+        }
+        const float y0 = __ldg(ys + (size_t)bt * sh.E);
+        for (int i = grp; live && i < ntok; i += NG) {
+            const size_t o = MASKED ? ((size_t)b * K + row_tok[(size_t)b * K + p0 + i]) * SL
+                                    : (dense_base(sh, b, t) >> 2) + (size_t)i * st4;
+            // every load of the token at once (one memory round trip per token)
+            float4 xv[U], zv[U], gv[U], sv[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                xv[u] = own[u] ? ld_stream(x4 + o + gt + G * u) : f4_zero();
+                zv[u] = own[u] ? ld_stream(z4 + o + gt + G * u) : f4_zero();
+                gv[u] = own[u] ? ld_stream(gy4 + o + gt + G * u) : f4_zero();
+            }
+            // pass 1: s and its moments about the token's first s value (the same in every thread)
+            const float Ks = fmaf(dsum[0].x, __ldg(x + o * 4), y0);
+            float m1 = 0.f, m2 = 0.f;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                sv[u] = f4_fma(ds4(u), xv[u], yv[u]);
+                if (own[u]) ln_accum(sv[u], Ks, m1, m2);
+            }
+            group_sum2(m1, m2, 0);
+            const float d = m1 * invE;
+            const float mean = Ks + d;
+            const float rstd = rsqrtf(fmaxf(m2 * invE - d * d, 0.f) + eps);
+            // pass 2: the two means of gs = dy SiLU(z) gamma
+            float a1 = 0.f, a2 = 0.f;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const float sa[4] = {sv[u].x, sv[u].y, sv[u].z, sv[u].w}, za[4] = {zv[u].x, zv[u].y, zv[u].z, zv[u].w};
+                const float ga[4] = {gv[u].x, gv[u].y, gv[u].z, gv[u].w};
+                const float4 g = gm(u);
+                const float gma[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float shv = (sa[c] - mean) * rstd;
+                    const float gs = ga[c] * za[c] * sigmoid_fast(za[c]) * gma[c];
+                    a1 += gs;
+                    a2 = fmaf(gs, shv, a2);
+                }
+            }
+            group_sum2(a1, a2, 1);
+            const float mgs = a1 * invE, mgss = a2 * invE;
+            // pass 3: the outputs, from registers
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (!own[u]) continue;
+                const int slot = gt + G * u;
+                const float sa[4] = {sv[u].x, sv[u].y, sv[u].z, sv[u].w}, za[4] = {zv[u].x, zv[u].y, zv[u].z, zv[u].w};
+                const float ga[4] = {gv[u].x, gv[u].y, gv[u].z, gv[u].w}, xa[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
+                const float4 g = gm(u), be = bm(u), dd = ds4(u);
+                const float gma[4] = {g.x, g.y, g.z, g.w}, bma[4] = {be.x, be.y, be.z, be.w};
+                const float dsa[4] = {dd.x, dd.y, dd.z, dd.w};
+                float dzo[4], dxo[4], dso[4], dno[4], sho[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float shv = (sa[c] - mean) * rstd;
+                    const float sg = sigmoid_fast(za[c]);
+                    const float dn = ga[c] * za[c] * sg;
+                    const float n = fmaf(gma[c], shv, bma[c]);
+                    dzo[c] = ga[c] * n * sg * fmaf(za[c], 1.f - sg, 1.f);
+                    const float ds = (fmaf(dn, gma[c], -mgs) - shv * mgss) * rstd;
+                    dxo[c] = ds * dsa[c];
+                    dso[c] = ds;
+                    dno[c] = dn;
+                    sho[c] = shv;
+                }
+                st_stream(dz4 + o + slot, make_float4(dzo[0], dzo[1], dzo[2], dzo[3]));
+                st_stream(dx4 + o + slot, make_float4(dxo[0], dxo[1], dxo[2], dxo[3]));
+                f4_add(acc_y[u], make_float4(dso[0], dso[1], dso[2], dso[3]));
+                f4_add(acc_g[u], make_float4(dno[0] * sho[0], dno[1] * sho[1], dno[2] * sho[2], dno[3] * sho[3]));
+                f4_add(acc_b[u], make_float4(dno[0], dno[1], dno[2], dno[3]));
+                f4_add(acc_d[u], make_float4(dso[0] * xa[0], dso[1] * xa[1], dso[2] * xa[2], dso[3] * xa[3]));
+            }
+        }
+        // dys of the row: the groups' sums, added in group order
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (own[u]) rows[(size_t)grp * SL + gt + G * u] = acc_y[u];
+        __syncthreads();
+        for (int slot = threadIdx.x; slot < SL; slot += blockDim.x) {
+            float4 acc = rows[slot];
+            for (int q = 1; q < NG; ++q) f4_add(acc, rows[(size_t)q * SL + slot]);
+            reinterpret_cast<float4*>(dys)[(size_t)bt * SL + slot] = acc;
+        }
+        __syncthreads();
+    }
+    // the block's batch sums, dgamma | dbeta | dD, each added over the groups in group order
+    float4* out = reinterpret_cast<float4*>(part_ln + (size_t)blockIdx.x * 3 * sh.E);
+#pragma unroll
+    for (int which = 0; which < 3; ++which) {
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (own[u]) rows[(size_t)grp * SL + gt + G * u] = which == 0 ? acc_g[u] : which == 1 ? acc_b[u] : acc_d[u];
+        __syncthreads();
+        for (int slot = threadIdx.x; slot < SL; slot += blockDim.x) {
+            float4 acc = rows[slot];
+            for (int q = 1; q < NG; ++q) f4_add(acc, rows[(size_t)q * SL + slot]);
+            out[(size_t)which * SL + slot] = acc;
+        }
+        __syncthreads();
+    }
+}
+
 // ------------------------------------------------------------------------------------------
 // Adjoint of the scans
 // ------------------------------------------------------------------------------------------

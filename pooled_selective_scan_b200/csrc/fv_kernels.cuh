@@ -661,8 +661,8 @@ ln_epilogue_kernel(Shape sh, const float* __restrict__ x, const float* __restric
 // The same epilogue for rows of up to 1536 channels (without the Conv1D), with each lane's share of
 // the token's s = ys[t] + (sum D) x held in registers (NSL float4 slots per lane) instead of
 // shared-memory rows: eight warps per CTA and no per-warp shared memory, so occupancy is set by
-// registers alone.  Per token: x and ys are loaded, s and its shifted moments formed, the warp
-// reduction gives the mean and 1/sqrt(var + eps); then z is loaded and y stored.
+// registers alone.  Per token: x, ys and z are loaded at once, s and its shifted moments formed,
+// the warp reduction gives the mean and 1/sqrt(var + eps), and y is stored.
 constexpr int kLnRegWarps = 8;
 __host__ __device__ __forceinline__ int ln_reg_nsl(int SL) {
     const int need = (SL + 31) / 32;
@@ -715,11 +715,14 @@ ln_epilogue_reg_kernel(Shape sh, const float* __restrict__ x, const float* __res
         }
         const float4* xl = reinterpret_cast<const float4*>(x) + o;
         const float4* yl4 = reinterpret_cast<const float4*>(ys + ((size_t)b * sh.T + t) * sh.E) + lane;
-        float4 sv[NSL];
+        const float4* zl = reinterpret_cast<const float4*>(z) + o;
+        float4 sv[NSL], zv[NSL];
 #pragma unroll
-        for (int u = 0; u < NSL; ++u)
+        for (int u = 0; u < NSL; ++u) {  // x, ys and z at once: one memory round trip per token
             sv[u] = u < nsl ? f4_fma(dl[32 * u], ld_stream(xl + 32 * u), __ldcg(yl4 + 32 * u))
                             : make_float4(0.f, 0.f, 0.f, 0.f);
+            zv[u] = u < nsl ? ld_stream(zl + 32 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         // shift: the token's first s value, from lane 0
         const float K = __shfl_sync(0xffffffffu, sv[0].x, 0);
         float m1 = 0.f, m2 = 0.f;
@@ -728,10 +731,9 @@ ln_epilogue_reg_kernel(Shape sh, const float* __restrict__ x, const float* __res
             if (u < nsl) ln_accum(sv[u], K, m1, m2);
         float mean, rstd;
         ln_stats(m1, m2, K, invE, sh.ln_eps, mean, rstd);
-        const float4* zl = reinterpret_cast<const float4*>(z) + o;
 #pragma unroll
         for (int u = 0; u < NSL; ++u)
-            if (u < nsl) st_stream(yl + 32 * u, ln_gate4(sv[u], ld_stream(zl + 32 * u), gl[32 * u], bl[32 * u], mean, rstd));
+            if (u < nsl) st_stream(yl + 32 * u, ln_gate4(sv[u], zv[u], gl[32 * u], bl[32 * u], mean, rstd));
     }
 }
 

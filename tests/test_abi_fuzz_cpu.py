@@ -231,7 +231,7 @@ def test_gradient_validation_and_plan(a, pick):
     if a.B == 0:
         assert n == 0
     else:
-        first = ("bwd_ln_gate_kernel" if a.flags & nat.FV_FLAG_LAYERNORM else
+        first = (("bwd_ln_gate_reg_kernel" if a.E <= 2048 else "bwd_ln_gate_kernel") if a.flags & nat.FV_FLAG_LAYERNORM else
                  "bwd_gate_masked_kernel" if a.K else "bwd_gate_dense_kernel")
         mid = ["bwd_scan_kernel"] if FL.delta else ["dt_proj_kernel", "bwd_scan_kernel"]
         assert names[0] == first and names[1:1 + len(mid)] == mid and len(names) == 6 + len(mid)

@@ -95,7 +95,9 @@ def test_launch_lists(lib):
     ln = args(flags=nat.FV_FLAG_LAYERNORM, ln_gamma=FAKE + 10 * SLOT, ln_beta=FAKE + 11 * SLOT, ln_eps=1e-5)
     names = [lib.fastvim_ssm_backward_launch_name(ctypes.byref(ln), i).decode() for i in range(8)]
     assert lib.fastvim_ssm_backward_launch_count(ctypes.byref(ln)) == 8
-    assert names[0] == "bwd_ln_gate_kernel" and names[1:] == dense[1:]
+    assert names[0] == "bwd_ln_gate_reg_kernel" and names[1:] == dense[1:]  # E = 384: tokens in registers
+    wide = args(E=2560, flags=nat.FV_FLAG_LAYERNORM, ln_gamma=FAKE + 10 * SLOT, ln_beta=FAKE + 11 * SLOT, ln_eps=1e-5)
+    assert lib.fastvim_ssm_backward_launch_name(ctypes.byref(wide), 0) == b"bwd_ln_gate_kernel"
     # dt_rank 48 on the staged path: the forward's step sizes are read, no dt_proj launch
     big = args(h=64, w=64, E=1536, R=48, K=1024, keep_idx=FAKE + 9 * SLOT)
     n = lib.fastvim_ssm_backward_launch_count(ctypes.byref(big))
