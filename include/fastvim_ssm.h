@@ -91,8 +91,8 @@ enum {
     FV_FLAG_LAYERNORM = 16u,  /* post-SSM LayerNorm before the gate (ln_gamma, ln_beta, ln_eps) */
     FV_FLAG_CONV_SILU = 32u   /* SiLU after the block's Conv1D (needs d_conv > 0)               */
 };
-/* Without a PATH flag a dense layer whose images hold >= 16 MiB of x runs the fused launch, every
- * other layer the staged kernels; both compute the same layer.  The fused launch gates image b
+/* Without a PATH flag a dense layer without FV_FLAG_LAYERNORM whose images hold >= 16 MiB of x
+ * runs the fused launch, every other layer the staged kernels; both compute the same layer.  The fused launch gates image b
  * L rounds after it pools it, L chosen from the layer's shape; the environment variable
  * FASTVIM_FUSED_LAG (an integer 3..64, read by every call that takes the fused launch) replaces
  * that choice.  It is a test hook: the tests run the schedule at its smallest safe lag (3) and at

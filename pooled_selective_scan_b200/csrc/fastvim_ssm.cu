@@ -184,12 +184,15 @@ bool fused_possible(const fv::Shape& sh) {
 
 // Which implementation runs: the fused single launch for dense layers with large images (>= 16 MiB
 // of x per image: there the overlap of projections and scans with streaming pays; measured on B200,
-// 2.19 vs 2.35 ms at 2048 px, while at 1024 px the staged kernels win, 1.41 vs 1.83 ms), the staged
-// kernels otherwise; flags can force either.
+// 2.19 vs 2.35 ms at 2048 px, while at 1024 px the staged kernels win, 1.41 vs 1.83 ms) without
+// the post-SSM LayerNorm, the staged kernels otherwise; flags can force either.
 Path choose_path(const fv::Shape& sh) {
     const bool ok = fused_possible(sh);
     if (sh.path_flags & FV_FLAG_PATH_STAGED) return Path::Staged;
     if (sh.path_flags & FV_FLAG_PATH_FUSED) return ok ? Path::Fused : Path::Invalid;
+    // with the post-SSM LayerNorm the staged epilogue (tokens in registers) is the faster one
+    // (2048 px: 2.20 ms staged vs 2.41 ms fused on B200)
+    if (sh.ln) return Path::Staged;
     const size_t img = (size_t)sh.h * sh.w * sh.E * sizeof(float);
     return (ok && img >= ((size_t)16 << 20)) ? Path::Fused : Path::Staged;
 }

@@ -232,8 +232,12 @@ def test_layernorm_launches(lib):
                      conv_b=FAKE + (13 << 32))
     n = lib.fastvim_ssm_launch_count(ctypes.byref(conv))
     assert lib.fastvim_ssm_launch_name(ctypes.byref(conv), n - 1).decode() == "ln_epilogue_kernel"
+    # large images: the staged kernels by default (their register epilogue is the faster one); the
+    # forced single launch does the LayerNorm in its gate tasks
     big = good_args(h=128, w=128, B=4, flags=LN, ln_gamma=g, ln_beta=b, ln_eps=1e-5)
-    assert lib.fastvim_ssm_launch_count(ctypes.byref(big)) == 1  # the fused launch does it in its gate tasks
+    assert lib.fastvim_ssm_launch_count(ctypes.byref(big)) == 4
+    big.flags = LN | nat.FV_FLAG_PATH_FUSED
+    assert lib.fastvim_ssm_launch_count(ctypes.byref(big)) == 1
 
 
 @pytest.mark.parametrize("masked,ln", [(False, False), (False, True), (True, False), (True, True)])

@@ -43,11 +43,13 @@ def test_layernorm_dense(E, pool_axis, dir_flags, path):
     assert_close(got["y"], ref_of(p, pool_axis, dir_flags))
 
 
-def test_layernorm_large_eps_and_fused_default():
-    # 2048 px FastVim-T images (fused by default), eps large enough to matter
+@pytest.mark.parametrize("path", ["auto", "fused"])
+def test_layernorm_large_eps_at_2048px(path):
+    # 2048 px FastVim-T images (the LayerNorm layer takes the staged kernels by default, and the
+    # single launch when forced), eps large enough to matter
     p = with_ln(rand_layer(320, B=2, h=128, w=128, E=384, N=16, R=12, dir_flags=3), 7, 384)
-    got = gpu_forward(p, 0, 3, intermediates=False, ln_eps=0.25)
-    assert got["launches"] == ["fused_layer_kernel"]
+    got = gpu_forward(p, 0, 3, intermediates=False, ln_eps=0.25, path=path)
+    assert got["launches"][-1] == ("fused_layer_kernel" if path == "fused" else "ln_epilogue_reg_kernel")
     assert_close(got["y"], ref_of(p, 0, 3, eps=0.25))
 
 
