@@ -229,7 +229,7 @@ FV_API fv_status fastvim_ssm_forward_host(const fv_ssm_args* host, const fv_ssm_
  * 16 MiB array in device memory, part of this library's device code, held until the process
  * exits.
  *   - Limit: fastvim_ssm_workspace_size(args) must be <= 16 MiB (e.g. the 224 px FastVim-T
- *     layer at batch 128 needs about 11 MiB); larger layers return FV_ERR_UNSUPPORTED with a
+ *     layer at batch 128 needs about 6 MiB); larger layers return FV_ERR_UNSUPPORTED with a
  *     message in fastvim_last_error() and queue nothing; split the batch or use
  *     fastvim_ssm_forward.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
