@@ -33,16 +33,16 @@ constexpr int kBsHalf = 8;       // steps per checkpoint (two per staged chunk)
 __host__ __device__ __forceinline__ int bs_nchunks(int T) { return (T + kBsChunk - 1) / kBsChunk; }
 // checkpoints per scan: one every 8 steps of the scan order
 __host__ __device__ __forceinline__ int bs_nckpt(int T) { return 2 * bs_nchunks(T); }
-// Row stride of the W_dt rows in shared memory: odd, so lanes reading 32 different rows at the
-// same column hit 32 different banks.
-__host__ __device__ __forceinline__ int bs_wstride(int R) { return R | 1; }
+// dt_rank rounded up to whole float4s (the dt_low rows and the dW_dt sums are read as float4).
+__host__ __device__ __forceinline__ int bs_r4(int R) { return (R + 3) & ~3; }
+constexpr int kBsWS = 64 + 4;  // row stride of W_dt transposed, [r][channel]: float4-aligned rows
 __host__ __device__ __forceinline__ size_t bs_smem_floats(int R) {
-    return (size_t)kBsCh * bs_wstride(R)      // W_dt rows of the CTA's channels
-           + (size_t)kBsChunk * R             // dt_low of the chunk's steps
+    return (size_t)R * kBsWS                  // W_dt of the CTA's channels, transposed
+           + (size_t)kBsChunk * bs_r4(R)      // dt_low of the chunk's steps (zero past R)
            + (size_t)kBsChunk * 32            // B | C of the chunk's steps
            + 6 * (size_t)kBsChunk * kBsCh     // xbar, dys, Delta, sig(v), dv, dxbar (scan share)
            + (size_t)(kBsThreads / 32) * kBsChunk * 32  // dB | dC sums of the chunk, one row per warp
-           + (size_t)kBsCh * (R + 1);         // dW_dt | db_dt sums of the CTA's channels
+           + (size_t)kBsCh * (bs_r4(R) + 4);  // dW_dt | db_dt sums of the CTA's channels
 }
 
 // sigmoid(v) = 1 / (1 + e^-v) on the SFU (v -> -inf gives 0, v -> +inf gives 1).
@@ -631,10 +631,10 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
     extern __shared__ float bsm[];
     const int b = blockIdx.x, k = blockIdx.y, e0 = blockIdx.z * kBsCh;
     const int T = sh.T, E = sh.E, N = sh.N, R = sh.R, J = sh.J;
-    const int WS = bs_wstride(R);
-    float* sw = bsm;                          // [64][WS]
-    float* sdtl = sw + kBsCh * WS;            // [16][R]
-    float* sbc = sdtl + kBsChunk * R;         // [16][32]
+    const int R4 = bs_r4(R), WA = R4 + 4;   // dt_low row stride; dW_dt | db_dt row stride
+    float* swT = bsm;                         // [R][kBsWS]: W_dt transposed
+    float* sdtl = swT + R * kBsWS;            // [16][R4]
+    float* sbc = sdtl + kBsChunk * R4;        // [16][32]
     float* sx = sbc + kBsChunk * 32;          // [16][64]
     float* sdy = sx + kBsChunk * kBsCh;       // [16][64]
     float* sdl = sdy + kBsChunk * kBsCh;      // [16][64]
@@ -642,7 +642,7 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
     float* sdv = ssg + kBsChunk * kBsCh;      // [16][64]
     float* sdx = sdv + kBsChunk * kBsCh;      // [16][64]
     float* sred = sdx + kBsChunk * kBsCh;     // [8 warps][16][32]
-    float* swacc = sred + (kBsThreads / 32) * kBsChunk * 32;  // [64][R + 1]
+    float* swacc = sred + (kBsThreads / 32) * kBsChunk * 32;  // [64][WA]: dW_dt row (R4) | db_dt
     const int tid = threadIdx.x;
     const int c = tid >> 2, q = tid & 3, lane = tid & 31;
     const int e = e0 + c;
@@ -657,9 +657,9 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
 
     for (int i = tid; i < kBsCh * R; i += kBsThreads) {
         const int row = i / R, r = i - row * R;
-        sw[row * WS + r] = (e0 + row < E) ? __ldg(W_dt + ((size_t)k * E + e0 + row) * R + r) : 0.f;
+        swT[r * kBsWS + row] = (e0 + row < E) ? __ldg(W_dt + ((size_t)k * E + e0 + row) * R + r) : 0.f;
     }
-    for (int i = tid; i < kBsCh * (R + 1); i += kBsThreads) swacc[i] = 0.f;
+    for (int i = tid; i < kBsCh * WA; i += kBsThreads) swacc[i] = 0.f;
 
     constexpr float kLog2e = 1.4426950408889634f;
     float A2[4], An[4], Ainv[4];
@@ -683,9 +683,9 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
     auto stage = [&](int it, bool pass2) {
         const int len = chunk_len(it);
         if (pass2)
-            for (int i = tid; i < kBsChunk * R; i += kBsThreads) {
-                const int s = i / R, r = i - s * R;
-                sdtl[i] = s < len ? ub[(size_t)t_of(it, s) * J + r] : 0.f;
+            for (int i = tid; i < kBsChunk * R4; i += kBsThreads) {
+                const int s = i / R4, r = i - s * R4;
+                sdtl[i] = (s < len && r < R) ? ub[(size_t)t_of(it, s) * J + r] : 0.f;
             }
         for (int i = tid; i < kBsChunk * 32; i += kBsThreads) {
             const int s = i >> 5, j = i & 31, n = j & 15;
@@ -838,29 +838,54 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
                 pdu[u_offset(sh, k, b, t_of(it, s)) + R + (j < 16 ? n : N + n)] = acc;
             }
         }
-        // dt_proj: d dt_low of the chunk's steps (this block's channels), dW_dt | db_dt partial sums
+        // dt_proj: d dt_low of the chunk's steps (this block's channels): one output per thread,
+        // W_dt's row r and the step's dv as float4 over the 64 channels
         for (int i = tid; i < len * R; i += kBsThreads) {
             const int s = i / R, r = i - s * R;
-            float acc = 0.f;
-            for (int cc = 0; cc < kBsCh; ++cc) acc = fmaf(sw[cc * WS + r], sdv[s * kBsCh + cc], acc);
-            pdu[u_offset(sh, k, b, t_of(it, s)) + r] = acc;
+            const float4* w4 = reinterpret_cast<const float4*>(swT + r * kBsWS);
+            const float4* d4 = reinterpret_cast<const float4*>(sdv + s * kBsCh);
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+            for (int c4 = 0; c4 < kBsCh / 4; ++c4) {
+                const float4 w = w4[c4], d = d4[c4];
+                a0 = fmaf(w.x, d.x, a0);
+                a1 = fmaf(w.y, d.y, a1);
+                a2 = fmaf(w.z, d.z, a2);
+                a3 = fmaf(w.w, d.w, a3);
+            }
+            pdu[u_offset(sh, k, b, t_of(it, s)) + r] = (a0 + a1) + (a2 + a3);
         }
-        for (int i = tid; i < kBsCh * (R + 1); i += kBsThreads) {
-            const int cc = i / (R + 1), r = i - cc * (R + 1);
-            float acc = swacc[i];
-            for (int s = 0; s < len; ++s) acc = fmaf(sdv[s * kBsCh + cc], r < R ? sdtl[s * R + r] : 1.f, acc);
-            swacc[i] = acc;
+        // dW_dt | db_dt partial sums over the chunk's steps: thread = (channel, 4 entries of the
+        // row; the last group is the bias), dt_low read as float4
+        const int ng = R4 / 4 + 1;
+        for (int i = tid; i < kBsCh * ng; i += kBsThreads) {
+            const int cc = i / ng, g = i - cc * ng;
+            float4* a = reinterpret_cast<float4*>(swacc + cc * WA + 4 * g);
+            float4 acc = *a;
+            if (g < R4 / 4) {
+                for (int s = 0; s < len; ++s) {
+                    const float dv = sdv[s * kBsCh + cc];
+                    const float4 d = *reinterpret_cast<const float4*>(sdtl + s * R4 + 4 * g);
+                    acc.x = fmaf(dv, d.x, acc.x);
+                    acc.y = fmaf(dv, d.y, acc.y);
+                    acc.z = fmaf(dv, d.z, acc.z);
+                    acc.w = fmaf(dv, d.w, acc.w);
+                }
+            } else {
+                for (int s = 0; s < len; ++s) acc.x += sdv[s * kBsCh + cc];
+            }
+            *a = acc;
         }
         __syncthreads();  // the buffers are refilled by the next stage()
     }
     // this image's dW_dt | db_dt and dA_log terms (part_wdt [B][nd][E][R], part_bdt [B][nd][E],
     // part_dA [B][nd][E][N]; bwd_reduce_kernel adds the images in order)
     const size_t img = (size_t)b * sh.nd + k;
-    for (int i = tid; i < kBsCh * (R + 1); i += kBsThreads) {  // each entry was summed by this thread
+    for (int i = tid; i < kBsCh * (R + 1); i += kBsThreads) {
         const int cc = i / (R + 1), r = i - cc * (R + 1);
         if (e0 + cc < E) {
-            if (r < R) part_wdt[(img * E + e0 + cc) * R + r] = swacc[i];
-            else part_bdt[img * E + e0 + cc] = swacc[i];
+            if (r < R) part_wdt[(img * E + e0 + cc) * R + r] = swacc[cc * WA + r];
+            else part_bdt[img * E + e0 + cc] = swacc[cc * WA + R4];
         }
     }
 #pragma unroll
