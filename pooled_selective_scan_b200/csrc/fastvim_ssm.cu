@@ -472,10 +472,11 @@ fv_status staged_back(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws_lay
     if (sh.ln && ln_uses_reg_kernel(sh)) {
         const size_t smem = (size_t)3 * sh.SL * sizeof(float4);
         const int nsl = fv::ln_reg_nsl(sh.SL);
-        auto kern = nsl == 1 ? fv::ln_epilogue_reg_kernel<1> : nsl == 2 ? fv::ln_epilogue_reg_kernel<2>
-                  : nsl == 3 ? fv::ln_epilogue_reg_kernel<3> : nsl == 4 ? fv::ln_epilogue_reg_kernel<4>
-                  : nsl == 6 ? fv::ln_epilogue_reg_kernel<6> : nsl == 8 ? fv::ln_epilogue_reg_kernel<8>
-                  : fv::ln_epilogue_reg_kernel<12>;
+        // the widest rows (12 slots per lane) take two warps per token at 6 slots each
+        auto kern = nsl == 1 ? fv::ln_epilogue_reg_kernel<1, 1> : nsl == 2 ? fv::ln_epilogue_reg_kernel<2, 1>
+                  : nsl == 3 ? fv::ln_epilogue_reg_kernel<3, 1> : nsl == 4 ? fv::ln_epilogue_reg_kernel<4, 1>
+                  : nsl == 6 ? fv::ln_epilogue_reg_kernel<6, 1> : nsl == 8 ? fv::ln_epilogue_reg_kernel<8, 1>
+                  : fv::ln_epilogue_reg_kernel<6, 2>;
         cudaError_t e = ensure_smem(kern, smem);
         if (e != cudaSuccess) { note_cuda(e, "LayerNorm epilogue smem attribute"); return FV_ERR_CUDA; }
         int per_sm = 0;

@@ -669,12 +669,16 @@ __host__ __device__ __forceinline__ int ln_reg_nsl(int SL) {
     return need <= 4 ? need : (need <= 6 ? 6 : (need <= 8 ? 8 : (need <= 12 ? 12 : 0)));
 }
 
-template <int NSL>
+// WPT warps per token (WPT = 2 for the widest rows: half the registers per thread, so two CTAs
+// per SM instead of one); the group's moments meet behind a named barrier, in warp order.
+template <int NSL, int WPT>
 __global__ void __launch_bounds__(kLnRegWarps * 32)
 ln_epilogue_reg_kernel(Shape sh, const float* __restrict__ x, const float* __restrict__ z,
                        const float* __restrict__ ys, const float* __restrict__ D, const float* __restrict__ gamma,
                        const float* __restrict__ beta, const int32_t* __restrict__ row_of, float* __restrict__ y) {
+    constexpr int G = 32 * WPT, NG = kLnRegWarps / WPT;  // threads per token, tokens per block
     extern __shared__ float4 lrs[];
+    __shared__ float red[kLnRegWarps][2];
     const int SL = sh.SL;
     float4* dsum = lrs;
     float4* g4 = dsum + SL;
@@ -686,16 +690,16 @@ ln_epilogue_reg_kernel(Shape sh, const float* __restrict__ x, const float* __res
     }
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int grp = warp / WPT, wig = warp - grp * WPT, gt = wig * 32 + lane;
     const long long per_img = sh.K > 0 ? (long long)sh.K : (long long)sh.h * sh.w;
     const long long ntok = (long long)sh.B * per_img;
     const float invE = 1.f / (float)sh.E;
-    // this lane's slots are lane + 32 u: one base pointer per tensor, constant offsets per slot
-    const int nsl = (SL - lane + 31) >> 5;  // slots of this lane
-    const float4* dl = dsum + lane;
-    const float4* gl = g4 + lane;
-    const float4* bl = b4 + lane;
-    for (long long tok = (long long)blockIdx.x * kLnRegWarps + warp; tok < ntok;
-         tok += (long long)gridDim.x * kLnRegWarps) {
+    // this thread's slots are gt + G u: one base pointer per tensor, constant offsets per slot
+    const int nsl = (SL - gt + G - 1) / G;  // slots of this thread
+    const float4* dl = dsum + gt;
+    const float4* gl = g4 + gt;
+    const float4* bl = b4 + gt;
+    for (long long tok = (long long)blockIdx.x * NG + grp; tok < ntok; tok += (long long)gridDim.x * NG) {
         const int b = (int)(tok / per_img);
         const long long r = tok - (long long)b * per_img;
         int t;
@@ -705,35 +709,62 @@ ln_epilogue_reg_kernel(Shape sh, const float* __restrict__ x, const float* __res
             const int i = (int)(r / sh.w), j = (int)(r - (long long)i * sh.w);
             t = sh.pool_axis == 0 ? i : j;
         }
-        const size_t o = (size_t)tok * SL + lane;
+        const size_t o = (size_t)tok * SL + gt;
         float4* yl = reinterpret_cast<float4*>(y) + o;
         if (t < 0) {
 #pragma unroll
             for (int u = 0; u < NSL; ++u)
-                if (u < nsl) st_stream(yl + 32 * u, make_float4(0.f, 0.f, 0.f, 0.f));
+                if (u < nsl) st_stream(yl + G * u, make_float4(0.f, 0.f, 0.f, 0.f));
             continue;
         }
         const float4* xl = reinterpret_cast<const float4*>(x) + o;
-        const float4* yl4 = reinterpret_cast<const float4*>(ys + ((size_t)b * sh.T + t) * sh.E) + lane;
+        const float* ysr = ys + ((size_t)b * sh.T + t) * sh.E;
+        const float4* yl4 = reinterpret_cast<const float4*>(ysr) + gt;
         const float4* zl = reinterpret_cast<const float4*>(z) + o;
         float4 sv[NSL], zv[NSL];
 #pragma unroll
         for (int u = 0; u < NSL; ++u) {  // x, ys and z at once: one memory round trip per token
-            sv[u] = u < nsl ? f4_fma(dl[32 * u], ld_stream(xl + 32 * u), __ldcg(yl4 + 32 * u))
+            sv[u] = u < nsl ? f4_fma(dl[G * u], ld_stream(xl + G * u), __ldcg(yl4 + G * u))
                             : make_float4(0.f, 0.f, 0.f, 0.f);
-            zv[u] = u < nsl ? ld_stream(zl + 32 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+            zv[u] = u < nsl ? ld_stream(zl + G * u) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        // shift: the token's first s value, from lane 0
-        const float K = __shfl_sync(0xffffffffu, sv[0].x, 0);
+        // shift: the token's first s value (lane 0 of the group's first warp holds it)
+        const float K = WPT == 1 ? __shfl_sync(0xffffffffu, sv[0].x, 0)
+                                 : fmaf(dsum[0].x, __ldcg(x + (size_t)tok * sh.E), __ldcg(ysr));
         float m1 = 0.f, m2 = 0.f;
 #pragma unroll
         for (int u = 0; u < NSL; ++u)
             if (u < nsl) ln_accum(sv[u], K, m1, m2);
         float mean, rstd;
-        ln_stats(m1, m2, K, invE, sh.ln_eps, mean, rstd);
+        if (WPT == 1) {
+            ln_stats(m1, m2, K, invE, sh.ln_eps, mean, rstd);
+        } else {
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                m1 += __shfl_xor_sync(0xffffffffu, m1, off);
+                m2 += __shfl_xor_sync(0xffffffffu, m2, off);
+            }
+            if (lane == 0) {
+                red[warp][0] = m1;
+                red[warp][1] = m2;
+            }
+            asm volatile("bar.sync %0, %1;" : : "r"(1 + grp), "r"(G) : "memory");
+            m1 = red[grp * WPT][0];
+            m2 = red[grp * WPT][1];
+#pragma unroll
+            for (int w = 1; w < WPT; ++w) {
+                m1 += red[grp * WPT + w][0];
+                m2 += red[grp * WPT + w][1];
+            }
+            // the slots are read again only after the group's next barrier
+            asm volatile("bar.sync %0, %1;" : : "r"(1 + grp), "r"(G) : "memory");
+            const float d = m1 * invE;
+            mean = K + d;
+            rstd = rsqrtf(fmaxf(m2 * invE - d * d, 0.f) + sh.ln_eps);
+        }
 #pragma unroll
         for (int u = 0; u < NSL; ++u)
-            if (u < nsl) st_stream(yl + 32 * u, ln_gate4(sv[u], zv[u], gl[32 * u], bl[32 * u], mean, rstd));
+            if (u < nsl) st_stream(yl + G * u, ln_gate4(sv[u], zv[u], gl[G * u], bl[G * u], mean, rstd));
     }
 }
 
