@@ -1101,7 +1101,9 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
         const size_t smem = fv::bwd_lnr_smem_bytes(sh.SL);
         const int32_t* row_off = sh.K > 0 ? (const int32_t*)(fw + FL.row_off) : nullptr;
         const int32_t* row_tok = sh.K > 0 ? (const int32_t*)(fw + FL.row_tok) : nullptr;
-        auto kern = sh.K > 0 ? fv::bwd_ln_gate_reg_kernel<true> : fv::bwd_ln_gate_reg_kernel<false>;
+        const bool one = fv::bwd_lnr_nsl(sh.SL) == 1;
+        auto kern = sh.K > 0 ? (one ? fv::bwd_ln_gate_reg_kernel<1, true> : fv::bwd_ln_gate_reg_kernel<2, true>)
+                             : (one ? fv::bwd_ln_gate_reg_kernel<1, false> : fv::bwd_ln_gate_reg_kernel<2, false>);
         if ((e = ensure_smem(kern, smem)) != cudaSuccess) {
             note_cuda(e, "LayerNorm gradient smem attribute");
             return FV_ERR_CUDA;

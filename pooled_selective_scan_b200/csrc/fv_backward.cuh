@@ -388,7 +388,7 @@ bwd_ln_gate_kernel(Shape sh, const float* __restrict__ x, const float* __restric
 }
 
 // The same gradient with each token's values in registers.  A group of WPT warps takes one token
-// (thread gt of the group owns float4 slots gt + 32 WPT u, u < 2: E <= 256 WPT); a
+// (thread gt of the group owns float4 slots gt + 32 WPT u, u < U: E <= 128 U WPT); a
 // block of NG groups is persistent over pooled rows, its groups taking the row's tokens in turn.
 // Per token: x, z and dy are loaded at once; pass 1 forms s and its shifted moments, pass 2 the
 // two means of gs, pass 3 writes dz, dx from the registers.  The group's sums (moments, means) go
@@ -396,9 +396,15 @@ bwd_ln_gate_kernel(Shape sh, const float* __restrict__ x, const float* __restric
 // dys of the current row and the batch sums of dgamma, dbeta, dD stay in each thread's registers;
 // the groups' dys meet in shared memory at the end of each row, the batch sums at the end of the
 // kernel (row blockIdx.x of part_ln, in group order).  No per-warp shared rows: occupancy is set
-// by registers, and the group spans any E up to 2 x 32 x WPT x 4 channels.
-constexpr int kBlrNsl = 2;  // float4 slots per thread
-__host__ __device__ __forceinline__ int bwd_lnr_wpt(int SL) { return (SL + 32 * kBlrNsl - 1) / (32 * kBlrNsl); }
+// by registers, and the group spans any E up to U x 32 x WPT x 4 channels.  U = 1 (64 registers,
+// four blocks per SM) for 513-1,024 channels, U = 2 (128 registers, two blocks) otherwise:
+// measured on B200, E = 768 streams at 0.60 of the copy rate with U = 1 against 0.53 with U = 2,
+// E = 384 at 0.68 with U = 2 against 0.65 with U = 1.
+__host__ __device__ __forceinline__ int bwd_lnr_nsl(int SL) { return (SL > 128 && SL <= 256) ? 1 : 2; }
+__host__ __device__ __forceinline__ int bwd_lnr_wpt(int SL) {
+    const int u = bwd_lnr_nsl(SL);
+    return (SL + 32 * u - 1) / (32 * u);
+}
 // groups per block: about 8 warps, at most 15 (named barrier ids 1..15)
 __host__ __device__ __forceinline__ int bwd_lnr_groups(int SL) {
     const int w = bwd_lnr_wpt(SL);
@@ -414,15 +420,14 @@ __device__ __forceinline__ void group_bar(int id, int threads) {
     asm volatile("bar.sync %0, %1;" : : "r"(id), "r"(threads) : "memory");
 }
 
-template <bool MASKED>
-__global__ void __launch_bounds__(256, 2)
+template <int U, bool MASKED>
+__global__ void __launch_bounds__(256, U == 1 ? 4 : 2)
 bwd_ln_gate_reg_kernel(Shape sh, const float* __restrict__ x, const float* __restrict__ z,
                        const float* __restrict__ dy, const float* __restrict__ ys, const float* __restrict__ D,
                        const float* __restrict__ gamma, const float* __restrict__ beta,
                        const int32_t* __restrict__ row_off, const int32_t* __restrict__ row_tok,
                        float* __restrict__ dx, float* __restrict__ dz, float* __restrict__ dys,
                        float* __restrict__ part_ln) {
-    constexpr int U = kBlrNsl;
     extern __shared__ float4 lrs[];
     const int SL = sh.SL, WPT = bwd_lnr_wpt(SL), NG = bwd_lnr_groups(SL), G = 32 * WPT;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
