@@ -1039,7 +1039,7 @@ constexpr int kMaxRedSegs = 8;
 struct RedSegs {
     RedSeg seg[kMaxRedSegs];
 };
-// Grid (x, number of segments): blockIdx.y picks the segment.  Few partials (P <= 32): one
+// Grid (x, number of segments): blockIdx.y picks the segment.  Up to 128 partials: one
 // thread per output adds them in order.  Many: a block takes 32 consecutive outputs at a time (one
 // per lane: coalesced loads) and splits the P partials over its 8 warps (warp w adds partials
 // w, w + 8, ... in order); the 8 warp sums are then added in warp order.  Either grouping depends
@@ -1049,7 +1049,7 @@ __global__ void __launch_bounds__(kRedWarps * 32)
 bwd_reduce_kernel(RedSegs segs) {
     __shared__ float wsum[kRedWarps][32];
     const RedSeg g = segs.seg[blockIdx.y];
-    if (g.P <= 32) {
+    if (g.P <= 128) {
         for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < g.L;
              i += (long long)gridDim.x * blockDim.x) {
             float acc = 0.f;
