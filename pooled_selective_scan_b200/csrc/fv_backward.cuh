@@ -36,11 +36,14 @@ __host__ __device__ __forceinline__ int bs_nckpt(int T) { return 2 * bs_nchunks(
 // dt_rank rounded up to whole float4s (the dt_low rows and the dW_dt sums are read as float4).
 __host__ __device__ __forceinline__ int bs_r4(int R) { return (R + 3) & ~3; }
 constexpr int kBsWS = 64 + 4;  // row stride of W_dt transposed, [r][channel]: float4-aligned rows
+// one staged chunk: dt_low [16][R4] (zero past R), B | C [16][32], then xbar, dys, Delta [16][64]
+__host__ __device__ __forceinline__ int bs_stage_floats(int R) {
+    return kBsChunk * bs_r4(R) + kBsChunk * 32 + 3 * kBsChunk * kBsCh;
+}
 __host__ __device__ __forceinline__ size_t bs_smem_floats(int R) {
     return (size_t)R * kBsWS                  // W_dt of the CTA's channels, transposed
-           + (size_t)kBsChunk * bs_r4(R)      // dt_low of the chunk's steps (zero past R)
-           + (size_t)kBsChunk * 32            // B | C of the chunk's steps
-           + 6 * (size_t)kBsChunk * kBsCh     // xbar, dys, Delta, sig(v), dv, dxbar (scan share)
+           + 2 * (size_t)bs_stage_floats(R)   // two staged chunks (copies of the next one in flight)
+           + 3 * (size_t)kBsChunk * kBsCh     // sig(v), dv, dxbar (scan share) of the chunk
            + (size_t)(kBsThreads / 32) * kBsChunk * 32  // dB | dC sums of the chunk, one row per warp
            + (size_t)kBsCh * (bs_r4(R) + 4);  // dW_dt | db_dt sums of the CTA's channels
 }
@@ -638,12 +641,8 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
     const int T = sh.T, E = sh.E, N = sh.N, R = sh.R, J = sh.J;
     const int R4 = bs_r4(R), WA = R4 + 4;   // dt_low row stride; dW_dt | db_dt row stride
     float* swT = bsm;                         // [R][kBsWS]: W_dt transposed
-    float* sdtl = swT + R * kBsWS;            // [16][R4]
-    float* sbc = sdtl + kBsChunk * R4;        // [16][32]
-    float* sx = sbc + kBsChunk * 32;          // [16][64]
-    float* sdy = sx + kBsChunk * kBsCh;       // [16][64]
-    float* sdl = sdy + kBsChunk * kBsCh;      // [16][64]
-    float* ssg = sdl + kBsChunk * kBsCh;      // [16][64]
+    float* sstage = swT + R * kBsWS;          // [2] staged chunks, bs_stage_floats(R) each
+    float* ssg = sstage + 2 * bs_stage_floats(R);  // [16][64]
     float* sdv = ssg + kBsChunk * kBsCh;      // [16][64]
     float* sdx = sdv + kBsChunk * kBsCh;      // [16][64]
     float* sred = sdx + kBsChunk * kBsCh;     // [8 warps][16][32]
@@ -682,34 +681,54 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
     auto chunk_len = [&](int it) { return min(kBsChunk, T - chunk_t0(it)); };
     auto t_of = [&](int it, int i) { return fwd ? chunk_t0(it) + i : chunk_t0(it) + chunk_len(it) - 1 - i; };
 
-    // stage a chunk's per-step inputs: Delta (written by the forward's or this call's dt_proj
-    // kernel), and in pass 2 dt_low, dys and softplus'(v) = sigmoid(v) = 1 - e^-Delta (as -expm1,
-    // exact for small Delta)
-    auto stage = [&](int it, bool pass2) {
-        const int len = chunk_len(it);
-        if (pass2)
+    // The chunks in the order they are used: pass 1 takes chunks 0 .. n-1 (scan order), pass 2
+    // n-1 .. 0; stage number si <-> chunk si (pass 1) or 2n-1-si (pass 2).  stage(si) queues the
+    // copies of the chunk's per-step inputs into buffer si & 1 (slots past the chunk and channels
+    // past E read as zero): B | C, xbar and Delta (written by the forward's or this call's dt_proj
+    // kernel), and in pass 2 dt_low and dys.  The next stage's copies run during a stage's steps.
+    const int nstages = 2 * nchunks;
+    auto chunk_of = [&](int si) { return si < nchunks ? si : nstages - 1 - si; };
+    auto stage = [&](int si) {
+        const int it = chunk_of(si), len = chunk_len(it);
+        float* sb = sstage + (si & 1) * bs_stage_floats(R);
+        float* dtl = sb;
+        float* bc = dtl + kBsChunk * R4;
+        float* rows = bc + kBsChunk * 32;  // xbar | dys | Delta
+        if (si >= nchunks)
             for (int i = tid; i < kBsChunk * R4; i += kBsThreads) {
                 const int s = i / R4, r = i - s * R4;
-                sdtl[i] = (s < len && r < R) ? ub[(size_t)t_of(it, s) * J + r] : 0.f;
+                const bool ok = s < len && r < R;
+                cp_async4z(dtl + i, ok ? ub + (size_t)t_of(it, s) * J + r : ub, ok);
             }
         for (int i = tid; i < kBsChunk * 32; i += kBsThreads) {
             const int s = i >> 5, j = i & 31, n = j & 15;
-            sbc[i] = (s < len && n < N) ? ub[(size_t)t_of(it, s) * J + R + (j < 16 ? n : N + n)] : 0.f;
+            const bool ok = s < len && n < N;
+            cp_async4z(bc + i, ok ? ub + (size_t)t_of(it, s) * J + R + (j < 16 ? n : N + n) : ub, ok);
         }
-        for (int i = tid; i < kBsChunk * kBsCh; i += kBsThreads) {
-            const int s = i / kBsCh, cc = i - s * kBsCh;
-            const bool ok = s < len && e0 + cc < E;
+        for (int i = tid; i < 3 * kBsChunk * (kBsCh / 4); i += kBsThreads) {
+            const int which = i / (kBsChunk * (kBsCh / 4)), v = i - which * (kBsChunk * (kBsCh / 4));
+            const int s = v / (kBsCh / 4), c4 = 4 * (v - s * (kBsCh / 4));
+            if (which == 1 && si < nchunks) continue;  // dys: pass 2 only
+            const bool ok = s < len && e0 + c4 < E;
             const int t = ok ? t_of(it, s) : 0;
-            const size_t o = ((size_t)b * T + t) * E + e0 + cc;
-            sx[i] = ok ? xbar[o] : 0.f;
-            const float dl = ok ? delta[delta_offset(sh, k, b, t) + e0 + cc] : 0.f;
-            sdl[i] = dl;
-            if (pass2) {
-                sdy[i] = ok ? dys[o] : 0.f;
-                ssg[i] = -expm1f(-dl);
-            }
+            const float* src = which == 0 ? xbar + ((size_t)b * T + t) * E
+                               : which == 1 ? dys + ((size_t)b * T + t) * E
+                                            : delta + delta_offset(sh, k, b, t);
+            cp_async16(rows + (which * kBsChunk + s) * kBsCh + c4, ok ? (const void*)(src + e0 + c4) : (const void*)ub,
+                       ok ? 16u : 0u);
+        }
+        cp_async_commit();
+    };
+    // wait for stage si's copies (the next stage's stay in flight) and return its buffer
+    auto arrive = [&](int si) {
+        if (si + 1 < nstages) {
+            stage(si + 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
         }
         __syncthreads();
+        return sstage + (si & 1) * bs_stage_floats(R);
     };
 
     // the input term of one step and state
@@ -717,10 +736,14 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
         return ZOH_EXACT ? expm1f(dt * An[j]) * Ainv[j] * Bn * xv : dt * Bn * xv;
     };
 
+    stage(0);
     // ---- pass 1: states entering each chunk ----
     float h[4] = {0.f, 0.f, 0.f, 0.f};
     for (int it = 0; it < nchunks; ++it) {
-        stage(it, false);
+        const float* sb = arrive(it);
+        const float* sbc = sb + kBsChunk * R4;
+        const float* sx = sbc + kBsChunk * 32;
+        const float* sdl = sx + 2 * kBsChunk * kBsCh;
         const int len = chunk_len(it);
         for (int i = 0; i < len; ++i) {
             if (live && (i == 0 || i == kBsHalf))
@@ -732,7 +755,7 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
                 h[j] = fmaf(ex2_approx(dt * A2[j]), h[j], qterm(dt, Bn, xv, j));
             }
         }
-        __syncthreads();  // the buffers are refilled by the next stage()
+        __syncthreads();  // the buffer is refilled by the stage after next
     }
 
     // ---- pass 2: the adjoint, chunks in reverse scan order ----
@@ -741,8 +764,15 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
     const int v_idx = (b2 ? 1 : 0) + (b3 ? 2 : 0) + (b4 ? 4 : 0);  // value this lane ends up holding
     const int red_n = 4 * q + (v_idx & 3), red_w = v_idx >> 2;       // state, and 0 = dB / 1 = dC
     for (int it = nchunks - 1; it >= 0; --it) {
-        stage(it, true);
+        const float* sdtl = arrive(nstages - 1 - it);
+        const float* sbc = sdtl + kBsChunk * R4;
+        const float* sx = sbc + kBsChunk * 32;
+        const float* sdy = sx + kBsChunk * kBsCh;
+        const float* sdl = sdy + kBsChunk * kBsCh;
         const int len = chunk_len(it);
+        // softplus'(v) = sigmoid(v) = 1 - e^-Delta (as -expm1, exact for small Delta) of the steps
+        // whose dv this thread writes (steps i = q mod 4 of its channel): no barrier needed
+        for (int i = q; i < len; i += 4) ssg[i * kBsCh + c] = -expm1f(-sdl[i * kBsCh + c]);
         for (int half = (len - 1) / kBsHalf; half >= 0; --half) {
             const int i0 = half * kBsHalf, hl = min(kBsHalf, len - i0);
             float hin[4] = {0.f, 0.f, 0.f, 0.f};
@@ -805,7 +835,7 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
                     ddt += __shfl_xor_sync(0xffffffffu, ddt, 2);
                     dxb += __shfl_xor_sync(0xffffffffu, dxb, 1);
                     dxb += __shfl_xor_sync(0xffffffffu, dxb, 2);
-                    if (q == 0) {
+                    if (q == (i & 3)) {  // every lane of the channel holds the sums
                         sdv[i * kBsCh + c] = ddt * ssg[i * kBsCh + c];
                         sdx[i * kBsCh + c] = dxb;
                     }
@@ -881,7 +911,7 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
             }
             *a = acc;
         }
-        __syncthreads();  // the buffers are refilled by the next stage()
+        __syncthreads();  // the buffers are refilled by the next stage(s)
     }
     // this image's dW_dt | db_dt and dA_log terms (part_wdt [B][nd][E][R], part_bdt [B][nd][E],
     // part_dA [B][nd][E][N]; bwd_reduce_kernel adds the images in order)
