@@ -84,12 +84,8 @@ def kernel_work(name: str, cfg, pool_axis: int):
         return "hbm", 4 * (-(-cfg.E // 64) + 1) * cfg.nd * cfg.B * T * (cfg.R + 2 * cfg.N)
     if name == "bwd_reduce_kernel:params":            # per-image partials of dA_log, dW_dt, db_dt read
         return "hbm", 4 * cfg.B * cfg.nd * cfg.E * (cfg.N + cfg.R + 1)
-    if name.startswith("bwd_gemm_kernel"):
-        J = cfg.R + 2 * cfg.N
-        M = cfg.B * T
-        flops = {"bwd_gemm_kernel:W_x": 2 * M * cfg.E * J * cfg.nd,
-                 "bwd_gemm_kernel:xbar": 2 * M * cfg.E * J * cfg.nd}
-        return "fma", flops.get(name, 0)
+    if name in ("bwd_dwx_kernel", "bwd_dxbar_kernel"):   # dW_x = du^T xbar, dxbar = du W_x
+        return "fma", 2 * cfg.B * T * cfg.E * (cfg.R + 2 * cfg.N) * cfg.nd
     return None, 0
 
 

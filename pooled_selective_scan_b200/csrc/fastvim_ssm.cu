@@ -937,10 +937,10 @@ bool bwd_ln_uses_reg(const fv::Shape& sh) { return fv::bwd_lnr_wpt(sh.SL) <= 8; 
 int bwd_launch_count_of(const fv::Shape& sh) { return sh.B == 0 ? 0 : (fwd_has_delta(sh) ? 7 : 8); }
 const char* bwd_launch_name_of(const fv::Shape& sh, int i) {
     static const char* dense[] = {"bwd_gate_dense_kernel", "dt_proj_kernel", "bwd_scan_kernel", "bwd_reduce_kernel:du",
-                                  "bwd_gemm_kernel:W_x", "bwd_gemm_kernel:xbar", "bwd_pool_dense_kernel",
+                                  "bwd_dwx_kernel", "bwd_dxbar_kernel", "bwd_pool_dense_kernel",
                                   "bwd_reduce_kernel:params"};
     static const char* masked[] = {"bwd_gate_masked_kernel", "dt_proj_kernel", "bwd_scan_kernel", "bwd_reduce_kernel:du",
-                                   "bwd_gemm_kernel:W_x", "bwd_gemm_kernel:xbar", "bwd_pool_masked_kernel",
+                                   "bwd_dwx_kernel", "bwd_dxbar_kernel", "bwd_pool_masked_kernel",
                                    "bwd_reduce_kernel:params"};
     const int n = bwd_launch_count_of(sh);
     if (i < 0 || i >= n) return "";
@@ -987,22 +987,34 @@ int device_sm_count() {
     return sms;
 }
 
-// K per split (a multiple of the GEMM's k-step) for about `splits` splits of Kd; the splits that
-// result are ceil(Kd / chunk).
-int bwd_kchunk(int Kd, int splits) {
-    const int kchunk = (Kd + splits - 1) / splits;
-    return (kchunk + fv::kBgK - 1) / fv::kBgK * fv::kBgK;
+// Tokens per split of dW_x (a multiple of the kernel's 16-token k-step) for about `splits` splits of
+// M; the splits that result are ceil(M / chunk).
+int bwd_kchunk(int M, int splits) {
+    const int kchunk = (M + splits - 1) / splits;
+    return (kchunk + fv::kGwK - 1) / fv::kGwK * fv::kGwK;
 }
 
-template <class AOp, class BOp, class COp>
-fv_status launch_bwd_gemm(int M, int Nc, int Kd, int nz, int splits, AOp A, BOp Bm, COp C, cudaStream_t st,
-                          const char* where) {
-    if (M <= 0 || Nc <= 0 || Kd <= 0) return FV_OK;
-    const int kchunk = bwd_kchunk(Kd, splits);
-    splits = (Kd + kchunk - 1) / kchunk;
-    const dim3 grid((M + fv::kBgTile - 1) / fv::kBgTile, (Nc + fv::kBgTile - 1) / fv::kBgTile, nz * splits);
-    fv::bwd_gemm_kernel<<<grid, fv::kThreads, 0, st>>>(M, Nc, Kd, splits, kchunk, A, Bm, C);
-    FV_LAUNCH_CHECK(where);
+// dW_x partials: one instantiation per row count ceil(J / 16) (J <= kMaxJ = 96)
+fv_status launch_bwd_dwx(const fv::Shape& sh, const float* du, const float* xbar, float* part, int splits,
+                         int kchunk, cudaStream_t st) {
+    const dim3 grid((sh.E + fv::kGwE - 1) / fv::kGwE, sh.nd * splits);
+    const bool vec = (sh.J & 3) == 0;
+#define FV_DWX(RT)                                                                                      \
+    case RT:                                                                                            \
+        if (vec) fv::bwd_dwx_kernel<RT, true><<<grid, fv::kThreads, 0, st>>>(sh, du, xbar, part, splits, kchunk); \
+        else fv::bwd_dwx_kernel<RT, false><<<grid, fv::kThreads, 0, st>>>(sh, du, xbar, part, splits, kchunk); \
+        break;
+    switch ((sh.J + 15) / 16) {
+        FV_DWX(1)
+        FV_DWX(2)
+        FV_DWX(3)
+        FV_DWX(4)
+        FV_DWX(5)
+        FV_DWX(6)
+        default: return FV_ERR_UNSUPPORTED;
+    }
+#undef FV_DWX
+    FV_LAUNCH_CHECK("bwd_dwx_kernel");
     return FV_OK;
 }
 
@@ -1198,16 +1210,16 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
         FV_MARK_CALL(marks, st, reduce(segs, 1, "bwd_reduce_kernel (du)"));
     }
     // 3. x_proj: dW_x = du^T xbar (split-K partials), dxbar = the scans' share + sum_k du[k] W_x[k]
-    const int wx_tiles = ((sh.J + 63) / 64) * ((sh.E + 63) / 64) * sh.nd;
+    const int wx_tiles = ((sh.E + fv::kGwE - 1) / fv::kGwE) * sh.nd;
     const int wx_chunk = bwd_kchunk(M, std::min(bwd_splits(M, wx_tiles, sms), kMaxWxSplits));
     const int wx_splits = (M + wx_chunk - 1) / wx_chunk;
-    FV_MARK_CALL(marks, st, launch_bwd_gemm(sh.J, sh.E, M, sh.nd, wx_splits, fv::OpDuJM{du, sh},
-                                            fv::OpXbar{xbar, sh.E},
-                                            fv::OutWx{(float*)(ws + L.part_wx), sh.J, sh.E, sh.nd, wx_splits}, st,
-                                            "bwd_gemm_kernel (W_x)"));
-    FV_MARK_CALL(marks, st, launch_bwd_gemm(M, sh.E, sh.nd * sh.J, 1, 1, fv::OpDuMK{du, sh}, fv::OpWx{a->W_x, sh.E},
-                                            fv::OutDxbar{dxbar, dxs, sh.T, sh.E, sh.nd}, st,
-                                            "bwd_gemm_kernel (xbar)"));
+    FV_MARK_CALL(marks, st, launch_bwd_dwx(sh, du, xbar, (float*)(ws + L.part_wx), wx_splits, wx_chunk, st));
+    FV_MARK_CALL(marks, st, ([&]() -> fv_status {
+        const dim3 grid((M + fv::kGxM - 1) / fv::kGxM, (sh.E + fv::kGxE - 1) / fv::kGxE);
+        fv::bwd_dxbar_kernel<<<grid, fv::kThreads, 0, st>>>(sh, du, a->W_x, dxs, dxbar);
+        FV_LAUNCH_CHECK("bwd_dxbar_kernel");
+        return FV_OK;
+    })());
     // 4. pooling
     if (sh.K == 0) {
         const int threads = fv::bwd_groups(sh.SL) * fv::bwd_slot_width(sh.SL);

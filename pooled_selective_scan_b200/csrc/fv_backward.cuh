@@ -12,7 +12,7 @@
 //   bwd_scan_kernel                                  adjoint of both scans: dDelta, and through
 //                                                    dt_proj + softplus d dt_low, dW_dt, db_dt; dB,
 //                                                    dC, dA_log and the scans' share of dxbar
-//   bwd_gemm_kernel (2 launches)                     x_proj: dW_x, dxbar
+//   bwd_dwx_kernel, bwd_dxbar_kernel                 x_proj: dW_x (split-K partials), dxbar
 //   bwd_pool_dense_kernel / bwd_pool_masked_kernel   pooling: dx += pool_scale / S dxbar of the
 //                                                    token's row
 // Inputs of the forward that the gradient reuses (xbar, the projections u, ys and, masked, the
@@ -931,124 +931,232 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
 }
 
 // ------------------------------------------------------------------------------------------
-// Projection gradients: small GEMMs out[i][j] = sum_kk A(i, kk) B(kk, j)
+// Projection gradients (x_proj: u[k] = xbar W_x[k]^T, J = R + 2N outputs per direction)
 // ------------------------------------------------------------------------------------------
 
-constexpr int kBgTile = 64, kBgK = 16, kBgPad = kBgTile + 4;
+constexpr int kGxM = 128, kGxE = 128, kGxK = 16;  // dxbar tile (tokens x channels) and k-step
+constexpr int kGwE = 128, kGwK = 16;              // dW_x tile columns, tokens per k-step
 
-// Operand accessors.  kContig: the operand is contiguous along kk (A) or along j (B), which picks
-// the coalesced loading order.  k is the direction slot of the launch (blockIdx.z / splits).
-
-// A = du[k][m][jj] as (i = jj, kk = m), for dW_x = du^T xbar
-struct OpDuJM {
-    static constexpr bool kContig = false;
-    const float* du; Shape sh;
-    __device__ float operator()(int k, int i, int kk) const {
-        const int b = kk / sh.T, t = kk - b * sh.T;
-        return du[u_offset(sh, k, b, t) + i];
-    }
-};
-// B = xbar[m][e] as (kk = m, j = e)
-struct OpXbar {
-    static constexpr bool kContig = true;
-    const float* xbar; int E;
-    __device__ float operator()(int, int kk, int j) const { return xbar[(size_t)kk * E + j]; }
-};
-// A = du[k'][m][jj] as (i = m, kk = k' J + jj), for dxbar = sum_k' du[k'] W_x[k']
-struct OpDuMK {
-    static constexpr bool kContig = true;
-    const float* du; Shape sh;
-    __device__ float operator()(int, int i, int kk) const {
-        const int kd = kk / sh.J, jj = kk - kd * sh.J;
-        const int b = i / sh.T, t = i - b * sh.T;
-        return du[u_offset(sh, kd, b, t) + jj];
-    }
-};
-// B = W_x[k'][jj][e] as (kk = k' J + jj, j = e)
-struct OpWx {
-    static constexpr bool kContig = true;
-    const float* W_x; int E;
-    __device__ float operator()(int, int kk, int j) const { return W_x[(size_t)kk * E + j]; }
-};
-
-// Outputs.
-struct OutWx {  // split-K partial sums of dW_x: part [splits][nd][J][E], added in split order later
-    static constexpr bool kVec4 = true;  // 4 consecutive j at once (E is a multiple of 4)
-    float* part; int J, E, nd, splits;
-    __device__ float* at(int k, int i, int j) const {
-        const int s = (int)blockIdx.z % splits;  // the GEMM's grid z is (direction, split)
-        return part + (((size_t)s * nd + k) * J + i) * E + j;
-    }
-    __device__ void operator()(int k, int i, int j, float v) const { *at(k, i, j) = v; }
-    __device__ void store4(int k, int i, int j, float4 v) const { *reinterpret_cast<float4*>(at(k, i, j)) = v; }
-};
-struct OutDxbar {  // dxbar = the scans' share (summed over directions) + the projections' share
-    static constexpr bool kVec4 = false;
-    float* dxbar; const float* dxs; int T, E, nd;
-    __device__ void operator()(int, int i, int j, float v) const {
-        const int b = i / T, t = i - b * T;
-        for (int k = 0; k < nd; ++k) v += dxs[(((size_t)b * nd + k) * T + t) * E + j];
-        dxbar[(size_t)i * E + j] = v;
-    }
-};
-
-// 64 x 64 output tile per block of 256 threads (4 x 4 per thread), k-steps of 16 through shared
-// memory.  Grid (ceil(M / 64), ceil(Nc / 64), nd * splits); split s of direction k covers
-// kk in [s * kchunk, min(Kd, (s + 1) * kchunk)).
-template <class AOp, class BOp, class COp>
-__global__ void __launch_bounds__(kThreads)
-bwd_gemm_kernel(int M, int Nc, int Kd, int splits, int kchunk, AOp A, BOp Bm, COp C) {
-    __shared__ __align__(16) float As[kBgK][kBgPad];
-    __shared__ __align__(16) float Bs[kBgK][kBgPad];
-    const int k = blockIdx.z / splits, s = blockIdx.z - k * splits;
-    const int i0 = blockIdx.x * kBgTile, j0 = blockIdx.y * kBgTile;
-    const int kbeg = s * kchunk, kend = min(Kd, kbeg + kchunk);
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    float acc[4][4];
+// dxbar[m][e] = sum_k sum_jj du[k][m][jj] W_x[k][jj][e] + sum_k dxs[b][k][t][e] (m = b T + t): the
+// projections' share, then the scans' share added in direction order.  Grid (ceil(M / 128),
+// ceil(E / 128)), 256 threads; thread (ty, tx) = (tid / 16, tid % 16) holds 8 x 8 outputs: tokens
+// 4 ty .. and 64 + 4 ty .., channels 4 tx .. and 64 + 4 tx ...  The k loop takes 16 projection
+// outputs of one direction per step (zero past J) through a cp.async double buffer: du transposed
+// to [16][128 tokens] by 4-byte copies (each thread copies 8 entries of one token's row), W_x rows
+// [16][128 channels] by 16-byte copies.  The k order is that of the plain sum (direction, then jj).
+__global__ void __launch_bounds__(kThreads, 2)
+bwd_dxbar_kernel(Shape sh, const float* __restrict__ du, const float* __restrict__ W_x,
+                 const float* __restrict__ dxs, float* __restrict__ dxbar) {
+    __shared__ __align__(16) float As[2][kGxK][kGxM];
+    __shared__ __align__(16) float Bs[2][kGxK][kGxE];
+    const int T = sh.T, E = sh.E, J = sh.J, nd = sh.nd;
+    const int M = sh.B * T;
+    const int m0 = blockIdx.x * kGxM, e0 = blockIdx.y * kGxE;
+    const int tid = threadIdx.x;
+    // the token whose du entries this thread copies (k rows ck, ck + 2, ..)
+    const int cm = tid & (kGxM - 1), ck = tid >> 7;
+    const int gm = m0 + cm;
+    const bool m_ok = gm < M;
+    const int cb = m_ok ? gm / T : 0;
+    const float* du_row = du + u_offset(sh, 0, cb, m_ok ? gm - cb * T : 0);  // direction 0
+    const size_t ubs = u_block_stride(T, J);                                  // next direction
+    const int jsteps = (J + kGxK - 1) / kGxK, nsteps = nd * jsteps;
+    auto stage = [&](int si) {
+        const int k = si / jsteps, jj0 = (si - k * jsteps) * kGxK, buf = si & 1;
+        const float* src = du_row + k * ubs + jj0;
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+        for (int l = 0; l < kGxK / 2; ++l) {
+            const int kk = ck + 2 * l;
+            const bool ok = m_ok && jj0 + kk < J;
+            cp_async4z(&As[buf][kk][cm], ok ? src + kk : du, ok);
+        }
 #pragma unroll
-        for (int bq = 0; bq < 4; ++bq) acc[a][bq] = 0.f;
-    for (int kk0 = kbeg; kk0 < kend; kk0 += kBgK) {
+        for (int l = 0; l < 2; ++l) {
+            const int idx = tid + kThreads * l;
+            const int kk = idx >> 5, c4 = (idx & 31) * 4;
+            const bool ok = jj0 + kk < J && e0 + c4 < E;
+            const float* w = W_x + ((size_t)k * J + jj0 + kk) * E + e0 + c4;
+            cp_async16(&Bs[buf][kk][c4], ok ? (const void*)w : (const void*)W_x, ok ? 16u : 0u);
+        }
+        cp_async_commit();
+    };
+    const int tx = tid & 15, ty = tid >> 4;
+    float acc[8][8];
 #pragma unroll
-        for (int l = 0; l < 4; ++l) {
-            const int idx = threadIdx.x + l * kThreads;
-            int ii, kk;
-            if (AOp::kContig) { kk = idx & 15; ii = idx >> 4; }
-            else { ii = idx & 63; kk = idx >> 6; }
-            const int gi = i0 + ii, gk = kk0 + kk;
-            As[kk][ii] = (gi < M && gk < kend) ? A(k, gi, gk) : 0.f;
-            int jj;
-            if (BOp::kContig) { jj = idx & 63; kk = idx >> 6; }
-            else { kk = idx & 15; jj = idx >> 4; }
-            const int gj = j0 + jj, gk2 = kk0 + kk;
-            Bs[kk][jj] = (gj < Nc && gk2 < kend) ? Bm(k, gk2, gj) : 0.f;
+    for (int p = 0; p < 8; ++p)
+#pragma unroll
+        for (int r = 0; r < 8; ++r) acc[p][r] = 0.f;
+    stage(0);
+    for (int si = 0; si < nsteps; ++si) {
+        if (si + 1 < nsteps) {
+            stage(si + 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
         }
         __syncthreads();
+        const int buf = si & 1;
 #pragma unroll
-        for (int kk = 0; kk < kBgK; ++kk) {
-            const float4 a = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
-            const float4 bv = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
-            const float av[4] = {a.x, a.y, a.z, a.w}, bw[4] = {bv.x, bv.y, bv.z, bv.w};
+        for (int kk = 0; kk < kGxK; ++kk) {
+            const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][4 * ty]);
+            const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + 4 * ty]);
+            const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][4 * tx]);
+            const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + 4 * tx]);
+            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-            for (int p = 0; p < 4; ++p)
+            for (int p = 0; p < 8; ++p)
 #pragma unroll
-                for (int r = 0; r < 4; ++r) acc[p][r] = fmaf(av[p], bw[r], acc[p][r]);
+                for (int r = 0; r < 8; ++r) acc[p][r] = fmaf(av[p], bv[r], acc[p][r]);
         }
-        __syncthreads();
+        __syncthreads();  // the buffer is refilled by the stage after next
     }
+    // two rows at a time: their scan shares (up to 8 float4, read once: streaming loads) are all
+    // requested before the first is used
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        const int gi = i0 + ty * 4 + p, gj = j0 + tx * 4;
-        if constexpr (COp::kVec4) {
-            if (gi < M && gj + 3 < Nc) {
-                C.store4(k, gi, gj, make_float4(acc[p][0], acc[p][1], acc[p][2], acc[p][3]));
-                continue;
+    for (int p0 = 0; p0 < 8; p0 += 2) {
+        float4 sv[2][2][2];
+        int mrow[2];
+#pragma unroll
+        for (int pp = 0; pp < 2; ++pp) {
+            const int p = p0 + pp;
+            const int m = m0 + (p < 4 ? 4 * ty + p : 64 + 4 * ty + p - 4);
+            mrow[pp] = m;
+            const int b = m < M ? m / T : 0, t = m - b * T;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int e = e0 + 64 * hf + 4 * tx;
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    // E is a multiple of 4: e < E covers e + 3
+                    sv[pp][hf][k] = (m < M && e < E && k < nd)
+                                        ? __ldcs(reinterpret_cast<const float4*>(dxs + (((size_t)b * nd + k) * T + t) * E + e))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
             }
         }
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
-            if (gi < M && gj + r < Nc) C(k, gi, gj + r, acc[p][r]);
+        for (int pp = 0; pp < 2; ++pp) {
+            const int p = p0 + pp, m = mrow[pp];
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int e = e0 + 64 * hf + 4 * tx;
+                if (m >= M || e >= E) continue;
+                float4 v = make_float4(acc[p][4 * hf], acc[p][4 * hf + 1], acc[p][4 * hf + 2], acc[p][4 * hf + 3]);
+                f4_add(v, sv[pp][hf][0]);  // the directions' shares in order (+0 past nd)
+                if (nd > 1) f4_add(v, sv[pp][hf][1]);
+                *reinterpret_cast<float4*>(dxbar + (size_t)m * E + e) = v;
+            }
+        }
+    }
+}
+
+// Split-K partial sums of dW_x[k][jj][e] = sum_m du[k][m][jj] xbar[m][e]: split s sums the tokens
+// [s kchunk, min(M, (s + 1) kchunk)) in order into part [splits][nd][J][E] (bwd_reduce_kernel adds
+// the splits in order).  Grid (ceil(E / 128), nd * splits), 256 threads, RT = ceil(J / 16): thread
+// (ty, tx) = (tid / 16, tid % 16) holds rows RT ty .. RT ty + RT - 1 and channels 4 tx .. and
+// 64 + 4 tx ...  Each k-step stages 16 tokens through a cp.async double buffer: their du rows
+// [16][16 RT] (zero past J; 16-byte copies when VEC: J a multiple of 4, else 4-byte ones) and their
+// xbar rows [16][128] (16-byte copies).
+template <int RT, bool VEC>
+__global__ void __launch_bounds__(kThreads)
+bwd_dwx_kernel(Shape sh, const float* __restrict__ du, const float* __restrict__ xbar, float* __restrict__ part,
+               int splits, int kchunk) {
+    constexpr int JP = 16 * RT;
+    __shared__ __align__(16) float As[2][kGwK][JP];
+    __shared__ __align__(16) float Bs[2][kGwK][kGwE];
+    const int T = sh.T, E = sh.E, J = sh.J;
+    const int M = sh.B * T;
+    const int k = blockIdx.y / splits, s = blockIdx.y - k * splits;
+    const int e0 = blockIdx.x * kGwE;
+    const int mbeg = s * kchunk, mend = min(M, mbeg + kchunk);
+    const int nsteps = (max(mend - mbeg, 0) + kGwK - 1) / kGwK;
+    const int tid = threadIdx.x;
+    auto stage = [&](int si) {
+        const int m0 = mbeg + si * kGwK, buf = si & 1;
+        const int b0 = m0 / T, t0 = m0 - b0 * T;
+        if (VEC) {  // J a multiple of 4: 16-byte copies of the du rows
+            for (int idx = tid; idx < kGwK * (JP / 4); idx += kThreads) {
+                const int kk = idx / (JP / 4), j4 = 4 * (idx - kk * (JP / 4));
+                const bool ok = m0 + kk < mend && j4 < J;
+                const float* src = du;
+                if (ok) {
+                    int b = b0, t = t0 + kk;
+                    while (t >= T) {
+                        t -= T;
+                        ++b;
+                    }
+                    src = du + u_offset(sh, k, b, t) + j4;
+                }
+                cp_async16(&As[buf][kk][j4], src, ok ? 16u : 0u);
+            }
+        } else {
+            for (int idx = tid; idx < kGwK * JP; idx += kThreads) {
+                const int kk = idx / JP, jj = idx - kk * JP;
+                const bool ok = m0 + kk < mend && jj < J;
+                const float* src = du;
+                if (ok) {
+                    int b = b0, t = t0 + kk;
+                    while (t >= T) {
+                        t -= T;
+                        ++b;
+                    }
+                    src = du + u_offset(sh, k, b, t) + jj;
+                }
+                cp_async4z(&As[buf][kk][jj], src, ok);
+            }
+        }
+#pragma unroll
+        for (int l = 0; l < 2; ++l) {
+            const int idx = tid + kThreads * l;
+            const int kk = idx >> 5, c4 = (idx & 31) * 4;
+            const bool ok = m0 + kk < mend && e0 + c4 < E;
+            const float* x = xbar + (size_t)(m0 + kk) * E + e0 + c4;
+            cp_async16(&Bs[buf][kk][c4], ok ? (const void*)x : (const void*)xbar, ok ? 16u : 0u);
+        }
+        cp_async_commit();
+    };
+    const int tx = tid & 15, ty = tid >> 4;
+    float acc[RT][8];
+#pragma unroll
+    for (int p = 0; p < RT; ++p)
+#pragma unroll
+        for (int r = 0; r < 8; ++r) acc[p][r] = 0.f;
+    if (nsteps > 0) stage(0);
+    for (int si = 0; si < nsteps; ++si) {
+        if (si + 1 < nsteps) {
+            stage(si + 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const int buf = si & 1;
+#pragma unroll
+        for (int kk = 0; kk < kGwK; ++kk) {
+            const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][4 * tx]);
+            const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + 4 * tx]);
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int p = 0; p < RT; ++p) {
+                const float av = As[buf][kk][RT * ty + p];
+#pragma unroll
+                for (int r = 0; r < 8; ++r) acc[p][r] = fmaf(av, bv[r], acc[p][r]);
+            }
+        }
+        __syncthreads();  // the buffer is refilled by the stage after next
+    }
+#pragma unroll
+    for (int p = 0; p < RT; ++p) {
+        const int jj = RT * ty + p;
+        if (jj >= J) continue;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const int e = e0 + 64 * hf + 4 * tx;
+            if (e >= E) continue;
+            *reinterpret_cast<float4*>(part + (((size_t)s * sh.nd + k) * J + jj) * E + e) =
+                make_float4(acc[p][4 * hf], acc[p][4 * hf + 1], acc[p][4 * hf + 2], acc[p][4 * hf + 3]);
+        }
     }
 }
 

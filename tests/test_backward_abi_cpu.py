@@ -85,7 +85,7 @@ def test_launch_lists(lib):
     dense = [lib.fastvim_ssm_backward_launch_name(ctypes.byref(args()), i).decode() for i in range(8)]
     assert lib.fastvim_ssm_backward_launch_count(ctypes.byref(args())) == 8
     assert dense == ["bwd_gate_dense_kernel", "dt_proj_kernel", "bwd_scan_kernel", "bwd_reduce_kernel:du",
-                     "bwd_gemm_kernel:W_x", "bwd_gemm_kernel:xbar", "bwd_pool_dense_kernel",
+                     "bwd_dwx_kernel", "bwd_dxbar_kernel", "bwd_pool_dense_kernel",
                      "bwd_reduce_kernel:params"]
     m = args(K=49, keep_idx=FAKE + 9 * SLOT)
     masked = [lib.fastvim_ssm_backward_launch_name(ctypes.byref(m), i).decode() for i in range(8)]
