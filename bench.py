@@ -18,9 +18,10 @@ CUDA-event time.  Rank 0 prints one JSON line.
 --impl reference times the fp64 CPU oracle on the host cores instead (rank 0 only), on a bounded
 sample of images of the same workload per step.
 
---grad times a training step of the layer instead: the forward call and then the gradient call
-(fastvim_ssm_backward: dx, dz and the parameter gradients for a seeded upstream gradient dy) over
-the same batch, and prints its own line for that.
+--grad times a training step of the layer instead: the forward call (keeping the scan states,
+FV_FLAG_KEEP_STATES, unless --recompute-states) and then the gradient call (fastvim_ssm_backward:
+dx, dz and the parameter gradients for a seeded upstream gradient dy) over the same batch, and
+prints its own line for that.
 """
 from __future__ import annotations
 
@@ -125,6 +126,9 @@ def parse(argv=None):
                          "workloads and reports them under 'configs')")
     ap.add_argument("--grad", action="store_true",
                     help="time a training step: the forward call, then the gradient call on its workspace")
+    ap.add_argument("--recompute-states", action="store_true",
+                    help="--grad without FV_FLAG_KEEP_STATES: the gradient reruns the recurrences for their "
+                         "states instead of reading the ones the forward kept")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -697,7 +701,7 @@ def run_grad(a, cfg, pool_axis):
     dy = workload.upstream_grad(cfg, dev)
     keep = t.get("keep_idx")
     shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, cfg.dir_flags, keep, cfg.h, cfg.w, path=a.path,
-                            ln=a.ln)
+                            ln=a.ln, keep_states=not a.recompute_states)
     y = torch.empty_like(t["x"])
     fws = ssm.alloc_workspace(shape, dev)
     bws = torch.empty(max(ssm.backward_workspace_size(shape), 256), dtype=torch.uint8, device=dev)
@@ -769,6 +773,8 @@ def run_grad(a, cfg, pool_axis):
         "ms_per_step": ms / a.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic (seeded N(0,1) x, z, dy; Mamba-style parameter init)",
         "config": dict(workload_desc(cfg, pool_axis), step="forward call + gradient call",
+                       scan_states="kept by the forward (FV_FLAG_KEEP_STATES)" if shape.keep_states
+                       else "recomputed by the gradient",
                        l2=("no flush (inputs > 2 x L2)" if flush is None else "L2 flushed before every step")),
         "gradient": {"ms": bwd_ms, "hbm_floor_ms": 5 * 4 * cfg.E * tokens / (peak * 1e9) * 1e3,
                      "floor_note": "x, z, dy read once, dx, dz written once at the measured copy rate"},

@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define FASTVIM_SSM_ABI_VERSION 5
+#define FASTVIM_SSM_ABI_VERSION 6
 
 #if defined(__GNUC__)
 #define FV_API __attribute__((visibility("default")))
@@ -89,7 +89,11 @@ enum {
     FV_FLAG_TRACE = 8u,       /* fused launch: record one entry per task in the workspace
                                  (fv_ws_layout.trace); costs a little time, for profiling      */
     FV_FLAG_LAYERNORM = 16u,  /* post-SSM LayerNorm before the gate (ln_gamma, ln_beta, ln_eps) */
-    FV_FLAG_CONV_SILU = 32u   /* SiLU after the block's Conv1D (needs d_conv > 0)               */
+    FV_FLAG_CONV_SILU = 32u,  /* SiLU after the block's Conv1D (needs d_conv > 0)               */
+    FV_FLAG_KEEP_STATES = 64u /* training: the scans also store their 16 states before every 8th
+                                 step (fv_ws_layout.ckpt, B nd 2 ceil(T/16) E 64 bytes more
+                                 workspace) so that the gradient call reads them instead of
+                                 running the recurrences a first time; y is unchanged          */
 };
 /* Without a PATH flag a dense layer without FV_FLAG_LAYERNORM whose images hold >= 16 MiB of x
  * runs the fused launch, every other layer the staged kernels; both compute the same layer.  The fused launch gates image b
@@ -166,7 +170,9 @@ typedef struct {
                             w1 = SM id << 32 | CTA id, w2 = start (ns, %globaltimer),
                             w3 = wait_ns << 40 | total_ns (from start to the task's end)        */
     size_t trace_records;  /* number of trace entries (tasks of the call), else 0               */
-    size_t scan_bc;      /* reserved, 0                                                      */
+    size_t ckpt;         /* FV_FLAG_KEEP_STATES: fp32 [B][nd][2 ceil(T/16)][E][16], the 16 states
+                            of each scan entering its steps 0, 8, 16, .. (scan order), zero
+                            past N; else 0                                                  */
     size_t scan_dt;      /* reserved, 0                                                      */
     int T, S, nd;        /* pooled length, pooled-over length, number of directions          */
 } fv_ws_layout;
@@ -297,7 +303,8 @@ typedef struct {
     size_t dxbar;        /* float [B][T][E]   dL/dxbar                                         */
     size_t du;           /* float, the layout of the forward's u: d dt_low | dB | dC           */
     size_t dxs;          /* float [B][nd][T][E]  the scans' share of dL/dxbar per direction     */
-    size_t ckpt;         /* float [B][nd][2 ceil(T/16)][E][16]  scan state entering every 8 steps */
+    size_t ckpt;         /* float [B][nd][2 ceil(T/16)][E][16]  scan state entering every 8 steps;
+                            0 with FV_FLAG_KEEP_STATES (the forward's are read)               */
     size_t status;       /* uint32 device status word (FV_ERR_TIMEOUT from a bounded wait), read
                             by fastvim_get_device_status(ws, stream); the call clears it       */
     size_t delta;        /* float [nd][B][T][E] step sizes Delta, computed by the gradient call
@@ -319,7 +326,7 @@ FV_API const char* fastvim_ssm_backward_launch_name(const fv_ssm_args* args, int
  * args: the forward call's arguments (the same tensors; y is not read and may be NULL).
  * fwd_ws: the workspace of a fastvim_ssm_forward (or _events) call with these args that is
  *   complete or queued earlier on `stream`: the gradient reads its pooled tokens, projections,
- *   scan outputs and (masked) row lists.  fwd_ws_bytes >= fastvim_ssm_workspace_size(args).
+ *   scan outputs, (masked) row lists and, with FV_FLAG_KEEP_STATES, the scan states.  fwd_ws_bytes >= fastvim_ssm_workspace_size(args).
  * ws: the gradient's own workspace, >= fastvim_ssm_backward_workspace_size(args) bytes, 256-byte
  *   aligned, no initial contents; fwd_ws and ws must not overlap.
  * grads: device arrays, 16-byte aligned; dx and dz must not overlap each other, x, z or dy.

@@ -29,6 +29,7 @@ FV_FLAG_PATH_FUSED = 4
 FV_FLAG_TRACE = 8
 FV_FLAG_LAYERNORM = 16
 FV_FLAG_CONV_SILU = 32
+FV_FLAG_KEEP_STATES = 64
 
 # Every exported symbol of the ABI, as the header declares it.
 EXPORTS = (
@@ -81,7 +82,7 @@ class FvWsLayout(ctypes.Structure):
         ("u", ctypes.c_size_t), ("ys", ctypes.c_size_t), ("row_of", ctypes.c_size_t),
         ("row_off", ctypes.c_size_t), ("row_tok", ctypes.c_size_t),
         ("delta", ctypes.c_size_t), ("ctrl", ctypes.c_size_t), ("trace", ctypes.c_size_t),
-        ("trace_records", ctypes.c_size_t), ("scan_bc", ctypes.c_size_t), ("scan_dt", ctypes.c_size_t),
+        ("trace_records", ctypes.c_size_t), ("ckpt", ctypes.c_size_t), ("scan_dt", ctypes.c_size_t),
         ("T", ctypes.c_int), ("S", ctypes.c_int), ("nd", ctypes.c_int),
     ]
 

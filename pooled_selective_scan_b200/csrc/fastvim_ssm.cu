@@ -45,7 +45,7 @@ fv_status make_shape(const fv_ssm_args* a, fv::Shape* sh) {
     if (a->pool_axis != FV_POOL_W && a->pool_axis != FV_POOL_H) return FV_ERR_SHAPE;
     if (a->dir_flags == 0 || (a->dir_flags & ~3u) != 0) return FV_ERR_SHAPE;
     if ((a->flags & ~(unsigned)(FV_FLAG_ZOH_EXACT | FV_FLAG_PATH_STAGED | FV_FLAG_PATH_FUSED | FV_FLAG_TRACE |
-                                FV_FLAG_LAYERNORM | FV_FLAG_CONV_SILU)) != 0)
+                                FV_FLAG_LAYERNORM | FV_FLAG_CONV_SILU | FV_FLAG_KEEP_STATES)) != 0)
         return FV_ERR_SHAPE;
     if (a->d_conv < 0) return FV_ERR_SHAPE;
     if (a->d_conv == 0 && (a->flags & FV_FLAG_CONV_SILU)) return FV_ERR_SHAPE;  // SiLU of no Conv1D
@@ -78,6 +78,7 @@ fv_status make_shape(const fv_ssm_args* a, fv::Shape* sh) {
     sh->dc = a->d_conv;
     sh->conv_silu = (a->flags & FV_FLAG_CONV_SILU) ? 1 : 0;
     sh->nx = a->d_conv > 0 ? sh->nd : 1;
+    sh->keep = (a->flags & FV_FLAG_KEEP_STATES) ? 1 : 0;
     if (a->d_conv > fv::kMaxConv) return FV_ERR_UNSUPPORTED;
     if (a->d_conv > 0 && a->K > 0) return FV_ERR_UNSUPPORTED;  // the Conv1D is for dense grids
     if (sh->T > kMaxT) return FV_ERR_UNSUPPORTED;
@@ -124,6 +125,9 @@ fv_status plan_layout(const fv::Shape& sh, fv_ws_layout* L) {
     L->ys = off; off = round256(off + (size_t)sh.B * sh.T * sh.E * sizeof(float));
     if (choose_path(sh) != Path::Fused && fv::staged_delta_kernel(sh)) {  // step sizes of the staged dt_proj kernel
         L->delta = off; off = round256(off + (size_t)sh.nd * sh.B * sh.T * sh.E * sizeof(float));
+    }
+    if (sh.keep) {  // the scan states every 8 steps, for the gradient
+        L->ckpt = off; off = round256(off + (size_t)sh.B * sh.nd * fv::ckpt_count(sh.T) * sh.E * 16 * sizeof(float));
     }
     if (sh.K > 0) {
         L->row_of = off; off = round256(off + (size_t)sh.B * sh.K * sizeof(int32_t));
@@ -347,6 +351,7 @@ fv::FusedPtrs fused_ptrs(const fv_ssm_args* a, const fv_ws_layout& L, char* ws) 
     p.status = (unsigned*)(ws + L.status);
     p.ctrl = L.ctrl ? (unsigned*)(ws + L.ctrl) : nullptr;
     p.trace = L.trace_records ? (unsigned long long*)(ws + L.trace) : nullptr;
+    p.ckpt = L.ckpt ? (float*)(ws + L.ckpt) : nullptr;
     return p;
 }
 
@@ -376,7 +381,8 @@ fv_status launch_scan_seq(const fv::Shape& sh, const fv_ssm_args* a, const fv_ws
     if (grid >= (1ll << 31)) return FV_ERR_UNSUPPORTED;
     kern<<<(unsigned)grid, fv::kSeqThreads, smem, st>>>(sh, (const float*)(ws + L.u), (const float*)(ws + L.xbar),
                                                          a->A_log, a->W_dt, a->b_dt,
-                                                         din ? (const float*)(ws + L.delta) : nullptr, ys);
+                                                         din ? (const float*)(ws + L.delta) : nullptr, ys,
+                                                         L.ckpt ? (float*)(ws + L.ckpt) : nullptr);
     FV_LAUNCH_CHECK("scan_seq_kernel");
     return FV_OK;
 }
@@ -909,8 +915,10 @@ BwdLayout plan_bwd(const fv::Shape& sh) {
     L.dxbar = off; off = round256(off + bte);
     L.du = off; off = round256(off + (size_t)sh.nd * sh.B * fv::u_block_stride(sh.T, sh.J) * sizeof(float));
     L.dxs = off; off = round256(off + (size_t)sh.nd * bte);
-    L.ckpt = off;
-    off = round256(off + (size_t)sh.B * sh.nd * fv::bs_nckpt(sh.T) * sh.E * 16 * sizeof(float));
+    if (!sh.keep) {  // else the forward kept the scan states in its workspace
+        L.ckpt = off;
+        off = round256(off + (size_t)sh.B * sh.nd * fv::bs_nckpt(sh.T) * sh.E * 16 * sizeof(float));
+    }
     if (!fwd_has_delta(sh)) {
         L.delta = off;
         off = round256(off + (size_t)sh.nd * sh.B * sh.T * sh.E * sizeof(float));
@@ -1073,7 +1081,9 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
     float* dxbar = (float*)(ws + L.dxbar);
     float* du = (float*)(ws + L.du);
     float* dxs = (float*)(ws + L.dxs);
-    float* ckpt = (float*)(ws + L.ckpt);
+    // the scan states every 8 steps: kept by the forward (FV_FLAG_KEEP_STATES), else pass 1 of
+    // bwd_scan_kernel writes them here
+    float* ckpt = sh.keep ? (float*)(fw + FL.ckpt) : (float*)(ws + L.ckpt);
     // the step sizes: the forward's (staged, dt_rank >= 32), else computed below into ws
     const float* delta = L.delta ? (const float*)(ws + L.delta) : (const float*)(fw + FL.delta);
     float* part_du = (float*)(ws + L.part_du);

@@ -31,8 +31,9 @@ constexpr int kBsChunk = 16;     // steps per staged chunk
 constexpr int kBsHalf = 8;       // steps per checkpoint (two per staged chunk)
 
 __host__ __device__ __forceinline__ int bs_nchunks(int T) { return (T + kBsChunk - 1) / kBsChunk; }
-// checkpoints per scan: one every 8 steps of the scan order
-__host__ __device__ __forceinline__ int bs_nckpt(int T) { return 2 * bs_nchunks(T); }
+// checkpoints per scan: one every 8 steps of the scan order (the forward's kept-state layout)
+__host__ __device__ __forceinline__ int bs_nckpt(int T) { return ckpt_count(T); }
+static_assert(kBsChunk == 2 * kCkptSteps && kBsHalf == kCkptSteps, "checkpoint layout");
 // dt_rank rounded up to whole float4s (the dt_low rows and the dW_dt sums are read as float4).
 __host__ __device__ __forceinline__ int bs_r4(int R) { return (R + 3) & ~3; }
 constexpr int kBsWS = 64 + 4;  // row stride of W_dt transposed, [r][channel]: float4-aligned rows
@@ -617,7 +618,8 @@ bwd_ln_gate_reg_kernel(Shape sh, const float* __restrict__ x, const float* __res
 // Delta comes from a buffer: the forward's (staged path, dt_rank >= 32) or the one the gradient call
 // fills first with dt_proj_kernel; sig(v) = softplus'(v) = 1 - e^-Delta.
 // Pass 1 runs the recurrence in scan order and stores the state entering every 8 steps
-// (ckpt [B][nd][2 nchunks][E][16]).  Pass 2 walks the 16-step staged chunks in reverse, each as two
+// (ckpt [B][nd][2 nchunks][E][16]); with FV_FLAG_KEEP_STATES the forward stored them (ckpt is
+// then its buffer) and pass 1 is skipped.  Pass 2 walks the 16-step staged chunks in reverse, each as two
 // halves of 8 steps, last half first: it recomputes the half's states from its checkpoint (8 steps
 // x 4 states in registers, which keeps the kernel at two resident blocks per SM) and steps the
 // adjoint back through them.  Per step: dDelta and the scans' dxbar are summed over the 4 lanes of
@@ -652,12 +654,12 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
     const int e = e0 + c;
     const bool live = e < E;
     const bool fwd = sh.nd == 2 ? k == 0 : (sh.dir_flags & 1u) != 0;
-    const int nchunks = bs_nchunks(T), nckpt = bs_nckpt(T);
+    const int nchunks = bs_nchunks(T);
     const float* ub = u + u_offset(sh, k, b, 0);
     // this CTA's share of du (dB, dC and d dt_low summed over its 64 channels): part_du holds one
     // copy of du's layout per 64-channel tile
     float* pdu = part_du + (size_t)blockIdx.z * sh.nd * sh.B * u_block_stride(T, J);
-    auto ckpt_at = [&](int c) { return ckpt + ((((size_t)b * sh.nd + k) * nckpt + c) * E + e) * 16 + 4 * q; };
+    auto ckpt_at = [&](int c) { return ckpt + ckpt_offset(sh, b, k, c, e) + 4 * q; };
 
     for (int i = tid; i < kBsCh * R; i += kBsThreads) {
         const int row = i / R, r = i - row * R;
@@ -736,10 +738,10 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
         return ZOH_EXACT ? expm1f(dt * An[j]) * Ainv[j] * Bn * xv : dt * Bn * xv;
     };
 
-    stage(0);
-    // ---- pass 1: states entering each chunk ----
+    // ---- pass 1: states entering each chunk (skipped when the forward kept them) ----
+    stage(sh.keep ? nchunks : 0);
     float h[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int it = 0; it < nchunks; ++it) {
+    for (int it = 0; it < (sh.keep ? 0 : nchunks); ++it) {
         const float* sb = arrive(it);
         const float* sbc = sb + kBsChunk * R4;
         const float* sx = sbc + kBsChunk * 32;

@@ -32,6 +32,7 @@ struct Shape {
     int dc;            // taps of the block's Conv1D in front of the layer (0: x is its output)
     int conv_silu;     // FV_FLAG_CONV_SILU: SiLU after the Conv1D
     int nx;            // pooled-token sets: nd with the Conv1D (one per direction), else 1
+    int keep;          // FV_FLAG_KEEP_STATES: the scans store their states for the gradient
 };
 
 constexpr int kMaxConv = 4;  // Conv1D taps at most
@@ -39,6 +40,15 @@ constexpr int kMaxConv = 4;  // Conv1D taps at most
 // Pooled tokens of image b, set kx (the direction's own with the Conv1D, else 0): [T][E] rows.
 __host__ __device__ __forceinline__ size_t xbar_offset(const Shape& sh, int b, int kx, int t) {
     return (((size_t)b * sh.nx + kx) * sh.T + t) * (size_t)sh.E;
+}
+
+// Scan states kept for the gradient (FV_FLAG_KEEP_STATES): the 16 states of (image b, direction
+// k, channel e) entering steps 0, 8, 16, .. of the scan order (slot c: the state before the
+// scan's step 8c), [B][nd][2 ceil(T / 16)][E][16], zero for states n >= N.
+constexpr int kCkptSteps = 8;
+__host__ __device__ __forceinline__ int ckpt_count(int T) { return 2 * ((T + 15) / 16); }
+__host__ __device__ __forceinline__ size_t ckpt_offset(const Shape& sh, int b, int k, int c, int e) {
+    return ((((size_t)b * sh.nd + k) * ckpt_count(sh.T) + c) * sh.E + e) * 16;
 }
 
 // Projections u of (image b, direction k) are one block of T x J floats, image-major (so the

@@ -89,6 +89,7 @@ struct FusedPtrs {
     unsigned* status;
     unsigned* ctrl;
     unsigned long long* trace;  // NULL, or 4 words per ticket
+    float* ckpt;                // NULL, or the kept scan states (FV_FLAG_KEEP_STATES)
 };
 
 // Per-CTA state of the TMA ring, kept across tasks.
@@ -479,7 +480,7 @@ __device__ __forceinline__ void fused_scan(const Shape& sh, const FusedPlan& pl,
                                            float* smem) {
     const int e0 = tile * pl.ECH;
     seq_scan<kFusedThreads, ND, ZOH_EXACT>(sh, p.u, p.xbar, p.A_log, p.W_dt, p.b_dt, nullptr, p.ys + (size_t)b * sh.T * sh.E + e0,
-                                           sh.E, b, e0, 0, smem);
+                                           sh.E, b, e0, 0, smem, p.ckpt);
     cta_signal(p.ctrl ? p.ctrl + kCtrlHeaderWords + 2 * sh.B + b : nullptr);
 }
 

@@ -878,11 +878,12 @@ proj_gemm_kernel(Shape sh, const float* __restrict__ xbar, const float* __restri
 
 // ---- Staged scans: one CTA per (image, 128-channel tile, direction) ----------------------------
 // DT_IN: Delta from dt_proj_kernel's buffer; else dt_proj + softplus per chunk in the scan.
+// ckpt: NULL, or where the scans keep their states for the gradient (FV_FLAG_KEEP_STATES).
 template <bool ZOH_EXACT, bool DT_IN>
 __global__ void __launch_bounds__(kSeqThreads)
 scan_seq_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__ xbar,
                 const float* __restrict__ A_log, const float* __restrict__ W_dt, const float* __restrict__ b_dt,
-                const float* __restrict__ delta, float* __restrict__ ys) {
+                const float* __restrict__ delta, float* __restrict__ ys, float* __restrict__ ckpt) {
     extern __shared__ __align__(16) float smem[];
     const int tiles = (sh.E + kSeqThreads - 1) / kSeqThreads;
     const int k = blockIdx.x % sh.nd;
@@ -890,7 +891,7 @@ scan_seq_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
     const int b = blockIdx.x / (sh.nd * tiles);
     const int e0 = tile * kSeqThreads;
     seq_scan<kSeqThreads, 1, ZOH_EXACT, DT_IN>(sh, u, xbar, A_log, W_dt, b_dt, delta,
-                                               ys + (size_t)b * sh.T * sh.E + e0, sh.E, b, e0, k, smem);
+                                               ys + (size_t)b * sh.T * sh.E + e0, sh.E, b, e0, k, smem, ckpt);
 }
 
 // Device math self-test: out[i] = f(in[i]) for the SFU-based helpers the layer uses

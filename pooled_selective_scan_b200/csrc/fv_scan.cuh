@@ -88,6 +88,15 @@ __device__ __forceinline__ float seq_step(float dt, float xv, const float* __res
     return (yp4[0] + yp4[1]) + (yp4[2] + yp4[3]);
 }
 
+// Store a thread's 16 states at `ck` (the chunk loops skip it when the states are not kept or the
+// channel is past E).
+__device__ __forceinline__ void keep_state(float* ck, const float (&h)[kSeqStates]) {
+    static_assert(kSeqStates == 16 && kSeqChunk == 2 * kCkptSteps, "checkpoint layout");
+    float4* d = reinterpret_cast<float4*>(ck);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) d[q] = make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+}
+
 // dt_proj + softplus and the recurrence over one staged chunk of `len` steps (LEN = 16 for a full
 // chunk, 0 for a shorter one).  Slot i holds the i-th step taken; y of slot i goes to yp + i * ystep.
 template <int LEN, int XSTRIDE, bool ZOH_EXACT>
@@ -95,7 +104,8 @@ __device__ __forceinline__ void seq_chunk(const float* __restrict__ bc, const fl
                                           const float* __restrict__ xs, const float* __restrict__ wrow, int R4,
                                           float bias, int len, const float (&A2)[kSeqStates],
                                           const float (&An)[kSeqStates], const float (&Ainv)[kSeqStates],
-                                          float (&h)[kSeqStates], float* yp, ptrdiff_t ystep, bool live, bool add) {
+                                          float (&h)[kSeqStates], float* yp, ptrdiff_t ystep, bool live, bool add,
+                                          float* ck, size_t ck_stride) {
     const int n_steps = LEN ? LEN : len;
     float dl[kSeqChunk];
 #pragma unroll
@@ -119,6 +129,7 @@ __device__ __forceinline__ void seq_chunk(const float* __restrict__ bc, const fl
 #pragma unroll
     for (int i = 0; i < kSeqChunk; ++i) {
         if (LEN || i < n_steps) {
+            if (i % kCkptSteps == 0 && ck) keep_state(ck + (i / kCkptSteps) * ck_stride, h);
             const float y = seq_step<ZOH_EXACT>(softplus_fast(dl[i]), xs[i * XSTRIDE], bc + i * 2 * kSeqStates, A2,
                                                 An, Ainv, h);
             if (live) {
@@ -136,11 +147,13 @@ template <int LEN, int XSTRIDE, bool ZOH_EXACT>
 __device__ __forceinline__ void seq_chunk_dt(const float* __restrict__ bc, const float* __restrict__ dts,
                                              const float* __restrict__ xs, int len, const float (&A2)[kSeqStates],
                                              const float (&An)[kSeqStates], const float (&Ainv)[kSeqStates],
-                                             float (&h)[kSeqStates], float* yp, ptrdiff_t ystep, bool live, bool add) {
+                                             float (&h)[kSeqStates], float* yp, ptrdiff_t ystep, bool live, bool add,
+                                             float* ck, size_t ck_stride) {
     const int n_steps = LEN ? LEN : len;
 #pragma unroll
     for (int i = 0; i < kSeqChunk; ++i) {
         if (LEN || i < n_steps) {
+            if (i % kCkptSteps == 0 && ck) keep_state(ck + (i / kCkptSteps) * ck_stride, h);
             const float y = seq_step<ZOH_EXACT>(dts[i * XSTRIDE], xs[i * XSTRIDE], bc + i * 2 * kSeqStates, A2, An,
                                                 Ainv, h);
             if (live) {
@@ -160,11 +173,14 @@ __device__ __forceinline__ void seq_chunk_dt(const float* __restrict__ bc, const
 // softplus run here per chunk.  The output of step t, channel e0 + c goes to ys0[t * ys_stride + c]
 // ([T][E] rows: ys0 = ys + b T E + e0), zeroed by the caller when both directions add into it.
 // smem: seq_smem_floats_dt(NT, NDC) floats with DT_IN, else seq_smem_floats(NT, NDC, R).
+// ckpt: NULL, or the kept states (ckpt_offset layout; FV_FLAG_KEEP_STATES), written before every
+// 8th step.
 template <int NT, int NDC, bool ZOH_EXACT, bool DT_IN = false>
 __device__ __forceinline__ void seq_scan(const Shape& sh, const float* __restrict__ u, const float* __restrict__ xbar,
                                          const float* __restrict__ A_log, const float* __restrict__ W_dt,
                                          const float* __restrict__ b_dt, const float* __restrict__ delta,
-                                         float* __restrict__ ys0, int ys_stride, int b, int e0, int k0, float* smem) {
+                                         float* __restrict__ ys0, int ys_stride, int b, int e0, int k0, float* smem,
+                                         float* __restrict__ ckpt) {
     constexpr int NS = kSeqStates;
     constexpr int ECH = NT / NDC;             // channels per direction
     const int T = sh.T, E = sh.E, N = sh.N, R = sh.R, J = sh.J;
@@ -262,21 +278,25 @@ __device__ __forceinline__ void seq_scan(const Shape& sh, const float* __restric
         const ptrdiff_t ystep = fwd ? (ptrdiff_t)ys_stride : -(ptrdiff_t)ys_stride;
         const float* bcb = sbc + (buf * NDC + kk) * kSeqChunk * 2 * kSeqStates;
         const float* xb = sxs + (buf * NDC + kk) * kSeqChunk * ECH + c;
+        // the chunk's two kept states (before its steps 0 and 8), or none
+        float* ck = (ckpt && live) ? ckpt + ckpt_offset(sh, b, k, 2 * it, e) : nullptr;
+        const size_t cks = (size_t)E * 16;
         if (DT_IN) {
             const float* db = sdt + (buf * NDC + kk) * kSeqChunk * ECH + c;
             if (len == kSeqChunk)
-                seq_chunk_dt<kSeqChunk, ECH, ZOH_EXACT>(bcb, db, xb, len, A2, An, Ainv, h, yp, ystep, live, add);
+                seq_chunk_dt<kSeqChunk, ECH, ZOH_EXACT>(bcb, db, xb, len, A2, An, Ainv, h, yp, ystep, live, add, ck,
+                                                        cks);
             else
-                seq_chunk_dt<0, ECH, ZOH_EXACT>(bcb, db, xb, len, A2, An, Ainv, h, yp, ystep, live, add);
+                seq_chunk_dt<0, ECH, ZOH_EXACT>(bcb, db, xb, len, A2, An, Ainv, h, yp, ystep, live, add, ck, cks);
         } else {
             const float* dtb = sdt + (buf * NDC + kk) * R4 * kSeqChunk;
             const float* wrow = sw + threadIdx.x * WS;
             if (len == kSeqChunk)
                 seq_chunk<kSeqChunk, ECH, ZOH_EXACT>(bcb, dtb, xb, wrow, R4, bias, len, A2, An, Ainv, h, yp, ystep,
-                                                     live, add);
+                                                     live, add, ck, cks);
             else
                 seq_chunk<0, ECH, ZOH_EXACT>(bcb, dtb, xb, wrow, R4, bias, len, A2, An, Ainv, h, yp, ystep, live,
-                                             add);
+                                             add, ck, cks);
         }
         __syncthreads();  // the buffer is refilled by the next iteration's stage()
     }

@@ -70,6 +70,7 @@ class LayerShape:
     ln_eps: float = 1e-5
     d_conv: int = 0     # taps of the block's Conv1D in front of the layer (0: none)
     conv_silu: bool = False  # SiLU after the Conv1D (FV_FLAG_CONV_SILU)
+    keep_states: bool = False  # the forward keeps the scan states for the gradient (FV_FLAG_KEEP_STATES)
 
     @property
     def nd(self) -> int:
@@ -91,7 +92,8 @@ class LayerShape:
         a.K = self.K
         a.pool_scale = float(self.pool_scale)
         a.flags = ((nat.FV_FLAG_ZOH_EXACT if self.zoh_exact else 0) | _PATH_FLAGS[self.path] |
-                   (nat.FV_FLAG_LAYERNORM if self.ln else 0) | (nat.FV_FLAG_CONV_SILU if self.conv_silu else 0))
+                   (nat.FV_FLAG_LAYERNORM if self.ln else 0) | (nat.FV_FLAG_CONV_SILU if self.conv_silu else 0) |
+                   (nat.FV_FLAG_KEEP_STATES if self.keep_states else 0))
         a.x, a.z, a.A_log, a.D, a.W_x, a.W_dt, a.b_dt, a.keep_idx, a.y = (
             _ptr(x), _ptr(z), _ptr(A_log), _ptr(D), _ptr(W_x), _ptr(W_dt), _ptr(b_dt), _ptr(keep_idx), _ptr(y))
         a.ln_gamma, a.ln_beta = _ptr(ln_gamma), _ptr(ln_beta)
@@ -102,7 +104,8 @@ class LayerShape:
 
 
 def infer_shape(x, A_log, W_dt, pool_axis, dir_flags, keep_idx=None, h=None, w=None, pool_scale=1.0,
-                zoh_exact=False, path="auto", ln=False, ln_eps=1e-5, d_conv=0, conv_silu=False) -> LayerShape:
+                zoh_exact=False, path="auto", ln=False, ln_eps=1e-5, d_conv=0, conv_silu=False,
+                keep_states=False) -> LayerShape:
     nd, E, N = A_log.shape
     R = W_dt.shape[2]
     if keep_idx is None:
@@ -121,7 +124,7 @@ def infer_shape(x, A_log, W_dt, pool_axis, dir_flags, keep_idx=None, h=None, w=N
     if path not in _PATH_FLAGS:
         raise ValueError(f"path must be one of {sorted(_PATH_FLAGS)}")
     s = LayerShape(B, h, w, E, N, R, pool_axis, dir_flags, K, pool_scale, zoh_exact, path, bool(ln), float(ln_eps),
-                   int(d_conv), bool(conv_silu))
+                   int(d_conv), bool(conv_silu), bool(keep_states))
     if s.nd != nd:
         raise ValueError(f"dir_flags={dir_flags} enables {s.nd} directions, parameters stack {nd}")
     return s
@@ -158,10 +161,13 @@ def alloc_workspace(shape: LayerShape, device=None) -> torch.Tensor:
 
 def forward(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis=POOL_W, dir_flags=DIR_FWD | DIR_BWD, keep_idx=None,
             h=None, w=None, pool_scale=1.0, zoh_exact=False, y=None, workspace=None, stream=None, path="auto",
-            ln_gamma=None, ln_beta=None, ln_eps=1e-5, conv_w=None, conv_b=None, conv_silu=False):
+            ln_gamma=None, ln_beta=None, ln_eps=1e-5, conv_w=None, conv_b=None, conv_silu=False,
+            keep_states=False):
     """Queue the layer on ``stream`` (default: the current stream) and return y.  Passing
     ln_gamma and ln_beta ([E]) adds the post-SSM LayerNorm before the gate; conv_w [nd,E,d_conv]
-    and conv_b [nd,E] put the block's Conv1D in front (x is then the Conv1D's input)."""
+    and conv_b [nd,E] put the block's Conv1D in front (x is then the Conv1D's input).
+    keep_states=True also stores the scan states in the workspace for a later ``backward``
+    with keep_states=True (training)."""
     dev = x.device
     for name, t in (("x", x), ("z", z), ("A_log", A_log), ("D", D), ("W_x", W_x), ("W_dt", W_dt), ("b_dt", b_dt)):
         _check_tensor(name, t, torch.float32, dev)
@@ -181,7 +187,7 @@ def forward(x, z, A_log, D, W_x, W_dt, b_dt, pool_axis=POOL_W, dir_flags=DIR_FWD
         _check_tensor("conv_b", conv_b, torch.float32, dev)
         d_conv = conv_w.shape[-1]
     shape = infer_shape(x, A_log, W_dt, pool_axis, dir_flags, keep_idx, h, w, pool_scale, zoh_exact, path, ln, ln_eps,
-                        d_conv, conv_silu)
+                        d_conv, conv_silu, keep_states)
     if z.shape != x.shape:
         raise ValueError("z must have the shape of x")
     if y is None:
@@ -260,11 +266,11 @@ def _grads(dy, grads: dict) -> nat.FvSsmGrads:
 
 def backward(x, z, A_log, D, W_x, W_dt, b_dt, dy, fwd_workspace, pool_axis=POOL_W, dir_flags=DIR_FWD | DIR_BWD,
              keep_idx=None, h=None, w=None, pool_scale=1.0, zoh_exact=False, path="auto", grads=None,
-             workspace=None, stream=None, ln_gamma=None, ln_beta=None, ln_eps=1e-5) -> dict:
+             workspace=None, stream=None, ln_gamma=None, ln_beta=None, ln_eps=1e-5, keep_states=False) -> dict:
     """Queue the gradient of the layer for the upstream gradient dy on ``stream`` and return the
     dict {dx, dz, dA_log, dD, dW_x, dW_dt, db_dt} (+ dln_gamma, dln_beta with the post-SSM
     LayerNorm).  fwd_workspace is the workspace of a forward call with the same tensors and
-    options, queued earlier on the same stream."""
+    options (keep_states included), queued earlier on the same stream."""
     dev = x.device
     for name, t in (("x", x), ("z", z), ("A_log", A_log), ("D", D), ("W_x", W_x), ("W_dt", W_dt), ("b_dt", b_dt),
                     ("dy", dy)):
@@ -277,7 +283,8 @@ def backward(x, z, A_log, D, W_x, W_dt, b_dt, dy, fwd_workspace, pool_axis=POOL_
             raise ValueError("the LayerNorm needs both ln_gamma and ln_beta")
         _check_tensor("ln_gamma", ln_gamma, torch.float32, dev)
         _check_tensor("ln_beta", ln_beta, torch.float32, dev)
-    shape = infer_shape(x, A_log, W_dt, pool_axis, dir_flags, keep_idx, h, w, pool_scale, zoh_exact, path, ln, ln_eps)
+    shape = infer_shape(x, A_log, W_dt, pool_axis, dir_flags, keep_idx, h, w, pool_scale, zoh_exact, path, ln, ln_eps,
+                        keep_states=keep_states)
     if z.shape != x.shape or dy.shape != x.shape:
         raise ValueError("z and dy must have the shape of x")
     if grads is None:

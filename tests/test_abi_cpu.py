@@ -69,7 +69,7 @@ def test_status_strings(lib):
     assert nat.status_string(0) == "FV_OK"
     for s in range(1, 10):
         assert nat.status_string(s).startswith("FV_ERR_")
-    assert lib.fastvim_abi_version() == 5
+    assert lib.fastvim_abi_version() == 6
 
 
 # ---------------------------------------------------------------------------------------------
@@ -211,7 +211,7 @@ def test_layernorm_arguments(lib):
         assert validate(good_args(flags=LN, ln_gamma=g, ln_beta=b, ln_eps=eps)) == nat.FV_ERR_SHAPE
     assert validate(good_args(flags=LN, ln_gamma=g + 4, ln_beta=b, ln_eps=1e-5)) == nat.FV_ERR_ALIGN
     assert validate(good_args(flags=LN, ln_gamma=g, ln_beta=b, ln_eps=1e-5, E=4100)) == nat.FV_ERR_UNSUPPORTED
-    assert lib.fastvim_abi_version() == 5
+    assert lib.fastvim_abi_version() == 6
 
 
 def test_layernorm_launches(lib):
@@ -278,6 +278,35 @@ def test_delta_kernel_from_dt_rank_32(lib, masked, R):
         assert L.total_bytes >= L.delta + 2 * 3 * 6 * 64 * 4
     else:
         assert L.delta == 0
+
+
+@pytest.mark.parametrize("K", [0, 37])
+@pytest.mark.parametrize("flags", [2, 4])
+def test_kept_scan_states_layout(lib, K, flags):
+    """FV_FLAG_KEEP_STATES adds the scan states every 8 steps to the forward workspace
+    ([B][nd][2 ceil(T/16)][E][16] fp32, on either path) and drops the gradient's own copy; the
+    launches stay the same."""
+    if K and flags == 4:
+        flags = 0  # masked layers run staged
+    kw = dict(B=3, h=20, w=9, E=64, R=4, flags=flags)
+    if K:
+        kw.update(K=K, keep_idx=FAKE + (9 << 32))
+    a, ak = good_args(**kw), good_args(**dict(kw, flags=flags | nat.FV_FLAG_KEEP_STATES))
+    L, Lk = nat.FvWsLayout(), nat.FvWsLayout()
+    assert lib.fastvim_ssm_workspace_layout(ctypes.byref(a), ctypes.byref(L)) == nat.FV_OK
+    assert lib.fastvim_ssm_workspace_layout(ctypes.byref(ak), ctypes.byref(Lk)) == nat.FV_OK
+    T = 20
+    size = 3 * 2 * (2 * 2) * 64 * 16 * 4
+    assert L.ckpt == 0 and Lk.ckpt % 256 == 0 and Lk.ckpt >= Lk.ys + 3 * T * 64 * 4
+    assert Lk.total_bytes >= Lk.ckpt + size and Lk.total_bytes - L.total_bytes >= size
+    names = [lib.fastvim_ssm_launch_name(ctypes.byref(a), i) for i in range(lib.fastvim_ssm_launch_count(ctypes.byref(a)))]
+    assert names == [lib.fastvim_ssm_launch_name(ctypes.byref(ak), i)
+                     for i in range(lib.fastvim_ssm_launch_count(ctypes.byref(ak)))]
+    B, Bk = nat.FvBwdWsLayout(), nat.FvBwdWsLayout()
+    assert lib.fastvim_ssm_backward_workspace_layout(ctypes.byref(a), ctypes.byref(B)) == nat.FV_OK
+    assert lib.fastvim_ssm_backward_workspace_layout(ctypes.byref(ak), ctypes.byref(Bk)) == nat.FV_OK
+    assert B.ckpt > 0 and Bk.ckpt == 0 and B.total_bytes - Bk.total_bytes >= size
+    assert lib.fastvim_ssm_validate(ctypes.byref(good_args(**dict(kw, flags=flags | 128)))) == nat.FV_ERR_SHAPE
 
 
 # ---------------------------------------------------------------------------------------------

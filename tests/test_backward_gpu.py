@@ -7,6 +7,8 @@ the gradient tolerance (fv_testlib).  Shapes cover ragged channel blocks (E not 
 64), partial state groups (N < 16), pooled lengths below, at and across the 16-step checkpoint
 chunks, one or two directions, exact ZOH, pool_scale, the fused forward's workspace, masked
 layers with empty rows and a rejected id, and the empty batch."""
+import ctypes
+
 import numpy as np
 import pytest
 
@@ -14,7 +16,7 @@ torch = pytest.importorskip("torch")
 
 import oracle  # noqa: E402
 from fv_testlib import GRAD_PARAM_ABS_RMS, assert_close  # noqa: E402
-from pooled_selective_scan_b200 import inputs, ssm  # noqa: E402
+from pooled_selective_scan_b200 import _native as nat, inputs, ssm  # noqa: E402
 
 pytestmark = [pytest.mark.gpu, pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
 
@@ -42,19 +44,22 @@ def make_inputs(seed, B, h, w, E, N, R, nd, K=0, drop_row=None, pool_axis=0):
     return d
 
 
-def gpu_grads(d, pool_axis, dir_flags, h, w, pool_scale=1.0, zoh_exact=False, path="auto", ln_eps=1e-5):
-    """d may hold ln_gamma and ln_beta: then the layer has the post-SSM LayerNorm."""
+def gpu_grads(d, pool_axis, dir_flags, h, w, pool_scale=1.0, zoh_exact=False, path="auto", ln_eps=1e-5,
+              keep_states=False, out=None):
+    """d may hold ln_gamma and ln_beta: then the layer has the post-SSM LayerNorm.  out (a dict),
+    if given, receives y and both workspaces."""
     dev = torch.device("cuda")
     t = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev) for k, v in d.items()}
     keep = t.get("keep_idx")
     ln = "ln_gamma" in t
     shape = ssm.infer_shape(t["x"], t["A_log"], t["W_dt"], pool_axis, dir_flags, keep, h, w, pool_scale, zoh_exact,
-                            path, ln, ln_eps)
-    lnkw = dict(ln_gamma=t.get("ln_gamma"), ln_beta=t.get("ln_beta"), ln_eps=ln_eps)
+                            path, ln, ln_eps, keep_states=keep_states)
+    lnkw = dict(ln_gamma=t.get("ln_gamma"), ln_beta=t.get("ln_beta"), ln_eps=ln_eps, keep_states=keep_states)
     fws = ssm.alloc_workspace(shape, dev)
     fws.fill_(0xFF)
-    ssm.forward(t["x"], t["z"], t["A_log"], t["D"], t["W_x"], t["W_dt"], t["b_dt"], pool_axis, dir_flags,
-                keep_idx=keep, h=h, w=w, pool_scale=pool_scale, zoh_exact=zoh_exact, workspace=fws, path=path, **lnkw)
+    y = ssm.forward(t["x"], t["z"], t["A_log"], t["D"], t["W_x"], t["W_dt"], t["b_dt"], pool_axis, dir_flags,
+                    keep_idx=keep, h=h, w=w, pool_scale=pool_scale, zoh_exact=zoh_exact, workspace=fws, path=path,
+                    **lnkw)
     fstatus = ssm.device_status(fws)
     bws = torch.full((max(ssm.backward_workspace_size(shape), 256),), 0xFF, dtype=torch.uint8, device=dev)
     grads = {"dx": torch.full_like(t["x"], float("nan")), "dz": torch.full_like(t["z"], float("nan"))}
@@ -64,6 +69,8 @@ def gpu_grads(d, pool_axis, dir_flags, h, w, pool_scale=1.0, zoh_exact=False, pa
                  dir_flags, keep_idx=keep, h=h, w=w, pool_scale=pool_scale, zoh_exact=zoh_exact, path=path,
                  grads=grads, workspace=bws, **lnkw)
     torch.cuda.synchronize()
+    if out is not None:
+        out.update(y=y.cpu().numpy(), fws=fws, bws=bws, shape=shape)
     return {k: v.cpu().numpy() for k, v in grads.items()}, fstatus, ssm.backward_launch_names(shape)
 
 
@@ -204,3 +211,54 @@ def test_layernorm_gradient(case):
     assert fst == 0 and names[0] == ("bwd_ln_gate_reg_kernel" if E <= 2048 else "bwd_ln_gate_kernel")
     ref = oracle_grads(d, axis, 3, h, w)
     compare(got, ref, f"layernorm {case}")
+
+
+KEEP_CASES = [
+    # B, h, w, E, N, R, pool_axis, dir_flags, zoh_exact, path, K
+    (2, 40, 3, 132, 16, 7, 0, 3, False, "staged", 0),    # T = 40: two whole chunks, then 8 steps
+    (3, 13, 7, 68, 5, 3, 1, 2, True, "staged", 0),       # T = 7 < 8, one direction, exact ZOH, N = 5
+    (2, 64, 64, 1024, 16, 64, 0, 3, False, "fused", 0),  # the fused launch keeps the states
+    (2, 64, 64, 1024, 16, 64, 0, 3, False, "staged", 0),  # step sizes from the dt_proj kernel
+    (2, 16, 16, 132, 16, 8, 1, 3, False, "auto", 100),   # masked
+]
+
+
+@pytest.mark.parametrize("case", KEEP_CASES, ids=lambda c: "x".join(map(str, c[:6])) + f"-{c[9]}K{c[10]}")
+def test_gradient_from_kept_states(case):
+    """FV_FLAG_KEEP_STATES: the forward stores the scan states every 8 steps and the gradient reads
+    them instead of running the recurrences a first time.  y keeps its bits, the gradient matches
+    the oracle, and the kept states match the ones the gradient computes itself without the flag
+    (slots of chunks shorter than 8 steps are never written)."""
+    B, h, w, E, N, R, axis, dirs, zoh, path, K = case
+    nd = bin(dirs).count("1")
+    d = make_inputs(23, B, h, w, E, N, R, nd, K=K)
+    kept, plain = {}, {}
+    got, fst, names = gpu_grads(d, axis, dirs, h, w, 1.0, zoh, path, keep_states=True, out=kept)
+    _, fst0, names0 = gpu_grads(d, axis, dirs, h, w, 1.0, zoh, path, out=plain)
+    assert fst == 0 and fst0 == 0 and names == names0
+    np.testing.assert_array_equal(kept["y"], plain["y"])
+    compare(got, oracle_grads(d, axis, dirs, h, w, 1.0, zoh), f"kept states {case}")
+    # the states themselves: forward's (kept) against the gradient call's own pass
+    T = h if axis == 0 else w
+    nck = 2 * (-(-T // 16))
+    L = nat.FvWsLayout()
+    a = kept["shape"].args()
+    assert nat.lib().fastvim_ssm_workspace_layout(ctypes.byref(a), ctypes.byref(L)) == nat.FV_OK
+    Lb = nat.FvBwdWsLayout()
+    a0 = plain["shape"].args()
+    assert nat.lib().fastvim_ssm_backward_workspace_layout(ctypes.byref(a0), ctypes.byref(Lb)) == nat.FV_OK
+    n = B * nd * nck * E * 16
+    fk = kept["fws"][L.ckpt:L.ckpt + 4 * n].view(torch.float32).cpu().numpy().reshape(B, nd, nck, E, 16)
+    bk = plain["bws"][Lb.ckpt:Lb.ckpt + 4 * n].view(torch.float32).cpu().numpy().reshape(B, nd, nck, E, 16)
+    fwd_slot = [k == 0 if nd == 2 else bool(dirs & 1) for k in range(nd)]
+    for k in range(nd):
+        for c in range(nck):
+            it = c // 2
+            ci = it if fwd_slot[k] else nck // 2 - 1 - it
+            if c % 2 == 1 and min(16, T - 16 * ci) <= 8:
+                continue  # no second half in this chunk
+            assert not np.isnan(fk[:, k, c]).any()
+            assert_close(fk[:, k, c], bk[:, k, c], f"states dir {k} slot {c}")
+            if c == 0:
+                assert not fk[:, k, c].any()  # every scan starts from zero
+            assert not fk[:, k, c, :, N:].any()  # states past N stay zero
