@@ -1177,9 +1177,10 @@ fv_status backward_impl(const fv_ssm_args* args, const fv_ssm_grads* g, const vo
     } else {
         const int32_t* row_off = (const int32_t*)(fw + FL.row_off);
         const int32_t* row_tok = (const int32_t*)(fw + FL.row_tok);
-        const int grid = gate_blocks = resident(fv::bwd_gate_masked_kernel, fv::kThreads);
+        const int threads = fv::bwd_mgroups(sh.SL) * fv::bwd_mslot_width(sh.SL);
+        const int grid = gate_blocks = resident(fv::bwd_gate_masked_kernel, threads);
         FV_MARK_CALL(marks, st, ([&]() -> fv_status {
-            fv::bwd_gate_masked_kernel<<<grid, fv::kThreads, 0, st>>>(sh, a->x, a->z, g->dy, ys, a->D, row_off, row_tok,
+            fv::bwd_gate_masked_kernel<<<grid, threads, 0, st>>>(sh, a->x, a->z, g->dy, ys, a->D, row_off, row_tok,
                                                                        g->dx, g->dz, dys, part_gate);
             FV_LAUNCH_CHECK("bwd_gate_masked_kernel");
             return FV_OK;

@@ -173,58 +173,82 @@ bwd_gate_dense_kernel(Shape sh, const float* __restrict__ x, const float* __rest
     }
 }
 
+// Masked layers: slots per pass and token groups, block = bwd_mgroups(SL) * bwd_mslot_width(SL)
+// threads (<= 512): up to 512 slots in one pass (every thread busy at E = 1536), several token
+// groups for narrow rows (SL <= 128), passes of 256 slots above 512.
+__host__ __device__ __forceinline__ int bwd_mslot_width(int SL) { return SL <= 2 * kThreads ? SL : kThreads; }
+__host__ __device__ __forceinline__ int bwd_mgroups(int SL) { return SL <= kThreads / 2 ? kThreads / SL : 1; }
+
 // Masked gate gradient, persistent over pooled rows (b, t): the row's kept tokens come from the
-// forward's row lists (row_off, row_tok).  A row without tokens gets dys = 0.  Tokens whose id was
-// rejected are in no row; bwd_pool_masked_kernel zeroes their dx and dz.
-__global__ void __launch_bounds__(kThreads)
+// forward's row lists (row_off, row_tok); token group g takes the row's tokens g, g + G, .. (two
+// in flight, six 128-bit loads).  dys of the row is the groups' sums added in group order (zero
+// for a row without tokens), and the block's dD sums go to row blockIdx.x of part_dD.  Tokens
+// whose id was rejected are in no row; bwd_pool_masked_kernel zeroes their dx and dz.
+__global__ void __launch_bounds__(2 * kThreads)
 bwd_gate_masked_kernel(Shape sh, const float* __restrict__ x, const float* __restrict__ z,
                        const float* __restrict__ dy, const float* __restrict__ ys, const float* __restrict__ D,
                        const int32_t* __restrict__ row_off, const int32_t* __restrict__ row_tok,
                        float* __restrict__ dx, float* __restrict__ dz, float* __restrict__ dys,
                        float* __restrict__ part_dD) {
+    __shared__ float4 part[kThreads];  // the groups' sums (G > 1 only: then G SW <= 256)
     const int SL = sh.SL, K = sh.K, T = sh.T;
+    const int SW = bwd_mslot_width(SL), G = bwd_mgroups(SL);
+    const int ls = threadIdx.x % SW, g = threadIdx.x / SW;
     const int rows = sh.B * T;
     const float4* x4 = reinterpret_cast<const float4*>(x);
     const float4* z4 = reinterpret_cast<const float4*>(z);
     const float4* g4 = reinterpret_cast<const float4*>(dy);
     float4* dx4 = reinterpret_cast<float4*>(dx);
     float4* dz4 = reinterpret_cast<float4*>(dz);
-    for (int s0 = 0; s0 < SL; s0 += kThreads) {
-        const int slot = s0 + threadIdx.x;
-        const bool act = slot < SL;
+    // the sum over the groups of v, in group order, to group 0 (G > 1; all threads take part)
+    auto group_sum = [&](const float4& v) {
+        part[threadIdx.x] = v;
+        __syncthreads();
+        float4 sum = part[ls];
+        for (int q = 1; q < G; ++q) f4_add(sum, part[q * SW + ls]);
+        __syncthreads();
+        return sum;
+    };
+    for (int s0 = 0; s0 < SL; s0 += SW) {
+        const int slot = s0 + ls;
+        const bool act = g < G && slot < SL;
         const float4 Ds = act ? bwd_dsum4(D, sh.nd, SL, slot) : f4_zero();
         float4 dDa = f4_zero();
         for (int bt = blockIdx.x; bt < rows; bt += gridDim.x) {
-            if (!act) continue;
-            const int b = bt / T, t = bt - b * T;
-            const int p0 = row_off[(size_t)b * (T + 1) + t], p1 = row_off[(size_t)b * (T + 1) + t + 1];
-            const int32_t* tok = row_tok + (size_t)b * K;
-            const float4 yv = reinterpret_cast<const float4*>(ys + (size_t)bt * sh.E)[slot];
             float4 acc = f4_zero();
-            int p = p0;
-            for (; p + 1 < p1; p += 2) {  // two tokens, six loads in flight
-                const size_t o0 = ((size_t)b * K + tok[p]) * SL + slot;
-                const size_t o1 = ((size_t)b * K + tok[p + 1]) * SL + slot;
-                const float4 xa = ld_stream(x4 + o0), za = ld_stream(z4 + o0), ga = ld_stream(g4 + o0);
-                const float4 xb = ld_stream(x4 + o1), zb = ld_stream(z4 + o1), gb = ld_stream(g4 + o1);
-                float4 dzv, dxv;
-                gate_grad4(xa, za, ga, yv, Ds, dzv, dxv, acc, dDa);
-                st_stream(dz4 + o0, dzv);
-                st_stream(dx4 + o0, dxv);
-                gate_grad4(xb, zb, gb, yv, Ds, dzv, dxv, acc, dDa);
-                st_stream(dz4 + o1, dzv);
-                st_stream(dx4 + o1, dxv);
+            if (act) {
+                const int b = bt / T, t = bt - b * T;
+                const int p0 = row_off[(size_t)b * (T + 1) + t], p1 = row_off[(size_t)b * (T + 1) + t + 1];
+                const int32_t* tok = row_tok + (size_t)b * K;
+                const float4 yv = reinterpret_cast<const float4*>(ys + (size_t)bt * sh.E)[slot];
+                int p = p0 + g;
+                for (; p + G < p1; p += 2 * G) {  // two tokens, six loads in flight
+                    const size_t o0 = ((size_t)b * K + tok[p]) * SL + slot;
+                    const size_t o1 = ((size_t)b * K + tok[p + G]) * SL + slot;
+                    const float4 xa = ld_stream(x4 + o0), za = ld_stream(z4 + o0), ga = ld_stream(g4 + o0);
+                    const float4 xb = ld_stream(x4 + o1), zb = ld_stream(z4 + o1), gb = ld_stream(g4 + o1);
+                    float4 dzv, dxv;
+                    gate_grad4(xa, za, ga, yv, Ds, dzv, dxv, acc, dDa);
+                    st_stream(dz4 + o0, dzv);
+                    st_stream(dx4 + o0, dxv);
+                    gate_grad4(xb, zb, gb, yv, Ds, dzv, dxv, acc, dDa);
+                    st_stream(dz4 + o1, dzv);
+                    st_stream(dx4 + o1, dxv);
+                }
+                if (p < p1) {
+                    const size_t o = ((size_t)b * K + tok[p]) * SL + slot;
+                    float4 dzv, dxv;
+                    gate_grad4(ld_stream(x4 + o), ld_stream(z4 + o), ld_stream(g4 + o), yv, Ds, dzv, dxv, acc, dDa);
+                    st_stream(dz4 + o, dzv);
+                    st_stream(dx4 + o, dxv);
+                }
             }
-            if (p < p1) {
-                const size_t o = ((size_t)b * K + tok[p]) * SL + slot;
-                float4 dzv, dxv;
-                gate_grad4(ld_stream(x4 + o), ld_stream(z4 + o), ld_stream(g4 + o), yv, Ds, dzv, dxv, acc, dDa);
-                st_stream(dz4 + o, dzv);
-                st_stream(dx4 + o, dxv);
-            }
-            reinterpret_cast<float4*>(dys + (size_t)bt * sh.E)[slot] = acc;
+            if (G > 1) acc = group_sum(acc);
+            if (g == 0 && slot < SL) reinterpret_cast<float4*>(dys + (size_t)bt * sh.E)[slot] = acc;
         }
-        if (act) reinterpret_cast<float4*>(part_dD + (size_t)blockIdx.x * sh.E)[slot] = dDa;  // this block's sums
+        if (G > 1) dDa = group_sum(dDa);
+        if (g == 0 && slot < SL)  // this block's sums
+            reinterpret_cast<float4*>(part_dD + (size_t)blockIdx.x * sh.E)[slot] = dDa;
     }
 }
 
