@@ -833,6 +833,8 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
                 if (ii < hl) {
                     const float dt = sdl[i * kBsCh + c], xv = sx[i * kBsCh + c], gy = sdy[i * kBsCh + c];
                     float ddt = 0.f, dxb = 0.f, vals[8];
+                    const float dtx = dt * xv;
+                    float lb = 0.f;  // Euler: sum_j lam_j B_j, the shared factor of dDelta and dxbar
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const float Bn = sbc[i * 32 + 4 * q + j], Cn = sbc[i * 32 + 16 + 4 * q + j];
@@ -851,11 +853,14 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
                             vals[j] = lam[j] * cf * xv;
                             dxb = fmaf(lam[j] * cf, Bn, dxb);
                         } else {
-                            ddt = fmaf(lam[j], Bn * xv, ddt);
-                            vals[j] = lam[j] * dt * xv;
-                            dxb = fmaf(lam[j] * dt, Bn, dxb);
+                            lb = fmaf(lam[j], Bn, lb);
+                            vals[j] = lam[j] * dtx;
                         }
                         Anext[j] = Ab;
+                    }
+                    if (!ZOH_EXACT) {  // dDelta += xbar sum_j lam_j B_j;  dxbar = Delta sum_j lam_j B_j
+                        ddt = fmaf(xv, lb, ddt);
+                        dxb = dt * lb;
                     }
                     ddt += __shfl_xor_sync(0xffffffffu, ddt, 1);
                     ddt += __shfl_xor_sync(0xffffffffu, ddt, 2);
@@ -916,26 +921,42 @@ bwd_scan_kernel(Shape sh, const float* __restrict__ u, const float* __restrict__
             }
             pdu[u_offset(sh, k, b, t_of(it, s)) + r] = (a0 + a1) + (a2 + a3);
         }
-        // dW_dt | db_dt partial sums over the chunk's steps: thread = (channel, 4 entries of the
-        // row; the last group is the bias), dt_low read as float4
+        // dW_dt | db_dt partial sums over the chunk's steps: thread = (4 channels, 4 entries of
+        // their rows; the last group is the bias), dv and dt_low read as float4: 16 FMA per pair
+        // of loads
         const int ng = R4 / 4 + 1;
-        for (int i = tid; i < kBsCh * ng; i += kBsThreads) {
-            const int cc = i / ng, g = i - cc * ng;
-            float4* a = reinterpret_cast<float4*>(swacc + cc * WA + 4 * g);
-            float4 acc = *a;
+        for (int i = tid; i < (kBsCh / 4) * ng; i += kBsThreads) {
+            const int cq = i / ng, g = i - cq * ng;
+            float4* a = reinterpret_cast<float4*>(swacc + 4 * cq * WA + 4 * g);  // rows 4 cq .. 4 cq + 3
+            const int aw = WA / 4;
             if (g < R4 / 4) {
+                float4 acc[4] = {a[0], a[aw], a[2 * aw], a[3 * aw]};
                 for (int s = 0; s < len; ++s) {
-                    const float dv = sdv[s * kBsCh + cc];
+                    const float4 dv = *reinterpret_cast<const float4*>(sdv + s * kBsCh + 4 * cq);
                     const float4 d = *reinterpret_cast<const float4*>(sdtl + s * R4 + 4 * g);
-                    acc.x = fmaf(dv, d.x, acc.x);
-                    acc.y = fmaf(dv, d.y, acc.y);
-                    acc.z = fmaf(dv, d.z, acc.z);
-                    acc.w = fmaf(dv, d.w, acc.w);
+                    const float dvs[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        acc[m].x = fmaf(dvs[m], d.x, acc[m].x);
+                        acc[m].y = fmaf(dvs[m], d.y, acc[m].y);
+                        acc[m].z = fmaf(dvs[m], d.z, acc[m].z);
+                        acc[m].w = fmaf(dvs[m], d.w, acc[m].w);
+                    }
                 }
-            } else {
-                for (int s = 0; s < len; ++s) acc.x += sdv[s * kBsCh + cc];
+#pragma unroll
+                for (int m = 0; m < 4; ++m) a[m * aw] = acc[m];
+            } else {  // the bias entries (column R4) of the 4 rows
+                float bs[4] = {a[0].x, a[aw].x, a[2 * aw].x, a[3 * aw].x};
+                for (int s = 0; s < len; ++s) {
+                    const float4 dv = *reinterpret_cast<const float4*>(sdv + s * kBsCh + 4 * cq);
+                    bs[0] += dv.x;
+                    bs[1] += dv.y;
+                    bs[2] += dv.z;
+                    bs[3] += dv.w;
+                }
+#pragma unroll
+                for (int m = 0; m < 4; ++m) a[m * aw].x = bs[m];
             }
-            *a = acc;
         }
         __syncthreads();  // the buffers are refilled by the next stage(s)
     }
