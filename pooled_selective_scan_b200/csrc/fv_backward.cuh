@@ -587,6 +587,16 @@ bwd_ln_gate_reg_kernel(Shape sh, const float* __restrict__ x, const float* __res
                     gv[u] = own[u] ? ld_stream(gy4 + o + gt + G * u) : f4_zero();
                 }
                 x0 = __ldg(x + o * 4);
+                if (i + NG < ntok) {  // the group's next token: into L2 while this one is processed
+                    const size_t on2 = tok_off(i + NG);
+#pragma unroll
+                    for (int u = 0; u < U; ++u)
+                        if (own[u]) {
+                            prefetch_l2(x4 + on2 + gt + G * u);
+                            prefetch_l2(z4 + on2 + gt + G * u);
+                            prefetch_l2(gy4 + on2 + gt + G * u);
+                        }
+                }
             }
             // pass 1: s and its moments about the token's first s value (the same in every thread)
             const float Ks = fmaf(dsum[0].x, x0, y0);

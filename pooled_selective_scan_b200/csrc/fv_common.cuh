@@ -199,6 +199,8 @@ __device__ __forceinline__ void cp_async4z(void* dst, const void* src, bool vali
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;"
                  : : "r"(smem_u32(dst)), "l"(src), "r"(valid ? 4u : 0u) : "memory");
 }
+// Bring the line holding p into L2 (no register, no wait).
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" : : "l"(p)); }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" : : : "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" : : "n"(N) : "memory"); }
