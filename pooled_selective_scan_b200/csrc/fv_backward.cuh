@@ -418,12 +418,11 @@ bwd_ln_gate_kernel(Shape sh, const float* __restrict__ x, const float* __restric
 // The same gradient with each token's values in registers.  A group of WPT warps takes one token
 // (thread gt of the group owns float4 slots gt + 32 WPT u, u < U: E <= 128 U WPT); a
 // block of NG groups is persistent over pooled rows, its groups taking the row's tokens in turn.
-// Per token: x, z and dy are loaded at once (U = 2), or (U = 1) arrive through the group's
-// shared-memory double buffer, the next token's copies in flight while this one is processed
-// (each thread copies and reads back only its own slots, so no barrier guards it; measured on
-// B200 it pays at U = 1, E = 768: 0.60 -> 0.66 of the copy rate, and costs at U = 2, E = 384 and
-// 1,536: 0.71 -> 0.69, 0.56 -> 0.54); pass 1 forms s and its shifted moments, pass 2 the two
-// means of gs, pass 3 writes dz, dx from the registers.  The group's sums (moments, means) go
+// Per token: x, z and dy are loaded at once (one memory round trip), and the group's next token
+// is prefetched into L2 meanwhile, so that its loads hit L2 (measured on B200: 0.71 -> 0.82 of the
+// copy rate at E = 384, 0.66 -> 0.75 at E = 768 against a shared-memory double buffer of the next
+// token, 0.56 -> 0.65 at E = 1,536; prefetching two tokens ahead measured slower); pass 1 forms s
+// and its shifted moments, pass 2 the two means of gs, pass 3 writes dz, dx from the registers.  The group's sums (moments, means) go
 // through a shared-memory slot per warp, added in warp order behind a named barrier of the group.
 // dys of the current row and the batch sums of dgamma, dbeta, dD stay in each thread's registers;
 // the groups' dys meet in shared memory at the end of each row, the batch sums at the end of the
@@ -446,8 +445,6 @@ __host__ __device__ __forceinline__ int bwd_lnr_groups(int SL) {
 __host__ __device__ __forceinline__ size_t bwd_lnr_smem_bytes(int SL) {
     const int ng = bwd_lnr_groups(SL), wpt = bwd_lnr_wpt(SL);
     return (size_t)(3 + ng) * SL * sizeof(float4)                // sum D, gamma, beta; the groups' rows
-           + (bwd_lnr_nsl(SL) == 1 ? (size_t)ng * 6 * SL * sizeof(float4) : 0)  // U = 1: x, z, dy of two
-                                                                                  // tokens per group
            + (size_t)ng * wpt * 4 * sizeof(float);               // the warps' partial sums
 }
 __device__ __forceinline__ void group_bar(int id, int threads) {
@@ -470,9 +467,7 @@ bwd_ln_gate_reg_kernel(Shape sh, const float* __restrict__ x, const float* __res
     float4* g4 = dsum + SL;
     float4* be4 = g4 + SL;
     float4* rows = be4 + SL;                                    // [NG][SL]
-    constexpr bool PF = U == 1;                                 // the double buffer (see above)
-    float4* stg = rows + (size_t)NG * SL + (size_t)grp * 6 * SL;  // PF: this group's [2 tokens][x | z | dy][SL]
-    float* red = reinterpret_cast<float*>(rows + (size_t)NG * (PF ? 7 : 1) * SL) + (size_t)grp * WPT * 4;  // [WPT][4]
+    float* red = reinterpret_cast<float*>(rows + (size_t)NG * SL) + (size_t)grp * WPT * 4;  // [WPT][4]
     for (int slot = threadIdx.x; slot < SL; slot += blockDim.x) {
         dsum[slot] = bwd_dsum4(D, sh.nd, SL, slot);
         g4[slot] = __ldg(reinterpret_cast<const float4*>(gamma) + slot);
@@ -534,69 +529,31 @@ bwd_ln_gate_reg_kernel(Shape sh, const float* __restrict__ x, const float* __res
             acc_y[u] = f4_zero();
         }
         const float y0 = __ldg(ys + (size_t)bt * sh.E);
-        // token i of the row: its float4 offset; the copies of its thread-owned slots into buffer buf
+        // token i of the row: its float4 offset
         auto tok_off = [&](int i) -> size_t {
             return MASKED ? ((size_t)b * K + row_tok[(size_t)b * K + p0 + i]) * SL
                           : (dense_base(sh, b, t) >> 2) + (size_t)i * st4;
         };
-        auto fetch = [&](size_t to, int buf) {
-            float4* sb = stg + (size_t)buf * 3 * SL;
+        for (int i = grp; live && i < ntok; i += NG) {
+            const size_t o = tok_off(i);
+            // every load of the token at once (one memory round trip per token)
+            float4 xv[U], zv[U], gv[U], sv[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                if (!own[u]) continue;
-                const int slot = gt + G * u;
-                cp_async16(sb + slot, x4 + to + slot, 16u);
-                cp_async16(sb + SL + slot, z4 + to + slot, 16u);
-                cp_async16(sb + 2 * SL + slot, gy4 + to + slot, 16u);
+                xv[u] = own[u] ? ld_stream(x4 + o + gt + G * u) : f4_zero();
+                zv[u] = own[u] ? ld_stream(z4 + o + gt + G * u) : f4_zero();
+                gv[u] = own[u] ? ld_stream(gy4 + o + gt + G * u) : f4_zero();
             }
-            cp_async_commit();
-        };
-        size_t o = 0;
-        float x0 = 0.f;  // x of the token's first channel (the shift of its moments)
-        if (PF && live && grp < ntok) {
-            o = tok_off(grp);
-            fetch(o, 0);
-            x0 = __ldg(x + o * 4);
-        }
-        for (int i = grp, it = 0; live && i < ntok; i += NG, ++it) {
-            size_t on = 0;
-            float x0n = 0.f;
-            float4 xv[U], zv[U], gv[U], sv[U];
-            if constexpr (PF) {
-                if (i + NG < ntok) {  // the group's next token: its copies fly during this one
-                    on = tok_off(i + NG);
-                    fetch(on, (it + 1) & 1);
-                    x0n = __ldg(x + on * 4);
-                    cp_async_wait<1>();
-                } else {
-                    cp_async_wait<0>();
-                }
-                const float4* sb = stg + (size_t)(it & 1) * 3 * SL;
+            const float x0 = __ldg(x + o * 4);  // x of the token's first channel (the shift of its moments)
+            if (i + NG < ntok) {  // the group's next token: into L2 while this one is processed
+                const size_t on = tok_off(i + NG);
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    xv[u] = own[u] ? sb[gt + G * u] : f4_zero();
-                    zv[u] = own[u] ? sb[SL + gt + G * u] : f4_zero();
-                    gv[u] = own[u] ? sb[2 * SL + gt + G * u] : f4_zero();
-                }
-            } else {  // every load of the token at once (one memory round trip per token)
-                o = tok_off(i);
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    xv[u] = own[u] ? ld_stream(x4 + o + gt + G * u) : f4_zero();
-                    zv[u] = own[u] ? ld_stream(z4 + o + gt + G * u) : f4_zero();
-                    gv[u] = own[u] ? ld_stream(gy4 + o + gt + G * u) : f4_zero();
-                }
-                x0 = __ldg(x + o * 4);
-                if (i + NG < ntok) {  // the group's next token: into L2 while this one is processed
-                    const size_t on2 = tok_off(i + NG);
-#pragma unroll
-                    for (int u = 0; u < U; ++u)
-                        if (own[u]) {
-                            prefetch_l2(x4 + on2 + gt + G * u);
-                            prefetch_l2(z4 + on2 + gt + G * u);
-                            prefetch_l2(gy4 + on2 + gt + G * u);
-                        }
-                }
+                for (int u = 0; u < U; ++u)
+                    if (own[u]) {
+                        prefetch_l2(x4 + on + gt + G * u);
+                        prefetch_l2(z4 + on + gt + G * u);
+                        prefetch_l2(gy4 + on + gt + G * u);
+                    }
             }
             // pass 1: s and its moments about the token's first s value (the same in every thread)
             const float Ks = fmaf(dsum[0].x, x0, y0);
@@ -658,10 +615,6 @@ bwd_ln_gate_reg_kernel(Shape sh, const float* __restrict__ x, const float* __res
                 f4_add(acc_g[u], make_float4(dno[0] * sho[0], dno[1] * sho[1], dno[2] * sho[2], dno[3] * sho[3]));
                 f4_add(acc_b[u], make_float4(dno[0], dno[1], dno[2], dno[3]));
                 f4_add(acc_d[u], make_float4(dso[0] * xa[0], dso[1] * xa[1], dso[2] * xa[2], dso[3] * xa[3]));
-            }
-            if (PF) {
-                o = on;
-                x0 = x0n;
             }
         }
         // dys of the row: the groups' sums, added in group order
