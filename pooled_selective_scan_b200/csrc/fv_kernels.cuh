@@ -160,7 +160,7 @@ mask_bucket_kernel(Shape sh, const int32_t* __restrict__ keep_idx, int32_t* row_
 // threads split the row's tokens; wider rows: one thread per slot (launched with SL threads
 // rounded up to whole warps, up to 1024), so no thread takes two slots while others take one.
 constexpr int kMaskPoolMaxThreads = 1024;
-__global__ void __launch_bounds__(kMaskPoolMaxThreads)
+__global__ void __launch_bounds__(kMaskPoolMaxThreads, 2)
 mask_pool_kernel(Shape sh, const float* __restrict__ x, const int32_t* __restrict__ row_off,
                  const int32_t* __restrict__ row_tok, float* __restrict__ xbar) {
     __shared__ float4 part[kThreads];
@@ -188,17 +188,16 @@ mask_pool_kernel(Shape sh, const float* __restrict__ x, const int32_t* __restric
         }
     } else {
         for (int slot = threadIdx.x; slot < SL; slot += blockDim.x) {
-            float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
+            float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f);
             int p = p0;
-            for (; p + 3 < p1; p += 4) {  // four kept tokens in flight
+            for (; p + 3 < p1; p += 4) {  // four kept tokens in flight, added in kept order
                 const float4 v0 = ld_stream(xb + (size_t)tok[p] * SL + slot);
                 const float4 v1 = ld_stream(xb + (size_t)tok[p + 1] * SL + slot);
                 const float4 v2 = ld_stream(xb + (size_t)tok[p + 2] * SL + slot);
                 const float4 v3 = ld_stream(xb + (size_t)tok[p + 3] * SL + slot);
-                f4_add(a0, v0); f4_add(a1, v1); f4_add(a2, v2); f4_add(a3, v3);
+                f4_add(a0, v0); f4_add(a0, v1); f4_add(a0, v2); f4_add(a0, v3);
             }
             for (; p < p1; ++p) f4_add(a0, ld_stream(xb + (size_t)tok[p] * SL + slot));
-            f4_add(a0, a1); f4_add(a2, a3); f4_add(a0, a2);
             out[slot] = f4_scale(a0, scale);
         }
     }
