@@ -43,7 +43,8 @@ def valid_layer(draw):
     a.flags = (draw(st.sampled_from([0, nat.FV_FLAG_PATH_STAGED, nat.FV_FLAG_PATH_FUSED]))
                | draw(st.sampled_from([0, nat.FV_FLAG_ZOH_EXACT]))
                | draw(st.sampled_from([0, nat.FV_FLAG_TRACE]))
-               | draw(st.sampled_from([0, nat.FV_FLAG_LAYERNORM])))
+               | draw(st.sampled_from([0, nat.FV_FLAG_LAYERNORM]))
+               | draw(st.sampled_from([0, nat.FV_FLAG_KEEP_STATES])))
     for i, name in enumerate(PTRS):
         setattr(a, name, FAKE + i * SLOT)
     if a.K:
@@ -66,6 +67,7 @@ BREAKS = [
     ("both paths forced", lambda a: True,
      _set("flags", lambda a: a.flags | nat.FV_FLAG_PATH_STAGED | nat.FV_FLAG_PATH_FUSED), nat.FV_ERR_SHAPE),
     ("unknown flag", lambda a: True, _set("flags", lambda a: a.flags | 32), nat.FV_ERR_SHAPE),
+    ("undefined flag bit", lambda a: True, _set("flags", lambda a: a.flags | 128), nat.FV_ERR_SHAPE),
     ("negative batch", lambda a: True, _set("B", -1), nat.FV_ERR_SHAPE),
     ("K above the grid", lambda a: True, _set("K", lambda a: a.h * a.w + 1), nat.FV_ERR_SHAPE),
     ("NaN pool scale", lambda a: True, _set("pool_scale", float("nan")), nat.FV_ERR_SHAPE),
@@ -108,6 +110,10 @@ def _check_layout(lib, a):
     if L.delta:  # the staged path's step sizes (dt_rank >= 32)
         assert a.R >= 32
         regions.append((L.delta, L.nd * B * T * E * 4))
+    # the scan states kept for the gradient: exactly with FV_FLAG_KEEP_STATES
+    assert (L.ckpt != 0) == bool(a.flags & nat.FV_FLAG_KEEP_STATES)
+    if L.ckpt:
+        regions.append((L.ckpt, B * L.nd * 2 * -(-T // 16) * E * 16 * 4))
     regions.sort()
     end = 0
     for off, n in regions:
@@ -213,8 +219,11 @@ def test_gradient_validation_and_plan(a, pick):
     nd = bin(a.dir_flags).count("1")
     ub = -(-T * (a.R + 2 * a.N) // 32) * 32
     bte = a.B * T * a.E * 4
-    regions = [(L.status, 8), (L.dys, bte), (L.dxbar, bte), (L.du, nd * a.B * ub * 4), (L.dxs, nd * bte),
-               (L.ckpt, a.B * nd * 2 * -(-T // 16) * a.E * 16 * 4)]
+    regions = [(L.status, 8), (L.dys, bte), (L.dxbar, bte), (L.du, nd * a.B * ub * 4), (L.dxs, nd * bte)]
+    # the scan states live in exactly one of the workspaces: the forward's with FV_FLAG_KEEP_STATES
+    assert (L.ckpt == 0) == bool(a.flags & nat.FV_FLAG_KEEP_STATES)
+    if L.ckpt:
+        regions.append((L.ckpt, a.B * nd * 2 * -(-T // 16) * a.E * 16 * 4))
     FL = nat.FvWsLayout()
     assert lib.fastvim_ssm_workspace_layout(ctypes.byref(a), ctypes.byref(FL)) == nat.FV_OK
     assert (L.delta == 0) == (FL.delta != 0)  # the step sizes live in exactly one of the workspaces
