@@ -174,9 +174,10 @@ bwd_gate_dense_kernel(Shape sh, const float* __restrict__ x, const float* __rest
 }
 
 // Masked layers: slots per pass and token groups, block = bwd_mgroups(SL) * bwd_mslot_width(SL)
-// threads (<= 512): up to 512 slots in one pass (every thread busy at E = 1536), several token
-// groups for narrow rows (SL <= 128), passes of 256 slots above 512.
-__host__ __device__ __forceinline__ int bwd_mslot_width(int SL) { return SL <= 2 * kThreads ? SL : kThreads; }
+// threads (<= 384): up to 384 slots in one pass (every thread busy at E = 1536; 56 registers,
+// three blocks per SM), several token groups for narrow rows (SL <= 128), passes of 256 slots
+// above 384.
+__host__ __device__ __forceinline__ int bwd_mslot_width(int SL) { return SL <= 3 * kThreads / 2 ? SL : kThreads; }
 __host__ __device__ __forceinline__ int bwd_mgroups(int SL) { return SL <= kThreads / 2 ? kThreads / SL : 1; }
 
 // Masked gate gradient, persistent over pooled rows (b, t): the row's kept tokens come from the
@@ -184,7 +185,7 @@ __host__ __device__ __forceinline__ int bwd_mgroups(int SL) { return SL <= kThre
 // in flight, six 128-bit loads).  dys of the row is the groups' sums added in group order (zero
 // for a row without tokens), and the block's dD sums go to row blockIdx.x of part_dD.  Tokens
 // whose id was rejected are in no row; bwd_pool_masked_kernel zeroes their dx and dz.
-__global__ void __launch_bounds__(2 * kThreads)
+__global__ void __launch_bounds__(3 * kThreads / 2, 3)
 bwd_gate_masked_kernel(Shape sh, const float* __restrict__ x, const float* __restrict__ z,
                        const float* __restrict__ dy, const float* __restrict__ ys, const float* __restrict__ D,
                        const int32_t* __restrict__ row_off, const int32_t* __restrict__ row_tok,
