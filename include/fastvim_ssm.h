@@ -223,7 +223,9 @@ FV_API fv_status fastvim_ssm_forward_events(const fv_ssm_args* args, void* ws, s
  * runs as chunks of whole images (about 64 MB of x each, at most 16 chunks) in a pipeline: the
  * upload of one chunk, the layer on the previous one (on `stream`) and the download of the one
  * before overlap, on two streams the call creates and destroys.  The device status word of ws
- * reports the first device error of any chunk. */
+ * reports the first device error of any chunk.  Each chunk reuses the workspace from its start,
+ * so with FV_FLAG_KEEP_STATES it holds the last chunk's scan states only (this entry point has no
+ * gradient counterpart). */
 FV_API fv_status fastvim_ssm_forward_host(const fv_ssm_args* host, const fv_ssm_args* dev, void* ws,
                                    size_t ws_bytes, void* stream);
 
