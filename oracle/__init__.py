@@ -58,6 +58,7 @@ def _load():
                 "fvo_pool_masked": [P, P, P, I, I, I, I, I, Dbl, P],
                 "fvo_proj": [P, I, I, I, I, I, I, P, P, P, P, P],
                 "fvo_scan": [P, P, P, P, I, I, I, I, I, I, U, I, P],
+                "fvo_scan_states": [P, P, P, P, I, I, I, I, I, I, U, I, P],
                 "fvo_gate_dense": [P, P, P, P, I, I, I, I, I, I, P, P, Dbl, P],
                 "fvo_gate_masked": [P, P, P, P, P, I, I, I, I, I, P, P, Dbl, P],
                 "fvo_forward": [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, U, Dbl, I, P, P, Dbl, I, P],
@@ -176,6 +177,20 @@ def scan(xbar, delta, u, A_log, R, N, dir_flags, zoh_exact=False):
                           int(dir_flags), int(bool(zoh_exact)), _p(ys))
     _check(st, "scan")
     return ys
+
+
+def scan_states(xbar, delta, u, A_log, R, N, dir_flags, zoh_exact=False):
+    """The scans' states [nd,B,T,E,N]: [k,b,s] = the state of direction slot k entering its s-th
+    step in scan order (zero at s = 0)."""
+    xbar, delta, u = _f64(xbar), _f64(delta), _f64(u)
+    A_log = _f32(A_log)
+    B, T, E = xbar.shape
+    nd = nd_of(dir_flags)
+    hin = np.empty((nd, B, T, E, N), np.float64)
+    st = _load().fvo_scan_states(_p(xbar), _p(delta), _p(u), _p(A_log), B, T, E, nd, R, N,
+                                 int(dir_flags), int(bool(zoh_exact)), _p(hin))
+    _check(st, "scan_states")
+    return hin
 
 
 def _ln(ln_gamma, ln_beta, E):

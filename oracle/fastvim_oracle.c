@@ -191,6 +191,43 @@ int fvo_scan(const double* xbar, const double* delta, const double* u, const flo
     return FVO_OK;
 }
 
+/* The states the scans above pass through (the same recurrences, stored instead of read out):
+ * hin[k][b][s][e][n] = the state of direction slot k entering its s-th step in scan order
+ * (time t = s forward, t = T-1-s backward), so hin[.][.][0] = 0.  For the gradient, which
+ * restarts the recurrence from stored states. */
+int fvo_scan_states(const double* xbar, const double* delta, const double* u, const float* A_log,
+                    int B, int T, int E, int nd, int R, int N, unsigned dir_flags, int zoh_exact,
+                    double* hin)
+{
+    if (B < 0 || T <= 0 || E <= 0 || R <= 0 || N <= 0 || (dir_flags & ~3u) != 0 ||
+        popcount2(dir_flags) != nd)
+        return FVO_BAD_SHAPE;
+    const int J = R + 2 * N;
+    const size_t rows = (size_t)B * T;
+    int slot = 0;
+    for (unsigned d = FVO_FWD; d <= FVO_BWD; d <<= 1) {
+        if ((dir_flags & d) == 0) continue;
+        for (int b = 0; b < B; ++b)
+            for (int e = 0; e < E; ++e)
+                for (int n = 0; n < N; ++n) {
+                    const double a_n = -exp((double)A_log[((size_t)slot * E + e) * N + n]);
+                    double h = 0.0;
+                    for (int s = 0; s < T; ++s) {
+                        hin[((((size_t)slot * B + b) * T + s) * E + e) * N + n] = h;
+                        const int t = d == FVO_FWD ? s : T - 1 - s;
+                        const size_t row = (size_t)b * T + t;
+                        const double dlt = delta[((size_t)slot * rows + row) * E + e];
+                        const double bn = u[((size_t)slot * rows + row) * J + R + n];
+                        const double ab = exp(dlt * a_n);
+                        const double q = zoh_exact ? (ab - 1.0) / a_n * bn : dlt * bn;
+                        h = ab * h + q * xbar[row * E + e];
+                    }
+                }
+        ++slot;
+    }
+    return FVO_OK;
+}
+
 /* Post-SSM LayerNorm over the E channels of one token (gptget.net summary of 2502.00594,
  * "方法详解" item 5: the repeated output goes through the skip connection and a LayerNorm;
  * pith.science verdict, referee report: the post-SSM LayerNorm is the one VMamba adds before

@@ -65,6 +65,12 @@ int fvo_scan(const double* xbar, const double* delta, const double* u, const flo
              int B, int T, int E, int nd, int R, int N, unsigned dir_flags, int zoh_exact,
              double* ys);
 
+/* The scans' states: hin [nd][B][T][E][N], hin[k][b][s] = the state of direction slot k entering
+ * its s-th step in scan order (zero at s = 0). */
+int fvo_scan_states(const double* xbar, const double* delta, const double* u, const float* A_log,
+                    int B, int T, int E, int nd, int R, int N, unsigned dir_flags, int zoh_exact,
+                    double* hin);
+
 /* Repeat + D x skip (+ the post-SSM LayerNorm over E when ln_gamma, ln_beta [E] are given,
  * both or neither, ln_eps >= 0) + SiLU(z) gate on the dense grid. */
 int fvo_gate_dense(const float* x, const float* z, const double* ys, const float* D, int B,

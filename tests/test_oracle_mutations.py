@@ -57,6 +57,11 @@ MUTATIONS = {
     "conv skip from the forward slot only": ("v += (double)D[(size_t)k * E + e] * xc[(size_t)k * all + g + e];",
                                              "v += (double)D[(size_t)k * E + e] * xc[g + e];"),
     "both directions pool the forward convolved tokens": ("fvo_pool_d(xc + (size_t)k * img, 1,", "fvo_pool_d(xc, 1,"),
+    "states stored after the update": ('                        hin[((((size_t)slot * B + b) * T + s) * E + e) * N + n] = h;\n                        const int t = d == FVO_FWD ? s : T - 1 - s;\n                        const size_t row = (size_t)b * T + t;\n                        const double dlt = delta[((size_t)slot * rows + row) * E + e];\n                        const double bn = u[((size_t)slot * rows + row) * J + R + n];\n                        const double ab = exp(dlt * a_n);\n                        const double q = zoh_exact ? (ab - 1.0) / a_n * bn : dlt * bn;\n                        h = ab * h + q * xbar[row * E + e];\n',
+                                       '                        const int t = d == FVO_FWD ? s : T - 1 - s;\n                        const size_t row = (size_t)b * T + t;\n                        const double dlt = delta[((size_t)slot * rows + row) * E + e];\n                        const double bn = u[((size_t)slot * rows + row) * J + R + n];\n                        const double ab = exp(dlt * a_n);\n                        const double q = zoh_exact ? (ab - 1.0) / a_n * bn : dlt * bn;\n                        h = ab * h + q * xbar[row * E + e];\n                        hin[((((size_t)slot * B + b) * T + s) * E + e) * N + n] = h;\n'),
+    "backward states in time order": ("const int t = d == FVO_FWD ? s : T - 1 - s;", "const int t = s;"),
+    "state input term from C": ("const double bn = u[((size_t)slot * rows + row) * J + R + n];",
+                                "const double bn = u[((size_t)slot * rows + row) * J + R + N + n];"),
     "pool scale ignored": ("pool_scale * acc / (double)S;\n            }\n    return FVO_OK;\n}\n\n/* Row of",
                            "acc / (double)S;\n            }\n    return FVO_OK;\n}\n\n/* Row of"),
 }

@@ -659,3 +659,61 @@ def test_p10_golden_hand_worked_conv_example(oracle_mod):
         full = oracle_mod.forward(x, inp["z"].reshape(x.shape), inp["A_log"], inp["D"], inp["W_x"], inp["W_dt"],
                                   inp["b_dt"], axis, g["dir_flags"], conv_w=inp["conv_w"], conv_b=inp["conv_b"])
         np.testing.assert_allclose(full.ravel(), y, rtol=1e-14)
+
+
+# ---------------------------------------------------------------------------------------------
+# p11: the scans' states (what a training forward keeps for the gradient), pinned to the scan
+#      output the pins above fix and to scipy's first-order filter.
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("dir_flags", [1, 2, 3])
+@pytest.mark.parametrize("T", [4, 9])
+def test_p11_states_read_out_by_C_give_the_scan_output(oracle_mod, dir_flags, T):
+    """ys[t] = sum over directions of C_t . (the state after the direction's step at t), and the
+    state after step s is the one entering step s + 1."""
+    rng = np.random.default_rng(300 + 10 * T + dir_flags)
+    B, E, N, R = 2, 3, 4, 2
+    nd = oracle_mod.nd_of(dir_flags)
+    A_log = rng.uniform(-1, 1, size=(nd, E, N)).astype(np.float32)
+    xbar = rng.standard_normal((B, T, E))
+    delta = rng.uniform(0.01, 0.8, size=(nd, B, T, E))
+    u = rng.standard_normal((nd, B, T, R + 2 * N))
+    for zoh in (False, True):
+        ys = oracle_mod.scan(xbar, delta, u, A_log, R, N, dir_flags, zoh)
+        hin = oracle_mod.scan_states(xbar, delta, u, A_log, R, N, dir_flags, zoh)
+        assert hin.shape == (nd, B, T, E, N) and not hin[:, :, 0].any()
+        fwd = [k == 0 if nd == 2 else dir_flags == 1 for k in range(nd)]
+        checked = 0
+        for t in range(T):
+            steps = [t if fwd[k] else T - 1 - t for k in range(nd)]
+            if max(steps) + 1 >= T:
+                continue  # the state after a scan's last step is not stored
+            for b in range(B):
+                read = sum(np.einsum("en,n->e", hin[k, b, steps[k] + 1], u[k, b, t, R + N:]) for k in range(nd))
+                np.testing.assert_allclose(read, ys[b, t], rtol=1e-12, atol=1e-12)
+                checked += 1
+        assert checked > 0
+
+
+def test_p11_states_lti_match_scipy_lfilter(oracle_mod):
+    """Constant Delta and B: each state is a first-order IIR filter of the input in scan order,
+    h_after = lfilter([1], [1, -a], Delta B x), and the stored state is the one before the step."""
+    rng = np.random.default_rng(11)
+    B, T, E, N, R = 1, 23, 2, 3, 1
+    A_log = rng.uniform(-1, 1, size=(1, E, N)).astype(np.float32)
+    xbar = rng.standard_normal((B, T, E))
+    dval = rng.uniform(0.05, 0.5, size=E)
+    delta = np.broadcast_to(dval[None, None, None, :], (1, B, T, E)).copy()
+    Bn = rng.standard_normal(N)
+    u = rng.standard_normal((1, B, T, R + 2 * N))
+    u[0, 0, :, R:R + N] = Bn[None, :]
+    for dir_flags in (1, 2):
+        hin = oracle_mod.scan_states(xbar, delta, u, A_log, R, N, dir_flags)
+        for e in range(E):
+            for n in range(N):
+                a = math.exp(-dval[e] * math.exp(float(A_log[0, e, n])))
+                seq = xbar[0, :, e] * dval[e] * Bn[n]
+                if dir_flags == 2:
+                    seq = seq[::-1]  # scan order
+                after = scipy.signal.lfilter([1.0], [1.0, -a], seq)
+                ref = np.concatenate([[0.0], after[:-1]])
+                np.testing.assert_allclose(hin[0, 0, :, e, n], ref, rtol=1e-11, atol=1e-12)
