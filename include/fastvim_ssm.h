@@ -90,8 +90,8 @@ enum {
                                  (fv_ws_layout.trace); costs a little time, for profiling      */
     FV_FLAG_LAYERNORM = 16u,  /* post-SSM LayerNorm before the gate (ln_gamma, ln_beta, ln_eps) */
     FV_FLAG_CONV_SILU = 32u,  /* SiLU after the block's Conv1D (needs d_conv > 0)               */
-    FV_FLAG_KEEP_STATES = 64u /* training: the scans also store their 16 states before every 8th
-                                 step (fv_ws_layout.ckpt, B nd 2 ceil(T/16) E 64 bytes more
+    FV_FLAG_KEEP_STATES = 64u /* training: the scans also store their 16 states every 8 steps
+                                 (fv_ws_layout.ckpt, B nd 2 ceil(T/16) E 64 bytes more
                                  workspace) so that the gradient call reads them instead of
                                  running the recurrences a first time; y is unchanged          */
 };
@@ -170,9 +170,12 @@ typedef struct {
                             w1 = SM id << 32 | CTA id, w2 = start (ns, %globaltimer),
                             w3 = wait_ns << 40 | total_ns (from start to the task's end)        */
     size_t trace_records;  /* number of trace entries (tasks of the call), else 0               */
-    size_t ckpt;         /* FV_FLAG_KEEP_STATES: fp32 [B][nd][2 ceil(T/16)][E][16], the 16 states
-                            of each scan entering its steps 0, 8, 16, .. (scan order), zero
-                            past N; else 0                                                  */
+    size_t ckpt;         /* FV_FLAG_KEEP_STATES: fp32 [B][nd][2 ceil(T/16)][E][16], zero past N;
+                            slot 2i+h = the 16 states entering the h-th 8-step half of the
+                            i-th 16-step chunk [16c, 16c+16) of the time axis in the scan's
+                            order (forward: before step 16i+8h; the backward scan starts
+                            with the last, possibly shorter, chunk); a chunk of <= 8 steps
+                            has no slot 2i+1; else 0                                        */
     size_t scan_dt;      /* reserved, 0                                                      */
     int T, S, nd;        /* pooled length, pooled-over length, number of directions          */
 } fv_ws_layout;

@@ -42,9 +42,12 @@ __host__ __device__ __forceinline__ size_t xbar_offset(const Shape& sh, int b, i
     return (((size_t)b * sh.nx + kx) * sh.T + t) * (size_t)sh.E;
 }
 
-// Scan states kept for the gradient (FV_FLAG_KEEP_STATES): the 16 states of (image b, direction
-// k, channel e) entering steps 0, 8, 16, .. of the scan order (slot c: the state before the
-// scan's step 8c), [B][nd][2 ceil(T / 16)][E][16], zero for states n >= N.
+// Scan states kept for the gradient (FV_FLAG_KEEP_STATES), [B][nd][2 ceil(T / 16)][E][16], zero
+// for states n >= N.  Each scan walks the time axis' 16-step chunks [16 c, 16 c + 16) in its own
+// order (forward c = 0, 1, ..; backward from the last, possibly shorter, chunk down); slot 2 i + h
+// of (image b, direction k, channel e) holds the state entering the h-th 8-step half of the
+// scan's i-th chunk (forward: the state before step 16 i + 8 h).  A chunk of at most 8 steps has
+// no second slot.
 constexpr int kCkptSteps = 8;
 __host__ __device__ __forceinline__ int ckpt_count(int T) { return 2 * ((T + 15) / 16); }
 __host__ __device__ __forceinline__ size_t ckpt_offset(const Shape& sh, int b, int k, int c, int e) {

@@ -227,8 +227,9 @@ KEEP_CASES = [
 def test_gradient_from_kept_states(case):
     """FV_FLAG_KEEP_STATES: the forward stores the scan states every 8 steps and the gradient reads
     them instead of running the recurrences a first time.  y keeps its bits, the gradient matches
-    the oracle, and the kept states match the ones the gradient computes itself without the flag
-    (slots of chunks shorter than 8 steps are never written)."""
+    the oracle, and the kept states match the oracle's states at the steps their slots stand for
+    and the ones the gradient computes itself without the flag (slots of chunks of at most 8
+    steps are never written)."""
     B, h, w, E, N, R, axis, dirs, zoh, path, K = case
     nd = bin(dirs).count("1")
     d = make_inputs(23, B, h, w, E, N, R, nd, K=K)
@@ -250,14 +251,21 @@ def test_gradient_from_kept_states(case):
     n = B * nd * nck * E * 16
     fk = kept["fws"][L.ckpt:L.ckpt + 4 * n].view(torch.float32).cpu().numpy().reshape(B, nd, nck, E, 16)
     bk = plain["bws"][Lb.ckpt:Lb.ckpt + 4 * n].view(torch.float32).cpu().numpy().reshape(B, nd, nck, E, 16)
+    # the oracle's states entering every scan step, [nd][B][T][E][N]
+    inter = oracle.forward_intermediates(d["x"], d["z"], d["A_log"], d["D"], d["W_x"], d["W_dt"], d["b_dt"], axis,
+                                         dirs, keep_idx=d.get("keep_idx"), h=h, w=w, zoh_exact=zoh)
+    hin = oracle.scan_states(inter["xbar"], inter["delta"], inter["u"], d["A_log"], R, N, dirs, zoh)
     fwd_slot = [k == 0 if nd == 2 else bool(dirs & 1) for k in range(nd)]
+    nchunks = nck // 2
     for k in range(nd):
+        lens = [min(16, T - 16 * (it if fwd_slot[k] else nchunks - 1 - it)) for it in range(nchunks)]
         for c in range(nck):
-            it = c // 2
-            ci = it if fwd_slot[k] else nck // 2 - 1 - it
-            if c % 2 == 1 and min(16, T - 16 * ci) <= 8:
+            it, half = divmod(c, 2)
+            if half == 1 and lens[it] <= 8:
                 continue  # no second half in this chunk
+            step = sum(lens[:it]) + 8 * half  # the scan step the slot's state enters
             assert not np.isnan(fk[:, k, c]).any()
+            assert_close(fk[:, k, c, :, :N], hin[k, :, step], f"states dir {k} slot {c} vs oracle")
             assert_close(fk[:, k, c], bk[:, k, c], f"states dir {k} slot {c}")
             if c == 0:
                 assert not fk[:, k, c].any()  # every scan starts from zero
