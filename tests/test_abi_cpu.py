@@ -361,3 +361,28 @@ def test_conv_gradient_not_built(lib):
                                   ctypes.c_size_t(1 << 30), ctypes.c_void_p(FAKE + (41 << 32)), ctypes.c_size_t(1 << 30),
                                   None)
     assert st == nat.FV_ERR_UNSUPPORTED
+
+
+def test_binding_constants_and_every_struct_field_match_the_header(tmp_path):
+    """Every status, flag and struct field offset of the ctypes binding equals what a C compiler
+    makes of include/fastvim_ssm.h (the binding only marshals; a drifted offset would pass
+    arguments to the wrong fields)."""
+    consts = [n for n in dir(nat) if n.startswith(("FV_OK", "FV_ERR_", "FV_FLAG_"))]
+    structs = {"fv_ssm_args": nat.FvSsmArgs, "fv_ws_layout": nat.FvWsLayout, "fv_ssm_grads": nat.FvSsmGrads,
+               "fv_bwd_ws_layout": nat.FvBwdWsLayout}
+    lines = [f'printf("%lld\\n", (long long){n});' for n in consts]
+    for cname, cls in structs.items():
+        lines.append(f'printf("%zu\\n", sizeof({cname}));')
+        lines += [f'printf("%zu\\n", offsetof({cname}, {f[0]}));' for f in cls._fields_]
+    src = tmp_path / "abi.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "fastvim_ssm.h"\nint main(void){\n'
+                   + "\n".join(lines) + "\nreturn 0;}\n")
+    exe = tmp_path / "abi"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)],
+                   check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    want = [getattr(nat, n) for n in consts]
+    for cls in structs.values():
+        want.append(ctypes.sizeof(cls))
+        want += [getattr(cls, f[0]).offset for f in cls._fields_]
+    assert got == want
