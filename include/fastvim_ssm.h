@@ -257,7 +257,8 @@ FV_API fv_status fastvim_ssm_forward_host(const fv_ssm_args* host, const fv_ssm_
  *     clearing.
  *   - The device status word lives in the shared scratch and is not readable through this
  *     entry point; use fastvim_ssm_forward with a workspace where FV_ERR_INDEX or
- *     FV_ERR_TIMEOUT must be seen.
+ *     FV_ERR_TIMEOUT must be seen.  Likewise a gradient call needs the forward's workspace,
+ *     which this entry point does not expose: FV_FLAG_KEEP_STATES only costs scratch here.
  * Inputs, outputs and the returned status are as for fastvim_ssm_forward. */
 FV_API fv_status fastvim_ssm_forward_noalloc(const fv_ssm_args* args, void* stream);
 
